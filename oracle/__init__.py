@@ -1,0 +1,190 @@
+"""Plain fp64 CPU oracle for the CSA / HCA hot path (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s cpu_baseline /
+``--impl reference`` leg may import this package.  The product library never imports,
+links or calls it; the two share no code.  The arithmetic lives in ``csa_oracle.c``
+(compiled here with gcc into ``liboracle.so``); this module only marshals numpy arrays.
+
+Sources:
+  "DeepSeek-V4 Hybrid Attention: CSA and HCA from Scratch" (cited as [P1]) sections 3-12;
+  bhhxx.wiki "MHA -> ... -> CSA/HCA", section 6.2.2 (cited as [P4]).
+
+Parity pins: tests/test_oracle_pins.py (worked example in closed form, printed values,
+invariants, brute force against library routines, ledger).  No function here is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "csa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile csa_oracle.c with gcc (plain -O2, no fast-math) into liboracle.so."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            dp = ctypes.POINTER(ctypes.c_double)
+            i64 = ctypes.c_int64
+            lib.oracle_project.argtypes = [dp, dp, i64, i64, i64, dp]
+            lib.oracle_csa_compress.argtypes = [dp, dp, dp, dp, dp, dp, i64, i64, i64, i64, i64, dp]
+            lib.oracle_hca_compress.argtypes = [dp, dp, dp, i64, i64, i64, i64, i64, dp]
+            lib.oracle_visible.argtypes = [i64, i64, i64]
+            lib.oracle_visible.restype = i64
+            lib.oracle_index_scores.argtypes = [dp, dp, dp, i64, i64, i64, dp]
+            lib.oracle_topk.argtypes = [dp, i64, i64, ctypes.POINTER(ctypes.c_int32)]
+            lib.oracle_mqa.argtypes = [dp, dp, ctypes.POINTER(ctypes.c_int32), i64, i64, i64,
+                                       ctypes.c_double, dp, dp]
+            _lib = lib
+    return _lib
+
+
+def _d(a):
+    """Contiguous float64 copy (or view) of ``a``."""
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a, ctype=ctypes.c_double):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def project(H, W):
+    """out = H @ W by the plain triple loop ([P1] section 3)."""
+    H, W = _d(H), _d(W)
+    n, d = H.shape
+    d2, c = W.shape
+    assert d == d2
+    out = np.empty((n, c), np.float64)
+    _load().oracle_project(_ptr(H), _ptr(W), n, d, c, _ptr(out))
+    return out
+
+
+def csa_compress(Ca, Cb, Za, Zb, m, Ba=None, Bb=None, i0=0, i1=None):
+    """CSA overlapped compressor ([P1] sections 4-5): entries i0 <= i < i1, [i1-i0, c]."""
+    Ca, Cb, Za, Zb = _d(Ca), _d(Cb), _d(Za), _d(Zb)
+    n, c = Ca.shape
+    for a in (Cb, Za, Zb):
+        assert a.shape == (n, c)
+    if i1 is None:
+        i1 = n // m
+    assert 0 <= i0 <= i1 and m * i1 <= n
+    Ba = None if Ba is None else _d(Ba)
+    Bb = None if Bb is None else _d(Bb)
+    if Ba is not None:
+        assert Ba.shape == (m, c)
+    if Bb is not None:
+        assert Bb.shape == (m, c)
+    out = np.empty((i1 - i0, c), np.float64)
+    _load().oracle_csa_compress(_ptr(Ca), _ptr(Cb), _ptr(Za), _ptr(Zb), _ptr(Ba), _ptr(Bb),
+                                n, c, m, i0, i1, _ptr(out))
+    return out
+
+
+def hca_compress(C, Z, m_prime, Bias=None, i0=0, i1=None):
+    """HCA compressor ([P1] section 10): entries i0 <= i < i1, [i1-i0, c]."""
+    C, Z = _d(C), _d(Z)
+    n, c = C.shape
+    assert Z.shape == (n, c)
+    if i1 is None:
+        i1 = n // m_prime
+    assert 0 <= i0 <= i1 and m_prime * i1 <= n
+    Bias = None if Bias is None else _d(Bias)
+    if Bias is not None:
+        assert Bias.shape == (m_prime, c)
+    out = np.empty((i1 - i0, c), np.float64)
+    _load().oracle_hca_compress(_ptr(C), _ptr(Z), _ptr(Bias), n, c, m_prime, i0, i1, _ptr(out))
+    return out
+
+
+def visible(t, m, N_cap):
+    """Number of compressed entries query t may see: min(floor(t/m), N_cap) ([P1] s.7)."""
+    return int(_load().oracle_visible(int(t), int(m), int(N_cap)))
+
+
+def index_scores(qI, wI, KI, nvis=None):
+    """I[s] = sum_h w[h] ReLU(q[h].K[s]) for s < nvis ([P1] section 6.4)."""
+    qI, wI, KI = _d(qI), _d(wI), _d(KI)
+    n_hI, cI = qI.shape
+    assert wI.shape == (n_hI,)
+    if nvis is None:
+        nvis = KI.shape[0]
+    assert KI.shape[1] == cI and nvis <= KI.shape[0]
+    out = np.empty((nvis,), np.float64)
+    _load().oracle_index_scores(_ptr(qI), _ptr(wI), _ptr(KI), nvis, n_hI, cI, _ptr(out))
+    return out
+
+
+def topk(scores, k):
+    """Indices of the k largest scores, ties to the smaller index, -1 padded ([P1] s.7)."""
+    scores = _d(scores)
+    idx = np.empty((k,), np.int32)
+    _load().oracle_topk(_ptr(scores), scores.shape[0], k, _ptr(idx, ctypes.c_int32))
+    return idx
+
+
+def mqa(q, cache, sel, scale=None):
+    """Shared-KV MQA over the entries ``sel`` (-1 skipped) ([P1] section 8).
+
+    Returns (out [n_h, c], lse [n_h]); scale defaults to 1/sqrt(c).
+    """
+    q, cache = _d(q), _d(cache)
+    n_h, c = q.shape
+    assert cache.shape[1] == c
+    sel = np.ascontiguousarray(sel, dtype=np.int32)
+    assert sel.ndim == 1
+    if sel.size:
+        assert sel.max() < cache.shape[0]
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(c)
+    out = np.empty((n_h, c), np.float64)
+    lse = np.empty((n_h,), np.float64)
+    _load().oracle_mqa(_ptr(q), _ptr(cache) if cache.size else _ptr(np.zeros(1)),
+                       _ptr(sel, ctypes.c_int32) if sel.size else None, sel.size, n_h, c,
+                       float(scale), _ptr(out), _ptr(lse))
+    return out, lse
+
+
+def round_bf16(x):
+    """Round float64/float32 values to the nearest bfloat16 (ties to even), as float64.
+
+    This is the storage rounding of a bf16 compressed cache (the pages do not fix the
+    cache precision; the reading used is bf16 round-to-nearest-even).  Written here
+    independently of the CUDA library's conversion.
+    """
+    f = np.ascontiguousarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) >> 16) << 16
+    nan = np.isnan(f)
+    out = r.astype(np.uint32).view(np.float32).astype(np.float64)
+    out[nan] = np.nan
+    return out
+
+
+from .ledger import kv_ledger  # noqa: E402  (pure arithmetic of [P1] section 12)
+
+__all__ = ["build", "project", "csa_compress", "hca_compress", "visible", "index_scores",
+           "topk", "mqa", "round_bf16", "kv_ledger"]

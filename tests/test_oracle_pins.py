@@ -1,0 +1,390 @@
+"""Pins for the fp64 CPU oracle: what the pages and mathematics fix, not the oracle itself.
+
+Source: "DeepSeek-V4 Hybrid Attention: CSA and HCA from Scratch" ([P1]) - the six-token
+worked example (sections 3-10), its printed softmax vectors and entries, the indexer
+and top-k numerical checks (sections 6.4, 7), the single-element attention check
+(section 8) and the ledger (sections 1, 12.1).  Printed decimals are rounded on the
+page, so they are checked to 3e-3 while the closed forms derived from the same
+numbers are checked to 1e-12.  Each pin is chosen so that a plausible slip in the
+oracle (dropped b-stream, wrong block offset, softmax over the wrong axis, missing
+ReLU, wrong scale, off-by-one visibility, wrong tie order) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import logsumexp, softmax
+
+import oracle
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_example.json")))
+E = math.e
+TOL_PRINTED = GOLD["printed_tolerance"]
+
+
+def g(name):
+    return np.array(GOLD[name]["value"], dtype=np.float64)
+
+
+def streams():
+    H = g("H")
+    return (oracle.project(H, g("W_aKV")), oracle.project(H, g("W_bKV")),
+            oracle.project(H, g("W_aZ")), oracle.project(H, g("W_bZ")))
+
+
+# ----------------------------------------------------------------------------------
+# worked example: projections, compressors, indexer, top-k, attention
+# ----------------------------------------------------------------------------------
+def test_projection_reproduces_printed_streams():
+    Ca, Cb, Za, Zb = streams()
+    for name, got in (("Ca", Ca), ("Cb", Cb), ("Za", Za), ("Zb", Zb)):
+        np.testing.assert_array_equal(got, g(name), err_msg=name)
+
+
+def test_csa_entries_closed_form():
+    Ca, Cb, Za, Zb = streams()
+    C = oracle.csa_compress(Ca, Cb, Za, Zb, m=2)
+    assert C.shape == (3, 2)
+    want = np.array([
+        [E / (E + 1), 1.0],                                   # section 5, C_0
+        [(4 * E**2 + E) / (2 * E**2 + E + 1), 0.75],          # section 5, C_1
+        [3 * E / (1 + 3 * E), 1.0],                           # C_2 ("analogous", derived)
+    ])
+    np.testing.assert_allclose(C, want, rtol=0, atol=1e-12)
+
+
+def test_csa_entries_printed():
+    Ca, Cb, Za, Zb = streams()
+    C = oracle.csa_compress(Ca, Cb, Za, Zb, m=2)
+    np.testing.assert_allclose(C[:2], g("csa_entries"), rtol=0, atol=TOL_PRINTED)
+
+
+def _indicator_weights(compress, n, c, row_count, entry, col, **kw):
+    """Softmax weight of every candidate row, read off the compressor by feeding a value
+    stream that is 1 on one token row and 0 elsewhere (output = that row's weight)."""
+    out = []
+    for row in range(row_count):
+        ind = np.zeros((n, c))
+        ind[row, col] = 1.0
+        out.append(compress(ind, entry, **kw)[col])
+    return np.array(out)
+
+
+def test_csa_softmax_weights_printed():
+    Ca, Cb, Za, Zb = streams()
+    sm = GOLD["csa_softmax"]
+
+    def w_a(block, col):
+        # weight of a-stream rows 2*block, 2*block+1 (b-stream values zero)
+        ws = []
+        for r in range(2):
+            ind = np.zeros((6, 2)); ind[2 * block + r, col] = 1.0
+            ws.append(oracle.csa_compress(ind, np.zeros((6, 2)), Za, Zb, m=2)[block, col])
+        return ws
+
+    def w_b(block, col):
+        ws = []
+        for r in range(2):
+            row = 2 * (block - 1) + r
+            if row < 0:
+                ws.append(0.0)
+                continue
+            ind = np.zeros((6, 2)); ind[row, col] = 1.0
+            ws.append(oracle.csa_compress(np.zeros((6, 2)), ind, Za, Zb, m=2)[block, col])
+        return ws
+
+    for block in (0, 1):
+        for col in (0, 1):
+            got = np.array(w_a(block, col) + w_b(block, col))
+            want = np.array(sm["block%d_col%d" % (block, col)])
+            np.testing.assert_allclose(got, want, atol=TOL_PRINTED)
+            assert abs(got.sum() - 1.0) < 1e-12          # section 4 numerical check
+    # block 1 column 0 closed form: [e^2, e, 1, e^2] / (2e^2 + e + 1)
+    d = 2 * E**2 + E + 1
+    got = np.array(w_a(1, 0) + w_b(1, 0))
+    np.testing.assert_allclose(got, [E**2 / d, E / d, 1 / d, E**2 / d], atol=1e-12)
+
+
+def test_hca_entries_closed_form_and_printed():
+    H = g("H")
+    C = oracle.project(H, g("W_aKV"))
+    Z = oracle.project(H, g("W_aZ"))
+    out = oracle.hca_compress(C, Z, m_prime=3)
+    want = np.array([[(E + 2 * E**2) / (1 + E + E**2), 1.0], [2 * E / (2 * E + 1), 2.0 / 3.0]])
+    np.testing.assert_allclose(out, want, atol=1e-12)
+    np.testing.assert_allclose(out, g("hca_entries"), atol=TOL_PRINTED)
+
+
+def test_hca_softmax_weights_printed():
+    H = g("H")
+    Z = oracle.project(H, g("W_aZ"))
+    sm = GOLD["hca_softmax"]
+    for block in (0, 1):
+        for col in (0, 1):
+            ws = []
+            for r in range(3):
+                ind = np.zeros((6, 2)); ind[3 * block + r, col] = 1.0
+                ws.append(oracle.hca_compress(ind, Z, m_prime=3)[block, col])
+            np.testing.assert_allclose(ws, sm["block%d_col%d" % (block, col)], atol=TOL_PRINTED)
+            assert abs(sum(ws) - 1.0) < 1e-12
+
+
+def test_indexer_queries_scores_printed():
+    H = g("H")
+    t = GOLD["params"]["t"]
+    cQ = oracle.project(H[t:t + 1], g("W_DQ"))[0]
+    np.testing.assert_array_equal(cQ, g("cQ_5"))
+    qI = oracle.project(cQ[None], g("W_IUQ"))            # [1, n_hI * cI] = [1, 2]
+    np.testing.assert_array_equal(qI[0], g("qI_5"))
+    wI = oracle.project(H[t:t + 1], g("W_w"))[0]
+    assert wI[0] == GOLD["wI_5"]["value"]
+    s = oracle.index_scores(qI.reshape(1, 2), wI, g("KI"))
+    np.testing.assert_array_equal(s, g("index_scores"))
+
+
+def test_visibility_and_topk_printed():
+    p = GOLD["params"]
+    assert oracle.visible(p["t"], p["m"], 3) == GOLD["visible_csa"]["value"]
+    assert oracle.visible(p["t"], p["m_prime"], 2) == GOLD["visible_hca"]["value"]
+    s = oracle.index_scores(g("qI_5")[None], np.array([1.0]), g("KI"))
+    np.testing.assert_array_equal(oracle.topk(s, 1), g("topk_k1").astype(np.int32))
+
+
+def test_csa_attention_printed_and_k2_closed_form():
+    Ca, Cb, Za, Zb = streams()
+    C = oracle.csa_compress(Ca, Cb, Za, Zb, m=2)
+    q = oracle.project(g("cQ_5")[None], g("W_UQ"))       # [1, 2]
+    o, lse = oracle.mqa(q, C, np.array([1], np.int32))
+    np.testing.assert_allclose(o[0], C[1], atol=1e-15)   # single value: output = value
+    np.testing.assert_allclose(o[0], g("csa_output_k1"), atol=TOL_PRINTED)
+    # k = 2 at t = 5: logits q.C_s / sqrt(2), weights and output in closed form
+    c0 = E / (E + 1)
+    c1 = (4 * E**2 + E) / (2 * E**2 + E + 1)
+    l0, l1 = c0 / math.sqrt(2), c1 / math.sqrt(2)
+    w1 = 1.0 / (1.0 + math.exp(l0 - l1))
+    want = (1 - w1) * np.array([c0, 1.0]) + w1 * np.array([c1, 0.75])
+    o2, lse2 = oracle.mqa(q, C, np.array([0, 1], np.int32))
+    np.testing.assert_allclose(o2[0], want, atol=1e-12)
+    np.testing.assert_allclose(o2[0], [1.412288, 0.832019], atol=1e-6)
+    assert abs(lse2[0] - math.log(math.exp(l0) + math.exp(l1))) < 1e-12
+
+
+def test_hca_attention_printed():
+    H = g("H")
+    C = oracle.hca_compress(oracle.project(H, g("W_aKV")), oracle.project(H, g("W_aZ")), 3)
+    vis = oracle.visible(5, 3, C.shape[0])
+    o, _ = oracle.mqa(g("cQ_5")[None], C, np.arange(vis, dtype=np.int32))
+    np.testing.assert_allclose(o[0], C[0], atol=1e-15)
+    np.testing.assert_allclose(o[0], g("hca_output"), atol=TOL_PRINTED)
+
+
+# ----------------------------------------------------------------------------------
+# compressor invariants and reductions
+# ----------------------------------------------------------------------------------
+def rnd(seed, *shape):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+@pytest.mark.parametrize("m", [1, 2, 4])
+def test_csa_convex_and_constant(m):
+    n, c = 6 * m, 5
+    Ca, Cb, Za, Zb = (rnd(s, n, c) for s in range(4))
+    out = oracle.csa_compress(Ca, Cb, Za, Zb, m)
+    for i in range(n // m):
+        cand_a = Ca[m * i:m * i + m]
+        cand = cand_a if i == 0 else np.vstack([cand_a, Cb[m * (i - 1):m * i]])
+        assert np.all(out[i] <= cand.max(0) + 1e-12) and np.all(out[i] >= cand.min(0) - 1e-12)
+    const = np.tile(np.arange(c, dtype=np.float64), (n, 1))
+    out = oracle.csa_compress(const, const, Za, Zb, m)
+    np.testing.assert_allclose(out, np.tile(np.arange(c), (n // m, 1)), atol=1e-12)
+
+
+def test_csa_equal_logits_give_mean():
+    m, n, c = 4, 16, 3
+    Ca, Cb = rnd(1, n, c), rnd(2, n, c)
+    Z = np.full((n, c), 0.37)
+    out = oracle.csa_compress(Ca, Cb, Z, Z, m)
+    np.testing.assert_allclose(out[0], Ca[0:4].mean(0), atol=1e-12)      # padding excluded
+    for i in range(1, n // m):
+        want = np.vstack([Ca[4 * i:4 * i + 4], Cb[4 * i - 4:4 * i]]).mean(0)
+        np.testing.assert_allclose(out[i], want, atol=1e-12)
+
+
+def test_csa_one_hot_limits_through_logits_and_biases():
+    m, n, c = 4, 12, 3
+    Ca, Cb = rnd(3, n, c), rnd(4, n, c)
+    Za, Zb = np.zeros((n, c)), np.zeros((n, c))
+    Za[9, 1] = 60.0                  # entry 2, a-row r=1, column 1
+    Zb[6, 2] = 60.0                  # b-row of entry 2 (previous block rows 4..7), r=2
+    out = oracle.csa_compress(Ca, Cb, Za, Zb, m)
+    assert abs(out[2, 1] - Ca[9, 1]) < 1e-12
+    assert abs(out[2, 2] - Cb[6, 2]) < 1e-12
+    # the bias is indexed by position within the block and shared by every block
+    Ba, Bb = np.zeros((m, c)), np.zeros((m, c))
+    Ba[3, 0] = 60.0
+    out = oracle.csa_compress(Ca, Cb, np.zeros((n, c)), np.zeros((n, c)), m, Ba=Ba, Bb=Bb)
+    for i in range(n // m):
+        assert abs(out[i, 0] - Ca[m * i + 3, 0]) < 1e-12
+    Bb[0, 1] = 60.0
+    out = oracle.csa_compress(Ca, Cb, np.zeros((n, c)), np.zeros((n, c)), m, Ba=None, Bb=Bb)
+    for i in range(1, n // m):
+        assert abs(out[i, 1] - Cb[m * (i - 1), 1]) < 1e-12
+    # a per-column constant added to every logit leaves the softmax unchanged
+    Za, Zb = rnd(5, n, c), rnd(6, n, c)
+    shift = np.tile(rnd(7, 1, c), (m, 1))
+    np.testing.assert_allclose(oracle.csa_compress(Ca, Cb, Za, Zb, m, Ba=shift, Bb=shift),
+                               oracle.csa_compress(Ca, Cb, Za, Zb, m), atol=1e-12)
+
+
+def test_csa_reduces_to_hca_pooling_of_each_stream():
+    m, n, c = 4, 20, 6
+    Ca, Cb, Za, Zb = (rnd(10 + s, n, c) for s in range(4))
+    ninf = np.full((n, c), -np.inf)
+    # b-stream switched off: entry i = m-pooling of a-stream block i
+    np.testing.assert_allclose(oracle.csa_compress(Ca, Cb, Za, ninf, m),
+                               oracle.hca_compress(Ca, Za, m), atol=1e-12)
+    # a-stream switched off: entry i >= 1 = m-pooling of b-stream block i-1
+    out = oracle.csa_compress(Ca, Cb, ninf, Zb, m)
+    np.testing.assert_allclose(out[1:], oracle.hca_compress(Cb, Zb, m)[:-1], atol=1e-12)
+
+
+def test_csa_brute_force_against_scipy_softmax():
+    m, n, c = 3, 12, 4
+    Ca, Cb, Za, Zb = (rnd(20 + s, n, c) for s in range(4))
+    Ba, Bb = rnd(30, m, c), rnd(31, m, c)
+    out = oracle.csa_compress(Ca, Cb, Za, Zb, m, Ba=Ba, Bb=Bb)
+    for i in range(n // m):
+        la, va = Za[m * i:m * i + m] + Ba, Ca[m * i:m * i + m]
+        if i == 0:
+            L, V = la, va
+        else:
+            L = np.vstack([la, Zb[m * i - m:m * i] + Bb])
+            V = np.vstack([va, Cb[m * i - m:m * i]])
+        np.testing.assert_allclose(out[i], (softmax(L, axis=0) * V).sum(0), atol=1e-12)
+
+
+def test_compress_entry_ranges_are_consistent():
+    m, n, c = 4, 32, 5
+    Ca, Cb, Za, Zb = (rnd(40 + s, n, c) for s in range(4))
+    full = oracle.csa_compress(Ca, Cb, Za, Zb, m)
+    np.testing.assert_array_equal(oracle.csa_compress(Ca, Cb, Za, Zb, m, i0=3, i1=5), full[3:5])
+    fullh = oracle.hca_compress(Ca, Za, 8)
+    np.testing.assert_array_equal(oracle.hca_compress(Ca, Za, 8, i0=2, i1=4), fullh[2:4])
+
+
+def test_hca_brute_force_and_bias():
+    mp, n, c = 8, 32, 3
+    C, Z, Bias = rnd(50, n, c), rnd(51, n, c), rnd(52, mp, c)
+    out = oracle.hca_compress(C, Z, mp, Bias=Bias)
+    for i in range(n // mp):
+        L = Z[mp * i:mp * i + mp] + Bias
+        np.testing.assert_allclose(out[i], (softmax(L, axis=0) * C[mp * i:mp * i + mp]).sum(0),
+                                   atol=1e-12)
+
+
+# ----------------------------------------------------------------------------------
+# indexer, top-k, attention
+# ----------------------------------------------------------------------------------
+def test_index_scores_brute_force_relu_and_linearity():
+    n_hI, cI, N = 5, 7, 40
+    qI, KI, wI = rnd(60, n_hI, cI), rnd(61, N, cI), rnd(62, n_hI)
+    s = oracle.index_scores(qI, wI, KI)
+    np.testing.assert_allclose(s, np.maximum(KI @ qI.T, 0.0) @ wI, atol=1e-12)
+    # ReLU: a head whose dot products are all negative contributes nothing
+    KIpos = np.abs(KI)
+    qneg = qI.copy(); qneg[0] = -np.abs(qneg[0])
+    s1 = oracle.index_scores(qneg, wI, KIpos)
+    s2 = oracle.index_scores(qneg[1:], wI[1:], KIpos)
+    np.testing.assert_allclose(s1, s2, atol=1e-12)
+    # linear in w, and truncated at nvis
+    np.testing.assert_allclose(oracle.index_scores(qI, 2 * wI, KI), 2 * s, atol=1e-12)
+    np.testing.assert_array_equal(oracle.index_scores(qI, wI, KI, nvis=11), s[:11])
+
+
+def test_topk_against_stable_sort_ties_and_padding():
+    rng = np.random.default_rng(70)
+    s = rng.integers(0, 6, size=50).astype(np.float64)        # many exact ties
+    for k in (1, 7, 13, 50):
+        want = np.argsort(-s, kind="stable")[:k]
+        np.testing.assert_array_equal(oracle.topk(s, k), want.astype(np.int32))
+    got = oracle.topk(s[:5], 8)
+    assert sorted(got[:5].tolist()) == list(range(5)) and list(got[5:]) == [-1, -1, -1]
+    assert list(oracle.topk(np.zeros(0), 3)) == [-1, -1, -1]
+    # largest scores win regardless of position; ties resolved to the smaller index
+    s = np.array([0.5, 2.0, 2.0, -1.0, 3.0])
+    assert list(oracle.topk(s, 2)) == [4, 1]
+
+
+def test_visibility_floor_and_cap():
+    assert oracle.visible(0, 4, 10) == 0
+    assert oracle.visible(3, 4, 10) == 0
+    assert oracle.visible(4, 4, 10) == 1
+    assert oracle.visible(8192, 4, 4096) == 2048
+    assert oracle.visible(10**6, 4, 100) == 100
+    assert oracle.visible(131072, 128, 1024) == 1024
+
+
+def test_mqa_brute_force_lse_permutation_and_padding():
+    n_h, c, N = 4, 8, 30
+    q, cache = rnd(80, n_h, c), rnd(81, N, c)
+    sel = np.array([3, 17, 0, 29, 8], np.int32)
+    o, lse = oracle.mqa(q, cache, sel)
+    logits = q @ cache[sel].T / math.sqrt(c)
+    np.testing.assert_allclose(o, softmax(logits, axis=1) @ cache[sel], atol=1e-12)
+    np.testing.assert_allclose(lse, logsumexp(logits, axis=1), atol=1e-12)
+    o2, lse2 = oracle.mqa(q, cache, sel[::-1].copy())
+    np.testing.assert_allclose(o2, o, atol=1e-12)
+    o3, lse3 = oracle.mqa(q, cache, np.array([-1, 3, 17, -1, 0, 29, 8, -1], np.int32))
+    np.testing.assert_allclose(o3, o, atol=1e-12)
+    np.testing.assert_allclose(lse3, lse, atol=1e-12)
+    # zero query: uniform weights -> mean of the selected values
+    o4, _ = oracle.mqa(np.zeros((1, c)), cache, sel)
+    np.testing.assert_allclose(o4[0], cache[sel].mean(0), atol=1e-12)
+    # explicit scale
+    o5, lse5 = oracle.mqa(q, cache, sel, scale=0.25)
+    np.testing.assert_allclose(lse5, logsumexp(q @ cache[sel].T * 0.25, axis=1), atol=1e-12)
+    # nothing visible
+    o6, lse6 = oracle.mqa(q, cache, np.array([-1, -1], np.int32))
+    assert np.all(o6 == 0) and np.all(np.isneginf(lse6))
+
+
+def test_hca_dense_equals_sparse_over_all_visible():
+    n, c, mp = 64, 6, 8
+    C, Z, q = rnd(90, n, c), rnd(91, n, c), rnd(92, 3, c)
+    cache = oracle.hca_compress(C, Z, mp)
+    t = 45
+    vis = oracle.visible(t, mp, cache.shape[0])
+    assert vis == 5
+    o, _ = oracle.mqa(q, cache, np.arange(vis, dtype=np.int32))
+    o_perm, _ = oracle.mqa(q, cache, np.random.default_rng(0).permutation(vis).astype(np.int32))
+    np.testing.assert_allclose(o, o_perm, atol=1e-12)
+
+
+def test_round_bf16_ties_to_even():
+    vals = np.array([1.0, 1.0 + 2**-8, 1.0 + 3 * 2**-8, 1.0 + 2**-9, -2.5, 0.0, 65504.0])
+    got = oracle.round_bf16(vals)
+    np.testing.assert_array_equal(got, [1.0, 1.0, 1.0 + 4 * 2**-8, 1.0, -2.5, 0.0, 65536.0])
+
+
+# ----------------------------------------------------------------------------------
+# ledger ([P1] sections 1 and 12.1)
+# ----------------------------------------------------------------------------------
+def test_ledger_ratios():
+    L = GOLD["ledger"]
+    led = oracle.kv_ledger(n=1)
+    assert led["csa_bytes"] == L["csa_bytes_per_token_layer"]
+    assert led["hca_bytes"] == L["hca_bytes_per_token_layer"]
+    assert led["csa_over_gqa"] == L["csa_over_gqa"]
+    assert led["hca_over_gqa"] == 8 / 2048
+    assert abs(led["hca_over_gqa"] - L["hca_over_gqa_printed"]) < 1e-4
+    assert abs(led["mix_over_gqa"] - L["mix_numerator"] / L["mix_denominator"]) < 1e-15
+    assert abs(led["mix_over_gqa"] - L["mix_over_gqa_printed"]) < 1e-3
+    led2 = oracle.kv_ledger(n=1, kv_factor=2)
+    assert led2["gqa_bytes"] == L["gqa_bytes_per_token_layer_section1"]
+    assert led2["csa_over_gqa"] == 0.0625
+    assert led["indexer_key_bytes"] == 64
+    from oracle.ledger import raw_request_bytes
+    assert raw_request_bytes() == 10**6 * 61 * 4096
+    assert abs(raw_request_bytes() - L["raw_request_bytes_1M_61_layers"]) / 2.5e11 < 0.01
