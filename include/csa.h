@@ -1,0 +1,178 @@
+/*
+ * csa.h - C ABI of the B200 (sm_100a) kernels for the DeepSeek-V4 hybrid-attention hot
+ * path: CSA / HCA sequence compression, lightning-indexer scoring with top-k
+ * selection, and shared-KV multi-query attention over compressed entries.
+ *
+ * Sources (page title, then section / equation):
+ *   [P1] "DeepSeek-V4 Hybrid Attention: CSA and HCA from Scratch"
+ *   [P4] bhhxx.wiki "MHA -> ... -> CSA/HCA" (Chinese), sections 6.1 and 6.2.2
+ *
+ * Conventions shared by every entry point
+ *   - Tensor pointers are DEVICE pointers owned by the caller; the library never
+ *     allocates, frees or keeps them.  Scratch comes from a caller workspace whose size
+ *     the matching *_workspace_size() call returns.
+ *   - Every call is asynchronous on `stream` and returns an int status: CSA_OK (0) or a
+ *     negative CSA_ERR_* code.  Argument errors are detected on the host before any
+ *     launch and leave every output untouched.  CSA_ERR_CUDA reports a launch failure
+ *     (cudaGetLastError after the launch).  No call aborts the process.
+ *   - `dtype` (CSA_BF16 or CSA_F32) is the element type of every floating-point tensor
+ *     argument of a call except those typed `float*` in the prototype, which are
+ *     always fp32.  bf16 data is IEEE bfloat16 bit patterns.
+ *   - All arithmetic is fp32 (softmax, accumulation, scores); bf16 outputs are rounded
+ *     to nearest even.  Inputs must be finite.
+ *   - Row-major layouts, last dimension contiguous.  Pointers must be aligned to their
+ *     element size (CSA_ERR_ALIGN otherwise), workspaces to 16 bytes.  The fast paths
+ *     use 16-byte vector accesses and are taken when every pointer and row stride of
+ *     the call is 16-byte aligned; other layouts run an element-wise path.
+ *   - Stateless and thread-safe; calls that share a workspace must not overlap on the
+ *     GPU.
+ */
+#ifndef CSA_B200_H
+#define CSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (same ABI); NULL is the legacy default stream. */
+typedef struct CUstream_st* csa_stream_t;
+
+enum csa_dtype { CSA_BF16 = 0, CSA_F32 = 1 };
+
+enum csa_status {
+    CSA_OK = 0,
+    CSA_ERR_ARG = -1,         /* null pointer, negative or inconsistent size */
+    CSA_ERR_ALIGN = -2,       /* pointer or stride not 16-byte aligned */
+    CSA_ERR_DTYPE = -3,       /* unknown dtype, or out_bf16 with CSA_F32 */
+    CSA_ERR_WORKSPACE = -4,   /* workspace NULL or smaller than *_workspace_size() */
+    CSA_ERR_CUDA = -5,        /* a CUDA launch or runtime call failed */
+    CSA_ERR_UNSUPPORTED = -6  /* shape outside what the kernels implement */
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* csa_status_string(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int csa_version(void);
+
+/* ---------------------------------------------------------------------------------
+ * csa_compress - CSA overlapped compression ([P1] section 4, boxed sum of section 5;
+ * [P4] section 6.2.2 compressor path).
+ *
+ * For every batch b and entry i in [entry_begin, entry_end), and column j < c:
+ *   logits  = [ Za[m*i + r][j] + Ba[r][j]      for r < m   (block i, stream a)
+ *               Zb[m*(i-1) + r][j] + Bb[r][j]  for r < m ] (block i-1, stream b)
+ *   S       = softmax over those 2m logits (one softmax per column)
+ *   out[i][j] = sum_r S_a[r] * Ca[m*i + r][j] + sum_r S_b[r] * Cb[m*(i-1) + r][j]
+ * For i == 0 the b-rows are absent (logit -inf, value 0: the padding rule of [P1]).
+ *
+ * Ca, Cb, Za, Zb : token rows of the four projected streams (dtype).  Row r of batch b
+ *                  of stream X is at X + b*ld_batch + (r - tok0)*ld_row (elements).
+ *                  Rows tok0 .. n-1 must be readable; the call reads rows
+ *                  m*(entry_begin-1) (or 0 when entry_begin == 0) .. m*entry_end - 1,
+ *                  so tok0 <= that first row and m*entry_end <= n are required.
+ *                  One interleaved [n, 4c] projection output works with ld_row = 4c.
+ * Ba, Bb         : fp32 [m, c] per-position-in-block biases, or NULL for zero.
+ * out            : compressed cache (dtype); entry i of batch b is written at
+ *                  out + b*out_ld_batch + i*c.  Entries outside the range are untouched
+ *                  (prefill: [0, n/m); incremental decode: [i, i+1)).
+ * Constraints    : c >= 1, 1 <= m <= 4096.
+ * The indexer keys K^I are produced by the same call with their own streams and c^I
+ * ([P1] section 6.4: "the same compression operation ... a separate set of weights").
+ * ------------------------------------------------------------------------------- */
+int csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                 int64_t ld_row, int64_t ld_batch, int64_t tok0, int64_t n,
+                 const float* Ba, const float* Bb,
+                 void* out, int64_t out_ld_batch,
+                 int B, int c, int m, int64_t entry_begin, int64_t entry_end,
+                 int dtype, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * hca_compress - HCA compression ([P1] section 10, boxed equations; [P4] section 6.1):
+ * non-overlapping blocks of m' tokens, one stream, per-column softmax over the m'
+ * logits Z[m'*i + r][j] + Bias[r][j], weighted sum of C[m'*i + r][j].
+ *
+ * C, Z   : token rows (dtype), row r of batch b at X + b*ld_batch + (r - tok0)*ld_row;
+ *          rows m'*entry_begin .. m'*entry_end - 1 are read (tok0 <= m'*entry_begin,
+ *          m'*entry_end <= n).
+ * Bias   : fp32 [m', c] or NULL.
+ * out    : entry i of batch b at out + b*out_ld_batch + i*c (dtype).
+ * ------------------------------------------------------------------------------- */
+int hca_compress(const void* C, const void* Z,
+                 int64_t ld_row, int64_t ld_batch, int64_t tok0, int64_t n,
+                 const float* Bias,
+                 void* out, int64_t out_ld_batch,
+                 int B, int c, int m_prime, int64_t entry_begin, int64_t entry_end,
+                 int dtype, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * csa_indexer_topk - lightning-indexer scores and top-k selection ([P1] section 6.4
+ * boxed score, section 7 selection and causal rule; [P4] section 6.2.2 indexer).
+ *
+ * For query g = b*nq + q at position t[g], with visible = min(floor(t[g]/m), N_cap):
+ *   I[s] = sum_{h < n_hI} wI[g][h] * max(0, qI[g][h] . KI[b][s])     for s < visible
+ *   idx_out[g] = the k indices s of largest I[s].  Ties go to the smaller s.  If
+ *   visible <= k, idx_out[g][s] = s for s < visible and -1 after.  Otherwise the k
+ *   indices are in unspecified order.
+ *
+ * qI         : [B, nq, n_hI, cI] (dtype)      wI : fp32 [B, nq, n_hI]
+ * KI         : [B, N_cap, cI] (dtype), compressed indexer keys
+ * t          : DEVICE int64 [B*nq] query token positions (read on the GPU, so a captured
+ *              CUDA graph can advance them between replays)
+ * idx_out    : int32 [B, nq, k]
+ * scores_out : fp32 [B, nq, k] score of each idx_out entry (-inf for padding), or NULL
+ * workspace  : >= csa_indexer_topk_workspace_size(B, nq, N_cap, k) bytes of device
+ *              memory, ZERO-FILLED before its first use (csa_workspace_zero).  Each
+ *              call leaves its counters zeroed again for the next call.
+ * Scores are fp32.  bf16 products are exact in fp32; sums accumulate in fp32 (tensor
+ * cores when dtype is bf16 and n_hI % 16 == 0, 16 <= n_hI <= 256, cI % 64 == 0,
+ * cI <= 256; CUDA cores otherwise).  Requires 1 <= k, N_cap < 2^31.
+ * ------------------------------------------------------------------------------- */
+size_t csa_indexer_topk_workspace_size(int B, int nq, int64_t N_cap, int k);
+int csa_indexer_topk(const void* qI, const float* wI, const void* KI, const int64_t* t,
+                     int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
+                     int32_t* idx_out, float* scores_out,
+                     void* workspace, size_t ws_bytes, int dtype, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * csa_sparse_attn - shared-KV multi-query attention over the selected compressed
+ * entries ([P1] section 8):
+ *   o[g][h] = sum_{s in idx[g]} softmax_s(scale * q[g][h] . C[b][s]) * C[b][s]
+ * key = value = the compressed entry.  scale <= 0 selects 1/sqrt(c).
+ *
+ * q     : [B, nq, n_h, c] (dtype)            cache : [B, N_cap, c] (dtype)
+ * idx   : int32 [B, nq, k]; values < 0 or >= N_cap are treated as padding (skipped)
+ * out   : [B, nq, n_h, c], fp32, or bf16 when out_bf16 != 0 (dtype must be bf16)
+ * lse   : fp32 [B, nq, n_h] natural-log sum of exp(scaled logits), or NULL
+ * A query with no valid entry gets out = 0 and lse = -inf.
+ * workspace : >= csa_attn_workspace_size(B, nq, n_h, c, k) bytes (no zeroing needed).
+ * Constraints: 1 <= c <= 512, n_h >= 1.
+ * ------------------------------------------------------------------------------- */
+size_t csa_attn_workspace_size(int B, int nq, int n_h, int c, int64_t max_entries);
+int csa_sparse_attn(const void* q, const void* cache, const int32_t* idx,
+                    int B, int nq, int n_h, int c, int64_t N_cap, int k, float scale,
+                    void* out, float* lse, void* workspace, size_t ws_bytes,
+                    int dtype, int out_bf16, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * hca_dense_attn - dense shared-KV MQA over every visible HCA entry ([P1] section 10,
+ * "every query attends to all compressed blocks densely"; causal rule s < floor(t/m')).
+ * Same arguments as csa_sparse_attn with the index list replaced by the visible range
+ * [0, min(floor(t[g]/m_prime), N_cap)) read from the DEVICE int64 array t [B*nq].
+ * workspace : >= csa_attn_workspace_size(B, nq, n_h, c, N_cap) bytes.
+ * ------------------------------------------------------------------------------- */
+int hca_dense_attn(const void* q, const void* cache, const int64_t* t,
+                   int B, int nq, int n_h, int c, int64_t N_cap, int m_prime, float scale,
+                   void* out, float* lse, void* workspace, size_t ws_bytes,
+                   int dtype, int out_bf16, csa_stream_t stream);
+
+/* Zero `bytes` of device memory on `stream` (cudaMemsetAsync); for first-use workspaces. */
+int csa_workspace_zero(void* workspace, size_t bytes, csa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_B200_H */

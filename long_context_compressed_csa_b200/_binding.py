@@ -1,0 +1,192 @@
+"""ctypes marshalling for libcsa_b200.so: pointers, sizes and the current stream only."""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libcsa_b200.so")
+
+CSA_BF16 = 0
+CSA_F32 = 1
+
+_lock = threading.Lock()
+_lib = None
+
+i32, i64, f32, vp, sz = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+_SIGS = {
+    "csa_status_string": ([i32], ctypes.c_char_p),
+    "csa_version": ([], i32),
+    "csa_workspace_zero": ([vp, sz, vp], i32),
+    "csa_compress": ([vp, vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, i64, i32, i32, i32, i64, i64,
+                      i32, vp], i32),
+    "hca_compress": ([vp, vp, i64, i64, i64, i64, vp, vp, i64, i32, i32, i32, i64, i64, i32, vp], i32),
+    "csa_indexer_topk_workspace_size": ([i32, i32, i64, i32], sz),
+    "csa_indexer_topk": ([vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, i32, vp, vp, vp, sz, i32, vp],
+                         i32),
+    "csa_attn_workspace_size": ([i32, i32, i32, i32, i64], sz),
+    "csa_sparse_attn": ([vp, vp, vp, i32, i32, i32, i32, i64, i32, f32, vp, vp, vp, sz, i32, i32, vp],
+                        i32),
+    "hca_dense_attn": ([vp, vp, vp, i32, i32, i32, i32, i64, i32, f32, vp, vp, vp, sz, i32, i32, vp],
+                       i32),
+}
+
+
+class CSAError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (fn, csa_status_string(status), status))
+
+
+def library():
+    """Load libcsa_b200.so (raises if it has not been built: there is no fallback)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(library_path):
+                raise ImportError("libcsa_b200.so not found at %s; build it with "
+                                  "`python -m long_context_compressed_csa_b200.build`" % library_path)
+            lib = ctypes.CDLL(library_path)
+            for name, (args, res) in _SIGS.items():
+                fn = getattr(lib, name)
+                fn.argtypes = args
+                fn.restype = res
+            _lib = lib
+    return _lib
+
+
+def csa_status_string(status: int) -> str:
+    return library().csa_status_string(int(status)).decode()
+
+
+def csa_version() -> int:
+    return int(library().csa_version())
+
+
+def _check(fn, status):
+    if status != 0:
+        raise CSAError(fn, status)
+
+
+def _dtype(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return CSA_BF16
+    if t.dtype == torch.float32:
+        return CSA_F32
+    raise TypeError("unsupported dtype %s (bf16 or fp32)" % t.dtype)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+
+
+def csa_workspace_zero(ws, stream=None):
+    _cuda(ws)
+    _check("csa_workspace_zero", library().csa_workspace_zero(_ptr(ws), ws.numel() * ws.element_size(),
+                                                              _stream(stream)))
+
+
+def csa_compress(Ca, Cb, Za, Zb, out, m, entry_begin=0, entry_end=None, Ba=None, Bb=None,
+                 tok0=0, stream=None):
+    """CSA overlapped compression into ``out[:, entry_begin:entry_end]``.
+
+    Ca, Cb, Za, Zb: [B, rows, c] views (same strides, last dim contiguous) holding token
+    rows tok0 .. tok0+rows-1.  out: [B, N_cap, c] of the same dtype.  Ba, Bb: fp32 [m, c].
+    """
+    _cuda(Ca, Cb, Za, Zb, out, Ba, Bb)
+    B, rows, c = Ca.shape
+    for x in (Cb, Za, Zb):
+        assert x.shape == Ca.shape and x.stride() == Ca.stride() and x.dtype == Ca.dtype
+    assert Ca.stride(2) == 1 and out.stride(2) == 1 and out.dtype == Ca.dtype
+    n = tok0 + rows
+    if entry_end is None:
+        entry_end = n // m
+    assert out.shape[0] == B and out.shape[2] == c and out.shape[1] >= entry_end
+    _check("csa_compress", library().csa_compress(
+        _ptr(Ca), _ptr(Cb), _ptr(Za), _ptr(Zb), Ca.stride(1), Ca.stride(0), tok0, n,
+        _ptr(Ba), _ptr(Bb), _ptr(out), out.stride(0), B, c, m, entry_begin, entry_end,
+        _dtype(Ca), _stream(stream)))
+
+
+def hca_compress(C, Z, out, m_prime, entry_begin=0, entry_end=None, Bias=None, tok0=0,
+                 stream=None):
+    """HCA compression into ``out[:, entry_begin:entry_end]`` (see csa_compress)."""
+    _cuda(C, Z, out, Bias)
+    B, rows, c = C.shape
+    assert Z.shape == C.shape and Z.stride() == C.stride() and Z.dtype == C.dtype
+    assert C.stride(2) == 1 and out.stride(2) == 1 and out.dtype == C.dtype
+    n = tok0 + rows
+    if entry_end is None:
+        entry_end = n // m_prime
+    assert out.shape[0] == B and out.shape[2] == c and out.shape[1] >= entry_end
+    _check("hca_compress", library().hca_compress(
+        _ptr(C), _ptr(Z), C.stride(1), C.stride(0), tok0, n, _ptr(Bias), _ptr(out), out.stride(0),
+        B, c, m_prime, entry_begin, entry_end, _dtype(C), _stream(stream)))
+
+
+def csa_indexer_topk_workspace_size(B, nq, N_cap, k) -> int:
+    return int(library().csa_indexer_topk_workspace_size(B, nq, N_cap, k))
+
+
+def csa_indexer_topk(qI, wI, KI, t, m, k, idx_out, workspace, scores_out=None, stream=None):
+    """Indexer scores + top-k.  qI [B,nq,n_hI,cI], wI fp32 [B,nq,n_hI], KI [B,N_cap,cI],
+    t int64 [B,nq] (device), idx_out int32 [B,nq,k], workspace uint8 (zeroed once)."""
+    _cuda(qI, wI, KI, t, idx_out, workspace, scores_out)
+    B, nq, n_hI, cI = qI.shape
+    N_cap = KI.shape[1]
+    assert KI.shape == (B, N_cap, cI) and KI.is_contiguous() and qI.is_contiguous()
+    assert wI.shape == (B, nq, n_hI) and wI.is_contiguous()
+    assert t.numel() == B * nq and idx_out.shape == (B, nq, k) and idx_out.is_contiguous()
+    _check("csa_indexer_topk", library().csa_indexer_topk(
+        _ptr(qI), _ptr(wI), _ptr(KI), _ptr(t), B, nq, N_cap, n_hI, cI, m, k, _ptr(idx_out),
+        _ptr(scores_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _dtype(qI), _stream(stream)))
+
+
+def csa_attn_workspace_size(B, nq, n_h, c, max_entries) -> int:
+    return int(library().csa_attn_workspace_size(B, nq, n_h, c, max_entries))
+
+
+def csa_sparse_attn(q, cache, idx, out, workspace, lse=None, scale=0.0, stream=None):
+    """MQA of q [B,nq,n_h,c] over cache [B,N_cap,c] rows idx int32 [B,nq,k] (-1 = pad)."""
+    _cuda(q, cache, idx, out, workspace, lse)
+    B, nq, n_h, c = q.shape
+    N_cap = cache.shape[1]
+    k = idx.shape[2]
+    assert q.is_contiguous() and cache.is_contiguous() and idx.is_contiguous() and out.is_contiguous()
+    assert cache.shape[0] == B and cache.shape[2] == c and idx.shape[:2] == (B, nq) and out.shape == q.shape
+    out_bf16 = 1 if out.dtype.itemsize == 2 else 0
+    _check("csa_sparse_attn", library().csa_sparse_attn(
+        _ptr(q), _ptr(cache), _ptr(idx), B, nq, n_h, c, N_cap, k, float(scale), _ptr(out), _ptr(lse),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _dtype(q), out_bf16,
+        _stream(stream)))
+
+
+def hca_dense_attn(q, cache, t, m_prime, out, workspace, lse=None, scale=0.0, stream=None):
+    """Dense MQA of q [B,nq,n_h,c] over cache [B,N_cap,c] rows s < floor(t/m')."""
+    _cuda(q, cache, t, out, workspace, lse)
+    B, nq, n_h, c = q.shape
+    N_cap = cache.shape[1]
+    assert q.is_contiguous() and cache.is_contiguous() and out.is_contiguous()
+    assert t.numel() == B * nq and cache.shape[0] == B and cache.shape[2] == c and out.shape == q.shape
+    out_bf16 = 1 if out.dtype.itemsize == 2 else 0
+    _check("hca_dense_attn", library().hca_dense_attn(
+        _ptr(q), _ptr(cache), _ptr(t), B, nq, n_h, c, N_cap, m_prime, float(scale), _ptr(out),
+        _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(), _dtype(q),
+        out_bf16, _stream(stream)))

@@ -1,0 +1,326 @@
+// Shared-KV multi-query attention over compressed entries
+// ("DeepSeek-V4 Hybrid Attention: CSA and HCA from Scratch", section 8 for CSA over the
+// top-k set, section 10 for HCA over every visible entry; key = value = the entry,
+// logits scaled by 1/sqrt(c)).
+//
+// Split-KV decode: the entry list of each query is cut into `splits` ranges; each CTA
+// produces, for its heads, an unnormalised partial output O_i and its (max, sum) in the
+// base-2 domain, and a combine kernel merges the splits with the usual log-sum-exp
+// rescaling.  bf16 inputs with tensor-core shapes run the tcgen05 kernel (attn_tc.cu);
+// everything else (the fp32 exact path, odd shapes) runs the CUDA-core kernel here.
+#include "attn.cuh"
+
+namespace csa {
+
+AttnPlan attn_plan_cuda_core(int G, int n_h, int64_t entries)
+{
+    AttnPlan p;
+    p.head_groups = (n_h + kCcHeads - 1) / kCcHeads;
+    int64_t want = (2 * kNumSMs + (int64_t)G * p.head_groups - 1) / ((int64_t)G * p.head_groups);
+    int64_t max_splits = (entries + kCcChunk - 1) / kCcChunk;
+    if (max_splits < 1) max_splits = 1;
+    if (want > max_splits) want = max_splits;
+    if (want < 1) want = 1;
+    p.per_split = (entries + want - 1) / want;
+    p.per_split = (p.per_split + kCcChunk - 1) / kCcChunk * kCcChunk;
+    if (p.per_split < kCcChunk) p.per_split = kCcChunk;
+    p.splits = (int)((entries + p.per_split - 1) / p.per_split);
+    if (p.splits < 1) p.splits = 1;
+    return p;
+}
+
+size_t attn_ws_bytes(int G, int n_h, int c, int splits)
+{
+    return align_up((size_t)G * splits * n_h * c * sizeof(float), 256) +
+           align_up((size_t)G * splits * n_h * sizeof(float2), 256);
+}
+
+namespace {
+
+// ----------------------------------------------------------------------------------
+// CUDA-core split kernel.  CTA = (split, head group of kCcHeads heads, query).  The
+// chunk of kCcChunk entries is staged in shared memory as fp32 with a padded row
+// stride, so that lane-per-entry dot products and lane-per-column accumulation are both
+// bank-conflict free.  Each warp owns kCcHeads/8 heads; a lane keeps c/32 output
+// columns of each of them in registers.
+// ----------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256)
+attn_cuda_core(AttnArgs a)
+{
+    extern __shared__ float smem[];
+    constexpr int HPW = kCcHeads / 8;  // heads per warp
+    constexpr int CPL = kMaxC / 32;    // output columns per lane
+    const int c = a.c;
+    const int cs = c + 1;                    // padded row stride
+    float* sC = smem;                        // [kCcChunk][cs]
+    float* sQ = smem + kCcChunk * cs;        // [kCcHeads][c]
+    __shared__ int s_ent[kCcChunk];
+
+    const int split = blockIdx.x, hg = blockIdx.y, g = blockIdx.z;
+    const int64_t b = g / a.nq;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h_base = hg * kCcHeads;
+
+    int64_t count;  // number of list positions for this query
+    if (a.dense) {
+        const int64_t tt = a.t[g];
+        const int64_t v = tt < 0 ? 0 : tt / a.m_prime;
+        count = v < a.N_cap ? v : a.N_cap;
+    } else {
+        count = a.k;
+    }
+    const int64_t p_begin = (int64_t)split * a.per_split;
+    const int64_t p_end = min(count, p_begin + a.per_split);
+
+    // stage q rows of this head group
+    const T* qg = static_cast<const T*>(a.q) + ((int64_t)g * a.n_h) * c;
+    for (int i = threadIdx.x; i < kCcHeads * c; i += 256) {
+        const int hh = i / c, j = i % c;
+        sQ[i] = (h_base + hh < a.n_h) ? to_f32(qg[(int64_t)(h_base + hh) * c + j]) : 0.f;
+    }
+
+    float m_run[HPW], l_run[HPW], o[HPW][CPL];
+#pragma unroll
+    for (int x = 0; x < HPW; ++x) {
+        m_run[x] = -INFINITY;
+        l_run[x] = 0.f;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) o[x][i] = 0.f;
+    }
+
+    const T* cache = static_cast<const T*>(a.cache) + b * a.N_cap * c;
+    for (int64_t p0 = p_begin; p0 < p_end; p0 += kCcChunk) {
+        __syncthreads();  // previous chunk fully consumed (and sQ staged on entry)
+        if (threadIdx.x < kCcChunk) {
+            const int64_t p = p0 + threadIdx.x;
+            int e = -1;
+            if (p < p_end) {
+                if (a.dense) {
+                    e = (int)p;
+                } else {
+                    const int32_t v = a.idx[(int64_t)g * a.k + p];
+                    e = (v >= 0 && v < a.N_cap) ? v : -1;
+                }
+            }
+            s_ent[threadIdx.x] = e;
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < kCcChunk * c; i += 256) {
+            const int r = i / c, j = i % c;
+            const int e = s_ent[r];
+            sC[r * cs + j] = e >= 0 ? to_f32(cache[(int64_t)e * c + j]) : 0.f;
+        }
+        __syncthreads();
+        const bool valid = s_ent[lane] >= 0;
+#pragma unroll
+        for (int x = 0; x < HPW; ++x) {
+            const int hh = warp * HPW + x;
+            const float* qr = sQ + hh * c;
+            const float* cr = sC + lane * cs;
+            float dot = 0.f;
+            for (int j = 0; j < c; ++j) dot = fmaf(qr[j], cr[j], dot);
+            const float logit = valid ? dot * a.scale_log2 : -INFINITY;
+            float cmax = logit;
+#pragma unroll
+            for (int off = 16; off; off >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, off));
+            const float m_new = fmaxf(m_run[x], cmax);
+            if (m_new == -INFINITY) continue;  // nothing valid yet
+            const float alpha = exp2f(m_run[x] - m_new);
+            const float pl = valid ? exp2f(logit - m_new) : 0.f;
+            float psum = pl;
+#pragma unroll
+            for (int off = 16; off; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
+            l_run[x] = l_run[x] * alpha + psum;
+            m_run[x] = m_new;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) o[x][i] *= alpha;
+            for (int e = 0; e < kCcChunk; ++e) {
+                const float pe = __shfl_sync(0xffffffffu, pl, e);
+                const float* ce = sC + e * cs;
+#pragma unroll
+                for (int i = 0; i < CPL; ++i) {
+                    const int j = lane + 32 * i;
+                    if (j < c) o[x][i] = fmaf(pe, ce[j], o[x][i]);
+                }
+            }
+        }
+    }
+
+    // write partials: O_i unnormalised, (m, l) in base-2 units of the scaled logits
+#pragma unroll
+    for (int x = 0; x < HPW; ++x) {
+        const int h = h_base + warp * HPW + x;
+        if (h >= a.n_h) continue;
+        const size_t row = ((size_t)g * a.splits + split) * a.n_h + h;
+        float* po = a.part_o + row * c;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int j = lane + 32 * i;
+            if (j < c) po[j] = o[x][i];
+        }
+        if (lane == 0) a.part_ml[row] = make_float2(m_run[x], l_run[x]);
+    }
+}
+
+// ----------------------------------------------------------------------------------
+// combine: out[g][h] = sum_i 2^(m_i - M) O_i / sum_i 2^(m_i - M) l_i ; lse in natural log
+// ----------------------------------------------------------------------------------
+template <typename TO>
+__global__ void __launch_bounds__(128)
+attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_ml, int splits,
+             int n_h, int c, TO* __restrict__ out, float* __restrict__ lse)
+{
+    const int h = blockIdx.x, g = blockIdx.y;
+    __shared__ float s_w[kMaxSplits];
+    __shared__ float s_inv;
+    const size_t base = (size_t)g * splits * n_h + h;
+    if (threadIdx.x < 32) {
+        float M = -INFINITY;
+        for (int i = threadIdx.x; i < splits; i += 32) M = fmaxf(M, part_ml[base + (size_t)i * n_h].x);
+#pragma unroll
+        for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        float L = 0.f;
+        for (int i = threadIdx.x; i < splits; i += 32) {
+            const float2 ml = part_ml[base + (size_t)i * n_h];
+            const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+            s_w[i] = w;
+            L += w * ml.y;
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+        if (threadIdx.x == 0) {
+            s_inv = L > 0.f ? 1.f / L : 0.f;
+            if (lse) lse[(size_t)g * n_h + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+        }
+    }
+    __syncthreads();
+    const float inv = s_inv;
+    for (int j = threadIdx.x; j < c; j += blockDim.x) {
+        float acc = 0.f;
+        for (int i = 0; i < splits; ++i) {
+            const float w = s_w[i];
+            if (w != 0.f) acc = fmaf(w, part_o[(base + (size_t)i * n_h) * c + j], acc);
+        }
+        const float v = acc * inv;
+        if constexpr (sizeof(TO) == 2)
+            out[((size_t)g * n_h + h) * c + j] = __float2bfloat16_rn(v);
+        else
+            out[((size_t)g * n_h + h) * c + j] = v;
+    }
+}
+
+int launch_cuda_core(AttnArgs a, const AttnPlan& plan, int dtype, cudaStream_t stream)
+{
+    a.splits = plan.splits;
+    a.per_split = plan.per_split;
+    const int G = a.B * a.nq;
+    dim3 grid((unsigned)plan.splits, (unsigned)plan.head_groups, (unsigned)G);
+    const size_t smem = ((size_t)kCcChunk * (a.c + 1) + (size_t)kCcHeads * a.c) * sizeof(float);
+    if (dtype == CSA_BF16) {
+        auto kern = attn_cuda_core<__nv_bfloat16>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kern<<<grid, 256, smem, stream>>>(a);
+    } else {
+        auto kern = attn_cuda_core<float>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kern<<<grid, 256, smem, stream>>>(a);
+    }
+    return launch_status();
+}
+
+}  // namespace
+
+int launch_attn_combine(const AttnArgs& a, void* out, int out_bf16, float* lse,
+                        cudaStream_t stream)
+{
+    const int G = a.B * a.nq;
+    dim3 grid((unsigned)a.n_h, (unsigned)G);
+    if (out_bf16)
+        attn_combine<__nv_bfloat16><<<grid, 128, 0, stream>>>(
+            a.part_o, a.part_ml, a.splits, a.n_h, a.c, static_cast<__nv_bfloat16*>(out), lse);
+    else
+        attn_combine<float><<<grid, 128, 0, stream>>>(a.part_o, a.part_ml, a.splits, a.n_h, a.c,
+                                                      static_cast<float*>(out), lse);
+    return launch_status();
+}
+
+// Shared host path of both exports.
+int attn_run(AttnArgs a, float scale, void* out, float* lse, void* workspace, size_t ws_bytes,
+             int dtype, int out_bf16, int64_t entries, cudaStream_t stream)
+{
+    if (dtype != CSA_BF16 && dtype != CSA_F32) return CSA_ERR_DTYPE;
+    if (out_bf16 && dtype != CSA_BF16) return CSA_ERR_DTYPE;
+    if (a.B < 0 || a.nq < 0 || a.n_h <= 0 || a.c <= 0 || a.N_cap < 0 || entries < 0)
+        return CSA_ERR_ARG;
+    if (a.c > kMaxC) return CSA_ERR_UNSUPPORTED;
+    if (a.B == 0 || a.nq == 0) return CSA_OK;
+    if (!a.q || !a.cache || !out || (!a.dense && !a.idx) || (a.dense && !a.t)) return CSA_ERR_ARG;
+    const uintptr_t eb = (uintptr_t)elem_bytes(dtype) - 1;
+    if ((((uintptr_t)a.q | (uintptr_t)a.cache) & eb) || ((uintptr_t)out & (out_bf16 ? 1 : 3)) ||
+        ((uintptr_t)lse & 3) || ((uintptr_t)a.idx & 3) || ((uintptr_t)a.t & 7))
+        return CSA_ERR_ALIGN;
+    const int G = a.B * a.nq;
+    if (!workspace || ws_bytes < csa_attn_workspace_size(a.B, a.nq, a.n_h, a.c, entries))
+        return CSA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return CSA_ERR_ALIGN;
+    a.scale_log2 = (scale > 0.f ? scale : 1.0f / sqrtf((float)a.c)) * kLog2e;
+
+    const bool tc = dtype == CSA_BF16 && attn_tc_supported(a.n_h, a.c);
+    AttnPlan plan = tc ? attn_plan_tc(G, a.n_h, a.c, entries) : attn_plan_cuda_core(G, a.n_h, entries);
+    char* ws = static_cast<char*>(workspace);
+    a.part_o = reinterpret_cast<float*>(ws);
+    a.part_ml = reinterpret_cast<float2*>(ws + align_up((size_t)G * plan.splits * a.n_h * a.c * sizeof(float), 256));
+    a.splits = plan.splits;
+    a.per_split = plan.per_split;
+    int st = tc ? launch_attn_tc(a, plan, stream) : launch_cuda_core(a, plan, dtype, stream);
+    if (st != CSA_OK) return st;
+    return launch_attn_combine(a, out, out_bf16, lse, stream);
+}
+
+}  // namespace csa
+
+extern "C" size_t csa_attn_workspace_size(int B, int nq, int n_h, int c, int64_t max_entries)
+{
+    using namespace csa;
+    if (B <= 0 || nq <= 0 || n_h <= 0 || c <= 0 || max_entries < 0) return 0;
+    const int G = B * nq;
+    AttnPlan p1 = attn_plan_cuda_core(G, n_h, max_entries);
+    size_t bytes = attn_ws_bytes(G, n_h, c, p1.splits);
+    if (attn_tc_supported(n_h, c)) {
+        AttnPlan p2 = attn_plan_tc(G, n_h, c, max_entries);
+        size_t b2 = attn_ws_bytes(G, n_h, c, p2.splits);
+        if (b2 > bytes) bytes = b2;
+    }
+    return bytes;
+}
+
+extern "C" int csa_sparse_attn(const void* q, const void* cache, const int32_t* idx, int B,
+                               int nq, int n_h, int c, int64_t N_cap, int k, float scale,
+                               void* out, float* lse, void* workspace, size_t ws_bytes,
+                               int dtype, int out_bf16, csa_stream_t stream)
+{
+    using namespace csa;
+    if (k < 0) return CSA_ERR_ARG;
+    AttnArgs a{};
+    a.q = q; a.cache = cache; a.idx = idx; a.t = nullptr;
+    a.B = B; a.nq = nq; a.n_h = n_h; a.c = c; a.N_cap = N_cap; a.k = k; a.m_prime = 1;
+    a.dense = 0;
+    return attn_run(a, scale, out, lse, workspace, ws_bytes, dtype, out_bf16, k,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int hca_dense_attn(const void* q, const void* cache, const int64_t* t, int B, int nq,
+                              int n_h, int c, int64_t N_cap, int m_prime, float scale, void* out,
+                              float* lse, void* workspace, size_t ws_bytes, int dtype,
+                              int out_bf16, csa_stream_t stream)
+{
+    using namespace csa;
+    if (m_prime <= 0) return CSA_ERR_ARG;
+    AttnArgs a{};
+    a.q = q; a.cache = cache; a.idx = nullptr; a.t = t;
+    a.B = B; a.nq = nq; a.n_h = n_h; a.c = c; a.N_cap = N_cap; a.k = 0; a.m_prime = m_prime;
+    a.dense = 1;
+    return attn_run(a, scale, out, lse, workspace, ws_bytes, dtype, out_bf16, N_cap,
+                    reinterpret_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,44 @@
+// Internal interface of the attention kernels (split-KV partials + combine).
+#pragma once
+#include "common.cuh"
+
+namespace csa {
+
+constexpr int kMaxC = 512;        // widest compressed entry the kernels hold on chip
+constexpr int kMaxSplits = 1024;  // splits per query the combine kernel accepts
+constexpr int kCcHeads = 16;      // CUDA-core kernel: heads per CTA
+constexpr int kCcChunk = 32;      // CUDA-core kernel: entries per shared-memory chunk
+
+struct AttnArgs {
+    const void* q;        // [G][n_h][c]
+    const void* cache;    // [B][N_cap][c]
+    const int32_t* idx;   // sparse: [G][k]
+    const int64_t* t;     // dense: [G] query positions (device)
+    int B, nq, n_h, c;
+    int64_t N_cap;
+    int k, m_prime;
+    int dense;
+    float scale_log2;     // softmax scale * log2(e)
+    int splits;
+    int64_t per_split;    // list positions per split
+    float* part_o;        // [G][splits][n_h][c]
+    float2* part_ml;      // [G][splits][n_h] (max, sum) of 2^(scaled logit)
+};
+
+struct AttnPlan {
+    int splits = 1;
+    int64_t per_split = 1;
+    int head_groups = 1;
+};
+
+AttnPlan attn_plan_cuda_core(int G, int n_h, int64_t entries);
+AttnPlan attn_plan_tc(int G, int n_h, int c, int64_t entries);
+bool attn_tc_supported(int n_h, int c);
+size_t attn_ws_bytes(int G, int n_h, int c, int splits);
+int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, cudaStream_t stream);
+int launch_attn_combine(const AttnArgs& a, void* out, int out_bf16, float* lse,
+                        cudaStream_t stream);
+
+}  // namespace csa
+
+extern "C" size_t csa_attn_workspace_size(int B, int nq, int n_h, int c, int64_t max_entries);

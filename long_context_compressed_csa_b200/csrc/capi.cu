@@ -1,0 +1,26 @@
+// Status strings, version and workspace helpers of the C ABI.
+#include "common.cuh"
+
+extern "C" const char* csa_status_string(int status)
+{
+    switch (status) {
+        case CSA_OK: return "CSA_OK";
+        case CSA_ERR_ARG: return "CSA_ERR_ARG: null pointer, negative or inconsistent size";
+        case CSA_ERR_ALIGN: return "CSA_ERR_ALIGN: pointer or stride not 16-byte aligned";
+        case CSA_ERR_DTYPE: return "CSA_ERR_DTYPE: unknown dtype or output type";
+        case CSA_ERR_WORKSPACE: return "CSA_ERR_WORKSPACE: workspace missing or too small";
+        case CSA_ERR_CUDA: return "CSA_ERR_CUDA: CUDA launch or runtime error";
+        case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED: shape not implemented";
+        default: return "CSA_ERR_UNKNOWN";
+    }
+}
+
+extern "C" int csa_version(void) { return 100; }
+
+extern "C" int csa_workspace_zero(void* workspace, size_t bytes, csa_stream_t stream)
+{
+    if (bytes == 0) return CSA_OK;
+    if (!workspace) return CSA_ERR_ARG;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, bytes, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+}

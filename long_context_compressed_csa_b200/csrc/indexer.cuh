@@ -1,0 +1,35 @@
+// Internal interface between the indexer scan kernels and the top-k select kernel.
+#pragma once
+#include "common.cuh"
+
+namespace csa {
+
+constexpr int kBins = 4096;  // 12-bit radix digits
+constexpr int kCtrs = 8;     // per query: [0] emitted, [1] candidates, [2] ticket
+
+// Workspace of csa_indexer_topk, carved from one caller buffer.
+struct TopkWs {
+    uint32_t* hist0;  // [G][kBins] digit-0 histogram (zero between calls)
+    uint32_t* hist1;  // [G][kBins] digit-1 histogram of the candidates (zero between calls)
+    uint32_t* ctr;    // [G][kCtrs] counters (zero between calls)
+    float* scores;    // [G][ld] fp32 scores of the visible entries
+    uint2* cand;      // [G][ld] (score key, index) candidates
+    uint2* cand2;     // [G][ld] second candidate buffer
+    int64_t ld;       // per-query stride of scores / cand (N_cap rounded up to 64)
+    size_t bytes;     // total bytes used
+    size_t zero_bytes;  // leading bytes that must be zero before a call
+};
+
+TopkWs topk_ws_layout(void* base, int G, int64_t N_cap);
+
+bool indexer_tc_supported(int n_hI, int cI);
+int launch_scan_tc(const void* qI, const float* wI, const void* KI, const int64_t* t, int B,
+                   int nq, int64_t N_cap, int n_hI, int cI, int m, int k, const TopkWs& ws,
+                   cudaStream_t stream);
+int launch_scan_cuda_core(const void* qI, const float* wI, const void* KI, const int64_t* t,
+                          int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
+                          const TopkWs& ws, int dtype, cudaStream_t stream);
+int launch_topk_select(const TopkWs& ws, const int64_t* t, int G, int m, int k, int64_t N_cap,
+                       int32_t* idx_out, float* scores_out, cudaStream_t stream);
+
+}  // namespace csa

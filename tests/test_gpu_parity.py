@@ -1,0 +1,372 @@
+"""GPU parity: every C-ABI entry point against the fp64 CPU oracle on seeded inputs.
+
+Tolerances (stated by the workload's target): attention outputs within 2e-2 max
+relative error per (query, head) row for bf16 inputs with fp32 accumulation, 1e-5 for
+the fp32 path; compressed entries by the same metric per entry; top-k index sets
+identical except for near-ties (tests/helpers.check_topk_sets).  Integer-valued inputs
+make every score exact in fp32 and fp64 alike, so there the top-k sets, tie order
+included, must match exactly.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_compressed_csa_b200 import (csa_attn_workspace_size, csa_compress,
+                                              csa_indexer_topk, csa_indexer_topk_workspace_size,
+                                              csa_sparse_attn, csa_workspace_zero, hca_compress,
+                                              hca_dense_attn)
+from long_context_compressed_csa_b200.synth import randint_values, randn, to_f64
+from tests.helpers import check_topk_sets, max_rel_rowwise, score_error_bound
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+TOL = {torch.bfloat16: 2e-2, torch.float32: 1e-5}
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_example.json")))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from long_context_compressed_csa_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def gv(name):
+    return torch.tensor(GOLD[name]["value"], dtype=torch.float32)
+
+
+def dev(x):
+    return x.to(DEV).contiguous()
+
+
+# ==================================================================================
+# compression
+# ==================================================================================
+def run_csa_compress(Ca, Cb, Za, Zb, m, Ba=None, Bb=None, i0=0, i1=None, tok0=0, N_cap=None):
+    B, rows, c = Ca.shape
+    n = tok0 + rows
+    if i1 is None:
+        i1 = n // m
+    N_cap = N_cap or max(i1, 1)
+    out = torch.full((B, N_cap, c), float("nan"), dtype=Ca.dtype, device=DEV)
+    csa_compress(Ca, Cb, Za, Zb, out, m, i0, i1, Ba=Ba, Bb=Bb, tok0=tok0)
+    torch.cuda.synchronize()
+    return out
+
+
+def test_worked_example_compressors_fp32():
+    H = gv("H")
+    Ca = dev(H @ gv("W_aKV"))[None]
+    Cb = dev(H @ gv("W_bKV"))[None]
+    Za = dev(H @ gv("W_aZ"))[None]
+    Zb = dev(H @ gv("W_bZ"))[None]
+    out = run_csa_compress(Ca, Cb, Za, Zb, m=2)[0].cpu().double().numpy()
+    e = math.e
+    want = [[e / (e + 1), 1.0], [(4 * e**2 + e) / (2 * e**2 + e + 1), 0.75], [3 * e / (1 + 3 * e), 1.0]]
+    np.testing.assert_allclose(out, want, rtol=1e-6, atol=1e-6)
+    np.testing.assert_allclose(out[:2], GOLD["csa_entries"]["value"], atol=3e-3)
+    hout = torch.full((1, 2, 2), float("nan"), device=DEV)
+    hca_compress(Ca, Za, hout, 3)
+    h = hout[0].cpu().double().numpy()
+    np.testing.assert_allclose(h, [[(e + 2 * e**2) / (1 + e + e**2), 1.0], [2 * e / (2 * e + 1), 2 / 3]],
+                               rtol=1e-6, atol=1e-6)
+
+
+@pytest.mark.parametrize("dtype,c,m", [(torch.bfloat16, 512, 4), (torch.float32, 512, 4),
+                                       (torch.bfloat16, 136, 3), (torch.float32, 6, 2),
+                                       (torch.bfloat16, 3, 4), (torch.bfloat16, 128, 1)])
+def test_csa_compress_random(dtype, c, m):
+    B, n = 2, 37 * m + m - 1          # ragged: a trailing partial block is not compressed
+    S = [randn((B, n, c), 100 + i, dtype) for i in range(4)]
+    Ba = randn((m, c), 110, torch.float32)
+    Bb = randn((m, c), 111, torch.float32)
+    out = run_csa_compress(*(dev(x) for x in S), m, Ba=dev(Ba), Bb=dev(Bb))
+    N = n // m
+    for b in range(B):
+        ref = oracle.csa_compress(*(to_f64(x[b]) for x in S), m, Ba=to_f64(Ba), Bb=to_f64(Bb))
+        err = max_rel_rowwise(out[b, :N].cpu().double().numpy(), ref)
+        assert err.max() <= TOL[dtype], err.max()
+
+
+def test_csa_compress_interleaved_layout_and_incremental_ranges():
+    """One [n, 4c] projection buffer (ld_row = 4c), then decode-style single entries
+    computed from a window of rows that starts at tok0 > 0."""
+    B, n, c, m = 2, 64, 128, 4
+    P = randn((B, n, 4 * c), 120, torch.bfloat16)
+    Pd = dev(P)
+    Ca, Cb, Za, Zb = (Pd[:, :, i * c:(i + 1) * c] for i in range(4))
+    full = run_csa_compress(Ca, Cb, Za, Zb, m, N_cap=n // m)
+    for b in range(B):
+        ref = oracle.csa_compress(*(to_f64(P[b, :, i * c:(i + 1) * c]) for i in range(4)), m)
+        assert max_rel_rowwise(full[b].cpu().double().numpy(), ref).max() <= 2e-2
+    # entry i from rows m(i-1) .. m(i+1)-1 only (a ring of the last 2m token rows)
+    for i in (1, 7, 15):
+        lo = m * (i - 1)
+        win = Pd[:, lo:m * (i + 1)]
+        part = run_csa_compress(*(win[:, :, j * c:(j + 1) * c] for j in range(4)), m, i0=i,
+                                i1=i + 1, tok0=lo, N_cap=n // m)
+        torch.testing.assert_close(part[:, i], full[:, i], rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("dtype,c,mp", [(torch.bfloat16, 512, 128), (torch.float32, 64, 128),
+                                        (torch.bfloat16, 24, 5)])
+def test_hca_compress_random(dtype, c, mp):
+    B, n = 3, 5 * mp + 17
+    C, Z = randn((B, n, c), 130, dtype), randn((B, n, c), 131, dtype)
+    Bias = randn((mp, c), 132, torch.float32)
+    N = n // mp
+    out = torch.full((B, N, c), float("nan"), dtype=dtype, device=DEV)
+    hca_compress(dev(C), dev(Z), out, mp, Bias=dev(Bias))
+    for b in range(B):
+        ref = oracle.hca_compress(to_f64(C[b]), to_f64(Z[b]), mp, Bias=to_f64(Bias))
+        assert max_rel_rowwise(out[b].cpu().double().numpy(), ref).max() <= TOL[dtype]
+    # one incremental entry from a window starting at tok0 = m' * i
+    i = 3
+    part = torch.zeros((B, N, c), dtype=dtype, device=DEV)
+    hca_compress(dev(C[:, mp * i:mp * (i + 1)]), dev(Z[:, mp * i:mp * (i + 1)]), part, mp, i, i + 1,
+                 Bias=dev(Bias), tok0=mp * i)
+    torch.testing.assert_close(part[:, i], out[:, i], rtol=0, atol=0)
+
+
+def test_compress_extreme_logits_one_hot():
+    B, n, c, m = 1, 32, 64, 4
+    Ca, Cb = randn((B, n, c), 140, torch.float32), randn((B, n, c), 141, torch.float32)
+    Za, Zb = torch.zeros(B, n, c), torch.zeros(B, n, c)
+    Za[0, 9, 5] = 80.0
+    Zb[0, 6, 7] = 80.0
+    out = run_csa_compress(dev(Ca), dev(Cb), dev(Za), dev(Zb), m)[0].cpu()
+    assert abs(out[2, 5] - Ca[0, 9, 5]) < 1e-5 and abs(out[2, 7] - Cb[0, 6, 7]) < 1e-5
+
+
+# ==================================================================================
+# indexer + top-k
+# ==================================================================================
+def run_indexer(qI, wI, KI, t, m, k, ws=None, scores=True):
+    B, nq = qI.shape[:2]
+    N_cap = KI.shape[1]
+    if ws is None:
+        ws = torch.zeros(csa_indexer_topk_workspace_size(B, nq, N_cap, k), dtype=torch.uint8, device=DEV)
+    idx = torch.full((B, nq, k), -7, dtype=torch.int32, device=DEV)
+    sc = torch.full((B, nq, k), float("nan"), dtype=torch.float32, device=DEV) if scores else None
+    tt = torch.tensor(t, dtype=torch.int64, device=DEV).reshape(B, nq)
+    csa_indexer_topk(qI, wI, KI, tt, m, k, idx, ws, scores_out=sc)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), (sc.cpu().numpy() if scores else None), ws
+
+
+def test_worked_example_indexer_fp32():
+    qI = dev(gv("qI_5").reshape(1, 1, 1, 2))
+    wI = dev(torch.ones(1, 1, 1))
+    KI = dev(gv("KI").reshape(1, 2, 2))
+    idx, sc, _ = run_indexer(qI, wI, KI, [5], m=2, k=1)
+    assert idx.tolist() == [[[1]]] and sc.tolist() == [[[1.0]]]
+    idx, sc, _ = run_indexer(qI, wI, KI, [5], m=2, k=2)
+    assert idx.tolist() == [[[0, 1]]] and sc.tolist() == [[[0.5, 1.0]]]
+    idx, _, _ = run_indexer(qI, wI, KI, [3], m=2, k=1)   # floor(3/2) = 1 visible
+    assert idx.tolist() == [[[0]]]
+
+
+@pytest.mark.parametrize("dtype,n_hI,cI", [(torch.bfloat16, 64, 128), (torch.bfloat16, 8, 24),
+                                           (torch.float32, 16, 32)])
+def test_indexer_topk_exact_on_integer_inputs(dtype, n_hI, cI):
+    """Small-integer q, K, w: every score is an exact integer in fp32, so the selected set
+    (with many exact ties resolved to the smaller index) must equal the oracle's."""
+    B, nq, N_cap, m, k = 2, 2, 3000, 4, 257
+    qI = randint_values((B, nq, n_hI, cI), 200, -2, 3, dtype)
+    KI = randint_values((B, N_cap, cI), 201, -2, 3, dtype)
+    wI = randint_values((B, nq, n_hI), 202, -2, 3, torch.float32)
+    t = [4 * N_cap, 4 * 700 + 3, 4 * 257 + 1, 4 * 100]     # vis: 3000, 700, 257 (= k), 100
+    idx, sc, ws = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k)
+    for b in range(B):
+        for q in range(nq):
+            g = b * nq + q
+            vis = oracle.visible(t[g], m, N_cap)
+            s = oracle.index_scores(to_f64(qI[b, q]), to_f64(wI[b, q]), to_f64(KI[b]), vis)
+            want = oracle.topk(s, k)
+            got = idx[b, q]
+            if vis <= k:
+                assert got.tolist() == want.tolist()
+            else:
+                assert sorted(got.tolist()) == sorted(want.tolist())
+            ok = got >= 0
+            np.testing.assert_array_equal(sc[b, q][ok], s[got[ok]])
+            assert np.all(np.isneginf(sc[b, q][~ok]))
+    # the workspace is left clean: a second call gives the same sets
+    idx2, _, _ = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k, ws=ws)
+    for g in range(B * nq):
+        assert sorted(idx2.reshape(-1, k)[g].tolist()) == sorted(idx.reshape(-1, k)[g].tolist())
+
+
+@pytest.mark.parametrize("dtype,n_hI,cI,N_cap,k", [(torch.bfloat16, 64, 128, 20000, 512),
+                                                   (torch.float32, 16, 32, 5000, 100),
+                                                   (torch.bfloat16, 32, 64, 1500, 1024)])
+def test_indexer_topk_random(dtype, n_hI, cI, N_cap, k):
+    B, nq, m = 1, 2, 4
+    qI = randn((B, nq, n_hI, cI), 210, dtype)
+    KI = randn((B, N_cap, cI), 211, dtype)
+    wI = randn((B, nq, n_hI), 212, torch.float32)
+    t = [4 * N_cap + 2, 4 * (N_cap // 2) + 1]
+    idx, sc, _ = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k)
+    for q in range(nq):
+        vis = oracle.visible(t[q], m, N_cap)
+        q64, w64, K64 = to_f64(qI[0, q]), to_f64(wI[0, q]), to_f64(KI[0])
+        s = oracle.index_scores(q64, w64, K64, vis)
+        check_topk_sets(idx[0, q], s, k, lambda d: score_error_bound(q64, w64, K64, d))
+        got = idx[0, q][idx[0, q] >= 0]
+        band = score_error_bound(q64, w64, K64, got) + 1e-6 * np.abs(s[got])
+        assert np.all(np.abs(sc[0, q][:len(got)] - s[got]) <= band)
+
+
+def test_indexer_degenerate_cases():
+    dtype, n_hI, cI, N_cap, m = torch.bfloat16, 64, 128, 700, 4
+    qI = randn((1, 3, n_hI, cI), 220, dtype)
+    KI = torch.zeros((1, N_cap, cI), dtype=dtype)      # all scores exactly 0: ties everywhere
+    wI = randn((1, 3, n_hI), 221, torch.float32)
+    idx, sc, _ = run_indexer(dev(qI), dev(wI), dev(KI), [0, 4 * 5, 4 * N_cap], m, 64)
+    assert idx[0, 0].tolist() == [-1] * 64                     # nothing visible
+    assert idx[0, 1].tolist() == list(range(5)) + [-1] * 59    # fewer visible than k
+    assert sorted(idx[0, 2].tolist()) == list(range(64))       # all tied: smallest indices
+    assert np.all(sc[0, 2] == 0)
+
+
+# ==================================================================================
+# attention
+# ==================================================================================
+def run_sparse(q, cache, idx, out_dtype=torch.float32, scale=0.0):
+    B, nq, n_h, c = q.shape
+    k = idx.shape[2]
+    ws = torch.empty(csa_attn_workspace_size(B, nq, n_h, c, k), dtype=torch.uint8, device=DEV)
+    out = torch.full((B, nq, n_h, c), float("nan"), dtype=out_dtype, device=DEV)
+    lse = torch.full((B, nq, n_h), float("nan"), device=DEV)
+    csa_sparse_attn(q, cache, idx, out, ws, lse=lse, scale=scale)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def run_dense(q, cache, t, mp, out_dtype=torch.float32):
+    B, nq, n_h, c = q.shape
+    N_cap = cache.shape[1]
+    ws = torch.empty(csa_attn_workspace_size(B, nq, n_h, c, N_cap), dtype=torch.uint8, device=DEV)
+    out = torch.full((B, nq, n_h, c), float("nan"), dtype=out_dtype, device=DEV)
+    lse = torch.full((B, nq, n_h), float("nan"), device=DEV)
+    tt = torch.tensor(t, dtype=torch.int64, device=DEV).reshape(B, nq)
+    hca_dense_attn(q, cache, tt, mp, out, ws, lse=lse)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def test_worked_example_attention_fp32():
+    e = math.e
+    C = torch.tensor([[e / (e + 1), 1.0], [(4 * e**2 + e) / (2 * e**2 + e + 1), 0.75],
+                      [3 * e / (1 + 3 * e), 1.0]], dtype=torch.float32)
+    q = dev(gv("cQ_5").reshape(1, 1, 1, 2))
+    o, lse = run_sparse(q, dev(C[None]), dev(torch.tensor([[[1]]], dtype=torch.int32)))
+    np.testing.assert_allclose(o[0, 0, 0], C[1].numpy(), rtol=1e-6)
+    np.testing.assert_allclose(o[0, 0, 0], GOLD["csa_output_k1"]["value"], atol=3e-3)
+    o, _ = run_sparse(q, dev(C[None]), dev(torch.tensor([[[0, 1]]], dtype=torch.int32)))
+    np.testing.assert_allclose(o[0, 0, 0], [1.412288, 0.832019], atol=2e-6)
+    Hc = torch.tensor([[(e + 2 * e**2) / (1 + e + e**2), 1.0], [2 * e / (2 * e + 1), 2 / 3]])
+    o, _ = run_dense(q, dev(Hc[None]), [5], 3)
+    np.testing.assert_allclose(o[0, 0, 0], Hc[0].numpy(), rtol=1e-6)
+
+
+def _ref_attn(q, cache, sel, scale=None):
+    out, lse = oracle.mqa(q, cache, sel, scale)
+    return out, lse
+
+
+@pytest.mark.parametrize("dtype,n_h,c,k", [(torch.bfloat16, 128, 512, 1024),
+                                           (torch.bfloat16, 128, 512, 200),
+                                           (torch.float32, 8, 64, 300),
+                                           (torch.bfloat16, 20, 40, 77)])
+def test_sparse_attn_random(dtype, n_h, c, k):
+    B, nq, N_cap = 2, 1, 3000
+    q = randn((B, nq, n_h, c), 300, dtype)
+    cache = randn((B, N_cap, c), 301, dtype)
+    g = torch.Generator().manual_seed(302)
+    idx = torch.stack([torch.randperm(N_cap, generator=g)[:k] for _ in range(B * nq)]).reshape(B, nq, k)
+    idx = idx.to(torch.int32)
+    idx[0, 0, ::7] = -1                                  # padding slots are skipped
+    o, lse = run_sparse(dev(q), dev(cache), dev(idx))
+    for b in range(B):
+        ref, ref_lse = _ref_attn(to_f64(q[b, 0]), to_f64(cache[b]), idx[b, 0].numpy())
+        assert max_rel_rowwise(o[b, 0], ref).max() <= TOL[dtype]
+        np.testing.assert_allclose(lse[b, 0], ref_lse, atol=2e-3 if dtype == torch.bfloat16 else 1e-5,
+                                   rtol=0)
+
+
+def test_sparse_attn_bf16_output_scale_and_empty():
+    B, nq, n_h, c, N_cap, k = 1, 2, 128, 512, 500, 64
+    q = randn((B, nq, n_h, c), 310, torch.bfloat16)
+    cache = randn((B, N_cap, c), 311, torch.bfloat16)
+    idx = torch.randint(0, N_cap, (B, nq, k), generator=torch.Generator().manual_seed(312)).to(torch.int32)
+    idx[0, 1] = -1                                       # query 1: nothing selected
+    o, lse = run_sparse(dev(q), dev(cache), dev(idx), out_dtype=torch.bfloat16, scale=0.03)
+    ref, ref_lse = _ref_attn(to_f64(q[0, 0]), to_f64(cache[0]), idx[0, 0].numpy(), 0.03)
+    assert max_rel_rowwise(o[0, 0], ref).max() <= 2e-2
+    np.testing.assert_allclose(lse[0, 0], ref_lse, atol=2e-3)
+    assert np.all(o[0, 1] == 0) and np.all(np.isneginf(lse[0, 1]))
+
+
+@pytest.mark.parametrize("dtype,n_h,c", [(torch.bfloat16, 128, 512), (torch.float32, 16, 64)])
+def test_dense_attn_random(dtype, n_h, c):
+    B, nq, N_cap, mp = 3, 1, 1024, 128
+    q = randn((B, nq, n_h, c), 320, dtype)
+    cache = randn((B, N_cap, c), 321, dtype)
+    t = [mp * N_cap + 5, mp * 333 + 127, 100]            # vis 1024, 333, 0
+    o, lse = run_dense(dev(q), dev(cache), t, mp)
+    for b in range(B):
+        vis = oracle.visible(t[b], mp, N_cap)
+        if vis == 0:
+            assert np.all(o[b, 0] == 0) and np.all(np.isneginf(lse[b, 0]))
+            continue
+        ref, ref_lse = _ref_attn(to_f64(q[b, 0]), to_f64(cache[b]), np.arange(vis, dtype=np.int32))
+        assert max_rel_rowwise(o[b, 0], ref).max() <= TOL[dtype]
+        np.testing.assert_allclose(lse[b, 0], ref_lse, atol=2e-3 if dtype == torch.bfloat16 else 1e-5,
+                                   rtol=0)
+
+
+# ==================================================================================
+# end to end: streams -> caches -> indexer/top-k -> sparse attention; HCA likewise
+# ==================================================================================
+def test_end_to_end_csa_and_hca_decode():
+    dtype = torch.bfloat16
+    B, n, m, mp, c, cI, n_h, n_hI, k = 1, 4096, 4, 128, 512, 128, 128, 64, 128
+    S = [randn((B, n, c), 400 + i, dtype) for i in range(4)]
+    SI = [randn((B, n, cI), 410 + i, dtype) for i in range(4)]
+    H = [randn((B, n, c), 420 + i, dtype) for i in range(2)]
+    q = randn((B, 1, n_h, c), 430, dtype)
+    qI = randn((B, 1, n_hI, cI), 431, dtype)
+    wI = randn((B, 1, n_hI), 432, torch.float32)
+    N, Nh, t = n // m, n // mp, n
+    cache = torch.empty((B, N, c), dtype=dtype, device=DEV)
+    kI = torch.empty((B, N, cI), dtype=dtype, device=DEV)
+    hcache = torch.empty((B, Nh, c), dtype=dtype, device=DEV)
+    csa_compress(*(dev(x) for x in S), cache, m)
+    csa_compress(*(dev(x) for x in SI), kI, m)
+    hca_compress(dev(H[0]), dev(H[1]), hcache, mp)
+    idx, _, _ = run_indexer(dev(qI), dev(wI), kI, [t], m, k)
+    o, _ = run_sparse(dev(q), cache, dev(torch.from_numpy(idx)))
+    oh, _ = run_dense(dev(q), hcache, [t], mp)
+
+    # oracle pipeline; caches stored in bf16 (round to nearest even) like the GPU's
+    ref_cache = oracle.round_bf16(oracle.csa_compress(*(to_f64(x[0]) for x in S), m))
+    ref_kI = oracle.round_bf16(oracle.csa_compress(*(to_f64(x[0]) for x in SI), m))
+    ref_h = oracle.round_bf16(oracle.hca_compress(to_f64(H[0][0]), to_f64(H[1][0]), mp))
+    assert max_rel_rowwise(cache[0].float().cpu().numpy(), ref_cache).max() <= 1e-2
+    q64, w64 = to_f64(qI[0, 0]), to_f64(wI[0, 0])
+    s = oracle.index_scores(q64, w64, ref_kI, oracle.visible(t, m, N))
+    band = lambda d: score_error_bound(q64, w64, ref_kI, d) + 1e-5 * np.abs(s[d])
+    ndiff = check_topk_sets(idx[0, 0], s, k, band)
+    sel = oracle.topk(s, k)
+    if ndiff == 0:
+        ref_o, _ = oracle.mqa(to_f64(q[0, 0]), ref_cache, sel)
+        assert max_rel_rowwise(o[0, 0], ref_o).max() <= 2e-2
+    ref_oh, _ = oracle.mqa(to_f64(q[0, 0]), ref_h, np.arange(oracle.visible(t, mp, Nh), dtype=np.int32))
+    assert max_rel_rowwise(oh[0, 0], ref_oh).max() <= 2e-2
