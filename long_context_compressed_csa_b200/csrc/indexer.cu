@@ -381,13 +381,13 @@ int launch_scan_cuda_core(const void* qI, const float* wI, const void* KI, const
     const bool vec = cI % (16 / elem_bytes(dtype)) == 0 && aligned16(KI);
     if (dtype == CSA_BF16) {
         auto kern = vec ? scan_cuda_core<__nv_bfloat16, 8> : scan_cuda_core<__nv_bfloat16, 1>;
-        if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         kern<<<grid, kScanThreads, smem, stream>>>(static_cast<const __nv_bfloat16*>(qI), wI,
                                                    static_cast<const __nv_bfloat16*>(KI), t, nq,
                                                    N_cap, n_hI, cI, m, k, ws);
     } else {
         auto kern = vec ? scan_cuda_core<float, 4> : scan_cuda_core<float, 1>;
-        if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         kern<<<grid, kScanThreads, smem, stream>>>(static_cast<const float*>(qI), wI,
                                                    static_cast<const float*>(KI), t, nq, N_cap,
                                                    n_hI, cI, m, k, ws);

@@ -190,8 +190,9 @@ def test_indexer_topk_exact_on_integer_inputs(dtype, n_hI, cI):
             s = oracle.index_scores(to_f64(qI[b, q]), to_f64(wI[b, q]), to_f64(KI[b]), vis)
             want = oracle.topk(s, k)
             got = idx[b, q]
-            if vis <= k:
-                assert got.tolist() == want.tolist()
+            if vis <= k:   # all visible, in index order, -1 padded
+                assert got.tolist() == list(range(vis)) + [-1] * (k - vis)
+                assert sorted(want[:vis].tolist()) == list(range(vis))
             else:
                 assert sorted(got.tolist()) == sorted(want.tolist())
             ok = got >= 0
