@@ -177,8 +177,8 @@ class HybridDecode:
             lib.hca_compress(H[0], H[1], P["hcache"], mp, lo // mp, hi // mp, tok0=lo)
             del H
 
-    # one step: token j through layer pair p
-    def step(self, p, j, q=None, qh=None, qI=None, wI=None, events=None):
+    # one step: token j through layer pair p (part 0: indexer + top-k, part 1: the rest)
+    def step(self, p, j, q=None, qh=None, qI=None, wI=None, part=None):
         lib = self.lib
         P = self.pairs[p]
         qs = j % self.nQ
@@ -187,11 +187,10 @@ class HybridDecode:
         qI = self.qI[qs] if qI is None else qI
         wI = self.wI[qs] if wI is None else wI
         t = self.tpos[j]
-        if events is not None:
-            events[0].record()
-        lib.csa_indexer_topk(qI, wI, P["kI"], t, self.m, self.k, self.idx, self.ws_topk)
-        if events is not None:
-            events[1].record()
+        if part in (None, 0):
+            lib.csa_indexer_topk(qI, wI, P["kI"], t, self.m, self.k, self.idx, self.ws_topk)
+        if part == 0:
+            return
         lib.csa_sparse_attn(q, P["cache"], self.idx, self.o, self.ws_attn)
         lib.hca_dense_attn(qh, P["hcache"], t, self.mp, self.oh, self.ws_hattn)
         tok = self.n + j
@@ -309,14 +308,17 @@ def main():
     dec = HybridDecode(torch, W + K, seed=5000 + 17 * rank)
     stream = torch.cuda.current_stream()
 
-    # ---- capture one CUDA graph per step (every pointer and position is baked in) ----
+    # ---- capture CUDA graphs per step (every pointer and position is baked in): one for
+    # the indexer call, one for the rest, so events between them time the indexer ----
     def make_graph(j_step):
         p, j = j_step % N_PAIRS, j_step // N_PAIRS
-        g = torch.cuda.CUDAGraph()
+        ga, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ga):
+            dec.step(p, j, part=0)
+        with torch.cuda.graph(gb):
+            dec.step(p, j, part=1)
         ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-        with torch.cuda.graph(g):
-            dec.step(p, j, events=ev)
-        return g, ev
+        return ga, gb, ev
 
     # eager warm-up of every code path once (outside any graph), then build graphs
     for s in range(min(W, 8)):
@@ -331,6 +333,7 @@ def main():
 
     for s in range(W):
         graphs[s][0].replay()
+        graphs[s][1].replay()
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
@@ -341,14 +344,18 @@ def main():
     torch.cuda.synchronize()
     start.record()
     for s in range(W, W + K):
-        graphs[s][0].replay()
+        ga, gb, ev = graphs[s]
+        ev[0].record()
+        ga.replay()
+        ev[1].record()
+        gb.replay()
     end.record()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
     ms = start.elapsed_time(end)
-    idx_ms = np.array([graphs[s][1][0].elapsed_time(graphs[s][1][1]) for s in range(W, W + K)])
+    idx_ms = np.array([graphs[s][2][0].elapsed_time(graphs[s][2][1]) for s in range(W, W + K)])
     t_max = torch.tensor([ms], dtype=torch.float64, device="cuda")
     if world > 1:
         dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
@@ -356,6 +363,8 @@ def main():
 
     bytes_total = sum(dec.step_bytes(s // N_PAIRS) for s in range(W, W + K))
     launches = sum(kernel_launches_per_step(dec, s // N_PAIRS) for s in range(W, W + K))
+    log("indexer+topk per launch: mean %.2f us, median %.2f us; step %.2f us" %
+        (idx_ms.mean() * 1e3, np.median(idx_ms) * 1e3, ms * 1e3 / K))
     hbm, tf, src = peaks()
     steps_all = K * world
     value = steps_all / (ms_all / 1000.0)

@@ -49,7 +49,8 @@ enum csa_status {
     CSA_ERR_DTYPE = -3,       /* unknown dtype, or out_bf16 with CSA_F32 */
     CSA_ERR_WORKSPACE = -4,   /* workspace NULL or smaller than *_workspace_size() */
     CSA_ERR_CUDA = -5,        /* a CUDA launch or runtime call failed */
-    CSA_ERR_UNSUPPORTED = -6  /* shape outside what the kernels implement */
+    CSA_ERR_UNSUPPORTED = -6, /* shape outside what the kernels implement */
+    CSA_ERR_TIMEOUT = -7      /* a bounded device-side wait gave up (see *_status) */
 };
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -132,6 +133,11 @@ int hca_compress(const void* C, const void* Z,
  * cI <= 256; CUDA cores otherwise).  Requires 1 <= k, N_cap < 2^31.
  * ------------------------------------------------------------------------------- */
 size_t csa_indexer_topk_workspace_size(int B, int nq, int64_t N_cap, int k);
+
+/* Device status of an indexer workspace: synchronises `stream`, returns CSA_OK, or
+ * CSA_ERR_TIMEOUT if a tensor-core scan of an earlier call abandoned a bounded wait
+ * (its outputs are then invalid).  The flag stays set until csa_workspace_zero. */
+int csa_indexer_topk_status(const void* workspace, csa_stream_t stream);
 int csa_indexer_topk(const void* qI, const float* wI, const void* KI, const int64_t* t,
                      int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
                      int32_t* idx_out, float* scores_out,

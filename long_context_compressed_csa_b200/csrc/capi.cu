@@ -11,6 +11,7 @@ extern "C" const char* csa_status_string(int status)
         case CSA_ERR_WORKSPACE: return "CSA_ERR_WORKSPACE: workspace missing or too small";
         case CSA_ERR_CUDA: return "CSA_ERR_CUDA: CUDA launch or runtime error";
         case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED: shape not implemented";
+        case CSA_ERR_TIMEOUT: return "CSA_ERR_TIMEOUT: a bounded device-side wait gave up";
         default: return "CSA_ERR_UNKNOWN";
     }
 }

@@ -31,6 +31,7 @@ TopkWs topk_ws_layout(void* base, int G, int64_t N_cap)
     const int64_t Np = (int64_t)align_up((size_t)(N_cap > 0 ? N_cap : 1), 64);
     char* p = static_cast<char*>(base);
     w.ld = Np;
+    w.status = reinterpret_cast<uint32_t*>(p); p += 256;
     w.hist0 = reinterpret_cast<uint32_t*>(p);  p += (size_t)G * kBins * 4;
     w.hist1 = reinterpret_cast<uint32_t*>(p);  p += (size_t)G * kBins * 4;
     w.ctr = reinterpret_cast<uint32_t*>(p);    p += (size_t)G * kCtrs * 4;
@@ -39,7 +40,7 @@ TopkWs topk_ws_layout(void* base, int G, int64_t N_cap)
     w.cand = reinterpret_cast<uint2*>(p);      p += (size_t)G * Np * 8;
     w.cand2 = reinterpret_cast<uint2*>(p);     p += (size_t)G * Np * 8;
     w.bytes = (size_t)(p - static_cast<char*>(base));
-    w.zero_bytes = (size_t)G * (2 * kBins + kCtrs) * 4;
+    w.zero_bytes = 256 + (size_t)G * (2 * kBins + kCtrs) * 4;
     return w;
 }
 
@@ -433,4 +434,15 @@ extern "C" int csa_indexer_topk(const void* qI, const float* wI, const void* KI,
         st = launch_scan_cuda_core(qI, wI, KI, t, B, nq, N_cap, n_hI, cI, m, k, ws, dtype, stream);
     if (st != CSA_OK) return st;
     return launch_topk_select(ws, t, G, m, k, N_cap, idx_out, scores_out, stream);
+}
+
+extern "C" int csa_indexer_topk_status(const void* workspace, csa_stream_t stream)
+{
+    if (!workspace) return CSA_ERR_ARG;
+    uint32_t st = 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&st, workspace, sizeof(st), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    return st ? CSA_ERR_TIMEOUT : CSA_OK;
 }

@@ -9,6 +9,7 @@ constexpr int kCtrs = 8;     // per query: [0] emitted, [1] candidates, [2] tick
 
 // Workspace of csa_indexer_topk, carved from one caller buffer.
 struct TopkWs {
+    uint32_t* status; // sticky device status: nonzero after a bounded wait timed out
     uint32_t* hist0;  // [G][kBins] digit-0 histogram (zero between calls)
     uint32_t* hist1;  // [G][kBins] digit-1 histogram of the candidates (zero between calls)
     uint32_t* ctr;    // [G][kCtrs] counters (zero between calls)

@@ -1,18 +1,263 @@
-// tcgen05 indexer scan (bf16): placeholder until the tensor-core kernel lands.
+// Lightning-indexer scan on the 5th-generation tensor cores (tcgen05, bf16 in, fp32 out)
+// ("DeepSeek-V4 Hybrid Attention: CSA and HCA from Scratch", section 6.4 boxed score).
+//
+// For one query the score of every compressed key is sum_h w[h] * ReLU(q[h] . K[s]):
+// a dense [keys x c^I] x [c^I x n_h^I] contraction followed by a ReLU-weighted row
+// reduction.  At n_h^I = 64 heads it performs 64 flop per byte of key read, six times
+// the fp32 CUDA-core ridge of a B200, so the contraction runs on tcgen05:
+//
+//   warp 0   TMA producer: 128-key tiles of K^I (two 64-column panels for c^I = 128,
+//            128-byte swizzle) into a STAGES-deep shared-memory ring;
+//   warp 1   MMA issuer: D[128 keys x n_h^I] = K_tile * q^T with M = 128, N = n_h^I,
+//            K = 16 per instruction, accumulating in TMEM; two accumulator buffers so
+//            the next tile's MMAs overlap the previous tile's epilogue;
+//   warps 2-5 epilogue: one thread per key row reads its n_h^I fp32 dot products from
+//            TMEM (tcgen05.ld), applies ReLU and the head weights, writes the fp32
+//            score and adds its top-12-bit radix digit to a shared-memory histogram.
+//
+// q^I (the B operand) is staged once per CTA into the same swizzled layout.  Each CTA
+// walks a strided set of key tiles of one query.  Every barrier wait is bounded; a
+// timeout sets the workspace status word and every role drains and exits.
 #include "indexer.cuh"
+#include "tc_utils.cuh"
 
 namespace csa {
+namespace {
+
+constexpr int kTcThreads = 192;
+constexpr int kTileKeys = 128;
+
+template <int NH, int CI>
+struct ScanCfg {
+    static constexpr int kPanels = CI / 64;
+    static constexpr int kAStage = kTileKeys * CI * 2;      // bytes of one key tile
+    static constexpr int kBBytes = NH * CI * 2;             // q^I tile
+    static constexpr int kFixed = 1024 + kBBytes + NH * 4 + kBins * 4 + 256;
+    static constexpr int kStagesRaw = (220 * 1024 - kFixed) / kAStage;
+    static constexpr int kStages = kStagesRaw > 6 ? 6 : kStagesRaw;
+    static constexpr int kSmem = kFixed + kStages * kAStage;
+    static constexpr int kTmemCols = (2 * NH) < 32 ? 32 : (2 * NH);
+    static_assert(kStages >= 2, "not enough shared memory for a 2-stage ring");
+    static_assert((kTmemCols & (kTmemCols - 1)) == 0, "TMEM columns must be a power of 2");
+};
+
+CSA_DEV int64_t visible_of(const int64_t* t, int g, int m, int64_t N_cap)
+{
+    const int64_t tt = t[g];
+    if (tt < 0) return 0;
+    const int64_t v = tt / m;
+    return v < N_cap ? v : N_cap;
+}
+
+template <int NH, int CI>
+__global__ void __launch_bounds__(kTcThreads, 1)
+scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __restrict__ qI,
+               const float* __restrict__ wI, const int64_t* __restrict__ t, int nq, int64_t N_cap,
+               int m, int k, TopkWs ws)
+{
+    using Cfg = ScanCfg<NH, CI>;
+    constexpr int S = Cfg::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + S * Cfg::kAStage;
+    float* sw = reinterpret_cast<float*>(sB + Cfg::kBBytes);
+    uint32_t* sh = reinterpret_cast<uint32_t*>(sw + NH);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sh + kBins);
+    uint64_t* empty = full + S;
+    uint64_t* tfull = empty + S;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    const int g = blockIdx.y;
+    const int64_t b = g / nq;
+    const int64_t vis = visible_of(t, g, m, N_cap);
+    const int ntiles = (int)((vis + kTileKeys - 1) / kTileKeys);
+    if ((int)blockIdx.x >= ntiles) return;  // whole CTA idle for this query
+    const bool need_hist = vis > k;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            tc::mbar_init(&tfull[a], 1);
+            tc::mbar_init(&tempty[a], 128);
+        }
+        tc::mbar_init(done, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+        tc::tma_prefetch_desc(&tmap);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, Cfg::kTmemCols);
+        tc::tmem_relinquish();
+    }
+    // q^I of this query into the 128-byte-swizzled K-major layout, w^I, histogram
+    {
+        const __nv_bfloat16* qg = qI + (int64_t)g * NH * CI;
+        constexpr int kChunks = NH * CI / 8;  // 16-byte chunks
+        for (int i = threadIdx.x; i < kChunks; i += kTcThreads) {
+            const int row = i / (CI / 8), cc = i % (CI / 8);
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(qg + (int64_t)row * CI + cc * 8));
+            *reinterpret_cast<uint4*>(sB + (cc / 8) * (NH * 128) + tc::sw128_offset(row, cc % 8)) = v;
+        }
+        for (int i = threadIdx.x; i < NH; i += kTcThreads) sw[i] = wI[(int64_t)g * NH + i];
+        if (need_hist)
+            for (int i = threadIdx.x; i < kBins; i += kTcThreads) sh[i] = 0;
+    }
+    tc::fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int it = 0;
+            for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+                const int s = it % S;
+                const uint32_t ph = (it / S) & 1;
+                if (*abort_flag) break;
+                if (!tc::mbar_wait(&empty[s], ph ^ 1, tc::kWaitBudget)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc::mbar_arrive_expect_tx(&full[s], Cfg::kAStage);
+                const int row0 = (int)(b * N_cap) + tile * kTileKeys;
+#pragma unroll
+                for (int p = 0; p < Cfg::kPanels; ++p)
+                    tc::tma_load_2d(sA + s * Cfg::kAStage + p * (kTileKeys * 128), &tmap, &full[s], 64 * p, row0);
+            }
+            // drain: every issued load has landed before the CTA may exit
+            for (int j = it - S < 0 ? 0 : it - S; j < it; ++j)
+                if (!tc::mbar_wait(&full[j % S], (j / S) & 1, tc::kWaitBudget)) *abort_flag = 1;
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, NH, false, false);
+            int it = 0;
+            for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+                const int s = it % S;
+                const uint32_t ph = (it / S) & 1;
+                const int acc = it & 1;
+                const uint32_t aph = (it >> 1) & 1;
+                if (*abort_flag) break;
+                if (!tc::mbar_wait(&tempty[acc], aph ^ 1, tc::kWaitBudget) ||
+                    !tc::mbar_wait(&full[s], ph, tc::kWaitBudget)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc::fence_after_sync();
+                const uint32_t d = tmem_base + acc * NH;
+                const uint32_t a0 = tc::smem_u32(sA + s * Cfg::kAStage);
+                const uint32_t b0 = tc::smem_u32(sB);
+#pragma unroll
+                for (int p = 0; p < Cfg::kPanels; ++p) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = tc::smem_desc_sw128(a0 + p * (kTileKeys * 128) + kk * 32, 16, 1024);
+                        const uint64_t bd = tc::smem_desc_sw128(b0 + p * (NH * 128) + kk * 32, 16, 1024);
+                        tc::mma_bf16_ss(d, ad, bd, kIdesc, (p | kk) ? 1u : 0u);
+                    }
+                }
+                tc::mma_commit(&empty[s]);     // smem stage free once these MMAs finish
+                tc::mma_commit(&tfull[acc]);   // accumulator ready for the epilogue
+            }
+            tc::mma_commit(done);              // all issued MMAs complete before TMEM is freed
+            if (!tc::mbar_wait(done, 0, tc::kWaitBudget)) *abort_flag = 1;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;          // TMEM lane quarter this warp may access
+        const int row = quarter * 32 + lane;
+        float* scores = ws.scores + (int64_t)g * ws.ld;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+            const int acc = it & 1;
+            const uint32_t aph = (it >> 1) & 1;
+            if (*abort_flag) break;
+            if (!tc::mbar_wait(&tfull[acc], aph, tc::kWaitBudget)) {
+                *abort_flag = 1;
+                break;
+            }
+            tc::fence_after_sync();
+            float v[NH];
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * NH;
+#pragma unroll
+            for (int c0 = 0; c0 < NH; c0 += 16) tc::tmem_ld16(taddr + c0, v + c0);
+            tc::tmem_wait_ld();
+            tc::fence_before_sync();
+            tc::mbar_arrive(&tempty[acc]);
+            float sc = 0.f;
+#pragma unroll
+            for (int h = 0; h < NH; ++h) sc = fmaf(sw[h], fmaxf(v[h], 0.f), sc);
+            const int64_t sidx = (int64_t)tile * kTileKeys + row;
+            if (sidx < vis) {
+                scores[sidx] = sc;
+                if (need_hist) atomicAdd(&sh[order_key(sc) >> 20], 1u);
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (*abort_flag && threadIdx.x == 0) atomicExch(ws.status, 1u);
+    if (need_hist)
+        for (int i = threadIdx.x; i < kBins; i += kTcThreads)
+            if (sh[i]) atomicAdd(&ws.hist0[(size_t)g * kBins + i], sh[i]);
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    }
+}
+
+template <int NH, int CI>
+int launch_nh_ci(const CUtensorMap& tmap, const void* qI, const float* wI, const int64_t* t, int B, int nq,
+                 int64_t N_cap, int m, int k, const TopkWs& ws, cudaStream_t stream)
+{
+    using Cfg = ScanCfg<NH, CI>;
+    const int G = B * nq;
+    int64_t ctas = (kNumSMs + G - 1) / G;
+    const int64_t tiles = (N_cap + kTileKeys - 1) / kTileKeys;
+    if (ctas > tiles) ctas = tiles;
+    if (ctas < 1) ctas = 1;
+    auto kern = scan_tc_kernel<NH, CI>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+    dim3 grid((unsigned)ctas, (unsigned)G);
+    kern<<<grid, kTcThreads, Cfg::kSmem, stream>>>(tmap, static_cast<const __nv_bfloat16*>(qI), wI, t, nq, N_cap,
+                                                    m, k, ws);
+    return launch_status();
+}
+
+}  // namespace
 
 bool indexer_tc_supported(int n_hI, int cI)
 {
-    (void)n_hI;
-    (void)cI;
-    return false;
+    return (n_hI == 16 || n_hI == 32 || n_hI == 64 || n_hI == 128) && (cI == 64 || cI == 128 || cI == 256);
 }
 
-int launch_scan_tc(const void*, const float*, const void*, const int64_t*, int, int, int64_t,
-                   int, int, int, int, const TopkWs&, cudaStream_t)
+int launch_scan_tc(const void* qI, const float* wI, const void* KI, const int64_t* t, int B, int nq,
+                   int64_t N_cap, int n_hI, int cI, int m, int k, const TopkWs& ws, cudaStream_t stream)
 {
+    if (N_cap == 0) return CSA_OK;
+    if ((int64_t)B * N_cap + kTileKeys >= (int64_t(1) << 31) || !aligned16(qI) || !aligned16(KI))
+        return launch_scan_cuda_core(qI, wI, KI, t, B, nq, N_cap, n_hI, cI, m, k, ws, CSA_BF16, stream);
+    CUtensorMap tmap;
+    if (!make_tmap_bf16_2d(&tmap, KI, (uint64_t)B * N_cap, cI, cI, 64, kTileKeys)) return CSA_ERR_CUDA;
+#define CSA_SCAN_CASE(NH_, CI_) \
+    if (n_hI == NH_ && cI == CI_) return launch_nh_ci<NH_, CI_>(tmap, qI, wI, t, B, nq, N_cap, m, k, ws, stream);
+    CSA_SCAN_CASE(16, 64) CSA_SCAN_CASE(16, 128) CSA_SCAN_CASE(16, 256)
+    CSA_SCAN_CASE(32, 64) CSA_SCAN_CASE(32, 128) CSA_SCAN_CASE(32, 256)
+    CSA_SCAN_CASE(64, 64) CSA_SCAN_CASE(64, 128) CSA_SCAN_CASE(64, 256)
+    CSA_SCAN_CASE(128, 64) CSA_SCAN_CASE(128, 128) CSA_SCAN_CASE(128, 256)
+#undef CSA_SCAN_CASE
     return CSA_ERR_UNSUPPORTED;
 }
 

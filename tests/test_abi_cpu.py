@@ -43,7 +43,7 @@ def test_every_declared_symbol_is_exported(lib):
 def test_status_strings_and_version(lib):
     from long_context_compressed_csa_b200 import csa_status_string, csa_version
     assert csa_status_string(0) == "CSA_OK"
-    for code in range(-1, -7, -1):
+    for code in range(-1, -8, -1):
         assert csa_status_string(code).startswith("CSA_ERR_")
     assert csa_status_string(-99) == "CSA_ERR_UNKNOWN"
     assert csa_version() >= 100
