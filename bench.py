@@ -264,6 +264,80 @@ def cpu_baseline(n_steps=2, seed=77):
 
 
 # ----------------------------------------------------------------------------------
+# single-kernel micro runs (profiling and per-kernel rooflines)
+# ----------------------------------------------------------------------------------
+def micro(kind, iters, rotate=4):
+    """Time one entry point alone on the 1M workload's shapes (compress kernels on the
+    B=16 x 128K HCA and B=4 x 256K CSA prefill shapes), rotating over `rotate` input
+    sets so repeated launches do not hit L2.  Prints one JSON line (not the bench line)."""
+    import torch
+    import long_context_compressed_csa_b200 as lib
+    from long_context_compressed_csa_b200 import build
+    from long_context_compressed_csa_b200.synth import randn
+    build.build()
+    bf16 = torch.bfloat16
+    dev = "cuda"
+    n, m, mp, c, cI, n_h, n_hI, k = 1 << 20, 4, 128, 512, 128, 128, 64, 1024
+    N, Nh = n // m, n // mp
+    t = torch.full((1, 1), n, dtype=torch.int64, device=dev)
+    calls, nbytes = [], 0
+    if kind == "indexer":
+        KIs = [randn((1, N, cI), 900 + r, bf16, dev) for r in range(rotate)]
+        qI, wI = randn((1, 1, n_hI, cI), 890, bf16, dev), randn((1, 1, n_hI), 891, torch.float32, dev)
+        idx = torch.empty((1, 1, k), dtype=torch.int32, device=dev)
+        ws = torch.zeros(lib.csa_indexer_topk_workspace_size(1, 1, N, k), dtype=torch.uint8, device=dev)
+        calls = [lambda r=r: lib.csa_indexer_topk(qI, wI, KIs[r], t, m, k, idx, ws) for r in range(rotate)]
+        nbytes = N * cI * 2
+    elif kind == "sparse":
+        caches = [randn((1, N, c), 910 + r, bf16, dev) for r in range(rotate)]
+        q = randn((1, 1, n_h, c), 920, bf16, dev)
+        g = torch.Generator(device="cpu").manual_seed(921)
+        idx = torch.randperm(N, generator=g)[:k].to(torch.int32).reshape(1, 1, k).to(dev)
+        o = torch.empty((1, 1, n_h, c), dtype=torch.float32, device=dev)
+        ws = torch.empty(lib.csa_attn_workspace_size(1, 1, n_h, c, k), dtype=torch.uint8, device=dev)
+        calls = [lambda r=r: lib.csa_sparse_attn(q, caches[r], idx, o, ws) for r in range(rotate)]
+        nbytes = k * c * 2
+    elif kind == "dense":
+        caches = [randn((1, Nh, c), 930 + r, bf16, dev) for r in range(rotate * 4)]
+        q = randn((1, 1, n_h, c), 940, bf16, dev)
+        o = torch.empty((1, 1, n_h, c), dtype=torch.float32, device=dev)
+        ws = torch.empty(lib.csa_attn_workspace_size(1, 1, n_h, c, Nh), dtype=torch.uint8, device=dev)
+        calls = [lambda r=r: lib.hca_dense_attn(q, caches[r], t, mp, o, ws) for r in range(rotate * 4)]
+        nbytes = Nh * c * 2
+    elif kind == "hca_compress":
+        B, nn = 16, 131072
+        C, Z = randn((B, nn, c), 950, bf16, dev), randn((B, nn, c), 951, bf16, dev)
+        out = torch.empty((B, nn // mp, c), dtype=bf16, device=dev)
+        calls = [lambda: lib.hca_compress(C, Z, out, mp)]
+        nbytes = 2 * B * nn * c * 2 + B * (nn // mp) * c * 2
+    elif kind == "csa_compress":
+        B, nn = 4, 262144
+        S = [randn((B, nn, c), 960 + i, bf16, dev) for i in range(4)]
+        out = torch.empty((B, nn // m, c), dtype=bf16, device=dev)
+        calls = [lambda: lib.csa_compress(*S, out, m)]
+        nbytes = 4 * B * nn * c * 2 + B * (nn // m) * c * 2
+    else:
+        raise SystemExit("unknown --micro kind %r" % kind)
+    for f in calls:
+        f()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for i in range(iters):
+        evs[i][0].record()
+        calls[i % len(calls)]()
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    us = np.array([a.elapsed_time(b) * 1e3 for a, b in evs])
+    hbm, _, src = peaks()
+    gbs = nbytes / (np.median(us) * 1e-6) / 1e9
+    print(json.dumps({"micro": kind, "iters": iters, "us_median": float(np.median(us)),
+                      "us_mean": float(us.mean()), "us_min": float(us.min()),
+                      "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "peak_gbs": hbm,
+                      "frac": gbs / hbm, "peak_source": src}), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -272,7 +346,12 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--micro", default=None,
+                    help="time one entry point alone: indexer, sparse, dense, csa_compress, hca_compress")
+    ap.add_argument("--iters", type=int, default=20)
     args = ap.parse_args()
+    if args.micro:
+        return micro(args.micro, args.iters)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
