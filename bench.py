@@ -152,9 +152,9 @@ class HybridDecode:
         self.oh = torch.empty((1, 1, self.n_h, c), dtype=torch.float32, device=device)
         self.ws_topk = torch.zeros(lib.csa_indexer_topk_workspace_size(1, 1, self.N_cap, self.k),
                                    dtype=torch.uint8, device=device)
-        self.ws_attn = torch.empty(lib.csa_attn_workspace_size(1, 1, self.n_h, c, self.k),
+        self.ws_attn = torch.zeros(lib.csa_attn_workspace_size(1, 1, self.n_h, c, self.k),
                                    dtype=torch.uint8, device=device)
-        self.ws_hattn = torch.empty(lib.csa_attn_workspace_size(1, 1, self.n_h, c, self.Nh_cap),
+        self.ws_hattn = torch.zeros(lib.csa_attn_workspace_size(1, 1, self.n_h, c, self.Nh_cap),
                                     dtype=torch.uint8, device=device)
 
     def _prefill(self, P, s):
@@ -294,14 +294,14 @@ def micro(kind, iters, rotate=4):
         g = torch.Generator(device="cpu").manual_seed(921)
         idx = torch.randperm(N, generator=g)[:k].to(torch.int32).reshape(1, 1, k).to(dev)
         o = torch.empty((1, 1, n_h, c), dtype=torch.float32, device=dev)
-        ws = torch.empty(lib.csa_attn_workspace_size(1, 1, n_h, c, k), dtype=torch.uint8, device=dev)
+        ws = torch.zeros(lib.csa_attn_workspace_size(1, 1, n_h, c, k), dtype=torch.uint8, device=dev)
         calls = [lambda r=r: lib.csa_sparse_attn(q, caches[r], idx, o, ws) for r in range(rotate)]
         nbytes = k * c * 2
     elif kind == "dense":
         caches = [randn((1, Nh, c), 930 + r, bf16, dev) for r in range(rotate * 4)]
         q = randn((1, 1, n_h, c), 940, bf16, dev)
         o = torch.empty((1, 1, n_h, c), dtype=torch.float32, device=dev)
-        ws = torch.empty(lib.csa_attn_workspace_size(1, 1, n_h, c, Nh), dtype=torch.uint8, device=dev)
+        ws = torch.zeros(lib.csa_attn_workspace_size(1, 1, n_h, c, Nh), dtype=torch.uint8, device=dev)
         calls = [lambda r=r: lib.hca_dense_attn(q, caches[r], t, mp, o, ws) for r in range(rotate * 4)]
         nbytes = Nh * c * 2
     elif kind == "hca_compress":

@@ -134,10 +134,6 @@ int hca_compress(const void* C, const void* Z,
  * ------------------------------------------------------------------------------- */
 size_t csa_indexer_topk_workspace_size(int B, int nq, int64_t N_cap, int k);
 
-/* Device status of an indexer workspace: synchronises `stream`, returns CSA_OK, or
- * CSA_ERR_TIMEOUT if a tensor-core scan of an earlier call abandoned a bounded wait
- * (its outputs are then invalid).  The flag stays set until csa_workspace_zero. */
-int csa_indexer_topk_status(const void* workspace, csa_stream_t stream);
 int csa_indexer_topk(const void* qI, const float* wI, const void* KI, const int64_t* t,
                      int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
                      int32_t* idx_out, float* scores_out,
@@ -154,7 +150,8 @@ int csa_indexer_topk(const void* qI, const float* wI, const void* KI, const int6
  * out   : [B, nq, n_h, c], fp32, or bf16 when out_bf16 != 0 (dtype must be bf16)
  * lse   : fp32 [B, nq, n_h] natural-log sum of exp(scaled logits), or NULL
  * A query with no valid entry gets out = 0 and lse = -inf.
- * workspace : >= csa_attn_workspace_size(B, nq, n_h, c, k) bytes (no zeroing needed).
+ * workspace : >= csa_attn_workspace_size(B, nq, n_h, c, k) bytes; zero its first 4 bytes
+ *             (the status word) before first use.
  * Constraints: 1 <= c <= 512, n_h >= 1.
  * ------------------------------------------------------------------------------- */
 size_t csa_attn_workspace_size(int B, int nq, int n_h, int c, int64_t max_entries);
@@ -174,6 +171,12 @@ int hca_dense_attn(const void* q, const void* cache, const int64_t* t,
                    int B, int nq, int n_h, int c, int64_t N_cap, int m_prime, float scale,
                    void* out, float* lse, void* workspace, size_t ws_bytes,
                    int dtype, int out_bf16, csa_stream_t stream);
+
+/* Device status of a workspace of csa_indexer_topk, csa_sparse_attn or hca_dense_attn:
+ * synchronises `stream` and returns CSA_OK, or CSA_ERR_TIMEOUT if a tensor-core kernel
+ * of an earlier call gave up a bounded wait (its outputs are then invalid).  The status
+ * word is the first 4 bytes of the workspace and stays set until it is zeroed. */
+int csa_workspace_status(const void* workspace, csa_stream_t stream);
 
 /* Zero `bytes` of device memory on `stream` (cudaMemsetAsync); for first-use workspaces. */
 int csa_workspace_zero(void* workspace, size_t bytes, csa_stream_t stream);

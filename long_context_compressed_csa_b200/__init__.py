@@ -13,11 +13,11 @@ from ._binding import (  # noqa: F401
     csa_attn_workspace_size,
     csa_compress,
     csa_indexer_topk,
-    csa_indexer_topk_status,
     csa_indexer_topk_workspace_size,
     csa_sparse_attn,
     csa_status_string,
     csa_version,
+    csa_workspace_status,
     csa_workspace_zero,
     hca_compress,
     hca_dense_attn,

@@ -24,7 +24,7 @@ _SIGS = {
                       i32, vp], i32),
     "hca_compress": ([vp, vp, i64, i64, i64, i64, vp, vp, i64, i32, i32, i32, i64, i64, i32, vp], i32),
     "csa_indexer_topk_workspace_size": ([i32, i32, i64, i32], sz),
-    "csa_indexer_topk_status": ([vp, vp], i32),
+    "csa_workspace_status": ([vp, vp], i32),
     "csa_indexer_topk": ([vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, i32, vp, vp, vp, sz, i32, vp],
                          i32),
     "csa_attn_workspace_size": ([i32, i32, i32, i32, i64], sz),
@@ -160,9 +160,9 @@ def csa_indexer_topk(qI, wI, KI, t, m, k, idx_out, workspace, scores_out=None, s
         _dtype(qI), _stream(stream)))
 
 
-def csa_indexer_topk_status(workspace, stream=None) -> int:
+def csa_workspace_status(workspace, stream=None) -> int:
     """0, or -7 (CSA_ERR_TIMEOUT) if a device-side wait of an earlier call gave up."""
-    return int(library().csa_indexer_topk_status(_ptr(workspace), _stream(stream)))
+    return int(library().csa_workspace_status(_ptr(workspace), _stream(stream)))
 
 
 def csa_attn_workspace_size(B, nq, n_h, c, max_entries) -> int:

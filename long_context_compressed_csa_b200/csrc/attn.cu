@@ -31,7 +31,7 @@ AttnPlan attn_plan_cuda_core(int G, int n_h, int64_t entries)
 
 size_t attn_ws_bytes(int G, int n_h, int c, int splits)
 {
-    return align_up((size_t)G * splits * n_h * c * sizeof(float), 256) +
+    return 256 + align_up((size_t)G * splits * n_h * c * sizeof(float), 256) +
            align_up((size_t)G * splits * n_h * sizeof(float2), 256);
 }
 
@@ -167,6 +167,15 @@ attn_cuda_core(AttnArgs a)
 // combine: out[g][h] = sum_i 2^(m_i - M) O_i / sum_i 2^(m_i - M) l_i ; lse in natural log
 // ----------------------------------------------------------------------------------
 template <typename TO>
+CSA_DEV void store_out(TO* p, float v);
+template <>
+CSA_DEV void store_out<float>(float* p, float v) { *p = v; }
+template <>
+CSA_DEV void store_out<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+// One CTA per (head, query).  Thread t owns columns 4t..4t+3 (float4 loads) and walks
+// the splits four at a time so that several independent loads are in flight.
+template <typename TO>
 __global__ void __launch_bounds__(128)
 attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_ml, int splits,
              int n_h, int c, TO* __restrict__ out, float* __restrict__ lse)
@@ -196,17 +205,47 @@ attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_m
     }
     __syncthreads();
     const float inv = s_inv;
-    for (int j = threadIdx.x; j < c; j += blockDim.x) {
-        float acc = 0.f;
-        for (int i = 0; i < splits; ++i) {
-            const float w = s_w[i];
-            if (w != 0.f) acc = fmaf(w, part_o[(base + (size_t)i * n_h) * c + j], acc);
+    TO* orow = out + ((size_t)g * n_h + h) * c;
+    if ((c & 3) == 0) {
+        for (int j = threadIdx.x * 4; j < c; j += blockDim.x * 4) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            int i = 0;
+            for (; i + 4 <= splits; i += 4) {
+                float4 v[4];
+                float w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    w[u] = s_w[i + u];
+                    v[u] = w[u] != 0.f ? __ldcs(reinterpret_cast<const float4*>(part_o + (base + (size_t)(i + u) * n_h) * c + j))
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    acc.x = fmaf(w[u], v[u].x, acc.x); acc.y = fmaf(w[u], v[u].y, acc.y);
+                    acc.z = fmaf(w[u], v[u].z, acc.z); acc.w = fmaf(w[u], v[u].w, acc.w);
+                }
+            }
+            for (; i < splits; ++i) {
+                const float w = s_w[i];
+                if (w == 0.f) continue;
+                const float4 v = __ldcs(reinterpret_cast<const float4*>(part_o + (base + (size_t)i * n_h) * c + j));
+                acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+                acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+            }
+            store_out<TO>(orow + j, acc.x * inv);
+            store_out<TO>(orow + j + 1, acc.y * inv);
+            store_out<TO>(orow + j + 2, acc.z * inv);
+            store_out<TO>(orow + j + 3, acc.w * inv);
         }
-        const float v = acc * inv;
-        if constexpr (sizeof(TO) == 2)
-            out[((size_t)g * n_h + h) * c + j] = __float2bfloat16_rn(v);
-        else
-            out[((size_t)g * n_h + h) * c + j] = v;
+    } else {
+        for (int j = threadIdx.x; j < c; j += blockDim.x) {
+            float acc = 0.f;
+            for (int i = 0; i < splits; ++i) {
+                const float w = s_w[i];
+                if (w != 0.f) acc = fmaf(w, part_o[(base + (size_t)i * n_h) * c + j], acc);
+            }
+            store_out<TO>(orow + j, acc * inv);
+        }
     }
 }
 
@@ -269,11 +308,13 @@ int attn_run(AttnArgs a, float scale, void* out, float* lse, void* workspace, si
     const bool tc = dtype == CSA_BF16 && attn_tc_supported(a.n_h, a.c);
     AttnPlan plan = tc ? attn_plan_tc(G, a.n_h, a.c, entries) : attn_plan_cuda_core(G, a.n_h, entries);
     char* ws = static_cast<char*>(workspace);
+    uint32_t* status = reinterpret_cast<uint32_t*>(ws);  // sticky device status word
+    ws += 256;
     a.part_o = reinterpret_cast<float*>(ws);
     a.part_ml = reinterpret_cast<float2*>(ws + align_up((size_t)G * plan.splits * a.n_h * a.c * sizeof(float), 256));
     a.splits = plan.splits;
     a.per_split = plan.per_split;
-    int st = tc ? launch_attn_tc(a, plan, stream) : launch_cuda_core(a, plan, dtype, stream);
+    int st = tc ? launch_attn_tc(a, plan, status, stream) : launch_cuda_core(a, plan, dtype, stream);
     if (st != CSA_OK) return st;
     return launch_attn_combine(a, out, out_bf16, lse, stream);
 }

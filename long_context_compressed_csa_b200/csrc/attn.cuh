@@ -35,7 +35,7 @@ AttnPlan attn_plan_cuda_core(int G, int n_h, int64_t entries);
 AttnPlan attn_plan_tc(int G, int n_h, int c, int64_t entries);
 bool attn_tc_supported(int n_h, int c);
 size_t attn_ws_bytes(int G, int n_h, int c, int splits);
-int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, cudaStream_t stream);
+int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cudaStream_t stream);
 int launch_attn_combine(const AttnArgs& a, void* out, int out_bf16, float* lse,
                         cudaStream_t stream);
 

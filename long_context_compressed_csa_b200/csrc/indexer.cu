@@ -207,11 +207,53 @@ CSA_DEV uint32_t digit_of(uint2 kv, int level)
     }
 }
 
+constexpr int kListCap = 1024;  // candidates kept in shared memory by the last CTA
+constexpr int kRankMax = 256;   // lists up to this size are finished by exact ranking
+
+// Emit every entry of a list (count entries) into the output slots counted by *s_out.
+CSA_DEV void emit_all(const uint2* list, bool in_smem, uint32_t count, uint32_t* s_out, int k,
+                      int32_t* idx_out, float* sc_out)
+{
+    for (uint32_t i = threadIdx.x; i < ((count + 31) & ~31u); i += kSelThreads) {
+        const bool in = i < count;
+        const uint2 kv = in ? (in_smem ? list[i] : __ldcg(&list[i])) : make_uint2(0, 0);
+        const uint32_t pos = warp_append(s_out, in);
+        if (in && pos < (uint32_t)k) {
+            idx_out[pos] = (int32_t)kv.y;
+            if (sc_out) sc_out[pos] = key_to_float(kv.x);
+        }
+    }
+}
+
+// Emit the `need` best entries of a shared-memory list of at most kSelThreads entries:
+// each entry counts the entries that beat it (higher score key, or equal key and a
+// smaller index) and is selected when fewer than `need` do.
+CSA_DEV void emit_by_rank(const uint2* list, uint32_t count, uint32_t need, uint32_t* s_out, int k,
+                          int32_t* idx_out, float* sc_out)
+{
+    const uint32_t i = threadIdx.x;
+    const bool in = i < count;
+    const uint2 me = in ? list[i] : make_uint2(0, 0);
+    uint32_t rank = 0;
+    if (in)
+        for (uint32_t j = 0; j < count; ++j) {
+            const uint2 o = list[j];
+            rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+        }
+    const bool take = in && rank < need;
+    const uint32_t pos = warp_append(s_out, take);
+    if (take && pos < (uint32_t)k) {
+        idx_out[pos] = (int32_t)me.y;
+        if (sc_out) sc_out[pos] = key_to_float(me.x);
+    }
+}
+
 __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
 {
     __shared__ uint32_t sh[kBins];
     __shared__ uint32_t s_scr[32];
-    __shared__ uint32_t s_bin, s_above, s_last, s_cnt;
+    __shared__ uint2 s_listA[kListCap], s_listB[kListCap];
+    __shared__ uint32_t s_bin, s_above, s_last, s_cnt, s_out;
     const int g = blockIdx.y;
     const int tid = threadIdx.x;
     const int64_t vis = visible_count(a.t, g, a.m, a.N_cap);
@@ -280,65 +322,66 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
     __threadfence();
 
     if (vis > k) {
-        uint32_t need = (uint32_t)k - __ldcg(&ctr[0]);
+        // Resolve the candidates of the digit-0 threshold bin.  Emission slots now come
+        // from a shared-memory counter (this CTA is the only writer left); lists that fit
+        // are kept in shared memory so the remaining passes make no global round trips.
+        if (tid == 0) s_out = __ldcg(&ctr[0]);
         uint32_t count = __ldcg(&ctr[1]);
-        uint2* list = cand;
-        uint2* next = cand2;
         for (int i = tid; i < kBins; i += kSelThreads) sh[i] = __ldcg(&a.ws.hist1[(size_t)g * kBins + i]);
         __syncthreads();
-        for (int level = 1; level <= 6 && need > 0; ++level) {
+        uint32_t need = (uint32_t)k - s_out;
+        uint2* list = cand;
+        bool in_smem = false;
+        for (int level = 1; need > 0; ++level) {
+            if (need >= count) {  // every remaining candidate is selected
+                emit_all(list, in_smem, count, &s_out, k, idx_out, sc_out);
+                break;
+            }
+            if (in_smem && count <= kRankMax) {  // exact rank among a small list
+                emit_by_rank(list, count, need, &s_out, k, idx_out, sc_out);
+                break;
+            }
+            if (level > 6) break;  // unreachable: (score, index) keys are unique
             if (level >= 2) {
-                // 256-bin histogram of this level's digit over the current list
                 for (int i = tid; i < 256; i += kSelThreads) sh[i] = 0;
                 __syncthreads();
                 for (uint32_t i = tid; i < count; i += kSelThreads)
-                    atomicAdd(&sh[digit_of(__ldcg(&list[i]), level)], 1u);
+                    atomicAdd(&sh[digit_of(in_smem ? list[i] : __ldcg(&list[i]), level)], 1u);
                 __syncthreads();
-            }
-            if (need == count) break;  // every remaining candidate is selected
-            if (level == 1)
-                find_threshold_bin<kBins>(sh, need, &s_bin, &s_above, s_scr);
-            else
                 find_threshold_bin<256>(sh, need, &s_bin, &s_above, s_scr);
-            const uint32_t bt = s_bin;
-            const uint32_t above = s_above;
+            } else {
+                find_threshold_bin<kBins>(sh, need, &s_bin, &s_above, s_scr);
+            }
+            const uint32_t bt = s_bin, above = s_above, keep_n = sh[bt];
+            uint2* next;
+            bool next_smem = keep_n <= (uint32_t)kListCap;
+            if (next_smem)
+                next = (list == s_listA) ? s_listB : s_listA;
+            else
+                next = (list == cand) ? cand2 : cand;
             if (tid == 0) s_cnt = 0;
             __syncthreads();
-            const uint32_t rounded = (count + 31) & ~31u;
-            for (uint32_t i = tid; i < ((rounded + kSelThreads - 1) / kSelThreads) * kSelThreads;
-                 i += kSelThreads) {
+            for (uint32_t i = tid; i < ((count + kSelThreads - 1) / kSelThreads) * kSelThreads; i += kSelThreads) {
                 const bool in = i < count;
-                uint2 kv = in ? __ldcg(&list[i]) : make_uint2(0, 0);
+                const uint2 kv = in ? (in_smem ? list[i] : __ldcg(&list[i])) : make_uint2(0, 0);
                 const uint32_t d = digit_of(kv, level);
                 const bool take = in && d > bt;
                 const bool keep = in && d == bt;
-                const uint32_t pos = warp_append(&ctr[0], take);
+                const uint32_t pos = warp_append(&s_out, take);
                 if (take && pos < (uint32_t)k) {
                     idx_out[pos] = (int32_t)kv.y;
                     if (sc_out) sc_out[pos] = key_to_float(kv.x);
                 }
                 const uint32_t npos = warp_append(&s_cnt, keep);
-                if (keep && npos < (uint32_t)a.ws.ld) next[npos] = kv;
+                if (keep && npos < (next_smem ? (uint32_t)kListCap : (uint32_t)a.ws.ld)) next[npos] = kv;
             }
-            __syncthreads();
             __threadfence_block();
+            __syncthreads();
             need -= above;
             count = s_cnt;
-            uint2* tmp = list; list = next; next = tmp;
+            list = next;
+            in_smem = next_smem;
             __syncthreads();
-        }
-        // remaining candidates (need == count) are all selected
-        if (need > 0) {
-            __syncthreads();
-            for (uint32_t i = tid; i < ((count + 31) & ~31u); i += kSelThreads) {
-                const bool in = i < count;
-                uint2 kv = in ? __ldcg(&list[i]) : make_uint2(0, 0);
-                const uint32_t pos = warp_append(&ctr[0], in);
-                if (in && pos < (uint32_t)k) {
-                    idx_out[pos] = (int32_t)kv.y;
-                    if (sc_out) sc_out[pos] = key_to_float(kv.x);
-                }
-            }
         }
     }
     __syncthreads();
@@ -436,7 +479,7 @@ extern "C" int csa_indexer_topk(const void* qI, const float* wI, const void* KI,
     return launch_topk_select(ws, t, G, m, k, N_cap, idx_out, scores_out, stream);
 }
 
-extern "C" int csa_indexer_topk_status(const void* workspace, csa_stream_t stream)
+extern "C" int csa_workspace_status(const void* workspace, csa_stream_t stream)
 {
     if (!workspace) return CSA_ERR_ARG;
     uint32_t st = 0;

@@ -68,7 +68,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
     uint64_t* tfull = empty + S;
     uint64_t* tempty = tfull + 2;
     uint64_t* done = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* qready = done + 1;  // q^I and w^I staged by the epilogue warps
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qready + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const int g = blockIdx.y;
@@ -89,6 +90,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
             tc::mbar_init(&tempty[a], 128);
         }
         tc::mbar_init(done, 1);
+        tc::mbar_init(qready, 128);
         *abort_flag = 0;
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&tmap);
@@ -97,20 +99,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
         tc::tmem_alloc(tmem_slot, Cfg::kTmemCols);
         tc::tmem_relinquish();
     }
-    // q^I of this query into the 128-byte-swizzled K-major layout, w^I, histogram
-    {
-        const __nv_bfloat16* qg = qI + (int64_t)g * NH * CI;
-        constexpr int kChunks = NH * CI / 8;  // 16-byte chunks
-        for (int i = threadIdx.x; i < kChunks; i += kTcThreads) {
-            const int row = i / (CI / 8), cc = i % (CI / 8);
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(qg + (int64_t)row * CI + cc * 8));
-            *reinterpret_cast<uint4*>(sB + (cc / 8) * (NH * 128) + tc::sw128_offset(row, cc % 8)) = v;
-        }
-        for (int i = threadIdx.x; i < NH; i += kTcThreads) sw[i] = wI[(int64_t)g * NH + i];
-        if (need_hist)
-            for (int i = threadIdx.x; i < kBins; i += kTcThreads) sh[i] = 0;
-    }
-    tc::fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -142,6 +130,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, NH, false, false);
+            if (!tc::mbar_wait(qready, 0, tc::kWaitBudget)) *abort_flag = 1;
             int it = 0;
             for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
                 const int s = it % S;
@@ -175,6 +164,24 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // first stage q^I (128-byte-swizzled K-major), w^I and the histogram while the
+        // producer's first key tiles are already in flight
+        {
+            const int et = threadIdx.x - 64;  // 0..127
+            const __nv_bfloat16* qg = qI + (int64_t)g * NH * CI;
+            constexpr int kChunks = NH * CI / 8;  // 16-byte chunks
+            for (int i = et; i < kChunks; i += 128) {
+                const int r = i / (CI / 8), cc = i % (CI / 8);
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(qg + (int64_t)r * CI + cc * 8));
+                *reinterpret_cast<uint4*>(sB + (cc / 8) * (NH * 128) + tc::sw128_offset(r, cc % 8)) = v;
+            }
+            for (int i = et; i < NH; i += 128) sw[i] = wI[(int64_t)g * NH + i];
+            if (need_hist)
+                for (int i = et; i < kBins; i += 128) sh[i] = 0;
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(qready);
+            asm volatile("bar.sync 1, 128;" ::: "memory");  // epilogue warps only
+        }
         const int quarter = warp & 3;          // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;
         float* scores = ws.scores + (int64_t)g * ws.ld;
@@ -199,9 +206,12 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
 #pragma unroll
             for (int h = 0; h < NH; ++h) sc = fmaf(sw[h], fmaxf(v[h], 0.f), sc);
             const int64_t sidx = (int64_t)tile * kTileKeys + row;
-            if (sidx < vis) {
-                scores[sidx] = sc;
-                if (need_hist) atomicAdd(&sh[order_key(sc) >> 20], 1u);
+            if (sidx < vis) scores[sidx] = sc;
+            if (need_hist) {
+                // lanes with the same digit add once (scores cluster in few bins)
+                const uint32_t bin = sidx < vis ? order_key(sc) >> 20 : 0xffffffffu;
+                const unsigned peers = __match_any_sync(0xffffffffu, bin);
+                if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&sh[bin], (uint32_t)__popc(peers));
             }
         }
     }

@@ -18,7 +18,7 @@ import torch
 import oracle
 from long_context_compressed_csa_b200 import (csa_attn_workspace_size, csa_compress,
                                               csa_indexer_topk, csa_indexer_topk_workspace_size,
-                                              csa_sparse_attn, csa_workspace_zero, hca_compress,
+                                              csa_sparse_attn, csa_workspace_status, hca_compress,
                                               hca_dense_attn)
 from long_context_compressed_csa_b200.synth import randint_values, randn, to_f64
 from tests.helpers import check_topk_sets, max_rel_rowwise, score_error_bound
@@ -157,6 +157,7 @@ def run_indexer(qI, wI, KI, t, m, k, ws=None, scores=True):
     tt = torch.tensor(t, dtype=torch.int64, device=DEV).reshape(B, nq)
     csa_indexer_topk(qI, wI, KI, tt, m, k, idx, ws, scores_out=sc)
     torch.cuda.synchronize()
+    assert csa_workspace_status(ws) == 0
     return idx.cpu().numpy(), (sc.cpu().numpy() if scores else None), ws
 
 
@@ -242,23 +243,25 @@ def test_indexer_degenerate_cases():
 def run_sparse(q, cache, idx, out_dtype=torch.float32, scale=0.0):
     B, nq, n_h, c = q.shape
     k = idx.shape[2]
-    ws = torch.empty(csa_attn_workspace_size(B, nq, n_h, c, k), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(csa_attn_workspace_size(B, nq, n_h, c, k), dtype=torch.uint8, device=DEV)
     out = torch.full((B, nq, n_h, c), float("nan"), dtype=out_dtype, device=DEV)
     lse = torch.full((B, nq, n_h), float("nan"), device=DEV)
     csa_sparse_attn(q, cache, idx, out, ws, lse=lse, scale=scale)
     torch.cuda.synchronize()
+    assert csa_workspace_status(ws) == 0
     return out.float().cpu().numpy(), lse.cpu().numpy()
 
 
 def run_dense(q, cache, t, mp, out_dtype=torch.float32):
     B, nq, n_h, c = q.shape
     N_cap = cache.shape[1]
-    ws = torch.empty(csa_attn_workspace_size(B, nq, n_h, c, N_cap), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(csa_attn_workspace_size(B, nq, n_h, c, N_cap), dtype=torch.uint8, device=DEV)
     out = torch.full((B, nq, n_h, c), float("nan"), dtype=out_dtype, device=DEV)
     lse = torch.full((B, nq, n_h), float("nan"), device=DEV)
     tt = torch.tensor(t, dtype=torch.int64, device=DEV).reshape(B, nq)
     hca_dense_attn(q, cache, tt, mp, out, ws, lse=lse)
     torch.cuda.synchronize()
+    assert csa_workspace_status(ws) == 0
     return out.float().cpu().numpy(), lse.cpu().numpy()
 
 
