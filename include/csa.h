@@ -140,6 +140,31 @@ int csa_indexer_topk(const void* qI, const float* wI, const void* KI, const int6
                      void* workspace, size_t ws_bytes, int dtype, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * csa_indexer_topk_noalloc - csa_indexer_topk for callers that cannot allocate device
+ * memory (no counterpart in the pages: it only changes where scratch comes from).
+ *
+ * Some callers have no way to get a scratch buffer: an engine that reserved all device
+ * memory for its own pool and gives kernels no allocator, or a plugin that receives
+ * only tensor pointers.  This variant takes the same arguments as csa_indexer_topk
+ * minus the workspace and computes the same result, using scratch that lives in the
+ * library: a fixed 8 MiB device array per GPU, held from the first use of the library
+ * on that GPU until the process exits.  It calls no allocator (no cudaMalloc or
+ * cudaFree, nothing that allocates).
+ *   - Size limit: csa_indexer_topk_workspace_size(B, nq, N_cap, k) must be at most
+ *     8 MiB (about B*nq*(20*N_cap + 33 KB) bytes; e.g. one query over ~400K compressed
+ *     entries).  Larger problems return CSA_ERR_WORKSPACE before any launch.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress
+ *     with that device current) and caches it; make that first call before any stream
+ *     capture.
+ *   - Every call shares the one array and clears its counters at the start (an
+ *     asynchronous memset on `stream`), so calls whose GPU work overlaps, on any streams
+ *     or threads, race with each other: serialise them.
+ * ------------------------------------------------------------------------------- */
+int csa_indexer_topk_noalloc(const void* qI, const float* wI, const void* KI, const int64_t* t,
+                             int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
+                             int32_t* idx_out, float* scores_out, int dtype, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * csa_sparse_attn - shared-KV multi-query attention over the selected compressed
  * entries ([P1] section 8):
  *   o[g][h] = sum_{s in idx[g]} softmax_s(scale * q[g][h] . C[b][s]) * C[b][s]

@@ -13,6 +13,7 @@ from ._binding import (  # noqa: F401
     csa_attn_workspace_size,
     csa_compress,
     csa_indexer_topk,
+    csa_indexer_topk_noalloc,
     csa_indexer_topk_workspace_size,
     csa_sparse_attn,
     csa_status_string,

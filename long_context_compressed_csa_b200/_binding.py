@@ -27,6 +27,7 @@ _SIGS = {
     "csa_workspace_status": ([vp, vp], i32),
     "csa_indexer_topk": ([vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, i32, vp, vp, vp, sz, i32, vp],
                          i32),
+    "csa_indexer_topk_noalloc": ([vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, i32, vp, vp, i32, vp], i32),
     "csa_attn_workspace_size": ([i32, i32, i32, i32, i64], sz),
     "csa_sparse_attn": ([vp, vp, vp, i32, i32, i32, i32, i64, i32, f32, vp, vp, vp, sz, i32, i32, vp],
                         i32),
@@ -158,6 +159,21 @@ def csa_indexer_topk(qI, wI, KI, t, m, k, idx_out, workspace, scores_out=None, s
         _ptr(qI), _ptr(wI), _ptr(KI), _ptr(t), B, nq, N_cap, n_hI, cI, m, k, _ptr(idx_out),
         _ptr(scores_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _dtype(qI), _stream(stream)))
+
+
+def csa_indexer_topk_noalloc(qI, wI, KI, t, m, k, idx_out, scores_out=None, stream=None):
+    """csa_indexer_topk without a workspace argument, for callers that cannot allocate:
+    scratch comes from a fixed 8 MiB device array inside the library (one per GPU), so
+    calls must not overlap on the GPU and the problem must fit in it."""
+    _cuda(qI, wI, KI, t, idx_out, scores_out)
+    B, nq, n_hI, cI = qI.shape
+    N_cap = KI.shape[1]
+    assert KI.shape == (B, N_cap, cI) and KI.is_contiguous() and qI.is_contiguous()
+    assert wI.shape == (B, nq, n_hI) and wI.is_contiguous()
+    assert t.numel() == B * nq and idx_out.shape == (B, nq, k) and idx_out.is_contiguous()
+    _check("csa_indexer_topk_noalloc", library().csa_indexer_topk_noalloc(
+        _ptr(qI), _ptr(wI), _ptr(KI), _ptr(t), B, nq, N_cap, n_hI, cI, m, k, _ptr(idx_out),
+        _ptr(scores_out), _dtype(qI), _stream(stream)))
 
 
 def csa_workspace_status(workspace, stream=None) -> int:
