@@ -208,6 +208,9 @@ CSA_DEV uint32_t digit_of(uint2 kv, int level)
 }
 
 constexpr int kListCap = 1024;  // candidates kept in shared memory by the last CTA
+constexpr int kPer = 4;         // scores per thread per round of the first pass
+constexpr int kRound = kPer * kSelThreads;
+static_assert(kRound <= kListCap, "a round's staging must fit the shared lists");
 constexpr int kRankMax = 256;   // lists up to this size are finished by exact ranking
 
 // Emit every entry of a list (count entries) into the output slots counted by *s_out.
@@ -252,8 +255,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
 {
     __shared__ uint32_t sh[kBins];
     __shared__ uint32_t s_scr[32];
-    __shared__ uint2 s_listA[kListCap], s_listB[kListCap];
-    __shared__ uint32_t s_bin, s_above, s_last, s_cnt, s_out;
+    __shared__ uint2 s_listA[kListCap], s_listB[kListCap];  // first pass: staged takes / candidates
+    __shared__ uint32_t s_bin, s_above, s_last, s_cnt, s_out, s_nt, s_nc, s_bt, s_bc;
+    uint2* s_take = s_listA;
+    uint2* s_cand = s_listB;
     const int g = blockIdx.y;
     const int tid = threadIdx.x;
     const int64_t vis = visible_count(a.t, g, a.m, a.N_cap);
@@ -284,26 +289,55 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
         for (int i = tid; i < kBins; i += kSelThreads) sh[i] = 0;
         __syncthreads();
         // ---- emit above b0, collect b0 candidates with their digit-1 histogram ----
+        // Rounds of kRound scores: every thread loads its kPer scores at once, the
+        // selected entries and candidates are staged in shared memory, and one global
+        // atomic per list and round reserves their output slots.
         const int64_t s_begin = (int64_t)blockIdx.x * a.chunk;
         const int64_t s_end = min(vis, s_begin + a.chunk);
-        for (int64_t base = s_begin; base < s_end; base += kSelThreads) {
-            const int64_t s = base + tid;
-            uint32_t key = 0;
-            bool in = s < s_end;
-            if (in) key = order_key(scores[s]);
-            const uint32_t d0 = key >> 20;
-            const bool take = in && d0 > b0;
-            const bool cnd = in && d0 == b0;
-            const uint32_t pos = warp_append(&ctr[0], take);
-            if (take && pos < (uint32_t)k) {
-                idx_out[pos] = (int32_t)s;
-                if (sc_out) sc_out[pos] = key_to_float(key);
+        for (int64_t base = s_begin; base < s_end; base += kRound) {
+            uint32_t key[kPer];
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int64_t s = base + tid + u * kSelThreads;
+                key[u] = s < s_end ? order_key(scores[s]) : 0u;
             }
-            const uint32_t cpos = warp_append(&ctr[1], cnd);
-            if (cnd && cpos < (uint32_t)a.ws.ld) {
-                cand[cpos] = make_uint2(key, (uint32_t)s);
-                atomicAdd(&sh[(key >> 8) & 0xfffu], 1u);
+            if (tid == 0) {
+                s_nt = 0;
+                s_nc = 0;
             }
+            __syncthreads();
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int64_t s = base + tid + u * kSelThreads;
+                const bool in = s < s_end;
+                const uint32_t d0 = key[u] >> 20;
+                const bool take = in && d0 > b0;
+                const bool cnd = in && d0 == b0;
+                const uint32_t tp = warp_append(&s_nt, take);
+                if (take) s_take[tp] = make_uint2(key[u], (uint32_t)s);
+                const uint32_t cp = warp_append(&s_nc, cnd);
+                if (cnd) {
+                    s_cand[cp] = make_uint2(key[u], (uint32_t)s);
+                    atomicAdd(&sh[(key[u] >> 8) & 0xfffu], 1u);
+                }
+            }
+            __syncthreads();
+            if (tid == 0) {
+                s_bt = s_nt ? atomicAdd(&ctr[0], s_nt) : 0u;
+                s_bc = s_nc ? atomicAdd(&ctr[1], s_nc) : 0u;
+            }
+            __syncthreads();
+            for (uint32_t i = tid; i < s_nt; i += kSelThreads) {
+                const uint32_t pos = s_bt + i;
+                const uint2 kv = s_take[i];
+                if (pos < (uint32_t)k) {
+                    idx_out[pos] = (int32_t)kv.y;
+                    if (sc_out) sc_out[pos] = key_to_float(kv.x);
+                }
+            }
+            for (uint32_t i = tid; i < s_nc; i += kSelThreads)
+                if (s_bc + i < (uint32_t)a.ws.ld) cand[s_bc + i] = s_cand[i];
+            __syncthreads();
         }
         __syncthreads();
         for (int i = tid; i < kBins; i += kSelThreads)

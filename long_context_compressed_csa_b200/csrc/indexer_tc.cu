@@ -11,7 +11,8 @@
 //   warp 1   MMA issuer: D[128 keys x n_h^I] = K_tile * q^T with M = 128, N = n_h^I,
 //            K = 16 per instruction, accumulating in TMEM; two accumulator buffers so
 //            the next tile's MMAs overlap the previous tile's epilogue;
-//   warps 2-5 epilogue: one thread per key row reads its n_h^I fp32 dot products from
+//   warps 2-9 epilogue (two groups of four, one per accumulator buffer): one thread
+//            per key row reads its n_h^I fp32 dot products from
 //            TMEM (tcgen05.ld), applies ReLU and the head weights, writes the fp32
 //            score and adds its top-12-bit radix digit to a shared-memory histogram.
 //
@@ -24,7 +25,7 @@
 namespace csa {
 namespace {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 320;  // producer, MMA, two groups of 4 epilogue warps
 constexpr int kTileKeys = 128;
 
 template <int NH, int CI>
@@ -90,7 +91,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
             tc::mbar_init(&tempty[a], 128);
         }
         tc::mbar_init(done, 1);
-        tc::mbar_init(qready, 128);
+        tc::mbar_init(qready, 256);
         *abort_flag = 0;
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&tmap);
@@ -167,26 +168,29 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
         // first stage q^I (128-byte-swizzled K-major), w^I and the histogram while the
         // producer's first key tiles are already in flight
         {
-            const int et = threadIdx.x - 64;  // 0..127
+            const int et = threadIdx.x - 64;  // 0..255
             const __nv_bfloat16* qg = qI + (int64_t)g * NH * CI;
             constexpr int kChunks = NH * CI / 8;  // 16-byte chunks
-            for (int i = et; i < kChunks; i += 128) {
+            for (int i = et; i < kChunks; i += 256) {
                 const int r = i / (CI / 8), cc = i % (CI / 8);
                 const uint4 v = __ldg(reinterpret_cast<const uint4*>(qg + (int64_t)r * CI + cc * 8));
                 *reinterpret_cast<uint4*>(sB + (cc / 8) * (NH * 128) + tc::sw128_offset(r, cc % 8)) = v;
             }
-            for (int i = et; i < NH; i += 128) sw[i] = wI[(int64_t)g * NH + i];
+            for (int i = et; i < NH; i += 256) sw[i] = wI[(int64_t)g * NH + i];
             if (need_hist)
-                for (int i = et; i < kBins; i += 128) sh[i] = 0;
+                for (int i = et; i < kBins; i += 256) sh[i] = 0;
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(qready);
-            asm volatile("bar.sync 1, 128;" ::: "memory");  // epilogue warps only
+            asm volatile("bar.sync 1, 256;" ::: "memory");  // epilogue warps only
         }
+        // group 0 (warps 2-5) drains accumulator 0 (even tiles), group 1 (warps 6-9)
+        // accumulator 1 (odd tiles), so each group has two tile periods per tile
         const int quarter = warp & 3;          // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;
+        const int eg = (warp - 2) >> 2;
         float* scores = ws.scores + (int64_t)g * ws.ld;
-        int it = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        int it = eg;
+        for (int tile = blockIdx.x + eg * gridDim.x; tile < ntiles; tile += 2 * gridDim.x, it += 2) {
             const int acc = it & 1;
             const uint32_t aph = (it >> 1) & 1;
             if (*abort_flag) break;
