@@ -57,6 +57,8 @@ attn_cuda_core(AttnArgs a)
     float* sQ = smem + kCcChunk * cs;        // [kCcHeads][c]
     __shared__ int s_ent[kCcChunk];
 
+    pdl_launch_dependents();
+    pdl_wait();
     const int split = blockIdx.x, hg = blockIdx.y, g = blockIdx.z;
     const int64_t b = g / a.nq;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -173,13 +175,15 @@ CSA_DEV void store_out<float>(float* p, float v) { *p = v; }
 template <>
 CSA_DEV void store_out<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
-// One CTA per (head, query).  Thread t owns columns 4t..4t+3 (float4 loads) and walks
-// the splits four at a time so that several independent loads are in flight.
+// One CTA per (head, query).  Loads of the partial rows are spread over column quads and
+// split groups so that many independent loads are in flight.
 template <typename TO>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kCombineThreads)
 attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_ml, int splits,
              int n_h, int c, TO* __restrict__ out, float* __restrict__ lse)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     const int h = blockIdx.x, g = blockIdx.y;
     __shared__ float s_w[kMaxSplits];
     __shared__ float s_inv;
@@ -207,35 +211,56 @@ attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_m
     const float inv = s_inv;
     TO* orow = out + ((size_t)g * n_h + h) * c;
     if ((c & 3) == 0) {
-        for (int j = threadIdx.x * 4; j < c; j += blockDim.x * 4) {
+        // thread = (column quad, split group); each group walks every ngrp-th split with
+        // eight loads in flight, then the groups are summed through shared memory
+        __shared__ float4 s_red[kCombineThreads];
+        const int ncq = c / 4;
+        const int ngrp = ncq >= (int)blockDim.x ? 1 : (int)blockDim.x / ncq;
+        for (int cq0 = 0; cq0 < ncq; cq0 += blockDim.x / ngrp) {
+            const int cq = cq0 + (int)threadIdx.x % (blockDim.x / ngrp);
+            const int grp = (int)threadIdx.x / (blockDim.x / ngrp);
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            int i = 0;
-            for (; i + 4 <= splits; i += 4) {
-                float4 v[4];
-                float w[4];
+            if (grp < ngrp && cq < ncq) {
+                const int j = cq * 4;
+                int i = grp;
+                for (; i + 7 * ngrp < splits; i += 8 * ngrp) {
+                    float4 v[8];
+                    float w[8];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    w[u] = s_w[i + u];
-                    v[u] = w[u] != 0.f ? __ldcs(reinterpret_cast<const float4*>(part_o + (base + (size_t)(i + u) * n_h) * c + j))
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int u = 0; u < 8; ++u) {
+                        w[u] = s_w[i + u * ngrp];
+                        v[u] = w[u] != 0.f ? __ldcs(reinterpret_cast<const float4*>(
+                                                 part_o + (base + (size_t)(i + u * ngrp) * n_h) * c + j))
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        acc.x = fmaf(w[u], v[u].x, acc.x); acc.y = fmaf(w[u], v[u].y, acc.y);
+                        acc.z = fmaf(w[u], v[u].z, acc.z); acc.w = fmaf(w[u], v[u].w, acc.w);
+                    }
                 }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    acc.x = fmaf(w[u], v[u].x, acc.x); acc.y = fmaf(w[u], v[u].y, acc.y);
-                    acc.z = fmaf(w[u], v[u].z, acc.z); acc.w = fmaf(w[u], v[u].w, acc.w);
+                for (; i < splits; i += ngrp) {
+                    const float w = s_w[i];
+                    if (w == 0.f) continue;
+                    const float4 v = __ldcs(reinterpret_cast<const float4*>(part_o + (base + (size_t)i * n_h) * c + j));
+                    acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+                    acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
                 }
             }
-            for (; i < splits; ++i) {
-                const float w = s_w[i];
-                if (w == 0.f) continue;
-                const float4 v = __ldcs(reinterpret_cast<const float4*>(part_o + (base + (size_t)i * n_h) * c + j));
-                acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
-                acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+            s_red[threadIdx.x] = acc;
+            __syncthreads();
+            if (grp == 0 && cq < ncq) {
+                for (int q = 1; q < ngrp; ++q) {
+                    const float4 o = s_red[q * (blockDim.x / ngrp) + threadIdx.x];
+                    acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+                }
+                const int j = cq * 4;
+                store_out<TO>(orow + j, acc.x * inv);
+                store_out<TO>(orow + j + 1, acc.y * inv);
+                store_out<TO>(orow + j + 2, acc.z * inv);
+                store_out<TO>(orow + j + 3, acc.w * inv);
             }
-            store_out<TO>(orow + j, acc.x * inv);
-            store_out<TO>(orow + j + 1, acc.y * inv);
-            store_out<TO>(orow + j + 2, acc.z * inv);
-            store_out<TO>(orow + j + 3, acc.w * inv);
+            __syncthreads();
         }
     } else {
         for (int j = threadIdx.x; j < c; j += blockDim.x) {
@@ -259,11 +284,11 @@ int launch_cuda_core(AttnArgs a, const AttnPlan& plan, int dtype, cudaStream_t s
     if (dtype == CSA_BF16) {
         auto kern = attn_cuda_core<__nv_bfloat16>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<grid, 256, smem, stream>>>(a);
+        launch_pdl(kern, grid, dim3(256), smem, stream, a);
     } else {
         auto kern = attn_cuda_core<float>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<grid, 256, smem, stream>>>(a);
+        launch_pdl(kern, grid, dim3(256), smem, stream, a);
     }
     return launch_status();
 }
@@ -276,11 +301,11 @@ int launch_attn_combine(const AttnArgs& a, void* out, int out_bf16, float* lse,
     const int G = a.B * a.nq;
     dim3 grid((unsigned)a.n_h, (unsigned)G);
     if (out_bf16)
-        attn_combine<__nv_bfloat16><<<grid, 128, 0, stream>>>(
-            a.part_o, a.part_ml, a.splits, a.n_h, a.c, static_cast<__nv_bfloat16*>(out), lse);
+        launch_pdl(attn_combine<__nv_bfloat16>, grid, dim3(kCombineThreads), 0, stream, (const float*)a.part_o,
+                   (const float2*)a.part_ml, a.splits, a.n_h, a.c, static_cast<__nv_bfloat16*>(out), lse);
     else
-        attn_combine<float><<<grid, 128, 0, stream>>>(a.part_o, a.part_ml, a.splits, a.n_h, a.c,
-                                                      static_cast<float*>(out), lse);
+        launch_pdl(attn_combine<float>, grid, dim3(kCombineThreads), 0, stream, (const float*)a.part_o,
+                   (const float2*)a.part_ml, a.splits, a.n_h, a.c, static_cast<float*>(out), lse);
     return launch_status();
 }
 

@@ -36,7 +36,8 @@ constexpr int kThreads = 288;       // 4 loader warps, 4 softmax warps, 1 MMA wa
 constexpr int kQBytes = kHeads * kC * 2;          // 128 KB, 8 panels of 16 KB
 constexpr int kCBytes = kE * kC * 2;              // 32 KB, 8 panels of 4 KB
 constexpr int kPBytes = kHeads * 128;             // 16 KB (64 B of each 128 B row used)
-constexpr int kSmem = 1024 + kQBytes + 2 * kCBytes + kPBytes + 256;
+constexpr int kMaxIds = 1024;                     // entry ids of a CTA's range staged in smem
+constexpr int kSmem = 1024 + kQBytes + 2 * kCBytes + kPBytes + 256 + kMaxIds * 4;
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
 
 CSA_DEV void cp_async16(uint32_t dst, const void* src, bool valid)
@@ -63,13 +64,40 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
     uint64_t* Sempty = bars + 6;   // [2] softmax -> MMA      (count 128)
     uint64_t* Pfull = bars + 8;    // softmax -> MMA          (count 128)
     uint64_t* PVdone = bars + 9;   // MMA commit -> softmax
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+    uint64_t* idsready = bars + 10; // loaders -> softmax: entry ids staged (count 128)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
     volatile uint32_t* abort_flag = tmem_slot + 1;
+    int* s_ids = reinterpret_cast<int*>(sP + kPBytes + 256);  // [kMaxIds]
 
+    pdl_launch_dependents();
     const int split = blockIdx.x, half = blockIdx.y, g = blockIdx.z;
     const int64_t b = g / a.nq;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&Cfull[i], kLoaders);
+            tc::mbar_init(&Cempty[i], 1);
+            tc::mbar_init(&Sfull[i], 1);
+            tc::mbar_init(&Sempty[i], kHeads);
+        }
+        tc::mbar_init(Pfull, kHeads);
+        tc::mbar_init(PVdone, 1);
+        tc::mbar_init(idsready, kLoaders);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 8) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    // only shared memory and TMEM were touched so far (overlaps the previous kernel)
+    pdl_wait();
     int64_t count;
     if (a.dense) {
         const int64_t tt = a.t[g];
@@ -82,42 +110,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
     const int64_t p_end = min(count, p_begin + a.per_split);
     const int nchunks = p_end > p_begin ? (int)((p_end - p_begin + kE - 1) / kE) : 0;
     const size_t prow = ((size_t)g * a.splits + split) * kHeads;  // partial row of head 0
-    if (nchunks == 0) {
-        if (half == 0 && threadIdx.x < kHeads) a.part_ml[prow + threadIdx.x] = make_float2(-INFINITY, 0.f);
-        return;
-    }
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&Cfull[i], kLoaders);
-            tc::mbar_init(&Cempty[i], 1);
-            tc::mbar_init(&Sfull[i], 1);
-            tc::mbar_init(&Sempty[i], kHeads);
-        }
-        tc::mbar_init(Pfull, kHeads);
-        tc::mbar_init(PVdone, 1);
-        *abort_flag = 0;
-        tc::fence_mbar_init();
-    }
-    if (warp == 8) {
-        tc::tmem_alloc(tmem_slot, 512);
-        tc::tmem_relinquish();
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = *tmem_slot;
     const __nv_bfloat16* cache = static_cast<const __nv_bfloat16*>(a.cache) + b * a.N_cap * kC;
 
-    // entry id of list position p (-1: padding or outside the cache)
-    auto entry_of = [&](int64_t p) -> int64_t {
+    // entry id of list position p (-1: padding or outside the cache).  Sparse ranges of
+    // up to kMaxIds positions are staged in shared memory once by the loaders, so the
+    // gathers and the softmax masks make no dependent global loads per chunk.
+    const bool ids_staged = !a.dense && (p_end - p_begin) <= kMaxIds;
+    auto entry_global = [&](int64_t p) -> int64_t {
         if (p >= p_end) return -1;
         if (a.dense) return p;
         const int32_t v = __ldg(&a.idx[(int64_t)g * a.k + p]);
         return (v >= 0 && v < a.N_cap) ? v : -1;
     };
+    auto entry_of = [&](int64_t p) -> int64_t {
+        if (ids_staged) return p < p_end ? (int64_t)s_ids[p - p_begin] : -1;
+        return entry_global(p);
+    };
 
-    if (warp < 4) {
+    if (nchunks == 0) {
+        // empty range: an empty partial (max -inf, sum 0) that the combine skips
+        if (half == 0 && threadIdx.x < kHeads) a.part_ml[prow + threadIdx.x] = make_float2(-INFINITY, 0.f);
+    } else if (warp < 4) {
         // ------------------------------------------------------------ loaders
         const int lt = threadIdx.x;
         const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) + (int64_t)g * kHeads * kC;
@@ -126,6 +139,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
             const int row = i >> 6, cc = i & 63;
             cp_async16(q0 + (cc >> 3) * (kHeads * 128) + tc::sw128_offset(row, cc & 7), qg + row * kC + cc * 8, true);
         }
+        if (ids_staged)
+            for (int64_t i = lt; i < p_end - p_begin; i += kLoaders) s_ids[i] = (int)entry_global(p_begin + i);
+        tc::mbar_arrive(idsready);
+        asm volatile("bar.sync 2, 128;" ::: "memory");  // loader warps: ids visible to each other
         for (int j = 0; j < nchunks; ++j) {
             const int buf = j & 1;
             if (*abort_flag) break;
@@ -153,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
         const int h = quarter * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         float m_run = -INFINITY, l_run = 0.f;
-        bool ok = true;
+        bool ok = tc::mbar_wait(idsready, 0, tc::kWaitBudget);
         for (int j = 0; j < nchunks && ok; ++j) {
             const int buf = j & 1;
             if (*abort_flag || !tc::mbar_wait(&Sfull[buf], (j >> 1) & 1, tc::kWaitBudget)) {
@@ -334,7 +351,7 @@ int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cu
     if (!aligned16(a.q) || !aligned16(a.cache)) return CSA_ERR_ALIGN;
     cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     dim3 grid((unsigned)plan.splits, 2u, (unsigned)(a.B * a.nq));
-    attn_tc_kernel<<<grid, kThreads, kSmem, stream>>>(a, status);
+    launch_pdl(attn_tc_kernel, grid, dim3(kThreads), kSmem, stream, a, status);
     return launch_status();
 }
 

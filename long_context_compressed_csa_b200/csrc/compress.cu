@@ -148,6 +148,8 @@ CSA_DEV void pool_rows(const T* __restrict__ Z, const T* __restrict__ X,
 template <typename T, int V>
 __global__ void __launch_bounds__(kThreads) pool_kernel(PoolArgs p)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     const int vecs = p.c / V;
     const int64_t nent = p.e1 - p.e0;
     const int64_t total = (int64_t)p.B * nent * vecs;
@@ -209,11 +211,11 @@ int launch_pool(const PoolArgs& p, int dtype, cudaStream_t stream)
     const int64_t cap = (int64_t)kNumSMs * 64;
     if (blocks > cap) blocks = cap;
     if (dtype == CSA_BF16) {
-        if (vec) pool_kernel<__nv_bfloat16, 8><<<(unsigned)blocks, kThreads, 0, stream>>>(p);
-        else pool_kernel<__nv_bfloat16, 1><<<(unsigned)blocks, kThreads, 0, stream>>>(p);
+        launch_pdl(vec ? pool_kernel<__nv_bfloat16, 8> : pool_kernel<__nv_bfloat16, 1>, dim3((unsigned)blocks),
+                   dim3(kThreads), 0, stream, p);
     } else {
-        if (vec) pool_kernel<float, 4><<<(unsigned)blocks, kThreads, 0, stream>>>(p);
-        else pool_kernel<float, 1><<<(unsigned)blocks, kThreads, 0, stream>>>(p);
+        launch_pdl(vec ? pool_kernel<float, 4> : pool_kernel<float, 1>, dim3((unsigned)blocks), dim3(kThreads), 0,
+                   stream, p);
     }
     return launch_status();
 }

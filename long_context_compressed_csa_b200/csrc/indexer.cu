@@ -68,6 +68,8 @@ scan_cuda_core(const T* __restrict__ qI, const float* __restrict__ wI, const T* 
 {
     extern __shared__ float sq[];  // [n_hI * cI] q, then [n_hI] w
     __shared__ uint32_t sh[kBins];
+    pdl_launch_dependents();
+    pdl_wait();
     const int g = blockIdx.y;
     const int64_t b = g / nq;
     const int64_t vis = visible_count(t, g, m, N_cap);
@@ -259,6 +261,8 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
     __shared__ uint32_t s_bin, s_above, s_last, s_cnt, s_out, s_nt, s_nc, s_bt, s_bc;
     uint2* s_take = s_listA;
     uint2* s_cand = s_listB;
+    pdl_launch_dependents();
+    pdl_wait();
     const int g = blockIdx.y;
     const int tid = threadIdx.x;
     const int64_t vis = visible_count(a.t, g, a.m, a.N_cap);
@@ -444,7 +448,7 @@ int launch_topk_select(const TopkWs& ws, const int64_t* t, int G, int m, int k, 
     ctas = (N_cap + a.chunk - 1) / a.chunk;
     if (ctas < 1) ctas = 1;
     dim3 grid((unsigned)ctas, (unsigned)G);
-    topk_select<<<grid, kSelThreads, 0, stream>>>(a);
+    launch_pdl(topk_select, grid, dim3(kSelThreads), 0, stream, a);
     return launch_status();
 }
 
@@ -460,15 +464,13 @@ int launch_scan_cuda_core(const void* qI, const float* wI, const void* KI, const
     if (dtype == CSA_BF16) {
         auto kern = vec ? scan_cuda_core<__nv_bfloat16, 8> : scan_cuda_core<__nv_bfloat16, 1>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<grid, kScanThreads, smem, stream>>>(static_cast<const __nv_bfloat16*>(qI), wI,
-                                                   static_cast<const __nv_bfloat16*>(KI), t, nq,
-                                                   N_cap, n_hI, cI, m, k, ws);
+        launch_pdl(kern, grid, dim3(kScanThreads), smem, stream, static_cast<const __nv_bfloat16*>(qI), wI,
+                   static_cast<const __nv_bfloat16*>(KI), t, nq, N_cap, n_hI, cI, m, k, ws);
     } else {
         auto kern = vec ? scan_cuda_core<float, 4> : scan_cuda_core<float, 1>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<grid, kScanThreads, smem, stream>>>(static_cast<const float*>(qI), wI,
-                                                   static_cast<const float*>(KI), t, nq, N_cap,
-                                                   n_hI, cI, m, k, ws);
+        launch_pdl(kern, grid, dim3(kScanThreads), smem, stream, static_cast<const float*>(qI), wI,
+                   static_cast<const float*>(KI), t, nq, N_cap, n_hI, cI, m, k, ws);
     }
     return launch_status();
 }

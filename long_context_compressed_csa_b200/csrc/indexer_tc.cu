@@ -73,12 +73,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qready + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
+    pdl_launch_dependents();
     const int g = blockIdx.y;
     const int64_t b = g / nq;
-    const int64_t vis = visible_of(t, g, m, N_cap);
-    const int ntiles = (int)((vis + kTileKeys - 1) / kTileKeys);
-    if ((int)blockIdx.x >= ntiles) return;  // whole CTA idle for this query
-    const bool need_hist = vis > k;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -105,7 +102,17 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
     tc::fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == 0) {
+    // everything above only touched this CTA's own shared memory and TMEM, so it may
+    // overlap the previous kernel; global memory is read only after this point
+    pdl_wait();
+    const int64_t vis = visible_of(t, g, m, N_cap);
+    const int ntiles = (int)((vis + kTileKeys - 1) / kTileKeys);
+    const bool active = (int)blockIdx.x < ntiles;  // otherwise the CTA is idle for this query
+    const bool need_hist = active && vis > k;
+
+    if (!active) {
+        // no key tile for this CTA: fall through to the TMEM release
+    } else if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int it = 0;
@@ -222,7 +229,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
 
     tc::fence_before_sync();
     __syncthreads();
-    if (*abort_flag && threadIdx.x == 0) atomicExch(ws.status, 1u);
+    if (active && *abort_flag && threadIdx.x == 0) atomicExch(ws.status, 1u);
     if (need_hist)
         for (int i = threadIdx.x; i < kBins; i += kTcThreads)
             if (sh[i]) atomicAdd(&ws.hist0[(size_t)g * kBins + i], sh[i]);
@@ -245,8 +252,8 @@ int launch_nh_ci(const CUtensorMap& tmap, const void* qI, const float* wI, const
     auto kern = scan_tc_kernel<NH, CI>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
     dim3 grid((unsigned)ctas, (unsigned)G);
-    kern<<<grid, kTcThreads, Cfg::kSmem, stream>>>(tmap, static_cast<const __nv_bfloat16*>(qI), wI, t, nq, N_cap,
-                                                    m, k, ws);
+    launch_pdl(kern, grid, dim3(kTcThreads), Cfg::kSmem, stream, tmap, static_cast<const __nv_bfloat16*>(qI), wI,
+               t, nq, N_cap, m, k, ws);
     return launch_status();
 }
 
