@@ -175,8 +175,10 @@ CSA_DEV void store_out<float>(float* p, float v) { *p = v; }
 template <>
 CSA_DEV void store_out<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
-// One CTA per (head, query).  Loads of the partial rows are spread over column quads and
-// split groups so that many independent loads are in flight.
+// One CTA per (head, query).  Every split's (max, sum) is read in one round, the
+// weights 2^(m_i - M) are formed in shared memory, and the partial rows are read by
+// (column quad, split group) threads that issue all their loads before using them, so
+// the kernel costs two dependent global round trips rather than one per split.
 template <typename TO>
 __global__ void __launch_bounds__(kCombineThreads)
 attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_ml, int splits,
@@ -184,74 +186,87 @@ attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_m
 {
     pdl_launch_dependents();
     pdl_wait();
+    constexpr int kBatch = 16;  // loads issued per thread before the first use
     const int h = blockIdx.x, g = blockIdx.y;
-    __shared__ float s_w[kMaxSplits];
-    __shared__ float s_inv;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ float s_m[kMaxSplits], s_w[kMaxSplits];
+    __shared__ float s_red[kCombineThreads / 32];
+    __shared__ float4 s_acc[kCombineThreads];
+    __shared__ float s_M, s_inv;
     const size_t base = (size_t)g * splits * n_h + h;
-    if (threadIdx.x < 32) {
+
+    // (max, sum) of every split: one round of loads
+    float mloc = -INFINITY;
+    for (int i = tid; i < splits; i += kCombineThreads) {
+        const float2 ml = part_ml[base + (size_t)i * n_h];
+        s_m[i] = ml.x;
+        s_w[i] = ml.y;
+        mloc = fmaxf(mloc, ml.x);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, off));
+    if (lane == 0) s_red[warp] = mloc;
+    __syncthreads();
+    if (tid == 0) {
         float M = -INFINITY;
-        for (int i = threadIdx.x; i < splits; i += 32) M = fmaxf(M, part_ml[base + (size_t)i * n_h].x);
+        for (int w = 0; w < kCombineThreads / 32; ++w) M = fmaxf(M, s_red[w]);
+        s_M = M;
+    }
+    __syncthreads();
+    const float M = s_M;
+    float lloc = 0.f;
+    for (int i = tid; i < splits; i += kCombineThreads) {
+        const float w = s_m[i] == -INFINITY ? 0.f : exp2f(s_m[i] - M);
+        lloc = fmaf(w, s_w[i], lloc);
+        s_w[i] = w;
+    }
 #pragma unroll
-        for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    for (int off = 16; off; off >>= 1) lloc += __shfl_xor_sync(0xffffffffu, lloc, off);
+    __syncthreads();
+    if (lane == 0) s_red[warp] = lloc;
+    __syncthreads();
+    if (tid == 0) {
         float L = 0.f;
-        for (int i = threadIdx.x; i < splits; i += 32) {
-            const float2 ml = part_ml[base + (size_t)i * n_h];
-            const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-            s_w[i] = w;
-            L += w * ml.y;
-        }
-#pragma unroll
-        for (int off = 16; off; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-        if (threadIdx.x == 0) {
-            s_inv = L > 0.f ? 1.f / L : 0.f;
-            if (lse) lse[(size_t)g * n_h + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
-        }
+        for (int w = 0; w < kCombineThreads / 32; ++w) L += s_red[w];
+        s_inv = L > 0.f ? 1.f / L : 0.f;
+        if (lse) lse[(size_t)g * n_h + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
     }
     __syncthreads();
     const float inv = s_inv;
     TO* orow = out + ((size_t)g * n_h + h) * c;
     if ((c & 3) == 0) {
-        // thread = (column quad, split group); each group walks every ngrp-th split with
-        // eight loads in flight, then the groups are summed through shared memory
-        __shared__ float4 s_red[kCombineThreads];
         const int ncq = c / 4;
-        const int ngrp = ncq >= (int)blockDim.x ? 1 : (int)blockDim.x / ncq;
-        for (int cq0 = 0; cq0 < ncq; cq0 += blockDim.x / ngrp) {
-            const int cq = cq0 + (int)threadIdx.x % (blockDim.x / ngrp);
-            const int grp = (int)threadIdx.x / (blockDim.x / ngrp);
+        const int per = ncq < kCombineThreads ? ncq : kCombineThreads;  // column quads per pass
+        const int ngrp = kCombineThreads / per;                         // split groups
+        for (int cq0 = 0; cq0 < ncq; cq0 += per) {
+            const int cq = cq0 + tid % per;
+            const int grp = tid / per;
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             if (grp < ngrp && cq < ncq) {
-                const int j = cq * 4;
-                int i = grp;
-                for (; i + 7 * ngrp < splits; i += 8 * ngrp) {
-                    float4 v[8];
-                    float w[8];
+                const float* col = part_o + base * c + (size_t)cq * 4;
+                for (int i0 = grp; i0 < splits; i0 += kBatch * ngrp) {
+                    float4 v[kBatch];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        w[u] = s_w[i + u * ngrp];
-                        v[u] = w[u] != 0.f ? __ldcs(reinterpret_cast<const float4*>(
-                                                 part_o + (base + (size_t)(i + u * ngrp) * n_h) * c + j))
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int u = 0; u < kBatch; ++u) {
+                        const int i = i0 + u * ngrp;
+                        v[u] = (i < splits && s_w[i] != 0.f)
+                                   ? __ldcs(reinterpret_cast<const float4*>(col + (size_t)i * n_h * c))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
                     }
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        acc.x = fmaf(w[u], v[u].x, acc.x); acc.y = fmaf(w[u], v[u].y, acc.y);
-                        acc.z = fmaf(w[u], v[u].z, acc.z); acc.w = fmaf(w[u], v[u].w, acc.w);
+                    for (int u = 0; u < kBatch; ++u) {
+                        const int i = i0 + u * ngrp;
+                        const float w = i < splits ? s_w[i] : 0.f;
+                        acc.x = fmaf(w, v[u].x, acc.x); acc.y = fmaf(w, v[u].y, acc.y);
+                        acc.z = fmaf(w, v[u].z, acc.z); acc.w = fmaf(w, v[u].w, acc.w);
                     }
-                }
-                for (; i < splits; i += ngrp) {
-                    const float w = s_w[i];
-                    if (w == 0.f) continue;
-                    const float4 v = __ldcs(reinterpret_cast<const float4*>(part_o + (base + (size_t)i * n_h) * c + j));
-                    acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
-                    acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
                 }
             }
-            s_red[threadIdx.x] = acc;
+            s_acc[tid] = acc;
             __syncthreads();
             if (grp == 0 && cq < ncq) {
                 for (int q = 1; q < ngrp; ++q) {
-                    const float4 o = s_red[q * (blockDim.x / ngrp) + threadIdx.x];
+                    const float4 o = s_acc[q * per + tid];
                     acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
                 }
                 const int j = cq * 4;
@@ -263,7 +278,7 @@ attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_m
             __syncthreads();
         }
     } else {
-        for (int j = threadIdx.x; j < c; j += blockDim.x) {
+        for (int j = tid; j < c; j += kCombineThreads) {
             float acc = 0.f;
             for (int i = 0; i < splits; ++i) {
                 const float w = s_w[i];

@@ -209,8 +209,8 @@ CSA_DEV uint32_t digit_of(uint2 kv, int level)
     }
 }
 
-constexpr int kListCap = 1024;  // candidates kept in shared memory by the last CTA
-constexpr int kPer = 4;         // scores per thread per round of the first pass
+constexpr int kListCap = 2048;  // candidates kept in shared memory by the last CTA
+constexpr int kPer = 8;         // scores per thread per round of the first pass
 constexpr int kRound = kPer * kSelThreads;
 static_assert(kRound <= kListCap, "a round's staging must fit the shared lists");
 constexpr int kRankMax = 256;   // lists up to this size are finished by exact ranking
@@ -255,16 +255,29 @@ CSA_DEV void emit_by_rank(const uint2* list, uint32_t count, uint32_t need, uint
 
 __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
 {
-    __shared__ uint32_t sh[kBins];
+    extern __shared__ __align__(16) uint8_t sel_smem[];
+    uint32_t* sh = reinterpret_cast<uint32_t*>(sel_smem);               // [kBins]
+    uint2* s_listA = reinterpret_cast<uint2*>(sel_smem + kBins * 4);    // [kListCap]
+    uint2* s_listB = s_listA + kListCap;                                 // [kListCap]
     __shared__ uint32_t s_scr[32];
-    __shared__ uint2 s_listA[kListCap], s_listB[kListCap];  // first pass: staged takes / candidates
     __shared__ uint32_t s_bin, s_above, s_last, s_cnt, s_out, s_nt, s_nc, s_bt, s_bc;
-    uint2* s_take = s_listA;
-    uint2* s_cand = s_listB;
+    uint2* s_take = s_listA;  // first pass: staged selections
+    uint2* s_cand = s_listB;  // first pass: staged candidates
     pdl_launch_dependents();
     pdl_wait();
     const int g = blockIdx.y;
     const int tid = threadIdx.x;
+    // the first round's scores, the digit-0 histogram and t go out in one round trip
+    const float* scores0 = a.ws.scores + (int64_t)g * a.ws.ld;
+    const int64_t s_begin = (int64_t)blockIdx.x * a.chunk;
+    const int64_t s_lim = min(a.N_cap, s_begin + a.chunk);
+    uint32_t key0[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int64_t s = s_begin + tid + u * kSelThreads;
+        key0[u] = s < s_lim ? order_key(__ldcg(&scores0[s])) : 0u;
+    }
+    for (int i = tid; i < kBins; i += kSelThreads) sh[i] = __ldcg(&a.ws.hist0[(size_t)g * kBins + i]);
     const int64_t vis = visible_count(a.t, g, a.m, a.N_cap);
     const int k = a.k;
     int32_t* idx_out = a.idx_out + (int64_t)g * k;
@@ -285,7 +298,6 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
         }
     } else {
         // ---- digit 0 threshold from the scan's histogram ----
-        for (int i = tid; i < kBins; i += kSelThreads) sh[i] = __ldcg(&a.ws.hist0[(size_t)g * kBins + i]);
         __syncthreads();
         find_threshold_bin<kBins>(sh, (uint32_t)k, &s_bin, &s_above, s_scr);
         const uint32_t b0 = s_bin;
@@ -296,14 +308,13 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
         // Rounds of kRound scores: every thread loads its kPer scores at once, the
         // selected entries and candidates are staged in shared memory, and one global
         // atomic per list and round reserves their output slots.
-        const int64_t s_begin = (int64_t)blockIdx.x * a.chunk;
         const int64_t s_end = min(vis, s_begin + a.chunk);
         for (int64_t base = s_begin; base < s_end; base += kRound) {
             uint32_t key[kPer];
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
                 const int64_t s = base + tid + u * kSelThreads;
-                key[u] = s < s_end ? order_key(scores[s]) : 0u;
+                key[u] = base == s_begin ? key0[u] : (s < s_end ? order_key(__ldcg(&scores[s])) : 0u);
             }
             if (tid == 0) {
                 s_nt = 0;
@@ -326,9 +337,11 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
                 }
             }
             __syncthreads();
-            if (tid == 0) {
-                s_bt = s_nt ? atomicAdd(&ctr[0], s_nt) : 0u;
-                s_bc = s_nc ? atomicAdd(&ctr[1], s_nc) : 0u;
+            if (tid == 0) {  // both reservations in flight together
+                const uint32_t bt = s_nt ? atomicAdd(&ctr[0], s_nt) : 0u;
+                const uint32_t bc = s_nc ? atomicAdd(&ctr[1], s_nc) : 0u;
+                s_bt = bt;
+                s_bc = bc;
             }
             __syncthreads();
             for (uint32_t i = tid; i < s_nt; i += kSelThreads) {
@@ -440,15 +453,17 @@ int launch_topk_select(const TopkWs& ws, const int64_t* t, int G, int m, int k, 
     a.ws = ws; a.t = t; a.m = m; a.k = k; a.N_cap = N_cap;
     a.idx_out = idx_out; a.scores_out = scores_out;
     int64_t ctas = (2 * kNumSMs + G - 1) / G;
-    const int64_t by_size = (N_cap + 2047) / 2048;
+    const int64_t by_size = (N_cap + kRound - 1) / kRound;
     if (ctas > by_size) ctas = by_size;
     if (ctas < 1) ctas = 1;
     a.chunk = (N_cap + ctas - 1) / ctas;
-    a.chunk = (a.chunk + 255) / 256 * 256;
+    a.chunk = (a.chunk + kRound - 1) / kRound * kRound;  // whole rounds per CTA
     ctas = (N_cap + a.chunk - 1) / a.chunk;
     if (ctas < 1) ctas = 1;
     dim3 grid((unsigned)ctas, (unsigned)G);
-    launch_pdl(topk_select, grid, dim3(kSelThreads), 0, stream, a);
+    const size_t smem = kBins * 4 + 2 * kListCap * sizeof(uint2);
+    cudaFuncSetAttribute(topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    launch_pdl(topk_select, grid, dim3(kSelThreads), smem, stream, a);
     return launch_status();
 }
 
