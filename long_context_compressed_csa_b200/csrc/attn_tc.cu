@@ -65,7 +65,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
     uint64_t* Pfull = bars + 8;    // softmax -> MMA          (count 128)
     uint64_t* PVdone = bars + 9;   // MMA commit -> softmax
     uint64_t* idsready = bars + 10; // loaders -> softmax: entry ids staged (count 128)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+    uint64_t* staged = bars + 11;   // softmax warps: output half staged (count 128)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
     volatile uint32_t* abort_flag = tmem_slot + 1;
     int* s_ids = reinterpret_cast<int*>(sP + kPBytes + 256);  // [kMaxIds]
 
@@ -84,6 +85,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
         tc::mbar_init(Pfull, kHeads);
         tc::mbar_init(PVdone, 1);
         tc::mbar_init(idsready, kLoaders);
+        tc::mbar_init(staged, kHeads);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -245,7 +247,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
         }
         if (ok && !*abort_flag && tc::mbar_wait(PVdone, (nchunks - 1) & 1, tc::kWaitBudget)) {
             tc::fence_after_sync();
-            float* po = a.part_o + (prow + h) * a.c + half * kHalf;
+            // The last P C has completed, so every MMA reading q has too: the q tile (128 KB)
+            // is free and stages the 128 x 256 fp32 output half.  Rows are written with the
+            // 16-byte units XOR-swizzled by (row & 7), then copied out row by row with
+            // coalesced 16-byte stores (one thread per row would scatter 16 B pieces 1 KB
+            // apart).
+            float4* stage = reinterpret_cast<float4*>(sQ);  // [128 rows][64 float4]
             const uint32_t ob = tmem + lane_base + kHalf;
 #pragma unroll 1
             for (int c0 = 0; c0 < kHalf; c0 += 16) {
@@ -253,11 +260,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
                 tc::tmem_ld16(ob + c0, o);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; i += 4)
-                    *reinterpret_cast<float4*>(po + c0 + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+                for (int i = 0; i < 16; i += 4) {
+                    const int q4 = (c0 + i) >> 2;
+                    stage[h * 64 + (q4 ^ (h & 7))] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+                }
             }
             if (half == 0) a.part_ml[prow + h] = make_float2(m_run, l_run);
+            tc::mbar_arrive(staged);
+            if (tc::mbar_wait(staged, 0, tc::kWaitBudget)) {
+                const int st = threadIdx.x - 128;  // 0..127
+                float* po = a.part_o + prow * a.c + half * kHalf;
+#pragma unroll 4
+                for (int i = st; i < kHeads * 64; i += 128) {
+                    const int r = i >> 6, q4 = i & 63;
+                    *reinterpret_cast<float4*>(po + (size_t)r * a.c + q4 * 4) = stage[r * 64 + (q4 ^ (r & 7))];
+                }
+            } else {
+                *abort_flag = 1;
+            }
         } else {
+            tc::mbar_arrive(staged);
             *abort_flag = 1;
             if (half == 0) a.part_ml[prow + h] = make_float2(-INFINITY, 0.f);
         }
