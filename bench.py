@@ -321,10 +321,20 @@ def micro(kind, iters, rotate=4):
     for f in calls:
         f()
     torch.cuda.synchronize()
+    # each call captured once in a CUDA graph, so host launch latency is not timed
+    graphs = []
+    for f in calls:
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            f()
+        graphs.append(gr)
+    for gr in graphs:
+        gr.replay()
+    torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
     for i in range(iters):
         evs[i][0].record()
-        calls[i % len(calls)]()
+        graphs[i % len(graphs)].replay()
         evs[i][1].record()
     torch.cuda.synchronize()
     us = np.array([a.elapsed_time(b) * 1e3 for a, b in evs])
