@@ -4,23 +4,28 @@
 //
 // For one query, S = Q C^T (128 heads x entries, K = c = 512) and O = softmax(S) C
 // (128 heads x 512) are dense contractions against entries shared by every head, so
-// both run on tcgen05 with the heads as the M = 128 dimension.  The fp32 accumulator of
-// O for all 512 columns would fill the whole 512-column TMEM, leaving no room for S,
-// so a CTA owns one half of the output columns (N = 256) and recomputes S: work per
-// entry is 1.5x the minimum, which is cheap next to the entry traffic.
-//
-// CTA = (split of the entry list, output half, query).  Entries stream through in
-// chunks of 32 rows, gathered by index with 16-byte cp.async into a double-buffered
-// 128-byte-swizzled tile; the same bytes serve as the K-major B operand of S and as
-// the MN-major B operand of P C.
-//   warps 0-3 loaders  : q (once) and the entry chunks -> shared memory
-//   warps 4-7 softmax  : S rows from TMEM, online softmax with lazy rescaling (O is
-//                        rescaled in TMEM only when the running max grows by > 2^8),
-//                        P (bf16) -> shared memory; final O half -> partials
-//   warp 8    MMA      : S(j+1) is issued before P(j) C so the tensor core keeps busy
-// Partials (O unnormalised, running max and sum in base 2) are merged by the combine
-// kernel of attn.cu.  Every barrier wait is bounded; a timeout sets the workspace
-// status word and the CTA drains and exits.
+// both run on tcgen05 with the heads as the M = 128 dimension.  An fp32 accumulator for
+// all 512 output columns would fill the whole 512-column TMEM and leave no room for S,
+// so the work is split over a CTA pair (a thread-block cluster of 2) by halves of c:
+//   - CTA r holds q[:, 256r : 256r+256] and, for each chunk of 64 entries, only the
+//     same 256 columns of the entries, so every byte of q and of the cache is loaded
+//     once per pair;
+//   - it computes the partial logits S_r = q[:, half] C[:, half]^T (K = 256), sends them
+//     to its peer through distributed shared memory, and both form S = S_0 + S_1 (same
+//     operand order, bit-identical in both CTAs) and the same softmax;
+//   - it accumulates its own output half O[:, half] += P C[:, half] (N = 256) in TMEM.
+// Entries are gathered by index with 16-byte cp.async into a double-buffered
+// 128-byte-swizzled tile; the same bytes are the K-major B operand of S and the
+// MN-major B operand of P C.
+//   warps 0-3 loaders  : q half (once) and the entry chunks -> shared memory
+//   warps 4-7 softmax  : partial S rows from TMEM -> peer, S, online softmax with lazy
+//                        rescaling (O is rescaled in TMEM only when the running max grows
+//                        by more than 2^8), P (bf16) -> shared memory; final O half ->
+//                        partials through a shared-memory transpose
+//   warp 8    MMA      : S(j+1) is issued before P(j) C so the tensor core stays busy
+// CTA pairs split the entry list; their partials (O unnormalised, running max and sum
+// in base 2) are merged by the combine kernel of attn.cu.  Every barrier wait is
+// bounded; a timeout sets the workspace status word and the CTA drains and exits.
 #include "attn.cuh"
 #include "tc_utils.cuh"
 
@@ -28,50 +33,108 @@ namespace csa {
 namespace {
 
 constexpr int kC = 512;             // entry width handled by this kernel
-constexpr int kHalf = 256;          // output columns per CTA
+constexpr int kHalf = 256;          // columns of c owned by each CTA of the pair
 constexpr int kHeads = 128;         // M
-constexpr int kE = 32;              // entries per chunk (N of S)
+constexpr int kE = 64;              // entries per chunk (N of S, K of P C)
 constexpr int kLoaders = 128;
 constexpr int kThreads = 288;       // 4 loader warps, 4 softmax warps, 1 MMA warp
-constexpr int kQBytes = kHeads * kC * 2;          // 128 KB, 8 panels of 16 KB
-constexpr int kCBytes = kE * kC * 2;              // 32 KB, 8 panels of 4 KB
-constexpr int kPBytes = kHeads * 128;             // 16 KB (64 B of each 128 B row used)
-constexpr int kMaxIds = 1024;                     // entry ids of a CTA's range staged in smem
-constexpr int kSmem = 1024 + kQBytes + 2 * kCBytes + kPBytes + 256 + kMaxIds * 4;
+constexpr int kQBytes = kHeads * kHalf * 2;       // 64 KB: 4 panels of 128 rows x 128 B
+constexpr int kCBytes = kE * kHalf * 2;           // 32 KB: 4 panels of 64 rows x 128 B
+constexpr int kPBytes = kHeads * kE * 2;          // 16 KB: 128 rows x 128 B
+constexpr int kRBytes = kHeads * kE * 4;          // 32 KB: peer partial S, fp32
+constexpr int kMaxIds = 1024;                     // entry ids of a range staged in smem
+constexpr int kBarBytes = 256;
+constexpr int kSmem = 1024 + kQBytes + 2 * kCBytes + kPBytes + 2 * kRBytes + kBarBytes + kMaxIds * 4;
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
+static_assert(kQBytes + 2 * kCBytes >= kHeads * kHalf * 4, "output staging reuses q + chunks");
 
 CSA_DEV void cp_async16(uint32_t dst, const void* src, bool valid)
 {
     const int n = valid ? 16 : 0;  // 0 bytes read -> 16 zero bytes written
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
 }
-CSA_DEV void cp_async_wait_all()
+CSA_DEV void cp_async_wait_all() { asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory"); }
+
+// ---- cluster (distributed shared memory) helpers
+CSA_DEV uint32_t cluster_rank()
 {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+CSA_DEV uint32_t peer_addr(uint32_t local_smem_addr, uint32_t peer)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem_addr), "r"(peer));
+    return r;
+}
+CSA_DEV void st_cluster_v4(uint32_t addr, float4 v)
+{
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
+}
+CSA_DEV void mbar_arrive_remote(uint32_t remote_bar)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+CSA_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(tc::smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// bounded wait on a barrier that the peer CTA arrives on
+CSA_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, long long budget)
+{
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_cluster(bar, parity))
+        if (clock64() - t0 > budget) return false;
+    return true;
+}
+CSA_DEV void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32_t* status)
+// float4 q (0..15) of row h of a 64-float row, XOR-swizzled so that the 32 rows of a
+// warp spread over the banks
+CSA_DEV int rswz(int h, int q) { return h * 16 + (q ^ (h & 15)); }
+
+__global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint32_t* status)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
-    uint8_t* sC0 = sQ + kQBytes;  // chunk buffer `buf` at sC0 + buf * kCBytes
-    uint8_t* sP = sQ + kQBytes + 2 * kCBytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPBytes);
-    uint64_t* Cfull = bars;        // [2] loaders -> MMA      (count 128)
-    uint64_t* Cempty = bars + 2;   // [2] MMA commit -> loaders
-    uint64_t* Sfull = bars + 4;    // [2] MMA commit -> softmax
-    uint64_t* Sempty = bars + 6;   // [2] softmax -> MMA      (count 128)
-    uint64_t* Pfull = bars + 8;    // softmax -> MMA          (count 128)
-    uint64_t* PVdone = bars + 9;   // MMA commit -> softmax
-    uint64_t* idsready = bars + 10; // loaders -> softmax: entry ids staged (count 128)
-    uint64_t* staged = bars + 11;   // softmax warps: output half staged (count 128)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+    uint8_t* sC0 = sQ + kQBytes;                      // chunk buffer b at sC0 + b * kCBytes
+    uint8_t* sP = sC0 + 2 * kCBytes;
+    float4* sR = reinterpret_cast<float4*>(sP + kPBytes);  // [2][128][16] peer partial S
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPBytes + 2 * kRBytes);
+    uint64_t* Cfull = bars;         // [2] loaders -> MMA            (count 128)
+    uint64_t* Cempty = bars + 2;    // [2] MMA commit -> loaders
+    uint64_t* Sfull = bars + 4;     // [2] MMA commit -> softmax
+    uint64_t* Sempty = bars + 6;    // [2] softmax -> MMA            (count 128)
+    uint64_t* Rfull = bars + 8;     // [2] peer softmax -> softmax   (count 128, remote)
+    uint64_t* Rfree = bars + 10;    // [2] peer consumed our partial (count 128, remote)
+    uint64_t* Pfull = bars + 12;    // softmax -> MMA                (count 128)
+    uint64_t* PVdone = bars + 13;   // MMA commit -> softmax
+    uint64_t* idsready = bars + 14; // loaders -> softmax            (count 128)
+    uint64_t* staged = bars + 15;   // softmax warps: output staged  (count 128)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
     volatile uint32_t* abort_flag = tmem_slot + 1;
-    int* s_ids = reinterpret_cast<int*>(sP + kPBytes + 256);  // [kMaxIds]
+    int* s_ids = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);  // [kMaxIds]
 
     pdl_launch_dependents();
-    const int split = blockIdx.x, half = blockIdx.y, g = blockIdx.z;
+    const int split = blockIdx.x, g = blockIdx.z;
+    const int half = (int)cluster_rank();  // == blockIdx.y (cluster of 2 along y)
+    const uint32_t peer = (uint32_t)(half ^ 1);
     const int64_t b = g / a.nq;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -81,6 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
             tc::mbar_init(&Cempty[i], 1);
             tc::mbar_init(&Sfull[i], 1);
             tc::mbar_init(&Sempty[i], kHeads);
+            tc::mbar_init(&Rfull[i], kHeads);
+            tc::mbar_init(&Rfree[i], kHeads);
         }
         tc::mbar_init(Pfull, kHeads);
         tc::mbar_init(PVdone, 1);
@@ -94,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
         tc::tmem_relinquish();
     }
     tc::fence_before_sync();
-    __syncthreads();
+    cluster_sync();  // both CTAs' barriers are initialised before any remote arrival
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
@@ -112,11 +177,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
     const int64_t p_end = min(count, p_begin + a.per_split);
     const int nchunks = p_end > p_begin ? (int)((p_end - p_begin + kE - 1) / kE) : 0;
     const size_t prow = ((size_t)g * a.splits + split) * kHeads;  // partial row of head 0
-    const __nv_bfloat16* cache = static_cast<const __nv_bfloat16*>(a.cache) + b * a.N_cap * kC;
+    const __nv_bfloat16* cache = static_cast<const __nv_bfloat16*>(a.cache) + b * a.N_cap * kC + half * kHalf;
 
     // entry id of list position p (-1: padding or outside the cache).  Sparse ranges of
-    // up to kMaxIds positions are staged in shared memory once by the loaders, so the
-    // gathers and the softmax masks make no dependent global loads per chunk.
+    // up to kMaxIds positions are staged in shared memory once by the loaders.
     const bool ids_staged = !a.dense && (p_end - p_begin) <= kMaxIds;
     auto entry_global = [&](int64_t p) -> int64_t {
         if (p >= p_end) return -1;
@@ -135,10 +199,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
     } else if (warp < 4) {
         // ------------------------------------------------------------ loaders
         const int lt = threadIdx.x;
-        const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) + (int64_t)g * kHeads * kC;
+        const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) + (int64_t)g * kHeads * kC + half * kHalf;
         const uint32_t q0 = tc::smem_u32(sQ);
-        for (int i = lt; i < kHeads * (kC / 8); i += kLoaders) {
-            const int row = i >> 6, cc = i & 63;
+        for (int i = lt; i < kHeads * (kHalf / 8); i += kLoaders) {
+            const int row = i >> 5, cc = i & 31;
             cp_async16(q0 + (cc >> 3) * (kHeads * 128) + tc::sw128_offset(row, cc & 7), qg + row * kC + cc * 8, true);
         }
         if (ids_staged)
@@ -155,8 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
             const uint32_t c0 = tc::smem_u32(sC0 + buf * kCBytes);
             const int64_t p0 = p_begin + (int64_t)j * kE;
 #pragma unroll 4
-            for (int i = lt; i < kE * (kC / 8); i += kLoaders) {
-                const int row = i >> 6, cc = i & 63;
+            for (int i = lt; i < kE * (kHalf / 8); i += kLoaders) {
+                const int row = i >> 5, cc = i & 31;
                 const int64_t e = entry_of(p0 + row);
                 const __nv_bfloat16* src = cache + (e >= 0 ? e : 0) * kC + cc * 8;
                 cp_async16(c0 + (cc >> 3) * (kE * 128) + tc::sw128_offset(row, cc & 7), src, e >= 0);
@@ -175,30 +239,63 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
         bool ok = tc::mbar_wait(idsready, 0, tc::kWaitBudget);
         for (int j = 0; j < nchunks && ok; ++j) {
             const int buf = j & 1;
-            if (*abort_flag || !tc::mbar_wait(&Sfull[buf], (j >> 1) & 1, tc::kWaitBudget)) {
-                *abort_flag = 1;
+            const uint32_t ph = (j >> 1) & 1;
+            if (*abort_flag || !tc::mbar_wait(&Sfull[buf], ph, tc::kWaitBudget)) {
                 ok = false;
                 break;
             }
             tc::fence_after_sync();
             float s[kE];
-            tc::tmem_ld16(tmem + lane_base + buf * kE, s);
-            tc::tmem_ld16(tmem + lane_base + buf * kE + 16, s + 16);
+#pragma unroll
+            for (int c0 = 0; c0 < kE; c0 += 16) tc::tmem_ld16(tmem + lane_base + buf * kE + c0, s + c0);
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             tc::mbar_arrive(&Sempty[buf]);
+            // send this half's partial logits to the peer once its receive buffer `buf`
+            // is free (consumed at chunk j-2), then signal it
+            if (!mbar_wait_cluster(&Rfree[buf], ph ^ 1, tc::kWaitBudget)) {
+                ok = false;
+                break;
+            }
+            {
+                const uint32_t dst = peer_addr(tc::smem_u32(sR + buf * (kHeads * 16)), peer);
+#pragma unroll
+                for (int q = 0; q < kE / 4; ++q)
+                    st_cluster_v4(dst + 16u * (uint32_t)rswz(h, q),
+                                  make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]));
+                mbar_arrive_remote(peer_addr(tc::smem_u32(&Rfull[buf]), peer));
+            }
+            // the peer's partial logits, then S = S_0 + S_1 in the same order on both CTAs
+            if (!mbar_wait_cluster(&Rfull[buf], ph, tc::kWaitBudget)) {
+                ok = false;
+                break;
+            }
+            const float4* rrow = sR + buf * (kHeads * 16);
+#pragma unroll
+            for (int q = 0; q < kE / 4; ++q) {
+                const float4 o = rrow[rswz(h, q)];
+                if (half == 0) {
+                    s[4 * q] = s[4 * q] + o.x; s[4 * q + 1] = s[4 * q + 1] + o.y;
+                    s[4 * q + 2] = s[4 * q + 2] + o.z; s[4 * q + 3] = s[4 * q + 3] + o.w;
+                } else {
+                    s[4 * q] = o.x + s[4 * q]; s[4 * q + 1] = o.y + s[4 * q + 1];
+                    s[4 * q + 2] = o.z + s[4 * q + 2]; s[4 * q + 3] = o.w + s[4 * q + 3];
+                }
+            }
+            mbar_arrive_remote(peer_addr(tc::smem_u32(&Rfree[buf]), peer));  // our buffer is free again
             const int64_t p0 = p_begin + (int64_t)j * kE;
-            const unsigned vmask = __ballot_sync(0xffffffffu, entry_of(p0 + lane) >= 0);
+            const unsigned vlo = __ballot_sync(0xffffffffu, entry_of(p0 + lane) >= 0);
+            const unsigned vhi = __ballot_sync(0xffffffffu, entry_of(p0 + 32 + lane) >= 0);
             float cmax = -INFINITY;
 #pragma unroll
             for (int e = 0; e < kE; ++e) {
-                s[e] = ((vmask >> e) & 1u) ? s[e] * a.scale_log2 : -INFINITY;
+                const bool valid = (((e < 32) ? (vlo >> e) : (vhi >> (e - 32))) & 1u) != 0;
+                s[e] = valid ? s[e] * a.scale_log2 : -INFINITY;
                 cmax = fmaxf(cmax, s[e]);
             }
             if (j > 0) {
                 // P buffer and O are free once the previous chunk's P C has finished
                 if (!tc::mbar_wait(PVdone, (j - 1) & 1, tc::kWaitBudget)) {
-                    *abort_flag = 1;
                     ok = false;
                     break;
                 }
@@ -247,11 +344,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
         }
         if (ok && !*abort_flag && tc::mbar_wait(PVdone, (nchunks - 1) & 1, tc::kWaitBudget)) {
             tc::fence_after_sync();
-            // The last P C has completed, so every MMA reading q has too: the q tile (128 KB)
-            // is free and stages the 128 x 256 fp32 output half.  Rows are written with the
-            // 16-byte units XOR-swizzled by (row & 7), then copied out row by row with
-            // coalesced 16-byte stores (one thread per row would scatter 16 B pieces 1 KB
-            // apart).
+            // The last P C has completed, so every MMA reading q and the chunks has too:
+            // those 128 KB stage the 128 x 256 fp32 output half.  Rows are written with
+            // 16-byte units XOR-swizzled by (row & 7) and copied out row by row with
+            // coalesced 16-byte stores.
             float4* stage = reinterpret_cast<float4*>(sQ);  // [128 rows][64 float4]
             const uint32_t ob = tmem + lane_base + kHalf;
 #pragma unroll 1
@@ -298,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
                 tc::fence_after_sync();
                 const uint32_t c0 = tc::smem_u32(sC0 + buf * kCBytes);
 #pragma unroll
-                for (int p = 0; p < kC / 64; ++p) {
+                for (int p = 0; p < kHalf / 64; ++p) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t ad = tc::smem_desc_sw128(q0 + p * (kHeads * 128) + kk * 32, 16, 1024);
@@ -322,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
                 }
                 tc::fence_after_sync();
                 const int buf = j & 1;
-                const uint32_t c0 = tc::smem_u32(sC0 + buf * kCBytes) + half * 4 * (kE * 128);
+                const uint32_t c0 = tc::smem_u32(sC0 + buf * kCBytes);
 #pragma unroll
                 for (int kk = 0; kk < kE / 16; ++kk) {
                     const uint64_t ad = tc::smem_desc_sw128(p0 + kk * 32, 16, 1024);
@@ -343,6 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a, uint32
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, 512);
     }
+    cluster_sync();  // the peer may write into this CTA's shared memory until here
 }
 
 }  // namespace
@@ -355,7 +452,7 @@ AttnPlan attn_plan_tc(int G, int n_h, int c, int64_t entries)
     (void)c;
     AttnPlan p;
     const int64_t chunks = (entries + kE - 1) / kE;
-    int64_t splits = kNumSMs / (2 * (int64_t)G);
+    int64_t splits = kNumSMs / (2 * (int64_t)G);  // one CTA pair per split and query
     if (splits < 1) splits = 1;
     if (splits > chunks) splits = chunks;
     if (splits < 1) splits = 1;
@@ -371,9 +468,23 @@ AttnPlan attn_plan_tc(int G, int n_h, int c, int64_t entries)
 int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cudaStream_t stream)
 {
     if (!aligned16(a.q) || !aligned16(a.cache)) return CSA_ERR_ALIGN;
-    cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    dim3 grid((unsigned)plan.splits, 2u, (unsigned)(a.B * a.nq));
-    launch_pdl(attn_tc_kernel, grid, dim3(kThreads), kSmem, stream, a, status);
+    cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)plan.splits, 2u, (unsigned)(a.B * a.nq));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 2;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaLaunchKernelEx(&cfg, attn_pair_kernel, a, status);
     return launch_status();
 }
 

@@ -209,6 +209,19 @@ CSA_DEV uint32_t digit_of(uint2 kv, int level)
     }
 }
 
+// Copy a 4096-bin histogram from global to shared memory.  All loads are issued before
+// the first store so that the copy costs one round trip (a load-store loop would be
+// serialised into one round trip per iteration).
+CSA_DEV void load_hist(uint32_t* sh, const uint32_t* gh)
+{
+    constexpr int kPerThread = kBins / kSelThreads;
+    uint32_t v[kPerThread];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) v[u] = __ldcg(&gh[threadIdx.x + u * kSelThreads]);
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) sh[threadIdx.x + u * kSelThreads] = v[u];
+}
+
 constexpr int kListCap = 2048;  // candidates kept in shared memory by the last CTA
 constexpr int kPer = 8;         // scores per thread per round of the first pass
 constexpr int kRound = kPer * kSelThreads;
@@ -277,7 +290,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
         const int64_t s = s_begin + tid + u * kSelThreads;
         key0[u] = s < s_lim ? order_key(__ldcg(&scores0[s])) : 0u;
     }
-    for (int i = tid; i < kBins; i += kSelThreads) sh[i] = __ldcg(&a.ws.hist0[(size_t)g * kBins + i]);
+    load_hist(sh, a.ws.hist0 + (size_t)g * kBins);
     const int64_t vis = visible_count(a.t, g, a.m, a.N_cap);
     const int k = a.k;
     int32_t* idx_out = a.idx_out + (int64_t)g * k;
@@ -378,11 +391,29 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
         // are kept in shared memory so the remaining passes make no global round trips.
         if (tid == 0) s_out = __ldcg(&ctr[0]);
         uint32_t count = __ldcg(&ctr[1]);
-        for (int i = tid; i < kBins; i += kSelThreads) sh[i] = __ldcg(&a.ws.hist1[(size_t)g * kBins + i]);
+        load_hist(sh, a.ws.hist1 + (size_t)g * kBins);
         __syncthreads();
         uint32_t need = (uint32_t)k - s_out;
         uint2* list = cand;
         bool in_smem = false;
+        if (count <= (uint32_t)kListCap) {
+            // bring the candidates into shared memory with one batched round of loads
+            constexpr int kPerT = kListCap / kSelThreads;
+            uint2 v[kPerT];
+#pragma unroll
+            for (int u = 0; u < kPerT; ++u) {
+                const uint32_t i = tid + u * kSelThreads;
+                v[u] = i < count ? __ldcg(&cand[i]) : make_uint2(0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kPerT; ++u) {
+                const uint32_t i = tid + u * kSelThreads;
+                if (i < count) s_listA[i] = v[u];
+            }
+            __syncthreads();
+            list = s_listA;
+            in_smem = true;
+        }
         for (int level = 1; need > 0; ++level) {
             if (need >= count) {  // every remaining candidate is selected
                 emit_all(list, in_smem, count, &s_out, k, idx_out, sc_out);

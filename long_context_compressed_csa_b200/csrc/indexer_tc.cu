@@ -178,10 +178,23 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
             const int et = threadIdx.x - 64;  // 0..255
             const __nv_bfloat16* qg = qI + (int64_t)g * NH * CI;
             constexpr int kChunks = NH * CI / 8;  // 16-byte chunks
-            for (int i = et; i < kChunks; i += 256) {
-                const int r = i / (CI / 8), cc = i % (CI / 8);
-                const uint4 v = __ldg(reinterpret_cast<const uint4*>(qg + (int64_t)r * CI + cc * 8));
-                *reinterpret_cast<uint4*>(sB + (cc / 8) * (NH * 128) + tc::sw128_offset(r, cc % 8)) = v;
+            constexpr int kPer = (kChunks + 255) / 256;
+            uint4 v[kPer];
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {  // all loads first: one round trip
+                const int i = et + u * 256;
+                if (i < kChunks) {
+                    const int r = i / (CI / 8), cc = i % (CI / 8);
+                    v[u] = __ldg(reinterpret_cast<const uint4*>(qg + (int64_t)r * CI + cc * 8));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int i = et + u * 256;
+                if (i < kChunks) {
+                    const int r = i / (CI / 8), cc = i % (CI / 8);
+                    *reinterpret_cast<uint4*>(sB + (cc / 8) * (NH * 128) + tc::sw128_offset(r, cc % 8)) = v[u];
+                }
             }
             for (int i = et; i < NH; i += 256) sw[i] = wI[(int64_t)g * NH + i];
             if (need_hist)
