@@ -54,6 +54,8 @@ CSA_DEV void cp_async16(uint32_t dst, const void* src, bool valid)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
 }
 CSA_DEV void cp_async_wait_all() { asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory"); }
+CSA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+CSA_DEV void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }  // all but the newest group
 
 // ---- cluster (distributed shared memory) helpers
 CSA_DEV uint32_t cluster_rank()
@@ -209,6 +211,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
             for (int64_t i = lt; i < p_end - p_begin; i += kLoaders) s_ids[i] = (int)entry_global(p_begin + i);
         tc::mbar_arrive(idsready);
         asm volatile("bar.sync 2, 128;" ::: "memory");  // loader warps: ids visible to each other
+        // chunk j is issued before chunk j-1 is waited for and signalled, so two chunk
+        // loads are in flight whenever both buffers are free
+        int issued = 0;
         for (int j = 0; j < nchunks; ++j) {
             const int buf = j & 1;
             if (*abort_flag) break;
@@ -225,11 +230,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
                 const __nv_bfloat16* src = cache + (e >= 0 ? e : 0) * kC + cc * 8;
                 cp_async16(c0 + (cc >> 3) * (kE * 128) + tc::sw128_offset(row, cc & 7), src, e >= 0);
             }
-            cp_async_wait_all();
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(&Cfull[buf]);
+            cp_async_commit();
+            issued = j + 1;
+            if (j > 0) {
+                cp_async_wait_prev();  // chunk j-1 (and q with chunk 0) has landed
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(&Cfull[(j - 1) & 1]);
+            }
         }
         cp_async_wait_all();
+        if (issued > 0) {
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(&Cfull[(issued - 1) & 1]);
+        }
     } else if (warp < 8) {
         // ------------------------------------------------------------ softmax
         const int quarter = warp & 3;

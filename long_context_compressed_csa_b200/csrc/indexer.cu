@@ -222,6 +222,31 @@ CSA_DEV void load_hist(uint32_t* sh, const uint32_t* gh)
     for (int u = 0; u < kPerThread; ++u) sh[threadIdx.x + u * kSelThreads] = v[u];
 }
 
+// Exclusive prefix sum of v over the kSelThreads threads of the block (thread order);
+// *total receives the block sum.  s_warp: 32 words of shared scratch.  All threads call.
+CSA_DEV uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp, uint32_t* total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+    }
+    __syncthreads();  // s_warp may still be read by a previous use
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    uint32_t base = 0, sum = 0;
+#pragma unroll
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+        const uint32_t x = s_warp[w];
+        base += w < warp ? x : 0u;
+        sum += x;
+    }
+    if (threadIdx.x == 0) *total = sum;
+    return base + incl - v;
+}
+
 constexpr int kListCap = 2048;  // candidates kept in shared memory by the last CTA
 constexpr int kPer = 8;         // scores per thread per round of the first pass
 constexpr int kRound = kPer * kSelThreads;
@@ -329,25 +354,33 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
                 const int64_t s = base + tid + u * kSelThreads;
                 key[u] = base == s_begin ? key0[u] : (s < s_end ? order_key(__ldcg(&scores[s])) : 0u);
             }
-            if (tid == 0) {
-                s_nt = 0;
-                s_nc = 0;
-            }
-            __syncthreads();
+            // slots from one block-wide exclusive scan of (selected, candidate) counts
+            // packed in 16-bit halves, instead of one shared atomic per element
+            uint32_t cnt = 0;
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
                 const int64_t s = base + tid + u * kSelThreads;
-                const bool in = s < s_end;
                 const uint32_t d0 = key[u] >> 20;
-                const bool take = in && d0 > b0;
-                const bool cnd = in && d0 == b0;
-                const uint32_t tp = warp_append(&s_nt, take);
-                if (take) s_take[tp] = make_uint2(key[u], (uint32_t)s);
-                const uint32_t cp = warp_append(&s_nc, cnd);
-                if (cnd) {
-                    s_cand[cp] = make_uint2(key[u], (uint32_t)s);
+                if (s < s_end) cnt += d0 > b0 ? 1u : (d0 == b0 ? 0x10000u : 0u);
+            }
+            uint32_t excl = block_excl_scan(cnt, s_scr, &s_nt);
+            uint32_t tp = excl & 0xffffu, cp = excl >> 16;
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int64_t s = base + tid + u * kSelThreads;
+                if (s >= s_end) continue;
+                const uint32_t d0 = key[u] >> 20;
+                if (d0 > b0) {
+                    s_take[tp++] = make_uint2(key[u], (uint32_t)s);
+                } else if (d0 == b0) {
+                    s_cand[cp++] = make_uint2(key[u], (uint32_t)s);
                     atomicAdd(&sh[(key[u] >> 8) & 0xfffu], 1u);
                 }
+            }
+            if (tid == 0) {
+                const uint32_t tot = s_nt;
+                s_nt = tot & 0xffffu;
+                s_nc = tot >> 16;
             }
             __syncthreads();
             if (tid == 0) {  // both reservations in flight together
