@@ -211,9 +211,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
             for (int64_t i = lt; i < p_end - p_begin; i += kLoaders) s_ids[i] = (int)entry_global(p_begin + i);
         tc::mbar_arrive(idsready);
         asm volatile("bar.sync 2, 128;" ::: "memory");  // loader warps: ids visible to each other
-        // chunk j is issued before chunk j-1 is waited for and signalled, so two chunk
-        // loads are in flight whenever both buffers are free
-        int issued = 0;
+        // Chunks 0 and 1 are loaded concurrently (both buffers start free); from chunk 2
+        // on, chunk j is issued once P C of chunk j-2 has released its buffer and is
+        // signalled when it has landed.  Chunk j-1 is always signalled before the wait for
+        // a buffer, because that wait depends on the MMA having consumed chunk j-1.
         for (int j = 0; j < nchunks; ++j) {
             const int buf = j & 1;
             if (*abort_flag) break;
@@ -231,18 +232,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
                 cp_async16(c0 + (cc >> 3) * (kE * 128) + tc::sw128_offset(row, cc & 7), src, e >= 0);
             }
             cp_async_commit();
-            issued = j + 1;
-            if (j > 0) {
-                cp_async_wait_prev();  // chunk j-1 (and q with chunk 0) has landed
+            if (j == 0 && nchunks > 1) continue;  // issue chunk 1 before waiting for chunk 0
+            if (j == 1) {
+                cp_async_wait_prev();  // chunk 0 (with q) has landed; chunk 1 may be in flight
                 tc::fence_proxy_async_smem();
-                tc::mbar_arrive(&Cfull[(j - 1) & 1]);
+                tc::mbar_arrive(&Cfull[0]);
             }
+            cp_async_wait_all();
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(&Cfull[buf]);
         }
         cp_async_wait_all();
-        if (issued > 0) {
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(&Cfull[(issued - 1) & 1]);
-        }
     } else if (warp < 8) {
         // ------------------------------------------------------------ softmax
         const int quarter = warp & 3;
