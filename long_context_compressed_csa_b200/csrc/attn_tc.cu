@@ -97,13 +97,35 @@ CSA_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, long long budget)
 {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait_cluster(bar, parity))
+    for (int polls = 0; !mbar_try_wait_cluster(bar, parity); ++polls) {
         if (clock64() - t0 > budget) return false;
+        if (polls >= 8) __nanosleep(32);
+    }
     return true;
 }
+// One bulk copy of `bytes` from this CTA's shared memory to a peer CTA's shared memory;
+// completion is counted in bytes on the peer's mbarrier.
+CSA_DEV void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes, uint32_t mbar_cluster)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t"
+        "cp.async.bulk.commit_group;" ::"r"(dst_cluster),
+        "r"(src_cta), "r"(bytes), "r"(mbar_cluster)
+        : "memory");
+}
+// Wait until every bulk copy this thread issued has finished reading its source.
+CSA_DEV void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 CSA_DEV void cluster_sync()
 {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 2^x with the hardware exponential unit (arguments here are <= 8, results >= 0)
+CSA_DEV float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // float4 q (0..15) of row h of a 64-float row, XOR-swizzled so that the 32 rows of a
@@ -117,14 +139,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
     uint8_t* sQ = smem;
     uint8_t* sC0 = sQ + kQBytes;                      // chunk buffer b at sC0 + b * kCBytes
     uint8_t* sP = sC0 + 2 * kCBytes;
-    float4* sR = reinterpret_cast<float4*>(sP + kPBytes);  // [2][128][16] peer partial S
+    float4* sR = reinterpret_cast<float4*>(sP + kPBytes);  // [128][16] peer partial S (received)
+    float4* sX = sR + kHeads * 16;                         // [128][16] own partial S (to send)
     uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPBytes + 2 * kRBytes);
     uint64_t* Cfull = bars;         // [2] loaders -> MMA            (count 128)
     uint64_t* Cempty = bars + 2;    // [2] MMA commit -> loaders
     uint64_t* Sfull = bars + 4;     // [2] MMA commit -> softmax
     uint64_t* Sempty = bars + 6;    // [2] softmax -> MMA            (count 128)
-    uint64_t* Rfull = bars + 8;     // [2] peer softmax -> softmax   (count 128, remote)
-    uint64_t* Rfree = bars + 10;    // [2] peer consumed our partial (count 128, remote)
+    uint64_t* Rfull = bars + 8;     // peer's bulk copy landed in sR (count 1 + bytes)
+    uint64_t* Xready = bars + 9;    // own partial staged in sX      (count 128)
+    uint64_t* Rfree = bars + 10;    // peer consumed what we sent    (count 128, remote)
+    uint64_t* Xfree = bars + 11;    // our bulk copy has read sX     (count 1)
     uint64_t* Pfull = bars + 12;    // softmax -> MMA                (count 128)
     uint64_t* PVdone = bars + 13;   // MMA commit -> softmax
     uint64_t* idsready = bars + 14; // loaders -> softmax            (count 128)
@@ -146,9 +171,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
             tc::mbar_init(&Cempty[i], 1);
             tc::mbar_init(&Sfull[i], 1);
             tc::mbar_init(&Sempty[i], kHeads);
-            tc::mbar_init(&Rfull[i], kHeads);
-            tc::mbar_init(&Rfree[i], kHeads);
         }
+        tc::mbar_init(Rfull, 1);
+        tc::mbar_init(Xready, kHeads);
+        tc::mbar_init(Rfree, kHeads);
+        tc::mbar_init(Xfree, 1);
         tc::mbar_init(Pfull, kHeads);
         tc::mbar_init(PVdone, 1);
         tc::mbar_init(idsready, kLoaders);
@@ -264,29 +291,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             tc::mbar_arrive(&Sempty[buf]);
-            // send this half's partial logits to the peer once its receive buffer `buf`
-            // is free (consumed at chunk j-2), then signal it
-            if (!mbar_wait_cluster(&Rfree[buf], ph ^ 1, tc::kWaitBudget)) {
+            // Exchange of the partial logits with the peer: this half's rows are staged in
+            // sX and moved by one bulk copy into the peer's sR, which signals the peer's
+            // Rfull with the byte count; one receive and one send buffer, so each side
+            // waits until the other has consumed the previous chunk.
+            const uint32_t xph = j & 1;
+            if (threadIdx.x == 128) tc::mbar_arrive_expect_tx(Rfull, kRBytes);  // arm this chunk's receive
+            if (j > 0 && !tc::mbar_wait(Xfree, xph ^ 1, tc::kWaitBudget)) {       // previous copy has read sX
                 ok = false;
                 break;
             }
-            {
-                const uint32_t dst = peer_addr(tc::smem_u32(sR + buf * (kHeads * 16)), peer);
 #pragma unroll
-                for (int q = 0; q < kE / 4; ++q)
-                    st_cluster_v4(dst + 16u * (uint32_t)rswz(h, q),
-                                  make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]));
-                mbar_arrive_remote(peer_addr(tc::smem_u32(&Rfull[buf]), peer));
+            for (int q = 0; q < kE / 4; ++q)
+                sX[rswz(h, q)] = make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(Xready);
+            if (threadIdx.x == 128) {
+                if (!tc::mbar_wait(Xready, xph, tc::kWaitBudget) || !mbar_wait_cluster(Rfree, xph ^ 1, tc::kWaitBudget)) {
+                    *abort_flag = 1;
+                } else {
+                    bulk_copy_to_peer(peer_addr(tc::smem_u32(sR), peer), tc::smem_u32(sX), kRBytes,
+                                      peer_addr(tc::smem_u32(Rfull), peer));
+                    bulk_wait_read();
+                }
+                tc::mbar_arrive(Xfree);
             }
             // the peer's partial logits, then S = S_0 + S_1 in the same order on both CTAs
-            if (!mbar_wait_cluster(&Rfull[buf], ph, tc::kWaitBudget)) {
+            if (!mbar_wait_cluster(Rfull, xph, tc::kWaitBudget)) {
                 ok = false;
                 break;
             }
-            const float4* rrow = sR + buf * (kHeads * 16);
 #pragma unroll
             for (int q = 0; q < kE / 4; ++q) {
-                const float4 o = rrow[rswz(h, q)];
+                const float4 o = sR[rswz(h, q)];
                 if (half == 0) {
                     s[4 * q] = s[4 * q] + o.x; s[4 * q + 1] = s[4 * q + 1] + o.y;
                     s[4 * q + 2] = s[4 * q + 2] + o.z; s[4 * q + 3] = s[4 * q + 3] + o.w;
@@ -295,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
                     s[4 * q + 2] = o.z + s[4 * q + 2]; s[4 * q + 3] = o.w + s[4 * q + 3];
                 }
             }
-            mbar_arrive_remote(peer_addr(tc::smem_u32(&Rfree[buf]), peer));  // our buffer is free again
+            mbar_arrive_remote(peer_addr(tc::smem_u32(Rfree), peer));  // our receive buffer is free again
             const int64_t p0 = p_begin + (int64_t)j * kE;
             const unsigned vlo = __ballot_sync(0xffffffffu, entry_of(p0 + lane) >= 0);
             const unsigned vhi = __ballot_sync(0xffffffffu, entry_of(p0 + 32 + lane) >= 0);
@@ -339,8 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
             uint32_t packed[kE / 2];
 #pragma unroll
             for (int e = 0; e < kE; e += 2) {
-                const float p0f = (s[e] == -INFINITY) ? 0.f : exp2f(s[e] - m_run);
-                const float p1f = (s[e + 1] == -INFINITY) ? 0.f : exp2f(s[e + 1] - m_run);
+                const float p0f = (s[e] == -INFINITY) ? 0.f : ex2_approx(s[e] - m_run);
+                const float p1f = (s[e + 1] == -INFINITY) ? 0.f : ex2_approx(s[e + 1] - m_run);
                 psum += p0f + p1f;
                 __nv_bfloat162 pr = __floats2bfloat162_rn(p0f, p1f);
                 packed[e / 2] = *reinterpret_cast<uint32_t*>(&pr);

@@ -47,8 +47,10 @@ CSA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, long long budget)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity))
+    for (int polls = 0; !mbar_try_wait(bar, parity); ++polls) {
         if (clock64() - t0 > budget) return false;
+        if (polls >= 8) __nanosleep(32);  // long waits yield issue slots to working warps
+    }
     return true;
 }
 
