@@ -5,13 +5,17 @@
 namespace csa {
 
 constexpr int kBins = 4096;  // 12-bit radix digits
-constexpr int kCtrs = 8;     // per query: [0] emitted, [1] candidates, [2] ticket
+constexpr int kCtrs = 8;     // per query: [0] emitted, [1] candidates, [2] ticket, [3] arrivals
+
+// Slot of a 12-bit digit in a 4096-bin histogram.  Bins are stored transposed
+// ([16][256]) so that the threshold search, in which thread t reads the 16 consecutive
+// bins 16u .. 16u + 15 (u = 255 - t), touches 32 different banks per warp access.
+CSA_DEV uint32_t hist_slot(uint32_t bin) { return (bin & 15u) * 256u + (bin >> 4); }
 
 // Workspace of csa_indexer_topk, carved from one caller buffer.
 struct TopkWs {
     uint32_t* status; // sticky device status: nonzero after a bounded wait timed out
     uint32_t* hist0;  // [G][kBins] digit-0 histogram (zero between calls)
-    uint32_t* hist1;  // [G][kBins] digit-1 histogram of the candidates (zero between calls)
     uint32_t* ctr;    // [G][kCtrs] counters (zero between calls)
     float* scores;    // [G][ld] fp32 scores of the visible entries
     uint2* cand;      // [G][ld] (score key, index) candidates
@@ -24,9 +28,11 @@ struct TopkWs {
 TopkWs topk_ws_layout(void* base, int G, int64_t N_cap);
 
 bool indexer_tc_supported(int n_hI, int cI);
+// tcgen05 scan; *fused is set when the scan kernel also performed the top-k select
+// (idx_out / scores_out written), otherwise launch_topk_select must follow.
 int launch_scan_tc(const void* qI, const float* wI, const void* KI, const int64_t* t, int B,
                    int nq, int64_t N_cap, int n_hI, int cI, int m, int k, const TopkWs& ws,
-                   cudaStream_t stream);
+                   int32_t* idx_out, float* scores_out, bool* fused, cudaStream_t stream);
 int launch_scan_cuda_core(const void* qI, const float* wI, const void* KI, const int64_t* t,
                           int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
                           const TopkWs& ws, int dtype, cudaStream_t stream);

@@ -20,6 +20,7 @@
 // walks a strided set of key tiles of one query.  Every barrier wait is bounded; a
 // timeout sets the workspace status word and every role drains and exits.
 #include "indexer.cuh"
+#include "select.cuh"
 #include "tc_utils.cuh"
 
 namespace csa {
@@ -33,14 +34,45 @@ struct ScanCfg {
     static constexpr int kPanels = CI / 64;
     static constexpr int kAStage = kTileKeys * CI * 2;      // bytes of one key tile
     static constexpr int kBBytes = NH * CI * 2;             // q^I tile
-    static constexpr int kFixed = 1024 + kBBytes + NH * 4 + kBins * 4 + 256;
-    static constexpr int kStagesRaw = (220 * 1024 - kFixed) / kAStage;
+    static constexpr int kBudget = 220 * 1024;
+    static constexpr int kFixed0 = 1024 + kBBytes + NH * 4 + kBins * 4 + 256;
+    // scores of the CTA's first kCacheTiles tiles stay in shared memory for the in-place
+    // select, when that still leaves a 3-stage ring
+    static constexpr int kCacheTiles = (kBudget - kFixed0 - 3 * kAStage) >= 32 * kTileKeys * 4 ? 32 : 0;
+    static constexpr int kFixed = kFixed0 + kCacheTiles * kTileKeys * 4;
+    static constexpr int kStagesRaw = (kBudget - kFixed) / kAStage;
     static constexpr int kStages = kStagesRaw > 6 ? 6 : kStagesRaw;
     static constexpr int kSmem = kFixed + kStages * kAStage;
     static constexpr int kTmemCols = (2 * NH) < 32 ? 32 : (2 * NH);
     static_assert(kStages >= 2, "not enough shared memory for a 2-stage ring");
     static_assert((kTmemCols & (kTmemCols - 1)) == 0, "TMEM columns must be a power of 2");
+    static_assert(kStages * kAStage >= 2 * sel::kListCap * 8, "select lists reuse the ring");
 };
+
+CSA_DEV void red_release_add(uint32_t* p, uint32_t v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+CSA_DEV uint32_t atom_acq_rel_add(uint32_t* p, uint32_t v)
+{
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+// Bounded wait until *p >= target (acquire, GPU scope); false after `budget` cycles.
+CSA_DEV bool wait_count_geq(const uint32_t* p, uint32_t target, long long budget)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    if (v >= target) return true;
+    const long long t0 = clock64();
+    for (;;) {
+        __nanosleep(64);
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+        if (v >= target) return true;
+        if (clock64() - t0 > budget) return false;
+    }
+}
 
 CSA_DEV int64_t visible_of(const int64_t* t, int g, int m, int64_t N_cap)
 {
@@ -50,11 +82,18 @@ CSA_DEV int64_t visible_of(const int64_t* t, int g, int m, int64_t N_cap)
     return v < N_cap ? v : N_cap;
 }
 
+// Outputs of the in-place top-k select (fused = 0: scores only, for topk_select).
+struct SelOut {
+    int32_t* idx_out;
+    float* scores_out;
+    int fused;
+};
+
 template <int NH, int CI>
 __global__ void __launch_bounds__(kTcThreads, 1)
 scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __restrict__ qI,
                const float* __restrict__ wI, const int64_t* __restrict__ t, int nq, int64_t N_cap,
-               int m, int k, TopkWs ws)
+               int m, int k, TopkWs ws, SelOut so)
 {
     using Cfg = ScanCfg<NH, CI>;
     constexpr int S = Cfg::kStages;
@@ -62,7 +101,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + S * Cfg::kAStage;
-    float* sw = reinterpret_cast<float*>(sB + Cfg::kBBytes);
+    float* s_sc = reinterpret_cast<float*>(sB + Cfg::kBBytes);  // [kCacheTiles * 128] own scores
+    float* sw = s_sc + Cfg::kCacheTiles * kTileKeys;
     uint32_t* sh = reinterpret_cast<uint32_t*>(sw + NH);
     uint64_t* full = reinterpret_cast<uint64_t*>(sh + kBins);
     uint64_t* empty = full + S;
@@ -230,12 +270,23 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
 #pragma unroll
             for (int h = 0; h < NH; ++h) sc = fmaf(sw[h], fmaxf(v[h], 0.f), sc);
             const int64_t sidx = (int64_t)tile * kTileKeys + row;
-            if (sidx < vis) scores[sidx] = sc;
+            if (sidx < vis) {
+                if (!so.fused) {
+                    scores[sidx] = sc;
+                } else if (vis <= k) {  // everything visible is selected, in index order
+                    so.idx_out[(int64_t)g * k + sidx] = (int32_t)sidx;
+                    if (so.scores_out) so.scores_out[(int64_t)g * k + sidx] = sc;
+                } else if (it < Cfg::kCacheTiles) {
+                    s_sc[it * kTileKeys + row] = sc;
+                } else {
+                    scores[sidx] = sc;
+                }
+            }
             if (need_hist) {
                 // lanes with the same digit add once (scores cluster in few bins)
                 const uint32_t bin = sidx < vis ? order_key(sc) >> 20 : 0xffffffffu;
                 const unsigned peers = __match_any_sync(0xffffffffu, bin);
-                if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&sh[bin], (uint32_t)__popc(peers));
+                if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&sh[hist_slot(bin)], (uint32_t)__popc(peers));
             }
         }
     }
@@ -250,23 +301,104 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem_base, Cfg::kTmemCols);
     }
+    if (!so.fused) return;
+    __syncthreads();  // the arrival below releases every thread's histogram atomics
+    if (warp < 2) return;
+
+    // ---------------------------------------------------------------- in-place top-k
+    // The epilogue warps (256 threads, named barrier 1) select from this CTA's scores.
+    // Every CTA of the query is resident (the launch keeps the grid within one wave), so
+    // they can meet at a counter once all digit-0 histograms are merged; the wait is
+    // bounded.  Then each CTA classifies its own keys against the threshold bin, and the
+    // last one (atomic ticket) resolves the candidates and resets the workspace.
+    using Bar = sel::NamedBar<1>;
+    __shared__ sel::Shared ss;
+    const int tid = threadIdx.x - 64;
+    const sel::Query q = sel::query_view(ws, g, k, so.idx_out, so.scores_out);
+    if (vis <= k) {  // padding after the visible entries (written by the epilogue above)
+        for (int64_t p = vis + (int64_t)blockIdx.x * sel::kSelThreads + tid; p < k;
+             p += (int64_t)gridDim.x * sel::kSelThreads) {
+            q.idx_out[p] = -1;
+            if (q.sc_out) q.sc_out[p] = -INFINITY;
+        }
+        return;
+    }
+    if (tid == 0) {
+        red_release_add(&q.ctr[3], 1u);
+        const bool ok = wait_count_geq(&q.ctr[3], gridDim.x, tc::kWaitBudget);
+        if (!ok) atomicExch(ws.status, 1u);
+        ss.ok = ok;
+    }
+    Bar::sync();
+    const bool ok = ss.ok != 0;
+    uint2* s_listA = reinterpret_cast<uint2*>(sA);  // the ring is idle now
+    uint2* s_listB = s_listA + sel::kListCap;
+    if (ok) {
+        sel::load_hist(sh, q.hist0, tid);
+        Bar::sync();
+        sel::find_threshold_bin<kBins, Bar>(sh, (uint32_t)k, &ss, tid);
+        const uint32_t b0 = ss.bin;
+        const float* scores = ws.scores + (int64_t)g * ws.ld;
+        const int my_tiles = active ? (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+        const int npos = my_tiles * kTileKeys;  // CTA-local positions: tile ordinal * 128 + row
+        for (int base = 0; base < npos; base += sel::kRound) {
+            uint32_t key[sel::kPer], eidx[sel::kPer];
+            bool valid[sel::kPer];
+#pragma unroll
+            for (int u = 0; u < sel::kPer; ++u) {
+                const int j = base + tid + u * sel::kSelThreads;
+                const int ord = j / kTileKeys;
+                const int64_t s = ((int64_t)blockIdx.x + (int64_t)ord * gridDim.x) * kTileKeys + (j % kTileKeys);
+                valid[u] = j < npos && s < vis;
+                eidx[u] = (uint32_t)s;
+                key[u] = valid[u] ? order_key(ord < Cfg::kCacheTiles ? s_sc[j] : __ldcg(&scores[s])) : 0u;
+            }
+            sel::classify_round<Bar>(q, key, eidx, valid, b0, s_listA, s_listB, &ss, tid);
+        }
+    }
+    Bar::sync();  // the ticket releases this CTA's candidate writes (and acquires the others')
+    if (tid == 0) ss.last = atom_acq_rel_add(&q.ctr[2], 1u) == gridDim.x - 1;
+    Bar::sync();
+    if (!ss.last) return;
+    if (ok) sel::resolve_candidates<Bar>(q, sh, s_listA, s_listB, &ss, tid);
+    Bar::sync();
+    sel::reset_query(q, tid);
 }
 
 template <int NH, int CI>
 int launch_nh_ci(const CUtensorMap& tmap, const void* qI, const float* wI, const int64_t* t, int B, int nq,
-                 int64_t N_cap, int m, int k, const TopkWs& ws, cudaStream_t stream)
+                 int64_t N_cap, int m, int k, const TopkWs& ws, int32_t* idx_out, float* scores_out,
+                 bool* fused, cudaStream_t stream)
 {
     using Cfg = ScanCfg<NH, CI>;
-    const int G = B * nq;
-    int64_t ctas = (kNumSMs + G - 1) / G;
-    const int64_t tiles = (N_cap + kTileKeys - 1) / kTileKeys;
-    if (ctas > tiles) ctas = tiles;
-    if (ctas < 1) ctas = 1;
     auto kern = scan_tc_kernel<NH, CI>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+    const int G = B * nq;
+    const int64_t tiles = (N_cap + kTileKeys - 1) / kTileKeys;
+    // The in-place select makes the CTAs of a query wait for one another, so it is used
+    // only when the whole grid fits in one wave of resident CTAs.
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kTcThreads, Cfg::kSmem);
+    const int64_t resident = (int64_t)sms * per_sm;
+    int64_t ctas;
+    if (resident >= G) {
+        ctas = resident / G;
+        *fused = true;
+    } else {
+        ctas = (kNumSMs + G - 1) / G;
+        *fused = false;
+    }
+    if (ctas > tiles) ctas = tiles;
+    if (ctas < 1) ctas = 1;
+    SelOut so;
+    so.idx_out = idx_out;
+    so.scores_out = scores_out;
+    so.fused = *fused ? 1 : 0;
     dim3 grid((unsigned)ctas, (unsigned)G);
     launch_pdl(kern, grid, dim3(kTcThreads), Cfg::kSmem, stream, tmap, static_cast<const __nv_bfloat16*>(qI), wI,
-               t, nq, N_cap, m, k, ws);
+               t, nq, N_cap, m, k, ws, so);
     return launch_status();
 }
 
@@ -278,15 +410,17 @@ bool indexer_tc_supported(int n_hI, int cI)
 }
 
 int launch_scan_tc(const void* qI, const float* wI, const void* KI, const int64_t* t, int B, int nq,
-                   int64_t N_cap, int n_hI, int cI, int m, int k, const TopkWs& ws, cudaStream_t stream)
+                   int64_t N_cap, int n_hI, int cI, int m, int k, const TopkWs& ws, int32_t* idx_out,
+                   float* scores_out, bool* fused, cudaStream_t stream)
 {
+    *fused = false;
     if (N_cap == 0) return CSA_OK;
     if ((int64_t)B * N_cap + kTileKeys >= (int64_t(1) << 31) || !aligned16(qI) || !aligned16(KI))
         return launch_scan_cuda_core(qI, wI, KI, t, B, nq, N_cap, n_hI, cI, m, k, ws, CSA_BF16, stream);
     CUtensorMap tmap;
     if (!make_tmap_bf16_2d(&tmap, KI, (uint64_t)B * N_cap, cI, cI, 64, kTileKeys)) return CSA_ERR_CUDA;
 #define CSA_SCAN_CASE(NH_, CI_) \
-    if (n_hI == NH_ && cI == CI_) return launch_nh_ci<NH_, CI_>(tmap, qI, wI, t, B, nq, N_cap, m, k, ws, stream);
+    if (n_hI == NH_ && cI == CI_) return launch_nh_ci<NH_, CI_>(tmap, qI, wI, t, B, nq, N_cap, m, k, ws, idx_out, scores_out, fused, stream);
     CSA_SCAN_CASE(16, 64) CSA_SCAN_CASE(16, 128) CSA_SCAN_CASE(16, 256)
     CSA_SCAN_CASE(32, 64) CSA_SCAN_CASE(32, 128) CSA_SCAN_CASE(32, 256)
     CSA_SCAN_CASE(64, 64) CSA_SCAN_CASE(64, 128) CSA_SCAN_CASE(64, 256)

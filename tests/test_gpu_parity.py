@@ -225,6 +225,40 @@ def test_indexer_topk_random(dtype, n_hI, cI, N_cap, k):
         assert np.all(np.abs(sc[0, q][:len(got)] - s[got]) <= band)
 
 
+@pytest.mark.parametrize("B,nq,N_cap,k,seed", [(2, 8, 40000, 512, 230), (3, 50, 1000, 100, 240)])
+def test_indexer_topk_many_queries(B, nq, N_cap, k, seed):
+    """16 queries: each query's scan CTAs own more key tiles than they keep on chip, so
+    the in-place select also reads scores back from the workspace.  150 queries: more
+    queries than resident CTAs, so the scan is followed by the stand-alone select."""
+    dtype, n_hI, cI, m = torch.bfloat16, 64, 128, 4
+    qI = randn((B, nq, n_hI, cI), seed, dtype)
+    KI = randn((B, N_cap, cI), seed + 1, dtype)
+    wI = randn((B, nq, n_hI), seed + 2, torch.float32)
+    rng = np.random.default_rng(seed + 3)
+    t = [int(x) for x in rng.integers(0, 4 * N_cap + 8, size=B * nq)]
+    t[0], t[1] = 4 * N_cap, 4 * (k // 2) + 3          # everything visible; fewer than k
+    idx, sc, ws = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k)
+    for b in range(B):
+        K64 = to_f64(KI[b])
+        for q in range(nq):
+            g = b * nq + q
+            vis = oracle.visible(t[g], m, N_cap)
+            q64, w64 = to_f64(qI[b, q]), to_f64(wI[b, q])
+            s = oracle.index_scores(q64, w64, K64, vis)
+            got = idx[b, q]
+            if vis <= k:
+                assert got.tolist() == list(range(vis)) + [-1] * (k - vis)
+            else:
+                check_topk_sets(got, s, k, lambda d: score_error_bound(q64, w64, K64, d))
+            sel = got[got >= 0]
+            band = score_error_bound(q64, w64, K64, sel) + 1e-6 * np.abs(s[sel])
+            assert np.all(np.abs(sc[b, q][:len(sel)] - s[sel]) <= band)
+            assert np.all(np.isneginf(sc[b, q][len(sel):]))
+    # the workspace is left clean for the next call
+    idx2, _, _ = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k, ws=ws)
+    assert np.array_equal(np.sort(idx2, axis=-1), np.sort(idx, axis=-1))
+
+
 def test_indexer_degenerate_cases():
     dtype, n_hI, cI, N_cap, m = torch.bfloat16, 64, 128, 700, 4
     qI = randn((1, 3, n_hI, cI), 220, dtype)
