@@ -341,17 +341,24 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
         const float* scores = ws.scores + (int64_t)g * ws.ld;
         const int my_tiles = active ? (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
         const int npos = my_tiles * kTileKeys;  // CTA-local positions: tile ordinal * 128 + row
+        const uint32_t vis32 = (uint32_t)vis;   // < 2^31 (checked by the host)
+        // position j = tile ordinal * 128 + row holds key (blockIdx.x + ordinal * gridDim.x) * 128 + row;
+        // kSelThreads = 2 tiles, so from one u to the next the key advances by 2 * gridDim.x tiles
+        static_assert(sel::kSelThreads == 2 * kTileKeys, "two tiles per classification step");
+        const uint32_t key_step = 2u * gridDim.x * kTileKeys;
         for (int base = 0; base < npos; base += sel::kRound) {
+            const int j0 = base + tid;
+            const int ord0 = j0 / kTileKeys;
+            const uint32_t s0 = (blockIdx.x + (uint32_t)ord0 * gridDim.x) * kTileKeys + (uint32_t)(j0 % kTileKeys);
             uint32_t key[sel::kPer], eidx[sel::kPer];
             bool valid[sel::kPer];
 #pragma unroll
             for (int u = 0; u < sel::kPer; ++u) {
-                const int j = base + tid + u * sel::kSelThreads;
-                const int ord = j / kTileKeys;
-                const int64_t s = ((int64_t)blockIdx.x + (int64_t)ord * gridDim.x) * kTileKeys + (j % kTileKeys);
-                valid[u] = j < npos && s < vis;
-                eidx[u] = (uint32_t)s;
-                key[u] = valid[u] ? order_key(ord < Cfg::kCacheTiles ? s_sc[j] : __ldcg(&scores[s])) : 0u;
+                const int j = j0 + u * sel::kSelThreads;
+                const uint32_t s = s0 + (uint32_t)u * key_step;
+                valid[u] = j < npos && s < vis32;
+                eidx[u] = s;
+                key[u] = valid[u] ? order_key(ord0 + 2 * u < Cfg::kCacheTiles ? s_sc[j] : __ldcg(&scores[s])) : 0u;
             }
             sel::classify_round<Bar>(q, key, eidx, valid, b0, s_listA, s_listB, &ss, tid);
         }

@@ -131,31 +131,33 @@ CSA_DEV uint32_t warp_append(uint32_t* ctr, bool pred)
     return base + __popc(mask & ((1u << lane) - 1u));
 }
 
-// Radix digit of a key at a level: level 0 = key bits 31..20, level 1 = bits 19..8
-// (12-bit digits); levels 2..6 = key bits 7..0, then ~index bits 31..24, .., 7..0.
-CSA_DEV uint32_t digit_of(uint2 kv, int level)
+// Radix digits of the 64-bit key (kv.x << 32) | ~kv.y: level 0 = bits 63..52, level 1 =
+// bits 51..40 (12-bit digits), levels 2..6 = 8-bit digits from bit 39 down to bit 0.
+CSA_DEV uint32_t digit_shift(int level) { return level == 0 ? 52u : level == 1 ? 40u : (uint32_t)(48 - 8 * level); }
+CSA_DEV uint32_t digit_mask(int level) { return level < 2 ? 0xfffu : 0xffu; }
+CSA_DEV uint32_t digit_at(uint2 kv, uint32_t shift, uint32_t mask)
 {
-    switch (level) {
-        case 0: return kv.x >> 20;
-        case 1: return (kv.x >> 8) & 0xfffu;
-        case 2: return kv.x & 0xffu;
-        case 3: return (~kv.y >> 24) & 0xffu;
-        case 4: return (~kv.y >> 16) & 0xffu;
-        case 5: return (~kv.y >> 8) & 0xffu;
-        default: return ~kv.y & 0xffu;
-    }
+    const uint64_t key = ((uint64_t)kv.x << 32) | (uint32_t)~kv.y;
+    return (uint32_t)(key >> shift) & mask;
 }
+CSA_DEV uint32_t digit_of(uint2 kv, int level) { return digit_at(kv, digit_shift(level), digit_mask(level)); }
 
 // Global -> shared copy of a 4096-bin histogram with every load issued before the
 // first store (one round trip instead of one per iteration).
 CSA_DEV void load_hist(uint32_t* sh, const uint32_t* gh, int tid)
 {
-    constexpr int kPerThread = kBins / kSelThreads;
-    uint32_t v[kPerThread];
+    constexpr int kQuads = kBins / 4 / kSelThreads;
+    uint4 v[kQuads];
 #pragma unroll
-    for (int u = 0; u < kPerThread; ++u) v[u] = __ldcg(&gh[tid + u * kSelThreads]);
+    for (int u = 0; u < kQuads; ++u) v[u] = __ldcg(reinterpret_cast<const uint4*>(gh) + tid + u * kSelThreads);
 #pragma unroll
-    for (int u = 0; u < kPerThread; ++u) sh[tid + u * kSelThreads] = v[u];
+    for (int u = 0; u < kQuads; ++u) reinterpret_cast<uint4*>(sh)[tid + u * kSelThreads] = v[u];
+}
+
+// Zero n words of 16-byte-aligned memory (n a multiple of 4 * kSelThreads).
+CSA_DEV void zero_words(uint32_t* p, int n, int tid)
+{
+    for (int i = tid; i < n / 4; i += kSelThreads) reinterpret_cast<uint4*>(p)[i] = make_uint4(0, 0, 0, 0);
 }
 
 // Exclusive prefix sum of v over the group in thread order; total = group sum (every
@@ -340,7 +342,7 @@ CSA_DEV void resolve_candidates(const Query& q, uint32_t* sh, uint2* s_listA, ui
         const uint32_t i = tid + u * kSelThreads;
         v[u] = i < nload ? __ldcg(&q.cand[i]) : make_uint2(0, 0);
     }
-    for (int i = tid; i < kBins; i += kSelThreads) sh[i] = 0;
+    zero_words(sh, kBins, tid);
     if (tid == 0) s->out = out;
     Bar::sync();
     if (count > (uint32_t)kListCap) {
@@ -356,6 +358,7 @@ CSA_DEV void resolve_candidates(const Query& q, uint32_t* sh, uint2* s_listA, ui
             emit_by_rank(q, s_listA, count, need, s, tid);
             break;
         }
+        const uint32_t dsh = digit_shift(level), dmask = digit_mask(level);
         uint32_t bt = 0xffffffffu;  // need >= count: every entry is taken
         if (need < count) {
             const int nb = level == 1 ? kBins : 256;
@@ -365,7 +368,7 @@ CSA_DEV void resolve_candidates(const Query& q, uint32_t* sh, uint2* s_listA, ui
             }
 #pragma unroll
             for (int u = 0; u < kPerT; ++u) {
-                const uint32_t d = digit_of(v[u], level);
+                const uint32_t d = digit_at(v[u], dsh, dmask);
                 if (tid + u * kSelThreads < (int)count) atomicAdd(&sh[level == 1 ? hist_slot(d) : d], 1u);
             }
             Bar::sync();
@@ -379,7 +382,7 @@ CSA_DEV void resolve_candidates(const Query& q, uint32_t* sh, uint2* s_listA, ui
 #pragma unroll
         for (int u = 0; u < kPerT; ++u) {
             if (tid + u * kSelThreads >= (int)count) continue;
-            const uint32_t d = bt == 0xffffffffu ? 0x1000u : digit_of(v[u], level);
+            const uint32_t d = bt == 0xffffffffu ? 0x1000u : digit_at(v[u], dsh, dmask);
             cnt += d > bt || bt == 0xffffffffu ? 1u : (d == bt ? 0x10000u : 0u);
         }
         uint32_t tot;
@@ -388,7 +391,7 @@ CSA_DEV void resolve_candidates(const Query& q, uint32_t* sh, uint2* s_listA, ui
 #pragma unroll
         for (int u = 0; u < kPerT; ++u) {
             if (tid + u * kSelThreads >= (int)count) continue;
-            const uint32_t d = bt == 0xffffffffu ? 0x1000u : digit_of(v[u], level);
+            const uint32_t d = bt == 0xffffffffu ? 0x1000u : digit_at(v[u], dsh, dmask);
             if (d > bt || bt == 0xffffffffu)
                 emit(q, tp++, v[u]);
             else if (d == bt)
@@ -412,7 +415,7 @@ CSA_DEV void resolve_candidates(const Query& q, uint32_t* sh, uint2* s_listA, ui
 // Zero this query's histogram and counters for the next call.
 CSA_DEV void reset_query(const Query& q, int tid)
 {
-    for (int i = tid; i < kBins; i += kSelThreads) q.hist0[i] = 0;
+    zero_words(q.hist0, kBins, tid);
     if (tid < kCtrs) q.ctr[tid] = 0;
 }
 
