@@ -128,11 +128,33 @@ CSA_DEV float ex2_approx(float x)
     return y;
 }
 
+constexpr int kBoxBytes = 128 * 128;  // one 128-row x 32-column fp32 output box
+
+// Copy columns [col0, col0 + 128) of row h of the output half from TMEM (o_taddr: this
+// warp's lane quarter, first O column) into the staging boxes: eight 128-row x 32-column
+// fp32 boxes of 16 KB in the 128-byte swizzled layout of the output tensor map.
+CSA_DEV void stage_o_cols(uint8_t* stage, uint32_t o_taddr, int h, int col0)
+{
+#pragma unroll 1
+    for (int c0 = col0; c0 < col0 + 128; c0 += 16) {
+        float o[16];
+        tc::tmem_ld16(o_taddr + c0, o);
+        tc::tmem_wait_ld();
+        uint8_t* row = stage + (c0 >> 5) * kBoxBytes + h * 128;
+        const int q0 = (c0 & 31) >> 2;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4*>(row + (((q0 + i) ^ (h & 7)) << 4)) =
+                make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+    }
+}
+
 // float4 q (0..15) of row h of a 64-float row, XOR-swizzled so that the 32 rows of a
 // warp spread over the banks
 CSA_DEV int rswz(int h, int q) { return h * 16 + (q ^ (h & 15)); }
 
-__global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint32_t* status)
+__global__ void __launch_bounds__(kThreads, 1)
+attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_t* status)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -153,8 +175,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
     uint64_t* Pfull = bars + 12;    // softmax -> MMA                (count 128)
     uint64_t* PVdone = bars + 13;   // MMA commit -> softmax
     uint64_t* idsready = bars + 14; // loaders -> softmax            (count 128)
-    uint64_t* staged = bars + 15;   // softmax warps: output staged  (count 128)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+    uint64_t* staged = bars + 15;   // output half staged            (count 256: loaders + softmax)
+    uint64_t* Ofinal = bars + 16;   // softmax -> loaders: last P C done (count 128)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
     volatile uint32_t* abort_flag = tmem_slot + 1;
     int* s_ids = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);  // [kMaxIds]
 
@@ -179,7 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
         tc::mbar_init(Pfull, kHeads);
         tc::mbar_init(PVdone, 1);
         tc::mbar_init(idsready, kLoaders);
-        tc::mbar_init(staged, kHeads);
+        tc::mbar_init(staged, 2 * kHeads);
+        tc::mbar_init(Ofinal, kHeads);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -270,6 +294,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
             tc::mbar_arrive(&Cfull[buf]);
         }
         cp_async_wait_all();
+        // The output half leaves through TMA: these warps stage columns 0..127 and the
+        // softmax warps 128..255 once the last P C has completed, then thread 0 stores the
+        // eight 128 x 32 boxes.
+        if (!*abort_flag && tc::mbar_wait(Ofinal, 0, tc::kWaitBudget)) {
+            tc::fence_after_sync();
+            stage_o_cols(smem, tmem + ((uint32_t)(warp * 32) << 16) + kHalf, warp * 32 + lane, 0);
+        } else {
+            *abort_flag = 1;
+        }
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(staged);
+        if (threadIdx.x == 0) {
+            if (tc::mbar_wait(staged, 0, tc::kWaitBudget) && !*abort_flag) {
+                for (int p = 0; p < kHalf / 32; ++p)
+                    tc::tma_store_2d(&tmap_o, smem + p * kBoxBytes, half * kHalf + p * 32, (int)prow);
+                tc::bulk_store_commit_wait();
+            } else {
+                *abort_flag = 1;
+            }
+        }
     } else if (warp < 8) {
         // ------------------------------------------------------------ softmax
         const int quarter = warp & 3;
@@ -336,13 +380,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
             const int64_t p0 = p_begin + (int64_t)j * kE;
             const unsigned vlo = __ballot_sync(0xffffffffu, entry_of(p0 + lane) >= 0);
             const unsigned vhi = __ballot_sync(0xffffffffu, entry_of(p0 + 32 + lane) >= 0);
-            float cmax = -INFINITY;
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // 4 chains, not 1
 #pragma unroll
             for (int e = 0; e < kE; ++e) {
                 const bool valid = (((e < 32) ? (vlo >> e) : (vhi >> (e - 32))) & 1u) != 0;
                 s[e] = valid ? s[e] * a.scale_log2 : -INFINITY;
-                cmax = fmaxf(cmax, s[e]);
+                mx[e & 3] = fmaxf(mx[e & 3], s[e]);
             }
+            const float cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             if (j > 0) {
                 // P buffer and O are free once the previous chunk's P C has finished
                 if (!tc::mbar_wait(PVdone, (j - 1) & 1, tc::kWaitBudget)) {
@@ -372,17 +417,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
             } else {
                 m_run = cmax;
             }
-            float psum = 0.f;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
             uint32_t packed[kE / 2];
 #pragma unroll
             for (int e = 0; e < kE; e += 2) {
                 const float p0f = (s[e] == -INFINITY) ? 0.f : ex2_approx(s[e] - m_run);
                 const float p1f = (s[e + 1] == -INFINITY) ? 0.f : ex2_approx(s[e + 1] - m_run);
-                psum += p0f + p1f;
+                ps[(e >> 1) & 3] += p0f + p1f;
                 __nv_bfloat162 pr = __floats2bfloat162_rn(p0f, p1f);
                 packed[e / 2] = *reinterpret_cast<uint32_t*>(&pr);
             }
-            l_run += psum;
+            l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
 #pragma unroll
             for (int qc = 0; qc < kE / 8; ++qc) {
                 uint4 v = make_uint4(packed[4 * qc], packed[4 * qc + 1], packed[4 * qc + 2], packed[4 * qc + 3]);
@@ -393,42 +438,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pair_kernel(AttnArgs a, uint
             tc::mbar_arrive(Pfull);
         }
         if (ok && !*abort_flag && tc::mbar_wait(PVdone, (nchunks - 1) & 1, tc::kWaitBudget)) {
-            tc::fence_after_sync();
             // The last P C has completed, so every MMA reading q and the chunks has too:
-            // those 128 KB stage the 128 x 256 fp32 output half.  Rows are written with
-            // 16-byte units XOR-swizzled by (row & 7) and copied out row by row with
-            // coalesced 16-byte stores.
-            float4* stage = reinterpret_cast<float4*>(sQ);  // [128 rows][64 float4]
-            const uint32_t ob = tmem + lane_base + kHalf;
-#pragma unroll 1
-            for (int c0 = 0; c0 < kHalf; c0 += 16) {
-                float o[16];
-                tc::tmem_ld16(ob + c0, o);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 16; i += 4) {
-                    const int q4 = (c0 + i) >> 2;
-                    stage[h * 64 + (q4 ^ (h & 7))] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
-                }
-            }
+            // those 128 KB now stage the 128 x 256 fp32 output half (columns 128..255 here).
+            tc::mbar_arrive(Ofinal);
+            tc::fence_after_sync();
+            stage_o_cols(smem, tmem + lane_base + kHalf, h, 128);
             if (half == 0) a.part_ml[prow + h] = make_float2(m_run, l_run);
-            tc::mbar_arrive(staged);
-            if (tc::mbar_wait(staged, 0, tc::kWaitBudget)) {
-                const int st = threadIdx.x - 128;  // 0..127
-                float* po = a.part_o + prow * a.c + half * kHalf;
-#pragma unroll 4
-                for (int i = st; i < kHeads * 64; i += 128) {
-                    const int r = i >> 6, q4 = i & 63;
-                    *reinterpret_cast<float4*>(po + (size_t)r * a.c + q4 * 4) = stage[r * 64 + (q4 ^ (r & 7))];
-                }
-            } else {
-                *abort_flag = 1;
-            }
         } else {
-            tc::mbar_arrive(staged);
+            tc::mbar_arrive(Ofinal);
             *abort_flag = 1;
             if (half == 0) a.part_ml[prow + h] = make_float2(-INFINITY, 0.f);
         }
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(staged);
     } else {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -534,7 +556,10 @@ int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cu
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    cudaLaunchKernelEx(&cfg, attn_pair_kernel, a, status);
+    CUtensorMap tmap_o;  // partial outputs [G * splits * 128 rows][512] fp32, 32 x 128 boxes
+    const uint64_t rows = (uint64_t)a.B * a.nq * plan.splits * kHeads;
+    if (!make_tmap_f32_2d(&tmap_o, a.part_o, rows, kC, kC, 32, kHeads)) return CSA_ERR_CUDA;
+    cudaLaunchKernelEx(&cfg, attn_pair_kernel, tmap_o, a, status);
     return launch_status();
 }
 

@@ -69,6 +69,20 @@ CSA_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+// 2-D tiled bulk tensor store from this CTA's shared memory (completion tracked by the
+// issuing thread's bulk groups).  x (innermost) must be a multiple of 16 bytes / element size.
+CSA_DEV void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+// Close this thread's bulk group and wait until all its bulk stores have completed.
+CSA_DEV void bulk_store_commit_wait()
+{
+    asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
+}
 CSA_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------- tcgen05
@@ -176,5 +190,8 @@ constexpr long long kWaitBudget = 2000000000LL;  // ~1 s at 1.9 GHz
 // box of box_cols x box_rows and 128-byte swizzle; false if the driver call fails.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                        uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);
+// Same for a 2-D fp32 tensor.
+bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                      uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);
 
 }  // namespace csa
