@@ -155,7 +155,7 @@ attn_cuda_core(AttnArgs a)
         const int h = h_base + warp * HPW + x;
         if (h >= a.n_h) continue;
         const size_t row = ((size_t)g * a.splits + split) * a.n_h + h;
-        float* po = a.part_o + row * c;
+        float* po = static_cast<float*>(a.part_o) + row * c;
 #pragma unroll
         for (int i = 0; i < CPL; ++i) {
             const int j = lane + 32 * i;
@@ -166,7 +166,8 @@ attn_cuda_core(AttnArgs a)
 }
 
 // ----------------------------------------------------------------------------------
-// combine: out[g][h] = sum_i 2^(m_i - M) O_i / sum_i 2^(m_i - M) l_i ; lse in natural log
+// combine: out[g][h] = sum_i 2^(m_i - M) O_i / sum_i 2^(m_i - M) l_i ; lse in natural log.
+// Partials are fp32 O_i, or bf16 O_i / l_i, whose weight is then 2^(m_i - M) l_i.
 // ----------------------------------------------------------------------------------
 template <typename TO>
 CSA_DEV void store_out(TO* p, float v);
@@ -175,23 +176,44 @@ CSA_DEV void store_out<float>(float* p, float v) { *p = v; }
 template <>
 CSA_DEV void store_out<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
+// 16 bytes of consecutive partial values, streamed (read once); zeros when !valid
+CSA_DEV void load_vec_stream(const float* p, bool valid, float (&v)[4])
+{
+    const float4 x = valid ? __ldcs(reinterpret_cast<const float4*>(p)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+CSA_DEV void load_vec_stream(const __nv_bfloat16* p, bool valid, float (&v)[8])
+{
+    const uint4 x = valid ? __ldcs(reinterpret_cast<const uint4*>(p)) : make_uint4(0, 0, 0, 0);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);             // low bf16 of the pair
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);  // high bf16
+    }
+}
+CSA_DEV float load1(const float* p) { return *p; }
+CSA_DEV float load1(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
 // One CTA per (head, query).  Every split's (max, sum) is read in one round, the
 // weights 2^(m_i - M) are formed in shared memory, and the partial rows are read by
 // (column quad, split group) threads that issue all their loads before using them, so
 // the kernel costs two dependent global round trips rather than one per split.
-template <typename TO>
+template <typename TO, typename TP>
 __global__ void __launch_bounds__(kCombineThreads)
-attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_ml, int splits,
+attn_combine(const TP* __restrict__ part_o, const float2* __restrict__ part_ml, int splits,
              int n_h, int c, TO* __restrict__ out, float* __restrict__ lse)
 {
+    constexpr bool kNormalized = sizeof(TP) == 2;  // bf16 partials are O_i / l_i
     pdl_launch_dependents();
     pdl_wait();
-    constexpr int kBatch = 16;  // loads issued per thread before the first use
     const int h = blockIdx.x, g = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     __shared__ float s_m[kMaxSplits], s_w[kMaxSplits];
     __shared__ float s_red[kCombineThreads / 32];
-    __shared__ float4 s_acc[kCombineThreads];
+    constexpr int kV = 16 / sizeof(TP);  // partial values per 16-byte load
+    __shared__ float s_acc[kV * kCombineThreads];
+    constexpr int kBatch = 64 / kV;  // 16-byte loads issued per thread before the first use
     __shared__ float s_M, s_inv;
     const size_t base = (size_t)g * splits * n_h + h;
 
@@ -218,7 +240,7 @@ attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_m
     for (int i = tid; i < splits; i += kCombineThreads) {
         const float w = s_m[i] == -INFINITY ? 0.f : exp2f(s_m[i] - M);
         lloc = fmaf(w, s_w[i], lloc);
-        s_w[i] = w;
+        s_w[i] = kNormalized ? w * s_w[i] : w;
     }
 #pragma unroll
     for (int off = 16; off; off >>= 1) lloc += __shfl_xor_sync(0xffffffffu, lloc, off);
@@ -234,46 +256,44 @@ attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_m
     __syncthreads();
     const float inv = s_inv;
     TO* orow = out + ((size_t)g * n_h + h) * c;
-    if ((c & 3) == 0) {
-        const int ncq = c / 4;
-        const int per = ncq < kCombineThreads ? ncq : kCombineThreads;  // column quads per pass
+    if (c % kV == 0) {
+        // (column group of kV, split group) threads; kV = 16 bytes of partial per load
+        const int ncv = c / kV;
+        const int per = ncv < kCombineThreads ? ncv : kCombineThreads;  // column groups per pass
         const int ngrp = kCombineThreads / per;                         // split groups
-        for (int cq0 = 0; cq0 < ncq; cq0 += per) {
-            const int cq = cq0 + tid % per;
+        for (int cv0 = 0; cv0 < ncv; cv0 += per) {
+            const int cv = cv0 + tid % per;
             const int grp = tid / per;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (grp < ngrp && cq < ncq) {
-                const float* col = part_o + base * c + (size_t)cq * 4;
+            float acc[kV];
+#pragma unroll
+            for (int e = 0; e < kV; ++e) acc[e] = 0.f;
+            if (grp < ngrp && cv < ncv) {
+                const TP* col = part_o + base * c + (size_t)cv * kV;
                 for (int i0 = grp; i0 < splits; i0 += kBatch * ngrp) {
-                    float4 v[kBatch];
+                    float v[kBatch][kV];
 #pragma unroll
                     for (int u = 0; u < kBatch; ++u) {
                         const int i = i0 + u * ngrp;
-                        v[u] = (i < splits && s_w[i] != 0.f)
-                                   ? __ldcs(reinterpret_cast<const float4*>(col + (size_t)i * n_h * c))
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                        load_vec_stream(col + (size_t)i * n_h * c, i < splits && s_w[i] != 0.f, v[u]);
                     }
 #pragma unroll
                     for (int u = 0; u < kBatch; ++u) {
                         const int i = i0 + u * ngrp;
                         const float w = i < splits ? s_w[i] : 0.f;
-                        acc.x = fmaf(w, v[u].x, acc.x); acc.y = fmaf(w, v[u].y, acc.y);
-                        acc.z = fmaf(w, v[u].z, acc.z); acc.w = fmaf(w, v[u].w, acc.w);
+#pragma unroll
+                        for (int e = 0; e < kV; ++e) acc[e] = fmaf(w, v[u][e], acc[e]);
                     }
                 }
             }
-            s_acc[tid] = acc;
+#pragma unroll
+            for (int e = 0; e < kV; ++e) s_acc[e * kCombineThreads + tid] = acc[e];
             __syncthreads();
-            if (grp == 0 && cq < ncq) {
-                for (int q = 1; q < ngrp; ++q) {
-                    const float4 o = s_acc[q * per + tid];
-                    acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
-                }
-                const int j = cq * 4;
-                store_out<TO>(orow + j, acc.x * inv);
-                store_out<TO>(orow + j + 1, acc.y * inv);
-                store_out<TO>(orow + j + 2, acc.z * inv);
-                store_out<TO>(orow + j + 3, acc.w * inv);
+            if (grp == 0 && cv < ncv) {
+                for (int q = 1; q < ngrp; ++q)
+#pragma unroll
+                    for (int e = 0; e < kV; ++e) acc[e] += s_acc[e * kCombineThreads + q * per + tid];
+#pragma unroll
+                for (int e = 0; e < kV; ++e) store_out<TO>(orow + cv * kV + e, acc[e] * inv);
             }
             __syncthreads();
         }
@@ -282,7 +302,7 @@ attn_combine(const float* __restrict__ part_o, const float2* __restrict__ part_m
             float acc = 0.f;
             for (int i = 0; i < splits; ++i) {
                 const float w = s_w[i];
-                if (w != 0.f) acc = fmaf(w, part_o[(base + (size_t)i * n_h) * c + j], acc);
+                if (w != 0.f) acc = fmaf(w, load1(&part_o[(base + (size_t)i * n_h) * c + j]), acc);
             }
             store_out<TO>(orow + j, acc * inv);
         }
@@ -310,17 +330,30 @@ int launch_cuda_core(AttnArgs a, const AttnPlan& plan, int dtype, cudaStream_t s
 
 }  // namespace
 
-int launch_attn_combine(const AttnArgs& a, void* out, int out_bf16, float* lse,
+int launch_attn_combine(const AttnArgs& a, bool normalized, void* out, int out_bf16, float* lse,
                         cudaStream_t stream)
 {
     const int G = a.B * a.nq;
     dim3 grid((unsigned)a.n_h, (unsigned)G);
-    if (out_bf16)
-        launch_pdl(attn_combine<__nv_bfloat16>, grid, dim3(kCombineThreads), 0, stream, (const float*)a.part_o,
-                   (const float2*)a.part_ml, a.splits, a.n_h, a.c, static_cast<__nv_bfloat16*>(out), lse);
-    else
-        launch_pdl(attn_combine<float>, grid, dim3(kCombineThreads), 0, stream, (const float*)a.part_o,
-                   (const float2*)a.part_ml, a.splits, a.n_h, a.c, static_cast<float*>(out), lse);
+    dim3 block(kCombineThreads);
+    const float2* ml = a.part_ml;
+    if (normalized) {
+        const __nv_bfloat16* po = static_cast<const __nv_bfloat16*>(a.part_o);
+        if (out_bf16)
+            launch_pdl(attn_combine<__nv_bfloat16, __nv_bfloat16>, grid, block, 0, stream, po, ml, a.splits, a.n_h,
+                       a.c, static_cast<__nv_bfloat16*>(out), lse);
+        else
+            launch_pdl(attn_combine<float, __nv_bfloat16>, grid, block, 0, stream, po, ml, a.splits, a.n_h, a.c,
+                       static_cast<float*>(out), lse);
+    } else {
+        const float* po = static_cast<const float*>(a.part_o);
+        if (out_bf16)
+            launch_pdl(attn_combine<__nv_bfloat16, float>, grid, block, 0, stream, po, ml, a.splits, a.n_h, a.c,
+                       static_cast<__nv_bfloat16*>(out), lse);
+        else
+            launch_pdl(attn_combine<float, float>, grid, block, 0, stream, po, ml, a.splits, a.n_h, a.c,
+                       static_cast<float*>(out), lse);
+    }
     return launch_status();
 }
 
@@ -350,13 +383,13 @@ int attn_run(AttnArgs a, float scale, void* out, float* lse, void* workspace, si
     char* ws = static_cast<char*>(workspace);
     uint32_t* status = reinterpret_cast<uint32_t*>(ws);  // sticky device status word
     ws += 256;
-    a.part_o = reinterpret_cast<float*>(ws);
+    a.part_o = ws;
     a.part_ml = reinterpret_cast<float2*>(ws + align_up((size_t)G * plan.splits * a.n_h * a.c * sizeof(float), 256));
     a.splits = plan.splits;
     a.per_split = plan.per_split;
     int st = tc ? launch_attn_tc(a, plan, status, stream) : launch_cuda_core(a, plan, dtype, stream);
     if (st != CSA_OK) return st;
-    return launch_attn_combine(a, out, out_bf16, lse, stream);
+    return launch_attn_combine(a, tc, out, out_bf16, lse, stream);
 }
 
 }  // namespace csa

@@ -22,7 +22,7 @@ struct AttnArgs {
     float scale_log2;     // softmax scale * log2(e)
     int splits;
     int64_t per_split;    // list positions per split
-    float* part_o;        // [G][splits][n_h][c]
+    void* part_o;         // [G][splits][n_h][c]: fp32 O_i (CUDA-core path) or bf16 O_i / l_i (tcgen05 path)
     float2* part_ml;      // [G][splits][n_h] (max, sum) of 2^(scaled logit)
 };
 
@@ -37,7 +37,8 @@ AttnPlan attn_plan_tc(int G, int n_h, int c, int64_t entries);
 bool attn_tc_supported(int n_h, int c);
 size_t attn_ws_bytes(int G, int n_h, int c, int splits);
 int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cudaStream_t stream);
-int launch_attn_combine(const AttnArgs& a, void* out, int out_bf16, float* lse,
+// normalized: part_o holds bf16 O_i / l_i (tcgen05 path) instead of fp32 O_i.
+int launch_attn_combine(const AttnArgs& a, bool normalized, void* out, int out_bf16, float* lse,
                         cudaStream_t stream);
 
 }  // namespace csa

@@ -17,14 +17,18 @@
 // Entries are gathered by index with 16-byte cp.async into a double-buffered
 // 128-byte-swizzled tile; the same bytes are the K-major B operand of S and the
 // MN-major B operand of P C.
-//   warps 0-3 loaders  : q half (once) and the entry chunks -> shared memory
+//   warps 0-3 loaders  : q half (once) and the entry chunks -> shared memory; at the
+//                        end, output columns 0..127 -> staging; thread 0 issues the
+//                        TMA stores of the staged output half
 //   warps 4-7 softmax  : partial S rows from TMEM -> peer, S, online softmax with lazy
 //                        rescaling (O is rescaled in TMEM only when the running max grows
-//                        by more than 2^8), P (bf16) -> shared memory; final O half ->
-//                        partials through a shared-memory transpose
+//                        by more than 2^8), P (bf16) -> shared memory; at the end,
+//                        output columns 128..255 -> staging
 //   warp 8    MMA      : S(j+1) is issued before P(j) C so the tensor core stays busy
-// CTA pairs split the entry list; their partials (O unnormalised, running max and sum
-// in base 2) are merged by the combine kernel of attn.cu.  Every barrier wait is
+// CTA pairs split the entry list.  A split's partial is its normalised output O_i / l_i,
+// rounded to bf16 (relative error at most 2^-9 per element, the same as the bf16 P fed
+// to the tensor core) and written by TMA, with its running max and sum in base 2 in
+// fp32; the combine kernel of attn.cu merges the splits in fp32.  Every barrier wait is
 // bounded; a timeout sets the workspace status word and the CTA drains and exits.
 #include "attn.cuh"
 #include "tc_utils.cuh"
@@ -46,7 +50,7 @@ constexpr int kMaxIds = 1024;                     // entry ids of a range staged
 constexpr int kBarBytes = 256;
 constexpr int kSmem = 1024 + kQBytes + 2 * kCBytes + kPBytes + 2 * kRBytes + kBarBytes + kMaxIds * 4;
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
-static_assert(kQBytes + 2 * kCBytes >= kHeads * kHalf * 4, "output staging reuses q + chunks");
+static_assert(kQBytes + 2 * kCBytes >= kHeads * kHalf * 2, "output staging reuses q + chunks");
 
 CSA_DEV void cp_async16(uint32_t dst, const void* src, bool valid)
 {
@@ -128,24 +132,30 @@ CSA_DEV float ex2_approx(float x)
     return y;
 }
 
-constexpr int kBoxBytes = 128 * 128;  // one 128-row x 32-column fp32 output box
+constexpr int kBoxCols = 64;             // one output box: 128 rows x 64 bf16 columns (128 B)
+constexpr int kBoxBytes = kHeads * 128;  // 16 KB
 
 // Copy columns [col0, col0 + 128) of row h of the output half from TMEM (o_taddr: this
-// warp's lane quarter, first O column) into the staging boxes: eight 128-row x 32-column
-// fp32 boxes of 16 KB in the 128-byte swizzled layout of the output tensor map.
-CSA_DEV void stage_o_cols(uint8_t* stage, uint32_t o_taddr, int h, int col0)
+// warp's lane quarter, first O column), scaled by inv = 1 / l, into the staging boxes as
+// bf16: four 128-row x 64-column boxes in the 128-byte swizzled layout of the output
+// tensor map.
+CSA_DEV void stage_o_cols(uint8_t* stage, uint32_t o_taddr, int h, int col0, float inv)
 {
 #pragma unroll 1
     for (int c0 = col0; c0 < col0 + 128; c0 += 16) {
         float o[16];
         tc::tmem_ld16(o_taddr + c0, o);
         tc::tmem_wait_ld();
-        uint8_t* row = stage + (c0 >> 5) * kBoxBytes + h * 128;
-        const int q0 = (c0 & 31) >> 2;
+        uint32_t w[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<float4*>(row + (((q0 + i) ^ (h & 7)) << 4)) =
-                make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        for (int i = 0; i < 8; ++i) {
+            __nv_bfloat162 pr = __floats2bfloat162_rn(o[2 * i] * inv, o[2 * i + 1] * inv);
+            w[i] = *reinterpret_cast<uint32_t*>(&pr);
+        }
+        uint8_t* row = stage + (c0 / kBoxCols) * kBoxBytes + h * 128;
+        const int q0 = (c0 % kBoxCols) / 8;  // 16-byte chunk of the 128-byte box row
+        *reinterpret_cast<uint4*>(row + ((q0 ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(row + (((q0 + 1) ^ (h & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
     }
 }
 
@@ -180,6 +190,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
     volatile uint32_t* abort_flag = tmem_slot + 1;
     int* s_ids = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);  // [kMaxIds]
+    float* s_inv_l = reinterpret_cast<float*>(sP);  // [128] 1 / l per head, after the last P C
 
     pdl_launch_dependents();
     const int split = blockIdx.x, g = blockIdx.z;
@@ -299,7 +310,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
         // eight 128 x 32 boxes.
         if (!*abort_flag && tc::mbar_wait(Ofinal, 0, tc::kWaitBudget)) {
             tc::fence_after_sync();
-            stage_o_cols(smem, tmem + ((uint32_t)(warp * 32) << 16) + kHalf, warp * 32 + lane, 0);
+            const int h = warp * 32 + lane;
+            stage_o_cols(smem, tmem + ((uint32_t)(warp * 32) << 16) + kHalf, h, 0, s_inv_l[h]);
         } else {
             *abort_flag = 1;
         }
@@ -307,8 +319,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
         tc::mbar_arrive(staged);
         if (threadIdx.x == 0) {
             if (tc::mbar_wait(staged, 0, tc::kWaitBudget) && !*abort_flag) {
-                for (int p = 0; p < kHalf / 32; ++p)
-                    tc::tma_store_2d(&tmap_o, smem + p * kBoxBytes, half * kHalf + p * 32, (int)prow);
+                for (int p = 0; p < kHalf / kBoxCols; ++p)
+                    tc::tma_store_2d(&tmap_o, smem + p * kBoxBytes, half * kHalf + p * kBoxCols, (int)prow);
                 tc::bulk_store_commit_wait();
             } else {
                 *abort_flag = 1;
@@ -438,11 +450,14 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
             tc::mbar_arrive(Pfull);
         }
         if (ok && !*abort_flag && tc::mbar_wait(PVdone, (nchunks - 1) & 1, tc::kWaitBudget)) {
-            // The last P C has completed, so every MMA reading q and the chunks has too:
-            // those 128 KB now stage the 128 x 256 fp32 output half (columns 128..255 here).
+            // The last P C has completed, so every MMA reading q, the chunks and P has too:
+            // q + chunk buffers stage the output half as bf16 O / l (columns 128..255 here),
+            // and the P buffer passes 1 / l to the loader warps.
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            s_inv_l[h] = inv;
             tc::mbar_arrive(Ofinal);
             tc::fence_after_sync();
-            stage_o_cols(smem, tmem + lane_base + kHalf, h, 128);
+            stage_o_cols(smem, tmem + lane_base + kHalf, h, 128, inv);
             if (half == 0) a.part_ml[prow + h] = make_float2(m_run, l_run);
         } else {
             tc::mbar_arrive(Ofinal);
@@ -556,9 +571,9 @@ int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cu
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    CUtensorMap tmap_o;  // partial outputs [G * splits * 128 rows][512] fp32, 32 x 128 boxes
+    CUtensorMap tmap_o;  // partial outputs [G * splits * 128 rows][512] bf16, 64 x 128 boxes
     const uint64_t rows = (uint64_t)a.B * a.nq * plan.splits * kHeads;
-    if (!make_tmap_f32_2d(&tmap_o, a.part_o, rows, kC, kC, 32, kHeads)) return CSA_ERR_CUDA;
+    if (!make_tmap_bf16_2d(&tmap_o, a.part_o, rows, kC, kC, kBoxCols, kHeads)) return CSA_ERR_CUDA;
     cudaLaunchKernelEx(&cfg, attn_pair_kernel, tmap_o, a, status);
     return launch_status();
 }
