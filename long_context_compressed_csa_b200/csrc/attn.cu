@@ -176,15 +176,18 @@ CSA_DEV void store_out<float>(float* p, float v) { *p = v; }
 template <>
 CSA_DEV void store_out<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
-// 16 bytes of consecutive partial values, streamed (read once); zeros when !valid
-CSA_DEV void load_vec_stream(const float* p, bool valid, float (&v)[4])
+CSA_DEV float load1(const float* p) { return *p; }
+CSA_DEV float load1(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+// 16 bytes of partial values as raw bits, streamed (read once); their values as floats
+CSA_DEV uint4 load_raw_stream(const void* p) { return __ldcs(reinterpret_cast<const uint4*>(p)); }
+CSA_DEV void raw_to_float(uint4 x, float (&v)[4])
 {
-    const float4 x = valid ? __ldcs(reinterpret_cast<const float4*>(p)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    v[0] = __uint_as_float(x.x); v[1] = __uint_as_float(x.y);
+    v[2] = __uint_as_float(x.z); v[3] = __uint_as_float(x.w);
 }
-CSA_DEV void load_vec_stream(const __nv_bfloat16* p, bool valid, float (&v)[8])
+CSA_DEV void raw_to_float(uint4 x, float (&v)[8])
 {
-    const uint4 x = valid ? __ldcs(reinterpret_cast<const uint4*>(p)) : make_uint4(0, 0, 0, 0);
     const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -192,32 +195,41 @@ CSA_DEV void load_vec_stream(const __nv_bfloat16* p, bool valid, float (&v)[8])
         v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);  // high bf16
     }
 }
-CSA_DEV float load1(const float* p) { return *p; }
-CSA_DEV float load1(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-// One CTA per (head, query).  Every split's (max, sum) is read in one round, the
-// weights 2^(m_i - M) are formed in shared memory, and the partial rows are read by
-// (column quad, split group) threads that issue all their loads before using them, so
-// the kernel costs two dependent global round trips rather than one per split.
+// One CTA per (head, slice of kCombineCols output columns, query), so that the partial
+// rows are read by ~4 CTAs per head spread over all SMs (a CTA reads at most the SM's
+// share of the L2 bandwidth).  Thread (column group of 16 bytes, split group) issues
+// its partial loads right after the (max, sum) loads of every split; the weights are
+// formed in shared memory meanwhile.  A split whose weight is 0 (empty range, nothing
+// written) is excluded by a select, not a multiply.
 template <typename TO, typename TP>
 __global__ void __launch_bounds__(kCombineThreads)
 attn_combine(const TP* __restrict__ part_o, const float2* __restrict__ part_ml, int splits,
              int n_h, int c, TO* __restrict__ out, float* __restrict__ lse)
 {
     constexpr bool kNormalized = sizeof(TP) == 2;  // bf16 partials are O_i / l_i
+    constexpr int kV = 16 / sizeof(TP);             // partial values per 16-byte load
+    constexpr int kBatch = 8;                       // 16-byte loads in flight per thread
+    constexpr int kGroups = kCombineCols / kV;      // column groups of a full slice
+    static_assert(kCombineThreads % kGroups == 0, "whole split groups");
     pdl_launch_dependents();
     pdl_wait();
     const int h = blockIdx.x, g = blockIdx.y;
+    const int c0 = blockIdx.z * kCombineCols;
+    const int width = min(kCombineCols, c - c0);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     __shared__ float s_m[kMaxSplits], s_w[kMaxSplits];
     __shared__ float s_red[kCombineThreads / 32];
-    constexpr int kV = 16 / sizeof(TP);  // partial values per 16-byte load
     __shared__ float s_acc[kV * kCombineThreads];
-    constexpr int kBatch = 64 / kV;  // 16-byte loads issued per thread before the first use
-    __shared__ float s_M, s_inv;
     const size_t base = (size_t)g * splits * n_h + h;
+    TO* orow = out + ((size_t)g * n_h + h) * c + c0;
+    const bool vec = c % kV == 0;
+    const int ngrp = kCombineThreads / kGroups;     // split groups
+    const int cv = tid % kGroups, grp = tid / kGroups;
+    const bool worker = vec && cv * kV < width;
+    const TP* col = part_o + base * c + c0 + (size_t)cv * kV;
+    const size_t split_stride = (size_t)n_h * c;
 
-    // (max, sum) of every split: one round of loads
     float mloc = -INFINITY;
     for (int i = tid; i < splits; i += kCombineThreads) {
         const float2 ml = part_ml[base + (size_t)i * n_h];
@@ -225,17 +237,19 @@ attn_combine(const TP* __restrict__ part_o, const float2* __restrict__ part_ml, 
         s_w[i] = ml.y;
         mloc = fmaxf(mloc, ml.x);
     }
+    uint4 raw[kBatch];  // first batch of partial rows, in flight while the weights form
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+        const int i = grp + u * ngrp;
+        raw[u] = worker && i < splits ? load_raw_stream(col + (size_t)i * split_stride) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
     for (int off = 16; off; off >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, off));
     if (lane == 0) s_red[warp] = mloc;
     __syncthreads();
-    if (tid == 0) {
-        float M = -INFINITY;
-        for (int w = 0; w < kCombineThreads / 32; ++w) M = fmaxf(M, s_red[w]);
-        s_M = M;
-    }
-    __syncthreads();
-    const float M = s_M;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCombineThreads / 32; ++w) M = fmaxf(M, s_red[w]);
     float lloc = 0.f;
     for (int i = tid; i < splits; i += kCombineThreads) {
         const float w = s_m[i] == -INFINITY ? 0.f : exp2f(s_m[i] - M);
@@ -247,62 +261,51 @@ attn_combine(const TP* __restrict__ part_o, const float2* __restrict__ part_ml, 
     __syncthreads();
     if (lane == 0) s_red[warp] = lloc;
     __syncthreads();
-    if (tid == 0) {
-        float L = 0.f;
-        for (int w = 0; w < kCombineThreads / 32; ++w) L += s_red[w];
-        s_inv = L > 0.f ? 1.f / L : 0.f;
-        if (lse) lse[(size_t)g * n_h + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
-    }
-    __syncthreads();
-    const float inv = s_inv;
-    TO* orow = out + ((size_t)g * n_h + h) * c;
-    if (c % kV == 0) {
-        // (column group of kV, split group) threads; kV = 16 bytes of partial per load
-        const int ncv = c / kV;
-        const int per = ncv < kCombineThreads ? ncv : kCombineThreads;  // column groups per pass
-        const int ngrp = kCombineThreads / per;                         // split groups
-        for (int cv0 = 0; cv0 < ncv; cv0 += per) {
-            const int cv = cv0 + tid % per;
-            const int grp = tid / per;
-            float acc[kV];
+    float L = 0.f;
 #pragma unroll
-            for (int e = 0; e < kV; ++e) acc[e] = 0.f;
-            if (grp < ngrp && cv < ncv) {
-                const TP* col = part_o + base * c + (size_t)cv * kV;
-                for (int i0 = grp; i0 < splits; i0 += kBatch * ngrp) {
-                    float v[kBatch][kV];
+    for (int w = 0; w < kCombineThreads / 32; ++w) L += s_red[w];
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    if (tid == 0 && blockIdx.z == 0 && lse)
+        lse[(size_t)g * n_h + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+
+    if (vec) {
+        float acc[kV];
 #pragma unroll
-                    for (int u = 0; u < kBatch; ++u) {
-                        const int i = i0 + u * ngrp;
-                        load_vec_stream(col + (size_t)i * n_h * c, i < splits && s_w[i] != 0.f, v[u]);
-                    }
+        for (int e = 0; e < kV; ++e) acc[e] = 0.f;
+        for (int i0 = grp; worker && i0 < splits; i0 += kBatch * ngrp) {
+            if (i0 != grp) {  // later batches (more than kBatch splits per split group)
 #pragma unroll
-                    for (int u = 0; u < kBatch; ++u) {
-                        const int i = i0 + u * ngrp;
-                        const float w = i < splits ? s_w[i] : 0.f;
-#pragma unroll
-                        for (int e = 0; e < kV; ++e) acc[e] = fmaf(w, v[u][e], acc[e]);
-                    }
+                for (int u = 0; u < kBatch; ++u) {
+                    const int i = i0 + u * ngrp;
+                    raw[u] = i < splits ? load_raw_stream(col + (size_t)i * split_stride) : make_uint4(0, 0, 0, 0);
                 }
             }
 #pragma unroll
-            for (int e = 0; e < kV; ++e) s_acc[e * kCombineThreads + tid] = acc[e];
-            __syncthreads();
-            if (grp == 0 && cv < ncv) {
-                for (int q = 1; q < ngrp; ++q)
+            for (int u = 0; u < kBatch; ++u) {
+                const int i = i0 + u * ngrp;
+                const float w = i < splits ? s_w[i] : 0.f;
+                float v[kV];
+                raw_to_float(raw[u], v);
 #pragma unroll
-                    for (int e = 0; e < kV; ++e) acc[e] += s_acc[e * kCombineThreads + q * per + tid];
-#pragma unroll
-                for (int e = 0; e < kV; ++e) store_out<TO>(orow + cv * kV + e, acc[e] * inv);
+                for (int e = 0; e < kV; ++e) acc[e] = w != 0.f ? fmaf(w, v[e], acc[e]) : acc[e];
             }
-            __syncthreads();
+        }
+#pragma unroll
+        for (int e = 0; e < kV; ++e) s_acc[e * kCombineThreads + tid] = acc[e];
+        __syncthreads();
+        if (grp == 0 && worker) {
+            for (int q = 1; q < ngrp; ++q)
+#pragma unroll
+                for (int e = 0; e < kV; ++e) acc[e] += s_acc[e * kCombineThreads + q * kGroups + tid];
+#pragma unroll
+            for (int e = 0; e < kV; ++e) store_out<TO>(orow + cv * kV + e, acc[e] * inv);
         }
     } else {
-        for (int j = tid; j < c; j += kCombineThreads) {
+        for (int j = tid; j < width; j += kCombineThreads) {
             float acc = 0.f;
             for (int i = 0; i < splits; ++i) {
                 const float w = s_w[i];
-                if (w != 0.f) acc = fmaf(w, load1(&part_o[(base + (size_t)i * n_h) * c + j]), acc);
+                if (w != 0.f) acc = fmaf(w, load1(&part_o[(base + (size_t)i * n_h) * c + c0 + j]), acc);
             }
             store_out<TO>(orow + j, acc * inv);
         }
@@ -334,7 +337,7 @@ int launch_attn_combine(const AttnArgs& a, bool normalized, void* out, int out_b
                         cudaStream_t stream)
 {
     const int G = a.B * a.nq;
-    dim3 grid((unsigned)a.n_h, (unsigned)G);
+    dim3 grid((unsigned)a.n_h, (unsigned)G, (unsigned)((a.c + kCombineCols - 1) / kCombineCols));
     dim3 block(kCombineThreads);
     const float2* ml = a.part_ml;
     if (normalized) {

@@ -8,7 +8,8 @@ constexpr int kMaxC = 512;        // widest compressed entry the kernels hold on
 constexpr int kMaxSplits = 1024;  // splits per query the combine kernel accepts
 constexpr int kCcHeads = 16;      // CUDA-core kernel: heads per CTA
 constexpr int kCcChunk = 32;      // CUDA-core kernel: entries per shared-memory chunk
-constexpr int kCombineThreads = 512;
+constexpr int kCombineThreads = 256;
+constexpr int kCombineCols = 128;  // output columns per combine CTA
 
 struct AttnArgs {
     const void* q;        // [G][n_h][c]
