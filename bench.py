@@ -321,21 +321,19 @@ def micro(kind, iters, rotate=4):
     for f in calls:
         f()
     torch.cuda.synchronize()
-    # each call captured once in a CUDA graph, so host launch latency is not timed
-    graphs = []
-    for f in calls:
-        gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr):
-            f()
-        graphs.append(gr)
-    for gr in graphs:
-        gr.replay()
+    # all timed calls captured in one CUDA graph with an event record node before and
+    # after each call, so neither host launch latency nor host pacing is timed
+    evs = [(torch.cuda.Event(enable_timing=True, external=True),
+            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(iters)]
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for i in range(iters):
+            evs[i][0].record()
+            calls[i % len(calls)]()
+            evs[i][1].record()
+    gr.replay()  # warm-up
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
-    for i in range(iters):
-        evs[i][0].record()
-        graphs[i % len(graphs)].replay()
-        evs[i][1].record()
+    gr.replay()
     torch.cuda.synchronize()
     us = np.array([a.elapsed_time(b) * 1e3 for a, b in evs])
     hbm, _, src = peaks()
