@@ -333,6 +333,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = tc::mbar_wait(idsready, 0, tc::kWaitBudget);
+        int sent = 0;  // chunks whose partial logits thread 128 sent to the peer
         for (int j = 0; j < nchunks && ok; ++j) {
             const int buf = j & 1;
             const uint32_t ph = (j >> 1) & 1;
@@ -369,6 +370,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
                     bulk_copy_to_peer(peer_addr(tc::smem_u32(sR), peer), tc::smem_u32(sX), kRBytes,
                                       peer_addr(tc::smem_u32(Rfull), peer));
                     bulk_wait_read();
+                    ++sent;
                 }
                 tc::mbar_arrive(Xfree);
             }
@@ -466,6 +468,11 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
         }
         tc::fence_proxy_async_smem();
         tc::mbar_arrive(staged);
+        // The peer's last access to this CTA's shared memory is its arrival on Rfree after
+        // consuming the last chunk sent; once it is in, this CTA may exit (no cluster-wide
+        // barrier at the end).
+        if (threadIdx.x == 128 && sent > 0 && !mbar_wait_cluster(Rfree, (sent - 1) & 1, tc::kWaitBudget))
+            *abort_flag = 1;
     } else {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -526,7 +533,6 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, 512);
     }
-    cluster_sync();  // the peer may write into this CTA's shared memory until here
 }
 
 }  // namespace
