@@ -370,6 +370,41 @@ def test_dense_attn_random(dtype, n_h, c):
                                    rtol=0)
 
 
+def test_attn_many_queries_and_workspace_reuse():
+    """80 queries of 128 heads in one call (one CTA pair per query, padding inside one
+    list); then one dense workspace reused across calls whose visible counts, hence split
+    plans, differ."""
+    dtype, n_h, c = torch.bfloat16, 128, 512
+    B, nq, N_cap, k = 1, 80, 512, 96
+    q = randn((B, nq, n_h, c), 330, dtype)
+    cache = randn((B, N_cap, c), 331, dtype)
+    g = torch.Generator().manual_seed(332)
+    idx = torch.stack([torch.randperm(N_cap, generator=g)[:k] for _ in range(nq)]).to(torch.int32)
+    idx[3, 5:20] = -1                                    # padding inside one list
+    o, lse = run_sparse(dev(q), dev(cache), dev(idx.reshape(B, nq, k)))
+    for j in (0, 3, 41, 79):
+        sel = idx[j].numpy()
+        ref, ref_lse = _ref_attn(to_f64(q[0, j]), to_f64(cache[0]), sel[sel >= 0])
+        assert max_rel_rowwise(o[0, j], ref).max() <= TOL[dtype]
+        np.testing.assert_allclose(lse[0, j], ref_lse, atol=2e-3, rtol=0)
+    # dense, one workspace, growing then shrinking visible counts
+    mp, Nh = 128, 4096
+    qd = randn((1, 1, n_h, c), 333, dtype)
+    cd = randn((1, Nh, c), 334, dtype)
+    ws = torch.zeros(csa_attn_workspace_size(1, 1, n_h, c, Nh), dtype=torch.uint8, device=DEV)
+    for tpos in (mp * 64 + 3, mp * Nh, mp * 700 + 1, mp * 65):
+        out = torch.full((1, 1, n_h, c), float("nan"), dtype=torch.float32, device=DEV)
+        lsed = torch.full((1, 1, n_h), float("nan"), device=DEV)
+        tt = torch.tensor([tpos], dtype=torch.int64, device=DEV).reshape(1, 1)
+        hca_dense_attn(dev(qd), dev(cd), tt, mp, out, ws, lse=lsed)
+        torch.cuda.synchronize()
+        assert csa_workspace_status(ws) == 0
+        vis = oracle.visible(tpos, mp, Nh)
+        ref, ref_lse = _ref_attn(to_f64(qd[0, 0]), to_f64(cd[0]), np.arange(vis, dtype=np.int32))
+        assert max_rel_rowwise(out.cpu().numpy()[0, 0], ref).max() <= TOL[dtype]
+        np.testing.assert_allclose(lsed.cpu().numpy()[0, 0], ref_lse, atol=2e-3, rtol=0)
+
+
 # ==================================================================================
 # end to end: streams -> caches -> indexer/top-k -> sparse attention; HCA likewise
 # ==================================================================================
