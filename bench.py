@@ -34,6 +34,10 @@ sys.path.insert(0, ROOT)
 METRIC = "CSA/HCA decode tokens/s at 128K–1M ctx; achieved HBM GB/s vs ~8 TB/s peak"
 WORKLOAD = "hybrid_1m_decode"
 N_PAIRS = 8
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one scan_tc_kernel launch
+# over 262144 keys, from one ncu capture of the current kernel (67.23 MB read, 0.71 MB
+# written; algorithmic 67.11 MB).  Must be retaken (or set to None) when the kernel changes.
+SCAN_TRAFFIC_BYTES = 67_940_608
 
 
 def log(*a):
@@ -478,9 +482,10 @@ def main():
                          "584 MiB between revisits of a pair)",
                    "step": "one token through one CSA+HCA layer pair (indexer+top-k, sparse MQA, "
                            "dense MQA, incremental compress at block ends)"},
-        "roofline": {"kernel": "csa_indexer_topk (indexer scan + top-k select)", "bound": "hbm",
+        "roofline": {"kernel": "csa_indexer_topk (scan_tc_kernel: indexer scan with the top-k "
+                               "select in place)", "bound": "hbm",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_source": src + " (burst copy)", "traffic": None,
+                     "peak_source": src + " (burst copy)", "traffic": SCAN_TRAFFIC_BYTES,
                      "algorithmic_bytes_per_launch": idx_bytes,
                      "avg_launch_us": idx_avg_s * 1e6},
         "step_roofline": {"achieved": step_gbs, "peak": hbm, "unit": "GB/s", "frac": step_gbs / hbm,
