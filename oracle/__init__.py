@@ -52,6 +52,8 @@ def _load():
             lib.oracle_hca_compress.argtypes = [dp, dp, dp, i64, i64, i64, i64, i64, dp]
             lib.oracle_visible.argtypes = [i64, i64, i64]
             lib.oracle_visible.restype = i64
+            lib.oracle_window.argtypes = [i64, i64, ctypes.POINTER(ctypes.c_int64)]
+            lib.oracle_window.restype = i64
             lib.oracle_index_scores.argtypes = [dp, dp, dp, i64, i64, i64, dp]
             lib.oracle_topk.argtypes = [dp, i64, i64, ctypes.POINTER(ctypes.c_int32)]
             lib.oracle_mqa.argtypes = [dp, dp, ctypes.POINTER(ctypes.c_int32), i64, i64, i64,
@@ -165,6 +167,26 @@ def mqa(q, cache, sel, scale=None):
                        _ptr(sel, ctypes.c_int32) if sel.size else None, sel.size, n_h, c,
                        float(scale), _ptr(out), _ptr(lse))
     return out, lse
+
+
+def window_positions(t, n_win):
+    """Token positions of the sliding-window branch for the query at position t:
+    max(0, t - n_win + 1) .. t (bhhxx.wiki "MHA -> ... -> CSA/HCA" section 6, W_t)."""
+    pos = np.empty((max(int(n_win), 1),), np.int64)
+    n = _load().oracle_window(int(t), int(n_win), _ptr(pos, ctypes.c_int64))
+    return pos[:n].copy()
+
+
+def mqa_window(q, cache, sel, win_rows, scale=None):
+    """MQA whose shared key/value set is the selected compressed entries ``sel`` (-1
+    skipped) concatenated with the sliding-window entries ``win_rows`` [n, c] (bhhxx.wiki
+    section 6: "concat sliding window key/value entries and compressed entries"), under
+    one softmax.  Returns (out [n_h, c], lse [n_h])."""
+    cache, win_rows = _d(cache), _d(win_rows).reshape(-1, _d(cache).shape[1])
+    sel = np.ascontiguousarray(sel, dtype=np.int32).reshape(-1)
+    keys = np.concatenate([cache, win_rows], axis=0)
+    sel2 = np.concatenate([sel, cache.shape[0] + np.arange(win_rows.shape[0], dtype=np.int32)])
+    return mqa(q, keys, sel2, scale)
 
 
 def round_bf16(x):

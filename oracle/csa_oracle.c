@@ -243,3 +243,19 @@ void oracle_mqa(const double* q, const double* cache, const int32_t* sel, int64_
     }
     free(logit);
 }
+
+/* Sliding-window branch: the raw-token positions the query at position t attends to
+ * besides the compressed entries.  bhhxx.wiki "MHA -> ... -> CSA/HCA", section 6 (HCA and
+ * CSA paths) defines W_t = {max(1, t - n_window + 1), ..., t} on 1-based positions; with
+ * this library's 0-based positions that is {max(0, t - n_win + 1), ..., t}, the current
+ * token included.  Writes the positions in ascending order into pos (capacity n_win)
+ * and returns their count (0 when t < 0 or n_win <= 0). */
+int64_t oracle_window(int64_t t, int64_t n_win, int64_t* pos)
+{
+    if (t < 0 || n_win <= 0) return 0;
+    int64_t lo = t - n_win + 1;
+    if (lo < 0) lo = 0;
+    int64_t n = 0;
+    for (int64_t p = lo; p <= t; ++p) pos[n++] = p;
+    return n;
+}

@@ -388,3 +388,64 @@ def test_ledger_ratios():
     from oracle.ledger import raw_request_bytes
     assert raw_request_bytes() == 10**6 * 61 * 4096
     assert abs(raw_request_bytes() - L["raw_request_bytes_1M_61_layers"]) / 2.5e11 < 0.01
+
+
+# ==================================================================================
+# sliding-window branch (bhhxx.wiki "MHA -> ... -> CSA/HCA" section 6: W_t and the
+# concatenation of window and compressed key/value entries under one softmax)
+# ==================================================================================
+def test_window_positions_pins():
+    # W_t = {max(1, t-n+1), ..., t} on 1-based positions, i.e. max(0, t-n+1) .. t here
+    assert oracle.window_positions(0, 128).tolist() == [0]
+    assert oracle.window_positions(5, 128).tolist() == [0, 1, 2, 3, 4, 5]
+    w = oracle.window_positions(1000, 128)
+    assert len(w) == 128 and w[0] == 873 and w[-1] == 1000 and np.all(np.diff(w) == 1)
+    assert oracle.window_positions(127, 128).tolist() == list(range(128))
+    assert oracle.window_positions(128, 128).tolist() == list(range(1, 129))
+    assert oracle.window_positions(7, 1).tolist() == [7]
+    assert oracle.window_positions(-1, 4).size == 0 and oracle.window_positions(9, 0).size == 0
+
+
+def test_window_mqa_closed_form_two_entries():
+    """One compressed entry and one window entry, c = 2, one head: the output is the
+    softmax(logit) mix of the two in closed form."""
+    a, b = 1.3, -0.4
+    q = np.array([[1.0, 2.0]])
+    cache = np.array([[a, 0.0]])           # logit = a / sqrt(2)
+    win = np.array([[0.0, b]])             # logit = 2b / sqrt(2)
+    out, lse = oracle.mqa_window(q, cache, np.array([0]), win)
+    la, lb = a / np.sqrt(2.0), 2 * b / np.sqrt(2.0)
+    pa = np.exp(la) / (np.exp(la) + np.exp(lb))
+    np.testing.assert_allclose(out[0], [pa * a, (1 - pa) * b], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse[0], np.log(np.exp(la) + np.exp(lb)), rtol=0, atol=1e-14)
+
+
+def test_window_mqa_invariants():
+    rng = np.random.default_rng(7)
+    n_h, c, N = 3, 8, 20
+    q, cache = rng.standard_normal((n_h, c)), rng.standard_normal((N, c))
+    win = rng.standard_normal((5, c))
+    sel = np.array([4, -1, 11, 2], dtype=np.int32)
+    out, lse = oracle.mqa_window(q, cache, sel, win)
+    # the order of the window rows (and of the selection) does not matter
+    out2, lse2 = oracle.mqa_window(q, cache, sel[::-1], win[::-1])
+    np.testing.assert_allclose(out2, out, atol=1e-13)
+    np.testing.assert_allclose(lse2, lse, atol=1e-13)
+    # window only (every compressed slot padded) equals plain MQA over the window rows
+    ow, lw = oracle.mqa_window(q, cache, np.full(3, -1, np.int32), win)
+    ow2, lw2 = oracle.mqa(q, win, np.arange(5, dtype=np.int32))
+    np.testing.assert_allclose(ow, ow2, atol=1e-13)
+    np.testing.assert_allclose(lw, lw2, atol=1e-13)
+    # no window rows: plain sparse MQA
+    o0, l0 = oracle.mqa_window(q, cache, sel, np.zeros((0, c)))
+    o1, l1 = oracle.mqa(q, cache, sel)
+    np.testing.assert_allclose(o0, o1, atol=1e-14)
+    np.testing.assert_allclose(l0, l1, atol=1e-14)
+    # a window row equal to a selected compressed row counts as that entry twice
+    od, ld = oracle.mqa_window(q, cache, np.array([4, 11], np.int32), cache[[4]])
+    oe, le = oracle.mqa(q, cache, np.array([4, 4, 11], np.int32))
+    np.testing.assert_allclose(od, oe, atol=1e-13)
+    np.testing.assert_allclose(ld, le, atol=1e-13)
+    # lse combines like a union: exp(lse) = exp(lse_comp) + exp(lse_win)
+    lc = oracle.mqa(q, cache, sel)[1]
+    np.testing.assert_allclose(np.exp(lse), np.exp(lc) + np.exp(lw2), rtol=1e-12)
