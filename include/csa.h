@@ -197,6 +197,36 @@ int hca_dense_attn(const void* q, const void* cache, const int64_t* t,
                    void* out, float* lse, void* workspace, size_t ws_bytes,
                    int dtype, int out_bf16, csa_stream_t stream);
 
+/* ---------------------------------------------------------------------------------
+ * csa_sparse_attn_window, hca_dense_attn_window - csa_sparse_attn / hca_dense_attn with the
+ * sliding-window branch.  The query at position t also attends, under the same softmax,
+ * to the window key/value entries of the raw tokens max(0, t - n_win + 1) .. t, the
+ * current token included.
+ *   Source: bhhxx.wiki "MHA -> ... -> CSA/HCA" section 6 gives W_t = {max(1, t - n_window
+ *   + 1), ..., t} on 1-based positions and concatenates the window entries with the
+ *   compressed entries as one shared key/value set.  dev.to "DSA, CSA, HCA and mHC"
+ *   section 4 gives the V4-Pro window: 128 tokens.
+ * win     : [B, win_cap, c] (dtype) ring buffer of window entries c_i^window = h_i
+ *           W^{window,KV} (projected by the caller); token p of sequence b is row
+ *           p % win_cap.  Requires 1 <= n_win <= win_cap < 2^31.  16-byte aligned for the
+ *           tensor-core path.
+ * t       : DEVICE int64 [B*nq] query positions (hca_dense_attn_window: the same t that
+ *           bounds the compressed entries).  t < 0: no window entry.
+ * workspace : >= csa_attn_workspace_size(B, nq, n_h, c, k + n_win) bytes (sparse), or
+ *             (..., N_cap + n_win) (dense).
+ * All other arguments, outputs and errors as for csa_sparse_attn / hca_dense_attn.
+ * ------------------------------------------------------------------------------- */
+int csa_sparse_attn_window(const void* q, const void* cache, const int32_t* idx,
+                           const void* win, const int64_t* t, int B, int nq, int n_h, int c,
+                           int64_t N_cap, int k, int n_win, int64_t win_cap, float scale,
+                           void* out, float* lse, void* workspace, size_t ws_bytes,
+                           int dtype, int out_bf16, csa_stream_t stream);
+int hca_dense_attn_window(const void* q, const void* cache, const int64_t* t, const void* win,
+                          int B, int nq, int n_h, int c, int64_t N_cap, int m_prime,
+                          int n_win, int64_t win_cap, float scale, void* out, float* lse,
+                          void* workspace, size_t ws_bytes, int dtype, int out_bf16,
+                          csa_stream_t stream);
+
 /* Device status of a workspace of csa_indexer_topk, csa_sparse_attn or hca_dense_attn:
  * synchronises `stream` and returns CSA_OK, or CSA_ERR_TIMEOUT if a tensor-core kernel
  * of an earlier call gave up a bounded wait (its outputs are then invalid).  The status

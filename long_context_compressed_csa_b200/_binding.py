@@ -33,6 +33,10 @@ _SIGS = {
                         i32),
     "hca_dense_attn": ([vp, vp, vp, i32, i32, i32, i32, i64, i32, f32, vp, vp, vp, sz, i32, i32, vp],
                        i32),
+    "csa_sparse_attn_window": ([vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i32, i32, i64, f32, vp, vp,
+                                vp, sz, i32, i32, vp], i32),
+    "hca_dense_attn_window": ([vp, vp, vp, vp, i32, i32, i32, i32, i64, i32, i32, i64, f32, vp, vp, vp,
+                               sz, i32, i32, vp], i32),
 }
 
 
@@ -185,30 +189,53 @@ def csa_attn_workspace_size(B, nq, n_h, c, max_entries) -> int:
     return int(library().csa_attn_workspace_size(B, nq, n_h, c, max_entries))
 
 
-def csa_sparse_attn(q, cache, idx, out, workspace, lse=None, scale=0.0, stream=None):
-    """MQA of q [B,nq,n_h,c] over cache [B,N_cap,c] rows idx int32 [B,nq,k] (-1 = pad)."""
-    _cuda(q, cache, idx, out, workspace, lse)
+def csa_sparse_attn(q, cache, idx, out, workspace, lse=None, scale=0.0, stream=None,
+                    win=None, t=None, n_win=0):
+    """MQA of q [B,nq,n_h,c] over cache [B,N_cap,c] rows idx int32 [B,nq,k] (-1 = pad).
+
+    With ``win`` [B,win_cap,c] (ring buffer, token p at row p % win_cap), device int64
+    positions ``t`` [B,nq] and ``n_win`` >= 1, the window entries of tokens
+    max(0, t-n_win+1) .. t join the same softmax (csa_sparse_attn_window)."""
+    _cuda(q, cache, idx, out, workspace, lse, win, t)
     B, nq, n_h, c = q.shape
     N_cap = cache.shape[1]
     k = idx.shape[2]
     assert q.is_contiguous() and cache.is_contiguous() and idx.is_contiguous() and out.is_contiguous()
     assert cache.shape[0] == B and cache.shape[2] == c and idx.shape[:2] == (B, nq) and out.shape == q.shape
     out_bf16 = 1 if out.dtype.itemsize == 2 else 0
-    _check("csa_sparse_attn", library().csa_sparse_attn(
-        _ptr(q), _ptr(cache), _ptr(idx), B, nq, n_h, c, N_cap, k, float(scale), _ptr(out), _ptr(lse),
-        _ptr(workspace), workspace.numel() * workspace.element_size(), _dtype(q), out_bf16,
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if win is None:
+        _check("csa_sparse_attn", library().csa_sparse_attn(
+            _ptr(q), _ptr(cache), _ptr(idx), B, nq, n_h, c, N_cap, k, float(scale), _ptr(out), _ptr(lse),
+            _ptr(workspace), ws_bytes, _dtype(q), out_bf16, _stream(stream)))
+        return
+    assert win.is_contiguous() and win.shape[0] == B and win.shape[2] == c and t.numel() == B * nq
+    _check("csa_sparse_attn_window", library().csa_sparse_attn_window(
+        _ptr(q), _ptr(cache), _ptr(idx), _ptr(win), _ptr(t), B, nq, n_h, c, N_cap, k, int(n_win),
+        win.shape[1], float(scale), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _dtype(q), out_bf16,
         _stream(stream)))
 
 
-def hca_dense_attn(q, cache, t, m_prime, out, workspace, lse=None, scale=0.0, stream=None):
-    """Dense MQA of q [B,nq,n_h,c] over cache [B,N_cap,c] rows s < floor(t/m')."""
-    _cuda(q, cache, t, out, workspace, lse)
+def hca_dense_attn(q, cache, t, m_prime, out, workspace, lse=None, scale=0.0, stream=None,
+                   win=None, n_win=0):
+    """Dense MQA of q [B,nq,n_h,c] over cache [B,N_cap,c] rows s < floor(t/m').
+
+    With ``win`` [B,win_cap,c] and ``n_win`` >= 1, the window entries of tokens
+    max(0, t-n_win+1) .. t join the same softmax (hca_dense_attn_window)."""
+    _cuda(q, cache, t, out, workspace, lse, win)
     B, nq, n_h, c = q.shape
     N_cap = cache.shape[1]
     assert q.is_contiguous() and cache.is_contiguous() and out.is_contiguous()
     assert t.numel() == B * nq and cache.shape[0] == B and cache.shape[2] == c and out.shape == q.shape
     out_bf16 = 1 if out.dtype.itemsize == 2 else 0
-    _check("hca_dense_attn", library().hca_dense_attn(
-        _ptr(q), _ptr(cache), _ptr(t), B, nq, n_h, c, N_cap, m_prime, float(scale), _ptr(out),
-        _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(), _dtype(q),
-        out_bf16, _stream(stream)))
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if win is None:
+        _check("hca_dense_attn", library().hca_dense_attn(
+            _ptr(q), _ptr(cache), _ptr(t), B, nq, n_h, c, N_cap, m_prime, float(scale), _ptr(out),
+            _ptr(lse), _ptr(workspace), ws_bytes, _dtype(q), out_bf16, _stream(stream)))
+        return
+    assert win.is_contiguous() and win.shape[0] == B and win.shape[2] == c
+    _check("hca_dense_attn_window", library().hca_dense_attn_window(
+        _ptr(q), _ptr(cache), _ptr(t), _ptr(win), B, nq, n_h, c, N_cap, m_prime, int(n_win), win.shape[1],
+        float(scale), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _dtype(q), out_bf16,
+        _stream(stream)))

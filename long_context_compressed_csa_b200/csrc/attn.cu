@@ -64,14 +64,25 @@ attn_cuda_core(AttnArgs a)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h_base = hg * kCcHeads;
 
-    int64_t count;  // number of list positions for this query
+    // list positions: [0, ncomp) compressed entries, then the sliding-window entries
+    int64_t ncomp;
     if (a.dense) {
         const int64_t tt = a.t[g];
         const int64_t v = tt < 0 ? 0 : tt / a.m_prime;
-        count = v < a.N_cap ? v : a.N_cap;
+        ncomp = v < a.N_cap ? v : a.N_cap;
     } else {
-        count = a.k;
+        ncomp = a.k;
     }
+    int64_t nwin = 0;
+    int wrow0 = 0;  // ring row of the window's first token
+    if (a.win) {
+        const int64_t tt = a.t[g];
+        if (tt >= 0) {
+            nwin = tt + 1 < a.n_win ? tt + 1 : a.n_win;
+            wrow0 = (int)((tt - nwin + 1) % a.win_cap);
+        }
+    }
+    const int64_t count = ncomp + nwin;
     const int64_t p_begin = (int64_t)split * a.per_split;
     const int64_t p_end = min(count, p_begin + a.per_split);
 
@@ -92,13 +103,18 @@ attn_cuda_core(AttnArgs a)
     }
 
     const T* cache = static_cast<const T*>(a.cache) + b * a.N_cap * c;
+    const T* wcache = a.win ? static_cast<const T*>(a.win) + b * (int64_t)a.win_cap * c : cache;
     for (int64_t p0 = p_begin; p0 < p_end; p0 += kCcChunk) {
         __syncthreads();  // previous chunk fully consumed (and sQ staged on entry)
         if (threadIdx.x < kCcChunk) {
             const int64_t p = p0 + threadIdx.x;
-            int e = -1;
+            int e = -1;  // >= 0 compressed entry, <= -2 window row -2 - e, -1 none
             if (p < p_end) {
-                if (a.dense) {
+                if (p >= ncomp) {  // window position: at most one wrap of the ring
+                    int r = wrow0 + (int)(p - ncomp);
+                    r = r >= a.win_cap ? r - a.win_cap : r;
+                    e = -2 - r;
+                } else if (a.dense) {
                     e = (int)p;
                 } else {
                     const int32_t v = a.idx[(int64_t)g * a.k + p];
@@ -111,10 +127,12 @@ attn_cuda_core(AttnArgs a)
         for (int i = threadIdx.x; i < kCcChunk * c; i += 256) {
             const int r = i / c, j = i % c;
             const int e = s_ent[r];
-            sC[r * cs + j] = e >= 0 ? to_f32(cache[(int64_t)e * c + j]) : 0.f;
+            sC[r * cs + j] = e >= 0    ? to_f32(cache[(int64_t)e * c + j])
+                             : e <= -2 ? to_f32(wcache[(int64_t)(-2 - e) * c + j])
+                                       : 0.f;
         }
         __syncthreads();
-        const bool valid = s_ent[lane] >= 0;
+        const bool valid = s_ent[lane] != -1;
 #pragma unroll
         for (int x = 0; x < HPW; ++x) {
             const int hh = warp * HPW + x;
@@ -439,5 +457,57 @@ extern "C" int hca_dense_attn(const void* q, const void* cache, const int64_t* t
     a.B = B; a.nq = nq; a.n_h = n_h; a.c = c; a.N_cap = N_cap; a.k = 0; a.m_prime = m_prime;
     a.dense = 1;
     return attn_run(a, scale, out, lse, workspace, ws_bytes, dtype, out_bf16, N_cap,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Sliding-window variants: the same calls with the window entries of tokens
+// max(0, t - n_win + 1) .. t joined to the entry set under one softmax.
+namespace {
+int window_args(csa::AttnArgs& a, const void* win, const int64_t* t, int n_win, int64_t win_cap,
+                int dtype)
+{
+    if (!win || !t || n_win < 1 || win_cap < n_win || win_cap >= (int64_t(1) << 31)) return CSA_ERR_ARG;
+    if (((uintptr_t)win & (uintptr_t)(csa::elem_bytes(dtype) - 1)) || ((uintptr_t)t & 7)) return CSA_ERR_ALIGN;
+    a.win = win;
+    a.t = t;  // the sparse path reads t only for the window
+    a.n_win = n_win;
+    a.win_cap = (int)win_cap;
+    return CSA_OK;
+}
+}  // namespace
+
+extern "C" int csa_sparse_attn_window(const void* q, const void* cache, const int32_t* idx,
+                                      const void* win, const int64_t* t, int B, int nq, int n_h,
+                                      int c, int64_t N_cap, int k, int n_win, int64_t win_cap,
+                                      float scale, void* out, float* lse, void* workspace,
+                                      size_t ws_bytes, int dtype, int out_bf16, csa_stream_t stream)
+{
+    using namespace csa;
+    if (k < 0) return CSA_ERR_ARG;
+    AttnArgs a{};
+    a.q = q; a.cache = cache; a.idx = idx; a.t = nullptr;
+    a.B = B; a.nq = nq; a.n_h = n_h; a.c = c; a.N_cap = N_cap; a.k = k; a.m_prime = 1;
+    a.dense = 0;
+    const int st = window_args(a, win, t, n_win, win_cap, dtype);
+    if (st != CSA_OK) return st;
+    return attn_run(a, scale, out, lse, workspace, ws_bytes, dtype, out_bf16, (int64_t)k + n_win,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int hca_dense_attn_window(const void* q, const void* cache, const int64_t* t, const void* win,
+                                     int B, int nq, int n_h, int c, int64_t N_cap, int m_prime,
+                                     int n_win, int64_t win_cap, float scale, void* out, float* lse,
+                                     void* workspace, size_t ws_bytes, int dtype, int out_bf16,
+                                     csa_stream_t stream)
+{
+    using namespace csa;
+    if (m_prime <= 0) return CSA_ERR_ARG;
+    AttnArgs a{};
+    a.q = q; a.cache = cache; a.idx = nullptr; a.t = t;
+    a.B = B; a.nq = nq; a.n_h = n_h; a.c = c; a.N_cap = N_cap; a.k = 0; a.m_prime = m_prime;
+    a.dense = 1;
+    const int st = window_args(a, win, t, n_win, win_cap, dtype);
+    if (st != CSA_OK) return st;
+    return attn_run(a, scale, out, lse, workspace, ws_bytes, dtype, out_bf16, N_cap + n_win,
                     reinterpret_cast<cudaStream_t>(stream));
 }

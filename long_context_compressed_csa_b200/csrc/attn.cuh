@@ -20,6 +20,11 @@ struct AttnArgs {
     int64_t N_cap;
     int k, m_prime;
     int dense;
+    // sliding-window branch (win == null: none): window entries of tokens
+    // max(0, t - n_win + 1) .. t (t from the array t above, also for the sparse path),
+    // token p at row p % win_cap of win [B][win_cap][c]
+    const void* win;
+    int n_win, win_cap;
     float scale_log2;     // softmax scale * log2(e)
     int splits;
     int64_t per_split;    // list positions per split

@@ -229,25 +229,45 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
 
     // only shared memory and TMEM were touched so far (overlaps the previous kernel)
     pdl_wait();
-    int64_t count;
+    // list positions: [0, ncomp) compressed entries, then [ncomp, count) the sliding-window
+    // entries of tokens wlo .. t (when a window is given)
+    int64_t ncomp;
     if (a.dense) {
         const int64_t tt = a.t[g];
         const int64_t v = tt < 0 ? 0 : tt / a.m_prime;
-        count = v < a.N_cap ? v : a.N_cap;
+        ncomp = v < a.N_cap ? v : a.N_cap;
     } else {
-        count = a.k;
+        ncomp = a.k;
     }
+    int64_t nwin = 0;
+    int wrow0 = 0;  // ring row of the window's first token
+    if (a.win) {
+        const int64_t tt = a.t[g];
+        if (tt >= 0) {
+            nwin = tt + 1 < a.n_win ? tt + 1 : a.n_win;
+            wrow0 = (int)((tt - nwin + 1) % a.win_cap);
+        }
+    }
+    const int64_t count = ncomp + nwin;
     const int64_t p_begin = (int64_t)split * a.per_split;
     const int64_t p_end = min(count, p_begin + a.per_split);
     const int nchunks = p_end > p_begin ? (int)((p_end - p_begin + kE - 1) / kE) : 0;
     const size_t prow = ((size_t)g * a.splits + split) * kHeads;  // partial row of head 0
     const __nv_bfloat16* cache = static_cast<const __nv_bfloat16*>(a.cache) + b * a.N_cap * kC + half * kHalf;
+    const __nv_bfloat16* wcache =
+        a.win ? static_cast<const __nv_bfloat16*>(a.win) + b * (int64_t)a.win_cap * kC + half * kHalf : cache;
 
-    // entry id of list position p (-1: padding or outside the cache).  Sparse ranges of
-    // up to kMaxIds positions are staged in shared memory once by the loaders.
+    // Code of list position p: e >= 0 compressed entry e, e <= -2 window row -2 - e, -1
+    // padding or outside the cache.  Sparse ranges of up to kMaxIds positions are staged in
+    // shared memory once by the loaders.
     const bool ids_staged = !a.dense && (p_end - p_begin) <= kMaxIds;
     auto entry_global = [&](int64_t p) -> int64_t {
         if (p >= p_end) return -1;
+        if (p >= ncomp) {  // window position: at most one wrap of the ring (n_win <= win_cap)
+            int r = wrow0 + (int)(p - ncomp);
+            r = r >= a.win_cap ? r - a.win_cap : r;
+            return -2 - (int64_t)r;
+        }
         if (a.dense) return p;
         const int32_t v = __ldg(&a.idx[(int64_t)g * a.k + p]);
         return (v >= 0 && v < a.N_cap) ? v : -1;
@@ -255,6 +275,11 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
     auto entry_of = [&](int64_t p) -> int64_t {
         if (ids_staged) return p < p_end ? (int64_t)s_ids[p - p_begin] : -1;
         return entry_global(p);
+    };
+    const bool plain = a.dense && !a.win;  // position p is entry p
+    // first element of this CTA's half of the row a code names (any valid row for -1)
+    auto row_of = [&](int64_t e) -> const __nv_bfloat16* {
+        return e >= 0 ? cache + e * kC : (e <= -2 ? wcache + (-2 - e) * kC : cache);
     };
 
     if (nchunks == 0) {
@@ -286,12 +311,22 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
             }
             const uint32_t c0 = tc::smem_u32(sC0 + buf * kCBytes);
             const int64_t p0 = p_begin + (int64_t)j * kE;
+            if (plain) {  // dense without a window: position p is entry p
 #pragma unroll 4
-            for (int i = lt; i < kE * (kHalf / 8); i += kLoaders) {
-                const int row = i >> 5, cc = i & 31;
-                const int64_t e = entry_of(p0 + row);
-                const __nv_bfloat16* src = cache + (e >= 0 ? e : 0) * kC + cc * 8;
-                cp_async16(c0 + (cc >> 3) * (kE * 128) + tc::sw128_offset(row, cc & 7), src, e >= 0);
+                for (int i = lt; i < kE * (kHalf / 8); i += kLoaders) {
+                    const int row = i >> 5, cc = i & 31;
+                    const int64_t p = p0 + row;
+                    cp_async16(c0 + (cc >> 3) * (kE * 128) + tc::sw128_offset(row, cc & 7),
+                               cache + (p < p_end ? p : 0) * kC + cc * 8, p < p_end);
+                }
+            } else {
+#pragma unroll 4
+                for (int i = lt; i < kE * (kHalf / 8); i += kLoaders) {
+                    const int row = i >> 5, cc = i & 31;
+                    const int64_t e = entry_of(p0 + row);
+                    cp_async16(c0 + (cc >> 3) * (kE * 128) + tc::sw128_offset(row, cc & 7), row_of(e) + cc * 8,
+                               e != -1);
+                }
             }
             cp_async_commit();
             if (j == 0 && nchunks > 1) continue;  // issue chunk 1 before waiting for chunk 0
@@ -392,8 +427,9 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
             }
             mbar_arrive_remote(peer_addr(tc::smem_u32(Rfree), peer));  // our receive buffer is free again
             const int64_t p0 = p_begin + (int64_t)j * kE;
-            const unsigned vlo = __ballot_sync(0xffffffffu, entry_of(p0 + lane) >= 0);
-            const unsigned vhi = __ballot_sync(0xffffffffu, entry_of(p0 + 32 + lane) >= 0);
+            const unsigned vlo = __ballot_sync(0xffffffffu, plain ? p0 + lane < p_end : entry_of(p0 + lane) != -1);
+            const unsigned vhi =
+                __ballot_sync(0xffffffffu, plain ? p0 + 32 + lane < p_end : entry_of(p0 + 32 + lane) != -1);
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // 4 chains, not 1
 #pragma unroll
             for (int e = 0; e < kE; ++e) {
@@ -560,7 +596,7 @@ AttnPlan attn_plan_tc(int G, int n_h, int c, int64_t entries)
 
 int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cudaStream_t stream)
 {
-    if (!aligned16(a.q) || !aligned16(a.cache)) return CSA_ERR_ALIGN;
+    if (!aligned16(a.q) || !aligned16(a.cache) || (a.win && !aligned16(a.win))) return CSA_ERR_ALIGN;
     cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
     cudaLaunchConfig_t cfg{};

@@ -96,6 +96,15 @@ def test_host_validation_rejects_bad_arguments_without_launching(lib):
                               8, 0, 0, None) == -4
     assert lib.hca_dense_attn(fake, fake, fake, 1, 1, 4, 64, 100, 0, 0.0, fake, None, fake,
                               1 << 30, 0, 0, None) == -1
+    # sliding window: n_win < 1, ring smaller than the window, no window buffer, misaligned t
+    assert lib.csa_sparse_attn_window(fake, fake, fake, fake, fake, 1, 1, 4, 64, 100, 8, 0, 16, 0.0,
+                                      fake, None, fake, 1 << 30, 0, 0, None) == -1
+    assert lib.csa_sparse_attn_window(fake, fake, fake, fake, fake, 1, 1, 4, 64, 100, 8, 32, 16, 0.0,
+                                      fake, None, fake, 1 << 30, 0, 0, None) == -1
+    assert lib.hca_dense_attn_window(fake, fake, fake, None, 1, 1, 4, 64, 100, 128, 8, 16, 0.0,
+                                     fake, None, fake, 1 << 30, 0, 0, None) == -1
+    assert lib.hca_dense_attn_window(fake, fake, vp(0x10004), fake, 1, 1, 4, 64, 100, 128, 8, 16, 0.0,
+                                     fake, None, fake, 1 << 30, 0, 0, None) == -2
     # empty problems succeed without touching memory
     assert lib.csa_compress(fake, fake, fake, fake, 8, 64, 0, 8, None, None, fake, 64, 0, 8, 4,
                             0, 2, 0, None) == 0

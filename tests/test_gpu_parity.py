@@ -405,6 +405,53 @@ def test_attn_many_queries_and_workspace_reuse():
         np.testing.assert_allclose(lsed.cpu().numpy()[0, 0], ref_lse, atol=2e-3, rtol=0)
 
 
+@pytest.mark.parametrize("dtype,n_h,c", [(torch.bfloat16, 128, 512), (torch.float32, 16, 64)])
+def test_sparse_and_dense_attn_with_window(dtype, n_h, c):
+    """Sliding-window branch: the window entries of tokens max(0, t-n_win+1) .. t, read
+    from a ring buffer (token p at row p % win_cap), join the softmax of the selected
+    (sparse) or visible (dense) compressed entries."""
+    B, nq, N_cap, k, mp, n_win, win_cap = 2, 2, 3000, 256, 16, 128, 160
+    q = randn((B, nq, n_h, c), 340, dtype)
+    cache = randn((B, N_cap, c), 341, dtype)
+    win = randn((B, win_cap, c), 342, dtype)
+    g = torch.Generator().manual_seed(343)
+    idx = torch.stack([torch.randperm(N_cap, generator=g)[:k] for _ in range(B * nq)]).to(torch.int32)
+    idx[1, :k] = -1                                       # only window entries for this query
+    idx[2, 100:] = -1
+    tpos = [1000, 40, 0, mp * N_cap + 7]                  # wrapped ring, partial window, t = 0, all visible
+    tt = torch.tensor(tpos, dtype=torch.int64, device=DEV).reshape(B, nq)
+    qd, cd, wd = dev(q), dev(cache), dev(win)
+    # sparse
+    ws = torch.zeros(csa_attn_workspace_size(B, nq, n_h, c, k + n_win), dtype=torch.uint8, device=DEV)
+    out = torch.full((B, nq, n_h, c), float("nan"), dtype=torch.float32, device=DEV)
+    lse = torch.full((B, nq, n_h), float("nan"), device=DEV)
+    csa_sparse_attn(qd, cd, dev(idx.reshape(B, nq, k)), out, ws, lse=lse, win=wd, t=tt, n_win=n_win)
+    torch.cuda.synchronize()
+    assert csa_workspace_status(ws) == 0
+    o, l = out.cpu().numpy(), lse.cpu().numpy()
+    for gq in range(B * nq):
+        b, j = divmod(gq, nq)
+        rows = to_f64(win[b])[oracle.window_positions(tpos[gq], n_win) % win_cap]
+        ref, ref_lse = oracle.mqa_window(to_f64(q[b, j]), to_f64(cache[b]), idx[gq].numpy(), rows)
+        assert max_rel_rowwise(o[b, j], ref).max() <= TOL[dtype]
+        np.testing.assert_allclose(l[b, j], ref_lse, atol=2e-3 if dtype == torch.bfloat16 else 1e-5, rtol=0)
+    # dense
+    ws2 = torch.zeros(csa_attn_workspace_size(B, nq, n_h, c, N_cap + n_win), dtype=torch.uint8, device=DEV)
+    out2 = torch.full((B, nq, n_h, c), float("nan"), dtype=torch.float32, device=DEV)
+    lse2 = torch.full((B, nq, n_h), float("nan"), device=DEV)
+    hca_dense_attn(qd, cd, tt, mp, out2, ws2, lse=lse2, win=wd, n_win=n_win)
+    torch.cuda.synchronize()
+    assert csa_workspace_status(ws2) == 0
+    o2, l2 = out2.cpu().numpy(), lse2.cpu().numpy()
+    for gq in range(B * nq):
+        b, j = divmod(gq, nq)
+        vis = oracle.visible(tpos[gq], mp, N_cap)
+        rows = to_f64(win[b])[oracle.window_positions(tpos[gq], n_win) % win_cap]
+        ref, ref_lse = oracle.mqa_window(to_f64(q[b, j]), to_f64(cache[b]), np.arange(vis, dtype=np.int32), rows)
+        assert max_rel_rowwise(o2[b, j], ref).max() <= TOL[dtype]
+        np.testing.assert_allclose(l2[b, j], ref_lse, atol=2e-3 if dtype == torch.bfloat16 else 1e-5, rtol=0)
+
+
 # ==================================================================================
 # end to end: streams -> caches -> indexer/top-k -> sparse attention; HCA likewise
 # ==================================================================================
