@@ -302,6 +302,27 @@ def micro(kind, iters, rotate=4):
         ws = torch.zeros(lib.csa_attn_workspace_size(1, 1, n_h, c, k), dtype=torch.uint8, device=dev)
         calls = [lambda r=r: lib.csa_sparse_attn(q, caches[r], idx, o, ws) for r in range(rotate)]
         nbytes = k * c * 2
+    elif kind in ("sparse_window", "dense_window"):
+        # the same calls with the sliding-window branch: 128 raw-token entries from a ring
+        # buffer join the softmax (V4-Pro window size)
+        n_win, win_cap = 128, 256
+        wins = [randn((1, win_cap, c), 915 + r, bf16, dev) for r in range(rotate)]
+        q = randn((1, 1, n_h, c), 920, bf16, dev)
+        o = torch.empty((1, 1, n_h, c), dtype=torch.float32, device=dev)
+        if kind == "sparse_window":
+            caches = [randn((1, N, c), 910 + r, bf16, dev) for r in range(rotate)]
+            g = torch.Generator(device="cpu").manual_seed(921)
+            idx = torch.randperm(N, generator=g)[:k].to(torch.int32).reshape(1, 1, k).to(dev)
+            ws = torch.zeros(lib.csa_attn_workspace_size(1, 1, n_h, c, k + n_win), dtype=torch.uint8, device=dev)
+            calls = [lambda r=r: lib.csa_sparse_attn(q, caches[r], idx, o, ws, win=wins[r], t=t, n_win=n_win)
+                     for r in range(rotate)]
+            nbytes = (k + n_win) * c * 2
+        else:
+            caches = [randn((1, Nh, c), 930 + r, bf16, dev) for r in range(rotate * 4)]
+            ws = torch.zeros(lib.csa_attn_workspace_size(1, 1, n_h, c, Nh + n_win), dtype=torch.uint8, device=dev)
+            calls = [lambda r=r: lib.hca_dense_attn(q, caches[r], t, mp, o, ws, win=wins[r % rotate], n_win=n_win)
+                     for r in range(rotate * 4)]
+            nbytes = (Nh + n_win) * c * 2
     elif kind == "dense":
         caches = [randn((1, Nh, c), 930 + r, bf16, dev) for r in range(rotate * 4)]
         q = randn((1, 1, n_h, c), 940, bf16, dev)
@@ -360,7 +381,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--micro", default=None,
-                    help="time one entry point alone: indexer, sparse, dense, csa_compress, hca_compress")
+                    help="time one entry point alone: indexer, sparse, dense, sparse_window, "
+                         "dense_window, csa_compress, hca_compress")
     ap.add_argument("--iters", type=int, default=20)
     args = ap.parse_args()
     if args.micro:
