@@ -164,7 +164,8 @@ CSA_DEV void stage_o_cols(uint8_t* stage, uint32_t o_taddr, int h, int col0, flo
 CSA_DEV int rswz(int h, int q) { return h * 16 + (q ^ (h & 15)); }
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_t* status)
+attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_q,
+                 const __grid_constant__ CUtensorMap tmap_c, AttnArgs a, uint32_t* status)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -187,7 +188,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
     uint64_t* idsready = bars + 14; // loaders -> softmax            (count 128)
     uint64_t* staged = bars + 15;   // output half staged            (count 256: loaders + softmax)
     uint64_t* Ofinal = bars + 16;   // softmax -> loaders: last P C done (count 128)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+    uint64_t* Qfull = bars + 17;    // q half landed (TMA, count 1 + bytes)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
     volatile uint32_t* abort_flag = tmem_slot + 1;
     int* s_ids = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);  // [kMaxIds]
     float* s_inv_l = reinterpret_cast<float*>(sP);  // [128] 1 / l per head, after the last P C
@@ -215,6 +217,9 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
         tc::mbar_init(idsready, kLoaders);
         tc::mbar_init(staged, 2 * kHeads);
         tc::mbar_init(Ofinal, kHeads);
+        tc::mbar_init(Qfull, 1);
+        tc::tma_prefetch_desc(&tmap_q);
+        tc::tma_prefetch_desc(&tmap_c);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -288,11 +293,11 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
     } else if (warp < 4) {
         // ------------------------------------------------------------ loaders
         const int lt = threadIdx.x;
-        const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) + (int64_t)g * kHeads * kC + half * kHalf;
-        const uint32_t q0 = tc::smem_u32(sQ);
-        for (int i = lt; i < kHeads * (kHalf / 8); i += kLoaders) {
-            const int row = i >> 5, cc = i & 31;
-            cp_async16(q0 + (cc >> 3) * (kHeads * 128) + tc::sw128_offset(row, cc & 7), qg + row * kC + cc * 8, true);
+        if (lt == 0) {  // q half: four 128-row x 64-column TMA boxes (128-byte swizzle)
+            tc::mbar_arrive_expect_tx(Qfull, kQBytes);
+#pragma unroll
+            for (int p = 0; p < kHalf / 64; ++p)
+                tc::tma_load_2d(sQ + p * (kHeads * 128), &tmap_q, Qfull, half * kHalf + p * 64, g * kHeads);
         }
         if (ids_staged)
             for (int64_t i = lt; i < p_end - p_begin; i += kLoaders) s_ids[i] = (int)entry_global(p_begin + i);
@@ -312,6 +317,21 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
             const uint32_t c0 = tc::smem_u32(sC0 + buf * kCBytes);
             const int64_t p0 = p_begin + (int64_t)j * kE;
             if (plain) {  // dense without a window: position p is entry p
+                if (p0 + kE <= p_end) {
+                    // a full chunk is one contiguous block of cache rows: four 64 x 64 TMA
+                    // boxes, counted in bytes on Cfull (the other loaders just arrive)
+                    if (lt == 0) {
+                        tc::mbar_arrive_expect_tx(&Cfull[buf], kCBytes);
+#pragma unroll
+                        for (int p = 0; p < kHalf / 64; ++p)
+                            tc::tma_load_2d(sC0 + buf * kCBytes + p * (kE * 128), &tmap_c, &Cfull[buf],
+                                            half * kHalf + p * 64, (int)(b * a.N_cap + p0));
+                    } else {
+                        tc::mbar_arrive(&Cfull[buf]);
+                    }
+                    continue;
+                }
+                // the last, partial chunk: rows past the end are zero-filled by cp.async
 #pragma unroll 4
                 for (int i = lt; i < kE * (kHalf / 8); i += kLoaders) {
                     const int row = i >> 5, cc = i & 31;
@@ -319,6 +339,10 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
                     cp_async16(c0 + (cc >> 3) * (kE * 128) + tc::sw128_offset(row, cc & 7),
                                cache + (p < p_end ? p : 0) * kC + cc * 8, p < p_end);
                 }
+                cp_async_wait_all();
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(&Cfull[buf]);
+                continue;
             } else {
 #pragma unroll 4
                 for (int i = lt; i < kE * (kHalf / 8); i += kLoaders) {
@@ -331,7 +355,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
             cp_async_commit();
             if (j == 0 && nchunks > 1) continue;  // issue chunk 1 before waiting for chunk 0
             if (j == 1) {
-                cp_async_wait_prev();  // chunk 0 (with q) has landed; chunk 1 may be in flight
+                cp_async_wait_prev();  // chunk 0 has landed; chunk 1 may be in flight
                 tc::fence_proxy_async_smem();
                 tc::mbar_arrive(&Cfull[0]);
             }
@@ -340,6 +364,10 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
             tc::mbar_arrive(&Cfull[buf]);
         }
         cp_async_wait_all();
+        // q has landed before the CTA may move on (its barrier is used once).  The TMA
+        // chunks were consumed by the MMA warp on the normal path; after an abort the
+        // bounded waits outlast any load in flight by many orders of magnitude.
+        if (lt == 0 && !tc::mbar_wait(Qfull, 0, tc::kWaitBudget)) *abort_flag = 1;
         // The output half leaves through TMA: these warps stage columns 0..127 and the
         // softmax warps 128..255 once the last P C has completed, then thread 0 stores the
         // eight 128 x 32 boxes.
@@ -535,7 +563,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnArgs a, uint32_
                 tc::mma_commit(&Sfull[buf]);
                 return true;
             };
-            bool ok = issue_S(0);
+            bool ok = tc::mbar_wait(Qfull, 0, tc::kWaitBudget) && issue_S(0);
             for (int j = 0; j < nchunks && ok; ++j) {
                 if (*abort_flag) break;
                 if (j + 1 < nchunks && !issue_S(j + 1)) {
@@ -616,7 +644,12 @@ int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cu
     CUtensorMap tmap_o;  // partial outputs [G * splits * 128 rows][512] bf16, 64 x 128 boxes
     const uint64_t rows = (uint64_t)a.B * a.nq * plan.splits * kHeads;
     if (!make_tmap_bf16_2d(&tmap_o, a.part_o, rows, kC, kC, kBoxCols, kHeads)) return CSA_ERR_CUDA;
-    cudaLaunchKernelEx(&cfg, attn_pair_kernel, tmap_o, a, status);
+    CUtensorMap tmap_q;  // queries [G * 128 rows][512] bf16, 64 x 128 boxes
+    if (!make_tmap_bf16_2d(&tmap_q, a.q, (uint64_t)a.B * a.nq * kHeads, kC, kC, 64, kHeads)) return CSA_ERR_CUDA;
+    CUtensorMap tmap_c;  // compressed cache [B * N_cap rows][512] bf16, 64 x 64 boxes (dense chunks)
+    if (!make_tmap_bf16_2d(&tmap_c, a.cache, (uint64_t)a.B * (uint64_t)(a.N_cap > 0 ? a.N_cap : 1), kC, kC, 64, kE))
+        return CSA_ERR_CUDA;
+    cudaLaunchKernelEx(&cfg, attn_pair_kernel, tmap_o, tmap_q, tmap_c, a, status);
     return launch_status();
 }
 
