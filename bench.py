@@ -38,7 +38,7 @@ N_PAIRS = 8
 # over 262144 keys, from one ncu capture of the current kernel (67.23 MB read, 0.71 MB
 # written; algorithmic 67.11 MB).  Must be retaken (or set to None) when the kernel changes.
 SCAN_TRAFFIC_BYTES = 67_940_608
-IDX_SAMPLE = 8  # the indexer call is timed by in-graph events on every 8th step
+IDX_SAMPLE = 8  # steps per CUDA graph; the indexer call of each graph's first step is timed
 
 
 def log(*a):
@@ -230,7 +230,7 @@ class HybridDecode:
 
 def kernel_launches_per_step(dec, j):
     tok = dec.n + j
-    n = 2 + 2 + 2  # indexer (scan + select), sparse attn (+combine), dense attn (+combine)
+    n = 1 + 2 + 2  # indexer (scan with the select in place), sparse attn (+combine), dense attn (+combine)
     if (tok + 1) % dec.m == 0:
         n += 2
     if (tok + 1) % dec.mp == 0:
@@ -422,25 +422,28 @@ def main():
     dec = HybridDecode(torch, W + K, seed=5000 + 17 * rank)
     stream = torch.cuda.current_stream()
 
-    # ---- capture one CUDA graph per step (every pointer and position is baked in).  On
-    # every IDX_SAMPLE-th step, event record nodes inside the graph bracket the indexer
-    # call to time it on the device; the other steps carry no event nodes, which would
-    # cut the programmatic overlap of the indexer with its neighbours. ----
-    def make_graph(j_step):
-        p, j = j_step % N_PAIRS, j_step // N_PAIRS
+    # ---- capture the steps in CUDA graphs of N_PAIRS consecutive steps (one token through
+    # the 8 layer pairs; every pointer and position is baked in), so the kernels of
+    # consecutive steps keep their programmatic overlap.  In the first step of each graph,
+    # event record nodes bracket the indexer call to time it on the device; the other
+    # steps carry no event nodes, which would cut that overlap. ----
+    def make_graph(s0, s1):
         g = torch.cuda.CUDAGraph()
-        ev = None
-        if j_step % IDX_SAMPLE == 0:
-            ev = (torch.cuda.Event(enable_timing=True, external=True),
-                  torch.cuda.Event(enable_timing=True, external=True))
+        ev = (torch.cuda.Event(enable_timing=True, external=True),
+              torch.cuda.Event(enable_timing=True, external=True))
         with torch.cuda.graph(g):
-            if ev:
-                ev[0].record()
-            dec.step(p, j, part=0)
-            if ev:
-                ev[1].record()
-            dec.step(p, j, part=1)
+            for s in range(s0, s1):
+                p, j = s % N_PAIRS, s // N_PAIRS
+                if s == s0:
+                    ev[0].record()
+                dec.step(p, j, part=0)
+                if s == s0:
+                    ev[1].record()
+                dec.step(p, j, part=1)
         return g, ev
+
+    def graph_ranges(lo, hi):
+        return [(s, min(s + IDX_SAMPLE, hi)) for s in range(lo, hi, IDX_SAMPLE)]
 
     # eager warm-up of every code path once (outside any graph), then build graphs
     for s in range(min(W, 8)):
@@ -449,12 +452,14 @@ def main():
     # re-run the prefill positions: eager steps above advanced nothing persistent except
     # the incremental entries they recomputed, which the graphs recompute identically.
     t0 = time.time()
-    graphs = [make_graph(s) for s in range(W + K)]
+    warm_graphs = [make_graph(a0, a1) for a0, a1 in graph_ranges(0, W)]
+    graphs = [make_graph(a0, a1) for a0, a1 in graph_ranges(W, W + K)]
     torch.cuda.synchronize()
-    log("captured %d step graphs in %.1f s" % (len(graphs), time.time() - t0))
+    log("captured %d graphs of up to %d steps in %.1f s" % (len(warm_graphs) + len(graphs), IDX_SAMPLE,
+                                                            time.time() - t0))
 
-    for s in range(W):
-        graphs[s][0].replay()
+    for g, _ in warm_graphs:
+        g.replay()
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
@@ -464,16 +469,15 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     start.record()
-    for s in range(W, W + K):
-        graphs[s][0].replay()
+    for g, _ in graphs:
+        g.replay()
     end.record()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
     ms = start.elapsed_time(end)
-    idx_ms = np.array([graphs[s][1][0].elapsed_time(graphs[s][1][1]) for s in range(W, W + K)
-                       if graphs[s][1] is not None])
+    idx_ms = np.array([ev[0].elapsed_time(ev[1]) for _, ev in graphs])
     t_max = torch.tensor([ms], dtype=torch.float64, device="cuda")
     if world > 1:
         dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
@@ -519,8 +523,8 @@ def main():
                      "algorithmic_bytes_per_launch": idx_bytes,
                      "avg_launch_us": idx_avg_s * 1e6,
                      "timed_launches": int(len(idx_ms)),
-                     "how": "in-graph event record nodes around the call on every %dth timed step"
-                            % IDX_SAMPLE},
+                     "how": "in-graph event record nodes around the call in the first step of "
+                            "each %d-step CUDA graph" % IDX_SAMPLE},
         "step_roofline": {"achieved": step_gbs, "peak": hbm, "unit": "GB/s", "frac": step_gbs / hbm,
                           "bytes_per_step": bytes_total / K},
         "gpu_launches": launches,
