@@ -189,6 +189,54 @@ def mqa_window(q, cache, sel, win_rows, scale=None):
     return mqa(q, keys, sel2, scale)
 
 
+# ----------------------------------------------------------------------------------
+# FP8 (E4M3) indexer keys and queries.  The pages run the indexer in FP4 ([P1] section 6.4:
+# scoring "performed in FP4 precision", viable because the scores are never
+# exponentiated) and note FP4 has the peak of FP8 on current hardware ([P1] section 12);
+# the block-scale format is not given.  The reading used: OCP E4M3 codes (1 sign, 4
+# exponent bits with bias 7, 3 mantissa bits, subnormals, largest finite 448, no
+# infinities) with one fp32 scale per row (per key, per query head) = max|x| / 448.
+# ----------------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def round_e4m3(x):
+    """Round fp32 values to the nearest E4M3 value, ties to even, saturating at +-448
+    (the format's definition; as float64)."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    a = np.abs(x)
+    # grid spacing at |x|: 2^(e - 3) for the binade [2^e, 2^(e+1)), e >= -6; 2^-9 below 2^-6
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)
+    step = np.exp2(e - 3.0)
+    r = np.round(a / step) * step          # np.round: half to even
+    r = np.minimum(r, E4M3_MAX)
+    return np.where(a > 0, np.copysign(r, x), 0.0 * x)
+
+
+def quantize_rows_e4m3(X):
+    """Per-row E4M3 quantisation: scale = max|x| / 448 in fp32, code = E4M3(x / scale) with
+    the division in fp32 (rows of zeros: scale 0, codes 0).  Returns (values of the codes
+    [rows, cols] float64, scales [rows] float64)."""
+    X = np.asarray(X, dtype=np.float32)
+    X2 = X.reshape(-1, X.shape[-1])
+    amax = np.max(np.abs(X2), axis=1).astype(np.float32)
+    scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = (X2 / safe[:, None]).astype(np.float32)
+    codes = np.where(scale[:, None] > 0, round_e4m3(q), 0.0)
+    return codes.reshape(X.shape), scale.astype(np.float64).reshape(X.shape[:-1])
+
+
+def index_scores_e4m3(qI, wI, KI, nvis=None):
+    """[P1] section 6.4 scores on E4M3 operands: q^I (per head) and K^I (per key) are
+    quantised by quantize_rows_e4m3 and the boxed formula is evaluated in fp64 on the
+    dequantised values (code x scale)."""
+    qc, qs = quantize_rows_e4m3(qI)
+    kc, ks = quantize_rows_e4m3(KI)
+    return index_scores(qc * qs[:, None], wI, kc * ks[:, None], nvis)
+
+
 def round_bf16(x):
     """Round float64/float32 values to the nearest bfloat16 (ties to even), as float64.
 

@@ -449,3 +449,72 @@ def test_window_mqa_invariants():
     # lse combines like a union: exp(lse) = exp(lse_comp) + exp(lse_win)
     lc = oracle.mqa(q, cache, sel)[1]
     np.testing.assert_allclose(np.exp(lse), np.exp(lc) + np.exp(lw2), rtol=1e-12)
+
+
+# ==================================================================================
+# FP8 (E4M3) indexer operands (reading of [P1] section 6.4 "FP4 indexer"; format chosen:
+# E4M3 codes with one fp32 scale per row)
+# ==================================================================================
+def _e4m3_table():
+    """Every finite E4M3 value, decoded from the 8-bit codes by the format definition
+    (sign, 4-bit exponent with bias 7, 3-bit mantissa, subnormals at exponent 0;
+    exponent 15 with mantissa 7 is NaN)."""
+    vals = []
+    for code in range(256):
+        s, e, m = code >> 7, (code >> 3) & 15, code & 7
+        if e == 15 and m == 7:
+            continue
+        v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7)
+        vals.append(-v if s else v)
+    return np.unique(np.array(vals))
+
+
+def test_e4m3_rounding_pins():
+    tab = _e4m3_table()
+    assert tab.max() == 448.0 and tab.min() == -448.0 and len(tab) == 253  # +-0 merge
+    # every representable value is a fixed point
+    np.testing.assert_array_equal(oracle.round_e4m3(tab.astype(np.float32)), tab)
+    # midpoints between neighbours round to the one with an even mantissa
+    pos = tab[tab >= 0]
+    mids = (pos[:-1] + pos[1:]) / 2
+    got = oracle.round_e4m3(mids.astype(np.float32))
+    for mid, g, a, b in zip(mids, got, pos[:-1], pos[1:]):
+        assert g in (a, b)
+        # the even neighbour: code mantissa bit 0 clear; on the grid, a/step even
+        e = max(np.floor(np.log2(a)) if a > 0 else -6, -6)
+        step = 2.0 ** (e - 3)
+        assert (g / step) % 2 == 0 or g == b == 2 ** (e + 1)
+    # saturation, sign symmetry, nearest rounding away from midpoints
+    np.testing.assert_array_equal(oracle.round_e4m3(np.float32([500.0, -1e6, 449.0])), [448, -448, 448])
+    rng = np.random.default_rng(3)
+    x = rng.uniform(-400, 400, 2000).astype(np.float32)
+    r = oracle.round_e4m3(x)
+    idx = np.abs(tab[None, :] - x[:, None].astype(np.float64)).argmin(axis=1)
+    dist_best = np.abs(tab[idx] - x)
+    np.testing.assert_array_equal(np.abs(r - x), dist_best)   # nearest (ties aside)
+    np.testing.assert_array_equal(oracle.round_e4m3(-x), -r)
+
+
+def test_e4m3_row_quantisation_and_scores():
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((50, 128)).astype(np.float32)
+    X[7] = 0.0
+    codes, scale = oracle.quantize_rows_e4m3(X)
+    assert scale[7] == 0 and np.all(codes[7] == 0)
+    amax = np.abs(X).max(axis=1)
+    np.testing.assert_array_equal(scale[:7], (amax[:7] / np.float32(448)).astype(np.float32))
+    # the largest entry of each row maps to +-448; every code is an E4M3 value
+    rows = np.arange(50) != 7
+    assert np.all(np.abs(codes[rows]).max(axis=1) == 448.0)
+    assert np.all(np.isin(codes, _e4m3_table()))
+    # relative error of E4M3 is at most 2^-4 of the value above the subnormal range
+    deq = codes * scale[:, None]
+    big = np.abs(X) >= 2.0 ** -6 * scale[:, None]
+    assert np.all(np.abs(deq - X)[big] <= 2.0 ** -4 * np.abs(X)[big] + 1e-30)
+    # scores on E4M3 operands stay within the operand error of the exact scores
+    qI, wI, KI = rng.standard_normal((16, 128)), rng.standard_normal(16), rng.standard_normal((300, 128))
+    s8 = oracle.index_scores_e4m3(qI, wI, KI)
+    s = oracle.index_scores(qI, wI, KI)
+    bound = np.abs(wI) @ (np.abs(qI) @ np.abs(KI).T) * (2 * 2.0 ** -4 + 2.0 ** -8) + 1e-9
+    assert np.all(np.abs(s8 - s) <= bound)
+    assert np.corrcoef(s8, s)[0, 1] > 0.99
