@@ -198,6 +198,42 @@ int hca_dense_attn(const void* q, const void* cache, const int64_t* t,
                    int dtype, int out_bf16, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * csa_quantize_e4m3 - per-row E4M3 (FP8) quantisation of indexer keys (or any rows).
+ *   Source: [P1] section 6.4 runs the indexer in FP4, which is viable because the scores
+ *   are never exponentiated; [P1] section 12 notes FP4 has the peak of FP8 on current
+ *   hardware.  The pages give no block-scale format.  The reading used: OCP E4M3 codes
+ *   (largest finite 448) with one fp32 scale per row, scale = max|x| / 448 (0 for an
+ *   all-zero row); code = E4M3(x / scale), the division in fp32, rounded to nearest even
+ *   and saturated.
+ * x      : [rows, cols] (dtype bf16 or fp32) with row stride ld (elements), cols % 4 == 0
+ * codes  : [rows, cols] E4M3 bytes, contiguous (4-byte aligned)
+ * scales : fp32 [rows]
+ * Quantising new compressed entries as they are appended keeps an E4M3 key cache in step.
+ * ------------------------------------------------------------------------------- */
+int csa_quantize_e4m3(const void* x, int64_t rows, int cols, int64_t ld, void* codes,
+                      float* scales, int dtype, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * csa_indexer_topk_e4m3 - csa_indexer_topk on E4M3 keys: the [P1] section 6.4 scores of
+ * the dequantised operands, then the same top-k (section 7).  q^I (bf16) is quantised per
+ * head inside the kernel with the csa_quantize_e4m3 rule; the products run on the tensor
+ * cores (E4M3 x E4M3 -> fp32), and the score is
+ *   KI_scale[s] * sum_h (w_h * scale_h) * ReLU(q8_h . K8_s),
+ * which equals the boxed formula on the dequantised values since the scales are >= 0.
+ * KI8      : [B, N_cap, cI] E4M3 codes (16-byte aligned), KI_scale: fp32 [B, N_cap]
+ * qI       : [B, nq, n_hI, cI] bf16 (16-byte aligned); other arguments, the workspace
+ *            (csa_indexer_topk_workspace_size) and the outputs as for csa_indexer_topk.
+ * Supported: n_hI in {16, 32, 64, 128}, cI in {128, 256}; CSA_ERR_UNSUPPORTED otherwise.
+ * Keys take 1 byte instead of 2: the scan of the 1M-token decode reads 34.6 MB instead of
+ * 67.1 MB.
+ * ------------------------------------------------------------------------------- */
+int csa_indexer_topk_e4m3(const void* qI, const float* wI, const void* KI8,
+                          const float* KI_scale, const int64_t* t, int B, int nq,
+                          int64_t N_cap, int n_hI, int cI, int m, int k, int32_t* idx_out,
+                          float* scores_out, void* workspace, size_t ws_bytes,
+                          csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * csa_sparse_attn_window, hca_dense_attn_window - csa_sparse_attn / hca_dense_attn with the
  * sliding-window branch.  The query at position t also attends, under the same softmax,
  * to the window key/value entries of the raw tokens max(0, t - n_win + 1) .. t, the

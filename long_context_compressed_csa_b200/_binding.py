@@ -33,6 +33,8 @@ _SIGS = {
                         i32),
     "hca_dense_attn": ([vp, vp, vp, i32, i32, i32, i32, i64, i32, f32, vp, vp, vp, sz, i32, i32, vp],
                        i32),
+    "csa_quantize_e4m3": ([vp, i64, i32, i64, vp, vp, i32, vp], i32),
+    "csa_indexer_topk_e4m3": ([vp, vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, i32, vp, vp, vp, sz, vp], i32),
     "csa_sparse_attn_window": ([vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i32, i32, i64, f32, vp, vp,
                                 vp, sz, i32, i32, vp], i32),
     "hca_dense_attn_window": ([vp, vp, vp, vp, i32, i32, i32, i32, i64, i32, i32, i64, f32, vp, vp, vp,
@@ -187,6 +189,30 @@ def csa_workspace_status(workspace, stream=None) -> int:
 
 def csa_attn_workspace_size(B, nq, n_h, c, max_entries) -> int:
     return int(library().csa_attn_workspace_size(B, nq, n_h, c, max_entries))
+
+
+def csa_quantize_e4m3(x, codes, scales, stream=None):
+    """Per-row E4M3 codes (uint8 tensor, same shape as x) and fp32 scales (x.shape[:-1]) of
+    x [..., cols] (bf16 or fp32, rows contiguous)."""
+    _cuda(x, codes, scales)
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols else 0
+    assert x.is_contiguous() and codes.is_contiguous() and scales.is_contiguous()
+    assert codes.shape == x.shape and codes.element_size() == 1 and scales.numel() == rows
+    _check("csa_quantize_e4m3", library().csa_quantize_e4m3(
+        _ptr(x), rows, cols, cols, _ptr(codes), _ptr(scales), _dtype(x), _stream(stream)))
+
+
+def csa_indexer_topk_e4m3(qI, wI, KI8, KI_scale, t, m, k, idx_out, workspace, scores_out=None, stream=None):
+    """csa_indexer_topk on E4M3 keys KI8 [B,N_cap,cI] (uint8) with scales [B,N_cap]; qI bf16."""
+    _cuda(qI, wI, KI8, KI_scale, t, idx_out, workspace, scores_out)
+    B, nq, n_hI, cI = qI.shape
+    N_cap = KI8.shape[1]
+    assert qI.is_contiguous() and KI8.is_contiguous() and KI_scale.is_contiguous()
+    assert KI8.shape == (B, N_cap, cI) and KI_scale.shape == (B, N_cap) and idx_out.shape == (B, nq, k)
+    _check("csa_indexer_topk_e4m3", library().csa_indexer_topk_e4m3(
+        _ptr(qI), _ptr(wI), _ptr(KI8), _ptr(KI_scale), _ptr(t), B, nq, N_cap, n_hI, cI, m, k, _ptr(idx_out),
+        _ptr(scores_out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def csa_sparse_attn(q, cache, idx, out, workspace, lse=None, scale=0.0, stream=None,

@@ -33,6 +33,12 @@ bool indexer_tc_supported(int n_hI, int cI);
 int launch_scan_tc(const void* qI, const float* wI, const void* KI, const int64_t* t, int B,
                    int nq, int64_t N_cap, int n_hI, int cI, int m, int k, const TopkWs& ws,
                    int32_t* idx_out, float* scores_out, bool* fused, cudaStream_t stream);
+// E4M3 keys (k_scale: one fp32 scale per key) with bf16 queries quantised per head.
+bool indexer_e4m3_supported(int n_hI, int cI);
+int launch_scan_tc_e4m3(const void* qI, const float* wI, const void* KI8, const float* k_scale,
+                        const int64_t* t, int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
+                        const TopkWs& ws, int32_t* idx_out, float* scores_out, bool* fused,
+                        cudaStream_t stream);
 int launch_scan_cuda_core(const void* qI, const float* wI, const void* KI, const int64_t* t,
                           int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
                           const TopkWs& ws, int dtype, cudaStream_t stream);

@@ -20,6 +20,7 @@
 // walks a strided set of key tiles of one query.  Every barrier wait is bounded; a
 // timeout sets the workspace status word and every role drains and exits.
 #include "indexer.cuh"
+#include "e4m3.cuh"
 #include "select.cuh"
 #include "tc_utils.cuh"
 
@@ -29,11 +30,13 @@ namespace {
 constexpr int kTcThreads = 320;  // producer, MMA, two groups of 4 epilogue warps
 constexpr int kTileKeys = 128;
 
-template <int NH, int CI>
+// KB: bytes per key / query element (2: bf16, 1: E4M3)
+template <int NH, int CI, int KB = 2>
 struct ScanCfg {
-    static constexpr int kPanels = CI / 64;
-    static constexpr int kAStage = kTileKeys * CI * 2;      // bytes of one key tile
-    static constexpr int kBBytes = NH * CI * 2;             // q^I tile
+    static constexpr int kPanels = CI * KB / 128;          // 128-byte column panels of a tile
+    static constexpr int kPanelElems = 128 / KB;             // elements per panel row
+    static constexpr int kAStage = kTileKeys * CI * KB;     // bytes of one key tile
+    static constexpr int kBBytes = NH * CI * KB;            // q^I tile
     static constexpr int kBudget = 220 * 1024;
     static constexpr int kFixed0 = 1024 + kBBytes + NH * 4 + kBins * 4 + 256;
     // scores of the CTA's first kCacheTiles tiles stay in shared memory for the in-place
@@ -89,13 +92,17 @@ struct SelOut {
     int fused;
 };
 
-template <int NH, int CI>
+// KB = 2: bf16 keys and queries (kind::f16).  KB = 1: E4M3 keys with one fp32 scale per
+// key (k_scale), bf16 queries quantised here per head to E4M3 (kind::f8f6f4); the score
+// is then k_scale[s] * sum_h (w_h * q_scale_h) ReLU(q8_h . k8_s), which equals the boxed
+// formula on the dequantised operands because the scales are non-negative.
+template <int NH, int CI, int KB>
 __global__ void __launch_bounds__(kTcThreads, 1)
 scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __restrict__ qI,
-               const float* __restrict__ wI, const int64_t* __restrict__ t, int nq, int64_t N_cap,
-               int m, int k, TopkWs ws, SelOut so)
+               const float* __restrict__ wI, const float* __restrict__ k_scale,
+               const int64_t* __restrict__ t, int nq, int64_t N_cap, int m, int k, TopkWs ws, SelOut so)
 {
-    using Cfg = ScanCfg<NH, CI>;
+    using Cfg = ScanCfg<NH, CI, KB>;
     constexpr int S = Cfg::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -168,7 +175,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
                 const int row0 = (int)(b * N_cap) + tile * kTileKeys;
 #pragma unroll
                 for (int p = 0; p < Cfg::kPanels; ++p)
-                    tc::tma_load_2d(sA + s * Cfg::kAStage + p * (kTileKeys * 128), &tmap, &full[s], 64 * p, row0);
+                    tc::tma_load_2d(sA + s * Cfg::kAStage + p * (kTileKeys * 128), &tmap, &full[s],
+                                    Cfg::kPanelElems * p, row0);
             }
             // drain: every issued load has landed before the CTA may exit
             for (int j = it - S < 0 ? 0 : it - S; j < it; ++j)
@@ -177,7 +185,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, NH, false, false);
+            constexpr uint32_t kIdesc = KB == 2 ? tc::idesc_bf16_f32(128, NH, false, false)
+                                                : tc::idesc_e4m3_f32(128, NH);
             if (!tc::mbar_wait(qready, 0, tc::kWaitBudget)) *abort_flag = 1;
             int it = 0;
             for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
@@ -201,7 +210,10 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t ad = tc::smem_desc_sw128(a0 + p * (kTileKeys * 128) + kk * 32, 16, 1024);
                         const uint64_t bd = tc::smem_desc_sw128(b0 + p * (NH * 128) + kk * 32, 16, 1024);
-                        tc::mma_bf16_ss(d, ad, bd, kIdesc, (p | kk) ? 1u : 0u);
+                        if constexpr (KB == 2)
+                            tc::mma_bf16_ss(d, ad, bd, kIdesc, (p | kk) ? 1u : 0u);
+                        else
+                            tc::mma_e4m3_ss(d, ad, bd, kIdesc, (p | kk) ? 1u : 0u);
                     }
                 }
                 tc::mma_commit(&empty[s]);     // smem stage free once these MMAs finish
@@ -217,26 +229,55 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
         {
             const int et = threadIdx.x - 64;  // 0..255
             const __nv_bfloat16* qg = qI + (int64_t)g * NH * CI;
-            constexpr int kChunks = NH * CI / 8;  // 16-byte chunks
-            constexpr int kPer = (kChunks + 255) / 256;
-            uint4 v[kPer];
+            if constexpr (KB == 2) {
+                constexpr int kChunks = NH * CI / 8;  // 16-byte chunks
+                constexpr int kPer = (kChunks + 255) / 256;
+                uint4 v[kPer];
 #pragma unroll
-            for (int u = 0; u < kPer; ++u) {  // all loads first: one round trip
-                const int i = et + u * 256;
-                if (i < kChunks) {
-                    const int r = i / (CI / 8), cc = i % (CI / 8);
-                    v[u] = __ldg(reinterpret_cast<const uint4*>(qg + (int64_t)r * CI + cc * 8));
+                for (int u = 0; u < kPer; ++u) {  // all loads first: one round trip
+                    const int i = et + u * 256;
+                    if (i < kChunks) {
+                        const int r = i / (CI / 8), cc = i % (CI / 8);
+                        v[u] = __ldg(reinterpret_cast<const uint4*>(qg + (int64_t)r * CI + cc * 8));
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kPer; ++u) {
+                    const int i = et + u * 256;
+                    if (i < kChunks) {
+                        const int r = i / (CI / 8), cc = i % (CI / 8);
+                        *reinterpret_cast<uint4*>(sB + (cc / 8) * (NH * 128) + tc::sw128_offset(r, cc % 8)) = v[u];
+                    }
+                }
+                for (int i = et; i < NH; i += 256) sw[i] = wI[(int64_t)g * NH + i];
+            } else {
+                // one warp per head: E4M3 codes of q_h / scale_h, scale_h = max|q_h| / 448,
+                // and the head weight folded with the scale (w_h * scale_h)
+                constexpr int V = CI / 32;  // elements per lane (4 or 8)
+                const int ew = et >> 5, el = et & 31;
+                for (int h = ew; h < NH; h += 8) {
+                    float x[V];
+#pragma unroll
+                    for (int u = 0; u < V; ++u) x[u] = __bfloat162float(qg[(int64_t)h * CI + el * V + u]);
+                    float amax = 0.f;
+#pragma unroll
+                    for (int u = 0; u < V; ++u) amax = fmaxf(amax, fabsf(x[u]));
+#pragma unroll
+                    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                    const float sc = e4m3_scale(amax);
+                    uint32_t w[V / 4];
+#pragma unroll
+                    for (int u = 0; u < V; u += 4)
+                        w[u / 4] = e4m3x2(x[u], x[u + 1], sc) | (e4m3x2(x[u + 2], x[u + 3], sc) << 16);
+                    const int byte = el * V;  // column of the first code = byte in the row
+                    uint8_t* dst = sB + (byte / 128) * (NH * 128) + tc::sw128_offset(h, (byte % 128) / 16) + byte % 16;
+                    if constexpr (V == 4)
+                        *reinterpret_cast<uint32_t*>(dst) = w[0];
+                    else
+                        *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+                    if (el == 0) sw[h] = wI[(int64_t)g * NH + h] * sc;
                 }
             }
-#pragma unroll
-            for (int u = 0; u < kPer; ++u) {
-                const int i = et + u * 256;
-                if (i < kChunks) {
-                    const int r = i / (CI / 8), cc = i % (CI / 8);
-                    *reinterpret_cast<uint4*>(sB + (cc / 8) * (NH * 128) + tc::sw128_offset(r, cc % 8)) = v[u];
-                }
-            }
-            for (int i = et; i < NH; i += 256) sw[i] = wI[(int64_t)g * NH + i];
             if (need_hist)
                 for (int i = et; i < kBins; i += 256) sh[i] = 0;
             tc::fence_proxy_async_smem();
@@ -253,6 +294,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
         for (int tile = blockIdx.x + eg * gridDim.x; tile < ntiles; tile += 2 * gridDim.x, it += 2) {
             const int acc = it & 1;
             const uint32_t aph = (it >> 1) & 1;
+            const int64_t sidx = (int64_t)tile * kTileKeys + row;
+            float ksc = 1.f;  // E4M3 keys: the key's scale, fetched before the wait
+            if constexpr (KB == 1) ksc = sidx < vis ? __ldg(&k_scale[b * N_cap + sidx]) : 0.f;
             if (*abort_flag) break;
             if (!tc::mbar_wait(&tfull[acc], aph, tc::kWaitBudget)) {
                 *abort_flag = 1;
@@ -269,7 +313,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
             float sc = 0.f;
 #pragma unroll
             for (int h = 0; h < NH; ++h) sc = fmaf(sw[h], fmaxf(v[h], 0.f), sc);
-            const int64_t sidx = (int64_t)tile * kTileKeys + row;
+            if constexpr (KB == 1) sc *= ksc;
             if (sidx < vis) {
                 if (!so.fused) {
                     scores[sidx] = sc;
@@ -372,13 +416,13 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
     sel::reset_query(q, tid);
 }
 
-template <int NH, int CI>
-int launch_nh_ci(const CUtensorMap& tmap, const void* qI, const float* wI, const int64_t* t, int B, int nq,
-                 int64_t N_cap, int m, int k, const TopkWs& ws, int32_t* idx_out, float* scores_out,
-                 bool* fused, cudaStream_t stream)
+template <int NH, int CI, int KB>
+int launch_nh_ci(const CUtensorMap& tmap, const void* qI, const float* wI, const float* k_scale, const int64_t* t,
+                 int B, int nq, int64_t N_cap, int m, int k, const TopkWs& ws, int32_t* idx_out,
+                 float* scores_out, bool* fused, cudaStream_t stream)
 {
-    using Cfg = ScanCfg<NH, CI>;
-    auto kern = scan_tc_kernel<NH, CI>;
+    using Cfg = ScanCfg<NH, CI, KB>;
+    auto kern = scan_tc_kernel<NH, CI, KB>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
     const int G = B * nq;
     const int64_t tiles = (N_cap + kTileKeys - 1) / kTileKeys;
@@ -405,7 +449,7 @@ int launch_nh_ci(const CUtensorMap& tmap, const void* qI, const float* wI, const
     so.fused = *fused ? 1 : 0;
     dim3 grid((unsigned)ctas, (unsigned)G);
     launch_pdl(kern, grid, dim3(kTcThreads), Cfg::kSmem, stream, tmap, static_cast<const __nv_bfloat16*>(qI), wI,
-               t, nq, N_cap, m, k, ws, so);
+               k_scale, t, nq, N_cap, m, k, ws, so);
     return launch_status();
 }
 
@@ -427,12 +471,37 @@ int launch_scan_tc(const void* qI, const float* wI, const void* KI, const int64_
     CUtensorMap tmap;
     if (!make_tmap_bf16_2d(&tmap, KI, (uint64_t)B * N_cap, cI, cI, 64, kTileKeys)) return CSA_ERR_CUDA;
 #define CSA_SCAN_CASE(NH_, CI_) \
-    if (n_hI == NH_ && cI == CI_) return launch_nh_ci<NH_, CI_>(tmap, qI, wI, t, B, nq, N_cap, m, k, ws, idx_out, scores_out, fused, stream);
+    if (n_hI == NH_ && cI == CI_)   \
+        return launch_nh_ci<NH_, CI_, 2>(tmap, qI, wI, nullptr, t, B, nq, N_cap, m, k, ws, idx_out, scores_out, fused, stream);
     CSA_SCAN_CASE(16, 64) CSA_SCAN_CASE(16, 128) CSA_SCAN_CASE(16, 256)
     CSA_SCAN_CASE(32, 64) CSA_SCAN_CASE(32, 128) CSA_SCAN_CASE(32, 256)
     CSA_SCAN_CASE(64, 64) CSA_SCAN_CASE(64, 128) CSA_SCAN_CASE(64, 256)
     CSA_SCAN_CASE(128, 64) CSA_SCAN_CASE(128, 128) CSA_SCAN_CASE(128, 256)
 #undef CSA_SCAN_CASE
+    return CSA_ERR_UNSUPPORTED;
+}
+
+bool indexer_e4m3_supported(int n_hI, int cI)
+{
+    return (n_hI == 16 || n_hI == 32 || n_hI == 64 || n_hI == 128) && (cI == 128 || cI == 256);
+}
+
+int launch_scan_tc_e4m3(const void* qI, const float* wI, const void* KI8, const float* k_scale, const int64_t* t,
+                        int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k, const TopkWs& ws,
+                        int32_t* idx_out, float* scores_out, bool* fused, cudaStream_t stream)
+{
+    *fused = false;
+    if (N_cap == 0) return CSA_OK;
+    if ((int64_t)B * N_cap + kTileKeys >= (int64_t(1) << 31)) return CSA_ERR_UNSUPPORTED;
+    if (!aligned16(qI) || !aligned16(KI8)) return CSA_ERR_ALIGN;
+    CUtensorMap tmap;  // E4M3 keys [B * N_cap rows][cI bytes], 128 x 128 boxes
+    if (!make_tmap_u8_2d(&tmap, KI8, (uint64_t)B * N_cap, cI, cI, 128, kTileKeys)) return CSA_ERR_CUDA;
+#define CSA_SCAN8_CASE(NH_, CI_) \
+    if (n_hI == NH_ && cI == CI_)   \
+        return launch_nh_ci<NH_, CI_, 1>(tmap, qI, wI, k_scale, t, B, nq, N_cap, m, k, ws, idx_out, scores_out, fused, stream);
+    CSA_SCAN8_CASE(16, 128) CSA_SCAN8_CASE(16, 256) CSA_SCAN8_CASE(32, 128) CSA_SCAN8_CASE(32, 256)
+    CSA_SCAN8_CASE(64, 128) CSA_SCAN8_CASE(64, 256) CSA_SCAN8_CASE(128, 128) CSA_SCAN8_CASE(128, 256)
+#undef CSA_SCAN8_CASE
     return CSA_ERR_UNSUPPORTED;
 }
 

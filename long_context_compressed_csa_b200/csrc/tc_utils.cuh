@@ -110,6 +110,16 @@ CSA_DEV void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem]^T, E4M3 inputs (kind::f8f6f4), fp32 accumulate; one thread.
+CSA_DEV void mma_e4m3_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 // Arrive on `bar` once every tcgen05 operation this thread issued so far has completed.
 CSA_DEV void mma_commit(uint64_t* bar)
 {
@@ -178,6 +188,15 @@ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, bool b_mn)
            | ((uint32_t)(M >> 4) << 24);// M / 16
 }
 
+// Instruction descriptor of kind::f8f6f4 with E4M3 A and B (format code 0), fp32 D, dense,
+// both operands K-major.
+constexpr uint32_t idesc_e4m3_f32(int M, int N)
+{
+    return (1u << 4)                    // D format: f32
+           | ((uint32_t)(N >> 3) << 17) // N / 8
+           | ((uint32_t)(M >> 4) << 24);// M / 16  (A and B format fields 0: E4M3)
+}
+
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128-byte-swizzled
 // panel whose base is 1024-byte aligned (the TMA SWIZZLE_128B pattern).
 CSA_DEV uint32_t sw128_offset(uint32_t row, uint32_t chunk) { return row * 128u + ((chunk ^ (row & 7u)) << 4); }
@@ -190,6 +209,9 @@ constexpr long long kWaitBudget = 2000000000LL;  // ~1 s at 1.9 GHz
 // box of box_cols x box_rows and 128-byte swizzle; false if the driver call fails.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                        uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);
+// Same for a 2-D tensor of bytes (E4M3 codes).
+bool make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                     uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);
 // Same for a 2-D fp32 tensor.
 bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                       uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);

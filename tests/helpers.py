@@ -46,3 +46,13 @@ def check_topk_sets(got_idx, oracle_scores, k, band_fn, rel=1e-6):
         assert np.all(gap <= band), "top-k differs beyond near-ties: %s" % list(
             zip(diff, gap.tolist(), band.tolist()))
     return len(diff)
+
+
+def decode_e4m3(codes):
+    """Values of E4M3 byte codes (numpy uint8 array), decoded from the format definition:
+    sign, 4-bit exponent with bias 7, 3-bit mantissa, subnormals at exponent 0."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    s, e, m = c >> 7, (c >> 3) & 15, c & 7
+    v = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1 + m / 8.0) * 2.0 ** (e - 7.0))
+    assert not np.any((e == 15) & (m == 7)), "NaN code"
+    return np.where(s == 1, -v, v)

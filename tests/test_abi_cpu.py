@@ -105,6 +105,11 @@ def test_host_validation_rejects_bad_arguments_without_launching(lib):
                                      fake, None, fake, 1 << 30, 0, 0, None) == -1
     assert lib.hca_dense_attn_window(fake, fake, vp(0x10004), fake, 1, 1, 4, 64, 100, 128, 8, 16, 0.0,
                                      fake, None, fake, 1 << 30, 0, 0, None) == -2
+    # E4M3: cols not a multiple of 4, bad dtype; indexer with an unsupported cI
+    assert lib.csa_quantize_e4m3(fake, 10, 6, 6, fake, fake, 0, None) == -1
+    assert lib.csa_quantize_e4m3(fake, 10, 8, 8, fake, fake, 9, None) == -3
+    assert lib.csa_indexer_topk_e4m3(fake, fake, fake, fake, fake, 1, 1, 100, 64, 64, 4, 8, fake, None,
+                                     fake, 1 << 30, None) == -6
     # empty problems succeed without touching memory
     assert lib.csa_compress(fake, fake, fake, fake, 8, 64, 0, 8, None, None, fake, 64, 0, 8, 4,
                             0, 2, 0, None) == 0

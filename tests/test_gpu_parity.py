@@ -17,11 +17,12 @@ import torch
 
 import oracle
 from long_context_compressed_csa_b200 import (csa_attn_workspace_size, csa_compress,
+                                              csa_indexer_topk_e4m3, csa_quantize_e4m3,
                                               csa_indexer_topk, csa_indexer_topk_workspace_size,
                                               csa_sparse_attn, csa_workspace_status, hca_compress,
                                               hca_dense_attn)
 from long_context_compressed_csa_b200.synth import randint_values, randn, to_f64
-from tests.helpers import check_topk_sets, max_rel_rowwise, score_error_bound
+from tests.helpers import check_topk_sets, decode_e4m3, max_rel_rowwise, score_error_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -257,6 +258,64 @@ def test_indexer_topk_many_queries(B, nq, N_cap, k, seed):
     # the workspace is left clean for the next call
     idx2, _, _ = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k, ws=ws)
     assert np.array_equal(np.sort(idx2, axis=-1), np.sort(idx, axis=-1))
+
+
+@pytest.mark.parametrize("dtype,cols", [(torch.bfloat16, 128), (torch.float32, 256), (torch.bfloat16, 44)])
+def test_quantize_e4m3_matches_oracle_bit_exactly(dtype, cols):
+    """E4M3 codes and fp32 row scales equal the oracle's (both divide in fp32 and round to
+    nearest even), including an all-zero row and a row of large values."""
+    X = randn((301, cols), 350, dtype, scale=3.0)
+    X[5] = 0
+    X[9] = X[9] * 1e4
+    codes = torch.empty((301, cols), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((301,), dtype=torch.float32, device=DEV)
+    csa_quantize_e4m3(dev(X), codes, scales)
+    torch.cuda.synchronize()
+    want_v, want_s = oracle.quantize_rows_e4m3(X.float().numpy())
+    np.testing.assert_array_equal(scales.cpu().numpy().astype(np.float64), want_s)
+    np.testing.assert_array_equal(decode_e4m3(codes.cpu().numpy()), want_v)
+
+
+@pytest.mark.parametrize("n_hI,cI,N_cap,k", [(64, 128, 20000, 512), (32, 256, 3000, 1024), (16, 128, 700, 64)])
+def test_indexer_topk_e4m3(n_hI, cI, N_cap, k):
+    """Top-k over E4M3 keys and in-kernel E4M3 queries against the oracle's scores of the
+    same quantised operands (sets identical except for fp32 near-ties)."""
+    B, nq, m = 2, 2, 4
+    qI = randn((B, nq, n_hI, cI), 360, torch.bfloat16)
+    KI = randn((B, N_cap, cI), 361, torch.bfloat16)
+    wI = randn((B, nq, n_hI), 362, torch.float32)
+    codes = torch.empty((B, N_cap, cI), dtype=torch.uint8, device=DEV)
+    ksc = torch.empty((B, N_cap), dtype=torch.float32, device=DEV)
+    csa_quantize_e4m3(dev(KI), codes, ksc)
+    t = [m * N_cap + 3, m * (N_cap // 3) + 1, m * (k // 2), 5]      # all, a third, fewer than k, t < m
+    tt = torch.tensor(t, dtype=torch.int64, device=DEV).reshape(B, nq)
+    ws = torch.zeros(csa_indexer_topk_workspace_size(B, nq, N_cap, k), dtype=torch.uint8, device=DEV)
+    idx = torch.full((B, nq, k), -7, dtype=torch.int32, device=DEV)
+    sc = torch.full((B, nq, k), float("nan"), dtype=torch.float32, device=DEV)
+    csa_indexer_topk_e4m3(dev(qI), dev(wI), codes, ksc, tt, m, k, idx, ws, scores_out=sc)
+    torch.cuda.synchronize()
+    assert csa_workspace_status(ws) == 0
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    for b in range(B):
+        kc, ks = oracle.quantize_rows_e4m3(KI[b].float().numpy())
+        K64 = kc * ks[:, None]
+        for q in range(nq):
+            g = b * nq + q
+            vis = oracle.visible(t[g], m, N_cap)
+            qc, qs = oracle.quantize_rows_e4m3(qI[b, q].float().numpy())
+            q64, w64 = qc * qs[:, None], to_f64(wI[b, q])
+            s = oracle.index_scores(q64, w64, K64, vis)
+            np.testing.assert_array_equal(s, oracle.index_scores_e4m3(qI[b, q].float().numpy(), w64,
+                                                                      KI[b].float().numpy(), vis))
+            check_topk_sets(idx[b, q], s, k, lambda d: score_error_bound(q64, w64, K64, d))
+            got = idx[b, q][idx[b, q] >= 0]
+            band = score_error_bound(q64, w64, K64, got) + 1e-6 * np.abs(s[got])
+            assert np.all(np.abs(sc[b, q][:len(got)] - s[got]) <= band)
+    # the workspace is left clean for the next call
+    idx2 = torch.full((B, nq, k), -7, dtype=torch.int32, device=DEV)
+    csa_indexer_topk_e4m3(dev(qI), dev(wI), codes, ksc, tt, m, k, idx2, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(np.sort(idx2.cpu().numpy(), axis=-1), np.sort(idx, axis=-1))
 
 
 def test_indexer_degenerate_cases():
