@@ -302,6 +302,20 @@ def micro(kind, iters, rotate=4):
         ws = torch.zeros(lib.csa_attn_workspace_size(1, 1, n_h, c, k), dtype=torch.uint8, device=dev)
         calls = [lambda r=r: lib.csa_sparse_attn(q, caches[r], idx, o, ws) for r in range(rotate)]
         nbytes = k * c * 2
+    elif kind == "indexer_e4m3":
+        # the same scan and top-k over E4M3 keys (1 byte per element + one fp32 scale per key)
+        KIs = [randn((1, N, cI), 900 + r, bf16, dev) for r in range(rotate)]
+        K8s = [torch.empty((1, N, cI), dtype=torch.uint8, device=dev) for _ in range(rotate)]
+        KSs = [torch.empty((1, N), dtype=torch.float32, device=dev) for _ in range(rotate)]
+        for r in range(rotate):
+            lib.csa_quantize_e4m3(KIs[r], K8s[r], KSs[r])
+        del KIs
+        qI, wI = randn((1, 1, n_hI, cI), 890, bf16, dev), randn((1, 1, n_hI), 891, torch.float32, dev)
+        idx = torch.empty((1, 1, k), dtype=torch.int32, device=dev)
+        ws = torch.zeros(lib.csa_indexer_topk_workspace_size(1, 1, N, k), dtype=torch.uint8, device=dev)
+        calls = [lambda r=r: lib.csa_indexer_topk_e4m3(qI, wI, K8s[r], KSs[r], t, m, k, idx, ws)
+                 for r in range(rotate)]
+        nbytes = N * (cI + 4)
     elif kind in ("sparse_window", "dense_window"):
         # the same calls with the sliding-window branch: 128 raw-token entries from a ring
         # buffer join the softmax (V4-Pro window size)
@@ -381,8 +395,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--micro", default=None,
-                    help="time one entry point alone: indexer, sparse, dense, sparse_window, "
-                         "dense_window, csa_compress, hca_compress")
+                    help="time one entry point alone: indexer, indexer_e4m3, sparse, dense, "
+                         "sparse_window, dense_window, csa_compress, hca_compress")
     ap.add_argument("--iters", type=int, default=20)
     args = ap.parse_args()
     if args.micro:

@@ -203,8 +203,8 @@ int hca_dense_attn(const void* q, const void* cache, const int64_t* t,
  *   are never exponentiated; [P1] section 12 notes FP4 has the peak of FP8 on current
  *   hardware.  The pages give no block-scale format.  The reading used: OCP E4M3 codes
  *   (largest finite 448) with one fp32 scale per row, scale = max|x| / 448 (0 for an
- *   all-zero row); code = E4M3(x / scale), the division in fp32, rounded to nearest even
- *   and saturated.
+ *   all-zero row); code = E4M3(x * (448 / max|x|)), the factor one fp32 division per row
+ *   and the product in fp32, rounded to nearest even and saturated.
  * x      : [rows, cols] (dtype bf16 or fp32) with row stride ld (elements), cols % 4 == 0
  * codes  : [rows, cols] E4M3 bytes, contiguous (4-byte aligned)
  * scales : fp32 [rows]

@@ -44,7 +44,10 @@ struct ScanCfg {
     static constexpr int kCacheTiles = (kBudget - kFixed0 - 3 * kAStage) >= 32 * kTileKeys * 4 ? 32 : 0;
     static constexpr int kFixed = kFixed0 + kCacheTiles * kTileKeys * 4;
     static constexpr int kStagesRaw = (kBudget - kFixed) / kAStage;
-    static constexpr int kStages = kStagesRaw > 6 ? 6 : kStagesRaw;
+    // the scan is bound by the bytes in flight per SM (ring depth / HBM latency), so the
+    // ring takes what shared memory allows, up to 12 stages (barrier area limit)
+    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+    static_assert((2 * kStages + 6) * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit 256 bytes");
     static constexpr int kSmem = kFixed + kStages * kAStage;
     static constexpr int kTmemCols = (2 * NH) < 32 ? 32 : (2 * NH);
     static_assert(kStages >= 2, "not enough shared memory for a 2-stage ring");
@@ -254,21 +257,41 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
                 // one warp per head: E4M3 codes of q_h / scale_h, scale_h = max|q_h| / 448,
                 // and the head weight folded with the scale (w_h * scale_h)
                 constexpr int V = CI / 32;  // elements per lane (4 or 8)
+                constexpr int HW = NH / 8;  // heads per warp
                 const int ew = et >> 5, el = et & 31;
-                for (int h = ew; h < NH; h += 8) {
+                // every load of this warp's heads first (one round trip), V bf16 per head
+                uint32_t raw[HW][V / 2];
+#pragma unroll
+                for (int i = 0; i < HW; ++i) {
+                    const __nv_bfloat16* src = qg + (int64_t)(ew + 8 * i) * CI + el * V;
+                    if constexpr (V == 4) {
+                        const uint2 u2 = __ldg(reinterpret_cast<const uint2*>(src));
+                        raw[i][0] = u2.x;
+                        raw[i][1] = u2.y;
+                    } else {
+                        const uint4 u4 = __ldg(reinterpret_cast<const uint4*>(src));
+                        raw[i][0] = u4.x; raw[i][1] = u4.y; raw[i][2] = u4.z; raw[i][3] = u4.w;
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < HW; ++i) {
+                    const int h = ew + 8 * i;
                     float x[V];
 #pragma unroll
-                    for (int u = 0; u < V; ++u) x[u] = __bfloat162float(qg[(int64_t)h * CI + el * V + u]);
+                    for (int u = 0; u < V / 2; ++u) {
+                        x[2 * u] = __uint_as_float(raw[i][u] << 16);
+                        x[2 * u + 1] = __uint_as_float(raw[i][u] & 0xffff0000u);
+                    }
                     float amax = 0.f;
 #pragma unroll
                     for (int u = 0; u < V; ++u) amax = fmaxf(amax, fabsf(x[u]));
 #pragma unroll
                     for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                    const float sc = e4m3_scale(amax);
+                    const float sc = e4m3_scale(amax), f = e4m3_factor(amax);
                     uint32_t w[V / 4];
 #pragma unroll
                     for (int u = 0; u < V; u += 4)
-                        w[u / 4] = e4m3x2(x[u], x[u + 1], sc) | (e4m3x2(x[u + 2], x[u + 3], sc) << 16);
+                        w[u / 4] = e4m3x2(x[u], x[u + 1], f) | (e4m3x2(x[u + 2], x[u + 3], f) << 16);
                     const int byte = el * V;  // column of the first code = byte in the row
                     uint8_t* dst = sB + (byte / 128) * (NH * 128) + tc::sw128_offset(h, (byte % 128) / 16) + byte % 16;
                     if constexpr (V == 4)
@@ -310,9 +333,10 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             tc::mbar_arrive(&tempty[acc]);
-            float sc = 0.f;
+            float part[4] = {0.f, 0.f, 0.f, 0.f};  // 4 independent chains, not one of NH
 #pragma unroll
-            for (int h = 0; h < NH; ++h) sc = fmaf(sw[h], fmaxf(v[h], 0.f), sc);
+            for (int h = 0; h < NH; ++h) part[h & 3] = fmaf(sw[h], fmaxf(v[h], 0.f), part[h & 3]);
+            float sc = (part[0] + part[1]) + (part[2] + part[3]);
             if constexpr (KB == 1) sc *= ksc;
             if (sidx < vis) {
                 if (!so.fused) {

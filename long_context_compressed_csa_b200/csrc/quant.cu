@@ -30,12 +30,12 @@ quant_rows_e4m3(const T* __restrict__ x, int64_t rows, int cols, int64_t ld, uin
             for (int u = 0; u < 4; ++u) amax = fmaxf(amax, fabsf(to_f32(xr[c + u])));
 #pragma unroll
         for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const float sc = e4m3_scale(amax);
+        const float f = e4m3_factor(amax);
         for (int c = lane * 4; c < cols; c += 128) {
             const float a = to_f32(xr[c]), b = to_f32(xr[c + 1]), d = to_f32(xr[c + 2]), e = to_f32(xr[c + 3]);
-            *reinterpret_cast<uint32_t*>(codes + r * cols + c) = e4m3x2(a, b, sc) | (e4m3x2(d, e, sc) << 16);
+            *reinterpret_cast<uint32_t*>(codes + r * cols + c) = e4m3x2(a, b, f) | (e4m3x2(d, e, f) << 16);
         }
-        if (lane == 0) scales[r] = sc;
+        if (lane == 0) scales[r] = e4m3_scale(amax);
     }
 }
 

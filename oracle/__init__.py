@@ -195,7 +195,8 @@ def mqa_window(q, cache, sel, win_rows, scale=None):
 # exponentiated) and note FP4 has the peak of FP8 on current hardware ([P1] section 12);
 # the block-scale format is not given.  The reading used: OCP E4M3 codes (1 sign, 4
 # exponent bits with bias 7, 3 mantissa bits, subnormals, largest finite 448, no
-# infinities) with one fp32 scale per row (per key, per query head) = max|x| / 448.
+# infinities) with one fp32 scale per row (per key, per query head) = max|x| / 448; the
+# codes are E4M3(x * (448 / max|x|)).
 # ----------------------------------------------------------------------------------
 E4M3_MAX = 448.0
 
@@ -215,16 +216,18 @@ def round_e4m3(x):
 
 
 def quantize_rows_e4m3(X):
-    """Per-row E4M3 quantisation: scale = max|x| / 448 in fp32, code = E4M3(x / scale) with
-    the division in fp32 (rows of zeros: scale 0, codes 0).  Returns (values of the codes
+    """Per-row E4M3 quantisation: dequantisation scale = max|x| / 448 and quantisation
+    factor r = 448 / max|x|, both one fp32 division per row; code = E4M3(x * r) with the
+    product in fp32 (rows of zeros: scale 0, codes 0).  Returns (values of the codes
     [rows, cols] float64, scales [rows] float64)."""
     X = np.asarray(X, dtype=np.float32)
     X2 = X.reshape(-1, X.shape[-1])
     amax = np.max(np.abs(X2), axis=1).astype(np.float32)
     scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
-    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
-    q = (X2 / safe[:, None]).astype(np.float32)
-    codes = np.where(scale[:, None] > 0, round_e4m3(q), 0.0)
+    safe = np.where(amax > 0, amax, np.float32(1.0)).astype(np.float32)
+    r = (np.float32(E4M3_MAX) / safe).astype(np.float32)
+    q = (X2 * r[:, None]).astype(np.float32)
+    codes = np.where(amax[:, None] > 0, round_e4m3(q), 0.0)
     return codes.reshape(X.shape), scale.astype(np.float64).reshape(X.shape[:-1])
 
 

@@ -262,8 +262,8 @@ def test_indexer_topk_many_queries(B, nq, N_cap, k, seed):
 
 @pytest.mark.parametrize("dtype,cols", [(torch.bfloat16, 128), (torch.float32, 256), (torch.bfloat16, 44)])
 def test_quantize_e4m3_matches_oracle_bit_exactly(dtype, cols):
-    """E4M3 codes and fp32 row scales equal the oracle's (both divide in fp32 and round to
-    nearest even), including an all-zero row and a row of large values."""
+    """E4M3 codes and fp32 row scales equal the oracle's (both form x * (448 / max|x|) in
+    fp32 and round to nearest even), including an all-zero row and a row of large values."""
     X = randn((301, cols), 350, dtype, scale=3.0)
     X[5] = 0
     X[9] = X[9] * 1e4
