@@ -271,7 +271,7 @@ def cpu_baseline(n_steps=2, seed=77):
 # ----------------------------------------------------------------------------------
 # single-kernel micro runs (profiling and per-kernel rooflines)
 # ----------------------------------------------------------------------------------
-def micro(kind, iters, rotate=4):
+def micro(kind, iters, rotate=4, nq_prefill=1024):
     """Time one entry point alone on the 1M workload's shapes (compress kernels on the
     B=16 x 128K HCA and B=4 x 256K CSA prefill shapes), rotating over `rotate` input
     sets so repeated launches do not hit L2.  Prints one JSON line (not the bench line)."""
@@ -285,8 +285,22 @@ def micro(kind, iters, rotate=4):
     n, m, mp, c, cI, n_h, n_hI, k = 1 << 20, 4, 128, 512, 128, 128, 64, 1024
     N, Nh = n // m, n // mp
     t = torch.full((1, 1), n, dtype=torch.int64, device=dev)
-    calls, nbytes = [], 0
-    if kind == "indexer":
+    calls, nbytes, flops = [], 0, 0
+    if kind == "indexer_prefill":
+        # a prefill chunk: the context's last nq_prefill query positions scored and
+        # selected in one call (the many-query tensor-core scan, then one select CTA per
+        # query); the contraction's flops are 2 * n_hI * cI per visible (query, key) pair
+        nq = nq_prefill
+        KIs = [randn((1, N, cI), 900 + r, bf16, dev) for r in range(rotate)]
+        qI, wI = randn((1, nq, n_hI, cI), 892, bf16, dev), randn((1, nq, n_hI), 893, torch.float32, dev)
+        tq = torch.arange(n - nq, n, dtype=torch.int64, device=dev).reshape(1, nq)
+        idx = torch.empty((1, nq, k), dtype=torch.int32, device=dev)
+        ws = torch.zeros(lib.csa_indexer_topk_workspace_size(1, nq, N, k), dtype=torch.uint8, device=dev)
+        calls = [lambda r=r: lib.csa_indexer_topk(qI, wI, KIs[r], tq, m, k, idx, ws) for r in range(rotate)]
+        vis = [min((n - nq + j) // m, N) for j in range(nq)]
+        nbytes = N * cI * 2 + nq * (n_hI * cI * 2 + n_hI * 4 + k * 4)
+        flops = 2 * n_hI * cI * sum(vis)
+    elif kind == "indexer":
         KIs = [randn((1, N, cI), 900 + r, bf16, dev) for r in range(rotate)]
         qI, wI = randn((1, 1, n_hI, cI), 890, bf16, dev), randn((1, 1, n_hI), 891, torch.float32, dev)
         idx = torch.empty((1, 1, k), dtype=torch.int32, device=dev)
@@ -376,12 +390,17 @@ def micro(kind, iters, rotate=4):
     gr.replay()
     torch.cuda.synchronize()
     us = np.array([a.elapsed_time(b) * 1e3 for a, b in evs])
-    hbm, _, src = peaks()
+    hbm, tf, src = peaks()
     gbs = nbytes / (np.median(us) * 1e-6) / 1e9
-    print(json.dumps({"micro": kind, "iters": iters, "us_median": float(np.median(us)),
-                      "us_mean": float(us.mean()), "us_min": float(us.min()),
-                      "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "peak_gbs": hbm,
-                      "frac": gbs / hbm, "peak_source": src}), flush=True)
+    line = {"micro": kind, "iters": iters, "us_median": float(np.median(us)),
+            "us_mean": float(us.mean()), "us_min": float(us.min()),
+            "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "peak_gbs": hbm,
+            "frac": gbs / hbm, "peak_source": src}
+    if flops:
+        tfs = flops / (np.median(us) * 1e-6) / 1e12
+        line.update({"queries": nq_prefill, "algorithmic_flops": flops, "achieved_tflops": tfs,
+                     "peak_tflops": tf, "tensor_frac": tfs / tf})
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -395,12 +414,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--micro", default=None,
-                    help="time one entry point alone: indexer, indexer_e4m3, sparse, dense, "
-                         "sparse_window, dense_window, csa_compress, hca_compress")
+                    help="time one entry point alone: indexer, indexer_e4m3, indexer_prefill, "
+                         "sparse, dense, sparse_window, dense_window, csa_compress, hca_compress")
+    ap.add_argument("--nq", type=int, default=1024,
+                    help="query positions of the indexer_prefill chunk")
     ap.add_argument("--iters", type=int, default=20)
     args = ap.parse_args()
     if args.micro:
-        return micro(args.micro, args.iters)
+        return micro(args.micro, args.iters, nq_prefill=args.nq)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

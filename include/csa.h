@@ -129,8 +129,14 @@ int hca_compress(const void* C, const void* Z,
  *              memory, ZERO-FILLED before its first use (csa_workspace_zero).  Each
  *              call leaves its counters zeroed again for the next call.
  * Scores are fp32.  bf16 products are exact in fp32; sums accumulate in fp32 (tensor
- * cores when dtype is bf16 and n_hI % 16 == 0, 16 <= n_hI <= 256, cI % 64 == 0,
- * cI <= 256; CUDA cores otherwise).  Requires 1 <= k, N_cap < 2^31.
+ * cores when dtype is bf16, n_hI in {16, 32, 64, 128} and cI in {64, 128, 256}; CUDA
+ * cores otherwise).  Requires 1 <= k, N_cap < 2^31 and B*nq <= 65535
+ * (CSA_ERR_UNSUPPORTED otherwise).
+ * Many queries (chunked prefill): when nq >= 16, dtype is bf16, n_hI is 32, 64 or 128,
+ * cI is 64 or 128, N_cap >= 128 and qI and KI are 16-byte aligned, the queries of a
+ * batch row are scored together.  Each block of 512/n_hI queries stays on chip while
+ * the key tiles stream past it, so a key is read once per block rather than once per
+ * query.  The result is the same set of indices.
  * ------------------------------------------------------------------------------- */
 size_t csa_indexer_topk_workspace_size(int B, int nq, int64_t N_cap, int k);
 
@@ -223,7 +229,8 @@ int csa_quantize_e4m3(const void* x, int64_t rows, int cols, int64_t ld, void* c
  * KI8      : [B, N_cap, cI] E4M3 codes (16-byte aligned), KI_scale: fp32 [B, N_cap]
  * qI       : [B, nq, n_hI, cI] bf16 (16-byte aligned); other arguments, the workspace
  *            (csa_indexer_topk_workspace_size) and the outputs as for csa_indexer_topk.
- * Supported: n_hI in {16, 32, 64, 128}, cI in {128, 256}; CSA_ERR_UNSUPPORTED otherwise.
+ * Supported: n_hI in {16, 32, 64, 128}, cI in {128, 256}, B*nq <= 65535;
+ * CSA_ERR_UNSUPPORTED otherwise.
  * Keys take 1 byte instead of 2: the scan of the 1M-token decode reads 34.6 MB instead of
  * 67.1 MB.
  * ------------------------------------------------------------------------------- */

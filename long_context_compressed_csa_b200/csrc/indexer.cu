@@ -140,6 +140,7 @@ struct SelArgs {
     int32_t* idx_out;
     float* scores_out;
     int64_t chunk;  // scores per CTA
+    int self_hist;  // one CTA per query builds its own digit-0 histogram from the scores
 };
 
 __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
@@ -164,9 +165,39 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
         const int64_t i = s_begin + tid + u * kSelThreads;
         key0[u] = i < s_lim ? order_key(__ldcg(&scores[i])) : 0u;
     }
-    sel::load_hist(sh, a.ws.hist0 + (size_t)g * kBins, tid);
     const int64_t vis = visible_count(a.t, g, a.m, a.N_cap);
     const int k = a.k;
+    if (!a.self_hist) {
+        sel::load_hist(sh, a.ws.hist0 + (size_t)g * kBins, tid);
+    } else {
+        // the many-query scan leaves no histogram: this CTA (the query's only one) counts
+        // the top-12-bit digits of its scores in one pass, four float4 loads in flight
+        sel::zero_words(sh, kBins, tid);
+        __syncthreads();
+        if (vis > k) {
+            const float4* s4 = reinterpret_cast<const float4*>(scores);
+            const int64_t n4 = vis >> 2;
+            for (int64_t i0 = 0; i0 < n4; i0 += 4 * kSelThreads) {
+                float4 v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int64_t i = i0 + tid + u * kSelThreads;
+                    v[u] = i < n4 ? __ldcg(&s4[i]) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (i0 + tid + u * kSelThreads < n4) {
+                        atomicAdd(&sh[hist_slot(order_key(v[u].x) >> 20)], 1u);
+                        atomicAdd(&sh[hist_slot(order_key(v[u].y) >> 20)], 1u);
+                        atomicAdd(&sh[hist_slot(order_key(v[u].z) >> 20)], 1u);
+                        atomicAdd(&sh[hist_slot(order_key(v[u].w) >> 20)], 1u);
+                    }
+                }
+            }
+            for (int64_t i = (n4 << 2) + tid; i < vis; i += kSelThreads)
+                atomicAdd(&sh[hist_slot(order_key(__ldcg(&scores[i])) >> 20)], 1u);
+        }
+    }
     const sel::Query q = sel::query_view(a.ws, g, k, a.idx_out, a.scores_out);
 
     if (vis <= k) {
@@ -211,18 +242,19 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
     __threadfence();
     if (vis > k) sel::resolve_candidates<Bar>(q, sh, s_listA, s_listB, &s, tid);
     __syncthreads();
-    sel::reset_query(q, tid);
+    sel::reset_query(q, tid, !a.self_hist);
 }
 
 }  // namespace
 
 int launch_topk_select(const TopkWs& ws, const int64_t* t, int G, int m, int k, int64_t N_cap,
-                       int32_t* idx_out, float* scores_out, cudaStream_t stream)
+                       int32_t* idx_out, float* scores_out, cudaStream_t stream, bool self_hist)
 {
     SelArgs a;
     a.ws = ws; a.t = t; a.m = m; a.k = k; a.N_cap = N_cap;
     a.idx_out = idx_out; a.scores_out = scores_out;
-    int64_t ctas = (2 * kNumSMs + G - 1) / G;
+    a.self_hist = self_hist ? 1 : 0;
+    int64_t ctas = self_hist ? 1 : (2 * kNumSMs + G - 1) / G;
     const int64_t by_size = (N_cap + kRound - 1) / kRound;
     if (ctas > by_size) ctas = by_size;
     if (ctas < 1) ctas = 1;
@@ -287,12 +319,18 @@ extern "C" int csa_indexer_topk(const void* qI, const float* wI, const void* KI,
     if ((((uintptr_t)qI | (uintptr_t)KI) & eb) || ((uintptr_t)wI & 3) || ((uintptr_t)t & 7) ||
         ((uintptr_t)idx_out & 3) || ((uintptr_t)scores_out & 3) || !aligned16(workspace))
         return CSA_ERR_ALIGN;
+    if ((int64_t)B * nq > 65535) return CSA_ERR_UNSUPPORTED;  // one grid row per query
     const int G = B * nq;
     if (!workspace || ws_bytes < csa_indexer_topk_workspace_size(B, nq, N_cap, k))
         return CSA_ERR_WORKSPACE;
     TopkWs ws = topk_ws_layout(workspace, G, N_cap);
     int st;
     bool fused = false;
+    if (dtype == CSA_BF16 && indexer_mq_eligible(qI, KI, B, nq, N_cap, n_hI, cI)) {
+        st = launch_scan_mq(qI, wI, KI, t, B, nq, N_cap, n_hI, cI, m, ws, stream);
+        if (st != CSA_OK) return st;
+        return launch_topk_select(ws, t, G, m, k, N_cap, idx_out, scores_out, stream, true);
+    }
     if (dtype == CSA_BF16 && indexer_tc_supported(n_hI, cI))
         st = launch_scan_tc(qI, wI, KI, t, B, nq, N_cap, n_hI, cI, m, k, ws, idx_out, scores_out, &fused, stream);
     else

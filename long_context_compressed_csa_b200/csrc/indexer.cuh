@@ -39,10 +39,19 @@ int launch_scan_tc_e4m3(const void* qI, const float* wI, const void* KI8, const 
                         const int64_t* t, int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
                         const TopkWs& ws, int32_t* idx_out, float* scores_out, bool* fused,
                         cudaStream_t stream);
+// Many queries of one batch row at once (chunked prefill): tcgen05 scores of a resident
+// block of queries against streamed key tiles, into ws.scores; the stand-alone select
+// with self_hist follows.
+constexpr int kMqMinQueries = 16;
+bool indexer_mq_eligible(const void* qI, const void* KI, int B, int nq, int64_t N_cap, int n_hI, int cI);
+int launch_scan_mq(const void* qI, const float* wI, const void* KI, const int64_t* t, int B, int nq,
+                   int64_t N_cap, int n_hI, int cI, int m, const TopkWs& ws, cudaStream_t stream);
 int launch_scan_cuda_core(const void* qI, const float* wI, const void* KI, const int64_t* t,
                           int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
                           const TopkWs& ws, int dtype, cudaStream_t stream);
+// self_hist: one CTA per query, which builds the digit-0 histogram from the scores itself
+// (after a scan that leaves ws.hist0 untouched).
 int launch_topk_select(const TopkWs& ws, const int64_t* t, int G, int m, int k, int64_t N_cap,
-                       int32_t* idx_out, float* scores_out, cudaStream_t stream);
+                       int32_t* idx_out, float* scores_out, cudaStream_t stream, bool self_hist = false);
 
 }  // namespace csa

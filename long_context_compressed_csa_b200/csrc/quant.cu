@@ -75,6 +75,7 @@ extern "C" int csa_indexer_topk_e4m3(const void* qI, const float* wI, const void
         return CSA_ERR_ARG;
     if (!indexer_e4m3_supported(n_hI, cI)) return CSA_ERR_UNSUPPORTED;
     if (B == 0 || nq == 0) return CSA_OK;
+    if ((int64_t)B * nq > 65535) return CSA_ERR_UNSUPPORTED;  // one grid row per query
     if (!qI || !wI || !KI8 || !KI_scale || !t || !idx_out) return CSA_ERR_ARG;
     if (((uintptr_t)wI & 3) || ((uintptr_t)KI_scale & 3) || ((uintptr_t)t & 7) || ((uintptr_t)idx_out & 3) ||
         ((uintptr_t)scores_out & 3) || !aligned16(workspace))

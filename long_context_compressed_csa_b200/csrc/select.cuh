@@ -413,9 +413,9 @@ CSA_DEV void resolve_candidates(const Query& q, uint32_t* sh, uint2* s_listA, ui
 }
 
 // Zero this query's histogram and counters for the next call.
-CSA_DEV void reset_query(const Query& q, int tid)
+CSA_DEV void reset_query(const Query& q, int tid, bool hist = true)
 {
-    zero_words(q.hist0, kBins, tid);
+    if (hist) zero_words(q.hist0, kBins, tid);
     if (tid < kCtrs) q.ctr[tid] = 0;
 }
 

@@ -87,6 +87,11 @@ def test_host_validation_rejects_bad_arguments_without_launching(lib):
                                 fake, 16, 0, None) == -4
     assert lib.csa_indexer_topk(fake, fake, fake, fake, 1, 1, 100, 4, 8, 4, 5, fake, None,
                                 fake, 1 << 30, 5, None) == -3
+    # more queries than one grid row per query allows (B * nq > 65535)
+    assert lib.csa_indexer_topk(fake, fake, fake, fake, 2, 40000, 100, 64, 128, 4, 5, fake, None,
+                                fake, 1 << 62, 0, None) == -6
+    assert lib.csa_indexer_topk_e4m3(fake, fake, fake, fake, fake, 2, 40000, 100, 64, 128, 4, 8, fake,
+                                     None, fake, 1 << 62, None) == -6
     # attention: out_bf16 with fp32, c too wide, workspace too small
     assert lib.csa_sparse_attn(fake, fake, fake, 1, 1, 4, 64, 100, 8, 0.0, fake, None, fake,
                                1 << 30, 1, 1, None) == -3

@@ -226,11 +226,14 @@ def test_indexer_topk_random(dtype, n_hI, cI, N_cap, k):
         assert np.all(np.abs(sc[0, q][:len(got)] - s[got]) <= band)
 
 
-@pytest.mark.parametrize("B,nq,N_cap,k,seed", [(2, 8, 40000, 512, 230), (3, 50, 1000, 100, 240)])
+@pytest.mark.parametrize("B,nq,N_cap,k,seed", [(2, 8, 40000, 512, 230), (150, 1, 1000, 100, 240),
+                                              (3, 50, 1000, 100, 250)])
 def test_indexer_topk_many_queries(B, nq, N_cap, k, seed):
     """16 queries: each query's scan CTAs own more key tiles than they keep on chip, so
-    the in-place select also reads scores back from the workspace.  150 queries: more
-    queries than resident CTAs, so the scan is followed by the stand-alone select."""
+    the in-place select also reads scores back from the workspace.  150 queries of one
+    each: more queries than resident CTAs, so the scan is followed by the stand-alone
+    select.  50 queries per row at random positions: the many-query scan (query blocks
+    whose visible ranges differ), then one select CTA per query."""
     dtype, n_hI, cI, m = torch.bfloat16, 64, 128, 4
     qI = randn((B, nq, n_hI, cI), seed, dtype)
     KI = randn((B, N_cap, cI), seed + 1, dtype)
@@ -274,6 +277,99 @@ def test_quantize_e4m3_matches_oracle_bit_exactly(dtype, cols):
     want_v, want_s = oracle.quantize_rows_e4m3(X.float().numpy())
     np.testing.assert_array_equal(scales.cpu().numpy().astype(np.float64), want_s)
     np.testing.assert_array_equal(decode_e4m3(codes.cpu().numpy()), want_v)
+
+
+def _oracle_scores(qI, wI, KI, b, q, vis):
+    return oracle.index_scores(to_f64(qI[b, q]), to_f64(wI[b, q]), to_f64(KI[b]), vis)
+
+
+@pytest.mark.parametrize("n_hI,cI,B,nq,N_cap,k,seed", [
+    (64, 128, 1, 40, 5000, 256, 400),    # 5 blocks of 8 queries
+    (64, 128, 2, 19, 3000, 1024, 410),   # 2 rows, ragged last block, visible counts crossing k
+    (32, 64, 1, 33, 2000, 100, 420),     # 16 queries per block, ragged
+    (128, 128, 1, 17, 1500, 64, 430),    # 4 queries per block
+])
+def test_indexer_topk_prefill_chunk(n_hI, cI, B, nq, N_cap, k, seed):
+    """A prefill chunk: nq consecutive query positions per batch row, scored together
+    (blocks of 512 / n_hI queries resident while the key tiles stream past), then one
+    select CTA per query.  Row 0 ends at the last key; row 1 starts just below k visible
+    entries, and its first queries see no entry at all."""
+    dtype, m = torch.bfloat16, 4
+    qI = randn((B, nq, n_hI, cI), seed, dtype)
+    KI = randn((B, N_cap, cI), seed + 1, dtype)
+    wI = randn((B, nq, n_hI), seed + 2, torch.float32)
+    starts = [4 * N_cap - 4 * nq + 3, 0][:B]
+    if B > 1:
+        starts[1] = 4 * (k - 3)
+    t = [t0 + j for t0 in starts for j in range(nq)]
+    if B > 1:
+        t[nq:nq + 3] = [0, 1, 3]             # t < m: nothing visible
+    idx, sc, ws = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k)
+    for b in range(B):
+        K64 = to_f64(KI[b])
+        for q in range(nq):
+            g = b * nq + q
+            vis = oracle.visible(t[g], m, N_cap)
+            q64, w64 = to_f64(qI[b, q]), to_f64(wI[b, q])
+            s = oracle.index_scores(q64, w64, K64, vis)
+            got = idx[b, q]
+            if vis <= k:
+                assert got.tolist() == list(range(vis)) + [-1] * (k - vis)
+            else:
+                check_topk_sets(got, s, k, lambda d: score_error_bound(q64, w64, K64, d))
+            sel = got[got >= 0]
+            band = score_error_bound(q64, w64, K64, sel) + 1e-6 * np.abs(s[sel])
+            assert np.all(np.abs(sc[b, q][:len(sel)] - s[sel]) <= band)
+            assert np.all(np.isneginf(sc[b, q][len(sel):]))
+    idx2, _, _ = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k, ws=ws)
+    assert np.array_equal(np.sort(idx2, axis=-1), np.sort(idx, axis=-1))
+
+
+def test_indexer_topk_prefill_exact_on_integer_inputs():
+    """Many-query path on small-integer q, K, w: every score is an exact integer, so the
+    selected sets, with ties resolved to the smaller index, and the scores must equal
+    the oracle's exactly."""
+    B, nq, N_cap, m, k, n_hI, cI = 2, 20, 3000, 4, 257, 64, 128
+    qI = randint_values((B, nq, n_hI, cI), 440, -2, 3, torch.bfloat16)
+    KI = randint_values((B, N_cap, cI), 441, -2, 3, torch.bfloat16)
+    wI = randint_values((B, nq, n_hI), 442, -2, 3, torch.float32)
+    t = [4 * N_cap - 40 + 2 * j for j in range(nq)] + [4 * 250 + 3 * j for j in range(nq)]
+    idx, sc, _ = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k)
+    for b in range(B):
+        for q in range(nq):
+            g = b * nq + q
+            vis = oracle.visible(t[g], m, N_cap)
+            s = _oracle_scores(qI, wI, KI, b, q, vis)
+            want = oracle.topk(s, k)
+            got = idx[b, q]
+            if vis <= k:
+                assert got.tolist() == list(range(vis)) + [-1] * (k - vis)
+            else:
+                assert sorted(got.tolist()) == sorted(want.tolist())
+            ok = got >= 0
+            np.testing.assert_array_equal(sc[b, q][ok], s[got[ok]])
+
+
+def test_indexer_topk_prefill_full_size_sampled():
+    """The 1M-token context's last 1024 query positions as one prefill chunk (262144
+    keys, k = 1024): the launch the prefill micro-benchmark times.  Four sampled
+    queries, one from each quarter of the chunk, are checked against the oracle."""
+    B, nq, N_cap, m, k, n_hI, cI = 1, 1024, 262144, 4, 1024, 64, 128
+    n = 1 << 20
+    qI = randn((B, nq, n_hI, cI), 450, torch.bfloat16, DEV)
+    KI = randn((B, N_cap, cI), 451, torch.bfloat16, DEV)
+    wI = randn((B, nq, n_hI), 452, torch.float32, DEV)
+    t = [n - nq + j for j in range(nq)]
+    idx, sc, _ = run_indexer(qI, wI, KI, t, m, k)
+    K64 = to_f64(KI[0].cpu())
+    for q in (0, 300, 700, 1023):
+        vis = oracle.visible(t[q], m, N_cap)
+        q64, w64 = to_f64(qI[0, q].cpu()), to_f64(wI[0, q].cpu())
+        s = oracle.index_scores(q64, w64, K64, vis)
+        check_topk_sets(idx[0, q], s, k, lambda d: score_error_bound(q64, w64, K64, d))
+        sel = idx[0, q]
+        band = score_error_bound(q64, w64, K64, sel) + 1e-6 * np.abs(s[sel])
+        assert np.all(np.abs(sc[0, q] - s[sel]) <= band)
 
 
 @pytest.mark.parametrize("n_hI,cI,N_cap,k", [(64, 128, 20000, 512), (32, 256, 3000, 1024), (16, 128, 700, 64)])
