@@ -140,7 +140,6 @@ struct SelArgs {
     int32_t* idx_out;
     float* scores_out;
     int64_t chunk;  // scores per CTA
-    int self_hist;  // one CTA per query builds its own digit-0 histogram from the scores
 };
 
 __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
@@ -167,37 +166,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
     }
     const int64_t vis = visible_count(a.t, g, a.m, a.N_cap);
     const int k = a.k;
-    if (!a.self_hist) {
-        sel::load_hist(sh, a.ws.hist0 + (size_t)g * kBins, tid);
-    } else {
-        // the many-query scan leaves no histogram: this CTA (the query's only one) counts
-        // the top-12-bit digits of its scores in one pass, four float4 loads in flight
-        sel::zero_words(sh, kBins, tid);
-        __syncthreads();
-        if (vis > k) {
-            const float4* s4 = reinterpret_cast<const float4*>(scores);
-            const int64_t n4 = vis >> 2;
-            for (int64_t i0 = 0; i0 < n4; i0 += 4 * kSelThreads) {
-                float4 v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int64_t i = i0 + tid + u * kSelThreads;
-                    v[u] = i < n4 ? __ldcg(&s4[i]) : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (i0 + tid + u * kSelThreads < n4) {
-                        atomicAdd(&sh[hist_slot(order_key(v[u].x) >> 20)], 1u);
-                        atomicAdd(&sh[hist_slot(order_key(v[u].y) >> 20)], 1u);
-                        atomicAdd(&sh[hist_slot(order_key(v[u].z) >> 20)], 1u);
-                        atomicAdd(&sh[hist_slot(order_key(v[u].w) >> 20)], 1u);
-                    }
-                }
-            }
-            for (int64_t i = (n4 << 2) + tid; i < vis; i += kSelThreads)
-                atomicAdd(&sh[hist_slot(order_key(__ldcg(&scores[i])) >> 20)], 1u);
-        }
-    }
+    sel::load_hist(sh, a.ws.hist0 + (size_t)g * kBins, tid);
     const sel::Query q = sel::query_view(a.ws, g, k, a.idx_out, a.scores_out);
 
     if (vis <= k) {
@@ -242,7 +211,143 @@ __global__ void __launch_bounds__(kSelThreads) topk_select(SelArgs a)
     __threadfence();
     if (vis > k) sel::resolve_candidates<Bar>(q, sh, s_listA, s_listB, &s, tid);
     __syncthreads();
-    sel::reset_query(q, tid, !a.self_hist);
+    sel::reset_query(q, tid);
+}
+
+
+// One CTA per query, after the many-query scan, which leaves the scores and, per 32
+// consecutive keys, their largest order key (in the query's second candidate buffer).
+//  1. Filter: at least k groups have a maximum at or above the lower edge T of the
+//     digit-0 bin holding the k-th largest group maximum, so at least k keys are >= T
+//     and the top k are among them.  (With fewer than k groups, T admits every key.)
+//  2. One pass over the scores, eight float4 loads in flight per thread, appends the
+//     keys >= T to the candidate list (warp-aggregated slots from a CTA-local counter:
+//     no other CTA shares the query) and counts their digits.
+//  3. The threshold bin among the candidates; those above it are emitted, those in it
+//     are compacted into the second buffer and resolved as in topk_select.
+// Per key this costs one compare; only the few candidates touch shared-memory atomics.
+__global__ void __launch_bounds__(kSelThreads) topk_select_row(SelArgs a)
+{
+    using Bar = sel::CtaBar;
+    extern __shared__ __align__(16) uint8_t sel_smem[];
+    uint32_t* sh = reinterpret_cast<uint32_t*>(sel_smem);               // [kBins]
+    uint2* s_listA = reinterpret_cast<uint2*>(sel_smem + kBins * 4);    // [kListCap]
+    uint2* s_listB = s_listA + kListCap;                                 // [kListCap]
+    __shared__ sel::Shared s;
+    constexpr int kVec = 8;  // float4 loads in flight per thread
+    pdl_launch_dependents();
+    pdl_wait();
+    const int g = blockIdx.x;
+    const int tid = threadIdx.x;
+    const float* scores = a.ws.scores + (int64_t)g * a.ws.ld;
+    const int64_t vis = visible_count(a.t, g, a.m, a.N_cap);
+    const int k = a.k;
+    sel::Query q = sel::query_view(a.ws, g, k, a.idx_out, a.scores_out);
+    if (vis <= k) {  // everything visible is selected, in index order, padded with -1
+        for (int64_t p = tid; p < k; p += kSelThreads) {
+            q.idx_out[p] = p < vis ? (int32_t)p : -1;
+            if (q.sc_out) q.sc_out[p] = p < vis ? __ldcg(&scores[p]) : -INFINITY;
+        }
+        return;
+    }
+    // ---- 1. filter threshold from the group maxima ----
+    const int64_t ng = (vis + 31) >> 5;
+    uint32_t T = 0;
+    if (ng >= k) {
+        const uint32_t* gm = reinterpret_cast<const uint32_t*>(q.cand2);
+        sel::zero_words(sh, kBins, tid);
+        __syncthreads();
+        for (int64_t i0 = 0; i0 < ng; i0 += 4 * kSelThreads) {
+            uint32_t v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t i = i0 + tid + u * kSelThreads;
+                v[u] = i < ng ? __ldcg(&gm[i]) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (i0 + tid + u * kSelThreads < ng) atomicAdd(&sh[v[u] >> 20], 1u);
+        }
+        __syncthreads();
+        sel::find_threshold_bin<kBins, Bar, true>(sh, (uint32_t)k, &s, tid);
+        T = s.bin << 20;
+    }
+    // ---- 2. candidates: every key >= T, with their digit-0 histogram ----
+    sel::zero_words(sh, kBins, tid);
+    if (tid == 0) s.cnt = 0;
+    __syncthreads();
+    const uint32_t cap = (uint32_t)q.ld;
+    auto keep_if = [&](uint32_t key, uint32_t e, bool in) {
+        const bool keep = in && key >= T;
+        const uint32_t pos = sel::warp_append(&s.cnt, keep);
+        if (keep) {
+            if (pos < cap) q.cand[pos] = make_uint2(key, e);
+            atomicAdd(&sh[key >> 20], 1u);
+        }
+    };
+    const float4* s4 = reinterpret_cast<const float4*>(scores);
+    const int64_t n4 = vis >> 2;  // whole float4 groups; the last vis % 4 scores separately
+    for (int64_t i0 = 0; i0 < n4; i0 += kVec * kSelThreads) {
+        float4 v[kVec];
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) {
+            const int64_t i = i0 + tid + u * kSelThreads;
+            v[u] = i < n4 ? __ldcg(&s4[i]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) {
+            const int64_t i = i0 + tid + u * kSelThreads;
+            const bool in = i < n4;
+            const uint32_t k0 = order_key(v[u].x), k1 = order_key(v[u].y);
+            const uint32_t k2 = order_key(v[u].z), k3 = order_key(v[u].w);
+            if (!__any_sync(0xffffffffu, in && max(max(k0, k1), max(k2, k3)) >= T)) continue;
+            const uint32_t e = (uint32_t)(i << 2);
+            keep_if(k0, e, in);
+            keep_if(k1, e + 1, in);
+            keep_if(k2, e + 2, in);
+            keep_if(k3, e + 3, in);
+        }
+    }
+    if (tid < 32) {  // the last vis % 4 scores (all lanes of warp 0 call)
+        const int64_t i = (n4 << 2) + tid;
+        keep_if(i < vis ? order_key(__ldcg(&scores[i])) : 0u, (uint32_t)i, i < vis);
+    }
+    __syncthreads();
+    const uint32_t nc = s.cnt;  // >= k; at most vis <= ld
+    sel::find_threshold_bin<kBins, Bar, true>(sh, (uint32_t)k, &s, tid);
+    const uint32_t b0 = s.bin;
+    // ---- 3. emit above b0; compact the b0 candidates into the second buffer ----
+    if (tid == 0) {
+        s.out = 0;
+        s.cnt = 0;
+    }
+    __syncthreads();
+    const uint32_t rounds = (nc + kSelThreads - 1) / kSelThreads;
+    for (uint32_t r = 0; r < rounds; ++r) {
+        const uint32_t i = r * kSelThreads + tid;
+        const bool in = i < nc;
+        const uint2 kv = in ? __ldcg(&q.cand[i]) : make_uint2(0, 0);
+        const uint32_t d0 = kv.x >> 20;
+        const bool take = in && d0 > b0;
+        const bool tie = in && d0 == b0;
+        const uint32_t pos = sel::warp_append(&s.out, take);
+        if (take) sel::emit(q, pos, kv);
+        const uint32_t tpos = sel::warp_append(&s.cnt, tie);
+        if (tie) q.cand2[tpos] = kv;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        q.ctr[0] = s.out;
+        q.ctr[1] = s.cnt;
+    }
+    __threadfence();
+    __syncthreads();
+    const uint2* tmp = q.cand;  // the tied candidates now sit in the second buffer
+    q.cand = q.cand2;
+    q.cand2 = const_cast<uint2*>(tmp);
+    sel::resolve_candidates<Bar>(q, sh, s_listA, s_listB, &s, tid);
+    __syncthreads();
+    sel::reset_query(q, tid, false);
 }
 
 }  // namespace
@@ -253,8 +358,14 @@ int launch_topk_select(const TopkWs& ws, const int64_t* t, int G, int m, int k, 
     SelArgs a;
     a.ws = ws; a.t = t; a.m = m; a.k = k; a.N_cap = N_cap;
     a.idx_out = idx_out; a.scores_out = scores_out;
-    a.self_hist = self_hist ? 1 : 0;
-    int64_t ctas = self_hist ? 1 : (2 * kNumSMs + G - 1) / G;
+    const size_t smem = kBins * 4 + 2 * kListCap * sizeof(uint2);
+    if (self_hist) {
+        a.chunk = N_cap;
+        cudaFuncSetAttribute(topk_select_row, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        launch_pdl(topk_select_row, dim3((unsigned)G), dim3(kSelThreads), smem, stream, a);
+        return launch_status();
+    }
+    int64_t ctas = (2 * kNumSMs + G - 1) / G;
     const int64_t by_size = (N_cap + kRound - 1) / kRound;
     if (ctas > by_size) ctas = by_size;
     if (ctas < 1) ctas = 1;
@@ -263,7 +374,6 @@ int launch_topk_select(const TopkWs& ws, const int64_t* t, int G, int m, int k, 
     ctas = (N_cap + a.chunk - 1) / a.chunk;
     if (ctas < 1) ctas = 1;
     dim3 grid((unsigned)ctas, (unsigned)G);
-    const size_t smem = kBins * 4 + 2 * kListCap * sizeof(uint2);
     cudaFuncSetAttribute(topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     launch_pdl(topk_select, grid, dim3(kSelThreads), smem, stream, a);
     return launch_status();

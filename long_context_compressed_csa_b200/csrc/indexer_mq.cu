@@ -20,9 +20,10 @@
 //            weights and writes one fp32 score per query of the half.
 //
 // Consecutive CTAs take consecutive query blocks of the same key range, so the key
-// tiles they stream are shared in L2.  The scores go to the workspace; the stand-alone
-// select (one CTA per query, histogram built from the scores) follows.  Every wait is
-// bounded; a timeout sets the workspace status word and every role drains and exits.
+// tiles they stream are shared in L2.  The scores go to the workspace, together with the
+// largest score of every 32 consecutive keys; the row select (one CTA per query)
+// follows.  Every wait is bounded; a timeout sets the workspace status word and every
+// role drains and exits.
 #include "indexer.cuh"
 #include "tc_utils.cuh"
 
@@ -227,12 +228,14 @@ scan_mq_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             vis[j] = jj < nvalid ? (int)mq_visible(a.t, g0 + jj, a.m, a.N_cap) : 0;
         }
         float* sc_base = a.ws.scores + (g0 + hf * QPM) * a.ws.ld;
+        // per query, the largest order key of every 32 consecutive keys, for the select's
+        // first filter (stored in the query's second candidate buffer, unused until then)
+        uint32_t* gm_base = reinterpret_cast<uint32_t*>(a.ws.cand2) + (g0 + hf * QPM) * 2 * a.ws.ld;
         const float* wh = sw + hf * QPM * NH;
         const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + hf * kMqN;
-        // the half's 256 columns in batches of BC (one query per batch at n_h^I = 64)
-        constexpr int BC = NH > 64 ? NH : 64;
-        constexpr int QPB = BC / NH;   // queries per batch
-        constexpr int NB = kMqN / BC;  // batches per half
+        // the half's 256 columns (QPM queries x NH heads) in 4 batches of 64; a query's
+        // partial sums carry over to the next batch when NH = 128
+        constexpr int kBatch = 64;
         int it = 0;
         for (int tile = tile0; tile < tile1; ++tile, ++it) {
             if (*abort_flag) break;
@@ -242,25 +245,30 @@ scan_mq_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             }
             tc::fence_after_sync();
             const int sidx = tile * kMqKeys + row;
+            float part[4] = {0.f, 0.f, 0.f, 0.f};  // 4 independent chains
 #pragma unroll
-            for (int bt = 0; bt < NB; ++bt) {
-                float v[BC];
+            for (int bt = 0; bt < kMqN / kBatch; ++bt) {
+                float v[kBatch];
 #pragma unroll
-                for (int c0 = 0; c0 < BC; c0 += 16) tc::tmem_ld16(taddr + bt * BC + c0, v + c0);
+                for (int c0 = 0; c0 < kBatch; c0 += 16) tc::tmem_ld16(taddr + bt * kBatch + c0, v + c0);
                 tc::tmem_wait_ld();
-                if (bt == NB - 1) {  // the whole half has been read: the MMA may refill it
+                if (bt == kMqN / kBatch - 1) {  // the whole half has been read: the MMA may refill it
                     tc::fence_before_sync();
                     tc::mbar_arrive(&tempty[hf]);
                 }
 #pragma unroll
-                for (int jj = 0; jj < QPB; ++jj) {
-                    const int j = bt * QPB + jj;
-                    const float* w = wh + j * NH;
-                    float part[4] = {0.f, 0.f, 0.f, 0.f};  // 4 independent chains
-#pragma unroll
-                    for (int h = 0; h < NH; ++h) part[h & 3] = fmaf(w[h], fmaxf(v[jj * NH + h], 0.f), part[h & 3]);
-                    const float sc = (part[0] + part[1]) + (part[2] + part[3]);
-                    if (sidx < vis[j]) sc_base[(int64_t)j * a.ws.ld + sidx] = sc;
+                for (int c = 0; c < kBatch; ++c) {
+                    const int j = (bt * kBatch + c) / NH, h = (bt * kBatch + c) % NH;
+                    part[h & 3] = fmaf(wh[j * NH + h], fmaxf(v[c], 0.f), part[h & 3]);
+                    if (h == NH - 1) {  // query j complete
+                        const float sc = (part[0] + part[1]) + (part[2] + part[3]);
+                        part[0] = part[1] = part[2] = part[3] = 0.f;
+                        const bool valid = sidx < vis[j];
+                        if (valid) sc_base[(int64_t)j * a.ws.ld + sidx] = sc;
+                        const uint32_t gk = __reduce_max_sync(0xffffffffu, valid ? order_key(sc) : 0u);
+                        if (lane == 0 && tile * kMqKeys + quarter * 32 < vis[j])
+                            gm_base[(int64_t)j * 2 * a.ws.ld + tile * 4 + quarter] = gk;
+                    }
                 }
             }
         }

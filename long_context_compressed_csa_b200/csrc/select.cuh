@@ -74,8 +74,8 @@ CSA_DEV void emit(const Query& q, uint32_t pos, uint2 kv)
 // Thread t owns PER consecutive bins, the top ones to thread 0, held in registers: one
 // warp scan and one exchange of warp totals locate the owning thread, which then walks
 // its own registers, so the dependent chain stays short.  A kBins histogram is in the
-// hist_slot layout, a 256-bin one in plain order.
-template <int NBINS, class Bar>
+// hist_slot layout (PLAIN: in plain order), a 256-bin one in plain order.
+template <int NBINS, class Bar, bool PLAIN = false>
 CSA_DEV void find_threshold_bin(const uint32_t* hist, uint32_t need, Shared* s, int tid)
 {
     constexpr int PER = NBINS / kSelThreads;
@@ -84,7 +84,7 @@ CSA_DEV void find_threshold_bin(const uint32_t* hist, uint32_t need, Shared* s, 
     const int lo = NBINS - (tid + 1) * PER;  // this thread covers [lo, lo + PER)
     uint32_t v[PER];
 #pragma unroll
-    for (int i = 0; i < PER; ++i) v[i] = NBINS == kBins ? hist[hist_slot((uint32_t)(lo + i))] : hist[lo + i];
+    for (int i = 0; i < PER; ++i) v[i] = NBINS == kBins && !PLAIN ? hist[hist_slot((uint32_t)(lo + i))] : hist[lo + i];
     uint32_t local = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) local += v[i];
