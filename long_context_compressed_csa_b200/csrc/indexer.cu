@@ -254,23 +254,52 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_row(SelArgs a)
     const int64_t ng = (vis + 31) >> 5;
     uint32_t T = 0;
     if (ng >= k) {
+        // The maxima crowd just below the largest one, M, so their histogram is taken over
+        // a window anchored there: distance bins d = (M - key) >> w, the last bin holding
+        // everything further down, in slot 4095 - d so that larger keys sit higher.  The
+        // first window (w = 12: 1/2048 octave bins, 2 octaves) is widened (w = 16, 20)
+        // only if the k-th largest maximum falls into the last bin.
         const uint32_t* gm = reinterpret_cast<const uint32_t*>(q.cand2);
-        sel::zero_words(sh, kBins, tid);
-        __syncthreads();
+        uint32_t mx = 0;
         for (int64_t i0 = 0; i0 < ng; i0 += 4 * kSelThreads) {
-            uint32_t v[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int64_t i = i0 + tid + u * kSelThreads;
-                v[u] = i < ng ? __ldcg(&gm[i]) : 0u;
+                if (i < ng) mx = max(mx, __ldcg(&gm[i]));
             }
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (i0 + tid + u * kSelThreads < ng) atomicAdd(&sh[v[u] >> 20], 1u);
         }
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if ((tid & 31) == 0) s.scr[tid >> 5] = mx;
         __syncthreads();
-        sel::find_threshold_bin<kBins, Bar, true>(sh, (uint32_t)k, &s, tid);
-        T = s.bin << 20;
+#pragma unroll
+        for (int w = 0; w < kSelThreads / 32; ++w) mx = max(mx, s.scr[w]);
+        for (int w = 12;; w += 4) {
+            sel::zero_words(sh, kBins, tid);
+            __syncthreads();
+            for (int64_t i0 = 0; i0 < ng; i0 += 4 * kSelThreads) {
+                uint32_t v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int64_t i = i0 + tid + u * kSelThreads;
+                    v[u] = i < ng ? __ldcg(&gm[i]) : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (i0 + tid + u * kSelThreads < ng) {
+                        const uint32_t d = min((mx - v[u]) >> w, (uint32_t)(kBins - 1));
+                        atomicAdd(&sh[kBins - 1 - d], 1u);
+                    }
+                }
+            }
+            __syncthreads();
+            sel::find_threshold_bin<kBins, Bar, true>(sh, (uint32_t)k, &s, tid);
+            const uint32_t d = kBins - 1 - s.bin;  // distance bin of the k-th largest maximum
+            if (d < kBins - 1 || w == 20) {
+                const uint64_t below = ((uint64_t)(d + 1) << w) - 1;  // T: lower edge of that bin
+                T = below > mx ? 0u : mx - (uint32_t)below;
+                break;
+            }
+        }
     }
     // ---- 2. candidates: every key >= T, with their digit-0 histogram ----
     sel::zero_words(sh, kBins, tid);
@@ -285,32 +314,64 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_row(SelArgs a)
             atomicAdd(&sh[key >> 20], 1u);
         }
     };
-    const float4* s4 = reinterpret_cast<const float4*>(scores);
-    const int64_t n4 = vis >> 2;  // whole float4 groups; the last vis % 4 scores separately
-    for (int64_t i0 = 0; i0 < n4; i0 += kVec * kSelThreads) {
-        float4 v[kVec];
+    if (ng >= k) {
+        // only groups whose maximum reaches T can hold a candidate: each warp takes 32
+        // group maxima at a time and reads the scores of the hits, up to 8 groups of 32
+        // scores in flight
+        const uint32_t* gm = reinterpret_cast<const uint32_t*>(q.cand2);
+        const int lane = tid & 31, warp = tid >> 5;
+        for (int64_t i0 = (int64_t)warp * 32; i0 < ng; i0 += kSelThreads) {
+            const int64_t gi = i0 + lane;
+            unsigned hit = __ballot_sync(0xffffffffu, gi < ng && __ldcg(&gm[gi]) >= T);
+            while (hit) {
+                int64_t si[8];
+                float v[8];
 #pragma unroll
-        for (int u = 0; u < kVec; ++u) {
-            const int64_t i = i0 + tid + u * kSelThreads;
-            v[u] = i < n4 ? __ldcg(&s4[i]) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+                for (int u = 0; u < 8; ++u) {
+                    si[u] = -1;
+                    if (hit) {
+                        si[u] = ((i0 + __ffs(hit) - 1) << 5) + lane;
+                        hit &= hit - 1;
+                    }
+                }
 #pragma unroll
-        for (int u = 0; u < kVec; ++u) {
-            const int64_t i = i0 + tid + u * kSelThreads;
-            const bool in = i < n4;
-            const uint32_t k0 = order_key(v[u].x), k1 = order_key(v[u].y);
-            const uint32_t k2 = order_key(v[u].z), k3 = order_key(v[u].w);
-            if (!__any_sync(0xffffffffu, in && max(max(k0, k1), max(k2, k3)) >= T)) continue;
-            const uint32_t e = (uint32_t)(i << 2);
-            keep_if(k0, e, in);
-            keep_if(k1, e + 1, in);
-            keep_if(k2, e + 2, in);
-            keep_if(k3, e + 3, in);
+                for (int u = 0; u < 8; ++u) v[u] = si[u] >= 0 && si[u] < vis ? __ldcg(&scores[si[u]]) : 0.f;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (si[u] == -1 && u > 0) break;  // warp-uniform: no more hits in this batch
+                    const bool in = si[u] >= 0 && si[u] < vis;
+                    keep_if(in ? order_key(v[u]) : 0u, (uint32_t)si[u], in);
+                }
+            }
         }
-    }
-    if (tid < 32) {  // the last vis % 4 scores (all lanes of warp 0 call)
-        const int64_t i = (n4 << 2) + tid;
-        keep_if(i < vis ? order_key(__ldcg(&scores[i])) : 0u, (uint32_t)i, i < vis);
+    } else {
+        const float4* s4 = reinterpret_cast<const float4*>(scores);
+        const int64_t n4 = vis >> 2;  // whole float4 groups; the last vis % 4 scores separately
+        for (int64_t i0 = 0; i0 < n4; i0 += kVec * kSelThreads) {
+            float4 v[kVec];
+#pragma unroll
+            for (int u = 0; u < kVec; ++u) {
+                const int64_t i = i0 + tid + u * kSelThreads;
+                v[u] = i < n4 ? __ldcg(&s4[i]) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < kVec; ++u) {
+                const int64_t i = i0 + tid + u * kSelThreads;
+                const bool in = i < n4;
+                const uint32_t k0 = order_key(v[u].x), k1 = order_key(v[u].y);
+                const uint32_t k2 = order_key(v[u].z), k3 = order_key(v[u].w);
+                if (!__any_sync(0xffffffffu, in && max(max(k0, k1), max(k2, k3)) >= T)) continue;
+                const uint32_t e = (uint32_t)(i << 2);
+                keep_if(k0, e, in);
+                keep_if(k1, e + 1, in);
+                keep_if(k2, e + 2, in);
+                keep_if(k3, e + 3, in);
+            }
+        }
+        if (tid < 32) {  // the last vis % 4 scores (all lanes of warp 0 call)
+            const int64_t i = (n4 << 2) + tid;
+            keep_if(i < vis ? order_key(__ldcg(&scores[i])) : 0u, (uint32_t)i, i < vis);
+        }
     }
     __syncthreads();
     const uint32_t nc = s.cnt;  // >= k; at most vis <= ld

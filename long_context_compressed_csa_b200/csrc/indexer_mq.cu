@@ -15,9 +15,11 @@
 //   warp 1   MMA issuer: per key tile two M = 128, N = 256 accumulations, one into
 //            each half of TMEM (columns 0-255 and 256-511), so one half's epilogue
 //            overlaps the other half's MMAs;
-//   warps 2-9 epilogue, four warps per half (one per TMEM lane quarter): each thread
-//            owns one key row, reads its 256 dot products, applies ReLU and the head
-//            weights and writes one fp32 score per query of the half.
+//   warps 2-17 epilogue, eight warps per half (one per TMEM lane quarter and column
+//            half): each thread owns one key row, reads 128 of its dot products,
+//            applies ReLU and the head weights and writes one fp32 score per query of
+//            its columns.  Two warps per scheduler drain a half, so a half's epilogue
+//            fits in the time of the other half's MMAs.
 //
 // Consecutive CTAs take consecutive query blocks of the same key range, so the key
 // tiles they stream are shared in L2.  The scores go to the workspace, together with the
@@ -30,7 +32,9 @@
 namespace csa {
 namespace {
 
-constexpr int kMqThreads = 320;  // producer, MMA, 8 epilogue warps
+constexpr int kMqColParts = 2;                         // epilogue warps per lane quarter and half
+constexpr int kMqEpiThreads = 2 * 4 * kMqColParts * 32;  // both halves
+constexpr int kMqThreads = 64 + kMqEpiThreads;           // producer, MMA, epilogue warps
 constexpr int kMqKeys = 128;     // keys per tile (MMA M)
 constexpr int kMqN = 256;        // (query, head) rows per accumulator half (MMA N)
 constexpr int kMqSmem = 232448;  // the opt-in shared-memory limit per block
@@ -112,7 +116,7 @@ scan_mq_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
         }
         for (int h = 0; h < 2; ++h) {
             tc::mbar_init(&tfull[h], 1);
-            tc::mbar_init(&tempty[h], 128);
+            tc::mbar_init(&tempty[h], kMqEpiThreads / 2);
         }
         tc::mbar_init(done, 1);
         tc::mbar_init(qfull, 1);
@@ -214,28 +218,33 @@ scan_mq_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int et = threadIdx.x - 64;  // 0..255
-        for (int i = et; i < QB * NH; i += 256)
+        const int et = threadIdx.x - 64;
+        for (int i = et; i < QB * NH; i += kMqEpiThreads)
             sw[i] = i / NH < nvalid ? __ldg(&a.wI[g0 * NH + i]) : 0.f;
-        asm volatile("bar.sync 1, 256;" ::: "memory");  // epilogue warps only
+        asm volatile("bar.sync 1, %0;" ::"n"(kMqEpiThreads) : "memory");  // epilogue warps only
         const int quarter = warp & 3;          // TMEM lane quarter this warp may access
-        const int hf = (warp - 2) >> 2;        // accumulator half: queries hf*QPM .. +QPM-1
+        const int hf = ((warp - 2) >> 2) & 1;  // accumulator half: queries hf*QPM .. +QPM-1
+        const int cp = (warp - 2) >> 3;        // column part of the half
         const int row = quarter * 32 + lane;   // key row of this thread within a tile
-        int vis[QPM];
+        constexpr int kCols = kMqN / kMqColParts;  // columns of this warp: whole queries
+        constexpr int kQW = kCols / NH;             // queries of this warp
+        static_assert(kCols % NH == 0, "a column part holds whole queries");
+        const int q0 = hf * QPM + cp * kQW;         // first query of this warp in the block
+        int vis[kQW];
 #pragma unroll
-        for (int j = 0; j < QPM; ++j) {
-            const int jj = hf * QPM + j;
-            vis[j] = jj < nvalid ? (int)mq_visible(a.t, g0 + jj, a.m, a.N_cap) : 0;
-        }
-        float* sc_base = a.ws.scores + (g0 + hf * QPM) * a.ws.ld;
+        for (int j = 0; j < kQW; ++j)
+            vis[j] = q0 + j < nvalid ? (int)mq_visible(a.t, g0 + q0 + j, a.m, a.N_cap) : 0;
+        float* sc_base = a.ws.scores + (g0 + q0) * a.ws.ld;
         // per query, the largest order key of every 32 consecutive keys, for the select's
         // first filter (stored in the query's second candidate buffer, unused until then)
-        uint32_t* gm_base = reinterpret_cast<uint32_t*>(a.ws.cand2) + (g0 + hf * QPM) * 2 * a.ws.ld;
-        const float* wh = sw + hf * QPM * NH;
-        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + hf * kMqN;
-        // the half's 256 columns (QPM queries x NH heads) in 4 batches of 64; a query's
-        // partial sums carry over to the next batch when NH = 128
-        constexpr int kBatch = 64;
+        uint32_t* gm_base = reinterpret_cast<uint32_t*>(a.ws.cand2) + (g0 + q0) * 2 * a.ws.ld;
+        const float* wh = sw + q0 * NH;
+        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + hf * kMqN + cp * kCols;
+        // This warp's columns in batches of 32, double buffered: the TMEM load of batch
+        // b + 1 is in flight while batch b is summed.  A query's partial sums carry over
+        // batches (NH = 64 or 128).
+        constexpr int kBatch = 32;
+        constexpr int kNB = kCols / kBatch;
         int it = 0;
         for (int tile = tile0; tile < tile1; ++tile, ++it) {
             if (*abort_flag) break;
@@ -245,30 +254,39 @@ scan_mq_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             }
             tc::fence_after_sync();
             const int sidx = tile * kMqKeys + row;
-            float part[4] = {0.f, 0.f, 0.f, 0.f};  // 4 independent chains
+            // 4 independent chains (heads h = 0, 1, 2, 3 mod 4), two per packed FMA
+            float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
+            uint32_t ra[32], rb[32];
+            tc::tmem_ld32_async(taddr, ra);
+            tc::tmem_wait_ld_regs(ra);
 #pragma unroll
-            for (int bt = 0; bt < kMqN / kBatch; ++bt) {
-                float v[kBatch];
+            for (int bt = 0; bt < kNB; ++bt) {
+                uint32_t(&cur)[32] = (bt & 1) ? rb : ra;
+                uint32_t(&nxt)[32] = (bt & 1) ? ra : rb;
+                if (bt + 1 < kNB) tc::tmem_ld32_async(taddr + (bt + 1) * kBatch, nxt);
 #pragma unroll
-                for (int c0 = 0; c0 < kBatch; c0 += 16) tc::tmem_ld16(taddr + bt * kBatch + c0, v + c0);
-                tc::tmem_wait_ld();
-                if (bt == kMqN / kBatch - 1) {  // the whole half has been read: the MMA may refill it
-                    tc::fence_before_sync();
-                    tc::mbar_arrive(&tempty[hf]);
-                }
-#pragma unroll
-                for (int c = 0; c < kBatch; ++c) {
-                    const int j = (bt * kBatch + c) / NH, h = (bt * kBatch + c) % NH;
-                    part[h & 3] = fmaf(wh[j * NH + h], fmaxf(v[c], 0.f), part[h & 3]);
-                    if (h == NH - 1) {  // query j complete
-                        const float sc = (part[0] + part[1]) + (part[2] + part[3]);
-                        part[0] = part[1] = part[2] = part[3] = 0.f;
+                for (int c = 0; c < kBatch; c += 4) {
+                    const int col = bt * kBatch + c;  // column within this warp's part
+                    const int j = col / NH, h = col % NH;  // query of this warp, head
+                    const float4 w4 = *reinterpret_cast<const float4*>(wh + j * NH + h);
+                    const float x0 = fmaxf(__uint_as_float(cur[c]), 0.f), x1 = fmaxf(__uint_as_float(cur[c + 1]), 0.f);
+                    const float x2 = fmaxf(__uint_as_float(cur[c + 2]), 0.f), x3 = fmaxf(__uint_as_float(cur[c + 3]), 0.f);
+                    p01 = tc::fma2(make_float2(x0, x1), make_float2(w4.x, w4.y), p01);
+                    p23 = tc::fma2(make_float2(x2, x3), make_float2(w4.z, w4.w), p23);
+                    if (h + 4 == NH) {  // query j complete
+                        const float sc = (p01.x + p01.y) + (p23.x + p23.y);
+                        p01 = p23 = make_float2(0.f, 0.f);
                         const bool valid = sidx < vis[j];
                         if (valid) sc_base[(int64_t)j * a.ws.ld + sidx] = sc;
                         const uint32_t gk = __reduce_max_sync(0xffffffffu, valid ? order_key(sc) : 0u);
                         if (lane == 0 && tile * kMqKeys + quarter * 32 < vis[j])
                             gm_base[(int64_t)j * 2 * a.ws.ld + tile * 4 + quarter] = gk;
                     }
+                }
+                if (bt + 1 < kNB) tc::tmem_wait_ld_regs(nxt);
+                if (bt + 2 == kNB) {  // the last batch is in registers: the MMA may refill the half
+                    tc::fence_before_sync();
+                    tc::mbar_arrive(&tempty[hf]);
                 }
             }
         }

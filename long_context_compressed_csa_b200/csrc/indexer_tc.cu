@@ -333,10 +333,15 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             tc::mbar_arrive(&tempty[acc]);
-            float part[4] = {0.f, 0.f, 0.f, 0.f};  // 4 independent chains, not one of NH
+            // 4 independent chains (h = 0, 1, 2, 3 mod 4), not one of NH; two per packed FMA
+            float2 p01 = make_float2(0.f, 0.f), p23 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int h = 0; h < NH; ++h) part[h & 3] = fmaf(sw[h], fmaxf(v[h], 0.f), part[h & 3]);
-            float sc = (part[0] + part[1]) + (part[2] + part[3]);
+            for (int h = 0; h < NH; h += 4) {
+                const float4 w4 = *reinterpret_cast<const float4*>(sw + h);
+                p01 = tc::fma2(make_float2(fmaxf(v[h], 0.f), fmaxf(v[h + 1], 0.f)), make_float2(w4.x, w4.y), p01);
+                p23 = tc::fma2(make_float2(fmaxf(v[h + 2], 0.f), fmaxf(v[h + 3], 0.f)), make_float2(w4.z, w4.w), p23);
+            }
+            float sc = (p01.x + p01.y) + (p23.x + p23.y);
             if constexpr (KB == 1) sc *= ksc;
             if (sidx < vis) {
                 if (!so.fused) {

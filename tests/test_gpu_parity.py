@@ -325,6 +325,28 @@ def test_indexer_topk_prefill_chunk(n_hI, cI, B, nq, N_cap, k, seed):
     assert np.array_equal(np.sort(idx2, axis=-1), np.sort(idx, axis=-1))
 
 
+def test_indexer_topk_prefill_negative_weights():
+    """Many-query path with every head weight negative: the scores are <= 0, the largest
+    ones cluster near zero, and the group maxima straddle the sign (the order keys of
+    +0 and of negative scores are far apart), so the select's maxima window widens."""
+    B, nq, N_cap, m, k, n_hI, cI = 1, 24, 6000, 4, 300, 64, 128
+    qI = randn((B, nq, n_hI, cI), 460, torch.bfloat16)
+    KI = randn((B, N_cap, cI), 461, torch.bfloat16)
+    wI = -randn((B, nq, n_hI), 462, torch.float32).abs()
+    wI[0, 1:4] = wI[0, 1:4] * 1e-3          # three queries with scores near zero
+    t = [4 * N_cap - 3 * j for j in range(nq)]
+    idx, sc, _ = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k)
+    K64 = to_f64(KI[0])
+    for q in range(nq):
+        vis = oracle.visible(t[q], m, N_cap)
+        q64, w64 = to_f64(qI[0, q]), to_f64(wI[0, q])
+        s = oracle.index_scores(q64, w64, K64, vis)
+        check_topk_sets(idx[0, q], s, k, lambda d: score_error_bound(q64, w64, K64, d))
+        sel = idx[0, q]
+        band = score_error_bound(q64, w64, K64, sel) + 1e-6 * np.abs(s[sel])
+        assert np.all(np.abs(sc[0, q] - s[sel]) <= band)
+
+
 def test_indexer_topk_prefill_exact_on_integer_inputs():
     """Many-query path on small-integer q, K, w: every score is an exact integer, so the
     selected sets, with ties resolved to the smaller index, and the scores must equal
