@@ -300,6 +300,21 @@ def micro(kind, iters, rotate=4, nq_prefill=1024):
         vis = [min((n - nq + j) // m, N) for j in range(nq)]
         nbytes = N * cI * 2 + nq * (n_hI * cI * 2 + n_hI * 4 + k * 4)
         flops = 2 * n_hI * cI * sum(vis)
+    elif kind == "sparse_prefill":
+        # sparse MQA for a prefill chunk: nq_prefill queries, each over its own k selected
+        # entries of the 1M-token CSA cache (indices drawn per query, as the prefill
+        # indexer returns them); flops 2 * 2 * n_h * c per (query, selected entry)
+        nq = nq_prefill
+        caches = [randn((1, N, c), 910 + r, bf16, dev) for r in range(2)]
+        q = randn((1, nq, n_h, c), 925, bf16, dev)
+        g = torch.Generator(device="cpu").manual_seed(926)
+        idx = torch.stack([torch.randperm(N, generator=g)[:k] for _ in range(nq)]).to(torch.int32)
+        idx = idx.reshape(1, nq, k).to(dev)
+        o = torch.empty((1, nq, n_h, c), dtype=torch.float32, device=dev)
+        ws = torch.zeros(lib.csa_attn_workspace_size(1, nq, n_h, c, k), dtype=torch.uint8, device=dev)
+        calls = [lambda r=r: lib.csa_sparse_attn(q, caches[r], idx, o, ws) for r in range(2)]
+        nbytes = nq * k * c * 2
+        flops = 4 * n_h * c * k * nq
     elif kind == "indexer":
         KIs = [randn((1, N, cI), 900 + r, bf16, dev) for r in range(rotate)]
         qI, wI = randn((1, 1, n_hI, cI), 890, bf16, dev), randn((1, 1, n_hI), 891, torch.float32, dev)
@@ -415,9 +430,10 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--micro", default=None,
                     help="time one entry point alone: indexer, indexer_e4m3, indexer_prefill, "
-                         "sparse, dense, sparse_window, dense_window, csa_compress, hca_compress")
+                         "sparse, sparse_prefill, dense, sparse_window, dense_window, csa_compress, "
+                         "hca_compress")
     ap.add_argument("--nq", type=int, default=1024,
-                    help="query positions of the indexer_prefill chunk")
+                    help="query positions of the indexer_prefill / sparse_prefill chunk")
     ap.add_argument("--iters", type=int, default=20)
     args = ap.parse_args()
     if args.micro:

@@ -1,7 +1,7 @@
 // Lightning-indexer scores for many queries at once (chunked prefill) on tcgen05
-// ("DeepSeek-V4 Hybrid Attention: CSA and HCA from Scratch", section 6.4 boxed score;
-// the indexer also scores every query of a prefill chunk, section 6.4 and the cost
-// discussion of section 11).
+// ("DeepSeek-V4 Hybrid Attention: CSA and HCA from Scratch", section 6.4: the boxed
+// score, and the cost paragraph there, by which each of the n queries scores every one
+// of the n/m compressed blocks).
 //
 // With many queries the score is a dense contraction over all of them:
 //   D[s, (j, h)] = K^I[s] . q^I[j, h]     (M = 128 keys, N = 256 query-head pairs, K = c^I)
