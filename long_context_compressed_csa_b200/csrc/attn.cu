@@ -408,8 +408,14 @@ int attn_run(AttnArgs a, float scale, void* out, float* lse, void* workspace, si
     a.part_ml = reinterpret_cast<float2*>(ws + align_up((size_t)G * plan.splits * a.n_h * a.c * sizeof(float), 256));
     a.splits = plan.splits;
     a.per_split = plan.per_split;
+    // one split per query (many queries): the tcgen05 kernel writes the final output and
+    // lse itself, with no combine pass
+    a.direct = tc && plan.splits == 1 && aligned16(out);
+    a.out = out;
+    a.out_bf16 = out_bf16;
+    a.lse = lse;
     int st = tc ? launch_attn_tc(a, plan, status, stream) : launch_cuda_core(a, plan, dtype, stream);
-    if (st != CSA_OK) return st;
+    if (st != CSA_OK || a.direct) return st;
     return launch_attn_combine(a, tc, out, out_bf16, lse, stream);
 }
 

@@ -30,6 +30,12 @@ struct AttnArgs {
     int64_t per_split;    // list positions per split
     void* part_o;         // [G][splits][n_h][c]: fp32 O_i (CUDA-core path) or bf16 O_i / l_i (tcgen05 path)
     float2* part_ml;      // [G][splits][n_h] (max, sum) of 2^(scaled logit)
+    // direct = 1 (tcgen05 path with one split per query): the split kernel writes the final
+    // output out [G][n_h][c] (fp32, or bf16 when out_bf16) and lse [G][n_h] itself
+    int direct;
+    void* out;
+    int out_bf16;
+    float* lse;
 };
 
 struct AttnPlan {

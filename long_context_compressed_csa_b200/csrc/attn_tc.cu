@@ -50,7 +50,7 @@ constexpr int kMaxIds = 1024;                     // entry ids of a range staged
 constexpr int kBarBytes = 256;
 constexpr int kSmem = 1024 + kQBytes + 2 * kCBytes + kPBytes + 2 * kRBytes + kBarBytes + kMaxIds * 4;
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
-static_assert(kQBytes + 2 * kCBytes >= kHeads * kHalf * 2, "output staging reuses q + chunks");
+static_assert(kQBytes + 2 * kCBytes >= kHeads * kHalf * 4, "output staging (fp32 included) reuses q + chunks");
 
 CSA_DEV void cp_async16(uint32_t dst, const void* src, bool valid)
 {
@@ -159,6 +159,23 @@ CSA_DEV void stage_o_cols(uint8_t* stage, uint32_t o_taddr, int h, int col0, flo
     }
 }
 
+// The same for an fp32 output: eight 128-row x 32-column boxes (128 B rows).
+CSA_DEV void stage_o_cols_f32(uint8_t* stage, uint32_t o_taddr, int h, int col0, float inv)
+{
+#pragma unroll 1
+    for (int c0 = col0; c0 < col0 + 128; c0 += 16) {
+        float o[16];
+        tc::tmem_ld16(o_taddr + c0, o);
+        tc::tmem_wait_ld();
+        uint8_t* row = stage + (c0 / 32) * kBoxBytes + h * 128;
+        const int q0 = (c0 % 32) / 4;  // 16-byte chunk of the 128-byte box row
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4*>(row + (((q0 + i) ^ (h & 7)) << 4)) =
+                make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
+    }
+}
+
 // float4 q (0..15) of row h of a 64-float row, XOR-swizzled so that the 32 rows of a
 // warp spread over the banks
 CSA_DEV int rswz(int h, int q) { return h * 16 + (q ^ (h & 15)); }
@@ -257,7 +274,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
     const int64_t p_begin = (int64_t)split * a.per_split;
     const int64_t p_end = min(count, p_begin + a.per_split);
     const int nchunks = p_end > p_begin ? (int)((p_end - p_begin + kE - 1) / kE) : 0;
-    const size_t prow = ((size_t)g * a.splits + split) * kHeads;  // partial row of head 0
+    const size_t prow = ((size_t)g * a.splits + split) * kHeads;  // partial (or output) row of head 0
+    const bool f32_out = a.direct && !a.out_bf16;                  // final fp32 output staged
     const __nv_bfloat16* cache = static_cast<const __nv_bfloat16*>(a.cache) + b * a.N_cap * kC + half * kHalf;
     const __nv_bfloat16* wcache =
         a.win ? static_cast<const __nv_bfloat16*>(a.win) + b * (int64_t)a.win_cap * kC + half * kHalf : cache;
@@ -288,8 +306,20 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
     };
 
     if (nchunks == 0) {
-        // empty range: an empty partial (max -inf, sum 0) that the combine skips
-        if (half == 0 && threadIdx.x < kHeads) a.part_ml[prow + threadIdx.x] = make_float2(-INFINITY, 0.f);
+        if (!a.direct) {
+            // empty range: an empty partial (max -inf, sum 0) that the combine skips
+            if (half == 0 && threadIdx.x < kHeads) a.part_ml[prow + threadIdx.x] = make_float2(-INFINITY, 0.f);
+        } else {
+            // nothing visible: output 0 and lse -inf (this CTA's half of every head row)
+            for (int i = threadIdx.x; i < kHeads * kHalf; i += kThreads) {
+                const size_t o = ((size_t)g * kHeads + i / kHalf) * kC + half * kHalf + i % kHalf;
+                if (a.out_bf16)
+                    static_cast<__nv_bfloat16*>(a.out)[o] = __float2bfloat16(0.f);
+                else
+                    static_cast<float*>(a.out)[o] = 0.f;
+            }
+            if (half == 0 && a.lse && threadIdx.x < kHeads) a.lse[(size_t)g * kHeads + threadIdx.x] = -INFINITY;
+        }
     } else if (warp < 4) {
         // ------------------------------------------------------------ loaders
         const int lt = threadIdx.x;
@@ -374,7 +404,10 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
         if (!*abort_flag && tc::mbar_wait(Ofinal, 0, tc::kWaitBudget)) {
             tc::fence_after_sync();
             const int h = warp * 32 + lane;
-            stage_o_cols(smem, tmem + ((uint32_t)(warp * 32) << 16) + kHalf, h, 0, s_inv_l[h]);
+            if (f32_out)
+                stage_o_cols_f32(smem, tmem + ((uint32_t)(warp * 32) << 16) + kHalf, h, 0, s_inv_l[h]);
+            else
+                stage_o_cols(smem, tmem + ((uint32_t)(warp * 32) << 16) + kHalf, h, 0, s_inv_l[h]);
         } else {
             *abort_flag = 1;
         }
@@ -382,8 +415,9 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
         tc::mbar_arrive(staged);
         if (threadIdx.x == 0) {
             if (tc::mbar_wait(staged, 0, tc::kWaitBudget) && !*abort_flag) {
-                for (int p = 0; p < kHalf / kBoxCols; ++p)
-                    tc::tma_store_2d(&tmap_o, smem + p * kBoxBytes, half * kHalf + p * kBoxCols, (int)prow);
+                const int bc = f32_out ? 32 : kBoxCols;  // columns per 128-byte box row
+                for (int p = 0; p < kHalf / bc; ++p)
+                    tc::tma_store_2d(&tmap_o, smem + p * kBoxBytes, half * kHalf + p * bc, (int)prow);
                 tc::bulk_store_commit_wait();
             } else {
                 *abort_flag = 1;
@@ -523,12 +557,20 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
             s_inv_l[h] = inv;
             tc::mbar_arrive(Ofinal);
             tc::fence_after_sync();
-            stage_o_cols(smem, tmem + lane_base + kHalf, h, 128, inv);
-            if (half == 0) a.part_ml[prow + h] = make_float2(m_run, l_run);
+            if (f32_out)
+                stage_o_cols_f32(smem, tmem + lane_base + kHalf, h, 128, inv);
+            else
+                stage_o_cols(smem, tmem + lane_base + kHalf, h, 128, inv);
+            if (half == 0) {
+                if (!a.direct)
+                    a.part_ml[prow + h] = make_float2(m_run, l_run);
+                else if (a.lse)  // natural-log lse of the scaled logits (m_run, l_run in base 2)
+                    a.lse[(size_t)g * kHeads + h] = l_run > 0.f ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+            }
         } else {
             tc::mbar_arrive(Ofinal);
             *abort_flag = 1;
-            if (half == 0) a.part_ml[prow + h] = make_float2(-INFINITY, 0.f);
+            if (half == 0 && !a.direct) a.part_ml[prow + h] = make_float2(-INFINITY, 0.f);
         }
         tc::fence_proxy_async_smem();
         tc::mbar_arrive(staged);
@@ -641,9 +683,19 @@ int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cu
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    CUtensorMap tmap_o;  // partial outputs [G * splits * 128 rows][512] bf16, 64 x 128 boxes
+    // partial outputs [G * splits * 128 rows][512] bf16 in 64 x 128 boxes, or with one
+    // split per query the final output [G * 128 rows][512] (bf16 boxes as above, fp32 in
+    // 32 x 128 boxes)
+    CUtensorMap tmap_o;
     const uint64_t rows = (uint64_t)a.B * a.nq * plan.splits * kHeads;
-    if (!make_tmap_bf16_2d(&tmap_o, a.part_o, rows, kC, kC, kBoxCols, kHeads)) return CSA_ERR_CUDA;
+    bool ok_o;
+    if (!a.direct)
+        ok_o = make_tmap_bf16_2d(&tmap_o, a.part_o, rows, kC, kC, kBoxCols, kHeads);
+    else if (a.out_bf16)
+        ok_o = make_tmap_bf16_2d(&tmap_o, a.out, rows, kC, kC, kBoxCols, kHeads);
+    else
+        ok_o = make_tmap_f32_2d(&tmap_o, a.out, rows, kC, kC, 32, kHeads);
+    if (!ok_o) return CSA_ERR_CUDA;
     CUtensorMap tmap_q;  // queries [G * 128 rows][512] bf16, 64 x 128 boxes
     if (!make_tmap_bf16_2d(&tmap_q, a.q, (uint64_t)a.B * a.nq * kHeads, kC, kC, 64, kHeads)) return CSA_ERR_CUDA;
     CUtensorMap tmap_c;  // compressed cache [B * N_cap rows][512] bf16, 64 x 64 boxes (dense chunks)

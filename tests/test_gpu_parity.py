@@ -582,6 +582,42 @@ def test_attn_many_queries_and_workspace_reuse():
         np.testing.assert_allclose(lsed.cpu().numpy()[0, 0], ref_lse, atol=2e-3, rtol=0)
 
 
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_attn_prefill_chunk_direct_output(out_dtype):
+    """A prefill chunk of 100 (sparse) and 90 (dense) queries: one CTA pair per query, so
+    the split kernel writes the final output and lse itself (no combine pass), over
+    several 64-entry chunks per pair.  Every query is checked, including dense queries
+    that see no entry (output 0, lse -inf) and a sparse list with padding."""
+    dtype, n_h, c = torch.bfloat16, 128, 512
+    B, nq, N_cap, k = 1, 100, 4096, 300
+    q = randn((B, nq, n_h, c), 470, dtype)
+    cache = randn((B, N_cap, c), 471, dtype)
+    g = torch.Generator().manual_seed(472)
+    idx = torch.stack([torch.randperm(N_cap, generator=g)[:k] for _ in range(nq)]).to(torch.int32)
+    idx[7, 100:250] = -1                                 # padding inside one list
+    o, lse = run_sparse(dev(q), dev(cache), dev(idx.reshape(B, nq, k)), out_dtype=out_dtype)
+    tol = TOL[dtype] if out_dtype == torch.float32 else TOL[dtype] + 2 ** -8
+    for j in range(nq):
+        sel = idx[j].numpy()
+        ref, ref_lse = _ref_attn(to_f64(q[0, j]), to_f64(cache[0]), sel[sel >= 0])
+        assert max_rel_rowwise(o[0, j], ref).max() <= tol
+        np.testing.assert_allclose(lse[0, j], ref_lse, atol=2e-3, rtol=0)
+    mp, Nh, nqd = 16, 1500, 90
+    qd = randn((1, nqd, n_h, c), 473, dtype)
+    cd = randn((1, Nh, c), 474, dtype)
+    t = [mp * 1500 - 40 * j for j in range(nqd)]
+    t[5], t[6] = 3, mp - 1                               # nothing visible
+    od, lsed = run_dense(dev(qd), dev(cd), t, mp, out_dtype=out_dtype)
+    for j in range(nqd):
+        vis = oracle.visible(t[j], mp, Nh)
+        if vis == 0:
+            assert np.all(od[0, j] == 0) and np.all(np.isneginf(lsed[0, j]))
+            continue
+        ref, ref_lse = _ref_attn(to_f64(qd[0, j]), to_f64(cd[0]), np.arange(vis, dtype=np.int32))
+        assert max_rel_rowwise(od[0, j], ref).max() <= tol
+        np.testing.assert_allclose(lsed[0, j], ref_lse, atol=2e-3, rtol=0)
+
+
 @pytest.mark.parametrize("dtype,n_h,c", [(torch.bfloat16, 128, 512), (torch.float32, 16, 64)])
 def test_sparse_and_dense_attn_with_window(dtype, n_h, c):
     """Sliding-window branch: the window entries of tokens max(0, t-n_win+1) .. t, read
