@@ -586,47 +586,61 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
             constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(kHeads, kHalf, false, true);
             const uint32_t q0 = tc::smem_u32(sQ);
             const uint32_t p0 = tc::smem_u32(sP);
-            auto issue_S = [&](int j) -> bool {
-                const int buf = j & 1;
-                if (!tc::mbar_wait(&Cfull[buf], (j >> 1) & 1, tc::kWaitBudget) ||
-                    !tc::mbar_wait(&Sempty[buf], ((j >> 1) & 1) ^ 1, tc::kWaitBudget))
-                    return false;
-                tc::fence_after_sync();
-                const uint32_t c0 = tc::smem_u32(sC0 + buf * kCBytes);
+            // The issuer runs whichever product is ready: S(j) once chunk j has landed and
+            // its TMEM buffer is free, P(j) C once the softmax has written P(j).  Neither
+            // waits on the other, so the gather of chunk j + 2 (which needs P(j) C to free
+            // its buffer) overlaps the softmax of chunk j + 1.
+            auto issue_S = [&](int j) {
+                const uint32_t c0 = tc::smem_u32(sC0 + (j & 1) * kCBytes);
 #pragma unroll
                 for (int p = 0; p < kHalf / 64; ++p) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t ad = tc::smem_desc_sw128(q0 + p * (kHeads * 128) + kk * 32, 16, 1024);
                         const uint64_t bd = tc::smem_desc_sw128(c0 + p * (kE * 128) + kk * 32, 16, 1024);
-                        tc::mma_bf16_ss(tmem + buf * kE, ad, bd, kIdescS, (p | kk) ? 1u : 0u);
+                        tc::mma_bf16_ss(tmem + (j & 1) * kE, ad, bd, kIdescS, (p | kk) ? 1u : 0u);
                     }
                 }
-                tc::mma_commit(&Sfull[buf]);
-                return true;
+                tc::mma_commit(&Sfull[j & 1]);
             };
-            bool ok = tc::mbar_wait(Qfull, 0, tc::kWaitBudget) && issue_S(0);
-            for (int j = 0; j < nchunks && ok; ++j) {
-                if (*abort_flag) break;
-                if (j + 1 < nchunks && !issue_S(j + 1)) {
-                    ok = false;
-                    break;
-                }
-                if (!tc::mbar_wait(Pfull, j & 1, tc::kWaitBudget)) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                const int buf = j & 1;
-                const uint32_t c0 = tc::smem_u32(sC0 + buf * kCBytes);
+            auto issue_PV = [&](int j) {
+                const uint32_t c0 = tc::smem_u32(sC0 + (j & 1) * kCBytes);
 #pragma unroll
                 for (int kk = 0; kk < kE / 16; ++kk) {
                     const uint64_t ad = tc::smem_desc_sw128(p0 + kk * 32, 16, 1024);
                     const uint64_t bd = tc::smem_desc_sw128(c0 + kk * 16 * 128, kE * 128, 1024);
                     tc::mma_bf16_ss(tmem + kHalf, ad, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                tc::mma_commit(&Cempty[buf]);
+                tc::mma_commit(&Cempty[j & 1]);
                 tc::mma_commit(PVdone);
+            };
+            bool ok = tc::mbar_wait(Qfull, 0, tc::kWaitBudget);
+            int nS = 0, nPV = 0;  // products issued so far
+            long long t_last = clock64();
+            int idle = 0;
+            while (ok && nPV < nchunks) {
+                bool progressed = false;
+                if (nS < nchunks) {
+                    const int buf = nS & 1;
+                    const uint32_t ph = (nS >> 1) & 1;
+                    if (tc::mbar_test(&Cfull[buf], ph) && tc::mbar_test(&Sempty[buf], ph ^ 1)) {
+                        tc::fence_after_sync();
+                        issue_S(nS++);
+                        progressed = true;
+                    }
+                }
+                if (nPV < nS && tc::mbar_test(Pfull, nPV & 1)) {
+                    tc::fence_after_sync();
+                    issue_PV(nPV++);
+                    progressed = true;
+                }
+                if (progressed) {
+                    t_last = clock64();
+                    idle = 0;
+                } else {
+                    if (*abort_flag || clock64() - t_last > tc::kWaitBudget) ok = false;
+                    if (++idle >= 8) __nanosleep(32);
+                }
             }
             if (!ok) *abort_flag = 1;
         }

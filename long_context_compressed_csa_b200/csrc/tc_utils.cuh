@@ -42,6 +42,19 @@ CSA_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity)
         : "memory");
     return ok != 0;
 }
+// Non-blocking test: has the phase with the given parity completed?
+CSA_DEV bool mbar_test(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 // Wait until the phase with the given parity has completed; false after `budget` cycles.
 CSA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, long long budget)
 {
