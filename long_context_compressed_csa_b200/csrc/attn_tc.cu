@@ -20,11 +20,12 @@
 //   warps 0-3 loaders  : q half (once) and the entry chunks -> shared memory; at the
 //                        end, output columns 0..127 -> staging; thread 0 issues the
 //                        TMA stores of the staged output half
-//   warps 4-7 softmax  : partial S rows from TMEM -> peer, S, online softmax with lazy
-//                        rescaling (O is rescaled in TMEM only when the running max grows
-//                        by more than 2^8), P (bf16) -> shared memory; at the end,
-//                        output columns 128..255 -> staging
-//   warp 8    MMA      : S(j+1) is issued before P(j) C so the tensor core stays busy
+//   warps 4-7, 9-12    : softmax, two groups (entries 0-31 and 32-63 of a chunk, one
+//                        thread per row in each): partial S from TMEM -> peer, S, online
+//                        softmax with lazy rescaling (O is rescaled in TMEM only when the
+//                        running max grows by more than 2^8), P (bf16) -> shared memory;
+//                        at the end, output columns 128..255 -> staging
+//   warp 8    MMA      : issues S(j) and P(j) C as soon as each is ready
 // CTA pairs split the entry list.  A split's partial is its normalised output O_i / l_i,
 // rounded to bf16 (relative error at most 2^-9 per element, the same as the bf16 P fed
 // to the tensor core) and written by TMA, with its running max and sum in base 2 in
@@ -41,14 +42,17 @@ constexpr int kHalf = 256;          // columns of c owned by each CTA of the pai
 constexpr int kHeads = 128;         // M
 constexpr int kE = 64;              // entries per chunk (N of S, K of P C)
 constexpr int kLoaders = 128;
-constexpr int kThreads = 288;       // 4 loader warps, 4 softmax warps, 1 MMA warp
+constexpr int kThreads = 416;       // 4 loader warps, 4 softmax warps, the MMA warp, 4 softmax warps
+constexpr int kMmaWarp = 8;
+constexpr int kSoftmax = 256;       // softmax threads: two per row
 constexpr int kQBytes = kHeads * kHalf * 2;       // 64 KB: 4 panels of 128 rows x 128 B
 constexpr int kCBytes = kE * kHalf * 2;           // 32 KB: 4 panels of 64 rows x 128 B
 constexpr int kPBytes = kHeads * kE * 2;          // 16 KB: 128 rows x 128 B
 constexpr int kRBytes = kHeads * kE * 4;          // 32 KB: peer partial S, fp32
 constexpr int kMaxIds = 1024;                     // entry ids of a range staged in smem
 constexpr int kBarBytes = 256;
-constexpr int kSmem = 1024 + kQBytes + 2 * kCBytes + kPBytes + 2 * kRBytes + kBarBytes + kMaxIds * 4;
+constexpr int kXBytes = (2 * 2 + 2) * kHeads * 4;   // row maxima [2 chunks][2 groups][128], sums [2][128]
+constexpr int kSmem = 1024 + kQBytes + 2 * kCBytes + kPBytes + 2 * kRBytes + kBarBytes + kMaxIds * 4 + kXBytes;
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
 static_assert(kQBytes + 2 * kCBytes >= kHeads * kHalf * 4, "output staging (fp32 included) reuses q + chunks");
 
@@ -135,14 +139,14 @@ CSA_DEV float ex2_approx(float x)
 constexpr int kBoxCols = 64;             // one output box: 128 rows x 64 bf16 columns (128 B)
 constexpr int kBoxBytes = kHeads * 128;  // 16 KB
 
-// Copy columns [col0, col0 + 128) of row h of the output half from TMEM (o_taddr: this
+// Copy columns [col0, col0 + ncols) of row h of the output half from TMEM (o_taddr: this
 // warp's lane quarter, first O column), scaled by inv = 1 / l, into the staging boxes as
 // bf16: four 128-row x 64-column boxes in the 128-byte swizzled layout of the output
 // tensor map.
-CSA_DEV void stage_o_cols(uint8_t* stage, uint32_t o_taddr, int h, int col0, float inv)
+CSA_DEV void stage_o_cols(uint8_t* stage, uint32_t o_taddr, int h, int col0, float inv, int ncols = 128)
 {
 #pragma unroll 1
-    for (int c0 = col0; c0 < col0 + 128; c0 += 16) {
+    for (int c0 = col0; c0 < col0 + ncols; c0 += 16) {
         float o[16];
         tc::tmem_ld16(o_taddr + c0, o);
         tc::tmem_wait_ld();
@@ -160,10 +164,10 @@ CSA_DEV void stage_o_cols(uint8_t* stage, uint32_t o_taddr, int h, int col0, flo
 }
 
 // The same for an fp32 output: eight 128-row x 32-column boxes (128 B rows).
-CSA_DEV void stage_o_cols_f32(uint8_t* stage, uint32_t o_taddr, int h, int col0, float inv)
+CSA_DEV void stage_o_cols_f32(uint8_t* stage, uint32_t o_taddr, int h, int col0, float inv, int ncols = 128)
 {
 #pragma unroll 1
-    for (int c0 = col0; c0 < col0 + 128; c0 += 16) {
+    for (int c0 = col0; c0 < col0 + ncols; c0 += 16) {
         float o[16];
         tc::tmem_ld16(o_taddr + c0, o);
         tc::tmem_wait_ld();
@@ -198,7 +202,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
     uint64_t* Sempty = bars + 6;    // [2] softmax -> MMA            (count 128)
     uint64_t* Rfull = bars + 8;     // peer's bulk copy landed in sR (count 1 + bytes)
     uint64_t* Xready = bars + 9;    // own partial staged in sX      (count 128)
-    uint64_t* Rfree = bars + 10;    // peer consumed what we sent    (count 128, remote)
+    uint64_t* Rfree = bars + 10;    // peer consumed what we sent    (count 8 warps, remote)
     uint64_t* Xfree = bars + 11;    // our bulk copy has read sX     (count 1)
     uint64_t* Pfull = bars + 12;    // softmax -> MMA                (count 128)
     uint64_t* PVdone = bars + 13;   // MMA commit -> softmax
@@ -206,10 +210,14 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
     uint64_t* staged = bars + 15;   // output half staged            (count 256: loaders + softmax)
     uint64_t* Ofinal = bars + 16;   // softmax -> loaders: last P C done (count 128)
     uint64_t* Qfull = bars + 17;    // q half landed (TMA, count 1 + bytes)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+    uint64_t* MXready = bars + 18;  // both softmax groups' row maxima written (count 256)
+    uint64_t* Lready = bars + 19;   // both softmax groups' row sums written (count 256)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
     volatile uint32_t* abort_flag = tmem_slot + 1;
     int* s_ids = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);  // [kMaxIds]
     float* s_inv_l = reinterpret_cast<float*>(sP);  // [128] 1 / l per head, after the last P C
+    float* s_mx = reinterpret_cast<float*>(s_ids + kMaxIds);  // [2][2][128] partial row maxima
+    float* s_lp = s_mx + 4 * kHeads;                          // [2][128] partial row sums
 
     pdl_launch_dependents();
     const int split = blockIdx.x, g = blockIdx.z;
@@ -223,16 +231,18 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
             tc::mbar_init(&Cfull[i], kLoaders);
             tc::mbar_init(&Cempty[i], 1);
             tc::mbar_init(&Sfull[i], 1);
-            tc::mbar_init(&Sempty[i], kHeads);
+            tc::mbar_init(&Sempty[i], kSoftmax);
         }
         tc::mbar_init(Rfull, 1);
-        tc::mbar_init(Xready, kHeads);
-        tc::mbar_init(Rfree, kHeads);
+        tc::mbar_init(Xready, kSoftmax);
+        tc::mbar_init(Rfree, kSoftmax / 32);
         tc::mbar_init(Xfree, 1);
-        tc::mbar_init(Pfull, kHeads);
+        tc::mbar_init(Pfull, kSoftmax);
         tc::mbar_init(PVdone, 1);
         tc::mbar_init(idsready, kLoaders);
-        tc::mbar_init(staged, 2 * kHeads);
+        tc::mbar_init(staged, kLoaders + kSoftmax);
+        tc::mbar_init(MXready, kSoftmax);
+        tc::mbar_init(Lready, kSoftmax);
         tc::mbar_init(Ofinal, kHeads);
         tc::mbar_init(Qfull, 1);
         tc::tma_prefetch_desc(&tmap_q);
@@ -240,7 +250,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         tc::tmem_alloc(tmem_slot, 512);
         tc::tmem_relinquish();
     }
@@ -423,11 +433,18 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
                 *abort_flag = 1;
             }
         }
-    } else if (warp < 8) {
+    } else if (warp != kMmaWarp) {
         // ------------------------------------------------------------ softmax
+        // Two groups of four warps: group sg owns entries [32 sg, 32 sg + 32) of every
+        // chunk for all 128 rows (thread = row).  The two threads of a row agree on the
+        // row maximum through a double-buffered shared exchange (bounded mbarrier wait),
+        // so they keep identical running maxima and rescale decisions; each keeps its own
+        // partial sum of the row.
+        const int sg = warp > kMmaWarp ? 1 : 0;
         const int quarter = warp & 3;
         const int h = quarter * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        constexpr int kEG = kE / 2;  // entries of a chunk per group
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = tc::mbar_wait(idsready, 0, tc::kWaitBudget);
         int sent = 0;  // chunks whose partial logits thread 128 sent to the peer
@@ -439,9 +456,9 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
                 break;
             }
             tc::fence_after_sync();
-            float s[kE];
+            float s[kEG];
 #pragma unroll
-            for (int c0 = 0; c0 < kE; c0 += 16) tc::tmem_ld16(tmem + lane_base + buf * kE + c0, s + c0);
+            for (int c0 = 0; c0 < kEG; c0 += 16) tc::tmem_ld16(tmem + lane_base + buf * kE + sg * kEG + c0, s + c0);
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             tc::mbar_arrive(&Sempty[buf]);
@@ -456,8 +473,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
                 break;
             }
 #pragma unroll
-            for (int q = 0; q < kE / 4; ++q)
-                sX[rswz(h, q)] = make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
+            for (int q = 0; q < kEG / 4; ++q)
+                sX[rswz(h, sg * (kEG / 4) + q)] = make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(Xready);
             if (threadIdx.x == 128) {
@@ -477,8 +494,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
                 break;
             }
 #pragma unroll
-            for (int q = 0; q < kE / 4; ++q) {
-                const float4 o = sR[rswz(h, q)];
+            for (int q = 0; q < kEG / 4; ++q) {
+                const float4 o = sR[rswz(h, sg * (kEG / 4) + q)];
                 if (half == 0) {
                     s[4 * q] = s[4 * q] + o.x; s[4 * q + 1] = s[4 * q + 1] + o.y;
                     s[4 * q + 2] = s[4 * q + 2] + o.z; s[4 * q + 3] = s[4 * q + 3] + o.w;
@@ -487,19 +504,27 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
                     s[4 * q + 2] = o.z + s[4 * q + 2]; s[4 * q + 3] = o.w + s[4 * q + 3];
                 }
             }
-            mbar_arrive_remote(peer_addr(tc::smem_u32(Rfree), peer));  // our receive buffer is free again
-            const int64_t p0 = p_begin + (int64_t)j * kE;
-            const unsigned vlo = __ballot_sync(0xffffffffu, plain ? p0 + lane < p_end : entry_of(p0 + lane) != -1);
-            const unsigned vhi =
-                __ballot_sync(0xffffffffu, plain ? p0 + 32 + lane < p_end : entry_of(p0 + 32 + lane) != -1);
+            // our receive buffer is free again: one release arrival per warp, after the
+            // warp's reads of sR (a remote arrival costs a cluster-scope release each)
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(peer_addr(tc::smem_u32(Rfree), peer));
+            const int64_t pg = p_begin + (int64_t)j * kE + sg * kEG;  // list position of entry 0 of the group
+            const unsigned vm = __ballot_sync(0xffffffffu, plain ? pg + lane < p_end : entry_of(pg + lane) != -1);
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // 4 chains, not 1
 #pragma unroll
-            for (int e = 0; e < kE; ++e) {
-                const bool valid = (((e < 32) ? (vlo >> e) : (vhi >> (e - 32))) & 1u) != 0;
-                s[e] = valid ? s[e] * a.scale_log2 : -INFINITY;
+            for (int e = 0; e < kEG; ++e) {
+                s[e] = ((vm >> e) & 1u) ? s[e] * a.scale_log2 : -INFINITY;
                 mx[e & 3] = fmaxf(mx[e & 3], s[e]);
             }
-            const float cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            // the row maximum of the chunk: both groups' partial maxima, same order in both
+            float* mxb = s_mx + (j & 1) * 2 * kHeads;
+            mxb[sg * kHeads + h] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            tc::mbar_arrive(MXready);
+            if (!tc::mbar_wait(MXready, j & 1, tc::kWaitBudget)) {
+                ok = false;
+                break;
+            }
+            const float cmax = fmaxf(mxb[h], mxb[kHeads + h]);
             if (j > 0) {
                 // P buffer and O are free once the previous chunk's P C has finished
                 if (!tc::mbar_wait(PVdone, (j - 1) & 1, tc::kWaitBudget)) {
@@ -509,10 +534,11 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
                 tc::fence_after_sync();
                 const bool need = cmax > m_run + kRescaleThreshold;
                 if (__any_sync(0xffffffffu, need)) {
+                    // each group rescales its 128 of the 256 output columns of the row
                     const float f = need ? (m_run == -INFINITY ? 0.f : exp2f(m_run - cmax)) : 1.f;
-                    const uint32_t ob = tmem + lane_base + kHalf;
+                    const uint32_t ob = tmem + lane_base + kHalf + sg * (kHalf / 2);
 #pragma unroll 1
-                    for (int c0 = 0; c0 < kHalf; c0 += 16) {
+                    for (int c0 = 0; c0 < kHalf / 2; c0 += 16) {
                         float o[16];
                         tc::tmem_ld16(ob + c0, o);
                         tc::tmem_wait_ld();
@@ -530,9 +556,9 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
                 m_run = cmax;
             }
             float ps[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t packed[kE / 2];
+            uint32_t packed[kEG / 2];
 #pragma unroll
-            for (int e = 0; e < kE; e += 2) {
+            for (int e = 0; e < kEG; e += 2) {
                 const float p0f = (s[e] == -INFINITY) ? 0.f : ex2_approx(s[e] - m_run);
                 const float p1f = (s[e + 1] == -INFINITY) ? 0.f : ex2_approx(s[e + 1] - m_run);
                 ps[(e >> 1) & 3] += p0f + p1f;
@@ -541,36 +567,49 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
             }
             l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
 #pragma unroll
-            for (int qc = 0; qc < kE / 8; ++qc) {
+            for (int qc = 0; qc < kEG / 8; ++qc) {
                 uint4 v = make_uint4(packed[4 * qc], packed[4 * qc + 1], packed[4 * qc + 2], packed[4 * qc + 3]);
-                *reinterpret_cast<uint4*>(sP + tc::sw128_offset(h, qc)) = v;
+                *reinterpret_cast<uint4*>(sP + tc::sw128_offset(h, sg * (kEG / 8) + qc)) = v;
             }
             tc::fence_proxy_async_smem();
             tc::fence_before_sync();
             tc::mbar_arrive(Pfull);
         }
-        if (ok && !*abort_flag && tc::mbar_wait(PVdone, (nchunks - 1) & 1, tc::kWaitBudget)) {
+        bool fin = ok && !*abort_flag && tc::mbar_wait(PVdone, (nchunks - 1) & 1, tc::kWaitBudget);
+        float l_tot = 0.f;
+        if (fin) {
+            // the row sum: both groups' partial sums, same order in both
+            s_lp[sg * kHeads + h] = l_run;
+            tc::mbar_arrive(Lready);
+            fin = tc::mbar_wait(Lready, 0, tc::kWaitBudget);
+            if (fin) l_tot = s_lp[h] + s_lp[kHeads + h];
+        } else {
+            tc::mbar_arrive(Lready);
+        }
+        if (fin) {
             // The last P C has completed, so every MMA reading q, the chunks and P has too:
-            // q + chunk buffers stage the output half as bf16 O / l (columns 128..255 here),
-            // and the P buffer passes 1 / l to the loader warps.
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            s_inv_l[h] = inv;
-            tc::mbar_arrive(Ofinal);
+            // q + chunk buffers stage the output half (columns 128..191 by group 0,
+            // 192..255 by group 1), and the P buffer passes 1 / l to the loader warps.
+            const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+            if (sg == 0) {
+                s_inv_l[h] = inv;
+                tc::mbar_arrive(Ofinal);
+            }
             tc::fence_after_sync();
             if (f32_out)
-                stage_o_cols_f32(smem, tmem + lane_base + kHalf, h, 128, inv);
+                stage_o_cols_f32(smem, tmem + lane_base + kHalf, h, 128 + sg * 64, inv, 64);
             else
-                stage_o_cols(smem, tmem + lane_base + kHalf, h, 128, inv);
-            if (half == 0) {
+                stage_o_cols(smem, tmem + lane_base + kHalf, h, 128 + sg * 64, inv, 64);
+            if (half == 0 && sg == 0) {
                 if (!a.direct)
-                    a.part_ml[prow + h] = make_float2(m_run, l_run);
-                else if (a.lse)  // natural-log lse of the scaled logits (m_run, l_run in base 2)
-                    a.lse[(size_t)g * kHeads + h] = l_run > 0.f ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+                    a.part_ml[prow + h] = make_float2(m_run, l_tot);
+                else if (a.lse)  // natural-log lse of the scaled logits (m_run, l_tot in base 2)
+                    a.lse[(size_t)g * kHeads + h] = l_tot > 0.f ? (m_run + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
             }
         } else {
-            tc::mbar_arrive(Ofinal);
+            if (sg == 0) tc::mbar_arrive(Ofinal);
             *abort_flag = 1;
-            if (half == 0 && !a.direct) a.part_ml[prow + h] = make_float2(-INFINITY, 0.f);
+            if (half == 0 && sg == 0 && !a.direct) a.part_ml[prow + h] = make_float2(-INFINITY, 0.f);
         }
         tc::fence_proxy_async_smem();
         tc::mbar_arrive(staged);
@@ -649,7 +688,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
     tc::fence_before_sync();
     __syncthreads();
     if (*abort_flag && threadIdx.x == 0) atomicExch(status, 1u);
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, 512);
     }
