@@ -41,6 +41,17 @@ SCAN_TRAFFIC_BYTES = 67_961_856
 IDX_SAMPLE = 8  # steps per CUDA graph; the indexer call of each graph's first step is timed
 
 
+def workload_config(world):
+    """The `config` object of both arms' JSON line (the 1M-token hybrid decode)."""
+    return {"workload": WORKLOAD, "n": 1 << 20, "B": 1, "c": 512, "m": 4, "m_prime": 128, "k": 1024,
+            "n_h": 128, "n_hI": 64, "cI": 128, "pairs_rotated": N_PAIRS,
+            "parallelism": "replicas" if world > 1 else "single",
+            "l2": "inputs larger than L2: 8 layer pairs rotated (73 MiB read per step, "
+                  "584 MiB between revisits of a pair)",
+            "step": "one token through one CSA+HCA layer pair (indexer+top-k, sparse MQA, "
+                    "dense MQA, incremental compress at block ends)"}
+
+
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
@@ -451,7 +462,7 @@ def main():
                 "n_gpus": args.gpus, "steps": max(1, min(args.steps, 3)), "warmup": 0,
                 "ms_per_step": 1000.0 / base["value"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": WORKLOAD, "n": 1 << 20, "B": 1, "pairs_rotated": N_PAIRS},
+                "config": workload_config(args.gpus),
                 "cpu_baseline": {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")},
                 "e2e": {"value": base["value"], "unit": base["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -560,13 +571,7 @@ def main():
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms_all / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "n": dec.n, "B": 1, "c": dec.c, "m": dec.m,
-                   "m_prime": dec.mp, "k": dec.k, "n_h": dec.n_h, "n_hI": dec.n_hI, "cI": dec.cI,
-                   "pairs_rotated": N_PAIRS, "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "inputs larger than L2: 8 layer pairs rotated (73 MiB read per step, "
-                         "584 MiB between revisits of a pair)",
-                   "step": "one token through one CSA+HCA layer pair (indexer+top-k, sparse MQA, "
-                           "dense MQA, incremental compress at block ends)"},
+        "config": workload_config(world),
         "roofline": {"kernel": "csa_indexer_topk (scan_tc_kernel: indexer scan with the top-k "
                                "select in place)", "bound": "hbm",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
