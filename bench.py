@@ -41,6 +41,22 @@ SCAN_TRAFFIC_BYTES = 67_961_856
 IDX_SAMPLE = 8  # steps per CUDA graph; the indexer call of each graph's first step is timed
 
 
+def max_over_ranks(x, device="cpu"):
+    """Max of a per-rank float over all ranks of the default process group (the value
+    itself on one rank).  The device is the group's: "cuda" under NCCL, "cpu" under gloo."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(steps_per_rank, world, ms_max):
+    """Steps per second of the whole job: every rank's steps over the slowest rank's time."""
+    return steps_per_rank * world / (ms_max / 1000.0)
+
+
 def workload_config(world):
     """The `config` object of both arms' JSON line (the 1M-token hybrid decode)."""
     return {"workload": WORKLOAD, "n": 1 << 20, "B": 1, "c": 512, "m": 4, "m_prime": 128, "k": 1024,
@@ -540,18 +556,14 @@ def main():
     clocks = sampler.stop()
     ms = start.elapsed_time(end)
     idx_ms = np.array([ev[0].elapsed_time(ev[1]) for _, ev in graphs])
-    t_max = torch.tensor([ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    ms_all = float(t_max.item())
+    ms_all = max_over_ranks(ms, "cuda")
 
     bytes_total = sum(dec.step_bytes(s // N_PAIRS) for s in range(W, W + K))
     launches = sum(kernel_launches_per_step(dec, s // N_PAIRS) for s in range(W, W + K))
     log("indexer+topk per launch: mean %.2f us, median %.2f us; step %.2f us" %
         (idx_ms.mean() * 1e3, np.median(idx_ms) * 1e3, ms * 1e3 / K))
     hbm, tf, src = peaks()
-    steps_all = K * world
-    value = steps_all / (ms_all / 1000.0)
+    value = whole_job_rate(K, world, ms_all)
 
     # ---- dominant kernel: the indexer (scan over every visible key, then top-k) ----
     vis = (dec.n + (W // N_PAIRS)) // dec.m
