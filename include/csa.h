@@ -110,6 +110,31 @@ int hca_compress(const void* C, const void* Z,
                  int dtype, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * hca_project_compress - hca_compress fused with the projections that produce its
+ * inputs ([P1] section 10: C = H W^KV and the pooling logits Z = H W^Z per token, then
+ * the boxed softmax pooling over each entry's m' tokens; [P1] section 3 states the
+ * projections H W of the CSA streams).  C and Z are computed on the tensor cores in fp32
+ * (bf16 products) and never written to memory.  The model width d is not given by the
+ * pages; any d that is a multiple of 64 is accepted.
+ *
+ * H      : bf16 token rows, row r of batch b at H + b*ld_batch + (r - tok0)*ld_row
+ *          (ld_row a multiple of 8, ld_batch a multiple of ld_row, 16-byte aligned);
+ *          rows m'*entry_begin .. m'*entry_end - 1 are read.
+ * Wc, Wz : bf16 [c, d], row j holds output column j's weights (16-byte aligned).
+ * Bias   : fp32 [m', c] or NULL.
+ * out    : bf16, entry i of batch b at out + b*out_ld_batch + i*c.
+ * workspace: >= 256 bytes of zero-filled device memory; csa_workspace_status reports a
+ *          bounded-wait timeout.
+ * Supported: m' = 128, c a multiple of 128, d a multiple of 64; CSA_ERR_UNSUPPORTED
+ * otherwise.
+ * ------------------------------------------------------------------------------- */
+int hca_project_compress(const void* H, int64_t ld_row, int64_t ld_batch, int64_t tok0,
+                         int64_t n, const void* Wc, const void* Wz, int d, const float* Bias,
+                         void* out, int64_t out_ld_batch, int B, int c, int m_prime,
+                         int64_t entry_begin, int64_t entry_end, void* workspace,
+                         size_t ws_bytes, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * csa_indexer_topk - lightning-indexer scores and top-k selection ([P1] section 6.4
  * boxed score, section 7 selection and causal rule; [P4] section 6.2.2 indexer).
  *

@@ -23,6 +23,8 @@ _SIGS = {
     "csa_compress": ([vp, vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, i64, i32, i32, i32, i64, i64,
                       i32, vp], i32),
     "hca_compress": ([vp, vp, i64, i64, i64, i64, vp, vp, i64, i32, i32, i32, i64, i64, i32, vp], i32),
+    "hca_project_compress": ([vp, i64, i64, i64, i64, vp, vp, i32, vp, vp, i64, i32, i32, i32, i64, i64, vp, sz,
+                              vp], i32),
     "csa_indexer_topk_workspace_size": ([i32, i32, i64, i32], sz),
     "csa_workspace_status": ([vp, vp], i32),
     "csa_indexer_topk": ([vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, i32, vp, vp, vp, sz, i32, vp],
@@ -146,6 +148,26 @@ def hca_compress(C, Z, out, m_prime, entry_begin=0, entry_end=None, Bias=None, t
     _check("hca_compress", library().hca_compress(
         _ptr(C), _ptr(Z), C.stride(1), C.stride(0), tok0, n, _ptr(Bias), _ptr(out), out.stride(0),
         B, c, m_prime, entry_begin, entry_end, _dtype(C), _stream(stream)))
+
+
+def hca_project_compress(H, Wc, Wz, out, m_prime, workspace, entry_begin=0, entry_end=None, Bias=None, tok0=0,
+                         stream=None):
+    """Fused HCA projection + compression into ``out[:, entry_begin:entry_end]``: H [B, rows, d]
+    bf16 token rows (token tok0 + r at row r), Wc and Wz [c, d] bf16 (output column j's weights
+    in row j), out [B, N', c] bf16, workspace >= 256 bytes (zeroed once)."""
+    _cuda(H, Wc, Wz, out, Bias, workspace)
+    B, rows, d = H.shape
+    c = Wc.shape[0]
+    assert Wc.shape == (c, d) and Wz.shape == (c, d) and Wc.is_contiguous() and Wz.is_contiguous()
+    assert H.stride(2) == 1 and out.stride(2) == 1 and H.dtype == Wc.dtype == Wz.dtype == out.dtype
+    n = tok0 + rows
+    if entry_end is None:
+        entry_end = n // m_prime
+    assert out.shape[0] == B and out.shape[2] == c and out.shape[1] >= entry_end
+    _check("hca_project_compress", library().hca_project_compress(
+        _ptr(H), H.stride(1), H.stride(0), tok0, n, _ptr(Wc), _ptr(Wz), d, _ptr(Bias), _ptr(out), out.stride(0),
+        B, c, m_prime, entry_begin, entry_end, _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
 
 
 def csa_indexer_topk_workspace_size(B, nq, N_cap, k) -> int:

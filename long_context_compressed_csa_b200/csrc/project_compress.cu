@@ -1,0 +1,291 @@
+// Fused HCA projection + compression on tcgen05 ("DeepSeek-V4 Hybrid Attention: CSA and
+// HCA from Scratch", section 10: one KV stream C = H W^KV and its pooling logits
+// Z = H W^Z, then the boxed per-column softmax over the m' = 128 tokens of an entry and
+// the weighted sum; section 3 states the projections H W for the CSA streams).
+//
+// The projections are a dense GEMM over the model width d, and the pooling only needs,
+// per output column, the 128 values of C and Z of one entry.  The products are computed
+// transposed, columns on the MMA M dimension and tokens on N:
+//   D_C[j, r] = sum_k W_C[j, k] H[r, k],   D_Z[j, r] = sum_k W_Z[j, k] H[r, k]
+// so that TMEM lane j holds a whole entry's C and Z values of column j and the softmax
+// over the entry's tokens runs inside one thread, with no cross-thread reduction.
+//
+//   warp 0    TMA producer: per 64-wide K panel, a 128 x 64 tile of W_C and of W_Z and
+//             a 256 x 64 tile of H (two entries' tokens), 128-byte swizzle, into a ring;
+//   warp 1    MMA issuer: M = 128 columns, N = 256 tokens, K = 16, two accumulators
+//             (C in TMEM columns 0-255, Z in 256-511);
+//   warps 2-5 epilogue: thread = column; per entry an online softmax over its 128 tokens
+//             (32 at a time from TMEM), then one bf16 entry value per column.
+// CTAs are persistent over tiles (token block, column block) with the column blocks of
+// one token block consecutive, so the CTAs running at the same time share H tiles in L2.
+// C and Z never leave the chip.  Every wait is bounded; a timeout sets the workspace
+// status word and every role drains and exits.
+#include "common.cuh"
+#include "tc_utils.cuh"
+
+namespace csa {
+namespace {
+
+constexpr int kPcThreads = 192;                  // TMA warp, MMA warp, 4 epilogue warps
+constexpr int kPcCols = 128;                     // output columns per tile (MMA M)
+constexpr int kPcMp = 128;                       // tokens per entry (m')
+constexpr int kPcTokens = 2 * kPcMp;             // tokens per tile (MMA N): two entries
+constexpr int kPcWBytes = kPcCols * 128;         // one 128 x 64 weight panel: 16 KB
+constexpr int kPcHBytes = kPcTokens * 128;       // one 256 x 64 H panel: 32 KB
+constexpr int kPcStage = 2 * kPcWBytes + kPcHBytes;  // 64 KB
+constexpr int kPcStages = 3;
+constexpr int kPcSmem = 1024 + kPcStages * kPcStage + 256;
+static_assert((2 * kPcStages + 3) * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit 256 bytes");
+
+struct PcArgs {
+    int64_t rows_per_batch;  // H rows of one batch in the buffer (ld_batch / ld_row)
+    int64_t tok0;            // token of buffer row 0 of each batch
+    int d;                   // model width (K)
+    int c;                   // output columns
+    const float* bias;       // [m'][c] or null
+    __nv_bfloat16* out;      // entry i of batch b at out + b * out_ld_batch + i * c
+    int64_t out_ld_batch;
+    int64_t e0, e1;          // entries [e0, e1) of every batch
+    int n_cb;                // column blocks of 128
+    int64_t n_tb;            // token blocks (two entries) per batch
+    int64_t tiles;           // B * n_tb * n_cb
+    uint32_t* status;
+};
+
+CSA_DEV void pc_tile(const PcArgs& a, int64_t t, int& b, int64_t& tb, int& cb)
+{
+    cb = (int)(t % a.n_cb);
+    const int64_t r = t / a.n_cb;
+    tb = r % a.n_tb;
+    b = (int)(r / a.n_tb);
+}
+
+__global__ void __launch_bounds__(kPcThreads, 1)
+hca_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ CUtensorMap tmap_wc,
+                            const __grid_constant__ CUtensorMap tmap_wz, PcArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPcStages * kPcStage);
+    uint64_t* empty = full + kPcStages;
+    uint64_t* tfull = empty + kPcStages;   // MMA -> epilogue: the tile's accumulators are complete
+    uint64_t* tempty = tfull + 1;          // epilogue -> MMA: TMEM read out (count 128)
+    uint64_t* done = tempty + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    pdl_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPcStages; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        tc::mbar_init(tfull, 1);
+        tc::mbar_init(tempty, 128);
+        tc::mbar_init(done, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+        tc::tma_prefetch_desc(&tmap_h);
+        tc::tma_prefetch_desc(&tmap_wc);
+        tc::tma_prefetch_desc(&tmap_wz);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();
+
+    const int kpanels = a.d / 64;
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int it = 0;
+            bool stop = false;
+            for (int64_t t = blockIdx.x; t < a.tiles && !stop; t += gridDim.x) {
+                int b, cb;
+                int64_t tb;
+                pc_tile(a, t, b, tb, cb);
+                const int hrow = (int)(b * a.rows_per_batch + kPcMp * (a.e0 + 2 * tb) - a.tok0);
+                const int wrow = cb * kPcCols;
+                for (int kp = 0; kp < kpanels; ++kp, ++it) {
+                    const int s = it % kPcStages;
+                    const uint32_t ph = (it / kPcStages) & 1;
+                    if (*abort_flag || !tc::mbar_wait(&empty[s], ph ^ 1, tc::kWaitBudget)) {
+                        *abort_flag = 1;
+                        stop = true;
+                        break;
+                    }
+                    uint8_t* st = smem + s * kPcStage;
+                    tc::mbar_arrive_expect_tx(&full[s], kPcStage);
+                    tc::tma_load_2d(st, &tmap_wc, &full[s], kp * 64, wrow);
+                    tc::tma_load_2d(st + kPcWBytes, &tmap_wz, &full[s], kp * 64, wrow);
+                    tc::tma_load_2d(st + 2 * kPcWBytes, &tmap_h, &full[s], kp * 64, hrow);
+                }
+            }
+            // drain: every issued load has landed before the CTA may exit
+            for (int j = it - kPcStages < 0 ? 0 : it - kPcStages; j < it; ++j)
+                if (!tc::mbar_wait(&full[j % kPcStages], (j / kPcStages) & 1, tc::kWaitBudget)) *abort_flag = 1;
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdesc = tc::idesc_bf16_f32(kPcCols, kPcTokens, false, false);
+            int it = 0, nt = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < a.tiles && ok; t += gridDim.x, ++nt) {
+                if (!tc::mbar_wait(tempty, (nt & 1) ^ 1, tc::kWaitBudget)) {  // TMEM read out
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                for (int kp = 0; kp < kpanels; ++kp, ++it) {
+                    const int s = it % kPcStages;
+                    const uint32_t ph = (it / kPcStages) & 1;
+                    if (*abort_flag || !tc::mbar_wait(&full[s], ph, tc::kWaitBudget)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    const uint32_t wc = tc::smem_u32(smem + s * kPcStage);
+                    const uint32_t wz = wc + kPcWBytes;
+                    const uint32_t hh = wc + 2 * kPcWBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t bd = tc::smem_desc_sw128(hh + kk * 32, 16, 1024);
+                        const uint32_t acc = (kp | kk) ? 1u : 0u;
+                        tc::mma_bf16_ss(tmem, tc::smem_desc_sw128(wc + kk * 32, 16, 1024), bd, kIdesc, acc);
+                        tc::mma_bf16_ss(tmem + kPcTokens, tc::smem_desc_sw128(wz + kk * 32, 16, 1024), bd, kIdesc, acc);
+                    }
+                    tc::mma_commit(&empty[s]);  // the stage is free once these MMAs finish
+                }
+                if (!ok) break;
+                tc::mma_commit(tfull);          // the tile's C and Z accumulators are complete
+            }
+            if (!ok) *abort_flag = 1;
+            tc::mma_commit(done);               // all issued MMAs complete before TMEM is freed
+            if (!tc::mbar_wait(done, 0, tc::kWaitBudget)) *abort_flag = 1;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        constexpr float kLog2e = 1.4426950408889634f;
+        const int quarter = warp & 3;
+        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
+        int nt = 0;
+        for (int64_t t = blockIdx.x; t < a.tiles; t += gridDim.x, ++nt) {
+            if (*abort_flag || !tc::mbar_wait(tfull, nt & 1, tc::kWaitBudget)) {
+                *abort_flag = 1;
+                break;
+            }
+            tc::fence_after_sync();
+            int b, cb;
+            int64_t tb;
+            pc_tile(a, t, b, tb, cb);
+            const int j = cb * kPcCols + quarter * 32 + lane;  // this thread's output column
+            float res[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                // online softmax over the entry's 128 tokens, 32 at a time
+                float m = -INFINITY, l = 0.f, acc = 0.f;
+#pragma unroll 1
+                for (int c0 = 0; c0 < kPcMp; c0 += 32) {
+                    uint32_t zr[32], cr[32];
+                    tc::tmem_ld32_async(taddr + kPcTokens + e * kPcMp + c0, zr);
+                    tc::tmem_ld32_async(taddr + e * kPcMp + c0, cr);
+                    tc::tmem_wait_ld_regs(zr);
+                    tc::tmem_wait_ld_regs(cr);
+                    float z[32];
+                    float cmax = -INFINITY;
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        z[u] = __uint_as_float(zr[u]) + (a.bias ? __ldg(&a.bias[(int64_t)(c0 + u) * a.c + j]) : 0.f);
+                        cmax = fmaxf(cmax, z[u]);
+                    }
+                    const float mn = fmaxf(m, cmax);
+                    const float f = m == -INFINITY ? 0.f : exp2f((m - mn) * kLog2e);
+                    l *= f;
+                    acc *= f;
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const float p = exp2f((z[u] - mn) * kLog2e);
+                        l += p;
+                        acc = fmaf(p, __uint_as_float(cr[u]), acc);
+                    }
+                    m = mn;
+                }
+                res[e] = acc / l;
+            }
+            tc::fence_before_sync();
+            tc::mbar_arrive(tempty);  // TMEM read out: the next tile's MMAs may start
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int64_t i = a.e0 + 2 * tb + e;
+                if (i < a.e1) a.out[(int64_t)b * a.out_ld_batch + i * a.c + j] = __float2bfloat16_rn(res[e]);
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (*abort_flag && threadIdx.x == 0) atomicExch(a.status, 1u);
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace
+}  // namespace csa
+
+extern "C" int hca_project_compress(const void* H, int64_t ld_row, int64_t ld_batch, int64_t tok0, int64_t n,
+                                    const void* Wc, const void* Wz, int d, const float* Bias, void* out,
+                                    int64_t out_ld_batch, int B, int c, int m_prime, int64_t entry_begin,
+                                    int64_t entry_end, void* workspace, size_t ws_bytes, csa_stream_t stream_)
+{
+    using namespace csa;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (B < 0 || c <= 0 || d <= 0 || m_prime <= 0 || n < 0 || entry_begin < 0 || entry_end < entry_begin)
+        return CSA_ERR_ARG;
+    if ((int64_t)m_prime * entry_end > n || tok0 < 0 || tok0 > (int64_t)m_prime * entry_begin)
+        return CSA_ERR_ARG;
+    if (ld_row < d || ld_batch < (n - tok0) * ld_row || out_ld_batch < entry_end * c) return CSA_ERR_ARG;
+    if (m_prime != kPcMp || c % kPcCols != 0 || d % 64 != 0 || ld_row % 8 != 0 || ld_batch % ld_row != 0)
+        return CSA_ERR_UNSUPPORTED;
+    if (B == 0 || entry_end == entry_begin) return CSA_OK;
+    if (!H || !Wc || !Wz || !out || !workspace) return CSA_ERR_ARG;
+    if (!aligned16(H) || !aligned16(Wc) || !aligned16(Wz) || !aligned16(workspace) || ((uintptr_t)Bias & 3) ||
+        ((uintptr_t)out & 1))
+        return CSA_ERR_ALIGN;
+    if (ws_bytes < 256) return CSA_ERR_WORKSPACE;
+    PcArgs a;
+    a.rows_per_batch = ld_batch / ld_row;
+    if ((int64_t)B * a.rows_per_batch + kPcTokens >= (int64_t(1) << 31)) return CSA_ERR_UNSUPPORTED;
+    a.tok0 = tok0;
+    a.d = d;
+    a.c = c;
+    a.bias = Bias;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.out_ld_batch = out_ld_batch;
+    a.e0 = entry_begin;
+    a.e1 = entry_end;
+    a.n_cb = c / kPcCols;
+    a.n_tb = (entry_end - entry_begin + 1) / 2;
+    a.tiles = (int64_t)B * a.n_tb * a.n_cb;
+    a.status = static_cast<uint32_t*>(workspace);
+    CUtensorMap th, twc, twz;
+    if (!make_tmap_bf16_2d(&th, H, (uint64_t)B * a.rows_per_batch, d, ld_row, 64, kPcTokens) ||
+        !make_tmap_bf16_2d(&twc, Wc, c, d, d, 64, kPcCols) || !make_tmap_bf16_2d(&twz, Wz, c, d, d, 64, kPcCols))
+        return CSA_ERR_CUDA;
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t grid = a.tiles < sms ? a.tiles : sms;
+    cudaFuncSetAttribute(hca_project_compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPcSmem);
+    launch_pdl(hca_project_compress_kernel, dim3((unsigned)grid), dim3(kPcThreads), (size_t)kPcSmem, stream, th, twc,
+               twz, a);
+    return launch_status();
+}

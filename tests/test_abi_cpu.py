@@ -115,6 +115,16 @@ def test_host_validation_rejects_bad_arguments_without_launching(lib):
     assert lib.csa_quantize_e4m3(fake, 10, 8, 8, fake, fake, 9, None) == -3
     assert lib.csa_indexer_topk_e4m3(fake, fake, fake, fake, fake, 1, 1, 100, 64, 64, 4, 8, fake, None,
                                      fake, 1 << 30, None) == -6
+    # fused projection + HCA compression: m' other than 128, d not a multiple of 64,
+    # no workspace, a workspace too small
+    assert lib.hca_project_compress(fake, 64, 64 * 256, 0, 256, fake, fake, 64, None, fake, 1024, 1, 128, 64,
+                                    0, 4, fake, 256, None) == -6
+    assert lib.hca_project_compress(fake, 96, 96 * 256, 0, 256, fake, fake, 96, None, fake, 1024, 1, 128, 128,
+                                    0, 2, fake, 256, None) == -6
+    assert lib.hca_project_compress(fake, 64, 64 * 256, 0, 256, fake, fake, 64, None, fake, 1024, 1, 128, 128,
+                                    0, 2, None, 256, None) == -1
+    assert lib.hca_project_compress(fake, 64, 64 * 256, 0, 256, fake, fake, 64, None, fake, 1024, 1, 128, 128,
+                                    0, 2, fake, 16, None) == -4
     # empty problems succeed without touching memory
     assert lib.csa_compress(fake, fake, fake, fake, 8, 64, 0, 8, None, None, fake, 64, 0, 8, 4,
                             0, 2, 0, None) == 0

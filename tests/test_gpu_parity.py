@@ -115,6 +115,46 @@ def test_csa_compress_interleaved_layout_and_incremental_ranges():
         torch.testing.assert_close(part[:, i], full[:, i], rtol=0, atol=0)
 
 
+def _ref_project_compress(H, Wc, Wz, mp, Bias, i0, i1):
+    """Oracle of the fused call: the plain projections, then the HCA compressor."""
+    C = oracle.project(H, Wc.T)
+    Z = oracle.project(H, Wz.T)
+    return oracle.hca_compress(C, Z, mp, Bias, i0, i1)
+
+
+@pytest.mark.parametrize("B,rows,d,c,bias,e0,e1,tok0", [
+    (2, 128 * 5 + 40, 256, 256, True, 0, None, 0),   # odd entry count, a partial block at the end
+    (1, 128 * 6, 64, 128, False, 1, 4, 128),         # one K panel, one column block, a sub-range
+    (3, 128 * 7, 1024, 512, True, 0, None, 0),       # several K panels and column blocks
+])
+def test_hca_project_compress_matches_oracle(B, rows, d, c, bias, e0, e1, tok0):
+    """Fused projection + HCA compression: C = H Wc^T and Z = H Wz^T in fp32 on the tensor
+    cores, never stored, then the per-column softmax pooling over each entry's 128
+    tokens, against the oracle's plain projections followed by its HCA compressor."""
+    from long_context_compressed_csa_b200 import hca_project_compress
+    mp = 128
+    H = randn((B, rows, d), 480, torch.bfloat16, scale=d ** -0.25)
+    Wc = randn((c, d), 481, torch.bfloat16, scale=d ** -0.25)
+    Wz = randn((c, d), 482, torch.bfloat16, scale=d ** -0.25)
+    Bias = randn((mp, c), 483, torch.float32) if bias else None
+    n = tok0 + rows
+    e1 = n // mp if e1 is None else e1
+    out = torch.full((B, n // mp + 1, c), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    hca_project_compress(dev(H), dev(Wc), dev(Wz), out, mp, ws, entry_begin=e0, entry_end=e1,
+                         Bias=dev(Bias) if bias else None, tok0=tok0)
+    torch.cuda.synchronize()
+    assert csa_workspace_status(ws) == 0
+    got = out.float().cpu().numpy()
+    for b in range(B):
+        # the oracle sees the tokens from 0: rows before tok0 are not read, so pad them
+        Hb = np.zeros((n, d))
+        Hb[tok0:] = to_f64(H[b])
+        ref = _ref_project_compress(Hb, to_f64(Wc), to_f64(Wz), mp, to_f64(Bias) if bias else None, e0, e1)
+        assert max_rel_rowwise(got[b, e0:e1], ref).max() <= TOL[torch.bfloat16]
+        assert np.all(np.isnan(got[b, :e0])) and np.all(np.isnan(got[b, e1:]))
+
+
 @pytest.mark.parametrize("dtype,c,mp", [(torch.bfloat16, 512, 128), (torch.float32, 64, 128),
                                         (torch.bfloat16, 24, 5)])
 def test_hca_compress_random(dtype, c, mp):
