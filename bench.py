@@ -298,7 +298,7 @@ def cpu_baseline(n_steps=2, seed=77):
 # ----------------------------------------------------------------------------------
 # single-kernel micro runs (profiling and per-kernel rooflines)
 # ----------------------------------------------------------------------------------
-def micro(kind, iters, rotate=4, nq_prefill=1024):
+def micro(kind, iters, rotate=4, nq_prefill=1024, batch=16):
     """Time one entry point alone on the 1M workload's shapes (compress kernels on the
     B=16 x 128K HCA and B=4 x 256K CSA prefill shapes), rotating over `rotate` input
     sets so repeated launches do not hit L2.  Prints one JSON line (not the bench line)."""
@@ -406,6 +406,17 @@ def micro(kind, iters, rotate=4, nq_prefill=1024):
         out = torch.empty((B, nn // mp, c), dtype=bf16, device=dev)
         calls = [lambda: lib.hca_compress(C, Z, out, mp)]
         nbytes = 2 * B * nn * c * 2 + B * (nn // mp) * c * 2
+    elif kind == "hca_project_compress":
+        # fused projection + HCA compression over the HCA prefill shape (B = 16 x 128K
+        # tokens) with model width d = 4096 (not given by the pages); flops 2 * d * 2c per token
+        B, nn, d = batch, 131072, 4096
+        H = randn((B, nn, d), 970, bf16, dev, scale=d ** -0.25)
+        Wc, Wz = randn((c, d), 971, bf16, dev, scale=d ** -0.25), randn((c, d), 972, bf16, dev, scale=d ** -0.25)
+        out = torch.empty((B, nn // mp, c), dtype=bf16, device=dev)
+        ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+        calls = [lambda: lib.hca_project_compress(H, Wc, Wz, out, mp, ws)]
+        nbytes = B * nn * d * 2 + 2 * c * d * 2 + B * (nn // mp) * c * 2
+        flops = 2 * B * nn * d * 2 * c
     elif kind == "csa_compress":
         B, nn = 4, 262144
         S = [randn((B, nn, c), 960 + i, bf16, dev) for i in range(4)]
@@ -440,8 +451,10 @@ def micro(kind, iters, rotate=4, nq_prefill=1024):
             "frac": gbs / hbm, "peak_source": src}
     if flops:
         tfs = flops / (np.median(us) * 1e-6) / 1e12
-        line.update({"queries": nq_prefill, "algorithmic_flops": flops, "achieved_tflops": tfs,
-                     "peak_tflops": tf, "tensor_frac": tfs / tf})
+        line.update({"algorithmic_flops": flops, "achieved_tflops": tfs, "peak_tflops": tf,
+                     "tensor_frac": tfs / tf})
+        if kind.endswith("_prefill"):
+            line["queries"] = nq_prefill
     print(json.dumps(line), flush=True)
     return 0
 
@@ -458,13 +471,15 @@ def main():
     ap.add_argument("--micro", default=None,
                     help="time one entry point alone: indexer, indexer_e4m3, indexer_prefill, "
                          "sparse, sparse_prefill, dense, sparse_window, dense_window, csa_compress, "
-                         "hca_compress")
+                         "hca_compress, hca_project_compress")
     ap.add_argument("--nq", type=int, default=1024,
                     help="query positions of the indexer_prefill / sparse_prefill chunk")
+    ap.add_argument("--batch", type=int, default=16,
+                    help="sequences of the hca_project_compress micro-benchmark")
     ap.add_argument("--iters", type=int, default=20)
     args = ap.parse_args()
     if args.micro:
-        return micro(args.micro, args.iters, nq_prefill=args.nq)
+        return micro(args.micro, args.iters, nq_prefill=args.nq, batch=args.batch)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -185,3 +185,24 @@ def test_hybrid_1m_decode_step():
     assert max_rel_rowwise(o[0, 0].cpu().numpy(), ref_o).max() <= 2e-2
     ref_h, _ = oracle.mqa(to_f64(q[0, 0]), to_f64(hcache[0]), np.arange(Nh, dtype=np.int32))
     assert max_rel_rowwise(oh[0, 0].cpu().numpy(), ref_h).max() <= 2e-2
+
+
+def test_hca_project_compress_b16_128k_sampled():
+    """The fused projection + HCA compression at the micro-benchmark's launch: B = 16
+    sequences of 131072 tokens, model width d = 4096, c = 512 (1024 entries each).
+    Sampled entries are recomputed by the oracle's projections and HCA compressor."""
+    B, n, d, c, mp = 16, 131072, 4096, 512, 128
+    H = randn((B, n, d), 970, BF16, DEV, scale=d ** -0.25)
+    Wc = randn((c, d), 971, BF16, DEV, scale=d ** -0.25)
+    Wz = randn((c, d), 972, BF16, DEV, scale=d ** -0.25)
+    Bias = randn((mp, c), 973, torch.float32, DEV)
+    out = torch.empty((B, n // mp, c), dtype=BF16, device=DEV)
+    ws = zeros_ws(256)
+    lib.hca_project_compress(H, Wc, Wz, out, mp, ws, Bias=Bias)
+    torch.cuda.synchronize()
+    assert lib.csa_workspace_status(ws) == 0
+    Wc64, Wz64, B64 = to_f64(Wc), to_f64(Wz), to_f64(Bias)
+    for b, i in ((0, 0), (3, 511), (7, 1), (15, 1023), (9, 700)):
+        rows = to_f64(H[b, mp * i:mp * (i + 1)])
+        ref = oracle.hca_compress(oracle.project(rows, Wc64.T), oracle.project(rows, Wz64.T), mp, B64, 0, 1)
+        assert max_rel_rowwise(to_f64(out[b, i:i + 1]), ref).max() <= 2e-2, (b, i)
