@@ -135,6 +135,28 @@ int hca_project_compress(const void* H, int64_t ld_row, int64_t ld_batch, int64_
                          size_t ws_bytes, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * csa_project_compress - csa_compress fused with the four projections that produce its
+ * streams ([P1] section 3: C^a = H W^{aKV}, C^b = H W^{bKV}, Z^a = H W^{aZ},
+ * Z^b = H W^{bZ}; sections 4-5: the overlapped 2m-logit softmax and weighted sum, entry 0
+ * without a b-part).  The streams are computed on the tensor cores in fp32 and never
+ * written to memory.
+ *
+ * H      : bf16 token rows as for hca_project_compress; rows m*(entry_begin-1) (m*0 for
+ *          entry_begin = 0) .. m*entry_end - 1 are read (tok0 <= the first of them).
+ * Wa_kv, Wb_kv, Wa_z, Wb_z : bf16 [c, d], row j holds output column j's weights.
+ * Ba, Bb : fp32 [m, c] or NULL.
+ * out, workspace : as for hca_project_compress.
+ * Supported: m = 4, c a multiple of 128, d a multiple of 64; CSA_ERR_UNSUPPORTED
+ * otherwise.
+ * ------------------------------------------------------------------------------- */
+int csa_project_compress(const void* H, int64_t ld_row, int64_t ld_batch, int64_t tok0,
+                         int64_t n, const void* Wa_kv, const void* Wb_kv, const void* Wa_z,
+                         const void* Wb_z, int d, const float* Ba, const float* Bb, void* out,
+                         int64_t out_ld_batch, int B, int c, int m, int64_t entry_begin,
+                         int64_t entry_end, void* workspace, size_t ws_bytes,
+                         csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * csa_indexer_topk - lightning-indexer scores and top-k selection ([P1] section 6.4
  * boxed score, section 7 selection and causal rule; [P4] section 6.2.2 indexer).
  *

@@ -24,6 +24,7 @@ from ._binding import (  # noqa: F401
     csa_workspace_zero,
     hca_compress,
     hca_project_compress,
+    csa_project_compress,
     hca_dense_attn,
     library,
     library_path,

@@ -25,6 +25,8 @@ _SIGS = {
     "hca_compress": ([vp, vp, i64, i64, i64, i64, vp, vp, i64, i32, i32, i32, i64, i64, i32, vp], i32),
     "hca_project_compress": ([vp, i64, i64, i64, i64, vp, vp, i32, vp, vp, i64, i32, i32, i32, i64, i64, vp, sz,
                               vp], i32),
+    "csa_project_compress": ([vp, i64, i64, i64, i64, vp, vp, vp, vp, i32, vp, vp, vp, i64, i32, i32, i32, i64, i64,
+                              vp, sz, vp], i32),
     "csa_indexer_topk_workspace_size": ([i32, i32, i64, i32], sz),
     "csa_workspace_status": ([vp, vp], i32),
     "csa_indexer_topk": ([vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, i32, vp, vp, vp, sz, i32, vp],
@@ -168,6 +170,27 @@ def hca_project_compress(H, Wc, Wz, out, m_prime, workspace, entry_begin=0, entr
         _ptr(H), H.stride(1), H.stride(0), tok0, n, _ptr(Wc), _ptr(Wz), d, _ptr(Bias), _ptr(out), out.stride(0),
         B, c, m_prime, entry_begin, entry_end, _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)))
+
+
+def csa_project_compress(H, Wa_kv, Wb_kv, Wa_z, Wb_z, out, m, workspace, entry_begin=0, entry_end=None, Ba=None,
+                         Bb=None, tok0=0, stream=None):
+    """Fused CSA projections + overlapped compression into ``out[:, entry_begin:entry_end]``:
+    H [B, rows, d] bf16 (token tok0 + r at row r), the four weights [c, d] bf16 (output column
+    j's weights in row j), out [B, N, c] bf16, workspace >= 256 bytes (zeroed once)."""
+    _cuda(H, Wa_kv, Wb_kv, Wa_z, Wb_z, out, Ba, Bb, workspace)
+    B, rows, d = H.shape
+    c = Wa_kv.shape[0]
+    for W in (Wa_kv, Wb_kv, Wa_z, Wb_z):
+        assert W.shape == (c, d) and W.is_contiguous() and W.dtype == H.dtype
+    assert H.stride(2) == 1 and out.stride(2) == 1 and out.dtype == H.dtype
+    n = tok0 + rows
+    if entry_end is None:
+        entry_end = n // m
+    assert out.shape[0] == B and out.shape[2] == c and out.shape[1] >= entry_end
+    _check("csa_project_compress", library().csa_project_compress(
+        _ptr(H), H.stride(1), H.stride(0), tok0, n, _ptr(Wa_kv), _ptr(Wb_kv), _ptr(Wa_z), _ptr(Wb_z), d,
+        _ptr(Ba), _ptr(Bb), _ptr(out), out.stride(0), B, c, m, entry_begin, entry_end, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def csa_indexer_topk_workspace_size(B, nq, N_cap, k) -> int:

@@ -238,6 +238,238 @@ hca_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __
     }
 }
 
+// ---------------------------------------------------------------------------------
+// CSA form ([P1] sections 3-5): four projections C^a = H W_a^KV, C^b = H W_b^KV,
+// Z^a = H W_a^Z, Z^b = H W_b^Z, then for entry i and column j the softmax over the 2m = 8
+// logits Z^a of block i (+ B^a) and Z^b of block i - 1 (+ B^b), and the weighted sum of
+// the matching C^a and C^b values; entry 0 has no b-part.  With m = 4, a tile of 128
+// tokens holds 32 blocks; block 0 only serves as the b-part of the tile's first entry,
+// so a tile yields 31 entries and consecutive tiles overlap by one block.  Four
+// accumulators of 128 tokens fill the 512 TMEM columns: C^a 0-127, C^b 128-255, Z^a
+// 256-383, Z^b 384-511.
+constexpr int kCsM = 4;                          // tokens per CSA block
+constexpr int kCsTokens = 128;                   // tokens per tile (MMA N)
+constexpr int kCsEntries = kCsTokens / kCsM - 1; // 31 entries per tile
+constexpr int kCsHBytes = kCsTokens * 128;       // one 128 x 64 H panel: 16 KB
+constexpr int kCsStage = 4 * kPcWBytes + kCsHBytes;  // 80 KB
+constexpr int kCsStages = 2;
+constexpr int kCsSmem = 1024 + kCsStages * kCsStage + 256;
+
+struct CsArgs {
+    int64_t rows_per_batch, tok0;
+    int d, c;
+    const float* ba;         // [m][c] or null
+    const float* bb;         // [m][c] or null
+    __nv_bfloat16* out;
+    int64_t out_ld_batch;
+    int64_t e0, e1;
+    int n_cb;
+    int64_t n_tb;            // tiles of 31 entries per batch
+    int64_t tiles;
+    uint32_t* status;
+};
+
+__global__ void __launch_bounds__(kPcThreads, 1)
+csa_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ CUtensorMap tmap_w0,
+                            const __grid_constant__ CUtensorMap tmap_w1, const __grid_constant__ CUtensorMap tmap_w2,
+                            const __grid_constant__ CUtensorMap tmap_w3, CsArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kCsStages * kCsStage);
+    uint64_t* empty = full + kCsStages;
+    uint64_t* tfull = empty + kCsStages;
+    uint64_t* tempty = tfull + 1;
+    uint64_t* done = tempty + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    pdl_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kCsStages; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        tc::mbar_init(tfull, 1);
+        tc::mbar_init(tempty, 128);
+        tc::mbar_init(done, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+        tc::tma_prefetch_desc(&tmap_h);
+        tc::tma_prefetch_desc(&tmap_w0);
+        tc::tma_prefetch_desc(&tmap_w1);
+        tc::tma_prefetch_desc(&tmap_w2);
+        tc::tma_prefetch_desc(&tmap_w3);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();
+
+    const int kpanels = a.d / 64;
+    auto tile_of = [&](int64_t t, int& b, int64_t& tb, int& cb) {
+        cb = (int)(t % a.n_cb);
+        const int64_t r = t / a.n_cb;
+        tb = r % a.n_tb;
+        b = (int)(r / a.n_tb);
+    };
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const CUtensorMap* wmaps[4] = {&tmap_w0, &tmap_w1, &tmap_w2, &tmap_w3};
+            int it = 0;
+            bool stop = false;
+            for (int64_t t = blockIdx.x; t < a.tiles && !stop; t += gridDim.x) {
+                int b, cb;
+                int64_t tb;
+                tile_of(t, b, tb, cb);
+                // block 0 of the tile is block (first entry - 1); rows before the batch's
+                // first token (entry 0) are read but never used
+                const int hrow = (int)(b * a.rows_per_batch + kCsM * (a.e0 + kCsEntries * tb - 1) - a.tok0);
+                const int wrow = cb * kPcCols;
+                for (int kp = 0; kp < kpanels; ++kp, ++it) {
+                    const int s = it % kCsStages;
+                    const uint32_t ph = (it / kCsStages) & 1;
+                    if (*abort_flag || !tc::mbar_wait(&empty[s], ph ^ 1, tc::kWaitBudget)) {
+                        *abort_flag = 1;
+                        stop = true;
+                        break;
+                    }
+                    uint8_t* st = smem + s * kCsStage;
+                    tc::mbar_arrive_expect_tx(&full[s], kCsStage);
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) tc::tma_load_2d(st + w * kPcWBytes, wmaps[w], &full[s], kp * 64, wrow);
+                    tc::tma_load_2d(st + 4 * kPcWBytes, &tmap_h, &full[s], kp * 64, hrow);
+                }
+            }
+            for (int j = it - kCsStages < 0 ? 0 : it - kCsStages; j < it; ++j)
+                if (!tc::mbar_wait(&full[j % kCsStages], (j / kCsStages) & 1, tc::kWaitBudget)) *abort_flag = 1;
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdesc = tc::idesc_bf16_f32(kPcCols, kCsTokens, false, false);
+            int it = 0, nt = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < a.tiles && ok; t += gridDim.x, ++nt) {
+                if (!tc::mbar_wait(tempty, (nt & 1) ^ 1, tc::kWaitBudget)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                for (int kp = 0; kp < kpanels; ++kp, ++it) {
+                    const int s = it % kCsStages;
+                    const uint32_t ph = (it / kCsStages) & 1;
+                    if (*abort_flag || !tc::mbar_wait(&full[s], ph, tc::kWaitBudget)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    const uint32_t w0 = tc::smem_u32(smem + s * kCsStage);
+                    const uint32_t hh = w0 + 4 * kPcWBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t bd = tc::smem_desc_sw128(hh + kk * 32, 16, 1024);
+                        const uint32_t acc = (kp | kk) ? 1u : 0u;
+#pragma unroll
+                        for (int w = 0; w < 4; ++w)
+                            tc::mma_bf16_ss(tmem + w * kCsTokens, tc::smem_desc_sw128(w0 + w * kPcWBytes + kk * 32, 16, 1024),
+                                            bd, kIdesc, acc);
+                    }
+                    tc::mma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                tc::mma_commit(tfull);
+            }
+            if (!ok) *abort_flag = 1;
+            tc::mma_commit(done);
+            if (!tc::mbar_wait(done, 0, tc::kWaitBudget)) *abort_flag = 1;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        constexpr float kLog2e = 1.4426950408889634f;
+        const int quarter = warp & 3;
+        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
+        int nt = 0;
+        for (int64_t t = blockIdx.x; t < a.tiles; t += gridDim.x, ++nt) {
+            if (*abort_flag || !tc::mbar_wait(tfull, nt & 1, tc::kWaitBudget)) {
+                *abort_flag = 1;
+                break;
+            }
+            tc::fence_after_sync();
+            int b, cb;
+            int64_t tb;
+            tile_of(t, b, tb, cb);
+            const int j = cb * kPcCols + quarter * 32 + lane;
+            float ba[kCsM], bb[kCsM];
+#pragma unroll
+            for (int r = 0; r < kCsM; ++r) {
+                ba[r] = a.ba ? __ldg(&a.ba[r * a.c + j]) : 0.f;
+                bb[r] = a.bb ? __ldg(&a.bb[r * a.c + j]) : 0.f;
+            }
+            const int64_t first = a.e0 + kCsEntries * tb;  // entry of tile block 1
+            __nv_bfloat16* orow = a.out + (int64_t)b * a.out_ld_batch + j;
+            float pcb[kCsM], pzb[kCsM];  // C^b, Z^b of the previous block
+#pragma unroll 1
+            for (int t0 = 0; t0 < kCsTokens; t0 += 16) {
+                uint32_t r_ca[16], r_cb[16], r_za[16], r_zb[16];
+                tc::tmem_ld16(taddr + 0 * kCsTokens + t0, reinterpret_cast<float*>(r_ca));
+                tc::tmem_ld16(taddr + 1 * kCsTokens + t0, reinterpret_cast<float*>(r_cb));
+                tc::tmem_ld16(taddr + 2 * kCsTokens + t0, reinterpret_cast<float*>(r_za));
+                tc::tmem_ld16(taddr + 3 * kCsTokens + t0, reinterpret_cast<float*>(r_zb));
+                tc::tmem_wait_ld();
+                if (t0 + 16 == kCsTokens) {  // the whole tile is in registers: the MMA may go on
+                    tc::fence_before_sync();
+                    tc::mbar_arrive(tempty);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {  // the 4 blocks of these 16 tokens
+                    const int kb = t0 / kCsM + q;  // tile block
+                    if (kb > 0) {
+                        const int64_t i = first + kb - 1;  // entry: a-part block kb, b-part block kb - 1
+                        float za[kCsM], zb[kCsM], mx = -INFINITY;
+#pragma unroll
+                        for (int r = 0; r < kCsM; ++r) {
+                            za[r] = __uint_as_float(r_za[q * kCsM + r]) + ba[r];
+                            zb[r] = i > 0 ? pzb[r] + bb[r] : -INFINITY;  // entry 0 has no b-part
+                            mx = fmaxf(mx, fmaxf(za[r], zb[r]));
+                        }
+                        float l = 0.f, acc = 0.f;
+#pragma unroll
+                        for (int r = 0; r < kCsM; ++r) {
+                            const float pa = exp2f((za[r] - mx) * kLog2e);
+                            const float pb = i > 0 ? exp2f((zb[r] - mx) * kLog2e) : 0.f;
+                            l += pa + pb;
+                            acc = fmaf(pa, __uint_as_float(r_ca[q * kCsM + r]), acc);
+                            if (i > 0) acc = fmaf(pb, pcb[r], acc);
+                        }
+                        if (i < a.e1) orow[i * a.c] = __float2bfloat16_rn(acc / l);
+                    }
+#pragma unroll
+                    for (int r = 0; r < kCsM; ++r) {
+                        pcb[r] = __uint_as_float(r_cb[q * kCsM + r]);
+                        pzb[r] = __uint_as_float(r_zb[q * kCsM + r]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (*abort_flag && threadIdx.x == 0) atomicExch(a.status, 1u);
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
 }  // namespace
 }  // namespace csa
 
@@ -287,5 +519,57 @@ extern "C" int hca_project_compress(const void* H, int64_t ld_row, int64_t ld_ba
     cudaFuncSetAttribute(hca_project_compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPcSmem);
     launch_pdl(hca_project_compress_kernel, dim3((unsigned)grid), dim3(kPcThreads), (size_t)kPcSmem, stream, th, twc,
                twz, a);
+    return launch_status();
+}
+
+extern "C" int csa_project_compress(const void* H, int64_t ld_row, int64_t ld_batch, int64_t tok0, int64_t n,
+                                    const void* Wa_kv, const void* Wb_kv, const void* Wa_z, const void* Wb_z, int d,
+                                    const float* Ba, const float* Bb, void* out, int64_t out_ld_batch, int B, int c,
+                                    int m, int64_t entry_begin, int64_t entry_end, void* workspace, size_t ws_bytes,
+                                    csa_stream_t stream_)
+{
+    using namespace csa;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (B < 0 || c <= 0 || d <= 0 || m <= 0 || n < 0 || entry_begin < 0 || entry_end < entry_begin || tok0 < 0)
+        return CSA_ERR_ARG;
+    const int64_t first_row = entry_begin == 0 ? 0 : (int64_t)m * (entry_begin - 1);
+    if ((int64_t)m * entry_end > n || (entry_end > entry_begin && tok0 > first_row)) return CSA_ERR_ARG;
+    if (ld_row < d || ld_batch < (n - tok0) * ld_row || out_ld_batch < entry_end * c) return CSA_ERR_ARG;
+    if (m != kCsM || c % kPcCols != 0 || d % 64 != 0 || ld_row % 8 != 0 || ld_batch % ld_row != 0)
+        return CSA_ERR_UNSUPPORTED;
+    if (B == 0 || entry_end == entry_begin) return CSA_OK;
+    if (!H || !Wa_kv || !Wb_kv || !Wa_z || !Wb_z || !out || !workspace) return CSA_ERR_ARG;
+    if (!aligned16(H) || !aligned16(Wa_kv) || !aligned16(Wb_kv) || !aligned16(Wa_z) || !aligned16(Wb_z) ||
+        !aligned16(workspace) || (((uintptr_t)Ba | (uintptr_t)Bb) & 3) || ((uintptr_t)out & 1))
+        return CSA_ERR_ALIGN;
+    if (ws_bytes < 256) return CSA_ERR_WORKSPACE;
+    CsArgs a;
+    a.rows_per_batch = ld_batch / ld_row;
+    if ((int64_t)B * a.rows_per_batch + kCsTokens >= (int64_t(1) << 31)) return CSA_ERR_UNSUPPORTED;
+    a.tok0 = tok0;
+    a.d = d;
+    a.c = c;
+    a.ba = Ba;
+    a.bb = Bb;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.out_ld_batch = out_ld_batch;
+    a.e0 = entry_begin;
+    a.e1 = entry_end;
+    a.n_cb = c / kPcCols;
+    a.n_tb = (entry_end - entry_begin + kCsEntries - 1) / kCsEntries;
+    a.tiles = (int64_t)B * a.n_tb * a.n_cb;
+    a.status = static_cast<uint32_t*>(workspace);
+    CUtensorMap th, tw[4];
+    const void* ws4[4] = {Wa_kv, Wb_kv, Wa_z, Wb_z};
+    if (!make_tmap_bf16_2d(&th, H, (uint64_t)B * a.rows_per_batch, d, ld_row, 64, kCsTokens)) return CSA_ERR_CUDA;
+    for (int w = 0; w < 4; ++w)
+        if (!make_tmap_bf16_2d(&tw[w], ws4[w], c, d, d, 64, kPcCols)) return CSA_ERR_CUDA;
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t grid = a.tiles < sms ? a.tiles : sms;
+    cudaFuncSetAttribute(csa_project_compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCsSmem);
+    launch_pdl(csa_project_compress_kernel, dim3((unsigned)grid), dim3(kPcThreads), (size_t)kCsSmem, stream, th,
+               tw[0], tw[1], tw[2], tw[3], a);
     return launch_status();
 }

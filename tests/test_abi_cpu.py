@@ -125,6 +125,11 @@ def test_host_validation_rejects_bad_arguments_without_launching(lib):
                                     0, 2, None, 256, None) == -1
     assert lib.hca_project_compress(fake, 64, 64 * 256, 0, 256, fake, fake, 64, None, fake, 1024, 1, 128, 128,
                                     0, 2, fake, 16, None) == -4
+    # fused CSA projections + compression: m other than 4, tok0 after the first row read
+    assert lib.csa_project_compress(fake, 64, 64 * 256, 0, 256, fake, fake, fake, fake, 64, None, None, fake,
+                                    1024, 1, 128, 8, 0, 4, fake, 256, None) == -6
+    assert lib.csa_project_compress(fake, 64, 64 * 256, 16, 256, fake, fake, fake, fake, 64, None, None, fake,
+                                    1024, 1, 128, 4, 2, 8, fake, 256, None) == -1
     # empty problems succeed without touching memory
     assert lib.csa_compress(fake, fake, fake, fake, 8, 64, 0, 8, None, None, fake, 64, 0, 8, 4,
                             0, 2, 0, None) == 0

@@ -123,6 +123,41 @@ def _ref_project_compress(H, Wc, Wz, mp, Bias, i0, i1):
 
 
 @pytest.mark.parametrize("B,rows,d,c,bias,e0,e1,tok0", [
+    (2, 4 * 70 + 3, 256, 256, True, 0, None, 0),      # 3 tiles of 31 entries (the last partial)
+    (1, 4 * 60, 64, 128, False, 5, 40, 16),           # a sub-range, tok0 at block e0 - 1
+    (3, 4 * 100, 1024, 512, True, 0, None, 0),        # several K panels and column blocks
+])
+def test_csa_project_compress_matches_oracle(B, rows, d, c, bias, e0, e1, tok0):
+    """Fused CSA projections + overlapped compression: the four streams H W^T in fp32 on
+    the tensor cores, never stored, then the 2m-logit softmax of entry i over block i
+    (a-part) and block i - 1 (b-part; none for entry 0), against the oracle's plain
+    projections followed by its CSA compressor."""
+    from long_context_compressed_csa_b200 import csa_project_compress
+    m = 4
+    H = randn((B, rows, d), 490, torch.bfloat16, scale=d ** -0.25)
+    Ws = [randn((c, d), 491 + w, torch.bfloat16, scale=d ** -0.25) for w in range(4)]
+    Ba = randn((m, c), 495, torch.float32) if bias else None
+    Bb = randn((m, c), 496, torch.float32) if bias else None
+    n = tok0 + rows
+    e1 = n // m if e1 is None else e1
+    out = torch.full((B, n // m + 1, c), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    csa_project_compress(dev(H), *[dev(W) for W in Ws], out, m, ws, entry_begin=e0, entry_end=e1,
+                         Ba=dev(Ba) if bias else None, Bb=dev(Bb) if bias else None, tok0=tok0)
+    torch.cuda.synchronize()
+    assert csa_workspace_status(ws) == 0
+    got = out.float().cpu().numpy()
+    W64 = [to_f64(W).T for W in Ws]
+    for b in range(B):
+        Hb = np.zeros((n, d))
+        Hb[tok0:] = to_f64(H[b])
+        streams = [oracle.project(Hb, W) for W in W64]
+        ref = oracle.csa_compress(*streams, m, to_f64(Ba) if bias else None, to_f64(Bb) if bias else None, e0, e1)
+        assert max_rel_rowwise(got[b, e0:e1], ref).max() <= TOL[torch.bfloat16]
+        assert np.all(np.isnan(got[b, :e0])) and np.all(np.isnan(got[b, e1:]))
+
+
+@pytest.mark.parametrize("B,rows,d,c,bias,e0,e1,tok0", [
     (2, 128 * 5 + 40, 256, 256, True, 0, None, 0),   # odd entry count, a partial block at the end
     (1, 128 * 6, 64, 128, False, 1, 4, 128),         # one K panel, one column block, a sub-range
     (3, 128 * 7, 1024, 512, True, 0, None, 0),       # several K panels and column blocks
