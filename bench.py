@@ -417,6 +417,17 @@ def micro(kind, iters, rotate=4, nq_prefill=1024, batch=16):
         calls = [lambda: lib.hca_project_compress(H, Wc, Wz, out, mp, ws)]
         nbytes = B * nn * d * 2 + 2 * c * d * 2 + B * (nn // mp) * c * 2
         flops = 2 * B * nn * d * 2 * c
+    elif kind == "csa_project_compress":
+        # fused CSA projections + compression over the CSA prefill shape (B = 4 x 256K
+        # tokens), d = 4096; flops 2 * d * 4c per token
+        B, nn, d = batch, 262144, 4096
+        H = randn((B, nn, d), 980, bf16, dev, scale=d ** -0.25)
+        Ws = [randn((c, d), 981 + w, bf16, dev, scale=d ** -0.25) for w in range(4)]
+        out = torch.empty((B, nn // m, c), dtype=bf16, device=dev)
+        ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+        calls = [lambda: lib.csa_project_compress(H, *Ws, out, m, ws)]
+        nbytes = B * nn * d * 2 + 4 * c * d * 2 + B * (nn // m) * c * 2
+        flops = 2 * B * nn * d * 4 * c
     elif kind == "csa_compress":
         B, nn = 4, 262144
         S = [randn((B, nn, c), 960 + i, bf16, dev) for i in range(4)]
@@ -471,15 +482,16 @@ def main():
     ap.add_argument("--micro", default=None,
                     help="time one entry point alone: indexer, indexer_e4m3, indexer_prefill, "
                          "sparse, sparse_prefill, dense, sparse_window, dense_window, csa_compress, "
-                         "hca_compress, hca_project_compress")
+                         "hca_compress, hca_project_compress, csa_project_compress")
     ap.add_argument("--nq", type=int, default=1024,
                     help="query positions of the indexer_prefill / sparse_prefill chunk")
-    ap.add_argument("--batch", type=int, default=16,
-                    help="sequences of the hca_project_compress micro-benchmark")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences of the *_project_compress micro-benchmarks (16 HCA, 4 CSA)")
     ap.add_argument("--iters", type=int, default=20)
     args = ap.parse_args()
     if args.micro:
-        return micro(args.micro, args.iters, nq_prefill=args.nq, batch=args.batch)
+        bdef = 4 if args.micro == "csa_project_compress" else 16
+        return micro(args.micro, args.iters, nq_prefill=args.nq, batch=args.batch or bdef)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
