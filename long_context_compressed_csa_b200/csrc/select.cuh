@@ -133,8 +133,12 @@ CSA_DEV uint32_t warp_append(uint32_t* ctr, bool pred)
 
 // Radix digits of the 64-bit key (kv.x << 32) | ~kv.y: level 0 = bits 63..52, level 1 =
 // bits 51..40 (12-bit digits), levels 2..6 = 8-bit digits from bit 39 down to bit 0.
-CSA_DEV uint32_t digit_shift(int level) { return level == 0 ? 52u : level == 1 ? 40u : (uint32_t)(48 - 8 * level); }
-CSA_DEV uint32_t digit_mask(int level) { return level < 2 ? 0xfffu : 0xffu; }
+// Digits of the 64-bit key (score key << 32 | ~index), most significant first: level 0
+// the top 12 bits (the scan's histogram), levels 1-6 eight bits each (bits 44-51 down
+// to 4-11), level 7 the last four.  The narrow digits after level 0 keep the per-level
+// histograms at 256 bins, which the threshold search covers with one bin per thread.
+CSA_DEV uint32_t digit_shift(int level) { return level == 0 ? 52u : level < 7 ? (uint32_t)(52 - 8 * level) : 0u; }
+CSA_DEV uint32_t digit_mask(int level) { return level == 0 ? 0xfffu : level < 7 ? 0xffu : 0xfu; }
 CSA_DEV uint32_t digit_at(uint2 kv, uint32_t shift, uint32_t mask)
 {
     const uint64_t key = ((uint64_t)kv.x << 32) | (uint32_t)~kv.y;
@@ -270,7 +274,7 @@ CSA_DEV void resolve_long_list(const Query& q, uint32_t* sh, uint2* s_listA, uin
                                int tid, uint32_t count)
 {
     for (uint32_t i = tid; i < count; i += kSelThreads)
-        atomicAdd(&sh[hist_slot(digit_of(__ldcg(&q.cand[i]), 1))], 1u);
+        atomicAdd(&sh[digit_of(__ldcg(&q.cand[i]), 1)], 1u);
     Bar::sync();
     uint32_t need = (uint32_t)q.k - s->out;
     uint2* list = q.cand;
@@ -284,18 +288,16 @@ CSA_DEV void resolve_long_list(const Query& q, uint32_t* sh, uint2* s_listA, uin
             emit_by_rank(q, list, count, need, s, tid);
             break;
         }
-        if (level > 6) break;  // unreachable: (score, index) keys are unique
+        if (level > 7) break;  // unreachable: (score, index) keys are unique
         if (level >= 2) {
             for (int i = tid; i < 256; i += kSelThreads) sh[i] = 0;
             Bar::sync();
             for (uint32_t i = tid; i < count; i += kSelThreads)
                 atomicAdd(&sh[digit_of(in_smem ? list[i] : __ldcg(&list[i]), level)], 1u);
             Bar::sync();
-            find_threshold_bin<256, Bar>(sh, need, s, tid);
-        } else {
-            find_threshold_bin<kBins, Bar>(sh, need, s, tid);
         }
-        const uint32_t bt = s->bin, above = s->above, keep_n = level >= 2 ? sh[bt] : sh[hist_slot(bt)];
+        find_threshold_bin<256, Bar>(sh, need, s, tid);
+        const uint32_t bt = s->bin, above = s->above, keep_n = sh[bt];
         const bool next_smem = keep_n <= (uint32_t)kListCap;
         uint2* next = next_smem ? (list == s_listA ? s_listB : s_listA) : (list == q.cand ? q.cand2 : q.cand);
         if (tid == 0) s->cnt = 0;
@@ -350,7 +352,7 @@ CSA_DEV void resolve_candidates(const Query& q, uint32_t* sh, uint2* s_listA, ui
         return;
     }
     uint32_t need = (uint32_t)q.k - out;
-    for (int level = 1; need > 0 && level <= 6; ++level) {
+    for (int level = 1; need > 0 && level <= 7; ++level) {
         // v[u] holds entry tid + u * kSelThreads of the current list (valid below count)
         if (need < count && count <= (uint32_t)kRankMax) {  // exact rank among a small list
             if (tid < (int)count) s_listA[tid] = v[0];
@@ -361,21 +363,17 @@ CSA_DEV void resolve_candidates(const Query& q, uint32_t* sh, uint2* s_listA, ui
         const uint32_t dsh = digit_shift(level), dmask = digit_mask(level);
         uint32_t bt = 0xffffffffu;  // need >= count: every entry is taken
         if (need < count) {
-            const int nb = level == 1 ? kBins : 256;
-            if (level > 1) {
-                for (int i = tid; i < nb; i += kSelThreads) sh[i] = 0;
+            if (level > 1) {  // (level 1 starts from the zeroed histogram)
+                for (int i = tid; i < 256; i += kSelThreads) sh[i] = 0;
                 Bar::sync();
             }
 #pragma unroll
             for (int u = 0; u < kPerT; ++u) {
                 const uint32_t d = digit_at(v[u], dsh, dmask);
-                if (tid + u * kSelThreads < (int)count) atomicAdd(&sh[level == 1 ? hist_slot(d) : d], 1u);
+                if (tid + u * kSelThreads < (int)count) atomicAdd(&sh[d], 1u);
             }
             Bar::sync();
-            if (level == 1)
-                find_threshold_bin<kBins, Bar>(sh, need, s, tid);
-            else
-                find_threshold_bin<256, Bar>(sh, need, s, tid);
+            find_threshold_bin<256, Bar>(sh, need, s, tid);
             bt = s->bin;
         }
         uint32_t cnt = 0;
