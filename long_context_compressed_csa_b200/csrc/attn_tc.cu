@@ -78,12 +78,6 @@ CSA_DEV uint32_t peer_addr(uint32_t local_smem_addr, uint32_t peer)
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem_addr), "r"(peer));
     return r;
 }
-CSA_DEV void st_cluster_v4(uint32_t addr, float4 v)
-{
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
-                 "f"(v.w)
-                 : "memory");
-}
 CSA_DEV void mbar_arrive_remote(uint32_t remote_bar)
 {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
