@@ -260,7 +260,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
                 constexpr int HW = NH / 8;  // heads per warp
                 const int ew = et >> 5, el = et & 31;
                 // every load of this warp's heads first (one round trip), V bf16 per head
+                // and the head weights
                 uint32_t raw[HW][V / 2];
+                float wv[HW];
+#pragma unroll
+                for (int i = 0; i < HW; ++i) wv[i] = __ldg(&wI[(int64_t)g * NH + ew + 8 * i]);
 #pragma unroll
                 for (int i = 0; i < HW; ++i) {
                     const __nv_bfloat16* src = qg + (int64_t)(ew + 8 * i) * CI + el * V;
@@ -298,7 +302,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
                         *reinterpret_cast<uint32_t*>(dst) = w[0];
                     else
                         *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
-                    if (el == 0) sw[h] = wI[(int64_t)g * NH + h] * sc;
+                    if (el == 0) sw[h] = wv[i] * sc;
                 }
             }
             if (need_hist)
@@ -355,12 +359,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
                     scores[sidx] = sc;
                 }
             }
-            if (need_hist) {
-                // lanes with the same digit add once (scores cluster in few bins)
-                const uint32_t bin = sidx < vis ? order_key(sc) >> 20 : 0xffffffffu;
-                const unsigned peers = __match_any_sync(0xffffffffu, bin);
-                if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&sh[hist_slot(bin)], (uint32_t)__popc(peers));
-            }
+            // the digit-0 histogram: one shared atomic per key (aggregating equal digits
+            // across the warp first measured slower)
+            if (need_hist && sidx < vis) atomicAdd(&sh[hist_slot(order_key(sc) >> 20)], 1u);
         }
     }
 
