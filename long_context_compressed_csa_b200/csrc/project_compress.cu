@@ -242,18 +242,31 @@ hca_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __
 // CSA form ([P1] sections 3-5): four projections C^a = H W_a^KV, C^b = H W_b^KV,
 // Z^a = H W_a^Z, Z^b = H W_b^Z, then for entry i and column j the softmax over the 2m = 8
 // logits Z^a of block i (+ B^a) and Z^b of block i - 1 (+ B^b), and the weighted sum of
-// the matching C^a and C^b values; entry 0 has no b-part.  With m = 4, a tile of 128
-// tokens holds 32 blocks; block 0 only serves as the b-part of the tile's first entry,
-// so a tile yields 31 entries and consecutive tiles overlap by one block.  Four
-// accumulators of 128 tokens fill the 512 TMEM columns: C^a 0-127, C^b 128-255, Z^a
-// 256-383, Z^b 384-511.
+// the matching C^a and C^b values; entry 0 has no b-part.
+//
+// With m = 4 a tile of 256 tokens holds 64 blocks.  Block 0 only serves as the b-part of
+// the tile's first entry, so a tile yields 63 entries and consecutive tiles overlap by
+// one block.  Only two accumulators of 256 tokens fit the 512 TMEM columns, so each tile
+// runs two passes over K, each of the shape of the HCA kernel above (C in TMEM columns
+// 0-255, Z in 256-511):
+//   pass b   C^b and Z^b: per block, the softmax statistics of its four b-logits, kept in
+//            the epilogue threads' registers as (value, log2 of the weight sum)
+//               v_b = sum_r e^{z_r - mx} C_r / sum_r e^{z_r - mx},
+//               s_b = mx log2(e) + log2(sum_r e^{z_r - mx});
+//   pass a   C^a and Z^a: per block i, the same sums over its four a-logits, merged with
+//            block i - 1's statistics into the softmax over all eight logits, then the
+//            bf16 entry.
+// The merge is the usual split softmax: with A = mx_a log2(e) and M = max(A, s_b), the
+// entry is (2^{A-M} acc_a + 2^{s_b-M} v_b) / (2^{A-M} l_a + 2^{s_b-M}).
+// Per 64-wide K panel a pass loads 32 KB of weights and a 32 KB H panel for 256 tokens,
+// the HCA kernel's ratio of bytes to products.  Eight epilogue warps (two per TMEM lane
+// quarter, each owning half of the tile's blocks) keep the TMEM drain between passes
+// short.
 constexpr int kCsM = 4;                          // tokens per CSA block
-constexpr int kCsTokens = 128;                   // tokens per tile (MMA N)
-constexpr int kCsEntries = kCsTokens / kCsM - 1; // 31 entries per tile
-constexpr int kCsHBytes = kCsTokens * 128;       // one 128 x 64 H panel: 16 KB
-constexpr int kCsStage = 4 * kPcWBytes + kCsHBytes;  // 80 KB
-constexpr int kCsStages = 2;
-constexpr int kCsSmem = 1024 + kCsStages * kCsStage + 256;
+constexpr int kCsTokens = kPcTokens;             // tokens per tile (MMA N): 64 blocks
+constexpr int kCsEntries = kCsTokens / kCsM - 1; // 63 entries per tile
+constexpr int kCsThreads = 64 + 256;             // TMA warp, MMA warp, 8 epilogue warps
+constexpr int kCsSmem = kPcSmem;                 // the HCA kernel's 3 x 64 KB ring
 
 struct CsArgs {
     int64_t rows_per_batch, tok0;
@@ -264,22 +277,113 @@ struct CsArgs {
     int64_t out_ld_batch;
     int64_t e0, e1;
     int n_cb;
-    int64_t n_tb;            // tiles of 31 entries per batch
+    int64_t n_tb;            // tiles of 63 entries per batch
     int64_t tiles;
     uint32_t* status;
 };
 
-__global__ void __launch_bounds__(kPcThreads, 1)
-csa_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ CUtensorMap tmap_w0,
-                            const __grid_constant__ CUtensorMap tmap_w1, const __grid_constant__ CUtensorMap tmap_w2,
-                            const __grid_constant__ CUtensorMap tmap_w3, CsArgs a)
+// Pass b for one epilogue thread.  Half 0 keeps blocks 0-30 (u = kb), half 1 blocks
+// 31-62 (u = kb - 31): the b-parts of the a-blocks 1-31 and 32-63 that the same thread
+// merges in pass a.  Loads are 16-column aligned, so half 1 starts at token 112.
+template <int HALF>
+CSA_DEV void cs_pass_b(uint32_t taddr, const float (&bb)[kCsM], float (&sv)[32], float (&ss)[32], uint64_t* tempty)
+{
+    constexpr float kLog2e = 1.4426950408889634f;
+    constexpr int kLo = HALF ? 7 : 0, kHi = HALF ? 15 : 7;
+#pragma unroll
+    for (int ch = kLo; ch <= kHi; ++ch) {
+        uint32_t rc[16], rz[16];
+        tc::tmem_ld16_async(taddr + ch * 16, rc);
+        tc::tmem_ld16_async(taddr + kCsTokens + ch * 16, rz);
+        tc::tmem_wait_ld_regs16(rc, rz);
+        if (ch == kHi) {  // this thread's TMEM reads are done
+            tc::fence_before_sync();
+            tc::mbar_arrive(tempty);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int kb = 4 * ch + q;
+            if (HALF == 0 ? kb > 30 : (kb < 31 || kb > 62)) continue;
+            const int u = HALF ? kb - 31 : kb;
+            float z[kCsM], mx = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < kCsM; ++r) {
+                z[r] = __uint_as_float(rz[4 * q + r]) + bb[r];
+                mx = fmaxf(mx, z[r]);
+            }
+            float l = 0.f, acc = 0.f;
+#pragma unroll
+            for (int r = 0; r < kCsM; ++r) {
+                const float p = exp2f((z[r] - mx) * kLog2e);
+                l += p;
+                acc = fmaf(p, __uint_as_float(rc[4 * q + r]), acc);
+            }
+            sv[u] = acc / l;
+            ss[u] = fmaf(mx, kLog2e, log2f(l));
+        }
+    }
+}
+
+// Pass a for one epilogue thread: half 0 writes the entries of a-blocks 1-31, half 1
+// those of a-blocks 32-63 (entry first + kb - 1, b-part in sv/ss[u]).
+template <int HALF>
+CSA_DEV void cs_pass_a(uint32_t taddr, const float (&ba)[kCsM], const float (&sv)[32], const float (&ss)[32],
+                       int64_t first, int64_t e1, int64_t ld_entry, __nv_bfloat16* orow, uint64_t* tempty)
+{
+    constexpr float kLog2e = 1.4426950408889634f;
+    constexpr int kLo = HALF ? 8 : 0, kHi = HALF ? 15 : 7;
+#pragma unroll
+    for (int ch = kLo; ch <= kHi; ++ch) {
+        uint32_t rc[16], rz[16];
+        tc::tmem_ld16_async(taddr + ch * 16, rc);
+        tc::tmem_ld16_async(taddr + kCsTokens + ch * 16, rz);
+        tc::tmem_wait_ld_regs16(rc, rz);
+        if (ch == kHi) {
+            tc::fence_before_sync();
+            tc::mbar_arrive(tempty);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int kb = 4 * ch + q;
+            if (HALF == 0 && kb == 0) continue;
+            const int u = HALF ? kb - 32 : kb - 1;
+            const int64_t i = first + kb - 1;
+            float z[kCsM], mx = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < kCsM; ++r) {
+                z[r] = __uint_as_float(rz[4 * q + r]) + ba[r];
+                mx = fmaxf(mx, z[r]);
+            }
+            float l = 0.f, acc = 0.f;
+#pragma unroll
+            for (int r = 0; r < kCsM; ++r) {
+                const float p = exp2f((z[r] - mx) * kLog2e);
+                l += p;
+                acc = fmaf(p, __uint_as_float(rc[4 * q + r]), acc);
+            }
+            float res = acc / l;
+            if (i > 0) {  // entry 0 has no b-part
+                const float A = mx * kLog2e;
+                const float M = fmaxf(A, ss[u]);
+                const float wa = exp2f(A - M), wb = exp2f(ss[u] - M);
+                res = fmaf(wa, acc, wb * sv[u]) / fmaf(wa, l, wb);
+            }
+            if (i < e1) orow[i * ld_entry] = __float2bfloat16_rn(res);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kCsThreads, 1)
+csa_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ CUtensorMap tmap_wa_kv,
+                            const __grid_constant__ CUtensorMap tmap_wb_kv, const __grid_constant__ CUtensorMap tmap_wa_z,
+                            const __grid_constant__ CUtensorMap tmap_wb_z, CsArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kCsStages * kCsStage);
-    uint64_t* empty = full + kCsStages;
-    uint64_t* tfull = empty + kCsStages;
-    uint64_t* tempty = tfull + 1;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPcStages * kPcStage);
+    uint64_t* empty = full + kPcStages;
+    uint64_t* tfull = empty + kPcStages;   // MMA -> epilogue: the pass's accumulators are complete
+    uint64_t* tempty = tfull + 1;          // epilogue -> MMA: TMEM read out (count 256)
     uint64_t* done = tempty + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
@@ -287,20 +391,20 @@ csa_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kCsStages; ++s) {
+        for (int s = 0; s < kPcStages; ++s) {
             tc::mbar_init(&full[s], 1);
             tc::mbar_init(&empty[s], 1);
         }
         tc::mbar_init(tfull, 1);
-        tc::mbar_init(tempty, 128);
+        tc::mbar_init(tempty, kCsThreads - 64);
         tc::mbar_init(done, 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&tmap_h);
-        tc::tma_prefetch_desc(&tmap_w0);
-        tc::tma_prefetch_desc(&tmap_w1);
-        tc::tma_prefetch_desc(&tmap_w2);
-        tc::tma_prefetch_desc(&tmap_w3);
+        tc::tma_prefetch_desc(&tmap_wa_kv);
+        tc::tma_prefetch_desc(&tmap_wb_kv);
+        tc::tma_prefetch_desc(&tmap_wa_z);
+        tc::tma_prefetch_desc(&tmap_wb_z);
     }
     if (warp == 1) {
         tc::tmem_alloc(tmem_slot, 512);
@@ -322,7 +426,6 @@ csa_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            const CUtensorMap* wmaps[4] = {&tmap_w0, &tmap_w1, &tmap_w2, &tmap_w3};
             int it = 0;
             bool stop = false;
             for (int64_t t = blockIdx.x; t < a.tiles && !stop; t += gridDim.x) {
@@ -333,59 +436,69 @@ csa_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __
                 // first token (entry 0) are read but never used
                 const int hrow = (int)(b * a.rows_per_batch + kCsM * (a.e0 + kCsEntries * tb - 1) - a.tok0);
                 const int wrow = cb * kPcCols;
-                for (int kp = 0; kp < kpanels; ++kp, ++it) {
-                    const int s = it % kCsStages;
-                    const uint32_t ph = (it / kCsStages) & 1;
-                    if (*abort_flag || !tc::mbar_wait(&empty[s], ph ^ 1, tc::kWaitBudget)) {
-                        *abort_flag = 1;
-                        stop = true;
-                        break;
+                for (int pass = 0; pass < 2 && !stop; ++pass) {
+                    const CUtensorMap* wkv = pass == 0 ? &tmap_wb_kv : &tmap_wa_kv;
+                    const CUtensorMap* wz = pass == 0 ? &tmap_wb_z : &tmap_wa_z;
+                    for (int kp = 0; kp < kpanels; ++kp, ++it) {
+                        const int s = it % kPcStages;
+                        const uint32_t ph = (it / kPcStages) & 1;
+                        if (*abort_flag || !tc::mbar_wait(&empty[s], ph ^ 1, tc::kWaitBudget)) {
+                            *abort_flag = 1;
+                            stop = true;
+                            break;
+                        }
+                        uint8_t* st = smem + s * kPcStage;
+                        tc::mbar_arrive_expect_tx(&full[s], kPcStage);
+                        // pass a walks K backwards: the H panels pass b read last are
+                        // the first ones it needs, while they are still in L2
+                        const int kx = (pass == 0 ? kp : kpanels - 1 - kp) * 64;
+                        tc::tma_load_2d(st, wkv, &full[s], kx, wrow);
+                        tc::tma_load_2d(st + kPcWBytes, wz, &full[s], kx, wrow);
+                        tc::tma_load_2d(st + 2 * kPcWBytes, &tmap_h, &full[s], kx, hrow);
                     }
-                    uint8_t* st = smem + s * kCsStage;
-                    tc::mbar_arrive_expect_tx(&full[s], kCsStage);
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) tc::tma_load_2d(st + w * kPcWBytes, wmaps[w], &full[s], kp * 64, wrow);
-                    tc::tma_load_2d(st + 4 * kPcWBytes, &tmap_h, &full[s], kp * 64, hrow);
                 }
             }
-            for (int j = it - kCsStages < 0 ? 0 : it - kCsStages; j < it; ++j)
-                if (!tc::mbar_wait(&full[j % kCsStages], (j / kCsStages) & 1, tc::kWaitBudget)) *abort_flag = 1;
+            // drain: every issued load has landed before the CTA may exit
+            for (int j = it - kPcStages < 0 ? 0 : it - kPcStages; j < it; ++j)
+                if (!tc::mbar_wait(&full[j % kPcStages], (j / kPcStages) & 1, tc::kWaitBudget)) *abort_flag = 1;
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdesc = tc::idesc_bf16_f32(kPcCols, kCsTokens, false, false);
-            int it = 0, nt = 0;
+            int it = 0, np = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < a.tiles && ok; t += gridDim.x, ++nt) {
-                if (!tc::mbar_wait(tempty, (nt & 1) ^ 1, tc::kWaitBudget)) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                for (int kp = 0; kp < kpanels; ++kp, ++it) {
-                    const int s = it % kCsStages;
-                    const uint32_t ph = (it / kCsStages) & 1;
-                    if (*abort_flag || !tc::mbar_wait(&full[s], ph, tc::kWaitBudget)) {
+            for (int64_t t = blockIdx.x; t < a.tiles && ok; t += gridDim.x) {
+                for (int pass = 0; pass < 2 && ok; ++pass, ++np) {
+                    if (!tc::mbar_wait(tempty, (np & 1) ^ 1, tc::kWaitBudget)) {  // TMEM read out
                         ok = false;
                         break;
                     }
                     tc::fence_after_sync();
-                    const uint32_t w0 = tc::smem_u32(smem + s * kCsStage);
-                    const uint32_t hh = w0 + 4 * kPcWBytes;
+                    for (int kp = 0; kp < kpanels; ++kp, ++it) {
+                        const int s = it % kPcStages;
+                        const uint32_t ph = (it / kPcStages) & 1;
+                        if (*abort_flag || !tc::mbar_wait(&full[s], ph, tc::kWaitBudget)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after_sync();
+                        const uint32_t wc = tc::smem_u32(smem + s * kPcStage);
+                        const uint32_t wz = wc + kPcWBytes;
+                        const uint32_t hh = wc + 2 * kPcWBytes;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t bd = tc::smem_desc_sw128(hh + kk * 32, 16, 1024);
-                        const uint32_t acc = (kp | kk) ? 1u : 0u;
-#pragma unroll
-                        for (int w = 0; w < 4; ++w)
-                            tc::mma_bf16_ss(tmem + w * kCsTokens, tc::smem_desc_sw128(w0 + w * kPcWBytes + kk * 32, 16, 1024),
-                                            bd, kIdesc, acc);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t bd = tc::smem_desc_sw128(hh + kk * 32, 16, 1024);
+                            const uint32_t acc = (kp | kk) ? 1u : 0u;
+                            tc::mma_bf16_ss(tmem, tc::smem_desc_sw128(wc + kk * 32, 16, 1024), bd, kIdesc, acc);
+                            tc::mma_bf16_ss(tmem + kCsTokens, tc::smem_desc_sw128(wz + kk * 32, 16, 1024), bd, kIdesc,
+                                            acc);
+                        }
+                        tc::mma_commit(&empty[s]);
                     }
-                    tc::mma_commit(&empty[s]);
+                    if (!ok) break;
+                    tc::mma_commit(tfull);
                 }
-                if (!ok) break;
-                tc::mma_commit(tfull);
             }
             if (!ok) *abort_flag = 1;
             tc::mma_commit(done);
@@ -393,16 +506,12 @@ csa_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        constexpr float kLog2e = 1.4426950408889634f;
-        const int quarter = warp & 3;
+        const int quarter = warp & 3;               // TMEM lanes this warp may read
+        const int half = (warp - 2) >> 2;           // which 32 blocks of the tile
         const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
-        int nt = 0;
-        for (int64_t t = blockIdx.x; t < a.tiles; t += gridDim.x, ++nt) {
-            if (*abort_flag || !tc::mbar_wait(tfull, nt & 1, tc::kWaitBudget)) {
-                *abort_flag = 1;
-                break;
-            }
-            tc::fence_after_sync();
+        float sv[32], ss[32];                       // pass b statistics, carried to pass a
+        int np = 0;
+        for (int64_t t = blockIdx.x; t < a.tiles; t += gridDim.x) {
             int b, cb;
             int64_t tb;
             tile_of(t, b, tb, cb);
@@ -413,51 +522,24 @@ csa_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __
                 ba[r] = a.ba ? __ldg(&a.ba[r * a.c + j]) : 0.f;
                 bb[r] = a.bb ? __ldg(&a.bb[r * a.c + j]) : 0.f;
             }
+            if (*abort_flag || !tc::mbar_wait(tfull, np & 1, tc::kWaitBudget)) {
+                *abort_flag = 1;
+                break;
+            }
+            ++np;
+            tc::fence_after_sync();
+            if (half == 0) cs_pass_b<0>(taddr, bb, sv, ss, tempty);
+            else cs_pass_b<1>(taddr, bb, sv, ss, tempty);
+            if (*abort_flag || !tc::mbar_wait(tfull, np & 1, tc::kWaitBudget)) {
+                *abort_flag = 1;
+                break;
+            }
+            ++np;
+            tc::fence_after_sync();
             const int64_t first = a.e0 + kCsEntries * tb;  // entry of tile block 1
             __nv_bfloat16* orow = a.out + (int64_t)b * a.out_ld_batch + j;
-            float pcb[kCsM], pzb[kCsM];  // C^b, Z^b of the previous block
-#pragma unroll 1
-            for (int t0 = 0; t0 < kCsTokens; t0 += 16) {
-                uint32_t r_ca[16], r_cb[16], r_za[16], r_zb[16];
-                tc::tmem_ld16(taddr + 0 * kCsTokens + t0, reinterpret_cast<float*>(r_ca));
-                tc::tmem_ld16(taddr + 1 * kCsTokens + t0, reinterpret_cast<float*>(r_cb));
-                tc::tmem_ld16(taddr + 2 * kCsTokens + t0, reinterpret_cast<float*>(r_za));
-                tc::tmem_ld16(taddr + 3 * kCsTokens + t0, reinterpret_cast<float*>(r_zb));
-                tc::tmem_wait_ld();
-                if (t0 + 16 == kCsTokens) {  // the whole tile is in registers: the MMA may go on
-                    tc::fence_before_sync();
-                    tc::mbar_arrive(tempty);
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {  // the 4 blocks of these 16 tokens
-                    const int kb = t0 / kCsM + q;  // tile block
-                    if (kb > 0) {
-                        const int64_t i = first + kb - 1;  // entry: a-part block kb, b-part block kb - 1
-                        float za[kCsM], zb[kCsM], mx = -INFINITY;
-#pragma unroll
-                        for (int r = 0; r < kCsM; ++r) {
-                            za[r] = __uint_as_float(r_za[q * kCsM + r]) + ba[r];
-                            zb[r] = i > 0 ? pzb[r] + bb[r] : -INFINITY;  // entry 0 has no b-part
-                            mx = fmaxf(mx, fmaxf(za[r], zb[r]));
-                        }
-                        float l = 0.f, acc = 0.f;
-#pragma unroll
-                        for (int r = 0; r < kCsM; ++r) {
-                            const float pa = exp2f((za[r] - mx) * kLog2e);
-                            const float pb = i > 0 ? exp2f((zb[r] - mx) * kLog2e) : 0.f;
-                            l += pa + pb;
-                            acc = fmaf(pa, __uint_as_float(r_ca[q * kCsM + r]), acc);
-                            if (i > 0) acc = fmaf(pb, pcb[r], acc);
-                        }
-                        if (i < a.e1) orow[i * a.c] = __float2bfloat16_rn(acc / l);
-                    }
-#pragma unroll
-                    for (int r = 0; r < kCsM; ++r) {
-                        pcb[r] = __uint_as_float(r_cb[q * kCsM + r]);
-                        pzb[r] = __uint_as_float(r_zb[q * kCsM + r]);
-                    }
-                }
-            }
+            if (half == 0) cs_pass_a<0>(taddr, ba, sv, ss, first, a.e1, a.c, orow, tempty);
+            else cs_pass_a<1>(taddr, ba, sv, ss, first, a.e1, a.c, orow, tempty);
         }
     }
 
@@ -569,7 +651,7 @@ extern "C" int csa_project_compress(const void* H, int64_t ld_row, int64_t ld_ba
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t grid = a.tiles < sms ? a.tiles : sms;
     cudaFuncSetAttribute(csa_project_compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCsSmem);
-    launch_pdl(csa_project_compress_kernel, dim3((unsigned)grid), dim3(kPcThreads), (size_t)kCsSmem, stream, th,
+    launch_pdl(csa_project_compress_kernel, dim3((unsigned)grid), dim3(kCsThreads), (size_t)kCsSmem, stream, th,
                tw[0], tw[1], tw[2], tw[3], a);
     return launch_status();
 }

@@ -211,7 +211,8 @@ def test_hca_project_compress_b16_128k_sampled():
 def test_csa_project_compress_b4_256k_sampled():
     """The fused CSA projections + compression at the micro-benchmark's launch: B = 4
     sequences of 262144 tokens, d = 4096, c = 512 (65536 entries each).  Sampled entries,
-    the first one (no b-part) and tile edges included, are recomputed by the oracle."""
+    the first one (no b-part), tile edges and the split between the two epilogue
+    halves of a tile included, are recomputed by the oracle."""
     B, n, d, c, m = 4, 262144, 4096, 512, 4
     H = randn((B, n, d), 980, BF16, DEV, scale=d ** -0.25)
     Ws = [randn((c, d), 981 + w, BF16, DEV, scale=d ** -0.25) for w in range(4)]
@@ -223,7 +224,7 @@ def test_csa_project_compress_b4_256k_sampled():
     assert lib.csa_workspace_status(ws) == 0
     W64 = [to_f64(W).T for W in Ws]
     Ba64, Bb64 = to_f64(Ba), to_f64(Bb)
-    for b, i in ((0, 0), (0, 30), (1, 31), (2, 62), (3, 65535), (2, 40000)):
+    for b, i in ((0, 0), (0, 30), (1, 31), (2, 62), (3, 63), (1, 125), (1, 126), (3, 65535), (2, 40000)):
         lo = max(0, m * (i - 1))
         rows = to_f64(H[b, lo:m * (i + 1)])
         streams = [oracle.project(rows, W) for W in W64]

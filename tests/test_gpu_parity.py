@@ -123,9 +123,11 @@ def _ref_project_compress(H, Wc, Wz, mp, Bias, i0, i1):
 
 
 @pytest.mark.parametrize("B,rows,d,c,bias,e0,e1,tok0", [
-    (2, 4 * 70 + 3, 256, 256, True, 0, None, 0),      # 3 tiles of 31 entries (the last partial)
+    (2, 4 * 70 + 3, 256, 256, True, 0, None, 0),      # 2 tiles of 63 entries (the last partial)
     (1, 4 * 60, 64, 128, False, 5, 40, 16),           # a sub-range, tok0 at block e0 - 1
     (3, 4 * 100, 1024, 512, True, 0, None, 0),        # several K panels and column blocks
+    (2, 4 * 320 + 1, 128, 128, True, 0, None, 0),     # 6 tiles: 5 full, one ragged
+    (2, 4 * 260, 192, 256, True, 70, 250, 4 * 69),    # a sub-range across 3 tiles, tok0 > 0
 ])
 def test_csa_project_compress_matches_oracle(B, rows, d, c, bias, e0, e1, tok0):
     """Fused CSA projections + overlapped compression: the four streams H W^T in fp32 on
