@@ -67,13 +67,6 @@ CSA_DEV void cp_async_wait_all() { asm volatile("cp.async.commit_group;\n\tcp.as
 CSA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 CSA_DEV void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }  // all but the newest group
 
-// 2^x with the hardware exponential unit (arguments here are <= 8, results >= 0)
-CSA_DEV float ex2_approx(float x)
-{
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 constexpr int kBoxCols = 64;             // one output box: 128 rows x 64 bf16 columns (128 B)
 constexpr int kBoxBytes = kHeads * 128;  // 16 KB
@@ -498,8 +491,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
             uint32_t packed[kEG / 2];
 #pragma unroll
             for (int e = 0; e < kEG; e += 2) {
-                const float p0f = (s[e] == -INFINITY) ? 0.f : ex2_approx(s[e] - m_run);
-                const float p1f = (s[e + 1] == -INFINITY) ? 0.f : ex2_approx(s[e + 1] - m_run);
+                const float p0f = (s[e] == -INFINITY) ? 0.f : tc::ex2_approx(s[e] - m_run);
+                const float p1f = (s[e + 1] == -INFINITY) ? 0.f : tc::ex2_approx(s[e + 1] - m_run);
                 ps[(e >> 1) & 3] += p0f + p1f;
                 __nv_bfloat162 pr = __floats2bfloat162_rn(p0f, p1f);
                 packed[e / 2] = *reinterpret_cast<uint32_t*>(&pr);

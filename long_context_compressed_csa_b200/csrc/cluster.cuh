@@ -63,5 +63,54 @@ CSA_DEV void cluster_sync()
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// ---- CTA pairs on one MMA (cta_group::2): rank 0 of a cluster of two is the leader ----
+// TMEM allocation of a CTA pair: both CTAs run it, from the same warp, into the same
+// shared memory offset, and receive the same column address.
+CSA_DEV void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tc::smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+CSA_DEV void tmem_relinquish_pair() { asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory"); }
+CSA_DEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D (+)= A B^T across the pair, issued by one leader thread: M = 256 rows of A, the
+// first 128 from the leader's shared memory and the next 128 from its peer's, both at
+// the descriptor's offset; the N rows of B split the same way (N/2 from each CTA).
+// Each CTA's TMEM receives its own 128 rows of D for all N columns.
+CSA_DEV void mma_bf16_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Once the pair MMAs this thread issued so far complete, arrive once on the barrier at
+// bar's offset in every CTA of cta_mask (bit r = cluster rank r).
+CSA_DEV void mma_commit_pair(uint64_t* bar, uint16_t cta_mask)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            tc::smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+// 2-D tiled TMA load into this CTA's shared memory whose transaction bytes complete on
+// an mbarrier of either CTA of the pair (bar_cluster: a shared::cluster address, e.g.
+// the leader's barrier from peer_addr).  No multicast: one destination CTA.
+CSA_DEV void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x, int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%3, %4}], [%2];" ::"r"(tc::smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+        : "memory");
+}
+
 }  // namespace cl
 }  // namespace csa

@@ -122,6 +122,48 @@ inline cudaError_t launch_pdl(void (*kern)(P...), dim3 grid, dim3 block, size_t 
     return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
 }
 
+// The same launch with thread-block clusters of two CTAs along x (CTA pairs).
+inline void pair_launch_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute (&attr)[2], dim3 grid, dim3 block,
+                               size_t smem, cudaStream_t stream)
+{
+    cfg = cudaLaunchConfig_t{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+}
+template <typename... P, typename... A>
+inline cudaError_t launch_pdl_pairs(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                    A&&... args)
+{
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[2];
+    pair_launch_config(cfg, attr, grid, block, smem, stream);
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+// CTA pairs of `kern` that fit on the device at once (0 if none, or on error).
+template <typename... P>
+inline int max_resident_pairs(void (*kern)(P...), dim3 block, size_t smem)
+{
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[2];
+    pair_launch_config(cfg, attr, dim3(2), block, smem, nullptr);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

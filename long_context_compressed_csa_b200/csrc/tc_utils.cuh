@@ -140,6 +140,27 @@ CSA_DEV void mma_commit(uint64_t* bar)
                  : "memory");
 }
 
+// Hardware approximations of the multi-function unit (flush-to-zero): 2^x and log2(x)
+// with about 2^-22 relative (absolute for log2) error, 1/x within 1 ulp.
+CSA_DEV float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+CSA_DEV float lg2_approx(float x)
+{
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+CSA_DEV float rcp_approx(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // 32 lanes x 16 consecutive 32-bit columns; thread i of the warp receives lane
 // (taddr.lane + i), columns taddr.col .. +15.
 CSA_DEV void tmem_ld16(uint32_t taddr, float* v)
