@@ -82,7 +82,13 @@ int csa_version(void);
  *                  (prefill: [0, n/m); incremental decode: [i, i+1)).
  * Constraints    : c >= 1, 1 <= m <= 4096.
  * The indexer keys K^I are produced by the same call with their own streams and c^I
- * ([P1] section 6.4: "the same compression operation ... a separate set of weights").
+ * ([P1] section 6.4: the indexer compresses its keys with this operation, under its own
+ * weights).
+ * Kernels        : prefill-sized bf16 calls with m = 4, c a multiple of 256, 16-byte
+ *                  aligned streams and row strides a multiple of 8 run a TMA-staged
+ *                  kernel (one CTA per SM); all other calls run a per-thread streaming
+ *                  kernel.  The staged kernel's waits are bounded: if one ever times out
+ *                  (not expected), the entries it did not finish are written as NaN.
  * ------------------------------------------------------------------------------- */
 int csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
                  int64_t ld_row, int64_t ld_batch, int64_t tok0, int64_t n,
@@ -239,8 +245,8 @@ int csa_sparse_attn(const void* q, const void* cache, const int32_t* idx,
                     int dtype, int out_bf16, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
- * hca_dense_attn - dense shared-KV MQA over every visible HCA entry ([P1] section 10,
- * "every query attends to all compressed blocks densely"; causal rule s < floor(t/m')).
+ * hca_dense_attn - dense shared-KV MQA over every visible HCA entry ([P1] section 10:
+ * no selection, each query sees all its compressed entries; causal rule s < floor(t/m')).
  * Same arguments as csa_sparse_attn with the index list replaced by the visible range
  * [0, min(floor(t[g]/m_prime), N_cap)) read from the DEVICE int64 array t [B*nq].
  * workspace : >= csa_attn_workspace_size(B, nq, n_h, c, N_cap) bytes.

@@ -19,6 +19,7 @@
 //     candidate count and the exp unit never becomes the limit;
 //   - fp32 state (running max, sum, weighted sum) per column, output rounded once.
 #include "common.cuh"
+#include "tc_utils.cuh"
 
 namespace csa {
 namespace {
@@ -39,6 +40,7 @@ struct PoolArgs {
     int B, c, m;
     int64_t e0, e1;
     int has_b;
+    int64_t n_rows;  // token rows of each batch in the buffers (n - tok0)
 };
 
 // Loads of V consecutive elements of one row: one 16-byte streaming load when the row
@@ -191,6 +193,208 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolArgs p)
     }
 }
 
+// ----------------------------------------------------------------------------------
+// TMA-staged streaming path for CSA (bf16, m = 4, c a multiple of 256, prefill-sized
+// calls).
+//
+// pool_kernel's per-thread walk keeps only 2 kUnroll 16-byte loads in flight per thread,
+// and a CSA entry has just 8 candidate rows, so it reaches 0.67 of the HBM copy rate.
+// Here a persistent CTA per SM streams the rows through a 6-stage ring of 32 KB TMA
+// boxes ({256 columns x 16 rows} of each of the four streams, unswizzled, so row r of a
+// stream is 512 contiguous bytes of shared memory), and eight compute warps pool them
+// with one thread per column of the 256-column slice.  A stage holds 16 rows of Z^a and
+// C^a (the blocks of 4 consecutive entries) and 16 rows of Z^b and C^b starting one block
+// earlier, so each of the 4 entries finds its 8 candidates in the same stage.  Entry 0's
+// b-rows (before the batch's first token) are loaded but never used.
+// Logits are taken in base 2 (zl = (z + B) log2 e) and every exponential is the
+// multi-function unit's ex2 (relative error about 2^-22).  Each compute warp releases a
+// stage with one arrival.  Waits are bounded; after a timeout (never expected) the
+// compute threads write NaN into every entry they have not finished, so a failure
+// cannot pass for a result.
+// (The same staging for HCA, 32 rows of Z and C per stage pooled online, measured 0.68
+// of the copy rate against pool_kernel's 0.73 and is not used.)
+constexpr int kSpCols = 256;                     // columns per slice: one per compute thread
+constexpr int kSpWarps = 8;                      // compute warps
+constexpr int kSpThreads = 32 * (kSpWarps + 1);  // + the producer warp
+constexpr int kSpStageBytes = 32768;
+constexpr int kSpStages = 6;
+constexpr int kSpSmem = kSpStages * kSpStageBytes + 128 + 128;
+constexpr int kSpCsaEntries = 64;                // CSA entries per work item (16 stages)
+
+struct SpArgs {
+    int64_t rows_per_batch, tok0;
+    const float* Ba;         // [m][c] or null
+    const float* Bb;         // [m][c] or null
+    __nv_bfloat16* out;
+    int64_t out_ld_batch;
+    int c, m;
+    int64_t e0, e1;
+    int n_slices;
+    int64_t groups;          // per (batch, slice): groups of kSpCsaEntries entries
+    int64_t items;           // B * groups * n_slices
+};
+
+__global__ void __launch_bounds__(kSpThreads, 1)
+stream_pool_kernel(const __grid_constant__ CUtensorMap t0, const __grid_constant__ CUtensorMap t1,
+                   const __grid_constant__ CUtensorMap t2, const __grid_constant__ CUtensorMap t3, SpArgs a)
+{
+    // t0 = Z^a, t1 = C^a, t2 = Z^b, t3 = C^b
+    constexpr int kStreams = 4;
+    constexpr int kRows = kSpStageBytes / (kStreams * kSpCols * 2);  // 16 rows: 4 blocks
+    constexpr int kStreamBytes = kRows * kSpCols * 2;
+    constexpr float kL2e = 1.4426950408889634f;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kSpStages * kSpStageBytes);
+    uint64_t* empty = full + kSpStages;
+    volatile uint32_t* abort_flag = reinterpret_cast<uint32_t*>(empty + kSpStages);
+
+    pdl_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kSpStages; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], kSpWarps);
+        }
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+        tc::tma_prefetch_desc(&t0);
+        tc::tma_prefetch_desc(&t1);
+        tc::tma_prefetch_desc(&t2);
+        tc::tma_prefetch_desc(&t3);
+    }
+    __syncthreads();
+    pdl_wait();
+
+    auto item_of = [&](int64_t t, int& b, int& sl, int64_t& g) {
+        sl = (int)(t % a.n_slices);
+        const int64_t r = t / a.n_slices;
+        g = r % a.groups;
+        b = (int)(r / a.groups);
+    };
+    // stages of an item and the entries it covers
+    auto item_span = [&](int64_t g, int64_t& ent0, int& nent, int& nst) {
+        ent0 = a.e0 + g * kSpCsaEntries;
+        const int64_t left = a.e1 - ent0;
+        nent = (int)(left < kSpCsaEntries ? left : kSpCsaEntries);
+        nst = (nent + 3) / 4;
+    };
+
+    if (warp == kSpWarps) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int it = 0;
+            bool stop = false;
+            for (int64_t t = blockIdx.x; t < a.items && !stop; t += gridDim.x) {
+                int b, sl, nent, nst;
+                int64_t g, ent0;
+                item_of(t, b, sl, g);
+                item_span(g, ent0, nent, nst);
+                const int x = sl * kSpCols;
+                const int ra = (int)(b * a.rows_per_batch + (int64_t)a.m * ent0 - a.tok0);  // first a-row
+                for (int j = 0; j < nst; ++j, ++it) {
+                    const int s = it % kSpStages;
+                    const uint32_t ph = (it / kSpStages) & 1;
+                    if (*abort_flag || !tc::mbar_wait(&empty[s], ph ^ 1, tc::kWaitBudget)) {
+                        *abort_flag = 1;
+                        stop = true;
+                        break;
+                    }
+                    uint8_t* st = smem + s * kSpStageBytes;
+                    tc::mbar_arrive_expect_tx(&full[s], kSpStageBytes);
+                    tc::tma_load_2d(st, &t0, &full[s], x, ra + kRows * j);
+                    tc::tma_load_2d(st + kStreamBytes, &t1, &full[s], x, ra + kRows * j);
+                    // b-rows one block (m = 4 rows) earlier
+                    tc::tma_load_2d(st + 2 * kStreamBytes, &t2, &full[s], x, ra - 4 + kRows * j);
+                    tc::tma_load_2d(st + 3 * kStreamBytes, &t3, &full[s], x, ra - 4 + kRows * j);
+                }
+            }
+            // drain: every issued load has landed before the CTA may exit
+            for (int j = it - kSpStages < 0 ? 0 : it - kSpStages; j < it; ++j)
+                if (!tc::mbar_wait(&full[j % kSpStages], (j / kSpStages) & 1, tc::kWaitBudget)) *abort_flag = 1;
+        }
+    } else {
+        // ------------------------------------------------------------ compute: thread = column
+        const int col = threadIdx.x;
+        int it = 0;
+        bool ok = true;
+        int64_t t = blockIdx.x;
+        for (; t < a.items && ok; t += gridDim.x) {
+            int b, sl, nent, nst;
+            int64_t g, ent0;
+            item_of(t, b, sl, g);
+            item_span(g, ent0, nent, nst);
+            const int j = sl * kSpCols + col;
+            __nv_bfloat16* orow = a.out + (int64_t)b * a.out_ld_batch + j;
+            {
+                float ba[4], bb[4];  // biases in base-2 units
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    ba[r] = a.Ba ? __ldg(&a.Ba[r * a.c + j]) * kL2e : 0.f;
+                    bb[r] = a.Bb ? __ldg(&a.Bb[r * a.c + j]) * kL2e : 0.f;
+                }
+                for (int js = 0; js < nst; ++js, ++it) {
+                    const int s = it % kSpStages;
+                    if (*abort_flag || !tc::mbar_wait(&full[s], (it / kSpStages) & 1, tc::kWaitBudget)) {
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    const __nv_bfloat16* st = reinterpret_cast<const __nv_bfloat16*>(smem + s * kSpStageBytes) + col;
+                    const __nv_bfloat16* za = st;
+                    const __nv_bfloat16* ca = st + kRows * kSpCols;
+                    const __nv_bfloat16* zb = st + 2 * kRows * kSpCols;
+                    const __nv_bfloat16* cb = st + 3 * kRows * kSpCols;
+                    float res[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int64_t i = ent0 + 4 * js + q;
+                        const bool has_b = i > 0;  // entry 0 has no b-part
+                        float zl[8], xv[8], mx = -INFINITY;
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            zl[r] = fmaf(__bfloat162float(za[(4 * q + r) * kSpCols]), kL2e, ba[r]);
+                            xv[r] = __bfloat162float(ca[(4 * q + r) * kSpCols]);
+                            zl[4 + r] = has_b ? fmaf(__bfloat162float(zb[(4 * q + r) * kSpCols]), kL2e, bb[r])
+                                              : -INFINITY;
+                            xv[4 + r] = has_b ? __bfloat162float(cb[(4 * q + r) * kSpCols]) : 0.f;
+                        }
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) mx = fmaxf(mx, zl[r]);
+                        float l = 0.f, acc = 0.f;
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) {
+                            const float p = tc::ex2_approx(zl[r] - mx);
+                            l += p;
+                            acc = fmaf(p, xv[r], acc);
+                        }
+                        res[q] = acc * tc::rcp_approx(l);  // l in [1, 8]
+                    }
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&empty[s]);  // this warp is done with the stage
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int64_t i = ent0 + 4 * js + q;
+                        if (4 * js + q < nent) orow[i * a.c] = __float2bfloat16_rn(res[q]);
+                    }
+                }
+            }
+            if (!ok) break;
+        }
+        if (!ok) {
+            // timeout: NaN into every entry of this item and of the CTA's later items
+            for (; t < a.items; t += gridDim.x) {
+                int b, sl, nent, nst;
+                int64_t g, ent0;
+                item_of(t, b, sl, g);
+                item_span(g, ent0, nent, nst);
+                __nv_bfloat16* orow = a.out + (int64_t)b * a.out_ld_batch + sl * kSpCols + col;
+                for (int e = 0; e < nent; ++e) orow[(ent0 + e) * a.c] = __float2bfloat16_rn(NAN);
+            }
+        }
+    }
+}
+
 // Vectorised (16-byte) path when every row offset of the call is 16-byte aligned,
 // element path otherwise.
 bool vector_ok(const PoolArgs& p, int dtype)
@@ -201,8 +405,52 @@ bool vector_ok(const PoolArgs& p, int dtype)
            aligned16(p.out) && (!p.Ba || aligned16(p.Ba)) && (!p.Bb || aligned16(p.Bb));
 }
 
+// The TMA-staged path for bf16 prefill-sized CSA calls; false when the call does not fit
+// it (not CSA, odd widths or strides, m other than 4, or too little work to fill the
+// SMs), which then runs pool_kernel.
+bool launch_stream_pool(const PoolArgs& p, cudaStream_t stream, int& status)
+{
+    if (!p.has_b || p.m != 4) return false;
+    if (p.c % kSpCols != 0 || p.ld_row % 8 != 0 || (p.B > 1 && p.ld_batch % p.ld_row != 0)) return false;
+    if (!aligned16(p.Xa) || !aligned16(p.Za) || !aligned16(p.Xb) || !aligned16(p.Zb)) return false;
+    const int64_t nent = p.e1 - p.e0;
+    SpArgs a;
+    a.n_slices = p.c / kSpCols;
+    a.groups = (nent + kSpCsaEntries - 1) / kSpCsaEntries;
+    a.items = (int64_t)p.B * a.groups * a.n_slices;
+    if (a.items < kNumSMs) return false;
+    a.rows_per_batch = p.B > 1 ? p.ld_batch / p.ld_row : p.n_rows;
+    const int64_t height = (int64_t)(p.B - 1) * a.rows_per_batch + p.n_rows;  // rows the buffers hold
+    if (height + kSpCols >= (int64_t(1) << 31)) return false;
+    a.tok0 = p.tok0;
+    a.Ba = p.Ba;
+    a.Bb = p.Bb;
+    a.out = static_cast<__nv_bfloat16*>(p.out);
+    a.out_ld_batch = p.out_ld_batch;
+    a.c = p.c;
+    a.m = p.m;
+    a.e0 = p.e0;
+    a.e1 = p.e1;
+    CUtensorMap tm[4];
+    const void* src[4] = {p.Za, p.Xa, p.Zb, p.Xb};
+    for (int i = 0; i < 4; ++i)
+        if (!make_tmap_bf16_2d_plain(&tm[i], src[i], (uint64_t)height, (uint64_t)p.c, (uint64_t)p.ld_row, kSpCols,
+                                     16)) {
+            status = CSA_ERR_CUDA;
+            return true;
+        }
+    const unsigned grid = (unsigned)(a.items < kNumSMs ? a.items : kNumSMs);
+    cudaFuncSetAttribute(stream_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSpSmem);
+    launch_pdl(stream_pool_kernel, dim3(grid), dim3(kSpThreads), (size_t)kSpSmem, stream, tm[0], tm[1], tm[2], tm[3],
+               a);
+    status = launch_status();
+    return true;
+}
+
 int launch_pool(const PoolArgs& p, int dtype, cudaStream_t stream)
 {
+    int status = CSA_OK;
+    if (dtype == CSA_BF16 && launch_stream_pool(p, stream, status)) return status;
     const bool vec = vector_ok(p, dtype);
     const int V = vec ? 16 / elem_bytes(dtype) : 1;
     const int64_t total = (int64_t)p.B * (p.e1 - p.e0) * (p.c / V);
@@ -260,6 +508,7 @@ extern "C" int csa_compress(const void* Ca, const void* Cb, const void* Za, cons
     p.ld_row = ld_row; p.ld_batch = ld_batch; p.tok0 = tok0;
     p.out = out; p.out_ld_batch = out_ld_batch;
     p.B = B; p.c = c; p.m = m; p.e0 = entry_begin; p.e1 = entry_end; p.has_b = 1;
+    p.n_rows = n - tok0;
     return launch_pool(p, dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -284,5 +533,6 @@ extern "C" int hca_compress(const void* C, const void* Z, int64_t ld_row, int64_
     p.ld_row = ld_row; p.ld_batch = ld_batch; p.tok0 = tok0;
     p.out = out; p.out_ld_batch = out_ld_batch;
     p.B = B; p.c = c; p.m = m_prime; p.e0 = entry_begin; p.e1 = entry_end; p.has_b = 0;
+    p.n_rows = n - tok0;
     return launch_pool(p, dtype, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -306,6 +306,10 @@ constexpr long long kWaitBudget = 2000000000LL;  // ~1 s at 1.9 GHz
 // box of box_cols x box_rows and 128-byte swizzle; false if the driver call fails.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                        uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);
+// Same without swizzle: the box lands row-major in shared memory (box_cols * 2 bytes per
+// row, a multiple of 16).
+bool make_tmap_bf16_2d_plain(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                             uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);
 // Same for a 2-D tensor of bytes (E4M3 codes).
 bool make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                      uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);

@@ -212,6 +212,55 @@ def test_hca_compress_random(dtype, c, mp):
     torch.testing.assert_close(part[:, i], out[:, i], rtol=0, atol=0)
 
 
+@pytest.mark.parametrize("B,nent,c,e0,e1,bias", [
+    (2, 5000, 256, 0, None, True),      # 79 groups of 64 entries per batch, the last ragged
+    (2, 5000, 256, 70, 4990, False),    # a sub-range, rows from block e0 - 1 (tok0 > 0)
+    (1, 9500, 512, 0, None, True),      # two 256-column slices
+])
+def test_csa_compress_streaming_path(B, nent, c, e0, e1, bias):
+    """Prefill-sized bf16 CSA compression, large enough (>= 148 work items of 64 entries
+    x 256 columns) to run the TMA-staged streaming kernel, against the oracle on every
+    entry: the b-rows loaded one block early, entry 0 without a b-part, ragged groups."""
+    m = 4
+    n = m * nent + 3
+    e1 = nent if e1 is None else e1
+    tok0 = 0 if e0 == 0 else m * (e0 - 1)
+    S = [randn((B, n, c), 150 + i, torch.bfloat16) for i in range(4)]
+    Ba = randn((m, c), 160, torch.float32) if bias else None
+    Bb = randn((m, c), 161, torch.float32) if bias else None
+    out = run_csa_compress(*(dev(x[:, tok0:]) for x in S), m, Ba=dev(Ba) if bias else None,
+                           Bb=dev(Bb) if bias else None, i0=e0, i1=e1, tok0=tok0, N_cap=nent + 1)
+    got = out.float().cpu().numpy()
+    for b in range(B):
+        ref = oracle.csa_compress(*(to_f64(x[b]) for x in S), m, Ba=to_f64(Ba) if bias else None,
+                                  Bb=to_f64(Bb) if bias else None, i0=e0, i1=e1)
+        assert max_rel_rowwise(got[b, e0:e1], ref).max() <= TOL[torch.bfloat16]
+        assert np.all(np.isnan(got[b, :e0])) and np.all(np.isnan(got[b, e1:]))
+
+
+@pytest.mark.parametrize("B,mp,nent,c,e0,bias", [
+    (2, 128, 100, 512, 0, True),
+    (3, 64, 120, 256, 7, False),        # a sub-range from tok0 = m' e0
+])
+def test_hca_compress_prefill_size(B, mp, nent, c, e0, bias):
+    """Prefill-sized bf16 HCA compression (hundreds of entries, m' = 128 and 64, a
+    sub-range from tok0 = m' e0) against the oracle on every entry."""
+    n = mp * nent + 17
+    tok0 = mp * e0
+    C, Z = randn((B, n, c), 170, torch.bfloat16), randn((B, n, c), 171, torch.bfloat16)
+    Bias = randn((mp, c), 172, torch.float32) if bias else None
+    out = torch.full((B, nent, c), float("nan"), dtype=torch.bfloat16, device=DEV)
+    hca_compress(dev(C[:, tok0:]), dev(Z[:, tok0:]), out, mp, e0, nent, Bias=dev(Bias) if bias else None,
+                 tok0=tok0)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy()
+    for b in range(B):
+        ref = oracle.hca_compress(to_f64(C[b]), to_f64(Z[b]), mp, Bias=to_f64(Bias) if bias else None,
+                                  i0=e0, i1=nent)
+        assert max_rel_rowwise(got[b, e0:], ref).max() <= TOL[torch.bfloat16]
+        assert np.all(np.isnan(got[b, :e0]))
+
+
 def test_compress_extreme_logits_one_hot():
     B, n, c, m = 1, 32, 64, 4
     Ca, Cb = randn((B, n, c), 140, torch.float32), randn((B, n, c), 141, torch.float32)
