@@ -326,57 +326,55 @@ stream_pool_kernel(const __grid_constant__ CUtensorMap t0, const __grid_constant
             item_span(g, ent0, nent, nst);
             const int j = sl * kSpCols + col;
             __nv_bfloat16* orow = a.out + (int64_t)b * a.out_ld_batch + j;
-            {
-                float ba[4], bb[4];  // biases in base-2 units
+            float ba[4], bb[4];  // biases in base-2 units
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    ba[r] = a.Ba ? __ldg(&a.Ba[r * a.c + j]) * kL2e : 0.f;
-                    bb[r] = a.Bb ? __ldg(&a.Bb[r * a.c + j]) * kL2e : 0.f;
+            for (int r = 0; r < 4; ++r) {
+                ba[r] = a.Ba ? __ldg(&a.Ba[r * a.c + j]) * kL2e : 0.f;
+                bb[r] = a.Bb ? __ldg(&a.Bb[r * a.c + j]) * kL2e : 0.f;
+            }
+            for (int js = 0; js < nst; ++js, ++it) {
+                const int s = it % kSpStages;
+                if (*abort_flag || !tc::mbar_wait(&full[s], (it / kSpStages) & 1, tc::kWaitBudget)) {
+                    *abort_flag = 1;
+                    ok = false;
+                    break;
                 }
-                for (int js = 0; js < nst; ++js, ++it) {
-                    const int s = it % kSpStages;
-                    if (*abort_flag || !tc::mbar_wait(&full[s], (it / kSpStages) & 1, tc::kWaitBudget)) {
-                        *abort_flag = 1;
-                        ok = false;
-                        break;
+                const __nv_bfloat16* st = reinterpret_cast<const __nv_bfloat16*>(smem + s * kSpStageBytes) + col;
+                const __nv_bfloat16* za = st;
+                const __nv_bfloat16* ca = st + kRows * kSpCols;
+                const __nv_bfloat16* zb = st + 2 * kRows * kSpCols;
+                const __nv_bfloat16* cb = st + 3 * kRows * kSpCols;
+                float res[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int64_t i = ent0 + 4 * js + q;
+                    const bool has_b = i > 0;  // entry 0 has no b-part
+                    float zl[8], xv[8], mx = -INFINITY;
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        zl[r] = fmaf(__bfloat162float(za[(4 * q + r) * kSpCols]), kL2e, ba[r]);
+                        xv[r] = __bfloat162float(ca[(4 * q + r) * kSpCols]);
+                        zl[4 + r] = has_b ? fmaf(__bfloat162float(zb[(4 * q + r) * kSpCols]), kL2e, bb[r])
+                                          : -INFINITY;
+                        xv[4 + r] = has_b ? __bfloat162float(cb[(4 * q + r) * kSpCols]) : 0.f;
                     }
-                    const __nv_bfloat16* st = reinterpret_cast<const __nv_bfloat16*>(smem + s * kSpStageBytes) + col;
-                    const __nv_bfloat16* za = st;
-                    const __nv_bfloat16* ca = st + kRows * kSpCols;
-                    const __nv_bfloat16* zb = st + 2 * kRows * kSpCols;
-                    const __nv_bfloat16* cb = st + 3 * kRows * kSpCols;
-                    float res[4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int64_t i = ent0 + 4 * js + q;
-                        const bool has_b = i > 0;  // entry 0 has no b-part
-                        float zl[8], xv[8], mx = -INFINITY;
+                    for (int r = 0; r < 8; ++r) mx = fmaxf(mx, zl[r]);
+                    float l = 0.f, acc = 0.f;
 #pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            zl[r] = fmaf(__bfloat162float(za[(4 * q + r) * kSpCols]), kL2e, ba[r]);
-                            xv[r] = __bfloat162float(ca[(4 * q + r) * kSpCols]);
-                            zl[4 + r] = has_b ? fmaf(__bfloat162float(zb[(4 * q + r) * kSpCols]), kL2e, bb[r])
-                                              : -INFINITY;
-                            xv[4 + r] = has_b ? __bfloat162float(cb[(4 * q + r) * kSpCols]) : 0.f;
-                        }
-#pragma unroll
-                        for (int r = 0; r < 8; ++r) mx = fmaxf(mx, zl[r]);
-                        float l = 0.f, acc = 0.f;
-#pragma unroll
-                        for (int r = 0; r < 8; ++r) {
-                            const float p = tc::ex2_approx(zl[r] - mx);
-                            l += p;
-                            acc = fmaf(p, xv[r], acc);
-                        }
-                        res[q] = acc * tc::rcp_approx(l);  // l in [1, 8]
+                    for (int r = 0; r < 8; ++r) {
+                        const float p = tc::ex2_approx(zl[r] - mx);
+                        l += p;
+                        acc = fmaf(p, xv[r], acc);
                     }
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(&empty[s]);  // this warp is done with the stage
+                    res[q] = acc * tc::rcp_approx(l);  // l in [1, 8]
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&empty[s]);  // this warp is done with the stage
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int64_t i = ent0 + 4 * js + q;
-                        if (4 * js + q < nent) orow[i * a.c] = __float2bfloat16_rn(res[q]);
-                    }
+                for (int q = 0; q < 4; ++q) {
+                    const int64_t i = ent0 + 4 * js + q;
+                    if (4 * js + q < nent) orow[i * a.c] = __float2bfloat16_rn(res[q]);
                 }
             }
             if (!ok) break;

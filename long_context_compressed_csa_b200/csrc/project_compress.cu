@@ -14,8 +14,9 @@
 //             a 256 x 64 tile of H (two entries' tokens), 128-byte swizzle, into a ring;
 //   warp 1    MMA issuer: M = 128 columns, N = 256 tokens, K = 16, two accumulators
 //             (C in TMEM columns 0-255, Z in 256-511);
-//   warps 2-5 epilogue: thread = column; per entry an online softmax over its 128 tokens
-//             (32 at a time from TMEM), then one bf16 entry value per column.
+//   warps 2-9 epilogue: thread = column of one of the tile's two entries (warps 2-5 the
+//             first, 6-9 the second); an online softmax over the entry's 128 tokens (32
+//             at a time from TMEM), then one bf16 entry value.
 // CTAs are persistent over tiles (token block, column block) with the column blocks of
 // one token block consecutive, so the CTAs running at the same time share H tiles in L2.
 // C and Z never leave the chip.  Every wait is bounded; a timeout sets the workspace
@@ -27,7 +28,7 @@
 namespace csa {
 namespace {
 
-constexpr int kPcThreads = 192;                  // TMA warp, MMA warp, 4 epilogue warps
+constexpr int kPcThreads = 320;                  // TMA warp, MMA warp, 8 epilogue warps
 constexpr int kPcCols = 128;                     // output columns per tile (MMA M)
 constexpr int kPcMp = 128;                       // tokens per entry (m')
 constexpr int kPcTokens = 2 * kPcMp;             // tokens per tile (MMA N): two entries
@@ -121,7 +122,7 @@ hca_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __
             tc::mbar_init(&empty[s], 1);
         }
         tc::mbar_init(tfull, 1);
-        tc::mbar_init(tempty, 128);
+        tc::mbar_init(tempty, kPcThreads - 64);
         tc::mbar_init(done, 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
@@ -211,7 +212,8 @@ hca_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int quarter = warp & 3;
+        const int quarter = warp & 3;        // TMEM lanes this warp may read
+        const int ent = (warp - 2) >> 2;     // which of the tile's two entries
         const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
         int nt = 0;
         for (int64_t t = blockIdx.x; t < a.tiles; t += gridDim.x, ++nt) {
@@ -224,16 +226,11 @@ hca_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __
             int64_t tb;
             pc_tile(a, t, b, tb, cb);
             const int j = cb * kPcCols + quarter * 32 + lane;  // this thread's output column
-            float res[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) res[e] = hca_entry(taddr + e * kPcMp, a.bias, a.c, j, a.bias != nullptr);
+            const float res = hca_entry(taddr + ent * kPcMp, a.bias, a.c, j, a.bias != nullptr);
             tc::fence_before_sync();
             tc::mbar_arrive(tempty);  // TMEM read out: the next tile's MMAs may start
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int64_t i = a.e0 + 2 * tb + e;
-                if (i < a.e1) a.out[(int64_t)b * a.out_ld_batch + i * a.c + j] = __float2bfloat16_rn(res[e]);
-            }
+            const int64_t i = a.e0 + 2 * tb + ent;
+            if (i < a.e1) a.out[(int64_t)b * a.out_ld_batch + i * a.c + j] = __float2bfloat16_rn(res);
         }
     }
 
