@@ -154,6 +154,7 @@ class HybridDecode:
         self.Nh_cap = self.Nh + T // self.mp + 1
         self.hist = 2 * self.m  # stream rows kept from before the decode (for block i-1)
         c, cI = self.c, self.cI
+        self.row_width = 4 * (c + cI) + 2 * c  # elements of one token's decode stream rows
         self.pairs = []
         t0 = time.time()
         for p in range(N_PAIRS):
@@ -164,10 +165,14 @@ class HybridDecode:
             P["hcache"] = torch.empty((1, self.Nh_cap, c), dtype=bf16, device=device)
             # prefill compress through the library (streams generated in slices)
             self._prefill(P, s)
-            # decode-time stream rows: tokens n - hist .. n + T - 1 (CSA), n .. n + T - 1 (HCA)
-            P["dec"] = [randn((1, self.hist + T, c), s + 10 + i, bf16, device) for i in range(4)]
-            P["decI"] = [randn((1, self.hist + T, cI), s + 20 + i, bf16, device) for i in range(4)]
-            P["decH"] = [randn((1, T, c), s + 30 + i, bf16, device) for i in range(2)]
+            # decode-time stream rows, one interleaved row per token (the 4 CSA streams, the
+            # 4 indexer-key streams, the 2 HCA streams), so that a token's new rows are one
+            # contiguous copy: tokens n - hist .. n + T - 1 (CSA), n .. n + T - 1 (HCA)
+            P["rows"] = randn((1, self.hist + T, self.row_width), s + 10, bf16, device)
+            R = P["rows"]
+            P["dec"] = [R[:, :, i * c:(i + 1) * c] for i in range(4)]
+            P["decI"] = [R[:, :, 4 * c + i * cI:4 * c + (i + 1) * cI] for i in range(4)]
+            P["decH"] = [R[:, self.hist:, 4 * (c + cI) + i * c:4 * (c + cI) + (i + 1) * c] for i in range(2)]
             self.pairs.append(P)
         torch.cuda.synchronize()
         log("prefill of %d layer pairs: %.1f s" % (N_PAIRS, time.time() - t0))
@@ -180,8 +185,8 @@ class HybridDecode:
         self.tpos = torch.arange(n, n + T, dtype=torch.int64, device=device).reshape(T, 1, 1)
         # outputs and workspaces (one set per pair so steps never share scratch in flight)
         self.idx = torch.empty((1, 1, self.k), dtype=torch.int32, device=device)
-        self.o = torch.empty((1, 1, self.n_h, c), dtype=torch.float32, device=device)
-        self.oh = torch.empty((1, 1, self.n_h, c), dtype=torch.float32, device=device)
+        self.obuf = torch.empty((2, 1, 1, self.n_h, c), dtype=torch.float32, device=device)
+        self.o, self.oh = self.obuf[0], self.obuf[1]  # CSA and HCA outputs, adjacent
         self.ws_topk = torch.zeros(lib.csa_indexer_topk_workspace_size(1, 1, self.N_cap, self.k),
                                    dtype=torch.uint8, device=device)
         self.ws_attn = torch.zeros(lib.csa_attn_workspace_size(1, 1, self.n_h, c, self.k),
@@ -639,52 +644,74 @@ def main():
 
 
 def run_e2e(torch, dec, W, K, world):
-    """Eager steps through the C ABI: each step's inputs from pinned host memory (the new
-    token's stream rows, q, q^I, w^I, the HCA query), both outputs back to pinned host."""
+    """Steps through the C ABI with each step's inputs from pinned host memory (the new
+    token's stream rows, q, q^I, w^I, the HCA query) and both outputs back to pinned host:
+    three copies per step (the four queries share one staging buffer, the new token's rows
+    of all ten streams are one interleaved row, the two outputs are adjacent)."""
     c, cI = dec.c, dec.cI
     nQ = 8
-    hq = dec.q[:nQ].cpu().pin_memory()
-    hqh = dec.qh[:nQ].cpu().pin_memory()
-    hqI = dec.qI[:nQ].cpu().pin_memory()
-    hwI = dec.wI[:nQ].cpu().pin_memory()
-    hrows = torch.randn((nQ, 4 * (c + cI) + 2 * c), dtype=torch.float32).to(torch.bfloat16).pin_memory()
-    ho = torch.empty((1, 1, dec.n_h, c), dtype=torch.float32).pin_memory()
-    hoh = torch.empty_like(ho).pin_memory()
-    dq = torch.empty_like(dec.q[0]); dqh = torch.empty_like(dec.qh[0])
-    dqI = torch.empty_like(dec.qI[0]); dwI = torch.empty_like(dec.wI[0])
-    h2d = (hq[0].numel() + hqh[0].numel() + hqI[0].numel()) * 2 + hwI[0].numel() * 4 + hrows[0].numel() * 2
-    d2h = 2 * ho.numel() * 4
+    parts = [dec.q[:nQ], dec.qh[:nQ], dec.qI[:nQ], dec.wI[:nQ]]
+    sizes = [x[0].numel() * x.element_size() for x in parts]
+    offs = [0]
+    for z in sizes:
+        offs.append(offs[-1] + (z + 255) // 256 * 256)
+    hstage = torch.empty((nQ, offs[-1]), dtype=torch.uint8).pin_memory()
+    for x, o0, z in zip(parts, offs, sizes):
+        hstage[:, o0:o0 + z].copy_(x.reshape(nQ, -1).view(torch.uint8).cpu())
+    dstage = torch.empty((offs[-1],), dtype=torch.uint8, device="cuda")
+    dq, dqh, dqI, dwI = (dstage[o0:o0 + z].view(x.dtype).view(x[0].shape)
+                         for x, o0, z in zip(parts, offs, sizes))
+    hrows = torch.randn((nQ, dec.row_width), dtype=torch.float32).to(torch.bfloat16).pin_memory()
+    hout = torch.empty(dec.obuf.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(sizes) + hrows[0].numel() * 2
+    d2h = hout.numel() * 4
 
     def one(s):
         p, j = s % N_PAIRS, s // N_PAIRS
         qs = s % nQ
-        dq.copy_(hq[qs], non_blocking=True)
-        dqh.copy_(hqh[qs], non_blocking=True)
-        dqI.copy_(hqI[qs], non_blocking=True)
-        dwI.copy_(hwI[qs], non_blocking=True)
+        dstage.copy_(hstage[qs], non_blocking=True)
         P = dec.pairs[p]
-        r = dec.hist + j  # the new token's rows in the decode stream buffers
-        off = 0
-        for x in P["dec"]:
-            x[0, r].copy_(hrows[qs, off:off + c], non_blocking=True); off += c
-        for x in P["decI"]:
-            x[0, r].copy_(hrows[qs, off:off + cI], non_blocking=True); off += cI
-        for x in P["decH"]:
-            x[0, j].copy_(hrows[qs, off:off + c], non_blocking=True); off += c
+        P["rows"][0, dec.hist + j].copy_(hrows[qs], non_blocking=True)  # the new token's rows
         dec.step(p, j, q=dq, qh=dqh, qI=dqI, wI=dwI)
-        ho.copy_(dec.o, non_blocking=True)
-        hoh.copy_(dec.oh, non_blocking=True)
+        hout.copy_(dec.obuf, non_blocking=True)
 
     for s in range(W):
         one(s)
     torch.cuda.synchronize()
+    # The same calls as a serving loop issues them: each group of IDX_SAMPLE steps (one
+    # token through the layer pairs) captured once, with its copies, in a CUDA graph and
+    # replayed; every replay still moves each step's inputs and outputs over PCIe.
+    how = ("C-ABI calls of each step with its pinned host->device input copies and "
+           "device->host output copies, captured in CUDA graphs of %d steps and replayed" % IDX_SAMPLE)
+    graphs = []
+    try:
+        for s0 in range(W, W + K, IDX_SAMPLE):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for s in range(s0, min(s0 + IDX_SAMPLE, W + K)):
+                    one(s)
+            graphs.append(g)
+        torch.cuda.synchronize()
+    except Exception as exc:  # capture refused: time the eager calls instead
+        log("e2e graph capture failed (%s); timing eager calls" % exc)
+        graphs = []
+        how = "eager C-ABI calls per step; pinned host->device inputs and device->host outputs inside the timed region"
+        torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if graphs:
+        graphs[0].replay()  # warm-up replay
+        torch.cuda.synchronize()
     a.record()
-    for s in range(W, W + K):
-        one(s)
+    if graphs:
+        for g in graphs:
+            g.replay()
+    else:
+        for s in range(W, W + K):
+            one(s)
     b.record()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
+    del graphs
     if world > 1:
         import torch.distributed as dist
         t = torch.tensor([ms], dtype=torch.float64, device="cuda")
@@ -692,8 +719,7 @@ def run_e2e(torch, dec, W, K, world):
         ms = float(t.item())
     return {"value": K * world / (ms / 1000.0), "unit": "layer-pair decode steps/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": K,
-            "how": "eager C-ABI calls per step; pinned host->device inputs and device->host "
-                   "outputs inside the timed region"}
+            "how": how}
 
 
 if __name__ == "__main__":
