@@ -201,8 +201,8 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolArgs p)
 // and a CSA entry has just 8 candidate rows, so it reaches 0.67 of the HBM copy rate.
 // Here a persistent CTA per SM streams the rows through a 6-stage ring of 32 KB TMA
 // boxes ({256 columns x 16 rows} of each of the four streams, unswizzled, so row r of a
-// stream is 512 contiguous bytes of shared memory), and eight compute warps pool them
-// with one thread per column of the 256-column slice.  A stage holds 16 rows of Z^a and
+// stream is 512 contiguous bytes of shared memory), and sixteen compute warps pool them:
+// one thread per column of the 256-column slice and per half of a stage's entries.  A stage holds 16 rows of Z^a and
 // C^a (the blocks of 4 consecutive entries) and 16 rows of Z^b and C^b starting one block
 // earlier, so each of the 4 entries finds its 8 candidates in the same stage.  Entry 0's
 // b-rows (before the batch's first token) are loaded but never used.
@@ -214,7 +214,8 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolArgs p)
 // (The same staging for HCA, 32 rows of Z and C per stage pooled online, measured 0.68
 // of the copy rate against pool_kernel's 0.73 and is not used.)
 constexpr int kSpCols = 256;                     // columns per slice: one per compute thread
-constexpr int kSpWarps = 8;                      // compute warps
+constexpr int kSpWarps = 16;                     // compute warps: two per column group
+constexpr int kSpEntPerThread = 2;               // of a stage's 4 entries
 constexpr int kSpThreads = 32 * (kSpWarps + 1);  // + the producer warp
 constexpr int kSpStageBytes = 32768;
 constexpr int kSpStages = 6;
@@ -315,7 +316,8 @@ stream_pool_kernel(const __grid_constant__ CUtensorMap t0, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------ compute: thread = column
-        const int col = threadIdx.x;
+        const int col = threadIdx.x % kSpCols;
+        const int q0 = (threadIdx.x / kSpCols) * kSpEntPerThread;  // this thread's first entry of a stage
         int it = 0;
         bool ok = true;
         int64_t t = blockIdx.x;
@@ -344,9 +346,10 @@ stream_pool_kernel(const __grid_constant__ CUtensorMap t0, const __grid_constant
                 const __nv_bfloat16* ca = st + kRows * kSpCols;
                 const __nv_bfloat16* zb = st + 2 * kRows * kSpCols;
                 const __nv_bfloat16* cb = st + 3 * kRows * kSpCols;
-                float res[4];
+                float res[kSpEntPerThread];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int qq = 0; qq < kSpEntPerThread; ++qq) {
+                    const int q = q0 + qq;
                     const int64_t i = ent0 + 4 * js + q;
                     const bool has_b = i > 0;  // entry 0 has no b-part
                     float zl[8], xv[8], mx = -INFINITY;
@@ -367,14 +370,15 @@ stream_pool_kernel(const __grid_constant__ CUtensorMap t0, const __grid_constant
                         l += p;
                         acc = fmaf(p, xv[r], acc);
                     }
-                    res[q] = acc * tc::rcp_approx(l);  // l in [1, 8]
+                    res[qq] = acc * tc::rcp_approx(l);  // l in [1, 8]
                 }
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&empty[s]);  // this warp is done with the stage
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int qq = 0; qq < kSpEntPerThread; ++qq) {
+                    const int q = q0 + qq;
                     const int64_t i = ent0 + 4 * js + q;
-                    if (4 * js + q < nent) orow[i * a.c] = __float2bfloat16_rn(res[q]);
+                    if (4 * js + q < nent) orow[i * a.c] = __float2bfloat16_rn(res[qq]);
                 }
             }
             if (!ok) break;
