@@ -194,25 +194,27 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolArgs p)
 }
 
 // ----------------------------------------------------------------------------------
-// TMA-staged streaming path for CSA (bf16, m = 4, c a multiple of 256, prefill-sized
-// calls).
+// TMA-staged streaming path (bf16, c a multiple of 256, prefill-sized calls; CSA with
+// m = 4, HCA with m' a multiple of 32).
 //
-// pool_kernel's per-thread walk keeps only 2 kUnroll 16-byte loads in flight per thread,
-// and a CSA entry has just 8 candidate rows, so it reaches 0.67 of the HBM copy rate.
-// Here a persistent CTA per SM streams the rows through a 6-stage ring of 32 KB TMA
-// boxes ({256 columns x 16 rows} of each of the four streams, unswizzled, so row r of a
-// stream is 512 contiguous bytes of shared memory), and sixteen compute warps pool them:
-// one thread per column of the 256-column slice and per half of a stage's entries.  A stage holds 16 rows of Z^a and
-// C^a (the blocks of 4 consecutive entries) and 16 rows of Z^b and C^b starting one block
-// earlier, so each of the 4 entries finds its 8 candidates in the same stage.  Entry 0's
-// b-rows (before the batch's first token) are loaded but never used.
+// pool_kernel's per-thread walk keeps only 2 kUnroll 16-byte loads in flight per thread:
+// it reaches 0.67 (CSA) and 0.72 (HCA) of the HBM copy rate.  Here a persistent CTA per
+// SM streams the rows through a 6-stage ring of 32 KB TMA boxes ({256 columns x R rows}
+// of each stream, unswizzled, so row r of a stream is 512 contiguous bytes of shared
+// memory), and sixteen compute warps pool them with one thread per column of the
+// 256-column slice:
+//   CSA   a stage holds 16 rows of Z^a and C^a (the blocks of 4 consecutive entries) and
+//         16 rows of Z^b and C^b starting one block earlier, so each of the 4 entries
+//         finds its 8 candidates in the same stage; each of the two warp groups takes 2
+//         of the 4 entries.  Entry 0's b-rows (before the batch's first token) are loaded
+//         but never used.
+//   HCA   a stage holds 32 rows of Z and C; an entry of m' rows is m'/32 consecutive
+//         stages, pooled online; the two warp groups take alternate entries.
 // Logits are taken in base 2 (zl = (z + B) log2 e) and every exponential is the
 // multi-function unit's ex2 (relative error about 2^-22).  Each compute warp releases a
 // stage with one arrival.  Waits are bounded; after a timeout (never expected) the
 // compute threads write NaN into every entry they have not finished, so a failure
 // cannot pass for a result.
-// (The same staging for HCA, 32 rows of Z and C per stage pooled online, measured 0.68
-// of the copy rate against pool_kernel's 0.73 and is not used.)
 constexpr int kSpCols = 256;                     // columns per slice: one per compute thread
 constexpr int kSpWarps = 16;                     // compute warps: two per column group
 constexpr int kSpEntPerThread = 2;               // of a stage's 4 entries
@@ -235,13 +237,14 @@ struct SpArgs {
     int64_t items;           // B * groups * n_slices
 };
 
+template <bool kCsa>
 __global__ void __launch_bounds__(kSpThreads, 1)
 stream_pool_kernel(const __grid_constant__ CUtensorMap t0, const __grid_constant__ CUtensorMap t1,
                    const __grid_constant__ CUtensorMap t2, const __grid_constant__ CUtensorMap t3, SpArgs a)
 {
-    // t0 = Z^a, t1 = C^a, t2 = Z^b, t3 = C^b
-    constexpr int kStreams = 4;
-    constexpr int kRows = kSpStageBytes / (kStreams * kSpCols * 2);  // 16 rows: 4 blocks
+    // CSA: t0 = Z^a, t1 = C^a, t2 = Z^b, t3 = C^b.  HCA: t0 = Z, t1 = C.
+    constexpr int kStreams = kCsa ? 4 : 2;
+    constexpr int kRows = kSpStageBytes / (kStreams * kSpCols * 2);  // CSA 16 rows (4 blocks), HCA 32
     constexpr int kStreamBytes = kRows * kSpCols * 2;
     constexpr float kL2e = 1.4426950408889634f;
     extern __shared__ uint8_t smem_raw[];
@@ -255,14 +258,16 @@ stream_pool_kernel(const __grid_constant__ CUtensorMap t0, const __grid_constant
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSpStages; ++s) {
             tc::mbar_init(&full[s], 1);
-            tc::mbar_init(&empty[s], kSpWarps);
+            tc::mbar_init(&empty[s], kCsa ? kSpWarps : kSpWarps / 2);  // HCA: one warp group per item
         }
         *abort_flag = 0;
         tc::fence_mbar_init();
         tc::tma_prefetch_desc(&t0);
         tc::tma_prefetch_desc(&t1);
-        tc::tma_prefetch_desc(&t2);
-        tc::tma_prefetch_desc(&t3);
+        if (kCsa) {
+            tc::tma_prefetch_desc(&t2);
+            tc::tma_prefetch_desc(&t3);
+        }
     }
     __syncthreads();
     pdl_wait();
@@ -275,10 +280,16 @@ stream_pool_kernel(const __grid_constant__ CUtensorMap t0, const __grid_constant
     };
     // stages of an item and the entries it covers
     auto item_span = [&](int64_t g, int64_t& ent0, int& nent, int& nst) {
-        ent0 = a.e0 + g * kSpCsaEntries;
-        const int64_t left = a.e1 - ent0;
-        nent = (int)(left < kSpCsaEntries ? left : kSpCsaEntries);
-        nst = (nent + 3) / 4;
+        if (kCsa) {
+            ent0 = a.e0 + g * kSpCsaEntries;
+            const int64_t left = a.e1 - ent0;
+            nent = (int)(left < kSpCsaEntries ? left : kSpCsaEntries);
+            nst = (nent + 3) / 4;
+        } else {  // one entry of m' rows
+            ent0 = a.e0 + g;
+            nent = 1;
+            nst = a.m / kRows;
+        }
     };
 
     if (warp == kSpWarps) {
@@ -305,17 +316,85 @@ stream_pool_kernel(const __grid_constant__ CUtensorMap t0, const __grid_constant
                     tc::mbar_arrive_expect_tx(&full[s], kSpStageBytes);
                     tc::tma_load_2d(st, &t0, &full[s], x, ra + kRows * j);
                     tc::tma_load_2d(st + kStreamBytes, &t1, &full[s], x, ra + kRows * j);
-                    // b-rows one block (m = 4 rows) earlier
-                    tc::tma_load_2d(st + 2 * kStreamBytes, &t2, &full[s], x, ra - 4 + kRows * j);
-                    tc::tma_load_2d(st + 3 * kStreamBytes, &t3, &full[s], x, ra - 4 + kRows * j);
+                    if (kCsa) {  // b-rows one block (m = 4 rows) earlier
+                        tc::tma_load_2d(st + 2 * kStreamBytes, &t2, &full[s], x, ra - 4 + kRows * j);
+                        tc::tma_load_2d(st + 3 * kStreamBytes, &t3, &full[s], x, ra - 4 + kRows * j);
+                    }
                 }
             }
             // drain: every issued load has landed before the CTA may exit
             for (int j = it - kSpStages < 0 ? 0 : it - kSpStages; j < it; ++j)
                 if (!tc::mbar_wait(&full[j % kSpStages], (j / kSpStages) & 1, tc::kWaitBudget)) *abort_flag = 1;
         }
+    } else if constexpr (!kCsa) {
+        // ------------------------------------------------------------ HCA compute
+        // The two warp groups take alternate items (one entry each), so each thread keeps
+        // one online softmax state per entry (thread = column); the rows of a stage are
+        // pooled 8 at a time: the chunk maximum rescales the state once, then one ex2 per
+        // row.
+        const int col = threadIdx.x % kSpCols;
+        const int grp = threadIdx.x / kSpCols;
+        bool ok = true;
+        int64_t t = blockIdx.x, tl = 0;  // tl: the CTA's item ordinal
+        for (; t < a.items; t += gridDim.x, ++tl) {
+            if ((int)(tl & 1) != grp) continue;
+            int b, sl, nent, nst;
+            int64_t g, ent0;
+            item_of(t, b, sl, g);
+            item_span(g, ent0, nent, nst);
+            const int j = sl * kSpCols + col;
+            float mx = -INFINITY, l = 0.f, acc = 0.f;
+            for (int js = 0; js < nst; ++js) {
+                const int64_t it = tl * nst + js;  // the producer's stage count
+                const int s = (int)(it % kSpStages);
+                if (*abort_flag || !tc::mbar_wait(&full[s], (uint32_t)(it / kSpStages) & 1, tc::kWaitBudget)) {
+                    *abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                const __nv_bfloat16* sz = reinterpret_cast<const __nv_bfloat16*>(smem + s * kSpStageBytes) + col;
+                const __nv_bfloat16* sc = sz + kRows * kSpCols;
+#pragma unroll
+                for (int r0 = 0; r0 < kRows; r0 += 8) {
+                    float zl[8], xv[8], cmax = -INFINITY;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int row = kRows * js + r0 + u;  // token within the entry
+                        const float bz = a.Ba ? __ldg(&a.Ba[(int64_t)row * a.c + j]) : 0.f;
+                        zl[u] = (__bfloat162float(sz[(r0 + u) * kSpCols]) + bz) * kL2e;
+                        xv[u] = __bfloat162float(sc[(r0 + u) * kSpCols]);
+                        cmax = fmaxf(cmax, zl[u]);
+                    }
+                    const float mn = fmaxf(mx, cmax);
+                    const float f = tc::ex2_approx(mx - mn);  // 0 while the state is empty
+                    l *= f;
+                    acc *= f;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const float p = tc::ex2_approx(zl[u] - mn);
+                        l += p;
+                        acc = fmaf(p, xv[u], acc);
+                    }
+                    mx = mn;
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&empty[s]);  // this warp is done with the stage
+            }
+            if (!ok) break;
+            a.out[(int64_t)b * a.out_ld_batch + ent0 * a.c + j] = __float2bfloat16_rn(acc * tc::rcp_approx(l));
+        }
+        if (!ok) {
+            // timeout: NaN into this group's unfinished entries
+            for (; t < a.items; t += gridDim.x, ++tl) {
+                if ((int)(tl & 1) != grp) continue;
+                int b, sl;
+                int64_t g;
+                item_of(t, b, sl, g);
+                a.out[(int64_t)b * a.out_ld_batch + (a.e0 + g) * a.c + sl * kSpCols + col] = __float2bfloat16_rn(NAN);
+            }
+        }
     } else {
-        // ------------------------------------------------------------ compute: thread = column
+        // ------------------------------------------------------------ CSA compute: thread = column
         const int col = threadIdx.x % kSpCols;
         const int q0 = (threadIdx.x / kSpCols) * kSpEntPerThread;  // this thread's first entry of a stage
         int it = 0;
@@ -407,18 +486,18 @@ bool vector_ok(const PoolArgs& p, int dtype)
            aligned16(p.out) && (!p.Ba || aligned16(p.Ba)) && (!p.Bb || aligned16(p.Bb));
 }
 
-// The TMA-staged path for bf16 prefill-sized CSA calls; false when the call does not fit
-// it (not CSA, odd widths or strides, m other than 4, or too little work to fill the
-// SMs), which then runs pool_kernel.
+// The TMA-staged path for bf16 prefill-sized calls; false when the call does not fit it
+// (odd widths or strides, m other than 4 for CSA or not a multiple of 32 for HCA, or too
+// little work to fill the SMs), which then runs pool_kernel.
 bool launch_stream_pool(const PoolArgs& p, cudaStream_t stream, int& status)
 {
-    if (!p.has_b || p.m != 4) return false;
+    if (p.has_b ? p.m != 4 : p.m % 32 != 0) return false;
     if (p.c % kSpCols != 0 || p.ld_row % 8 != 0 || (p.B > 1 && p.ld_batch % p.ld_row != 0)) return false;
     if (!aligned16(p.Xa) || !aligned16(p.Za) || !aligned16(p.Xb) || !aligned16(p.Zb)) return false;
     const int64_t nent = p.e1 - p.e0;
     SpArgs a;
     a.n_slices = p.c / kSpCols;
-    a.groups = (nent + kSpCsaEntries - 1) / kSpCsaEntries;
+    a.groups = p.has_b ? (nent + kSpCsaEntries - 1) / kSpCsaEntries : nent;
     a.items = (int64_t)p.B * a.groups * a.n_slices;
     if (a.items < kNumSMs) return false;
     a.rows_per_batch = p.B > 1 ? p.ld_batch / p.ld_row : p.n_rows;
@@ -434,17 +513,23 @@ bool launch_stream_pool(const PoolArgs& p, cudaStream_t stream, int& status)
     a.e0 = p.e0;
     a.e1 = p.e1;
     CUtensorMap tm[4];
-    const void* src[4] = {p.Za, p.Xa, p.Zb, p.Xb};
+    const void* src[4] = {p.Za, p.Xa, p.has_b ? p.Zb : p.Za, p.has_b ? p.Xb : p.Xa};
     for (int i = 0; i < 4; ++i)
         if (!make_tmap_bf16_2d_plain(&tm[i], src[i], (uint64_t)height, (uint64_t)p.c, (uint64_t)p.ld_row, kSpCols,
-                                     16)) {
+                                     p.has_b ? 16 : 32)) {
             status = CSA_ERR_CUDA;
             return true;
         }
     const unsigned grid = (unsigned)(a.items < kNumSMs ? a.items : kNumSMs);
-    cudaFuncSetAttribute(stream_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSpSmem);
-    launch_pdl(stream_pool_kernel, dim3(grid), dim3(kSpThreads), (size_t)kSpSmem, stream, tm[0], tm[1], tm[2], tm[3],
-               a);
+    if (p.has_b) {
+        cudaFuncSetAttribute(stream_pool_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSpSmem);
+        launch_pdl(stream_pool_kernel<true>, dim3(grid), dim3(kSpThreads), (size_t)kSpSmem, stream, tm[0], tm[1],
+                   tm[2], tm[3], a);
+    } else {
+        cudaFuncSetAttribute(stream_pool_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSpSmem);
+        launch_pdl(stream_pool_kernel<false>, dim3(grid), dim3(kSpThreads), (size_t)kSpSmem, stream, tm[0], tm[1],
+                   tm[2], tm[3], a);
+    }
     status = launch_status();
     return true;
 }
