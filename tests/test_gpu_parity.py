@@ -243,8 +243,10 @@ def test_csa_compress_streaming_path(B, nent, c, e0, e1, bias):
     (3, 64, 120, 256, 7, False),        # a sub-range from tok0 = m' e0
 ])
 def test_hca_compress_prefill_size(B, mp, nent, c, e0, bias):
-    """Prefill-sized bf16 HCA compression (hundreds of entries, m' = 128 and 64, a
-    sub-range from tok0 = m' e0) against the oracle on every entry."""
+    """Prefill-sized bf16 HCA compression, large enough (>= 148 work items of one entry x
+    256 columns) to run the TMA-staged streaming kernel: m' = 128 and 64 (4 and 2 stages
+    of 32 rows per entry, the two warp groups on alternate entries), a sub-range from
+    tok0 = m' e0, against the oracle on every entry."""
     n = mp * nent + 17
     tok0 = mp * e0
     C, Z = randn((B, n, c), 170, torch.bfloat16), randn((B, n, c), 171, torch.bfloat16)
