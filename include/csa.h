@@ -218,10 +218,22 @@ int csa_indexer_topk(const void* qI, const float* wI, const void* KI, const int6
  *   - Every call shares the one array and clears its counters at the start (an
  *     asynchronous memset on `stream`), so calls whose GPU work overlaps, on any streams
  *     or threads, race with each other: serialise them.
+ *   - Argument errors (every code csa_indexer_topk returns before a launch, and
+ *     CSA_ERR_WORKSPACE for problems beyond the array) are returned before anything is
+ *     enqueued on `stream`.
+ *   - A device-side timeout is reported by csa_indexer_topk_noalloc_status, not by the
+ *     return value.  The next call clears it, so read it before the next call.
  * ------------------------------------------------------------------------------- */
 int csa_indexer_topk_noalloc(const void* qI, const float* wI, const void* KI, const int64_t* t,
                              int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
                              int32_t* idx_out, float* scores_out, int dtype, csa_stream_t stream);
+
+/* csa_indexer_topk_noalloc_status - the status word of the current device's fixed
+ * scratch array after the work already enqueued on `stream` (this call waits for it):
+ * CSA_ERR_TIMEOUT if a bounded wait of the last csa_indexer_topk_noalloc call gave up
+ * (its idx_out is then invalid), CSA_OK otherwise; CSA_ERR_CUDA if the copy fails.  It
+ * allocates nothing and leaves the word as it is. */
+int csa_indexer_topk_noalloc_status(csa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * csa_sparse_attn - shared-KV multi-query attention over the selected compressed
@@ -328,6 +340,16 @@ int hca_dense_attn_window(const void* q, const void* cache, const int64_t* t, co
  * of an earlier call gave up a bounded wait (its outputs are then invalid).  The status
  * word is the first 4 bytes of the workspace and stays set until it is zeroed. */
 int csa_workspace_status(const void* workspace, csa_stream_t stream);
+
+/* Test hook of the failure detection (no counterpart in the pages): sets, on `stream`,
+ * the wait budget in SM clock cycles of the one grid-wide wait of csa_indexer_topk and
+ * csa_indexer_topk_e4m3 (the meeting of a query's CTAs before the in-place top-k), kept
+ * in bytes 8-15 of that call's workspace.  0 (the zero-filled default) keeps the ~1 s
+ * budget of every other device wait.  A budget of a few cycles makes the wait run out, so
+ * a test can see CSA_ERR_TIMEOUT from csa_workspace_status without faulting or hanging
+ * the GPU: after a timeout every CTA skips its remaining selection work and the call's
+ * idx_out is invalid.  workspace: 16-byte aligned; cycles >= 0 (CSA_ERR_ARG otherwise). */
+int csa_workspace_set_wait_budget(void* workspace, int64_t cycles, csa_stream_t stream);
 
 /* Zero `bytes` of device memory on `stream` (cudaMemsetAsync); for first-use workspaces. */
 int csa_workspace_zero(void* workspace, size_t bytes, csa_stream_t stream);

@@ -15,11 +15,13 @@ from ._binding import (  # noqa: F401
     csa_indexer_topk,
     csa_indexer_topk_e4m3,
     csa_indexer_topk_noalloc,
+    csa_indexer_topk_noalloc_status,
     csa_indexer_topk_workspace_size,
     csa_quantize_e4m3,
     csa_sparse_attn,
     csa_status_string,
     csa_version,
+    csa_workspace_set_wait_budget,
     csa_workspace_status,
     csa_workspace_zero,
     hca_compress,

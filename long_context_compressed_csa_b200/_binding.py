@@ -29,9 +29,11 @@ _SIGS = {
                               vp, sz, vp], i32),
     "csa_indexer_topk_workspace_size": ([i32, i32, i64, i32], sz),
     "csa_workspace_status": ([vp, vp], i32),
+    "csa_workspace_set_wait_budget": ([vp, i64, vp], i32),
     "csa_indexer_topk": ([vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, i32, vp, vp, vp, sz, i32, vp],
                          i32),
     "csa_indexer_topk_noalloc": ([vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, i32, vp, vp, i32, vp], i32),
+    "csa_indexer_topk_noalloc_status": ([vp], i32),
     "csa_attn_workspace_size": ([i32, i32, i32, i32, i64], sz),
     "csa_sparse_attn": ([vp, vp, vp, i32, i32, i32, i32, i64, i32, f32, vp, vp, vp, sz, i32, i32, vp],
                         i32),
@@ -227,9 +229,24 @@ def csa_indexer_topk_noalloc(qI, wI, KI, t, m, k, idx_out, scores_out=None, stre
         _ptr(scores_out), _dtype(qI), _stream(stream)))
 
 
+def csa_indexer_topk_noalloc_status(stream=None) -> int:
+    """Status word of the no-allocation variant's fixed scratch after the work enqueued on
+    the stream: 0, or -7 (CSA_ERR_TIMEOUT) if a device-side wait of the last
+    csa_indexer_topk_noalloc call gave up.  The next such call clears it."""
+    return int(library().csa_indexer_topk_noalloc_status(_stream(stream)))
+
+
 def csa_workspace_status(workspace, stream=None) -> int:
     """0, or -7 (CSA_ERR_TIMEOUT) if a device-side wait of an earlier call gave up."""
     return int(library().csa_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def csa_workspace_set_wait_budget(workspace, cycles, stream=None):
+    """Test hook: the wait budget (SM cycles) of the indexer's grid-wide meeting, kept in
+    the workspace; 0 restores the default."""
+    _cuda(workspace)
+    _check("csa_workspace_set_wait_budget",
+           library().csa_workspace_set_wait_budget(_ptr(workspace), int(cycles), _stream(stream)))
 
 
 def csa_attn_workspace_size(B, nq, n_h, c, max_entries) -> int:

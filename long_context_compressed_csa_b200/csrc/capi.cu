@@ -25,3 +25,16 @@ extern "C" int csa_workspace_zero(void* workspace, size_t bytes, csa_stream_t st
     cudaError_t e = cudaMemsetAsync(workspace, 0, bytes, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
+
+namespace {
+__global__ void store_i64(int64_t* p, int64_t v) { *p = v; }
+}  // namespace
+
+extern "C" int csa_workspace_set_wait_budget(void* workspace, int64_t cycles, csa_stream_t stream)
+{
+    if (!workspace || cycles < 0) return CSA_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return CSA_ERR_ALIGN;
+    store_i64<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<int64_t*>(static_cast<char*>(workspace) + 8), cycles);
+    return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+}

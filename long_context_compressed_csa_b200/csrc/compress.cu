@@ -258,7 +258,7 @@ stream_pool_kernel(const __grid_constant__ CUtensorMap t0, const __grid_constant
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSpStages; ++s) {
             tc::mbar_init(&full[s], 1);
-            tc::mbar_init(&empty[s], kCsa ? kSpWarps : kSpWarps / 2);  // HCA: one warp group per item
+            tc::mbar_init(&empty[s], kSpWarps);  // every compute warp passes every stage
         }
         *abort_flag = 0;
         tc::fence_mbar_init();
@@ -331,17 +331,35 @@ stream_pool_kernel(const __grid_constant__ CUtensorMap t0, const __grid_constant
         // The two warp groups take alternate items (one entry each), so each thread keeps
         // one online softmax state per entry (thread = column); the rows of a stage are
         // pooled 8 at a time: the chunk maximum rescales the state once, then one ex2 per
-        // row.
+        // row.  Each group still waits for every stage of the other group's items and
+        // releases it at once, so that it observes every phase of every slot in order: a
+        // slot's full barrier can then never be a whole phase behind the parity a group
+        // waits for (TMA loads of different stages complete in any order), and a slot is
+        // refilled only after both groups have passed it.
         const int col = threadIdx.x % kSpCols;
         const int grp = threadIdx.x / kSpCols;
         bool ok = true;
         int64_t t = blockIdx.x, tl = 0;  // tl: the CTA's item ordinal
         for (; t < a.items; t += gridDim.x, ++tl) {
-            if ((int)(tl & 1) != grp) continue;
             int b, sl, nent, nst;
             int64_t g, ent0;
             item_of(t, b, sl, g);
             item_span(g, ent0, nent, nst);
+            if ((int)(tl & 1) != grp) {  // the other group's item: pass its stages
+                for (int js = 0; js < nst && ok; ++js) {
+                    const int64_t it = tl * nst + js;
+                    const int s = (int)(it % kSpStages);
+                    if (*abort_flag || !tc::mbar_wait(&full[s], (uint32_t)(it / kSpStages) & 1, tc::kWaitBudget)) {
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&empty[s]);
+                }
+                if (!ok) break;
+                continue;
+            }
             const int j = sl * kSpCols + col;
             float mx = -INFINITY, l = 0.f, acc = 0.f;
             for (int js = 0; js < nst; ++js) {

@@ -463,23 +463,12 @@ int launch_scan_cuda_core(const void* qI, const float* wI, const void* KI, const
     return launch_status();
 }
 
-}  // namespace csa
-
-extern "C" size_t csa_indexer_topk_workspace_size(int B, int nq, int64_t N_cap, int k)
+// Host-side validation of csa_indexer_topk's arguments (every error it can return before
+// a launch), shared with the no-allocation variant.
+int indexer_topk_check(const void* qI, const float* wI, const void* KI, const int64_t* t, int B, int nq,
+                       int64_t N_cap, int n_hI, int cI, int m, int k, const int32_t* idx_out,
+                       const float* scores_out, const void* workspace, size_t ws_bytes, int dtype)
 {
-    (void)k;
-    if (B <= 0 || nq <= 0 || N_cap < 0) return 0;
-    return csa::topk_ws_layout(nullptr, B * nq, N_cap).bytes + 256;
-}
-
-extern "C" int csa_indexer_topk(const void* qI, const float* wI, const void* KI,
-                                const int64_t* t, int B, int nq, int64_t N_cap, int n_hI,
-                                int cI, int m, int k, int32_t* idx_out, float* scores_out,
-                                void* workspace, size_t ws_bytes, int dtype,
-                                csa_stream_t stream_)
-{
-    using namespace csa;
-    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (dtype != CSA_BF16 && dtype != CSA_F32) return CSA_ERR_DTYPE;
     if (B < 0 || nq < 0 || N_cap < 0 || N_cap >= (int64_t(1) << 31) || n_hI <= 0 || cI <= 0 ||
         m <= 0 || k <= 0)
@@ -491,9 +480,37 @@ extern "C" int csa_indexer_topk(const void* qI, const float* wI, const void* KI,
         ((uintptr_t)idx_out & 3) || ((uintptr_t)scores_out & 3) || !aligned16(workspace))
         return CSA_ERR_ALIGN;
     if ((int64_t)B * nq > 65535) return CSA_ERR_UNSUPPORTED;  // one grid row per query
-    const int G = B * nq;
     if (!workspace || ws_bytes < csa_indexer_topk_workspace_size(B, nq, N_cap, k))
         return CSA_ERR_WORKSPACE;
+    // the CUDA-core scan stages q^I and w^I of one query in shared memory
+    const bool tc_path = dtype == CSA_BF16 && indexer_tc_supported(n_hI, cI);
+    if (!tc_path && ((size_t)n_hI * cI + n_hI) * sizeof(float) > 160 * 1024) return CSA_ERR_UNSUPPORTED;
+    return CSA_OK;
+}
+
+}  // namespace csa
+
+extern "C" size_t csa_indexer_topk_workspace_size(int B, int nq, int64_t N_cap, int k)
+{
+    (void)k;
+    if (B <= 0 || nq <= 0 || N_cap < 0) return 0;
+    const int64_t G = (int64_t)B * nq;
+    if (G > 65535) return 0;  // beyond the supported number of queries per call
+    return csa::topk_ws_layout(nullptr, (int)G, N_cap).bytes + 256;
+}
+
+extern "C" int csa_indexer_topk(const void* qI, const float* wI, const void* KI,
+                                const int64_t* t, int B, int nq, int64_t N_cap, int n_hI,
+                                int cI, int m, int k, int32_t* idx_out, float* scores_out,
+                                void* workspace, size_t ws_bytes, int dtype,
+                                csa_stream_t stream_)
+{
+    using namespace csa;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    const int chk = indexer_topk_check(qI, wI, KI, t, B, nq, N_cap, n_hI, cI, m, k, idx_out, scores_out,
+                                       workspace, ws_bytes, dtype);
+    if (chk != CSA_OK || B == 0 || nq == 0) return chk;
+    const int G = B * nq;
     TopkWs ws = topk_ws_layout(workspace, G, N_cap);
     int st;
     bool fused = false;

@@ -14,7 +14,9 @@ CSA_DEV uint32_t hist_slot(uint32_t bin) { return (bin & 15u) * 256u + (bin >> 4
 
 // Workspace of csa_indexer_topk, carved from one caller buffer.
 struct TopkWs {
-    uint32_t* status; // sticky device status: nonzero after a bounded wait timed out
+    uint32_t* status; // 256-byte status block: word 0 the sticky device status (nonzero after
+                      // a bounded wait timed out); bytes 8-15 an int64 wait budget (SM cycles)
+                      // for the in-place select's grid meeting, 0 for the default
     uint32_t* hist0;  // [G][kBins] digit-0 histogram (zero between calls)
     uint32_t* ctr;    // [G][kCtrs] counters (zero between calls)
     float* scores;    // [G][ld] fp32 scores of the visible entries
@@ -49,6 +51,10 @@ int launch_scan_mq(const void* qI, const float* wI, const void* KI, const int64_
 int launch_scan_cuda_core(const void* qI, const float* wI, const void* KI, const int64_t* t,
                           int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
                           const TopkWs& ws, int dtype, cudaStream_t stream);
+// Every error csa_indexer_topk reports before a launch (CSA_OK when the call may run).
+int indexer_topk_check(const void* qI, const float* wI, const void* KI, const int64_t* t, int B, int nq,
+                       int64_t N_cap, int n_hI, int cI, int m, int k, const int32_t* idx_out,
+                       const float* scores_out, const void* workspace, size_t ws_bytes, int dtype);
 // self_hist: one CTA per query, which builds the digit-0 histogram from the scores itself
 // (after a scan that leaves ws.hist0 untouched).
 int launch_topk_select(const TopkWs& ws, const int64_t* t, int G, int m, int k, int64_t N_cap,

@@ -53,16 +53,35 @@ extern "C" int csa_indexer_topk_noalloc(const void* qI, const float* wI, const v
     using namespace csa;
     if (B < 0 || nq < 0 || N_cap < 0 || N_cap >= (int64_t(1) << 31)) return CSA_ERR_ARG;
     if (B == 0 || nq == 0) return CSA_OK;
+    if ((int64_t)B * nq > 65535) return CSA_ERR_UNSUPPORTED;  // before any size arithmetic
     const size_t need = csa_indexer_topk_workspace_size(B, nq, N_cap, k);
     if (need == 0 || need > kScratchBytes) return CSA_ERR_WORKSPACE;  // beyond the fixed scratch
     void* scratch = nullptr;
     int st = scratch_address(&scratch);
     if (st != CSA_OK) return st;
+    // Every argument error is reported here, before anything is enqueued on the stream.
+    st = indexer_topk_check(qI, wI, KI, t, B, nq, N_cap, n_hI, cI, m, k, idx_out, scores_out, scratch,
+                            kScratchBytes, dtype);
+    if (st != CSA_OK) return st;
     // The array keeps whatever the previous call left; the histograms, counters and the
-    // status word must start at zero.
+    // status word (which a previous call's timeout may have set) must start at zero.
     const size_t zero = topk_ws_layout(nullptr, B * nq, N_cap).zero_bytes;
     if (cudaMemsetAsync(scratch, 0, zero, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return CSA_ERR_CUDA;
     return csa_indexer_topk(qI, wI, KI, t, B, nq, N_cap, n_hI, cI, m, k, idx_out, scores_out, scratch,
                             kScratchBytes, dtype, stream);
+}
+
+extern "C" int csa_indexer_topk_noalloc_status(csa_stream_t stream)
+{
+    using namespace csa;
+    void* scratch = nullptr;
+    const int st = scratch_address(&scratch);
+    if (st != CSA_OK) return st;
+    uint32_t word = 0;  // the status word: the first 4 bytes of the scratch
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    return word ? CSA_ERR_TIMEOUT : CSA_OK;
 }

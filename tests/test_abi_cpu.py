@@ -92,6 +92,13 @@ def test_host_validation_rejects_bad_arguments_without_launching(lib):
                                 fake, 1 << 62, 0, None) == -6
     assert lib.csa_indexer_topk_e4m3(fake, fake, fake, fake, fake, 2, 40000, 100, 64, 128, 4, 8, fake,
                                      None, fake, 1 << 62, None) == -6
+    # the no-allocation variant: B * nq above the limit (checked before any size
+    # arithmetic, which would overflow), and a problem larger than its fixed scratch
+    assert lib.csa_indexer_topk_noalloc(fake, fake, fake, fake, 40000, 40000, 100, 64, 128, 4, 5, fake,
+                                        None, 0, None) == -6
+    assert lib.csa_indexer_topk_noalloc(fake, fake, fake, fake, 1, 1, 1 << 20, 64, 128, 4, 5, fake,
+                                        None, 0, None) == -4
+    assert lib.csa_indexer_topk_workspace_size(40000, 40000, 100, 5) == 0
     # attention: out_bf16 with fp32, c too wide, workspace too small
     assert lib.csa_sparse_attn(fake, fake, fake, 1, 1, 4, 64, 100, 8, 0.0, fake, None, fake,
                                1 << 30, 1, 1, None) == -3

@@ -23,7 +23,10 @@ def _run(fn_kind, qI, wI, KI, t, m, k):
                          device="cuda")
         csa_indexer_topk(qI, wI, KI, t, m, k, idx, ws, scores_out=sc)
     else:
+        from long_context_compressed_csa_b200 import csa_indexer_topk_noalloc_status
         csa_indexer_topk_noalloc(qI, wI, KI, t, m, k, idx, scores_out=sc)
+        # a device-side timeout would show here (the next call clears it)
+        assert csa_indexer_topk_noalloc_status() == 0
     torch.cuda.synchronize()
     return idx.cpu().numpy(), sc.cpu().numpy()
 
@@ -49,6 +52,11 @@ def test_noalloc_matches_workspace_entry_point_twice_in_a_row():
         # a second, different problem right after: CUDA-core path (fp32, 16 heads x 32)
         (randn((2, 1, 16, 32), 710, torch.float32), randn((2, 1, 16), 711, torch.float32),
          randn((2, 9000, 32), 712, torch.float32), [[4 * 9000 + 3], [4 * 5000]]),
+        # then a chunk of 16 queries (the many-query scan, which leaves the digit-0
+        # histograms untouched, then one select CTA per query), starting from the scratch
+        # the two calls above left behind; visible counts from below k to all keys
+        (randn((1, 16, 64, 128), 720, torch.bfloat16), randn((1, 16, 64), 721, torch.float32),
+         randn((1, 3000, 128), 722, torch.bfloat16), [[4 * 100 + 800 * j for j in range(16)]]),
     ]
     for qI, wI, KI, t in cases:
         qI, wI, KI = qI.cuda(), wI.cuda(), KI.cuda()
