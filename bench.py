@@ -273,33 +273,97 @@ def kernel_launches_per_step(dec, j):
 
 
 # ----------------------------------------------------------------------------------
-# CPU oracle baseline (bounded sample of the same workload)
+# CPU oracle baseline (bounded sample of the same workload, on the host's cores)
 # ----------------------------------------------------------------------------------
-def cpu_baseline(n_steps=2, seed=77):
+def _oracle_inputs(workload, seed):
+    """Seeded inputs of one decode step of `workload` for the oracle (float64 numpy)."""
     import torch
-    import oracle
     from long_context_compressed_csa_b200.synth import randn, to_f64
-    n, m, mp, c, cI, n_h, n_hI, k = 1 << 20, 4, 128, 512, 128, 128, 64, 1024
-    N, Nh = n // m, n // mp
-    KI = to_f64(randn((N, cI), seed, torch.bfloat16))
-    hc = to_f64(randn((Nh, c), seed + 1, torch.bfloat16))
-    rows = to_f64(randn((4096, c), seed + 2, torch.bfloat16))  # CSA entries, indexed mod 4096
-    q = to_f64(randn((n_h, c), seed + 3, torch.bfloat16))
-    qI = to_f64(randn((n_hI, cI), seed + 4, torch.bfloat16))
-    wI = to_f64(randn((n_hI,), seed + 5, torch.float32))
-    t0 = time.perf_counter()
-    for j in range(n_steps):
-        t = n + j
-        s = oracle.index_scores(qI, wI, KI, oracle.visible(t, m, N))
-        sel = oracle.topk(s, k)
-        oracle.mqa(q, rows[sel % rows.shape[0]], np.arange(k, dtype=np.int32))
-        oracle.mqa(q, hc, np.arange(oracle.visible(t, mp, Nh), dtype=np.int32))
-    dt = time.perf_counter() - t0
-    return {"value": n_steps / dt, "unit": "layer-pair decode steps/s", "cores": 1, "kind": "oracle",
-            "sample": "%d decode steps of one CSA+HCA layer pair at t=2^20 (indexer over 262144 "
-                      "keys, full-sort top-1024, 128-head MQA over 1024 + 8192 entries), fp64, "
-                      "single-threaded" % n_steps,
-            "seconds": dt}
+    bf = torch.bfloat16
+    if workload == "hybrid_1m_decode":
+        n, m, mp, c, cI, n_h, n_hI = 1 << 20, 4, 128, 512, 128, 128, 64
+        return {"KI": to_f64(randn((n // m, cI), seed, bf)), "hc": to_f64(randn((n // mp, c), seed + 1, bf)),
+                "rows": to_f64(randn((4096, c), seed + 2, bf)),  # CSA entries, indexed mod 4096
+                "q": to_f64(randn((n_h, c), seed + 3, bf)), "qI": to_f64(randn((n_hI, cI), seed + 4, bf)),
+                "wI": to_f64(randn((n_hI,), seed + 5, torch.float32))}
+    if workload in ("csa_decode_8k", "csa_prefill_decode_b4_256k"):
+        n = 8192 if workload == "csa_decode_8k" else 262144
+        m, c, cI, n_h, n_hI = 4, 512, 128, 128, 64
+        return {"KI": to_f64(randn((n // m, cI), seed, bf)), "cache": to_f64(randn((n // m, c), seed + 1, bf)),
+                "q": to_f64(randn((n_h, c), seed + 3, bf)), "qI": to_f64(randn((n_hI, cI), seed + 4, bf)),
+                "wI": to_f64(randn((n_hI,), seed + 5, torch.float32))}
+    if workload == "hca_decode_b16_128k":
+        return {"hc": to_f64(randn((1024, 512), seed + 1, bf)), "q": to_f64(randn((128, 512), seed + 3, bf))}
+    raise ValueError(workload)
+
+
+def _oracle_step(workload, x, j):
+    """One decode step of one sequence through the oracle (the unit of the workload's
+    metric divided by its batch)."""
+    import oracle
+    if workload == "hybrid_1m_decode":
+        t = (1 << 20) + j
+        s = oracle.index_scores(x["qI"], x["wI"], x["KI"], oracle.visible(t, 4, x["KI"].shape[0]))
+        sel = oracle.topk(s, 1024)
+        oracle.mqa(x["q"], x["rows"][sel % x["rows"].shape[0]], np.arange(1024, dtype=np.int32))
+        oracle.mqa(x["q"], x["hc"], np.arange(oracle.visible(t, 128, x["hc"].shape[0]), dtype=np.int32))
+    elif workload in ("csa_decode_8k", "csa_prefill_decode_b4_256k"):
+        k = 512 if workload == "csa_decode_8k" else 1024
+        N = x["KI"].shape[0]
+        s = oracle.index_scores(x["qI"], x["wI"], x["KI"], oracle.visible(4 * N + j, 4, N))
+        oracle.mqa(x["q"], x["cache"], oracle.topk(s, k))
+    else:
+        oracle.mqa(x["q"], x["hc"], np.arange(1024, dtype=np.int32))
+
+
+def _oracle_worker(workload, seed, steps, barrier, queue):
+    x = _oracle_inputs(workload, seed)
+    _oracle_step(workload, x, 0)  # warm: loads the oracle library
+    barrier.wait()
+    t0 = time.monotonic()
+    for j in range(steps):
+        _oracle_step(workload, x, j + 1)
+    queue.put((t0, time.monotonic(), steps))
+
+
+# per-sequence oracle steps of each workload in one worker, about 10-30 s of CPU work in all
+ORACLE_STEPS = {"hybrid_1m_decode": 1, "csa_decode_8k": 20, "hca_decode_b16_128k": 8,
+                "csa_prefill_decode_b4_256k": 3}
+ORACLE_MAX_WORKERS = 16
+
+
+def cpu_baseline(workload="hybrid_1m_decode", seed=77, steps=None):
+    """The oracle timed on the host's cores: one spawned process per core (at most
+    ORACLE_MAX_WORKERS), each running whole decode steps of its own sequence after a
+    common barrier; value = all steps / the wall time of the concurrent region, in the
+    workload's unit (a layer-pair step of the hybrid workload is one token)."""
+    import multiprocessing as mp_
+    host = len(os.sched_getaffinity(0))
+    P = max(1, min(host, ORACLE_MAX_WORKERS))
+    steps = steps or ORACLE_STEPS[workload]
+    ctx = mp_.get_context("spawn")  # never fork a process that has touched the GPU
+    barrier, queue = ctx.Barrier(P), ctx.Queue()
+    procs = [ctx.Process(target=_oracle_worker, args=(workload, seed + 1000 * w, steps, barrier, queue))
+             for w in range(P)]
+    for pr in procs:
+        pr.start()
+    res = [queue.get(timeout=600) for _ in range(P)]
+    for pr in procs:
+        pr.join()
+    wall = max(r[1] for r in res) - min(r[0] for r in res)
+    total = sum(r[2] for r in res)
+    unit = "layer-pair decode steps/s" if workload == "hybrid_1m_decode" else "decode tokens/s"
+    what = {"hybrid_1m_decode": "one CSA+HCA layer pair at t=2^20 (indexer over 262144 keys, full-sort "
+                                "top-1024, 128-head MQA over 1024 + 8192 entries)",
+            "csa_decode_8k": "one CSA layer at t=8192 (indexer over 2048 keys, top-512, 128-head MQA "
+                             "over 512 entries)",
+            "hca_decode_b16_128k": "one sequence's HCA dense MQA at t=131072 (128 heads over 1024 entries)",
+            "csa_prefill_decode_b4_256k": "one sequence's CSA step at t=262144 (indexer over 65536 keys, "
+                                          "top-1024, 128-head MQA over 1024 entries)"}[workload]
+    return {"value": total / wall, "unit": unit, "cores": P, "host_cores": host, "kind": "oracle",
+            "sample": "%d processes x %d decode steps of %s, fp64 oracle, one process per core"
+                      % (P, steps, what),
+            "seconds": wall}
 
 
 # ----------------------------------------------------------------------------------
@@ -478,12 +542,260 @@ def micro(kind, iters, rotate=4, nq_prefill=1024, batch=16):
 
 
 # ----------------------------------------------------------------------------------
+# timing helpers
+# ----------------------------------------------------------------------------------
+def graph_replay_ms(torch, fns, reps):
+    """Capture the calls `fns` once in one CUDA graph and replay it `reps` times, each
+    replay bracketed by CUDA events on the stream it is launched on; returns the
+    per-replay milliseconds (after one untimed replay)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for f in fns:
+            f()
+    g.replay()
+    torch.cuda.synchronize()
+    out = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        b.synchronize()
+        out.append(a.elapsed_time(b))
+    del g
+    return np.array(out)
+
+
+def back_to_back_launch_us(torch, fns, reps=8):
+    """Per-launch device time of a call issued back to back: `fns` (>= 64 calls, inputs
+    rotated so they stream from HBM) captured in one graph and replayed `reps` times;
+    each replay gives one sample = its duration / len(fns).  No event node sits between
+    the calls, so each launch keeps its overlap with its neighbours as in a step."""
+    ms = graph_replay_ms(torch, fns, reps)
+    per = ms * 1e3 / len(fns)
+    return {"median_us": float(np.median(per)), "mean_us": float(per.mean()), "min_us": float(per.min()),
+            "max_us": float(per.max()), "samples": int(reps), "timed_launches": int(reps * len(fns))}
+
+
+def time_step_graphs(torch, step, s_lo, s_hi, group=IDX_SAMPLE):
+    """Steps s_lo..s_hi-1 captured in CUDA graphs of `group` consecutive steps and replayed
+    in order between two CUDA events; returns the elapsed milliseconds."""
+    graphs = []
+    for a0 in range(s_lo, s_hi, group):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for s in range(a0, min(a0 + group, s_hi)):
+                step(s)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for g in graphs:
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del graphs
+    return a.elapsed_time(b)
+
+
+def roofline_obj(kernel, nbytes, t, hbm, src, traffic, how):
+    ach = nbytes / (t["mean_us"] * 1e-6) / 1e9
+    return {"kernel": kernel, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+            "frac": ach / hbm, "peak_source": src + " (burst copy)", "traffic": traffic,
+            "algorithmic_bytes_per_launch": nbytes, "avg_launch_us": t["mean_us"],
+            "median_launch_us": t["median_us"],
+            "frac_at_median": nbytes / (t["median_us"] * 1e-6) / 1e9 / hbm,
+            "timed_launches": t["timed_launches"], "samples": t["samples"], "how": how}
+
+
+HOW_B2B = ("%d back-to-back launches per CUDA graph (inputs rotated over independent layer caches, "
+           "no event node between calls), %d graph replays each timed by CUDA events on the launching "
+           "stream: avg = mean of the replays' per-launch times, median = their median")
+
+
+# ----------------------------------------------------------------------------------
+# presets: the other workload configurations, each with its own timed units
+# ----------------------------------------------------------------------------------
+def preset_config(name, extra=None):
+    from long_context_compressed_csa_b200.synth import WORKLOADS
+    cfg = {"workload": name}
+    cfg.update(WORKLOADS[name])
+    cfg.update(extra or {})
+    return cfg
+
+
+def run_preset(torch, name, args, world, rank):
+    """Configs other than the 1M hybrid decode (one layer, B sequences):
+      csa_decode_8k              prefill compress of both caches; step = indexer + top-k +
+                                 sparse MQA for the query at t = 8192
+      hca_decode_b16_128k        hca_compress over all 16 x 131072 tokens; step = dense MQA
+                                 of 16 queries (one per sequence) at t = 131072
+      csa_prefill_decode_b4_256k prefill compress of both caches; steps = 64 decode tokens per
+                                 sequence (indexer + top-k + sparse MQA of 4 queries, with the
+                                 incremental compression of both caches every m = 4 tokens)
+    Independent layer caches are rotated so that a step's inputs stream from HBM.
+    `value` = decode tokens per second (B tokens per step)."""
+    import long_context_compressed_csa_b200 as lib
+    from long_context_compressed_csa_b200.synth import randn
+    bf16, dev = torch.bfloat16, "cuda"
+    hbm, tf, src = peaks()
+    W = max(3, args.warmup)
+    seed = 7000 + 17 * rank
+    c, cI, n_h, n_hI, m, mp = 512, 128, 128, 64, 4, 128
+    if name == "hca_decode_b16_128k":
+        B, n = 16, 131072
+        Nh = n // mp
+        L = 8  # 8 x 16.8 MB of entries between revisits of a layer
+        caches = [torch.empty((B, Nh, c), dtype=bf16, device=dev) for _ in range(L)]
+        pre_ms = []
+        for l in range(L):  # prefill: 4.3 GB of C and Z per layer, compressed as one call
+            C = randn((B, n, c), seed + 10 * l, bf16, dev)
+            Z = randn((B, n, c), seed + 10 * l + 1, bf16, dev)
+            lib.hca_compress(C, Z, caches[l], mp)  # warm
+            pre_ms.append(float(np.median(graph_replay_ms(torch, [lambda: lib.hca_compress(C, Z, caches[l], mp)], 3))))
+            del C, Z
+        q = randn((L, B, 1, n_h, c), seed + 5, bf16, dev)
+        t = torch.full((B, 1), n, dtype=torch.int64, device=dev)
+        o = torch.empty((B, 1, n_h, c), dtype=torch.float32, device=dev)
+        ws = torch.zeros(lib.csa_attn_workspace_size(B, 1, n_h, c, Nh), dtype=torch.uint8, device=dev)
+        step = lambda s: lib.hca_dense_attn(q[s % L], caches[s % L], t, mp, o, ws)
+        step_bytes = B * Nh * c * 2
+        launches_per_step = 2
+        pre_bytes = 2 * B * n * c * 2 + B * Nh * c * 2
+        dom = ("hca_dense_attn (attn_pair_kernel + attn_combine), 16 queries x 1024 entries",
+               step_bytes, [lambda s=s: step(s) for s in range(64)])
+    else:
+        B, n, k = (1, 8192, 512) if name == "csa_decode_8k" else (4, 262144, 1024)
+        N = n // m
+        L = 64 if B == 1 else 4  # 64 x 2.5 MB, or 4 x 336 MB, between revisits of a layer
+        steps_dec = 64 if B == 4 else 0  # decode tokens appended per sequence
+        N_cap = N + steps_dec // m + 1
+        caches = [torch.empty((B, N_cap, c), dtype=bf16, device=dev) for _ in range(L)]
+        kIs = [torch.empty((B, N_cap, cI), dtype=bf16, device=dev) for _ in range(L)]
+        rw = 4 * (c + cI)  # one token's rows of the 4 cache streams and the 4 key streams
+        hist = 2 * m
+        rows = [randn((B, hist + steps_dec, rw), seed + 10 * l + 9, bf16, dev) for l in range(L)]
+        pre_ms = []
+        if B == 1:  # all layers' streams first, so none is still in L2 when compressed
+            S = [randn((B, n, rw), seed + 10 * l, bf16, dev) for l in range(L)]
+            fns = []
+            for l in range(L):
+                v = [S[l][:, :, i * c:(i + 1) * c] for i in range(4)]
+                vI = [S[l][:, :, 4 * c + i * cI:4 * c + (i + 1) * cI] for i in range(4)]
+                fns.append(lambda v=v, l=l: lib.csa_compress(*v, caches[l], m, 0, N))
+                fns.append(lambda vI=vI, l=l: lib.csa_compress(*vI, kIs[l], m, 0, N))
+            for f in fns:
+                f()
+            pre_ms = list(graph_replay_ms(torch, fns, 3) / L)
+            del S, fns
+        else:
+            for l in range(L):  # 5.4 GB of streams per layer, one layer at a time
+                S = randn((B, n, rw), seed + 10 * l, bf16, dev)
+                v = [S[:, :, i * c:(i + 1) * c] for i in range(4)]
+                vI = [S[:, :, 4 * c + i * cI:4 * c + (i + 1) * cI] for i in range(4)]
+                fns = [lambda: lib.csa_compress(*v, caches[l], m, 0, N),
+                       lambda: lib.csa_compress(*vI, kIs[l], m, 0, N)]
+                for f in fns:
+                    f()
+                pre_ms.append(float(np.median(graph_replay_ms(torch, fns, 3))))
+                del S, v, vI, fns
+        nQ = 16
+        q = randn((nQ, B, 1, n_h, c), seed + 5, bf16, dev)
+        qI = randn((nQ, B, 1, n_hI, cI), seed + 6, bf16, dev)
+        wI = randn((nQ, B, 1, n_hI), seed + 7, torch.float32, dev)
+        T = max(1, steps_dec)
+        tpos = torch.arange(n, n + T, dtype=torch.int64, device=dev).reshape(T, 1, 1).expand(T, B, 1).contiguous()
+        idx = torch.empty((B, 1, k), dtype=torch.int32, device=dev)
+        o = torch.empty((B, 1, n_h, c), dtype=torch.float32, device=dev)
+        ws_t = torch.zeros(lib.csa_indexer_topk_workspace_size(B, 1, N_cap, k), dtype=torch.uint8, device=dev)
+        ws_a = torch.zeros(lib.csa_attn_workspace_size(B, 1, n_h, c, k), dtype=torch.uint8, device=dev)
+
+        def step(s):
+            l, j = s % L, (s // L) % T  # token j of every sequence through layer l
+            lib.csa_indexer_topk(qI[s % nQ], wI[s % nQ], kIs[l], tpos[j], m, k, idx, ws_t)
+            lib.csa_sparse_attn(q[s % nQ], caches[l], idx, o, ws_a)
+            tok = n + j
+            if steps_dec and (tok + 1) % m == 0:  # the token completes entry i
+                i = (tok + 1) // m - 1
+                lo = m * (i - 1)
+                r0 = lo - (n - hist)
+                R = rows[l][:, r0:r0 + 2 * m]
+                lib.csa_compress(*[R[:, :, a * c:(a + 1) * c] for a in range(4)], caches[l], m, i, i + 1, tok0=lo)
+                lib.csa_compress(*[R[:, :, 4 * c + a * cI:4 * c + (a + 1) * cI] for a in range(4)], kIs[l], m,
+                                 i, i + 1, tok0=lo)
+
+        def bytes_of(s):
+            j = (s // L) % T
+            tok = n + j
+            b = B * ((tok // m) * cI * 2 + k * c * 2)
+            if steps_dec and (tok + 1) % m == 0:
+                b += B * (4 * 2 * m * (c + cI) * 2 + (c + cI) * 2)
+            return b
+        launches_per_step = 3
+        pre_bytes = B * (4 * n * (c + cI) * 2 + N * (c + cI) * 2)
+        dom = ("csa_indexer_topk (scan_tc_kernel with the top-k select in place), %d x %d keys" % (B, N),
+               B * N * cI * 2,
+               [lambda l=l: lib.csa_indexer_topk(qI[l % nQ], wI[l % nQ], kIs[l % L], tpos[0], m, k, idx, ws_t)
+                for l in range(64)])
+    # steps: a whole number of layer rotations, at least the requested count
+    K = max(args.steps, L)
+    if name == "csa_prefill_decode_b4_256k":
+        K = max(K, L * 64)  # 64 decode tokens per sequence through every layer
+    K = (K + L - 1) // L * L
+    for s in range(min(W, 8)):
+        step(s)
+    torch.cuda.synchronize()
+    time_step_graphs(torch, step, 0, W)
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    sampler.start()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    ms = time_step_graphs(torch, step, W, W + K)
+    clocks = sampler.stop()
+    ms_all = max_over_ranks(ms, "cuda")
+    if name == "hca_decode_b16_128k":
+        total_bytes = K * step_bytes
+        gpu_launches = K * launches_per_step
+    else:
+        total_bytes = sum(bytes_of(s) for s in range(W, W + K))
+        gpu_launches = sum(3 + (2 if steps_dec and (n + (s // L) % T + 1) % m == 0 else 0)
+                           for s in range(W, W + K))
+    t_dom = back_to_back_launch_us(torch, dom[2], reps=8)
+    step_gbs = total_bytes / (ms / 1e3) / 1e9
+    pre_us = float(np.median(pre_ms)) * 1e3
+    line = {
+        "metric": METRIC, "value": whole_job_rate(K * B, world, ms_all), "unit": "decode tokens/s",
+        "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms_all / K,
+        "us_per_step": ms_all / K * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": preset_config(name, {"layers_rotated": L, "parallelism": "replicas" if world > 1 else "single",
+                                       "l2": "inputs larger than L2: %d independent layer caches rotated" % L}),
+        "roofline": roofline_obj(dom[0], dom[1], t_dom, hbm, src, None, HOW_B2B % (len(dom[2]), 8)),
+        "step_roofline": {"achieved": step_gbs, "peak": hbm, "unit": "GB/s", "frac": step_gbs / hbm,
+                          "bytes_per_step": total_bytes / K},
+        "prefill_compress": {"us": pre_us, "bytes": pre_bytes, "achieved": pre_bytes / (pre_us * 1e-6) / 1e9,
+                             "peak": hbm, "unit": "GB/s", "frac": pre_bytes / (pre_us * 1e-6) / 1e9 / hbm},
+        "gpu_launches": gpu_launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        base = cpu_baseline(name)
+        line["cpu_baseline"] = {k2: base[k2] for k2 in ("value", "unit", "cores", "host_cores", "kind", "sample")}
+    return line
+
+
+# ----------------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2048)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=["hybrid_1m_decode", "csa_decode_8k", "hca_decode_b16_128k",
+                             "csa_prefill_decode_b4_256k"],
+                    help="the configuration timed (default: the 1M-token hybrid decode)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--micro", default=None,
@@ -507,13 +819,16 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        base = cpu_baseline(n_steps=max(1, min(args.steps, 3)))
+        import oracle
+        oracle.build()
+        base = cpu_baseline(args.workload)
+        cfg = workload_config(args.gpus) if args.workload == WORKLOAD else preset_config(args.workload)
         line = {"impl": "reference", "metric": METRIC, "value": base["value"], "unit": base["unit"],
-                "n_gpus": args.gpus, "steps": max(1, min(args.steps, 3)), "warmup": 0,
+                "n_gpus": args.gpus, "steps": base["cores"] * ORACLE_STEPS[args.workload], "warmup": 0,
                 "ms_per_step": 1000.0 / base["value"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": workload_config(args.gpus),
-                "cpu_baseline": {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "config": cfg,
+                "cpu_baseline": {k: base[k] for k in ("value", "unit", "cores", "host_cores", "kind", "sample")},
                 "e2e": {"value": base["value"], "unit": base["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -527,8 +842,20 @@ def main():
     from long_context_compressed_csa_b200 import build
     if rank == 0:
         build.build()
+        if not args.no_cpu:
+            import oracle
+            oracle.build()
     if world > 1:
         dist.barrier()
+
+    if args.workload != WORKLOAD:
+        line = run_preset(torch, args.workload, args, world, rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
 
     W, K = max(3, args.warmup), args.steps
     dec = HybridDecode(torch, W + K, seed=5000 + 17 * rank)
@@ -591,19 +918,23 @@ def main():
     ms = start.elapsed_time(end)
     idx_ms = np.array([ev[0].elapsed_time(ev[1]) for _, ev in graphs])
     ms_all = max_over_ranks(ms, "cuda")
+    del graphs, warm_graphs
 
     bytes_total = sum(dec.step_bytes(s // N_PAIRS) for s in range(W, W + K))
     launches = sum(kernel_launches_per_step(dec, s // N_PAIRS) for s in range(W, W + K))
-    log("indexer+topk per launch: mean %.2f us, median %.2f us; step %.2f us" %
-        (idx_ms.mean() * 1e3, np.median(idx_ms) * 1e3, ms * 1e3 / K))
     hbm, tf, src = peaks()
     value = whole_job_rate(K, world, ms_all)
 
-    # ---- dominant kernel: the indexer (scan over every visible key, then top-k) ----
-    vis = (dec.n + (W // N_PAIRS)) // dec.m
+    # ---- dominant kernel: the indexer (scan over every visible key, then top-k), timed
+    # back to back over the 8 layer pairs' keys at the first timed token position ----
+    j0 = W // N_PAIRS
+    vis = (dec.n + j0) // dec.m
     idx_bytes = vis * dec.cI * 2
-    idx_avg_s = float(idx_ms.mean()) / 1000.0
-    achieved = idx_bytes / idx_avg_s / 1e9
+    t_idx = back_to_back_launch_us(
+        torch, [lambda p=p: dec.step(p, j0, part=0) for _ in range(8) for p in range(N_PAIRS)], reps=8)
+    log("indexer+topk per launch: back to back mean %.2f us, median %.2f us; in the step (event nodes) "
+        "mean %.2f us over %d; step %.2f us" % (t_idx["mean_us"], t_idx["median_us"], idx_ms.mean() * 1e3,
+                                                len(idx_ms), ms * 1e3 / K))
     step_gbs = bytes_total / (ms / 1000.0) / 1e9
 
     # ---- end to end through the C ABI with host buffers ----
@@ -611,22 +942,17 @@ def main():
     if not args.no_e2e:
         e2e = run_e2e(torch, dec, W, min(K, 512), world)
 
-    del graphs
+    roof = roofline_obj("csa_indexer_topk (scan_tc_kernel: indexer scan with the top-k select in place)",
+                        idx_bytes, t_idx, hbm, src, SCAN_TRAFFIC_BYTES, HOW_B2B % (64, 8))
+    roof["in_step_event_nodes_us_mean"] = float(idx_ms.mean() * 1e3)
+    roof["in_step_event_nodes_samples"] = int(len(idx_ms))
     line = {
         "metric": METRIC, "value": value, "unit": "layer-pair decode steps/s",
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms_all / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": workload_config(world),
-        "roofline": {"kernel": "csa_indexer_topk (scan_tc_kernel: indexer scan with the top-k "
-                               "select in place)", "bound": "hbm",
-                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_source": src + " (burst copy)", "traffic": SCAN_TRAFFIC_BYTES,
-                     "algorithmic_bytes_per_launch": idx_bytes,
-                     "avg_launch_us": idx_avg_s * 1e6,
-                     "timed_launches": int(len(idx_ms)),
-                     "how": "in-graph event record nodes around the call in the first step of "
-                            "each %d-step CUDA graph" % IDX_SAMPLE},
+        "roofline": roof,
         "step_roofline": {"achieved": step_gbs, "peak": hbm, "unit": "GB/s", "frac": step_gbs / hbm,
                           "bytes_per_step": bytes_total / K},
         "gpu_launches": launches,
@@ -636,7 +962,7 @@ def main():
         line["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu:
         base = cpu_baseline()
-        line["cpu_baseline"] = {k: base[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        line["cpu_baseline"] = {k: base[k] for k in ("value", "unit", "cores", "host_cores", "kind", "sample")}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
