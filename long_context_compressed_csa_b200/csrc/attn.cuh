@@ -42,6 +42,7 @@ struct AttnPlan {
     int splits = 1;
     int64_t per_split = 1;
     int head_groups = 1;
+    int kernel = 0;  // 0: CUDA cores; 1: tcgen05, full-width splits (attn_tc.cu); 2: tcgen05 CTA pairs (attn_pair.cu)
 };
 
 AttnPlan attn_plan_cuda_core(int G, int n_h, int64_t entries);
@@ -49,6 +50,7 @@ AttnPlan attn_plan_tc(int G, int n_h, int c, int64_t entries);
 bool attn_tc_supported(int n_h, int c);
 size_t attn_ws_bytes(int G, int n_h, int c, int splits);
 int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cudaStream_t stream);
+int launch_attn_pair(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cudaStream_t stream);
 // normalized: part_o holds bf16 O_i / l_i (tcgen05 path) instead of fp32 O_i.
 int launch_attn_combine(const AttnArgs& a, bool normalized, void* out, int out_bf16, float* lse,
                         cudaStream_t stream);

@@ -6,145 +6,81 @@
 // (128 heads x 512) are dense contractions against entries shared by every head, so
 // both run on tcgen05 with the heads as the M = 128 dimension.  An fp32 accumulator for
 // all 512 output columns would fill the whole 512-column TMEM and leave no room for S,
-// so the work is split over a CTA pair (a thread-block cluster of 2) by halves of c:
-//   - CTA r holds q[:, 256r : 256r+256] and, for each chunk of 64 entries, only the
-//     same 256 columns of the entries, so every byte of q and of the cache is loaded
-//     once per pair;
-//   - it computes the partial logits S_r = q[:, half] C[:, half]^T (K = 256), sends them
-//     to its peer through distributed shared memory, and both form S = S_0 + S_1 (same
-//     operand order, bit-identical in both CTAs) and the same softmax;
-//   - it accumulates its own output half O[:, half] += P C[:, half] (N = 256) in TMEM.
-// Entries are gathered by index with 16-byte cp.async into a double-buffered
-// 128-byte-swizzled tile; the same bytes are the K-major B operand of S and the
-// MN-major B operand of P C.
-//   warps 0-3 loaders  : q half (once) and the entry chunks -> shared memory; at the
-//                        end, output columns 0..127 -> staging; thread 0 issues the
-//                        TMA stores of the staged output half
-//   warps 4-7, 9-12    : softmax, two groups (entries 0-31 and 32-63 of a chunk, one
-//                        thread per row in each): partial S from TMEM -> peer, S, online
-//                        softmax with lazy rescaling (O is rescaled in TMEM only when the
-//                        running max grows by more than 2^8), P (bf16) -> shared memory;
-//                        at the end, output columns 128..255 -> staging
+// so each range ("split") of the entry list is worked by two CTAs, one per half of c:
+//   - both CTAs hold the whole q (128 KB) and, for each chunk of 32 entries, the whole
+//     entry rows, and both compute the full logits S (K = 512) with the same MMAs in
+//     the same order, so their S, softmax and (max, sum) are bit-identical and the two
+//     CTAs never communicate;
+//   - CTA r accumulates only its half of the output, O[:, 256r : 256r+256] += P C[:, half]
+//     (N = 256), in TMEM.
+// The redundant S costs tensor-pipe time, which a decode query has to spare; in exchange
+// no partial logits cross between CTAs, which removes a dependent exchange from every
+// chunk and lets the two CTAs run anywhere on the GPU (no cluster).
+// Entries are gathered by index with 16-byte cp.async (contiguous dense chunks by TMA)
+// into a double-buffered 128-byte-swizzled tile; the same bytes are the K-major B
+// operand of S and, for the CTA's four 64-column panels, the MN-major B operand of P C.
+//   warps 0-3 loaders  : L2 prefetches, q (once) and the entry chunks -> shared memory;
+//                        at the end, output columns 0..127 -> staging; thread 0 issues
+//                        the TMA stores of the staged output half
+//   warps 4-7, 9-12    : softmax, two groups (entries 0-15 and 16-31 of a chunk, one
+//                        thread per row in each): S from TMEM, online softmax with lazy
+//                        rescaling (O is rescaled in TMEM only when the running max grows
+//                        by more than 2^8), P (bf16) -> shared memory; at the end, output
+//                        columns 128..255 -> staging
 //   warp 8    MMA      : issues S(j) and P(j) C as soon as each is ready
-// CTA pairs split the entry list.  A split's partial is its normalised output O_i / l_i,
-// rounded to bf16 (relative error at most 2^-9 per element, the same as the bf16 P fed
-// to the tensor core) and written by TMA, with its running max and sum in base 2 in
-// fp32; the combine kernel of attn.cu merges the splits in fp32.  Every barrier wait is
-// bounded; a timeout sets the workspace status word and the CTA drains and exits.
+// A split's partial is its normalised output O_i / l_i, rounded to bf16 (relative error
+// at most 2^-9 per element, the same as the bf16 P fed to the tensor core) and written
+// by TMA, with its running max and sum in base 2 in fp32; the combine kernel of attn.cu
+// merges the splits in fp32.  Every barrier wait is bounded; a
+// timeout sets the workspace status word and the CTA drains and exits.
 #include "attn.cuh"
-#include "cluster.cuh"
-#include "tc_utils.cuh"
+#include "attn_tc.cuh"
 
 namespace csa {
 namespace {
-using namespace cl;
+using namespace atc;
 
-constexpr int kC = 512;             // entry width handled by this kernel
-constexpr int kHalf = 256;          // columns of c owned by each CTA of the pair
-constexpr int kHeads = 128;         // M
-constexpr int kE = 64;              // entries per chunk (N of S, K of P C)
+constexpr int kE = 32;              // entries per chunk (N of S, K of P C)
+constexpr int kPanels = kC / 64;    // 128-byte column panels of q and of a chunk
 constexpr int kLoaders = 128;
 constexpr int kThreads = 416;       // 4 loader warps, 4 softmax warps, the MMA warp, 4 softmax warps
 constexpr int kMmaWarp = 8;
 constexpr int kSoftmax = 256;       // softmax threads: two per row
-constexpr int kQBytes = kHeads * kHalf * 2;       // 64 KB: 4 panels of 128 rows x 128 B
-constexpr int kCBytes = kE * kHalf * 2;           // 32 KB: 4 panels of 64 rows x 128 B
-constexpr int kPBytes = kHeads * kE * 2;          // 16 KB: 128 rows x 128 B
-constexpr int kRBytes = kHeads * kE * 4;          // 32 KB: peer partial S, fp32
+constexpr int kQBytes = kHeads * kC * 2;          // 128 KB: 8 panels of 128 rows x 128 B
+constexpr int kQPanel = kHeads * 128;             // 16 KB
+constexpr int kCBytes = kE * kC * 2;              // 32 KB: 8 panels of 32 rows x 128 B
+constexpr int kCPanel = kE * 128;                 // 4 KB
+constexpr int kPBytes = kHeads * 128;             // 16 KB: 128 rows x 128 B (the first 64 B used)
 constexpr int kMaxIds = 1024;                     // entry ids of a range staged in smem
 constexpr int kBarBytes = 256;
-constexpr int kXBytes = (2 * 2 + 2) * kHeads * 4;   // row maxima [2 chunks][2 groups][128], sums [2][128]
-constexpr int kSmem = 1024 + kQBytes + 2 * kCBytes + kPBytes + 2 * kRBytes + kBarBytes + kMaxIds * 4 + kXBytes;
-constexpr float kRescaleThreshold = 8.0f;         // log2 units
-static_assert(kQBytes + 2 * kCBytes >= kHeads * kHalf * 4, "output staging (fp32 included) reuses q + chunks");
-
-CSA_DEV void cp_async16(uint32_t dst, const void* src, bool valid)
-{
-    const int n = valid ? 16 : 0;  // 0 bytes read -> 16 zero bytes written
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
-}
-CSA_DEV void cp_async_wait_all() { asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory"); }
-CSA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-CSA_DEV void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }  // all but the newest group
-
-
-constexpr int kBoxCols = 64;             // one output box: 128 rows x 64 bf16 columns (128 B)
-constexpr int kBoxBytes = kHeads * 128;  // 16 KB
-
-// Copy columns [col0, col0 + ncols) of row h of the output half from TMEM (o_taddr: this
-// warp's lane quarter, first O column), scaled by inv = 1 / l, into the staging boxes as
-// bf16: four 128-row x 64-column boxes in the 128-byte swizzled layout of the output
-// tensor map.
-CSA_DEV void stage_o_cols(uint8_t* stage, uint32_t o_taddr, int h, int col0, float inv, int ncols = 128)
-{
-#pragma unroll 1
-    for (int c0 = col0; c0 < col0 + ncols; c0 += 16) {
-        float o[16];
-        tc::tmem_ld16(o_taddr + c0, o);
-        tc::tmem_wait_ld();
-        uint32_t w[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            __nv_bfloat162 pr = __floats2bfloat162_rn(o[2 * i] * inv, o[2 * i + 1] * inv);
-            w[i] = *reinterpret_cast<uint32_t*>(&pr);
-        }
-        uint8_t* row = stage + (c0 / kBoxCols) * kBoxBytes + h * 128;
-        const int q0 = (c0 % kBoxCols) / 8;  // 16-byte chunk of the 128-byte box row
-        *reinterpret_cast<uint4*>(row + ((q0 ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4*>(row + (((q0 + 1) ^ (h & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
-    }
-}
-
-// The same for an fp32 output: eight 128-row x 32-column boxes (128 B rows).
-CSA_DEV void stage_o_cols_f32(uint8_t* stage, uint32_t o_taddr, int h, int col0, float inv, int ncols = 128)
-{
-#pragma unroll 1
-    for (int c0 = col0; c0 < col0 + ncols; c0 += 16) {
-        float o[16];
-        tc::tmem_ld16(o_taddr + c0, o);
-        tc::tmem_wait_ld();
-        uint8_t* row = stage + (c0 / 32) * kBoxBytes + h * 128;
-        const int q0 = (c0 % 32) / 4;  // 16-byte chunk of the 128-byte box row
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<float4*>(row + (((q0 + i) ^ (h & 7)) << 4)) =
-                make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
-    }
-}
-
-// float4 q (0..15) of row h of a 64-float row, XOR-swizzled so that the 32 rows of a
-// warp spread over the banks
-CSA_DEV int rswz(int h, int q) { return h * 16 + (q ^ (h & 15)); }
+constexpr int kXBytes = (2 * 2 + 2) * kHeads * 4; // row maxima [2 chunks][2 groups][128], sums [2][128]
+constexpr int kSmem = 1024 + kQBytes + 2 * kCBytes + kPBytes + kBarBytes + kMaxIds * 4 + kXBytes;
+static_assert(kQBytes >= kHeads * kHalf * 4, "output staging (fp32 included) reuses q");
+static_assert(kSmem <= 227 * 1024, "shared memory of one CTA");
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_q,
-                 const __grid_constant__ CUtensorMap tmap_c, AttnArgs a, uint32_t* status)
+attn_split_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_q,
+                  const __grid_constant__ CUtensorMap tmap_c, AttnArgs a, uint32_t* status)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
     uint8_t* sC0 = sQ + kQBytes;                      // chunk buffer b at sC0 + b * kCBytes
     uint8_t* sP = sC0 + 2 * kCBytes;
-    float4* sR = reinterpret_cast<float4*>(sP + kPBytes);  // [128][16] peer partial S (received)
-    float4* sX = sR + kHeads * 16;                         // [128][16] own partial S (to send)
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPBytes + 2 * kRBytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPBytes);
     uint64_t* Cfull = bars;         // [2] loaders -> MMA            (count 128)
     uint64_t* Cempty = bars + 2;    // [2] MMA commit -> loaders
     uint64_t* Sfull = bars + 4;     // [2] MMA commit -> softmax
-    uint64_t* Sempty = bars + 6;    // [2] softmax -> MMA            (count 128)
-    uint64_t* Rfull = bars + 8;     // peer's bulk copy landed in sR (count 1 + bytes)
-    uint64_t* Xready = bars + 9;    // own partial staged in sX      (count 128)
-    uint64_t* Rfree = bars + 10;    // peer consumed what we sent    (count 8 warps, remote)
-    uint64_t* Xfree = bars + 11;    // our bulk copy has read sX     (count 1)
-    uint64_t* Pfull = bars + 12;    // softmax -> MMA                (count 128)
-    uint64_t* PVdone = bars + 13;   // MMA commit -> softmax
-    uint64_t* idsready = bars + 14; // loaders -> softmax            (count 128)
-    uint64_t* staged = bars + 15;   // output half staged            (count 256: loaders + softmax)
-    uint64_t* Ofinal = bars + 16;   // softmax -> loaders: last P C done (count 128)
-    uint64_t* Qfull = bars + 17;    // q half landed (TMA, count 1 + bytes)
-    uint64_t* MXready = bars + 18;  // both softmax groups' row maxima written (count 256)
-    uint64_t* Lready = bars + 19;   // both softmax groups' row sums written (count 256)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+    uint64_t* Sempty = bars + 6;    // [2] softmax -> MMA            (count 256)
+    uint64_t* Pfull = bars + 8;     // softmax -> MMA                (count 256)
+    uint64_t* PVdone = bars + 9;    // MMA commit -> softmax
+    uint64_t* idsready = bars + 10; // loaders -> softmax            (count 128)
+    uint64_t* staged = bars + 11;   // output half staged            (count 384: loaders + softmax)
+    uint64_t* Ofinal = bars + 12;   // softmax -> loaders: last P C done (count 128)
+    uint64_t* Qfull = bars + 13;    // q landed (TMA, count 1 + bytes)
+    uint64_t* MXready = bars + 14;  // both softmax groups' row maxima written (count 256)
+    uint64_t* Lready = bars + 15;   // both softmax groups' row sums written (count 256)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
     volatile uint32_t* abort_flag = tmem_slot + 1;
     int* s_ids = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);  // [kMaxIds]
     float* s_inv_l = reinterpret_cast<float*>(sP);  // [128] 1 / l per head, after the last P C
@@ -152,9 +88,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
     float* s_lp = s_mx + 4 * kHeads;                          // [2][128] partial row sums
 
     pdl_launch_dependents();
-    const int split = blockIdx.x, g = blockIdx.z;
-    const int half = (int)cluster_rank();  // == blockIdx.y (cluster of 2 along y)
-    const uint32_t peer = (uint32_t)(half ^ 1);
+    const int split = blockIdx.x, half = blockIdx.y, g = blockIdx.z;
     const int64_t b = g / a.nq;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -165,18 +99,15 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
             tc::mbar_init(&Sfull[i], 1);
             tc::mbar_init(&Sempty[i], kSoftmax);
         }
-        tc::mbar_init(Rfull, 1);
-        tc::mbar_init(Xready, kSoftmax);
-        tc::mbar_init(Rfree, kSoftmax / 32);
-        tc::mbar_init(Xfree, 1);
         tc::mbar_init(Pfull, kSoftmax);
         tc::mbar_init(PVdone, 1);
         tc::mbar_init(idsready, kLoaders);
-        tc::mbar_init(staged, kLoaders + kSoftmax);
         tc::mbar_init(MXready, kSoftmax);
         tc::mbar_init(Lready, kSoftmax);
         tc::mbar_init(Ofinal, kHeads);
+        tc::mbar_init(staged, kLoaders + kSoftmax);
         tc::mbar_init(Qfull, 1);
+        tc::tma_prefetch_desc(&tmap_o);
         tc::tma_prefetch_desc(&tmap_q);
         tc::tma_prefetch_desc(&tmap_c);
         *abort_flag = 0;
@@ -187,11 +118,26 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
         tc::tmem_relinquish();
     }
     tc::fence_before_sync();
-    cluster_sync();  // both CTAs' barriers are initialised before any remote arrival
+    __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    // only shared memory and TMEM were touched so far (overlaps the previous kernel)
+    // Only shared memory and TMEM were touched so far (overlaps the previous kernel).  The
+    // L2 prefetches of q and of a dense split's whole range (its compressed entries) go
+    // out now too, so their DRAM latency overlaps the previous kernel's tail.
+    if (threadIdx.x == 32) {
+        const char* qp = static_cast<const char*>(a.q) + (size_t)g * kHeads * kC * 2;
+#pragma unroll
+        for (int i = 0; i < kQBytes / 16384; ++i) tc::prefetch_l2(qp + i * 16384, 16384);
+        if (a.dense) {
+            const int64_t r0 = (int64_t)split * a.per_split;
+            const int64_t r1 = min(r0 + a.per_split, a.N_cap);
+            const char* cp = static_cast<const char*>(a.cache) + ((size_t)b * a.N_cap) * kC * 2;
+            // the two CTAs of the split prefetch alternate 16-entry blocks
+            for (int64_t r = r0 + 16 * half; r < r1; r += 32)
+                tc::prefetch_l2(cp + (size_t)r * kC * 2, (uint32_t)(min((int64_t)16, r1 - r) * kC * 2));
+        }
+    }
     pdl_wait();
     // list positions: [0, ncomp) compressed entries, then [ncomp, count) the sliding-window
     // entries of tokens wlo .. t (when a window is given)
@@ -217,10 +163,10 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
     const int64_t p_end = min(count, p_begin + a.per_split);
     const int nchunks = p_end > p_begin ? (int)((p_end - p_begin + kE - 1) / kE) : 0;
     const size_t prow = ((size_t)g * a.splits + split) * kHeads;  // partial (or output) row of head 0
-    const bool f32_out = a.direct && !a.out_bf16;                  // final fp32 output staged
-    const __nv_bfloat16* cache = static_cast<const __nv_bfloat16*>(a.cache) + b * a.N_cap * kC + half * kHalf;
+    const bool f32_out = a.direct && !a.out_bf16;                  // final output in fp32
+    const __nv_bfloat16* cache = static_cast<const __nv_bfloat16*>(a.cache) + b * a.N_cap * kC;
     const __nv_bfloat16* wcache =
-        a.win ? static_cast<const __nv_bfloat16*>(a.win) + b * (int64_t)a.win_cap * kC + half * kHalf : cache;
+        a.win ? static_cast<const __nv_bfloat16*>(a.win) + b * (int64_t)a.win_cap * kC : cache;
 
     // Code of list position p: e >= 0 compressed entry e, e <= -2 window row -2 - e, -1
     // padding or outside the cache.  Sparse ranges of up to kMaxIds positions are staged in
@@ -242,7 +188,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
         return entry_global(p);
     };
     const bool plain = a.dense && !a.win;  // position p is entry p
-    // first element of this CTA's half of the row a code names (any valid row for -1)
+    // first element of the row a code names (any valid row for -1)
     auto row_of = [&](int64_t e) -> const __nv_bfloat16* {
         return e >= 0 ? cache + e * kC : (e <= -2 ? wcache + (-2 - e) * kC : cache);
     };
@@ -265,11 +211,10 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
     } else if (warp < 4) {
         // ------------------------------------------------------------ loaders
         const int lt = threadIdx.x;
-        if (lt == 0) {  // q half: four 128-row x 64-column TMA boxes (128-byte swizzle)
+        if (lt == 0) {  // q: eight 128-row x 64-column TMA boxes (128-byte swizzle)
             tc::mbar_arrive_expect_tx(Qfull, kQBytes);
 #pragma unroll
-            for (int p = 0; p < kHalf / 64; ++p)
-                tc::tma_load_2d(sQ + p * (kHeads * 128), &tmap_q, Qfull, half * kHalf + p * 64, g * kHeads);
+            for (int p = 0; p < kPanels; ++p) tc::tma_load_2d(sQ + p * kQPanel, &tmap_q, Qfull, p * 64, g * kHeads);
         }
         if (ids_staged)
             for (int64_t i = lt; i < p_end - p_begin; i += kLoaders) s_ids[i] = (int)entry_global(p_begin + i);
@@ -288,41 +233,28 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
             }
             const uint32_t c0 = tc::smem_u32(sC0 + buf * kCBytes);
             const int64_t p0 = p_begin + (int64_t)j * kE;
-            if (plain) {  // dense without a window: position p is entry p
-                if (p0 + kE <= p_end) {
-                    // a full chunk is one contiguous block of cache rows: four 64 x 64 TMA
-                    // boxes, counted in bytes on Cfull (the other loaders just arrive)
-                    if (lt == 0) {
-                        tc::mbar_arrive_expect_tx(&Cfull[buf], kCBytes);
+            if (plain && p0 + kE <= p_end) {
+                // a full dense chunk is one contiguous block of cache rows: eight 32 x 64
+                // TMA boxes, counted in bytes on Cfull (the other loaders just arrive)
+                if (lt == 0) {
+                    tc::mbar_arrive_expect_tx(&Cfull[buf], kCBytes);
 #pragma unroll
-                        for (int p = 0; p < kHalf / 64; ++p)
-                            tc::tma_load_2d(sC0 + buf * kCBytes + p * (kE * 128), &tmap_c, &Cfull[buf],
-                                            half * kHalf + p * 64, (int)(b * a.N_cap + p0));
-                    } else {
-                        tc::mbar_arrive(&Cfull[buf]);
-                    }
-                    continue;
+                    for (int p = 0; p < kPanels; ++p)
+                        tc::tma_load_2d(sC0 + buf * kCBytes + p * kCPanel, &tmap_c, &Cfull[buf], p * 64,
+                                        (int)(b * a.N_cap + p0));
+                } else {
+                    tc::mbar_arrive(&Cfull[buf]);
                 }
-                // the last, partial chunk: rows past the end are zero-filled by cp.async
-#pragma unroll 4
-                for (int i = lt; i < kE * (kHalf / 8); i += kLoaders) {
-                    const int row = i >> 5, cc = i & 31;
-                    const int64_t p = p0 + row;
-                    cp_async16(c0 + (cc >> 3) * (kE * 128) + tc::sw128_offset(row, cc & 7),
-                               cache + (p < p_end ? p : 0) * kC + cc * 8, p < p_end);
-                }
-                cp_async_wait_all();
-                tc::fence_proxy_async_smem();
-                tc::mbar_arrive(&Cfull[buf]);
                 continue;
-            } else {
+            }
+            // gathered (or partial dense) chunk: 32 rows x 64 16-byte pieces, rows past
+            // the range or padding zero-filled
 #pragma unroll 4
-                for (int i = lt; i < kE * (kHalf / 8); i += kLoaders) {
-                    const int row = i >> 5, cc = i & 31;
-                    const int64_t e = entry_of(p0 + row);
-                    cp_async16(c0 + (cc >> 3) * (kE * 128) + tc::sw128_offset(row, cc & 7), row_of(e) + cc * 8,
-                               e != -1);
-                }
+            for (int i = lt; i < kE * (kC / 8); i += kLoaders) {
+                const int row = i >> 6, cc = i & 63;
+                const int64_t p = p0 + row;
+                const int64_t e = plain ? (p < p_end ? p : (int64_t)-1) : entry_of(p);
+                cp_async16(c0 + (cc >> 3) * kCPanel + tc::sw128_offset(row, cc & 7), row_of(e) + cc * 8, e != -1);
             }
             cp_async_commit();
             if (j == 0 && nchunks > 1) continue;  // issue chunk 1 before waiting for chunk 0
@@ -341,15 +273,16 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
         // bounded waits outlast any load in flight by many orders of magnitude.
         if (lt == 0 && !tc::mbar_wait(Qfull, 0, tc::kWaitBudget)) *abort_flag = 1;
         // The output half leaves through TMA: these warps stage columns 0..127 and the
-        // softmax warps 128..255 once the last P C has completed, then thread 0 stores the
-        // eight 128 x 32 boxes.
+        // softmax warps 128..255 once the last P C has completed (q is dead by then, so
+        // its buffer is the staging area), then thread 0 stores the boxes.
         if (!*abort_flag && tc::mbar_wait(Ofinal, 0, tc::kWaitBudget)) {
             tc::fence_after_sync();
             const int h = warp * 32 + lane;
+            const uint32_t ot = tmem + ((uint32_t)(warp * 32) << 16) + kHalf;
             if (f32_out)
-                stage_o_cols_f32(smem, tmem + ((uint32_t)(warp * 32) << 16) + kHalf, h, 0, s_inv_l[h]);
+                stage_o_cols_f32(smem, ot, h, 0, s_inv_l[h], 128);
             else
-                stage_o_cols(smem, tmem + ((uint32_t)(warp * 32) << 16) + kHalf, h, 0, s_inv_l[h]);
+                stage_o_cols(smem, ot, h, 0, s_inv_l[h], 128);
         } else {
             *abort_flag = 1;
         }
@@ -367,7 +300,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
         }
     } else if (warp != kMmaWarp) {
         // ------------------------------------------------------------ softmax
-        // Two groups of four warps: group sg owns entries [32 sg, 32 sg + 32) of every
+        // Two groups of four warps: group sg owns entries [16 sg, 16 sg + 16) of every
         // chunk for all 128 rows (thread = row).  The two threads of a row agree on the
         // row maximum through a double-buffered shared exchange (bounded mbarrier wait),
         // so they keep identical running maxima and rescale decisions; each keeps its own
@@ -379,69 +312,23 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
         constexpr int kEG = kE / 2;  // entries of a chunk per group
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = tc::mbar_wait(idsready, 0, tc::kWaitBudget);
-        int sent = 0;  // chunks whose partial logits thread 128 sent to the peer
         for (int j = 0; j < nchunks && ok; ++j) {
             const int buf = j & 1;
             const uint32_t ph = (j >> 1) & 1;
+            // the validity of this group's 16 entries, read while S is computed
+            const int64_t pg = p_begin + (int64_t)j * kE + sg * kEG;  // list position of entry 0 of the group
+            const unsigned vm =
+                __ballot_sync(0xffffffffu, lane < kEG && (plain ? pg + lane < p_end : entry_of(pg + lane) != -1));
             if (*abort_flag || !tc::mbar_wait(&Sfull[buf], ph, tc::kWaitBudget)) {
                 ok = false;
                 break;
             }
             tc::fence_after_sync();
             float s[kEG];
-#pragma unroll
-            for (int c0 = 0; c0 < kEG; c0 += 16) tc::tmem_ld16(tmem + lane_base + buf * kE + sg * kEG + c0, s + c0);
+            tc::tmem_ld16(tmem + lane_base + buf * kE + sg * kEG, s);
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             tc::mbar_arrive(&Sempty[buf]);
-            // Exchange of the partial logits with the peer: this half's rows are staged in
-            // sX and moved by one bulk copy into the peer's sR, which signals the peer's
-            // Rfull with the byte count; one receive and one send buffer, so each side
-            // waits until the other has consumed the previous chunk.
-            const uint32_t xph = j & 1;
-            if (threadIdx.x == 128) tc::mbar_arrive_expect_tx(Rfull, kRBytes);  // arm this chunk's receive
-            if (j > 0 && !tc::mbar_wait(Xfree, xph ^ 1, tc::kWaitBudget)) {       // previous copy has read sX
-                ok = false;
-                break;
-            }
-#pragma unroll
-            for (int q = 0; q < kEG / 4; ++q)
-                sX[rswz(h, sg * (kEG / 4) + q)] = make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(Xready);
-            if (threadIdx.x == 128) {
-                if (!tc::mbar_wait(Xready, xph, tc::kWaitBudget) || !mbar_wait_cluster(Rfree, xph ^ 1, tc::kWaitBudget)) {
-                    *abort_flag = 1;
-                } else {
-                    bulk_copy_to_peer(peer_addr(tc::smem_u32(sR), peer), tc::smem_u32(sX), kRBytes,
-                                      peer_addr(tc::smem_u32(Rfull), peer));
-                    bulk_wait_read();
-                    ++sent;
-                }
-                tc::mbar_arrive(Xfree);
-            }
-            // the peer's partial logits, then S = S_0 + S_1 in the same order on both CTAs
-            if (!mbar_wait_cluster(Rfull, xph, tc::kWaitBudget)) {
-                ok = false;
-                break;
-            }
-#pragma unroll
-            for (int q = 0; q < kEG / 4; ++q) {
-                const float4 o = sR[rswz(h, sg * (kEG / 4) + q)];
-                if (half == 0) {
-                    s[4 * q] = s[4 * q] + o.x; s[4 * q + 1] = s[4 * q + 1] + o.y;
-                    s[4 * q + 2] = s[4 * q + 2] + o.z; s[4 * q + 3] = s[4 * q + 3] + o.w;
-                } else {
-                    s[4 * q] = o.x + s[4 * q]; s[4 * q + 1] = o.y + s[4 * q + 1];
-                    s[4 * q + 2] = o.z + s[4 * q + 2]; s[4 * q + 3] = o.w + s[4 * q + 3];
-                }
-            }
-            // our receive buffer is free again: one release arrival per warp, after the
-            // warp's reads of sR (a remote arrival costs a cluster-scope release each)
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(peer_addr(tc::smem_u32(Rfree), peer));
-            const int64_t pg = p_begin + (int64_t)j * kE + sg * kEG;  // list position of entry 0 of the group
-            const unsigned vm = __ballot_sync(0xffffffffu, plain ? pg + lane < p_end : entry_of(pg + lane) != -1);
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // 4 chains, not 1
 #pragma unroll
             for (int e = 0; e < kEG; ++e) {
@@ -520,8 +407,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
         }
         if (fin) {
             // The last P C has completed, so every MMA reading q, the chunks and P has too:
-            // q + chunk buffers stage the output half (columns 128..191 by group 0,
-            // 192..255 by group 1), and the P buffer passes 1 / l to the loader warps.
+            // the q buffer stages the output half (columns 128..191 by group 0, 192..255 by
+            // group 1), and the P buffer passes 1 / l to the loader warps.
             const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
             if (sg == 0) {
                 s_inv_l[h] = inv;
@@ -545,11 +432,6 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
         }
         tc::fence_proxy_async_smem();
         tc::mbar_arrive(staged);
-        // The peer's last access to this CTA's shared memory is its arrival on Rfree after
-        // consuming the last chunk sent; once it is in, this CTA may exit (no cluster-wide
-        // barrier at the end).
-        if (threadIdx.x == 128 && sent > 0 && !mbar_wait_cluster(Rfree, (sent - 1) & 1, tc::kWaitBudget))
-            *abort_flag = 1;
     } else {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -564,22 +446,24 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
             auto issue_S = [&](int j) {
                 const uint32_t c0 = tc::smem_u32(sC0 + (j & 1) * kCBytes);
 #pragma unroll
-                for (int p = 0; p < kHalf / 64; ++p) {
+                for (int p = 0; p < kPanels; ++p) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t ad = tc::smem_desc_sw128(q0 + p * (kHeads * 128) + kk * 32, 16, 1024);
-                        const uint64_t bd = tc::smem_desc_sw128(c0 + p * (kE * 128) + kk * 32, 16, 1024);
+                        const uint64_t ad = tc::smem_desc_sw128(q0 + p * kQPanel + kk * 32, 16, 1024);
+                        const uint64_t bd = tc::smem_desc_sw128(c0 + p * kCPanel + kk * 32, 16, 1024);
                         tc::mma_bf16_ss(tmem + (j & 1) * kE, ad, bd, kIdescS, (p | kk) ? 1u : 0u);
                     }
                 }
                 tc::mma_commit(&Sfull[j & 1]);
             };
             auto issue_PV = [&](int j) {
-                const uint32_t c0 = tc::smem_u32(sC0 + (j & 1) * kCBytes);
+                // this CTA's four 64-column panels of the chunk, MN-major (64 columns x
+                // 8 entries per 1024-byte atom, panels kCPanel apart)
+                const uint32_t c0 = tc::smem_u32(sC0 + (j & 1) * kCBytes) + half * (kPanels / 2) * kCPanel;
 #pragma unroll
                 for (int kk = 0; kk < kE / 16; ++kk) {
                     const uint64_t ad = tc::smem_desc_sw128(p0 + kk * 32, 16, 1024);
-                    const uint64_t bd = tc::smem_desc_sw128(c0 + kk * 16 * 128, kE * 128, 1024);
+                    const uint64_t bd = tc::smem_desc_sw128(c0 + kk * 16 * 128, kCPanel, 1024);
                     tc::mma_bf16_ss(tmem + kHalf, ad, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 tc::mma_commit(&Cempty[j & 1]);
@@ -635,39 +519,36 @@ AttnPlan attn_plan_tc(int G, int n_h, int c, int64_t entries)
     (void)n_h;
     (void)c;
     AttnPlan p;
-    const int64_t chunks = (entries + kE - 1) / kE;
-    int64_t splits = kNumSMs / (2 * (int64_t)G);  // one CTA pair per split and query
-    if (splits < 1) splits = 1;
-    if (splits > chunks) splits = chunks;
+    p.head_groups = 1;
+    int64_t max_splits = kNumSMs / (2 * (int64_t)G);  // two CTAs per split and query
+    if (max_splits < 1) max_splits = 1;
+    // Short lists (a decode query's top-k): one 32-entry chunk per split on the
+    // full-width kernel, whose chain has no exchange.  Longer lists: the CTA-pair kernel
+    // of attn_pair.cu over 64-entry chunks, which does half the MMA work per entry.
+    const int64_t c32 = (entries + kE - 1) / kE;
+    if (c32 <= max_splits) {
+        p.kernel = 1;
+        p.per_split = kE;
+        p.splits = (int)(c32 > 0 ? c32 : 1);
+        return p;
+    }
+    constexpr int kPairE = 64;
+    const int64_t chunks = (entries + kPairE - 1) / kPairE;
+    int64_t splits = max_splits < chunks ? max_splits : chunks;
     if (splits < 1) splits = 1;
     const int64_t per_chunks = (chunks + splits - 1) / splits;
-    p.per_split = per_chunks * kE;
-    if (p.per_split < kE) p.per_split = kE;
+    p.kernel = 2;
+    p.per_split = per_chunks * kPairE;
     p.splits = (int)((entries + p.per_split - 1) / p.per_split);
     if (p.splits < 1) p.splits = 1;
-    p.head_groups = 1;
     return p;
 }
 
 int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cudaStream_t stream)
 {
+    if (plan.kernel == 2) return launch_attn_pair(a, plan, status, stream);
     if (!aligned16(a.q) || !aligned16(a.cache) || (a.win && !aligned16(a.win))) return CSA_ERR_ALIGN;
-    cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)plan.splits, 2u, (unsigned)(a.B * a.nq));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = 2;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cudaFuncSetAttribute(attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     // partial outputs [G * splits * 128 rows][512] bf16 in 64 x 128 boxes, or with one
     // split per query the final output [G * 128 rows][512] (bf16 boxes as above, fp32 in
     // 32 x 128 boxes)
@@ -683,10 +564,11 @@ int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cu
     if (!ok_o) return CSA_ERR_CUDA;
     CUtensorMap tmap_q;  // queries [G * 128 rows][512] bf16, 64 x 128 boxes
     if (!make_tmap_bf16_2d(&tmap_q, a.q, (uint64_t)a.B * a.nq * kHeads, kC, kC, 64, kHeads)) return CSA_ERR_CUDA;
-    CUtensorMap tmap_c;  // compressed cache [B * N_cap rows][512] bf16, 64 x 64 boxes (dense chunks)
+    CUtensorMap tmap_c;  // compressed cache [B * N_cap rows][512] bf16, 64 x 32 boxes (dense chunks)
     if (!make_tmap_bf16_2d(&tmap_c, a.cache, (uint64_t)a.B * (uint64_t)(a.N_cap > 0 ? a.N_cap : 1), kC, kC, 64, kE))
         return CSA_ERR_CUDA;
-    cudaLaunchKernelEx(&cfg, attn_pair_kernel, tmap_o, tmap_q, tmap_c, a, status);
+    launch_pdl(attn_split_kernel, dim3((unsigned)plan.splits, 2u, (unsigned)(a.B * a.nq)), dim3(kThreads),
+               (size_t)kSmem, stream, tmap_o, tmap_q, tmap_c, a, status);
     return launch_status();
 }
 

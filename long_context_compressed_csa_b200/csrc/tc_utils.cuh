@@ -97,6 +97,14 @@ CSA_DEV void bulk_store_commit_wait()
     asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
 }
 CSA_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Bulk prefetch of `bytes` (a multiple of 16) at the 16-byte aligned global address p into
+// L2: a hint that returns nothing to the SM.  L2 is the device's point of coherence, so it
+// may be issued before the kernel's dependency wait even for data the previous kernel is
+// still writing: later reads see the written values either way.
+CSA_DEV void prefetch_l2(const void* p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
 // ---------------------------------------------------------------------------- tcgen05
 CSA_DEV void tmem_alloc(uint32_t* dst_smem, uint32_t ncols)
