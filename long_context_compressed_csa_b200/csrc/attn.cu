@@ -399,7 +399,10 @@ int attn_run(AttnArgs a, float scale, void* out, float* lse, void* workspace, si
     if (!aligned16(workspace)) return CSA_ERR_ALIGN;
     a.scale_log2 = (scale > 0.f ? scale : 1.0f / sqrtf((float)a.c)) * kLog2e;
 
-    const bool tc = dtype == CSA_BF16 && attn_tc_supported(a.n_h, a.c);
+    // the tensor-core kernels address cache and window rows with 32-bit TMA coordinates
+    const bool tc = dtype == CSA_BF16 && attn_tc_supported(a.n_h, a.c) &&
+                    (int64_t)a.B * a.N_cap < (int64_t(1) << 31) - 64 &&
+                    (!a.win || (int64_t)a.B * a.win_cap < (int64_t(1) << 31));
     AttnPlan plan = tc ? attn_plan_tc(G, a.n_h, a.c, entries) : attn_plan_cuda_core(G, a.n_h, entries);
     char* ws = static_cast<char*>(workspace);
     uint32_t* status = reinterpret_cast<uint32_t*>(ws);  // sticky device status word

@@ -156,6 +156,15 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
                 tc::prefetch_l2(cp + (size_t)r * kC * 2, (uint32_t)(min((int64_t)16, r1 - r) * kC * 2));
         }
     }
+    if (threadIdx.x == 64) {
+        // the lines of t[g] and of this split's entry ids, likewise (a line the previous
+        // kernel writes afterwards is simply updated in L2)
+        if (a.t) asm volatile("prefetch.global.L2 [%0];" ::"l"(a.t + g) : "memory");
+        if (!a.dense)
+            for (int64_t p = (int64_t)split * a.per_split; p < min((int64_t)(split + 1) * a.per_split, (int64_t)a.k);
+                 p += 32)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(a.idx + (int64_t)g * a.k + p) : "memory");
+    }
     pdl_wait();
     // list positions: [0, ncomp) compressed entries, then [ncomp, count) the sliding-window
     // entries of tokens wlo .. t (when a window is given)

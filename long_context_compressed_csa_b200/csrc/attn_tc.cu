@@ -60,7 +60,8 @@ static_assert(kSmem <= 227 * 1024, "shared memory of one CTA");
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_split_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_q,
-                  const __grid_constant__ CUtensorMap tmap_c, AttnArgs a, uint32_t* status)
+                  const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ CUtensorMap tmap_g,
+                  const __grid_constant__ CUtensorMap tmap_w, AttnArgs a, uint32_t* status)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -110,6 +111,8 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_const
         tc::tma_prefetch_desc(&tmap_o);
         tc::tma_prefetch_desc(&tmap_q);
         tc::tma_prefetch_desc(&tmap_c);
+        tc::tma_prefetch_desc(&tmap_g);
+        if (a.win) tc::tma_prefetch_desc(&tmap_w);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -138,6 +141,15 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_const
                 tc::prefetch_l2(cp + (size_t)r * kC * 2, (uint32_t)(min((int64_t)16, r1 - r) * kC * 2));
         }
     }
+    if (threadIdx.x == 64) {
+        // the lines of t[g] and of this split's entry ids, likewise (a line the previous
+        // kernel writes afterwards is simply updated in L2)
+        if (a.t) asm volatile("prefetch.global.L2 [%0];" ::"l"(a.t + g) : "memory");
+        if (!a.dense)
+            for (int64_t p = (int64_t)split * a.per_split; p < min((int64_t)(split + 1) * a.per_split, (int64_t)a.k);
+                 p += 32)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(a.idx + (int64_t)g * a.k + p) : "memory");
+    }
     pdl_wait();
     // list positions: [0, ncomp) compressed entries, then [ncomp, count) the sliding-window
     // entries of tokens wlo .. t (when a window is given)
@@ -164,10 +176,6 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_const
     const int nchunks = p_end > p_begin ? (int)((p_end - p_begin + kE - 1) / kE) : 0;
     const size_t prow = ((size_t)g * a.splits + split) * kHeads;  // partial (or output) row of head 0
     const bool f32_out = a.direct && !a.out_bf16;                  // final output in fp32
-    const __nv_bfloat16* cache = static_cast<const __nv_bfloat16*>(a.cache) + b * a.N_cap * kC;
-    const __nv_bfloat16* wcache =
-        a.win ? static_cast<const __nv_bfloat16*>(a.win) + b * (int64_t)a.win_cap * kC : cache;
-
     // Code of list position p: e >= 0 compressed entry e, e <= -2 window row -2 - e, -1
     // padding or outside the cache.  Sparse ranges of up to kMaxIds positions are staged in
     // shared memory once by the loaders.
@@ -188,11 +196,6 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_const
         return entry_global(p);
     };
     const bool plain = a.dense && !a.win;  // position p is entry p
-    // first element of the row a code names (any valid row for -1)
-    auto row_of = [&](int64_t e) -> const __nv_bfloat16* {
-        return e >= 0 ? cache + e * kC : (e <= -2 ? wcache + (-2 - e) * kC : cache);
-    };
-
     if (nchunks == 0) {
         if (!a.direct) {
             // empty range: an empty partial (max -inf, sum 0) that the combine skips
@@ -220,10 +223,9 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_const
             for (int64_t i = lt; i < p_end - p_begin; i += kLoaders) s_ids[i] = (int)entry_global(p_begin + i);
         tc::mbar_arrive(idsready);
         asm volatile("bar.sync 2, 128;" ::: "memory");  // loader warps: ids visible to each other
-        // Chunks 0 and 1 are loaded concurrently (both buffers start free); from chunk 2
-        // on, chunk j is issued once P C of chunk j-2 has released its buffer and is
-        // signalled when it has landed.  Chunk j-1 is always signalled before the wait for
-        // a buffer, because that wait depends on the MMA having consumed chunk j-1.
+        // Every chunk arrives by TMA, counted in bytes on Cfull[buf]: chunks 0 and 1 are
+        // issued at once (both buffers start free), chunk j >= 2 once P C of chunk j-2 has
+        // released its buffer.  The loaders never wait for data themselves.
         for (int j = 0; j < nchunks; ++j) {
             const int buf = j & 1;
             if (*abort_flag) break;
@@ -247,30 +249,24 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_const
                 }
                 continue;
             }
-            // gathered (or partial dense) chunk: 32 rows x 64 16-byte pieces, rows past
-            // the range or padding zero-filled
-#pragma unroll 4
-            for (int i = lt; i < kE * (kC / 8); i += kLoaders) {
-                const int row = i >> 6, cc = i & 63;
+            // gathered (or partial dense) chunk: one TMA box of 1 row x 64 columns (128 B)
+            // per row and column panel, two per loader thread; a padding row (or a row
+            // past the range) is loaded from row -1, which TMA fills with zeros
+            {
+                const int row = lt >> 2, pp = (lt & 3) * 2;
                 const int64_t p = p0 + row;
                 const int64_t e = plain ? (p < p_end ? p : (int64_t)-1) : entry_of(p);
-                cp_async16(c0 + (cc >> 3) * kCPanel + tc::sw128_offset(row, cc & 7), row_of(e) + cc * 8, e != -1);
+                const CUtensorMap* m = e <= -2 ? &tmap_w : &tmap_g;
+                const int y = e >= 0 ? (int)(b * a.N_cap + e) : (e <= -2 ? (int)(b * a.win_cap + (-2 - e)) : -1);
+                uint8_t* dst = sC0 + buf * kCBytes + row * 128;
+                tc::mbar_arrive_expect_tx(&Cfull[buf], 2 * 128);
+                tc::tma_load_2d(dst + pp * kCPanel, m, &Cfull[buf], pp * 64, y);
+                tc::tma_load_2d(dst + (pp + 1) * kCPanel, m, &Cfull[buf], (pp + 1) * 64, y);
             }
-            cp_async_commit();
-            if (j == 0 && nchunks > 1) continue;  // issue chunk 1 before waiting for chunk 0
-            if (j == 1) {
-                cp_async_wait_prev();  // chunk 0 has landed; chunk 1 may be in flight
-                tc::fence_proxy_async_smem();
-                tc::mbar_arrive(&Cfull[0]);
-            }
-            cp_async_wait_all();
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(&Cfull[buf]);
         }
-        cp_async_wait_all();
-        // q has landed before the CTA may move on (its barrier is used once).  The TMA
-        // chunks were consumed by the MMA warp on the normal path; after an abort the
-        // bounded waits outlast any load in flight by many orders of magnitude.
+        // q has landed before the CTA may move on (its barrier is used once).  The chunks
+        // were consumed by the MMA warp on the normal path; after an abort the bounded
+        // waits outlast any load in flight by many orders of magnitude.
         if (lt == 0 && !tc::mbar_wait(Qfull, 0, tc::kWaitBudget)) *abort_flag = 1;
         // The output half leaves through TMA: these warps stage columns 0..127 and the
         // softmax warps 128..255 once the last P C has completed (q is dead by then, so
@@ -567,8 +563,14 @@ int launch_attn_tc(const AttnArgs& a, const AttnPlan& plan, uint32_t* status, cu
     CUtensorMap tmap_c;  // compressed cache [B * N_cap rows][512] bf16, 64 x 32 boxes (dense chunks)
     if (!make_tmap_bf16_2d(&tmap_c, a.cache, (uint64_t)a.B * (uint64_t)(a.N_cap > 0 ? a.N_cap : 1), kC, kC, 64, kE))
         return CSA_ERR_CUDA;
+    CUtensorMap tmap_g;  // the same rows, 64 x 1 boxes (gathered entries)
+    if (!make_tmap_bf16_2d(&tmap_g, a.cache, (uint64_t)a.B * (uint64_t)(a.N_cap > 0 ? a.N_cap : 1), kC, kC, 64, 1))
+        return CSA_ERR_CUDA;
+    CUtensorMap tmap_w = tmap_g;  // sliding-window ring [B * win_cap rows][512] bf16, 64 x 1 boxes
+    if (a.win && !make_tmap_bf16_2d(&tmap_w, a.win, (uint64_t)a.B * (uint64_t)a.win_cap, kC, kC, 64, 1))
+        return CSA_ERR_CUDA;
     launch_pdl(attn_split_kernel, dim3((unsigned)plan.splits, 2u, (unsigned)(a.B * a.nq)), dim3(kThreads),
-               (size_t)kSmem, stream, tmap_o, tmap_q, tmap_c, a, status);
+               (size_t)kSmem, stream, tmap_o, tmap_q, tmap_c, tmap_g, tmap_w, a, status);
     return launch_status();
 }
 

@@ -29,6 +29,7 @@ namespace {
 
 constexpr int kTcThreads = 320;  // producer, MMA, two groups of 4 epilogue warps
 constexpr int kTileKeys = 128;
+constexpr int kPrefetchTiles = 4;  // key tiles per CTA prefetched into L2 before the dependency wait
 
 // KB: bytes per key / query element (2: bf16, 1: E4M3)
 template <int NH, int CI, int KB = 2>
@@ -101,8 +102,8 @@ struct SelOut {
 // formula on the dequantised operands because the scales are non-negative.
 template <int NH, int CI, int KB>
 __global__ void __launch_bounds__(kTcThreads, 1)
-scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __restrict__ qI,
-               const float* __restrict__ wI, const float* __restrict__ k_scale,
+scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict__ tmap_base,
+               const __nv_bfloat16* __restrict__ qI, const float* __restrict__ wI, const float* __restrict__ k_scale,
                const int64_t* __restrict__ t, int nq, int64_t N_cap, int m, int k, TopkWs ws, SelOut so)
 {
     using Cfg = ScanCfg<NH, CI, KB>;
@@ -152,8 +153,23 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
     tc::fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
 
-    // everything above only touched this CTA's own shared memory and TMEM, so it may
-    // overlap the previous kernel; global memory is read only after this point
+    // Everything above only touched this CTA's own shared memory and TMEM, so it may
+    // overlap the previous kernel; global memory is read only after the wait below.  The
+    // first key tiles of this CTA (and its query) are prefetched into L2 before it: a
+    // hint that returns nothing, safe before the wait because L2 is the device's point of
+    // coherence (an entry the previous kernel appends is updated in L2), so their DRAM
+    // reads overlap the previous kernel instead of starting the scan.
+    if (threadIdx.x == 32) {
+        const char* kb = static_cast<const char*>(tmap_base) + (size_t)b * N_cap * CI * KB;
+        const int64_t tiles_cap = (N_cap + kTileKeys - 1) / kTileKeys;
+        for (int i = 0; i < kPrefetchTiles; ++i) {
+            const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
+            if (tile >= tiles_cap) break;
+            const int64_t rows = min((int64_t)kTileKeys, N_cap - tile * kTileKeys);
+            tc::prefetch_l2(kb + tile * kTileKeys * CI * KB, (uint32_t)(rows * CI * KB));
+        }
+        tc::prefetch_l2(qI + (int64_t)g * NH * CI, NH * CI * 2);
+    }
     pdl_wait();
     const int64_t vis = visible_of(t, g, m, N_cap);
     const int ntiles = (int)((vis + kTileKeys - 1) / kTileKeys);
@@ -450,7 +466,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __nv_bfloat16* __
 }
 
 template <int NH, int CI, int KB>
-int launch_nh_ci(const CUtensorMap& tmap, const void* qI, const float* wI, const float* k_scale, const int64_t* t,
+int launch_nh_ci(const CUtensorMap& tmap, const void* KI, const void* qI, const float* wI, const float* k_scale, const int64_t* t,
                  int B, int nq, int64_t N_cap, int m, int k, const TopkWs& ws, int32_t* idx_out,
                  float* scores_out, bool* fused, cudaStream_t stream)
 {
@@ -481,7 +497,7 @@ int launch_nh_ci(const CUtensorMap& tmap, const void* qI, const float* wI, const
     so.scores_out = scores_out;
     so.fused = *fused ? 1 : 0;
     dim3 grid((unsigned)ctas, (unsigned)G);
-    launch_pdl(kern, grid, dim3(kTcThreads), Cfg::kSmem, stream, tmap, static_cast<const __nv_bfloat16*>(qI), wI,
+    launch_pdl(kern, grid, dim3(kTcThreads), Cfg::kSmem, stream, tmap, KI, static_cast<const __nv_bfloat16*>(qI), wI,
                k_scale, t, nq, N_cap, m, k, ws, so);
     return launch_status();
 }
@@ -505,7 +521,7 @@ int launch_scan_tc(const void* qI, const float* wI, const void* KI, const int64_
     if (!make_tmap_bf16_2d(&tmap, KI, (uint64_t)B * N_cap, cI, cI, 64, kTileKeys)) return CSA_ERR_CUDA;
 #define CSA_SCAN_CASE(NH_, CI_) \
     if (n_hI == NH_ && cI == CI_)   \
-        return launch_nh_ci<NH_, CI_, 2>(tmap, qI, wI, nullptr, t, B, nq, N_cap, m, k, ws, idx_out, scores_out, fused, stream);
+        return launch_nh_ci<NH_, CI_, 2>(tmap, KI, qI, wI, nullptr, t, B, nq, N_cap, m, k, ws, idx_out, scores_out, fused, stream);
     CSA_SCAN_CASE(16, 64) CSA_SCAN_CASE(16, 128) CSA_SCAN_CASE(16, 256)
     CSA_SCAN_CASE(32, 64) CSA_SCAN_CASE(32, 128) CSA_SCAN_CASE(32, 256)
     CSA_SCAN_CASE(64, 64) CSA_SCAN_CASE(64, 128) CSA_SCAN_CASE(64, 256)
@@ -531,7 +547,7 @@ int launch_scan_tc_e4m3(const void* qI, const float* wI, const void* KI8, const 
     if (!make_tmap_u8_2d(&tmap, KI8, (uint64_t)B * N_cap, cI, cI, 128, kTileKeys)) return CSA_ERR_CUDA;
 #define CSA_SCAN8_CASE(NH_, CI_) \
     if (n_hI == NH_ && cI == CI_)   \
-        return launch_nh_ci<NH_, CI_, 1>(tmap, qI, wI, k_scale, t, B, nq, N_cap, m, k, ws, idx_out, scores_out, fused, stream);
+        return launch_nh_ci<NH_, CI_, 1>(tmap, KI8, qI, wI, k_scale, t, B, nq, N_cap, m, k, ws, idx_out, scores_out, fused, stream);
     CSA_SCAN8_CASE(16, 128) CSA_SCAN8_CASE(16, 256) CSA_SCAN8_CASE(32, 128) CSA_SCAN8_CASE(32, 256)
     CSA_SCAN8_CASE(64, 128) CSA_SCAN8_CASE(64, 256) CSA_SCAN8_CASE(128, 128) CSA_SCAN8_CASE(128, 256)
 #undef CSA_SCAN8_CASE
