@@ -35,9 +35,9 @@ METRIC = "CSA/HCA decode tokens/s at 128K–1M ctx; achieved HBM GB/s vs ~8 TB/s
 WORKLOAD = "hybrid_1m_decode"
 N_PAIRS = 8
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one scan_tc_kernel launch
-# over 262144 keys, from one ncu capture of the current kernel (67.22 MB read, 0.75 MB
+# over 262144 keys, from one ncu capture of the current kernel (67.22 MB read, 0.56 MB
 # written; algorithmic 67.11 MB).  Must be retaken (or set to None) when the kernel changes.
-SCAN_TRAFFIC_BYTES = 67_976_704
+SCAN_TRAFFIC_BYTES = 67_783_424
 IDX_SAMPLE = 8  # steps per CUDA graph; the indexer call of each graph's first step is timed
 
 
@@ -57,9 +57,9 @@ def whole_job_rate(steps_per_rank, world, ms_max):
     return steps_per_rank * world / (ms_max / 1000.0)
 
 
-def workload_config(world):
+def workload_config(world, kI_format="bf16"):
     """The `config` object of both arms' JSON line (the 1M-token hybrid decode)."""
-    return {"workload": WORKLOAD, "n": 1 << 20, "B": 1, "c": 512, "m": 4, "m_prime": 128, "k": 1024,
+    return {"workload": WORKLOAD, "kI_format": kI_format, "n": 1 << 20, "B": 1, "c": 512, "m": 4, "m_prime": 128, "k": 1024,
             "n_h": 128, "n_hI": 64, "cI": 128, "pairs_rotated": N_PAIRS,
             "parallelism": "replicas" if world > 1 else "single",
             "l2": "inputs larger than L2: 8 layer pairs rotated (73 MiB read per step, "
@@ -138,13 +138,14 @@ class ClockSampler:
 class HybridDecode:
     """Eight CSA + HCA layer pairs prefilled at n = 2^20, ready for decode steps."""
 
-    def __init__(self, torch, steps_total, seed=5000, n=1 << 20, device="cuda"):
+    def __init__(self, torch, steps_total, seed=5000, n=1 << 20, device="cuda", kI_format="bf16"):
         import long_context_compressed_csa_b200 as lib
         from long_context_compressed_csa_b200.synth import randn, randint_values
         self.torch, self.lib = torch, lib
         self.n, self.m, self.mp, self.c, self.cI = n, 4, 128, 512, 128
         self.n_h, self.n_hI, self.k = 128, 64, 1024
         self.dev = device
+        self.e4m3 = kI_format == "e4m3"  # indexer keys as E4M3 codes + one fp32 scale per key
         bf16 = torch.bfloat16
         self.tokens = (steps_total + N_PAIRS - 1) // N_PAIRS + 1
         T = self.tokens
@@ -165,6 +166,10 @@ class HybridDecode:
             P["hcache"] = torch.empty((1, self.Nh_cap, c), dtype=bf16, device=device)
             # prefill compress through the library (streams generated in slices)
             self._prefill(P, s)
+            if self.e4m3:  # quantise the prefill keys once; the bf16 cache stays the staging of new keys
+                P["kI8"] = torch.zeros((1, self.N_cap, cI), dtype=torch.uint8, device=device)
+                P["kIs"] = torch.zeros((1, self.N_cap), dtype=torch.float32, device=device)
+                lib.csa_quantize_e4m3(P["kI"][:, :self.N], P["kI8"][:, :self.N], P["kIs"][:, :self.N])
             # decode-time stream rows, one interleaved row per token (the 4 CSA streams, the
             # 4 indexer-key streams, the 2 HCA streams), so that a token's new rows are one
             # contiguous copy: tokens n - hist .. n + T - 1 (CSA), n .. n + T - 1 (HCA)
@@ -227,7 +232,10 @@ class HybridDecode:
         wI = self.wI[qs] if wI is None else wI
         t = self.tpos[j]
         if part in (None, 0):
-            lib.csa_indexer_topk(qI, wI, P["kI"], t, self.m, self.k, self.idx, self.ws_topk)
+            if self.e4m3:
+                lib.csa_indexer_topk_e4m3(qI, wI, P["kI8"], P["kIs"], t, self.m, self.k, self.idx, self.ws_topk)
+            else:
+                lib.csa_indexer_topk(qI, wI, P["kI"], t, self.m, self.k, self.idx, self.ws_topk)
         if part == 0:
             return
         lib.csa_sparse_attn(q, P["cache"], self.idx, o, self.ws_attn)
@@ -241,6 +249,8 @@ class HybridDecode:
             lib.csa_compress(*win, P["cache"], self.m, i, i + 1, tok0=lo)
             winI = [x[:, r0:r0 + 2 * self.m] for x in P["decI"]]
             lib.csa_compress(*winI, P["kI"], self.m, i, i + 1, tok0=lo)
+            if self.e4m3:  # the new key, quantised as it is formed
+                lib.csa_quantize_e4m3(P["kI"][:, i:i + 1], P["kI8"][:, i:i + 1], P["kIs"][:, i:i + 1])
         if (tok + 1) % self.mp == 0:
             i = (tok + 1) // self.mp - 1
             lo = self.mp * i
@@ -254,7 +264,7 @@ class HybridDecode:
         tok = self.n + j
         vis = tok // self.m
         visH = tok // self.mp
-        b = vis * self.cI * 2 + self.k * self.c * 2 + visH * self.c * 2
+        b = vis * (self.cI + 4 if self.e4m3 else self.cI * 2) + self.k * self.c * 2 + visH * self.c * 2
         if (tok + 1) % self.m == 0:
             b += 4 * 2 * self.m * (self.c + self.cI) * 2 + (self.c + self.cI) * 2
         if (tok + 1) % self.mp == 0:
@@ -266,7 +276,7 @@ def kernel_launches_per_step(dec, j):
     tok = dec.n + j
     n = 1 + 2 + 2  # indexer (scan with the select in place), sparse attn (+combine), dense attn (+combine)
     if (tok + 1) % dec.m == 0:
-        n += 2
+        n += 3 if dec.e4m3 else 2
     if (tok + 1) % dec.mp == 0:
         n += 1
     return n
@@ -297,13 +307,14 @@ def _oracle_inputs(workload, seed):
     raise ValueError(workload)
 
 
-def _oracle_step(workload, x, j):
+def _oracle_step(workload, x, j, kI_format="bf16"):
     """One decode step of one sequence through the oracle (the unit of the workload's
     metric divided by its batch)."""
     import oracle
     if workload == "hybrid_1m_decode":
         t = (1 << 20) + j
-        s = oracle.index_scores(x["qI"], x["wI"], x["KI"], oracle.visible(t, 4, x["KI"].shape[0]))
+        score = oracle.index_scores_e4m3 if kI_format == "e4m3" else oracle.index_scores
+        s = score(x["qI"], x["wI"], x["KI"], oracle.visible(t, 4, x["KI"].shape[0]))
         sel = oracle.topk(s, 1024)
         oracle.mqa(x["q"], x["rows"][sel % x["rows"].shape[0]], np.arange(1024, dtype=np.int32))
         oracle.mqa(x["q"], x["hc"], np.arange(oracle.visible(t, 128, x["hc"].shape[0]), dtype=np.int32))
@@ -316,13 +327,13 @@ def _oracle_step(workload, x, j):
         oracle.mqa(x["q"], x["hc"], np.arange(1024, dtype=np.int32))
 
 
-def _oracle_worker(workload, seed, steps, barrier, queue):
+def _oracle_worker(workload, seed, steps, barrier, queue, kI_format="bf16"):
     x = _oracle_inputs(workload, seed)
-    _oracle_step(workload, x, 0)  # warm: loads the oracle library
+    _oracle_step(workload, x, 0, kI_format)  # warm: loads the oracle library
     barrier.wait()
     t0 = time.monotonic()
     for j in range(steps):
-        _oracle_step(workload, x, j + 1)
+        _oracle_step(workload, x, j + 1, kI_format)
     queue.put((t0, time.monotonic(), steps))
 
 
@@ -332,7 +343,7 @@ ORACLE_STEPS = {"hybrid_1m_decode": 1, "csa_decode_8k": 20, "hca_decode_b16_128k
 ORACLE_MAX_WORKERS = 16
 
 
-def cpu_baseline(workload="hybrid_1m_decode", seed=77, steps=None):
+def cpu_baseline(workload="hybrid_1m_decode", seed=77, steps=None, kI_format="bf16"):
     """The oracle timed on the host's cores: one spawned process per core (at most
     ORACLE_MAX_WORKERS), each running whole decode steps of its own sequence after a
     common barrier; value = all steps / the wall time of the concurrent region, in the
@@ -343,7 +354,7 @@ def cpu_baseline(workload="hybrid_1m_decode", seed=77, steps=None):
     steps = steps or ORACLE_STEPS[workload]
     ctx = mp_.get_context("spawn")  # never fork a process that has touched the GPU
     barrier, queue = ctx.Barrier(P), ctx.Queue()
-    procs = [ctx.Process(target=_oracle_worker, args=(workload, seed + 1000 * w, steps, barrier, queue))
+    procs = [ctx.Process(target=_oracle_worker, args=(workload, seed + 1000 * w, steps, barrier, queue, kI_format))
              for w in range(P)]
     for pr in procs:
         pr.start()
@@ -353,8 +364,9 @@ def cpu_baseline(workload="hybrid_1m_decode", seed=77, steps=None):
     wall = max(r[1] for r in res) - min(r[0] for r in res)
     total = sum(r[2] for r in res)
     unit = "layer-pair decode steps/s" if workload == "hybrid_1m_decode" else "decode tokens/s"
-    what = {"hybrid_1m_decode": "one CSA+HCA layer pair at t=2^20 (indexer over 262144 keys, full-sort "
-                                "top-1024, 128-head MQA over 1024 + 8192 entries)",
+    what = {"hybrid_1m_decode": "one CSA+HCA layer pair at t=2^20 (indexer over 262144 %skeys, full-sort "
+                                "top-1024, 128-head MQA over 1024 + 8192 entries)"
+                                % ("E4M3-quantised " if kI_format == "e4m3" else ""),
             "csa_decode_8k": "one CSA layer at t=8192 (indexer over 2048 keys, top-512, 128-head MQA "
                              "over 512 entries)",
             "hca_decode_b16_128k": "one sequence's HCA dense MQA at t=131072 (128 heads over 1024 entries)",
@@ -796,6 +808,9 @@ def main():
                     choices=["hybrid_1m_decode", "csa_decode_8k", "hca_decode_b16_128k",
                              "csa_prefill_decode_b4_256k"],
                     help="the configuration timed (default: the 1M-token hybrid decode)")
+    ap.add_argument("--kI-format", default="bf16", choices=["bf16", "e4m3"],
+                    help="indexer keys of the hybrid decode: bf16 (default) or E4M3 codes with one fp32 "
+                         "scale per key, every appended key quantised as it is formed")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--micro", default=None,
@@ -821,8 +836,8 @@ def main():
             return 0
         import oracle
         oracle.build()
-        base = cpu_baseline(args.workload)
-        cfg = workload_config(args.gpus) if args.workload == WORKLOAD else preset_config(args.workload)
+        base = cpu_baseline(args.workload, kI_format=args.kI_format)
+        cfg = workload_config(args.gpus, args.kI_format) if args.workload == WORKLOAD else preset_config(args.workload)
         line = {"impl": "reference", "metric": METRIC, "value": base["value"], "unit": base["unit"],
                 "n_gpus": args.gpus, "steps": base["cores"] * ORACLE_STEPS[args.workload], "warmup": 0,
                 "ms_per_step": 1000.0 / base["value"], "higher_is_better": True,
@@ -858,7 +873,7 @@ def main():
         return 0
 
     W, K = max(3, args.warmup), args.steps
-    dec = HybridDecode(torch, W + K, seed=5000 + 17 * rank)
+    dec = HybridDecode(torch, W + K, seed=5000 + 17 * rank, kI_format=args.kI_format)
     stream = torch.cuda.current_stream()
 
     # ---- capture the steps in CUDA graphs of N_PAIRS consecutive steps (one token through
@@ -929,7 +944,7 @@ def main():
     # back to back over the 8 layer pairs' keys at the first timed token position ----
     j0 = W // N_PAIRS
     vis = (dec.n + j0) // dec.m
-    idx_bytes = vis * dec.cI * 2
+    idx_bytes = vis * (dec.cI + 4 if dec.e4m3 else dec.cI * 2)
     t_idx = back_to_back_launch_us(
         torch, [lambda p=p: dec.step(p, j0, part=0) for _ in range(8) for p in range(N_PAIRS)], reps=8)
     log("indexer+topk per launch: back to back mean %.2f us, median %.2f us; in the step (event nodes) "
@@ -942,8 +957,9 @@ def main():
     if not args.no_e2e:
         e2e = run_e2e(torch, dec, W, min(K, 512), world)
 
-    roof = roofline_obj("csa_indexer_topk (scan_tc_kernel: indexer scan with the top-k select in place)",
-                        idx_bytes, t_idx, hbm, src, SCAN_TRAFFIC_BYTES, HOW_B2B % (64, 8))
+    roof = roofline_obj("csa_indexer_topk%s (scan_tc_kernel: indexer scan with the top-k select in place)"
+                        % ("_e4m3" if dec.e4m3 else ""), idx_bytes, t_idx, hbm, src,
+                        None if dec.e4m3 else SCAN_TRAFFIC_BYTES, HOW_B2B % (64, 8))
     roof["in_step_event_nodes_us_mean"] = float(idx_ms.mean() * 1e3)
     roof["in_step_event_nodes_samples"] = int(len(idx_ms))
     line = {
@@ -951,7 +967,7 @@ def main():
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms_all / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": workload_config(world),
+        "config": workload_config(world, args.kI_format),
         "roofline": roof,
         "step_roofline": {"achieved": step_gbs, "peak": hbm, "unit": "GB/s", "frac": step_gbs / hbm,
                           "bytes_per_step": bytes_total / K},
@@ -961,7 +977,7 @@ def main():
     if e2e is not None:
         line["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu:
-        base = cpu_baseline()
+        base = cpu_baseline(kI_format=args.kI_format)
         line["cpu_baseline"] = {k: base[k] for k in ("value", "unit", "cores", "host_cores", "kind", "sample")}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -1083,14 +1099,27 @@ def run_e2e(torch, dec, W, K, world):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
     del graphs
+    # the same steps issued eagerly from the host, one C-ABI call at a time (no graphs):
+    # what a host-driven serving loop pays for launch latency
+    Ke = min(K, 256)
+    a2, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a2.record()
+    for s in range(W, W + Ke):
+        one(s)
+    b2.record()
+    torch.cuda.synchronize()
+    ms_e = a2.elapsed_time(b2)
     if world > 1:
         import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        t = torch.tensor([ms, ms_e], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms, ms_e = float(t[0].item()), float(t[1].item())
     return {"value": K * world / (ms / 1000.0), "unit": "layer-pair decode steps/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": K,
-            "how": how}
+            "how": how,
+            "eager": {"value": Ke * world / (ms_e / 1000.0), "steps": Ke,
+                      "how": "the same calls and copies issued eagerly from the host, one C-ABI call at a "
+                             "time on one stream (no CUDA graphs)"}}
 
 
 if __name__ == "__main__":
