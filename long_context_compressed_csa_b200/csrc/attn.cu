@@ -330,6 +330,158 @@ attn_combine(const TP* __restrict__ part_o, const float2* __restrict__ part_ml, 
     }
 }
 
+// Split merge of the tensor-core path (bf16 partials O_i / l_i), one warp per (output row,
+// slice of 32 * VPL columns): a lane keeps the (max, sum) of up to four splits in
+// registers, the first kBatch partial loads of its columns are in flight before the
+// weights are known, and each split's weight reaches the lanes by a shuffle.  The slice
+// width adapts the grid to the number of rows, so that one query (128 rows) and many
+// queries (thousands of rows) both spread over every SM in one wave.
+constexpr int kRowWarps = 4;        // warps per CTA (a lane keeps the weights of up to 4 x 32 splits)
+
+template <int VPL>
+struct RowRaw;
+template <>
+struct RowRaw<4> {
+    using T = uint2;
+    static CSA_DEV T load(const __nv_bfloat16* p) { return __ldcs(reinterpret_cast<const uint2*>(p)); }
+    static CSA_DEV void unpack(T x, float (&v)[4])
+    {
+        v[0] = __uint_as_float(x.x << 16); v[1] = __uint_as_float(x.x & 0xffff0000u);
+        v[2] = __uint_as_float(x.y << 16); v[3] = __uint_as_float(x.y & 0xffff0000u);
+    }
+};
+template <>
+struct RowRaw<8> {
+    using T = uint4;
+    static CSA_DEV T load(const __nv_bfloat16* p) { return __ldcs(reinterpret_cast<const uint4*>(p)); }
+    static CSA_DEV void unpack(T x, float (&v)[8])
+    {
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+
+// kBatch (16 or 32) partial loads are in flight per lane; a split count of at most
+// kBatch is merged in one round trip.
+template <typename TO, int VPL, int kBatch>
+__global__ void __launch_bounds__(32 * kRowWarps)
+attn_combine_rows(const __nv_bfloat16* __restrict__ part_o, const float2* __restrict__ part_ml, int splits, int n_h,
+                  int c, int items, TO* __restrict__ out, float* __restrict__ lse)
+{
+    constexpr int W = 32 * VPL;  // columns of one work item
+    static_assert(kBatch == 16 || kBatch == 32, "a batch never straddles two weight registers");
+    using R = RowRaw<VPL>;
+    pdl_launch_dependents();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int item = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+    if (item >= items) return;
+    const int slices = c / W;
+    const int sl = item % slices, row = item / slices;  // row = g * n_h + h
+    const int g = row / n_h, h = row - g * n_h;
+    const size_t base = (size_t)g * splits * n_h + h;   // partial row of split 0 (splits n_h rows apart)
+    const int col = sl * W + lane * VPL;
+    const __nv_bfloat16* src = part_o + base * c + col;
+    const size_t sstride = (size_t)n_h * c;
+    typename R::T raw[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) raw[u] = u < splits ? R::load(src + (size_t)u * sstride) : typename R::T{};
+    float m[4], l[4], M = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int i = lane + 32 * q;
+        const float2 ml = i < splits ? part_ml[base + (size_t)i * n_h] : make_float2(-INFINITY, 0.f);
+        m[q] = ml.x;
+        l[q] = ml.y;
+        M = fmaxf(M, ml.x);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float w[4], L = 0.f;  // weight of split lane + 32 q: 2^(m_i - M) l_i (0 for an empty split)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        w[q] = m[q] == -INFINITY ? 0.f : exp2f(m[q] - M) * l[q];
+        L += w[q];
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    float acc[VPL];
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) acc[e] = 0.f;
+    for (int i0 = 0; i0 < splits; i0 += kBatch) {
+        if (i0 > 0) {
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                raw[u] = i0 + u < splits ? R::load(src + (size_t)(i0 + u) * sstride) : typename R::T{};
+        }
+        const int q = i0 >> 5;  // the register holding the weights of this batch
+        const float wq = q == 0 ? w[0] : q == 1 ? w[1] : q == 2 ? w[2] : w[3];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const float wi = __shfl_sync(0xffffffffu, wq, (i0 + u) & 31);
+            if (i0 + u < splits && wi != 0.f) {
+                float v[VPL];
+                R::unpack(raw[u], v);
+#pragma unroll
+                for (int e = 0; e < VPL; ++e) acc[e] = fmaf(wi, v[e], acc[e]);
+            }
+        }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    TO* dst = out + (size_t)row * c + col;
+    if constexpr (sizeof(TO) == 4) {
+#pragma unroll
+        for (int e = 0; e < VPL; e += 4)
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(dst) + e) =
+                make_float4(acc[e] * inv, acc[e + 1] * inv, acc[e + 2] * inv, acc[e + 3] * inv);
+    } else {
+        uint32_t pk[VPL / 2];
+#pragma unroll
+        for (int e = 0; e < VPL; e += 2) {
+            __nv_bfloat162 pr = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+            pk[e / 2] = *reinterpret_cast<uint32_t*>(&pr);
+        }
+        if constexpr (VPL == 8)
+            *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        else
+            *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+    }
+    if (sl == 0 && lane == 0 && lse) lse[row] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+}
+
+// 128-column slices (32 loads in flight per lane) below 1024 rows, 256-column slices (16
+// loads in flight) from there on.  One query (128 rows) keeps the (head, column slice)
+// merge instead: its 256-thread CTAs leave room on every SM for the next kernel's CTAs to
+// become resident and start their prologue and prefetches, which the 106-register warps
+// of this merge do not (measured: the 1M sparse-then-dense pair of calls ~2.6 us slower).
+bool combine_rows_wide(const AttnArgs& a) { return a.B * a.nq * a.n_h >= 1024; }
+bool combine_rows_fits(const AttnArgs& a)
+{
+    return a.B * a.nq >= 4 && a.splits <= (combine_rows_wide(a) ? 16 : 32);
+}
+
+template <typename TO>
+int launch_combine_rows(const AttnArgs& a, TO* out, float* lse, cudaStream_t stream)
+{
+    const int rows = a.B * a.nq * a.n_h;
+    const bool wide = combine_rows_wide(a);
+    const int vpl = wide ? 8 : 4;
+    const int items = rows * (a.c / (32 * vpl));
+    const dim3 grid((unsigned)((items + kRowWarps - 1) / kRowWarps));
+    const __nv_bfloat16* po = static_cast<const __nv_bfloat16*>(a.part_o);
+    if (wide)
+        launch_pdl(attn_combine_rows<TO, 8, 16>, grid, dim3(32 * kRowWarps), 0, stream, po, a.part_ml, a.splits,
+                   a.n_h, a.c, items, out, lse);
+    else
+        launch_pdl(attn_combine_rows<TO, 4, 32>, grid, dim3(32 * kRowWarps), 0, stream, po, a.part_ml, a.splits,
+                   a.n_h, a.c, items, out, lse);
+    return launch_status();
+}
+
 int launch_cuda_core(AttnArgs a, const AttnPlan& plan, int dtype, cudaStream_t stream)
 {
     a.splits = plan.splits;
@@ -358,6 +510,13 @@ int launch_attn_combine(const AttnArgs& a, bool normalized, void* out, int out_b
     dim3 grid((unsigned)a.n_h, (unsigned)G, (unsigned)((a.c + kCombineCols - 1) / kCombineCols));
     dim3 block(kCombineThreads);
     const float2* ml = a.part_ml;
+    // bf16 partials of the tensor-core path, widths of whole 256-column slices, and few
+    // enough splits for one round of loads: the warp-per-row merge; otherwise the
+    // (head, column slice) CTAs below, which spread many splits over their threads
+    if (normalized && combine_rows_fits(a) && a.c % 256 == 0 && aligned16(out) && aligned16(a.part_o)) {
+        if (out_bf16) return launch_combine_rows(a, static_cast<__nv_bfloat16*>(out), lse, stream);
+        return launch_combine_rows(a, static_cast<float*>(out), lse, stream);
+    }
     if (normalized) {
         const __nv_bfloat16* po = static_cast<const __nv_bfloat16*>(a.part_o);
         if (out_bf16)
