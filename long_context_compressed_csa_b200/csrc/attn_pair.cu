@@ -57,14 +57,18 @@ constexpr int kCBytes = kE * kHalf * 2;           // 32 KB: 4 panels of 64 rows 
 constexpr int kPBytes = kHeads * kE * 2;          // 16 KB: 128 rows x 128 B
 constexpr int kRBytes = kHeads * kE * 4;          // 32 KB: peer partial S, fp32
 constexpr int kMaxIds = 1024;                     // entry ids of a range staged in smem
-constexpr int kBarBytes = 256;
+constexpr int kBarBytes = 512;
 constexpr int kXBytes = (2 * 2 + 2) * kHeads * 4;   // row maxima [2 chunks][2 groups][128], sums [2][128]
 constexpr int kSmem = 1024 + kQBytes + 2 * kCBytes + kPBytes + 2 * kRBytes + kBarBytes + kMaxIds * 4 + kXBytes;
 static_assert(kQBytes + 2 * kCBytes >= kHeads * kHalf * 4, "output staging (fp32 included) reuses q + chunks");
 
 // float4 q (0..15) of row h of a 64-float row, XOR-swizzled so that the 32 rows of a
 // warp spread over the banks
-CSA_DEV int rswz(int h, int q) { return h * 16 + (q ^ (h & 15)); }
+// Exchange blocks: softmax warp w (group sg, lane quarter qw; w = 4 sg + qw) owns one
+// 4 KB block of sX / sR, its 32 rows x its group's 32 entries as 8 float4 per row, the
+// float4 index XOR-swizzled by the row so that a warp's accesses spread over the banks.
+CSA_DEV int xblk(int w, int lane, int q) { return (w * 32 + lane) * 8 + (q ^ (lane & 7)); }
+constexpr int kXBlock = 32 * 32 * 4;  // 4 KB
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_q,
@@ -75,26 +79,24 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
     uint8_t* sQ = smem;
     uint8_t* sC0 = sQ + kQBytes;                      // chunk buffer b at sC0 + b * kCBytes
     uint8_t* sP = sC0 + 2 * kCBytes;
-    float4* sR = reinterpret_cast<float4*>(sP + kPBytes);  // [128][16] peer partial S (received)
-    float4* sX = sR + kHeads * 16;                         // [128][16] own partial S (to send)
+    float4* sR = reinterpret_cast<float4*>(sP + kPBytes);  // 8 blocks of 4 KB: peer partial S (received)
+    float4* sX = sR + kHeads * 16;                         // 8 blocks of 4 KB: own partial S (to send)
     uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPBytes + 2 * kRBytes);
     uint64_t* Cfull = bars;         // [2] loaders -> MMA            (count 128)
     uint64_t* Cempty = bars + 2;    // [2] MMA commit -> loaders
     uint64_t* Sfull = bars + 4;     // [2] MMA commit -> softmax
     uint64_t* Sempty = bars + 6;    // [2] softmax -> MMA            (count 128)
-    uint64_t* Rfull = bars + 8;     // peer's bulk copy landed in sR (count 1 + bytes)
-    uint64_t* Xready = bars + 9;    // own partial staged in sX      (count 128)
-    uint64_t* Rfree = bars + 10;    // peer consumed what we sent    (count 8 warps, remote)
-    uint64_t* Xfree = bars + 11;    // our bulk copy has read sX     (count 1)
-    uint64_t* Pfull = bars + 12;    // softmax -> MMA                (count 128)
-    uint64_t* PVdone = bars + 13;   // MMA commit -> softmax
-    uint64_t* idsready = bars + 14; // loaders -> softmax            (count 128)
-    uint64_t* staged = bars + 15;   // output half staged            (count 256: loaders + softmax)
-    uint64_t* Ofinal = bars + 16;   // softmax -> loaders: last P C done (count 128)
-    uint64_t* Qfull = bars + 17;    // q half landed (TMA, count 1 + bytes)
-    uint64_t* MXready = bars + 18;  // both softmax groups' row maxima written (count 256)
-    uint64_t* Lready = bars + 19;   // both softmax groups' row sums written (count 256)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+    uint64_t* Rfull = bars + 8;     // [8] the peer's block w landed in sR (count 1 + 4 KB)
+    uint64_t* Rfree = bars + 16;    // [8] the peer read our block w (count 1, remote arrival)
+    uint64_t* Pfull = bars + 24;    // softmax -> MMA                (count 128)
+    uint64_t* PVdone = bars + 25;   // MMA commit -> softmax
+    uint64_t* idsready = bars + 26; // loaders -> softmax            (count 128)
+    uint64_t* staged = bars + 27;   // output half staged            (count 256: loaders + softmax)
+    uint64_t* Ofinal = bars + 28;   // softmax -> loaders: last P C done (count 128)
+    uint64_t* Qfull = bars + 29;    // q half landed (TMA, count 1 + bytes)
+    uint64_t* MXready = bars + 30;  // both softmax groups' row maxima written (count 256)
+    uint64_t* Lready = bars + 31;   // both softmax groups' row sums written (count 256)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 32);
     volatile uint32_t* abort_flag = tmem_slot + 1;
     int* s_ids = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);  // [kMaxIds]
     float* s_inv_l = reinterpret_cast<float*>(sP);  // [128] 1 / l per head, after the last P C
@@ -115,10 +117,10 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
             tc::mbar_init(&Sfull[i], 1);
             tc::mbar_init(&Sempty[i], kSoftmax);
         }
-        tc::mbar_init(Rfull, 1);
-        tc::mbar_init(Xready, kSoftmax);
-        tc::mbar_init(Rfree, kSoftmax / 32);
-        tc::mbar_init(Xfree, 1);
+        for (int w = 0; w < 8; ++w) {
+            tc::mbar_init(&Rfull[w], 1);
+            tc::mbar_init(&Rfree[w], 1);
+        }
         tc::mbar_init(Pfull, kSoftmax);
         tc::mbar_init(PVdone, 1);
         tc::mbar_init(idsready, kLoaders);
@@ -350,9 +352,10 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
         const int h = quarter * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         constexpr int kEG = kE / 2;  // entries of a chunk per group
+        const int wb = sg * 4 + quarter;  // this warp's exchange block
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = tc::mbar_wait(idsready, 0, tc::kWaitBudget);
-        int sent = 0;  // chunks whose partial logits thread 128 sent to the peer
+        int sent = 0;  // chunks whose partial logits this warp's lane 0 sent to the peer
         for (int j = 0; j < nchunks && ok; ++j) {
             const int buf = j & 1;
             const uint32_t ph = (j >> 1) & 1;
@@ -367,40 +370,37 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             tc::mbar_arrive(&Sempty[buf]);
-            // Exchange of the partial logits with the peer: this half's rows are staged in
-            // sX and moved by one bulk copy into the peer's sR, which signals the peer's
-            // Rfull with the byte count; one receive and one send buffer, so each side
-            // waits until the other has consumed the previous chunk.
+            // Exchange of the partial logits with the peer, per warp: this warp's 32 rows x
+            // 32 entries are staged in its block of sX and moved by one 4 KB bulk copy into
+            // the same block of the peer's sR, counted in bytes on the peer's Rfull[w]; the
+            // peer's warp w does the same towards this CTA.  One receive and one send block
+            // per warp, so each warp waits until the peer's warp has read the previous one.
             const uint32_t xph = j & 1;
-            if (threadIdx.x == 128) tc::mbar_arrive_expect_tx(Rfull, kRBytes);  // arm this chunk's receive
-            if (j > 0 && !tc::mbar_wait(Xfree, xph ^ 1, tc::kWaitBudget)) {       // previous copy has read sX
-                ok = false;
-                break;
-            }
+            if (lane == 0) tc::mbar_arrive_expect_tx(&Rfull[wb], kXBlock);  // arm this chunk's receive
 #pragma unroll
             for (int q = 0; q < kEG / 4; ++q)
-                sX[rswz(h, sg * (kEG / 4) + q)] = make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
+                sX[xblk(wb, lane, q)] = make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
             tc::fence_proxy_async_smem();
-            tc::mbar_arrive(Xready);
-            if (threadIdx.x == 128) {
-                if (!tc::mbar_wait(Xready, xph, tc::kWaitBudget) || !mbar_wait_cluster(Rfree, xph ^ 1, tc::kWaitBudget)) {
+            __syncwarp();
+            if (lane == 0) {
+                if (!mbar_wait_cluster(&Rfree[wb], xph ^ 1, tc::kWaitBudget)) {
                     *abort_flag = 1;
                 } else {
-                    bulk_copy_to_peer(peer_addr(tc::smem_u32(sR), peer), tc::smem_u32(sX), kRBytes,
-                                      peer_addr(tc::smem_u32(Rfull), peer));
-                    bulk_wait_read();
+                    bulk_copy_to_peer(peer_addr(tc::smem_u32(sR + wb * 256), peer), tc::smem_u32(sX + wb * 256),
+                                      kXBlock, peer_addr(tc::smem_u32(&Rfull[wb]), peer));
+                    bulk_wait_read();  // the block may be rewritten for the next chunk
                     ++sent;
                 }
-                tc::mbar_arrive(Xfree);
             }
+            __syncwarp();
             // the peer's partial logits, then S = S_0 + S_1 in the same order on both CTAs
-            if (!mbar_wait_cluster(Rfull, xph, tc::kWaitBudget)) {
+            if (*abort_flag || !mbar_wait_cluster(&Rfull[wb], xph, tc::kWaitBudget)) {
                 ok = false;
                 break;
             }
 #pragma unroll
             for (int q = 0; q < kEG / 4; ++q) {
-                const float4 o = sR[rswz(h, sg * (kEG / 4) + q)];
+                const float4 o = sR[xblk(wb, lane, q)];
                 if (half == 0) {
                     s[4 * q] = s[4 * q] + o.x; s[4 * q + 1] = s[4 * q + 1] + o.y;
                     s[4 * q + 2] = s[4 * q + 2] + o.z; s[4 * q + 3] = s[4 * q + 3] + o.w;
@@ -409,10 +409,10 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
                     s[4 * q + 2] = o.z + s[4 * q + 2]; s[4 * q + 3] = o.w + s[4 * q + 3];
                 }
             }
-            // our receive buffer is free again: one release arrival per warp, after the
-            // warp's reads of sR (a remote arrival costs a cluster-scope release each)
+            // our receive block is free again: one release arrival on the peer warp's
+            // Rfree[w], after this warp's reads of it
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(peer_addr(tc::smem_u32(Rfree), peer));
+            if (lane == 0) mbar_arrive_remote(peer_addr(tc::smem_u32(&Rfree[wb]), peer));
             const int64_t pg = p_begin + (int64_t)j * kE + sg * kEG;  // list position of entry 0 of the group
             const unsigned vm = __ballot_sync(0xffffffffu, plain ? pg + lane < p_end : entry_of(pg + lane) != -1);
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // 4 chains, not 1
@@ -518,10 +518,10 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_consta
         }
         tc::fence_proxy_async_smem();
         tc::mbar_arrive(staged);
-        // The peer's last access to this CTA's shared memory is its arrival on Rfree after
-        // consuming the last chunk sent; once it is in, this CTA may exit (no cluster-wide
-        // barrier at the end).
-        if (threadIdx.x == 128 && sent > 0 && !mbar_wait_cluster(Rfree, (sent - 1) & 1, tc::kWaitBudget))
+        // The peer's last access to this CTA's shared memory is its warps' arrivals on
+        // Rfree after consuming the last block each was sent; once they are in, this CTA
+        // may exit (no cluster-wide barrier at the end).
+        if (lane == 0 && sent > 0 && !mbar_wait_cluster(&Rfree[wb], (sent - 1) & 1, tc::kWaitBudget))
             *abort_flag = 1;
     } else {
         // ------------------------------------------------------------ MMA issuer
