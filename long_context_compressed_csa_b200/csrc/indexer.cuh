@@ -5,7 +5,11 @@
 namespace csa {
 
 constexpr int kBins = 4096;  // 12-bit radix digits
-constexpr int kCtrs = 8;     // per query: [0] emitted, [1] candidates, [2] ticket, [3] arrivals
+// per query: [0] emitted, [1] candidates, [2] ticket, [3] arrivals at the first grid
+// meeting of the in-place select, [4] at its second, [5] nonzero when the workspace needs a
+// full reset (a timed-out wait or an aborted scan)
+constexpr int kCtrs = 8;
+constexpr int kCtrDirty = 5;
 
 // Slot of a 12-bit digit in a 4096-bin histogram.  Bins are stored transposed
 // ([16][256]) so that the threshold search, in which thread t reads the 16 consecutive

@@ -53,7 +53,14 @@ struct ScanCfg {
     static constexpr int kTmemCols = (2 * NH) < 32 ? 32 : (2 * NH);
     static_assert(kStages >= 2, "not enough shared memory for a 2-stage ring");
     static_assert((kTmemCols & (kTmemCols - 1)) == 0, "TMEM columns must be a power of 2");
-    static_assert(kStages * kAStage >= 2 * sel::kListCap * 8, "select lists reuse the ring");
+    // the in-place select reuses the ring: the fallback's two lists, the per-bin counts
+    // merged before this CTA's, the merged histogram and the threshold bin's candidates
+    static constexpr int kOldOff = 2 * sel::kListCap * 8;
+    static constexpr int kGhOff = kOldOff + kBins * 4;
+    static constexpr int kCandOff = kGhOff + kBins * 4;
+    static constexpr int kFastCapRaw = (kStages * kAStage - kCandOff) / 8;
+    static constexpr int kFastCap = kFastCapRaw > 4096 ? 4096 : kFastCapRaw;
+    static_assert(kFastCap >= 2048 && kFastCap % sel::kSelThreads == 0, "candidate list of the select's fast path");
 };
 
 CSA_DEV void red_release_add(uint32_t* p, uint32_t v)
@@ -124,6 +131,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict_
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qready + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
+    __shared__ sel::Shared ss;  // scalars of the in-place select
     pdl_launch_dependents();
     const int g = blockIdx.y;
     const int64_t b = g / nq;
@@ -181,6 +189,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict_
     } else if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
+            const uint64_t stream_policy = tc::l2_evict_first_policy();  // every key is read once
             int it = 0;
             for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
                 const int s = it % S;
@@ -194,8 +203,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict_
                 const int row0 = (int)(b * N_cap) + tile * kTileKeys;
 #pragma unroll
                 for (int p = 0; p < Cfg::kPanels; ++p)
-                    tc::tma_load_2d(sA + s * Cfg::kAStage + p * (kTileKeys * 128), &tmap, &full[s],
-                                    Cfg::kPanelElems * p, row0);
+                    tc::tma_load_2d_hint(sA + s * Cfg::kAStage + p * (kTileKeys * 128), &tmap, &full[s],
+                                         Cfg::kPanelElems * p, row0, stream_policy);
             }
             // drain: every issued load has landed before the CTA may exit
             for (int j = it - S < 0 ? 0 : it - S; j < it; ++j)
@@ -384,9 +393,30 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict_
     tc::fence_before_sync();
     __syncthreads();
     if (active && *abort_flag && threadIdx.x == 0) atomicExch(ws.status, 1u);
-    if (need_hist)
-        for (int i = threadIdx.x; i < kBins; i += kTcThreads)
-            if (sh[i]) atomicAdd(&ws.hist0[(size_t)g * kBins + i], sh[i]);
+    if (need_hist) {
+        uint32_t* gh = ws.hist0 + (size_t)g * kBins;
+        if (so.fused) {
+            // the in-place select places its keys from the counts merged before its own
+            // (the atomics' return values), kept per bin in the idle ring; every atomic
+            // is issued before the first return value is needed
+            uint32_t* s_old = reinterpret_cast<uint32_t*>(sA + Cfg::kOldOff);
+            constexpr int kM = (kBins + kTcThreads - 1) / kTcThreads;
+            uint32_t c[kM], o[kM];
+#pragma unroll
+            for (int u = 0; u < kM; ++u) {
+                const int i = threadIdx.x + u * kTcThreads;
+                c[u] = i < kBins ? sh[i] : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kM; ++u) o[u] = c[u] ? atomicAdd(&gh[threadIdx.x + u * kTcThreads], c[u]) : 0u;
+#pragma unroll
+            for (int u = 0; u < kM; ++u)
+                if (c[u]) s_old[threadIdx.x + u * kTcThreads] = o[u];
+        } else {
+            for (int i = threadIdx.x; i < kBins; i += kTcThreads)
+                if (sh[i]) atomicAdd(&gh[i], sh[i]);
+        }
+    }
     if (warp == 1) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem_base, Cfg::kTmemCols);
@@ -398,61 +428,166 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict_
     // ---------------------------------------------------------------- in-place top-k
     // The epilogue warps (256 threads, named barrier 1) select from this CTA's scores.
     // Every CTA of the query is resident (the launch keeps the grid within one wave), so
-    // they can meet at a counter once all digit-0 histograms are merged; the wait is
-    // bounded.  Then each CTA classifies its own keys against the threshold bin, and the
-    // last one (atomic ticket) resolves the candidates and resets the workspace.
+    // they can meet at counters; every wait is bounded.
     using Bar = sel::NamedBar<1>;
-    __shared__ sel::Shared ss;
+    constexpr int T = sel::kSelThreads;
     const int tid = threadIdx.x - 64;
     const sel::Query q = sel::query_view(ws, g, k, so.idx_out, so.scores_out);
     if (vis <= k) {  // padding after the visible entries (written by the epilogue above)
-        for (int64_t p = vis + (int64_t)blockIdx.x * sel::kSelThreads + tid; p < k;
-             p += (int64_t)gridDim.x * sel::kSelThreads) {
+        for (int64_t p = vis + (int64_t)blockIdx.x * T + tid; p < k; p += (int64_t)gridDim.x * T) {
             q.idx_out[p] = -1;
             if (q.sc_out) q.sc_out[p] = -INFINITY;
         }
         return;
     }
+    const float* scores = ws.scores + (int64_t)g * ws.ld;
+    const int my_tiles = active ? (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+    const int npos = my_tiles * kTileKeys;  // CTA-local positions: tile ordinal * 128 + row
+    const uint32_t vis32 = (uint32_t)vis;   // < 2^31 (checked by the host)
+    // position j = tile ordinal * 128 + row holds key (blockIdx.x + ordinal * gridDim.x) * 128 + row;
+    // kSelThreads = 2 tiles, so from one u to the next the key advances by 2 * gridDim.x tiles
+    static_assert(T == 2 * kTileKeys, "two tiles per classification step");
+    const uint32_t key_step = 2u * gridDim.x * kTileKeys;
+    auto load_keys = [&](int base, uint32_t (&key)[sel::kPer], uint32_t (&eidx)[sel::kPer], bool (&valid)[sel::kPer]) {
+        const int j0 = base + tid;
+        const int ord0 = j0 / kTileKeys;
+        const uint32_t s0 = (blockIdx.x + (uint32_t)ord0 * gridDim.x) * kTileKeys + (uint32_t)(j0 % kTileKeys);
+#pragma unroll
+        for (int u = 0; u < sel::kPer; ++u) {
+            const int j = j0 + u * T;
+            const uint32_t s = s0 + (uint32_t)u * key_step;
+            valid[u] = j < npos && s < vis32;
+            eidx[u] = s;
+            key[u] = valid[u] ? order_key(ord0 + 2 * u < Cfg::kCacheTiles ? s_sc[j] : __ldcg(&scores[s])) : 0u;
+        }
+    };
+
+    // first meeting: every CTA's histogram is merged
+    long long budget = tc::kWaitBudget;  // tid 0 runs both meetings
     if (tid == 0) {
-        // the wait budget of this meeting: the workspace's override when one is set (a
-        // test hook that makes the wait run out), else the ~1 s of every other wait
         const long long ov = *reinterpret_cast<const volatile long long*>(ws.status + 2);
+        if (ov > 0) budget = ov;  // a test hook that makes the waits run out
         red_release_add(&q.ctr[3], 1u);
-        const bool ok = wait_count_geq(&q.ctr[3], gridDim.x, ov > 0 ? ov : tc::kWaitBudget);
+        const bool ok = wait_count_geq(&q.ctr[3], gridDim.x, budget);
         if (!ok) atomicExch(ws.status, 1u);
+        // a timed-out meeting or an aborted scan leaves the query's workspace for the
+        // last CTA to clear in full
+        if (!ok || *abort_flag) q.ctr[kCtrDirty] = 1u;
         ss.ok = ok;
     }
     Bar::sync();
     const bool ok = ss.ok != 0;
-    uint2* s_listA = reinterpret_cast<uint2*>(sA);  // the ring is idle now
-    uint2* s_listB = s_listA + sel::kListCap;
+    uint32_t* s_old = reinterpret_cast<uint32_t*>(sA + Cfg::kOldOff);  // the ring is idle now
+    uint32_t* s_gh = reinterpret_cast<uint32_t*>(sA + Cfg::kGhOff);
+    uint2* s_cand = reinterpret_cast<uint2*>(sA + Cfg::kCandOff);
+    bool fast = false;
     if (ok) {
-        sel::load_hist(sh, q.hist0, tid);
+        sel::load_hist(s_gh, q.hist0, tid);
         Bar::sync();
-        sel::find_threshold_bin<kBins, Bar>(sh, (uint32_t)k, &ss, tid);
-        const uint32_t b0 = ss.bin;
-        const float* scores = ws.scores + (int64_t)g * ws.ld;
-        const int my_tiles = active ? (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
-        const int npos = my_tiles * kTileKeys;  // CTA-local positions: tile ordinal * 128 + row
-        const uint32_t vis32 = (uint32_t)vis;   // < 2^31 (checked by the host)
-        // position j = tile ordinal * 128 + row holds key (blockIdx.x + ordinal * gridDim.x) * 128 + row;
-        // kSelThreads = 2 tiles, so from one u to the next the key advances by 2 * gridDim.x tiles
-        static_assert(sel::kSelThreads == 2 * kTileKeys, "two tiles per classification step");
-        const uint32_t key_step = 2u * gridDim.x * kTileKeys;
+        sel::threshold_and_suffix<Bar>(s_gh, (uint32_t)k, &ss, tid);
+        fast = ss.cnt <= (uint32_t)Cfg::kFastCap;  // the same decision in every CTA
+    }
+
+    if (fast) {
+        // Every key's output slot follows from counts alone.  The merged histogram, turned
+        // into per-bin counts of the bins above (s_gh), orders the bins; inside a bin the
+        // CTAs are ordered by their merge atomics (s_old: the bin's count merged before
+        // this CTA's) and a CTA's own keys by a shared-memory countdown on its local
+        // histogram.  Keys above the threshold bin b0 are emitted at once; b0's keys go to
+        // the global candidate list at the same kind of slot.  After a second meeting
+        // every CTA loads that list (at most kFastCap entries) and ranks a 1/gridDim.x
+        // share of it against the whole list: the candidate of rank r (larger score
+        // first, ties to the smaller index) is selected when r < k - above and goes to
+        // slot above + r.  The last CTA by an atomic ticket (taken after the second
+        // meeting, read at the end) clears the counters; each CTA clears its share of the
+        // merged histogram.
+        const uint32_t b0 = ss.bin, above = ss.above, nb0 = ss.cnt;
         for (int base = 0; base < npos; base += sel::kRound) {
-            const int j0 = base + tid;
-            const int ord0 = j0 / kTileKeys;
-            const uint32_t s0 = (blockIdx.x + (uint32_t)ord0 * gridDim.x) * kTileKeys + (uint32_t)(j0 % kTileKeys);
             uint32_t key[sel::kPer], eidx[sel::kPer];
             bool valid[sel::kPer];
+            load_keys(base, key, eidx, valid);
 #pragma unroll
             for (int u = 0; u < sel::kPer; ++u) {
-                const int j = j0 + u * sel::kSelThreads;
-                const uint32_t s = s0 + (uint32_t)u * key_step;
-                valid[u] = j < npos && s < vis32;
-                eidx[u] = s;
-                key[u] = valid[u] ? order_key(ord0 + 2 * u < Cfg::kCacheTiles ? s_sc[j] : __ldcg(&scores[s])) : 0u;
+                const uint32_t d0 = key[u] >> 20;
+                if (!valid[u] || d0 < b0) continue;
+                const uint32_t sl = hist_slot(d0);
+                const uint32_t r = atomicSub(&sh[sl], 1u) - 1u;
+                const uint2 kv = make_uint2(key[u], eidx[u]);
+                if (d0 > b0) {
+                    sel::emit(q, s_gh[sl] + s_old[sl] + r, kv);
+                } else {
+                    const uint32_t c = s_old[sl] + r;
+                    if (c < nb0) q.cand[c] = kv;  // always, unless the scan was aborted
+                }
             }
+        }
+        Bar::sync();  // the arrival below releases every thread's candidate stores
+        uint32_t ticket = 0;
+        if (tid == 0) {
+            red_release_add(&q.ctr[4], 1u);
+            const bool ok2 = wait_count_geq(&q.ctr[4], gridDim.x, budget);
+            if (!ok2) {
+                atomicExch(ws.status, 1u);
+                q.ctr[kCtrDirty] = 1u;
+            }
+            ss.ok = ok2;
+            ticket = atom_acq_rel_add(&q.ctr[2], 1u);  // read at the end: the round trip overlaps the rest
+        }
+        Bar::sync();
+        if (ss.ok) {
+            // every CTA has read the merged histogram: clear this CTA's share of it
+            const uint32_t per4 = (kBins / 4 + gridDim.x - 1) / gridDim.x;
+            const uint32_t z0 = blockIdx.x * per4, z1 = min((uint32_t)(kBins / 4), z0 + per4);
+            for (uint32_t i = z0 + tid; i < z1; i += T)
+                reinterpret_cast<uint4*>(q.hist0)[i] = make_uint4(0, 0, 0, 0);
+            constexpr int kLd = Cfg::kFastCap / T;
+            uint2 v[kLd];
+#pragma unroll
+            for (int u = 0; u < kLd; ++u) {
+                const uint32_t i = tid + u * T;
+                v[u] = i < nb0 ? __ldcg(&q.cand[i]) : make_uint2(0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kLd; ++u) {
+                const uint32_t i = tid + u * T;
+                if (i < nb0) s_cand[i] = v[u];
+            }
+            Bar::sync();
+            const uint32_t need = (uint32_t)k - above;
+            const uint32_t per = (nb0 + gridDim.x - 1) / gridDim.x;
+            const uint32_t c0 = min(nb0, blockIdx.x * per), c1 = min(nb0, c0 + per);
+            const uint32_t wl = (uint32_t)tid & 31u;
+            for (uint32_t i = c0 + (uint32_t)(tid >> 5); i < c1; i += T / 32) {  // a warp per candidate
+                const uint2 me = s_cand[i];
+                uint32_t rank = 0;
+                for (uint32_t j = wl; j < nb0; j += 32) {
+                    const uint2 o = s_cand[j];
+                    rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+                }
+                rank = __reduce_add_sync(0xffffffffu, rank);
+                if (wl == 0 && rank < need) sel::emit(q, above + rank, me);
+            }
+        }
+        if (tid == 0) {
+            ss.last = ticket == gridDim.x - 1;
+            ss.nt = ss.last ? __ldcg(&q.ctr[kCtrDirty]) : 0u;  // read before the reset below
+        }
+        Bar::sync();
+        if (ss.last) sel::reset_query(q, tid, ss.nt != 0u);
+        return;
+    }
+    uint2* s_listA = reinterpret_cast<uint2*>(sA);
+    uint2* s_listB = s_listA + sel::kListCap;
+
+    // Fallback (a threshold bin of more than kFastCap keys, or a timed-out meeting): each
+    // CTA emits its keys above b0 and appends b0's to the candidate list through global
+    // counters; the last CTA (atomic ticket) resolves the candidates digit by digit.
+    if (ok) {
+        const uint32_t b0 = ss.bin;
+        for (int base = 0; base < npos; base += sel::kRound) {
+            uint32_t key[sel::kPer], eidx[sel::kPer];
+            bool valid[sel::kPer];
+            load_keys(base, key, eidx, valid);
             sel::classify_round<Bar>(q, key, eidx, valid, b0, s_listA, s_listB, &ss, tid);
         }
     }

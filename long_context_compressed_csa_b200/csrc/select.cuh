@@ -117,6 +117,48 @@ CSA_DEV void find_threshold_bin(const uint32_t* hist, uint32_t need, Shared* s, 
     Bar::sync();
 }
 
+// find_threshold_bin over a kBins histogram in the hist_slot layout that also replaces
+// each bin's count by the count of the bins above it (an exclusive suffix sum: the first
+// output slot of the bin's entries when entries are placed from the top bin down) and
+// sets s->cnt to the threshold bin's own count.
+template <class Bar>
+CSA_DEV void threshold_and_suffix(uint32_t* hist, uint32_t need, Shared* s, int tid)
+{
+    constexpr int PER = kBins / kSelThreads;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int lo = kBins - (tid + 1) * PER;  // this thread covers [lo, lo + PER)
+    uint32_t v[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) v[i] = hist[hist_slot((uint32_t)(lo + i))];
+    uint32_t local = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) local += v[i];
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+    }
+    if (lane == 31) s->scr[warp] = incl;
+    Bar::sync();
+    uint32_t base = 0;
+#pragma unroll
+    for (int w = 0; w < kSelThreads / 32; ++w) base += w < warp ? s->scr[w] : 0u;
+    uint32_t cum = base + incl - local;  // count in the bins above this thread's range
+#pragma unroll
+    for (int i = PER - 1; i >= 0; --i) {
+        const uint32_t bin = (uint32_t)(lo + i);
+        if (cum < need && need <= cum + v[i]) {
+            s->bin = bin;
+            s->above = cum;
+            s->cnt = v[i];
+        }
+        hist[hist_slot(bin)] = cum;
+        cum += v[i];
+    }
+    Bar::sync();
+}
+
 // Warp-aggregated append: this lane's slot in a list whose length counter is *ctr, for
 // lanes with pred true.  All lanes of the warp call.
 CSA_DEV uint32_t warp_append(uint32_t* ctr, bool pred)

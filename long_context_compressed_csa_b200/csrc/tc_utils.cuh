@@ -82,6 +82,23 @@ CSA_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+// L2 policy for data read once: its lines are the first to go, so a stream does not
+// push out what other work (code, counters, the next kernel's inputs) keeps in L2.
+CSA_DEV uint64_t l2_evict_first_policy()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// tma_load_2d with an L2 cache policy (l2_evict_first_policy) for the loaded lines.
+CSA_DEV void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
 // 2-D tiled bulk tensor store from this CTA's shared memory (completion tracked by the
 // issuing thread's bulk groups).  x (innermost) must be a multiple of 16 bytes / element size.
 CSA_DEV void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y)

@@ -340,6 +340,36 @@ def test_indexer_topk_exact_on_integer_inputs(dtype, n_hI, cI):
         assert sorted(idx2.reshape(-1, k)[g].tolist()) == sorted(idx.reshape(-1, k)[g].tolist())
 
 
+@pytest.mark.parametrize("k,lo,hi", [(1000, 2048, 4096), (4000, 4097, 30000)])
+def test_indexer_topk_wide_threshold_bin(k, lo, hi):
+    """Scores that crowd into a few digit-0 bins (0/1 inputs; unit weights for the first
+    query, -2..2 for the second), so the bin holding the k-th score is wide.  With
+    k = 1000 it holds 2000-4000 keys: every CTA of the in-place select ranks a share of
+    that candidate list.  With k = 4000 it holds over 4096: one CTA resolves it digit by
+    digit instead.  Scores are exact in fp32, so the sets (ties to the smaller index)
+    must equal the oracle's, and a second call on the same workspace must repeat them."""
+    B, nq, n_hI, cI, N_cap, m = 1, 2, 64, 128, 30000, 4
+    qI = randint_values((B, nq, n_hI, cI), 270, 0, 2, torch.bfloat16)
+    KI = randint_values((B, N_cap, cI), 271, 0, 2, torch.bfloat16)
+    wI = torch.ones((B, nq, n_hI), dtype=torch.float32)
+    wI[0, 1] = randint_values((n_hI,), 272, -2, 3, torch.float32)
+    t = [4 * N_cap, 4 * N_cap - 1]
+    idx, sc, ws = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k)
+    for q in range(nq):
+        vis = oracle.visible(t[q], m, N_cap)
+        s = oracle.index_scores(to_f64(qI[0, q]), to_f64(wI[0, q]), to_f64(KI[0]), vis)
+        want = oracle.topk(s, k)
+        # the threshold bin (top 12 bits of the fp32 order key) really has that width
+        u = s.astype(np.float32).view(np.uint32)
+        d0 = np.where(u >> 31, ~u, u | np.uint32(0x80000000)) >> 20
+        assert lo <= np.sum(d0 == d0[want[k - 1]]) <= hi
+        assert sorted(idx[0, q].tolist()) == sorted(want.tolist())
+        np.testing.assert_array_equal(sc[0, q], s[idx[0, q]])
+    idx2, _, _ = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k, ws=ws)
+    for q in range(nq):
+        assert sorted(idx2[0, q].tolist()) == sorted(idx[0, q].tolist())
+
+
 @pytest.mark.parametrize("dtype,n_hI,cI,N_cap,k", [(torch.bfloat16, 64, 128, 20000, 512),
                                                    (torch.float32, 16, 32, 5000, 100),
                                                    (torch.bfloat16, 32, 64, 1500, 1024)])
