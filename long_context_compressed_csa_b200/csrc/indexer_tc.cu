@@ -179,6 +179,10 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict_
         tc::prefetch_l2(qI + (int64_t)g * NH * CI, NH * CI * 2);
     }
     pdl_wait();
+    // the workspace's wait-budget override, a test hook read by the thread that later runs
+    // the select's meetings: issued here, where its round trip overlaps the scan
+    long long budget_ov = 0;
+    if (threadIdx.x == 64) budget_ov = *reinterpret_cast<const volatile long long*>(ws.status + 2);
     const int64_t vis = visible_of(t, g, m, N_cap);
     const int ntiles = (int)((vis + kTileKeys - 1) / kTileKeys);
     const bool active = (int)blockIdx.x < ntiles;  // otherwise the CTA is idle for this query
@@ -463,10 +467,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict_
     };
 
     // first meeting: every CTA's histogram is merged
-    long long budget = tc::kWaitBudget;  // tid 0 runs both meetings
+    // tid 0 (thread 64, which read the override) runs both meetings
+    const long long budget = budget_ov > 0 ? budget_ov : tc::kWaitBudget;
     if (tid == 0) {
-        const long long ov = *reinterpret_cast<const volatile long long*>(ws.status + 2);
-        if (ov > 0) budget = ov;  // a test hook that makes the waits run out
         red_release_add(&q.ctr[3], 1u);
         const bool ok = wait_count_geq(&q.ctr[3], gridDim.x, budget);
         if (!ok) atomicExch(ws.status, 1u);

@@ -340,6 +340,26 @@ def test_indexer_topk_exact_on_integer_inputs(dtype, n_hI, cI):
         assert sorted(idx2.reshape(-1, k)[g].tolist()) == sorted(idx.reshape(-1, k)[g].tolist())
 
 
+@pytest.mark.parametrize("k,N_cap,run", [(200, 40000, 300), (1024, 262144, 2048)])
+def test_indexer_topk_clustered_top_keys(k, N_cap, run):
+    """The top keys crowd into a few consecutive key tiles (a run of keys scaled by 3, so
+    every one of the k best lies inside it): the CTAs holding those tiles have far more
+    top keys than the others, which the in-place select must place exactly as well as
+    evenly spread ones.  Sets identical to the oracle's except for fp32 near-ties."""
+    B, nq, n_hI, cI, m, r0 = 1, 1, 64, 128, 4, 12345
+    qI = randn((B, nq, n_hI, cI), 280, torch.bfloat16)
+    KI = randn((B, N_cap, cI), 281, torch.bfloat16)
+    KI[0, r0:r0 + run] *= 3
+    wI = randn((B, nq, n_hI), 282, torch.float32).abs()
+    t = [4 * N_cap]
+    idx, sc, _ = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k)
+    q64, w64, K64 = to_f64(qI[0, 0]), to_f64(wI[0, 0]), to_f64(KI[0])
+    s = oracle.index_scores(q64, w64, K64, N_cap)
+    top = oracle.topk(s, k)
+    assert np.all((top >= r0) & (top < r0 + run))  # the run holds the top k
+    check_topk_sets(idx[0, 0], s, k, lambda d: score_error_bound(q64, w64, K64, d))
+
+
 @pytest.mark.parametrize("k,lo,hi", [(1000, 2048, 4096), (4000, 4097, 30000)])
 def test_indexer_topk_wide_threshold_bin(k, lo, hi):
     """Scores that crowd into a few digit-0 bins (0/1 inputs; unit weights for the first
