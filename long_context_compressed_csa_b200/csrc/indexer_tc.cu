@@ -29,7 +29,7 @@ namespace {
 
 constexpr int kTcThreads = 320;  // producer, MMA, two groups of 4 epilogue warps
 constexpr int kTileKeys = 128;
-constexpr int kPrefetchTiles = 4;  // key tiles per CTA prefetched into L2 before the dependency wait
+constexpr int kPrefetchTiles = 2;  // key tiles per CTA prefetched into L2 before the dependency wait
 
 // KB: bytes per key / query element (2: bf16, 1: E4M3)
 template <int NH, int CI, int KB = 2>
