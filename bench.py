@@ -35,9 +35,9 @@ METRIC = "CSA/HCA decode tokens/s at 128K–1M ctx; achieved HBM GB/s vs ~8 TB/s
 WORKLOAD = "hybrid_1m_decode"
 N_PAIRS = 8
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one scan_tc_kernel launch
-# over 262144 keys, from one ncu capture of the current kernel (67.22 MB read, 0.56 MB
+# over 262144 keys, from one ncu capture of the current kernel (67.21 MB read, 0.73 MB
 # written; algorithmic 67.11 MB).  Must be retaken (or set to None) when the kernel changes.
-SCAN_TRAFFIC_BYTES = None  # the select tail changed since the last capture
+SCAN_TRAFFIC_BYTES = 67_941_888
 IDX_SAMPLE = 8  # steps per CUDA graph; the indexer call of each graph's first step is timed
 
 
