@@ -240,6 +240,56 @@ def index_scores_e4m3(qI, wI, KI, nvis=None):
     return index_scores(qc * qs[:, None], wI, kc * ks[:, None], nvis)
 
 
+# ----------------------------------------------------------------------------------
+# FP4 (E2M1) indexer keys.  [P1] section 6.4 runs the indexer's products in FP4; the
+# element and scale formats are not given.  The reading used: OCP E2M1 codes (1 sign, 2
+# exponent bits with bias 1, 1 mantissa bit, one subnormal 0.5; values 0, 0.5, 1, 1.5,
+# 2, 3, 4, 6) with one fp32 scale per key = max|x| / 6; the codes are E2M1(x * (6 /
+# max|x|)), the product in fp32, rounded to nearest even and saturated at +-6.  The
+# query stays E4M3 per head (quantize_rows_e4m3): the key cache is what the scan streams,
+# the query is 16 KB.
+# ----------------------------------------------------------------------------------
+E2M1_MAX = 6.0
+E2M1_VALUES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)  # magnitudes of codes 0..7
+
+
+def round_e2m1(x):
+    """Round fp32 values to the nearest E2M1 value, ties to the even code (mantissa bit
+    0), saturating at +-6 (the format's definition; as float64)."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    a = np.minimum(np.abs(x), E2M1_MAX)
+    # grid spacing at |x|: 0.5 below 2, 1 in [2, 4), 2 in [4, 6]
+    step = np.where(a < 2.0, 0.5, np.where(a < 4.0, 1.0, 2.0))
+    r = np.round(a / step) * step  # np.round: half to even, which is the even code here
+    r = np.minimum(r, E2M1_MAX)
+    return np.where(a > 0, np.copysign(r, x), 0.0 * x)
+
+
+def quantize_rows_e2m1(X):
+    """Per-row E2M1 quantisation: dequantisation scale = max|x| / 6 and quantisation
+    factor r = 6 / max|x|, both one fp32 division per row; code = E2M1(x * r) with the
+    product in fp32 (rows of zeros: scale 0, codes 0).  Returns (values of the codes
+    [rows, cols] float64, scales [rows] float64)."""
+    X = np.asarray(X, dtype=np.float32)
+    X2 = X.reshape(-1, X.shape[-1])
+    amax = np.max(np.abs(X2), axis=1).astype(np.float32)
+    scale = (amax / np.float32(E2M1_MAX)).astype(np.float32)
+    safe = np.where(amax > 0, amax, np.float32(1.0)).astype(np.float32)
+    r = (np.float32(E2M1_MAX) / safe).astype(np.float32)
+    q = (X2 * r[:, None]).astype(np.float32)
+    codes = np.where(amax[:, None] > 0, round_e2m1(q), 0.0)
+    return codes.reshape(X.shape), scale.astype(np.float64).reshape(X.shape[:-1])
+
+
+def index_scores_e2m1(qI, wI, KI, nvis=None):
+    """[P1] section 6.4 scores with E2M1 keys (quantize_rows_e2m1, one scale per key) and
+    E4M3 query heads (quantize_rows_e4m3, one scale per head); the boxed formula is
+    evaluated in fp64 on the dequantised values (code x scale)."""
+    qc, qs = quantize_rows_e4m3(qI)
+    kc, ks = quantize_rows_e2m1(KI)
+    return index_scores(qc * qs[:, None], wI, kc * ks[:, None], nvis)
+
+
 def round_bf16(x):
     """Round float64/float32 values to the nearest bfloat16 (ties to even), as float64.
 

@@ -518,3 +518,67 @@ def test_e4m3_row_quantisation_and_scores():
     bound = np.abs(wI) @ (np.abs(qI) @ np.abs(KI).T) * (2 * 2.0 ** -4 + 2.0 ** -8) + 1e-9
     assert np.all(np.abs(s8 - s) <= bound)
     assert np.corrcoef(s8, s)[0, 1] > 0.99
+
+
+# ==================================================================================
+# FP4 (E2M1) indexer keys (reading of [P1] section 6.4 "FP4 indexer"; format chosen:
+# E2M1 codes with one fp32 scale per key, the query E4M3 per head)
+# ==================================================================================
+def _e2m1_table():
+    """Every E2M1 value, decoded from the 4-bit codes by the format definition (sign,
+    2-bit exponent with bias 1, 1-bit mantissa, subnormal at exponent 0)."""
+    vals = []
+    for code in range(16):
+        s, e, m = code >> 3, (code >> 1) & 3, code & 1
+        v = (m / 2.0) if e == 0 else (1 + m / 2.0) * 2.0 ** (e - 1)
+        vals.append(-v if s else v)
+    return np.unique(np.array(vals))
+
+
+def test_e2m1_rounding_pins():
+    tab = _e2m1_table()
+    np.testing.assert_array_equal(tab[tab >= 0], [0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    np.testing.assert_array_equal(oracle.round_e2m1(tab.astype(np.float32)), tab)
+    # midpoints go to the neighbour whose code has mantissa bit 0
+    mids = np.float32([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    np.testing.assert_array_equal(oracle.round_e2m1(mids), [0, 1, 1, 2, 2, 4, 4])
+    np.testing.assert_array_equal(oracle.round_e2m1(-mids), -np.array([0, 1, 1, 2, 2, 4, 4.0]))
+    # saturation and nearest rounding away from midpoints
+    np.testing.assert_array_equal(oracle.round_e2m1(np.float32([6.5, 100.0, -7.0, 5.01, 0.26, 0.24])),
+                                  [6, 6, -6, 6, 0.5, 0])
+    rng = np.random.default_rng(5)
+    x = rng.uniform(-6, 6, 4000).astype(np.float32)
+    r = oracle.round_e2m1(x)
+    idx = np.abs(tab[None, :] - x[:, None].astype(np.float64)).argmin(axis=1)
+    np.testing.assert_array_equal(np.abs(r - x), np.abs(tab[idx] - x))
+
+
+def test_e2m1_row_quantisation_and_scores():
+    # a hand-worked row: max|x| = 6, so the factor is 1 and the codes are E2M1(x)
+    codes, scale = oracle.quantize_rows_e2m1(np.float32([[6.0, 3.0, 1.4, -0.2, 0.0, 5.2, -2.6, 0.8]]))
+    assert scale[0] == 1.0
+    np.testing.assert_array_equal(codes[0], [6, 3, 1.5, -0, 0, 6, -3, 1])
+    rng = np.random.default_rng(6)
+    X = rng.standard_normal((60, 128)).astype(np.float32)
+    X[9] = 0.0
+    codes, scale = oracle.quantize_rows_e2m1(X)
+    assert scale[9] == 0 and np.all(codes[9] == 0)
+    amax = np.abs(X).max(axis=1)
+    rows = np.arange(60) != 9
+    np.testing.assert_array_equal(scale[rows], (amax[rows] / np.float32(6)).astype(np.float32))
+    assert np.all(np.abs(codes[rows]).max(axis=1) == 6.0)   # the largest entry maps to +-6
+    assert np.all(np.isin(codes, _e2m1_table()))
+    # E2M1 error: at most a quarter of max(|x|, scale) (half a grid step)
+    deq = codes * scale[:, None]
+    tol = 0.25 * np.maximum(np.abs(X), scale[:, None]) * (1 + 1e-6)
+    assert np.all(np.abs(deq - X) <= tol)
+    # scores with E2M1 keys and E4M3 queries stay within the operands' error
+    qI, wI, KI = rng.standard_normal((16, 128)), rng.standard_normal(16), rng.standard_normal((300, 128))
+    s4 = oracle.index_scores_e2m1(qI, wI, KI)
+    s = oracle.index_scores(qI, wI, KI)
+    kc, ks = oracle.quantize_rows_e2m1(KI)
+    dk = 0.25 * (np.abs(KI) + ks[:, None])                 # key error bound per element
+    dq = 2.0 ** -4 * np.abs(qI) + 2.0 ** -9 * np.abs(qI).max(axis=1, keepdims=True) / 448
+    bound = np.abs(wI) @ ((np.abs(qI) + dq) @ dk.T + dq @ np.abs(KI).T) + 1e-9
+    assert np.all(np.abs(s4 - s) <= bound)
+    assert np.corrcoef(s4, s)[0, 1] > 0.9
