@@ -285,6 +285,44 @@ int csa_quantize_e4m3(const void* x, int64_t rows, int cols, int64_t ld, void* c
                       float* scales, int dtype, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * csa_quantize_e2m1 - per-row E2M1 (FP4) quantisation of indexer keys (or any rows).
+ *   Source: [P1] section 6.4 runs the indexer in FP4; the element and scale formats are
+ *   not given.  The reading used: OCP E2M1 codes (values 0, 0.5, 1, 1.5, 2, 3, 4, 6 and
+ *   their negatives) with one fp32 scale per row, scale = max|x| / 6 (0 for an all-zero
+ *   row); code = E2M1(x * (6 / max|x|)), the factor one fp32 division per row and the
+ *   product in fp32, rounded to nearest even and saturated at +-6.
+ * x      : [rows, cols] (dtype bf16 or fp32) with row stride ld (elements), cols % 8 == 0
+ * codes  : [rows, cols / 2] bytes, contiguous (4-byte aligned); two codes per byte, the
+ *          even column in the low nibble (bits 0-2 magnitude, bit 3 sign)
+ * scales : fp32 [rows]
+ * ------------------------------------------------------------------------------- */
+int csa_quantize_e2m1(const void* x, int64_t rows, int cols, int64_t ld, void* codes,
+                      float* scales, int dtype, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * csa_indexer_topk_e2m1 - csa_indexer_topk on E2M1 keys: the [P1] section 6.4 scores of
+ * the dequantised operands, then the same top-k (section 7).  q^I (bf16) is quantised per
+ * head to E4M3 inside the kernel with the csa_quantize_e4m3 rule (the query is 16 KB; the
+ * key cache is what the scan streams).  The products run on the tensor cores (E2M1 x
+ * E4M3 -> fp32), and the score is
+ *   KI_scale[s] * sum_h (w_h * scale_h) * ReLU(q8_h . K4_s),
+ * which equals the boxed formula on the dequantised values since the scales are >= 0.
+ * KI4      : [B, N_cap, cI / 2] bytes of E2M1 codes as written by csa_quantize_e2m1
+ *            (32-byte aligned), KI_scale: fp32 [B, N_cap]
+ * qI       : [B, nq, n_hI, cI] bf16 (16-byte aligned); other arguments, the workspace
+ *            (csa_indexer_topk_workspace_size) and the outputs as for csa_indexer_topk.
+ * Supported: n_hI in {16, 32, 64, 128}, cI in {128, 256}, B*nq <= 65535;
+ * CSA_ERR_UNSUPPORTED otherwise.
+ * Keys take half a byte: the scan of the 1M-token decode reads 17.8 MB of codes and
+ * scales instead of 67.1 MB.
+ * ------------------------------------------------------------------------------- */
+int csa_indexer_topk_e2m1(const void* qI, const float* wI, const void* KI4,
+                          const float* KI_scale, const int64_t* t, int B, int nq,
+                          int64_t N_cap, int n_hI, int cI, int m, int k, int32_t* idx_out,
+                          float* scores_out, void* workspace, size_t ws_bytes,
+                          csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * csa_indexer_topk_e4m3 - csa_indexer_topk on E4M3 keys: the [P1] section 6.4 scores of
  * the dequantised operands, then the same top-k (section 7).  q^I (bf16) is quantised per
  * head inside the kernel with the csa_quantize_e4m3 rule; the products run on the tensor

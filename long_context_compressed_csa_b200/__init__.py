@@ -13,10 +13,12 @@ from ._binding import (  # noqa: F401
     csa_attn_workspace_size,
     csa_compress,
     csa_indexer_topk,
+    csa_indexer_topk_e2m1,
     csa_indexer_topk_e4m3,
     csa_indexer_topk_noalloc,
     csa_indexer_topk_noalloc_status,
     csa_indexer_topk_workspace_size,
+    csa_quantize_e2m1,
     csa_quantize_e4m3,
     csa_sparse_attn,
     csa_status_string,

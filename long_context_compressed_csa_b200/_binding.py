@@ -41,6 +41,8 @@ _SIGS = {
                        i32),
     "csa_quantize_e4m3": ([vp, i64, i32, i64, vp, vp, i32, vp], i32),
     "csa_indexer_topk_e4m3": ([vp, vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, i32, vp, vp, vp, sz, vp], i32),
+    "csa_quantize_e2m1": ([vp, i64, i32, i64, vp, vp, i32, vp], i32),
+    "csa_indexer_topk_e2m1": ([vp, vp, vp, vp, vp, i32, i32, i64, i32, i32, i32, i32, vp, vp, vp, sz, vp], i32),
     "csa_sparse_attn_window": ([vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i32, i32, i64, f32, vp, vp,
                                 vp, sz, i32, i32, vp], i32),
     "hca_dense_attn_window": ([vp, vp, vp, vp, i32, i32, i32, i32, i64, i32, i32, i64, f32, vp, vp, vp,
@@ -274,6 +276,31 @@ def csa_indexer_topk_e4m3(qI, wI, KI8, KI_scale, t, m, k, idx_out, workspace, sc
     assert KI8.shape == (B, N_cap, cI) and KI_scale.shape == (B, N_cap) and idx_out.shape == (B, nq, k)
     _check("csa_indexer_topk_e4m3", library().csa_indexer_topk_e4m3(
         _ptr(qI), _ptr(wI), _ptr(KI8), _ptr(KI_scale), _ptr(t), B, nq, N_cap, n_hI, cI, m, k, _ptr(idx_out),
+        _ptr(scores_out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def csa_quantize_e2m1(x, codes, scales, stream=None):
+    """Per-row E2M1 codes (uint8 tensor [..., cols / 2], two codes per byte) and fp32
+    scales (x.shape[:-1]) of x [..., cols] (bf16 or fp32, rows contiguous)."""
+    _cuda(x, codes, scales)
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols else 0
+    assert x.is_contiguous() and codes.is_contiguous() and scales.is_contiguous()
+    assert codes.shape == x.shape[:-1] + (cols // 2,) and codes.element_size() == 1 and scales.numel() == rows
+    _check("csa_quantize_e2m1", library().csa_quantize_e2m1(
+        _ptr(x), rows, cols, cols, _ptr(codes), _ptr(scales), _dtype(x), _stream(stream)))
+
+
+def csa_indexer_topk_e2m1(qI, wI, KI4, KI_scale, t, m, k, idx_out, workspace, scores_out=None, stream=None):
+    """csa_indexer_topk on E2M1 keys KI4 [B,N_cap,cI/2] (uint8, two codes per byte) with
+    scales [B,N_cap]; qI bf16."""
+    _cuda(qI, wI, KI4, KI_scale, t, idx_out, workspace, scores_out)
+    B, nq, n_hI, cI = qI.shape
+    N_cap = KI4.shape[1]
+    assert qI.is_contiguous() and KI4.is_contiguous() and KI_scale.is_contiguous()
+    assert KI4.shape == (B, N_cap, cI // 2) and KI_scale.shape == (B, N_cap) and idx_out.shape == (B, nq, k)
+    _check("csa_indexer_topk_e2m1", library().csa_indexer_topk_e2m1(
+        _ptr(qI), _ptr(wI), _ptr(KI4), _ptr(KI_scale), _ptr(t), B, nq, N_cap, n_hI, cI, m, k, _ptr(idx_out),
         _ptr(scores_out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 

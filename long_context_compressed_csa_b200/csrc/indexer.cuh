@@ -45,6 +45,14 @@ int launch_scan_tc_e4m3(const void* qI, const float* wI, const void* KI8, const 
                         const int64_t* t, int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
                         const TopkWs& ws, int32_t* idx_out, float* scores_out, bool* fused,
                         cudaStream_t stream);
+// E2M1 keys (two codes per byte, k_scale one fp32 scale per key) with bf16 queries
+// quantised here per head to E4M3: kind::f8f6f4 with an E2M1 A operand, the codes
+// unpacked by the TMA into the 16-byte-aligned layout that operand reads.
+bool indexer_e2m1_supported(int n_hI, int cI);
+int launch_scan_tc_e2m1(const void* qI, const float* wI, const void* KI4, const float* k_scale,
+                        const int64_t* t, int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k,
+                        const TopkWs& ws, int32_t* idx_out, float* scores_out, bool* fused,
+                        cudaStream_t stream);
 // Many queries of one batch row at once (chunked prefill): tcgen05 scores of a resident
 // block of queries against streamed key tiles, into ws.scores; the stand-alone select
 // with self_hist follows.

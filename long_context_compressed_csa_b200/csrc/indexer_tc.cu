@@ -107,7 +107,7 @@ struct SelOut {
 // key (k_scale), bf16 queries quantised here per head to E4M3 (kind::f8f6f4); the score
 // is then k_scale[s] * sum_h (w_h * q_scale_h) ReLU(q8_h . k8_s), which equals the boxed
 // formula on the dequantised operands because the scales are non-negative.
-template <int NH, int CI, int KB>
+template <int NH, int CI, int KB, bool KF4 = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
 scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict__ tmap_base,
                const __nv_bfloat16* __restrict__ qI, const float* __restrict__ wI, const float* __restrict__ k_scale,
@@ -168,13 +168,14 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict_
     // coherence (an entry the previous kernel appends is updated in L2), so their DRAM
     // reads overlap the previous kernel instead of starting the scan.
     if (threadIdx.x == 32) {
-        const char* kb = static_cast<const char*>(tmap_base) + (size_t)b * N_cap * CI * KB;
+        constexpr int kRowBytes = KF4 ? CI / 2 : CI * KB;  // one key in global memory
+        const char* kb = static_cast<const char*>(tmap_base) + (size_t)b * N_cap * kRowBytes;
         const int64_t tiles_cap = (N_cap + kTileKeys - 1) / kTileKeys;
         for (int i = 0; i < kPrefetchTiles; ++i) {
             const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
             if (tile >= tiles_cap) break;
             const int64_t rows = min((int64_t)kTileKeys, N_cap - tile * kTileKeys);
-            tc::prefetch_l2(kb + tile * kTileKeys * CI * KB, (uint32_t)(rows * CI * KB));
+            tc::prefetch_l2(kb + tile * kTileKeys * kRowBytes, (uint32_t)(rows * kRowBytes));
         }
         tc::prefetch_l2(qI + (int64_t)g * NH * CI, NH * CI * 2);
     }
@@ -203,7 +204,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict_
                     *abort_flag = 1;
                     break;
                 }
-                tc::mbar_arrive_expect_tx(&full[s], Cfg::kAStage);
+                // packed E2M1 codes count their global bytes (half the unpacked tile)
+                tc::mbar_arrive_expect_tx(&full[s], KF4 ? Cfg::kAStage / 2 : Cfg::kAStage);
                 const int row0 = (int)(b * N_cap) + tile * kTileKeys;
 #pragma unroll
                 for (int p = 0; p < Cfg::kPanels; ++p)
@@ -218,6 +220,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict_
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdesc = KB == 2 ? tc::idesc_bf16_f32(128, NH, false, false)
+                                        : KF4   ? tc::idesc_e2m1_e4m3_f32(128, NH)
                                                 : tc::idesc_e4m3_f32(128, NH);
             if (!tc::mbar_wait(qready, 0, tc::kWaitBudget)) *abort_flag = 1;
             int it = 0;
@@ -603,13 +606,13 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict_
     sel::reset_query(q, tid);
 }
 
-template <int NH, int CI, int KB>
+template <int NH, int CI, int KB, bool KF4 = false>
 int launch_nh_ci(const CUtensorMap& tmap, const void* KI, const void* qI, const float* wI, const float* k_scale, const int64_t* t,
                  int B, int nq, int64_t N_cap, int m, int k, const TopkWs& ws, int32_t* idx_out,
                  float* scores_out, bool* fused, cudaStream_t stream)
 {
     using Cfg = ScanCfg<NH, CI, KB>;
-    auto kern = scan_tc_kernel<NH, CI, KB>;
+    auto kern = scan_tc_kernel<NH, CI, KB, KF4>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
     const int G = B * nq;
     const int64_t tiles = (N_cap + kTileKeys - 1) / kTileKeys;
@@ -689,6 +692,30 @@ int launch_scan_tc_e4m3(const void* qI, const float* wI, const void* KI8, const 
     CSA_SCAN8_CASE(16, 128) CSA_SCAN8_CASE(16, 256) CSA_SCAN8_CASE(32, 128) CSA_SCAN8_CASE(32, 256)
     CSA_SCAN8_CASE(64, 128) CSA_SCAN8_CASE(64, 256) CSA_SCAN8_CASE(128, 128) CSA_SCAN8_CASE(128, 256)
 #undef CSA_SCAN8_CASE
+    return CSA_ERR_UNSUPPORTED;
+}
+
+bool indexer_e2m1_supported(int n_hI, int cI)
+{
+    return (n_hI == 16 || n_hI == 32 || n_hI == 64 || n_hI == 128) && (cI == 128 || cI == 256);
+}
+
+int launch_scan_tc_e2m1(const void* qI, const float* wI, const void* KI4, const float* k_scale, const int64_t* t,
+                        int B, int nq, int64_t N_cap, int n_hI, int cI, int m, int k, const TopkWs& ws,
+                        int32_t* idx_out, float* scores_out, bool* fused, cudaStream_t stream)
+{
+    *fused = false;
+    if (N_cap == 0) return CSA_OK;
+    if ((int64_t)B * N_cap + kTileKeys >= (int64_t(1) << 31)) return CSA_ERR_UNSUPPORTED;
+    if (!aligned16(qI) || ((uintptr_t)KI4 & 31)) return CSA_ERR_ALIGN;
+    CUtensorMap tmap;  // E2M1 codes [B * N_cap rows][cI codes], 128 x 128 boxes, unpacked to 1 byte per code
+    if (!make_tmap_e2m1_2d(&tmap, KI4, (uint64_t)B * N_cap, cI, kTileKeys)) return CSA_ERR_CUDA;
+#define CSA_SCAN4_CASE(NH_, CI_) \
+    if (n_hI == NH_ && cI == CI_)   \
+        return launch_nh_ci<NH_, CI_, 1, true>(tmap, KI4, qI, wI, k_scale, t, B, nq, N_cap, m, k, ws, idx_out, scores_out, fused, stream);
+    CSA_SCAN4_CASE(16, 128) CSA_SCAN4_CASE(16, 256) CSA_SCAN4_CASE(32, 128) CSA_SCAN4_CASE(32, 256)
+    CSA_SCAN4_CASE(64, 128) CSA_SCAN4_CASE(64, 256) CSA_SCAN4_CASE(128, 128) CSA_SCAN4_CASE(128, 256)
+#undef CSA_SCAN4_CASE
     return CSA_ERR_UNSUPPORTED;
 }
 

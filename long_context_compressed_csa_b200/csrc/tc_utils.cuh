@@ -310,6 +310,16 @@ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, bool b_mn)
            | ((uint32_t)(M >> 4) << 24);// M / 16
 }
 
+// Instruction descriptor of kind::f8f6f4 with an E2M1 A (format code 5) and an E4M3 B
+// (format code 0), fp32 D, dense, both operands K-major.
+constexpr uint32_t idesc_e2m1_e4m3_f32(int M, int N)
+{
+    return (1u << 4)                    // D format: f32
+           | (5u << 7)                  // A format: E2M1
+           | ((uint32_t)(N >> 3) << 17) // N / 8
+           | ((uint32_t)(M >> 4) << 24);// M / 16  (B format field 0: E4M3)
+}
+
 // Instruction descriptor of kind::f8f6f4 with E4M3 A and B (format code 0), fp32 D, dense,
 // both operands K-major.
 constexpr uint32_t idesc_e4m3_f32(int M, int N)
@@ -338,6 +348,11 @@ bool make_tmap_bf16_2d_plain(CUtensorMap* map, const void* base, uint64_t rows, 
 // Same for a 2-D tensor of bytes (E4M3 codes).
 bool make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                      uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);
+// Host: encode a 2-D tensor map of packed E2M1 codes (rows x cols codes, cols/2 bytes per
+// row, cols a multiple of 128, base 32-byte aligned) with 128 x box_rows boxes unpacked by
+// the TMA to 16 bytes per 16 codes in shared memory (the layout of an E2M1 operand of
+// kind::f8f6f4), 128-byte swizzle; false if the driver call fails.
+bool make_tmap_e2m1_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 // Same for a 2-D fp32 tensor.
 bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                       uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);

@@ -72,6 +72,20 @@ bool make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_e2m1_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    EncodeTiled fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};      // in codes
+    cuuint64_t strides[1] = {cols / 2};     // bytes per row
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                       uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows)
 {

@@ -56,3 +56,14 @@ def decode_e4m3(codes):
     v = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1 + m / 8.0) * 2.0 ** (e - 7.0))
     assert not np.any((e == 15) & (m == 7)), "NaN code"
     return np.where(s == 1, -v, v)
+
+
+def decode_e2m1(packed):
+    """Values of E2M1 codes packed two per byte (numpy uint8 array [..., n]), the even
+    element in the low nibble, decoded from the format definition: sign, 2-bit exponent
+    with bias 1, 1-bit mantissa, subnormal at exponent 0.  Returns [..., 2 n]."""
+    b = np.asarray(packed, dtype=np.uint8).astype(np.int64)
+    c = np.stack([b & 15, b >> 4], axis=-1).reshape(b.shape[:-1] + (2 * b.shape[-1],))
+    s, e, m = c >> 3, (c >> 1) & 3, c & 1
+    v = np.where(e == 0, m / 2.0, (1 + m / 2.0) * 2.0 ** (e - 1.0))
+    return np.where(s == 1, -v, v)

@@ -122,6 +122,16 @@ def test_host_validation_rejects_bad_arguments_without_launching(lib):
     assert lib.csa_quantize_e4m3(fake, 10, 8, 8, fake, fake, 9, None) == -3
     assert lib.csa_indexer_topk_e4m3(fake, fake, fake, fake, fake, 1, 1, 100, 64, 64, 4, 8, fake, None,
                                      fake, 1 << 30, None) == -6
+    # E2M1: cols not a multiple of 8, bad dtype; indexer with an unsupported cI, codes not
+    # 32-byte aligned, more queries than grid rows
+    assert lib.csa_quantize_e2m1(fake, 10, 12, 12, fake, fake, 0, None) == -1
+    assert lib.csa_quantize_e2m1(fake, 10, 16, 16, fake, fake, 9, None) == -3
+    assert lib.csa_indexer_topk_e2m1(fake, fake, fake, fake, fake, 1, 1, 100, 64, 64, 4, 8, fake, None,
+                                     fake, 1 << 30, None) == -6
+    assert lib.csa_indexer_topk_e2m1(fake, fake, vp(0x10010), fake, fake, 1, 1, 100, 64, 128, 4, 8, fake, None,
+                                     fake, 1 << 30, None) == -2
+    assert lib.csa_indexer_topk_e2m1(fake, fake, fake, fake, fake, 2, 40000, 100, 64, 128, 4, 8, fake,
+                                     None, fake, 1 << 62, None) == -6
     # fused projection + HCA compression: m' other than 128, d not a multiple of 64,
     # no workspace, a workspace too small
     assert lib.hca_project_compress(fake, 64, 64 * 256, 0, 256, fake, fake, 64, None, fake, 1024, 1, 128, 64,

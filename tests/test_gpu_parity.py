@@ -22,7 +22,7 @@ from long_context_compressed_csa_b200 import (csa_attn_workspace_size, csa_compr
                                               csa_sparse_attn, csa_workspace_status, hca_compress,
                                               hca_dense_attn)
 from long_context_compressed_csa_b200.synth import randint_values, randn, to_f64
-from tests.helpers import check_topk_sets, decode_e4m3, max_rel_rowwise, score_error_bound
+from tests.helpers import check_topk_sets, decode_e2m1, decode_e4m3, max_rel_rowwise, score_error_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -616,6 +616,68 @@ def test_indexer_topk_e4m3(n_hI, cI, N_cap, k):
     # the workspace is left clean for the next call
     idx2 = torch.full((B, nq, k), -7, dtype=torch.int32, device=DEV)
     csa_indexer_topk_e4m3(dev(qI), dev(wI), codes, ksc, tt, m, k, idx2, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(np.sort(idx2.cpu().numpy(), axis=-1), np.sort(idx, axis=-1))
+
+
+@pytest.mark.parametrize("dtype,cols", [(torch.bfloat16, 128), (torch.float32, 256), (torch.bfloat16, 8)])
+def test_quantize_e2m1_matches_oracle_bit_exactly(dtype, cols):
+    """E2M1 codes (two per byte, even column in the low nibble) and fp32 row scales equal
+    the oracle's (both form x * (6 / max|x|) in fp32 and round to nearest even, saturating
+    at 6), including an all-zero row and a row of large values."""
+    from long_context_compressed_csa_b200 import csa_quantize_e2m1
+    X = randn((301, cols), 370, dtype, scale=3.0)
+    X[5] = 0
+    X[9] = X[9] * 1e4
+    codes = torch.empty((301, cols // 2), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((301,), dtype=torch.float32, device=DEV)
+    csa_quantize_e2m1(dev(X), codes, scales)
+    torch.cuda.synchronize()
+    want_v, want_s = oracle.quantize_rows_e2m1(X.float().numpy())
+    np.testing.assert_array_equal(scales.cpu().numpy().astype(np.float64), want_s)
+    np.testing.assert_array_equal(decode_e2m1(codes.cpu().numpy()), want_v)
+
+
+@pytest.mark.parametrize("n_hI,cI,N_cap,k", [(64, 128, 20000, 512), (32, 256, 3000, 1024), (16, 128, 700, 64)])
+def test_indexer_topk_e2m1(n_hI, cI, N_cap, k):
+    """Top-k over E2M1 keys and in-kernel E4M3 queries against the oracle's scores of the
+    GPU's decoded keys and the oracle-quantised queries (sets identical except for fp32
+    near-ties); the scores returned match within the fp32 rounding bound."""
+    from long_context_compressed_csa_b200 import csa_indexer_topk_e2m1, csa_quantize_e2m1
+    B, nq, m = 2, 2, 4
+    qI = randn((B, nq, n_hI, cI), 365, torch.bfloat16)
+    KI = randn((B, N_cap, cI), 366, torch.bfloat16)
+    wI = randn((B, nq, n_hI), 367, torch.float32)
+    codes = torch.empty((B, N_cap, cI // 2), dtype=torch.uint8, device=DEV)
+    ksc = torch.empty((B, N_cap), dtype=torch.float32, device=DEV)
+    csa_quantize_e2m1(dev(KI), codes, ksc)
+    t = [m * N_cap + 3, m * (N_cap // 3) + 1, m * (k // 2), 5]      # all, a third, fewer than k, t < m
+    tt = torch.tensor(t, dtype=torch.int64, device=DEV).reshape(B, nq)
+    ws = torch.zeros(csa_indexer_topk_workspace_size(B, nq, N_cap, k), dtype=torch.uint8, device=DEV)
+    idx = torch.full((B, nq, k), -7, dtype=torch.int32, device=DEV)
+    sc = torch.full((B, nq, k), float("nan"), dtype=torch.float32, device=DEV)
+    csa_indexer_topk_e2m1(dev(qI), dev(wI), codes, ksc, tt, m, k, idx, ws, scores_out=sc)
+    torch.cuda.synchronize()
+    assert csa_workspace_status(ws) == 0
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    codes_h, ksc_h = codes.cpu().numpy(), ksc.cpu().numpy().astype(np.float64)
+    for b in range(B):
+        K64 = decode_e2m1(codes_h[b]) * ksc_h[b][:, None]
+        kc, ks = oracle.quantize_rows_e2m1(KI[b].float().numpy())
+        np.testing.assert_array_equal(K64, kc * ks[:, None])  # the GPU's keys are the oracle's
+        for q in range(nq):
+            g = b * nq + q
+            vis = oracle.visible(t[g], m, N_cap)
+            qc, qs = oracle.quantize_rows_e4m3(qI[b, q].float().numpy())
+            q64, w64 = qc * qs[:, None], to_f64(wI[b, q])
+            s = oracle.index_scores(q64, w64, K64, vis)
+            check_topk_sets(idx[b, q], s, k, lambda d: score_error_bound(q64, w64, K64, d))
+            got = idx[b, q][idx[b, q] >= 0]
+            band = score_error_bound(q64, w64, K64, got) + 1e-6 * np.abs(s[got])
+            assert np.all(np.abs(sc[b, q][:len(got)] - s[got]) <= band)
+    # the workspace is left clean for the next call
+    idx2 = torch.full((B, nq, k), -7, dtype=torch.int32, device=DEV)
+    csa_indexer_topk_e2m1(dev(qI), dev(wI), codes, ksc, tt, m, k, idx2, ws)
     torch.cuda.synchronize()
     assert np.array_equal(np.sort(idx2.cpu().numpy(), axis=-1), np.sort(idx, axis=-1))
 
