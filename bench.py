@@ -145,7 +145,10 @@ class HybridDecode:
         self.n, self.m, self.mp, self.c, self.cI = n, 4, 128, 512, 128
         self.n_h, self.n_hI, self.k = 128, 64, 1024
         self.dev = device
-        self.e4m3 = kI_format == "e4m3"  # indexer keys as E4M3 codes + one fp32 scale per key
+        # indexer keys as E4M3 (one byte) or E2M1 (half a byte) codes + one fp32 scale per key
+        self.kfmt = kI_format
+        self.e4m3, self.e2m1 = kI_format == "e4m3", kI_format == "e2m1"
+        self.quant = self.e4m3 or self.e2m1
         bf16 = torch.bfloat16
         self.tokens = (steps_total + N_PAIRS - 1) // N_PAIRS + 1
         T = self.tokens
@@ -166,10 +169,11 @@ class HybridDecode:
             P["hcache"] = torch.empty((1, self.Nh_cap, c), dtype=bf16, device=device)
             # prefill compress through the library (streams generated in slices)
             self._prefill(P, s)
-            if self.e4m3:  # quantise the prefill keys once; the bf16 cache stays the staging of new keys
-                P["kI8"] = torch.zeros((1, self.N_cap, cI), dtype=torch.uint8, device=device)
+            if self.quant:  # quantise the prefill keys once; the bf16 cache stays the staging of new keys
+                P["kI8"] = torch.zeros((1, self.N_cap, cI if self.e4m3 else cI // 2), dtype=torch.uint8,
+                                       device=device)
                 P["kIs"] = torch.zeros((1, self.N_cap), dtype=torch.float32, device=device)
-                lib.csa_quantize_e4m3(P["kI"][:, :self.N], P["kI8"][:, :self.N], P["kIs"][:, :self.N])
+                self._quantize(P, 0, self.N)
             # decode-time stream rows, one interleaved row per token (the 4 CSA streams, the
             # 4 indexer-key streams, the 2 HCA streams), so that a token's new rows are one
             # contiguous copy: tokens n - hist .. n + T - 1 (CSA), n .. n + T - 1 (HCA)
@@ -234,6 +238,8 @@ class HybridDecode:
         if part in (None, 0):
             if self.e4m3:
                 lib.csa_indexer_topk_e4m3(qI, wI, P["kI8"], P["kIs"], t, self.m, self.k, self.idx, self.ws_topk)
+            elif self.e2m1:
+                lib.csa_indexer_topk_e2m1(qI, wI, P["kI8"], P["kIs"], t, self.m, self.k, self.idx, self.ws_topk)
             else:
                 lib.csa_indexer_topk(qI, wI, P["kI"], t, self.m, self.k, self.idx, self.ws_topk)
         if part == 0:
@@ -249,8 +255,8 @@ class HybridDecode:
             lib.csa_compress(*win, P["cache"], self.m, i, i + 1, tok0=lo)
             winI = [x[:, r0:r0 + 2 * self.m] for x in P["decI"]]
             lib.csa_compress(*winI, P["kI"], self.m, i, i + 1, tok0=lo)
-            if self.e4m3:  # the new key, quantised as it is formed
-                lib.csa_quantize_e4m3(P["kI"][:, i:i + 1], P["kI8"][:, i:i + 1], P["kIs"][:, i:i + 1])
+            if self.quant:  # the new key, quantised as it is formed
+                self._quantize(P, i, i + 1)
         if (tok + 1) % self.mp == 0:
             i = (tok + 1) // self.mp - 1
             lo = self.mp * i
@@ -258,13 +264,21 @@ class HybridDecode:
             lib.hca_compress(P["decH"][0][:, r0:r0 + self.mp], P["decH"][1][:, r0:r0 + self.mp],
                              P["hcache"], self.mp, i, i + 1, tok0=lo)
 
+    def _quantize(self, P, lo, hi):
+        f = self.lib.csa_quantize_e4m3 if self.e4m3 else self.lib.csa_quantize_e2m1
+        f(P["kI"][:, lo:hi], P["kI8"][:, lo:hi], P["kIs"][:, lo:hi])
+
+    def key_bytes(self):
+        """HBM bytes of one indexer key as the scan reads it (codes + scale)."""
+        return self.cI + 4 if self.e4m3 else self.cI // 2 + 4 if self.e2m1 else self.cI * 2
+
     def step_bytes(self, j):
         """Algorithmic HBM bytes of step j: indexer keys scanned + selected entries +
         HCA entries read (+ the stream rows and entries of any compression)."""
         tok = self.n + j
         vis = tok // self.m
         visH = tok // self.mp
-        b = vis * (self.cI + 4 if self.e4m3 else self.cI * 2) + self.k * self.c * 2 + visH * self.c * 2
+        b = vis * self.key_bytes() + self.k * self.c * 2 + visH * self.c * 2
         if (tok + 1) % self.m == 0:
             b += 4 * 2 * self.m * (self.c + self.cI) * 2 + (self.c + self.cI) * 2
         if (tok + 1) % self.mp == 0:
@@ -276,7 +290,7 @@ def kernel_launches_per_step(dec, j):
     tok = dec.n + j
     n = 1 + 2 + 2  # indexer (scan with the select in place), sparse attn (+combine), dense attn (+combine)
     if (tok + 1) % dec.m == 0:
-        n += 3 if dec.e4m3 else 2
+        n += 3 if dec.quant else 2
     if (tok + 1) % dec.mp == 0:
         n += 1
     return n
@@ -313,7 +327,8 @@ def _oracle_step(workload, x, j, kI_format="bf16"):
     import oracle
     if workload == "hybrid_1m_decode":
         t = (1 << 20) + j
-        score = oracle.index_scores_e4m3 if kI_format == "e4m3" else oracle.index_scores
+        score = {"e4m3": oracle.index_scores_e4m3, "e2m1": oracle.index_scores_e2m1}.get(kI_format,
+                                                                                         oracle.index_scores)
         s = score(x["qI"], x["wI"], x["KI"], oracle.visible(t, 4, x["KI"].shape[0]))
         sel = oracle.topk(s, 1024)
         oracle.mqa(x["q"], x["rows"][sel % x["rows"].shape[0]], np.arange(1024, dtype=np.int32))
@@ -366,7 +381,7 @@ def cpu_baseline(workload="hybrid_1m_decode", seed=77, steps=None, kI_format="bf
     unit = "layer-pair decode steps/s" if workload == "hybrid_1m_decode" else "decode tokens/s"
     what = {"hybrid_1m_decode": "one CSA+HCA layer pair at t=2^20 (indexer over 262144 %skeys, full-sort "
                                 "top-1024, 128-head MQA over 1024 + 8192 entries)"
-                                % ("E4M3-quantised " if kI_format == "e4m3" else ""),
+                                % ({"e4m3": "E4M3-quantised ", "e2m1": "E2M1-quantised "}.get(kI_format, "")),
             "csa_decode_8k": "one CSA layer at t=8192 (indexer over 2048 keys, top-512, 128-head MQA "
                              "over 512 entries)",
             "hca_decode_b16_128k": "one sequence's HCA dense MQA at t=131072 (128 heads over 1024 entries)",
@@ -455,6 +470,20 @@ def micro(kind, iters, rotate=4, nq_prefill=1024, batch=16):
         calls = [lambda r=r: lib.csa_indexer_topk_e4m3(qI, wI, K8s[r], KSs[r], t, m, k, idx, ws)
                  for r in range(rotate)]
         nbytes = N * (cI + 4)
+    elif kind == "indexer_e2m1":
+        # the same scan and top-k over E2M1 keys (half a byte per element + one fp32 scale per key)
+        KIs = [randn((1, N, cI), 900 + r, bf16, dev) for r in range(rotate)]
+        K4s = [torch.empty((1, N, cI // 2), dtype=torch.uint8, device=dev) for _ in range(rotate)]
+        KSs = [torch.empty((1, N), dtype=torch.float32, device=dev) for _ in range(rotate)]
+        for r in range(rotate):
+            lib.csa_quantize_e2m1(KIs[r], K4s[r], KSs[r])
+        del KIs
+        qI, wI = randn((1, 1, n_hI, cI), 890, bf16, dev), randn((1, 1, n_hI), 891, torch.float32, dev)
+        idx = torch.empty((1, 1, k), dtype=torch.int32, device=dev)
+        ws = torch.zeros(lib.csa_indexer_topk_workspace_size(1, 1, N, k), dtype=torch.uint8, device=dev)
+        calls = [lambda r=r: lib.csa_indexer_topk_e2m1(qI, wI, K4s[r], KSs[r], t, m, k, idx, ws)
+                 for r in range(rotate)]
+        nbytes = N * (cI // 2 + 4)
     elif kind in ("sparse_window", "dense_window"):
         # the same calls with the sliding-window branch: 128 raw-token entries from a ring
         # buffer join the softmax (V4-Pro window size)
@@ -808,13 +837,13 @@ def main():
                     choices=["hybrid_1m_decode", "csa_decode_8k", "hca_decode_b16_128k",
                              "csa_prefill_decode_b4_256k"],
                     help="the configuration timed (default: the 1M-token hybrid decode)")
-    ap.add_argument("--kI-format", default="bf16", choices=["bf16", "e4m3"],
-                    help="indexer keys of the hybrid decode: bf16 (default) or E4M3 codes with one fp32 "
-                         "scale per key, every appended key quantised as it is formed")
+    ap.add_argument("--kI-format", default="bf16", choices=["bf16", "e4m3", "e2m1"],
+                    help="indexer keys of the hybrid decode: bf16 (default), E4M3 or E2M1 codes with one "
+                         "fp32 scale per key, every appended key quantised as it is formed")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--micro", default=None,
-                    help="time one entry point alone: indexer, indexer_e4m3, indexer_prefill, "
+                    help="time one entry point alone: indexer, indexer_e4m3, indexer_e2m1, indexer_prefill, "
                          "sparse, sparse_prefill, dense, sparse_window, dense_window, csa_compress, "
                          "hca_compress, hca_project_compress, csa_project_compress")
     ap.add_argument("--nq", type=int, default=1024,
@@ -944,7 +973,7 @@ def main():
     # back to back over the 8 layer pairs' keys at the first timed token position ----
     j0 = W // N_PAIRS
     vis = (dec.n + j0) // dec.m
-    idx_bytes = vis * (dec.cI + 4 if dec.e4m3 else dec.cI * 2)
+    idx_bytes = vis * dec.key_bytes()
     t_idx = back_to_back_launch_us(
         torch, [lambda p=p: dec.step(p, j0, part=0) for _ in range(8) for p in range(N_PAIRS)], reps=8)
     log("indexer+topk per launch: back to back mean %.2f us, median %.2f us; in the step (event nodes) "
@@ -958,8 +987,8 @@ def main():
         e2e = run_e2e(torch, dec, W, min(K, 512), world)
 
     roof = roofline_obj("csa_indexer_topk%s (scan_tc_kernel: indexer scan with the top-k select in place)"
-                        % ("_e4m3" if dec.e4m3 else ""), idx_bytes, t_idx, hbm, src,
-                        None if dec.e4m3 else SCAN_TRAFFIC_BYTES, HOW_B2B % (64, 8))
+                        % ("" if not dec.quant else "_" + dec.kfmt), idx_bytes, t_idx, hbm, src,
+                        None if dec.quant else SCAN_TRAFFIC_BYTES, HOW_B2B % (64, 8))
     roof["in_step_event_nodes_us_mean"] = float(idx_ms.mean() * 1e3)
     roof["in_step_event_nodes_samples"] = int(len(idx_ms))
     line = {

@@ -709,22 +709,28 @@ def test_indexer_wait_timeout_is_reported_then_cleared():
     check_topk_sets(idx[0, 0], s, k, lambda d: score_error_bound(q64, w64, K64, d))
 
 
-def test_e4m3_key_cache_decode_loop():
-    """A CSA decode loop whose indexer keys live as E4M3 codes with one fp32 scale per key:
-    the prefill keys are quantised once, and each key appended at a block end is formed
-    by csa_compress (bf16) and quantised by csa_quantize_e4m3 as it is formed.  Stage-wise
-    checks at every step: each new key's codes and scale are bit-exact against the
-    oracle's quantisation of the GPU's bf16 key, and the step's top-k set matches the
-    oracle's scores of the GPU's decoded keys and the oracle-quantised query (near-ties
-    within the fp32 rounding bound plus 1e-6 relative)."""
-    from long_context_compressed_csa_b200 import csa_quantize_e4m3 as quant
+@pytest.mark.parametrize("fmt", ["e4m3", "e2m1"])
+def test_low_precision_key_cache_decode_loop(fmt):
+    """A CSA decode loop whose indexer keys live as E4M3 (one byte) or E2M1 (half a byte)
+    codes with one fp32 scale per key: the prefill keys are quantised once, and each key
+    appended at a block end is formed by csa_compress (bf16) and quantised as it is
+    formed.  Stage-wise checks at every step: each new key's codes and scale are
+    bit-exact against the oracle's quantisation of the GPU's bf16 key, and the step's
+    top-k set matches the oracle's scores of the GPU's decoded keys and the
+    oracle-quantised query (near-ties within the fp32 rounding bound plus 1e-6
+    relative)."""
+    import long_context_compressed_csa_b200 as lib
+    quant = lib.csa_quantize_e4m3 if fmt == "e4m3" else lib.csa_quantize_e2m1
+    topk = lib.csa_indexer_topk_e4m3 if fmt == "e4m3" else lib.csa_indexer_topk_e2m1
+    decode = decode_e4m3 if fmt == "e4m3" else decode_e2m1
+    oquant = oracle.quantize_rows_e4m3 if fmt == "e4m3" else oracle.quantize_rows_e2m1
     B, m, cI, n_hI, k, N0, steps = 1, 4, 128, 64, 256, 3000, 13
     n0 = m * N0
     N_cap = N0 + steps // m + 2
     SI = [randn((B, n0 + steps, cI), 380 + i, torch.bfloat16) for i in range(4)]
     SId = [dev(x) for x in SI]
     kI = torch.empty((B, N_cap, cI), dtype=torch.bfloat16, device=DEV)
-    K8 = torch.zeros((B, N_cap, cI), dtype=torch.uint8, device=DEV)
+    K8 = torch.zeros((B, N_cap, cI if fmt == "e4m3" else cI // 2), dtype=torch.uint8, device=DEV)
     KS = torch.zeros((B, N_cap), dtype=torch.float32, device=DEV)
     csa_compress(*(x[:, :n0] for x in SId), kI, m, 0, N0)
     quant(kI[:, :N0], K8[:, :N0], KS[:, :N0])
@@ -735,11 +741,11 @@ def test_e4m3_key_cache_decode_loop():
         wI = randn((B, 1, n_hI), 400 + j, torch.float32)
         idx = torch.full((B, 1, k), -7, dtype=torch.int32, device=DEV)
         tt = torch.tensor([[t]], dtype=torch.int64, device=DEV)
-        csa_indexer_topk_e4m3(dev(qI), dev(wI), K8, KS, tt, m, k, idx, ws)
+        topk(dev(qI), dev(wI), K8, KS, tt, m, k, idx, ws)
         torch.cuda.synchronize()
         assert csa_workspace_status(ws) == 0
         vis = oracle.visible(t, m, N_cap)
-        K64 = decode_e4m3(K8[0, :vis].cpu().numpy()) * KS[0, :vis].cpu().numpy().astype(np.float64)[:, None]
+        K64 = decode(K8[0, :vis].cpu().numpy()) * KS[0, :vis].cpu().numpy().astype(np.float64)[:, None]
         qc, qs = oracle.quantize_rows_e4m3(qI[0, 0].float().numpy())
         q64, w64 = qc * qs[:, None], to_f64(wI[0, 0])
         s = oracle.index_scores(q64, w64, K64, vis)
@@ -750,8 +756,8 @@ def test_e4m3_key_cache_decode_loop():
             csa_compress(*(x[:, lo:lo + 2 * m] for x in SId), kI, m, i, i + 1, tok0=lo)
             quant(kI[:, i:i + 1], K8[:, i:i + 1], KS[:, i:i + 1])
             torch.cuda.synchronize()
-            rc, rs = oracle.quantize_rows_e4m3(kI[0, i].float().cpu().numpy())
-            np.testing.assert_array_equal(decode_e4m3(K8[0, i].cpu().numpy()), rc)
+            rc, rs = oquant(kI[0, i].float().cpu().numpy())
+            np.testing.assert_array_equal(decode(K8[0, i].cpu().numpy()), rc)
             assert KS[0, i].item() == np.float32(rs)
 
 
