@@ -19,6 +19,14 @@
 // q^I (the B operand) is staged once per CTA into the same swizzled layout.  Each CTA
 // walks a strided set of key tiles of one query.  Every barrier wait is bounded; a
 // timeout sets the workspace status word and every role drains and exits.
+//
+// Key formats: bf16 (kind::f16); E4M3 codes (kind::f8f6f4, q^I quantised per head to
+// E4M3 by the epilogue warps, the key's fp32 scale applied to the score); E2M1 codes,
+// two per byte in global memory, which the TMA unpacks into the 16-bytes-per-16-codes
+// layout of an E2M1 operand, so the tiles, swizzle and descriptors are the E4M3 ones.
+//
+// When the query's grid fits in one wave, the same kernel then selects the top k in
+// place (section 7): see the in-place top-k below.
 #include "indexer.cuh"
 #include "e4m3.cuh"
 #include "select.cuh"
