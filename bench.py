@@ -342,9 +342,14 @@ def _oracle_step(workload, x, j, kI_format="bf16"):
         oracle.mqa(x["q"], x["hc"], np.arange(1024, dtype=np.int32))
 
 
-def _oracle_worker(workload, seed, steps, barrier, queue, kI_format="bf16"):
+def _oracle_worker(workload, seed, steps, barrier, queue, kI_format="bf16", warmup=1, budget_s=None):
     x = _oracle_inputs(workload, seed)
-    _oracle_step(workload, x, 0, kI_format)  # warm: loads the oracle library
+    t_w = time.monotonic()
+    for j in range(max(1, warmup)):  # warm: loads the oracle library (untimed)
+        _oracle_step(workload, x, -1 - j, kI_format)
+    per_step = (time.monotonic() - t_w) / max(1, warmup)
+    if budget_s is not None:  # a bounded sample: as many of the steps as fit the budget
+        steps = max(1, min(steps, int(budget_s / max(per_step, 1e-9))))
     barrier.wait()
     t0 = time.monotonic()
     for j in range(steps):
@@ -358,18 +363,24 @@ ORACLE_STEPS = {"hybrid_1m_decode": 1, "csa_decode_8k": 20, "hca_decode_b16_128k
 ORACLE_MAX_WORKERS = 16
 
 
-def cpu_baseline(workload="hybrid_1m_decode", seed=77, steps=None, kI_format="bf16"):
+def cpu_baseline(workload="hybrid_1m_decode", seed=77, steps=None, kI_format="bf16", warmup=1, total=None,
+                 budget_s=None):
     """The oracle timed on the host's cores: one spawned process per core (at most
     ORACLE_MAX_WORKERS), each running whole decode steps of its own sequence after a
     common barrier; value = all steps / the wall time of the concurrent region, in the
-    workload's unit (a layer-pair step of the hybrid workload is one token)."""
+    workload's unit (a layer-pair step of the hybrid workload is one token).  With
+    `total`, the processes share that many steps; with `budget_s`, each runs at most the
+    steps that fit that many seconds (measured on its warm-up steps)."""
     import multiprocessing as mp_
     host = len(os.sched_getaffinity(0))
     P = max(1, min(host, ORACLE_MAX_WORKERS))
     steps = steps or ORACLE_STEPS[workload]
+    if total is not None:
+        steps = max(1, -(-total // P))
     ctx = mp_.get_context("spawn")  # never fork a process that has touched the GPU
     barrier, queue = ctx.Barrier(P), ctx.Queue()
-    procs = [ctx.Process(target=_oracle_worker, args=(workload, seed + 1000 * w, steps, barrier, queue, kI_format))
+    procs = [ctx.Process(target=_oracle_worker, args=(workload, seed + 1000 * w, steps, barrier, queue, kI_format,
+                                                      warmup, budget_s))
              for w in range(P)]
     for pr in procs:
         pr.start()
@@ -377,7 +388,6 @@ def cpu_baseline(workload="hybrid_1m_decode", seed=77, steps=None, kI_format="bf
     for pr in procs:
         pr.join()
     wall = max(r[1] for r in res) - min(r[0] for r in res)
-    total = sum(r[2] for r in res)
     unit = "layer-pair decode steps/s" if workload == "hybrid_1m_decode" else "decode tokens/s"
     what = {"hybrid_1m_decode": "one CSA+HCA layer pair at t=2^20 (indexer over 262144 %skeys, full-sort "
                                 "top-1024, 128-head MQA over 1024 + 8192 entries)"
@@ -387,10 +397,12 @@ def cpu_baseline(workload="hybrid_1m_decode", seed=77, steps=None, kI_format="bf
             "hca_decode_b16_128k": "one sequence's HCA dense MQA at t=131072 (128 heads over 1024 entries)",
             "csa_prefill_decode_b4_256k": "one sequence's CSA step at t=262144 (indexer over 65536 keys, "
                                           "top-1024, 128-head MQA over 1024 entries)"}[workload]
-    return {"value": total / wall, "unit": unit, "cores": P, "host_cores": host, "kind": "oracle",
+    done = sum(r[2] for r in res)
+    return {"value": done / wall, "unit": unit, "cores": P, "host_cores": host, "kind": "oracle",
             "sample": "%d processes x %d decode steps of %s, fp64 oracle, one process per core"
-                      % (P, steps, what),
-            "seconds": wall}
+                      % (P, -(-done // P), what) + ("" if budget_s is None else
+                                                     " (at most %.0f s of steps per process)" % budget_s),
+            "seconds": wall, "steps_done": done}
 
 
 # ----------------------------------------------------------------------------------
@@ -865,10 +877,14 @@ def main():
             return 0
         import oracle
         oracle.build()
-        base = cpu_baseline(args.workload, kI_format=args.kI_format)
+        # the K timed steps are shared by the host processes (each on its own sequence),
+        # after at most 2 untimed steps each; every process stops at ~90 s of steps, so a
+        # run with the default K still ends within a few minutes
+        base = cpu_baseline(args.workload, kI_format=args.kI_format, warmup=min(2, max(1, args.warmup)),
+                            total=max(1, args.steps), budget_s=90.0)
         cfg = workload_config(args.gpus, args.kI_format) if args.workload == WORKLOAD else preset_config(args.workload)
         line = {"impl": "reference", "metric": METRIC, "value": base["value"], "unit": base["unit"],
-                "n_gpus": args.gpus, "steps": base["cores"] * ORACLE_STEPS[args.workload], "warmup": 0,
+                "n_gpus": args.gpus, "steps": base["steps_done"], "warmup": min(2, max(1, args.warmup)),
                 "ms_per_step": 1000.0 / base["value"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": cfg,
