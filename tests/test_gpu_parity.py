@@ -340,6 +340,37 @@ def test_indexer_topk_exact_on_integer_inputs(dtype, n_hI, cI):
         assert sorted(idx2.reshape(-1, k)[g].tolist()) == sorted(idx.reshape(-1, k)[g].tolist())
 
 
+def test_indexer_topk_mixed_select_paths_in_one_launch():
+    """Two queries of one launch whose threshold bins differ in width: the first (0/1
+    query, unit weights) crowds ~4800 keys into its threshold bin and is resolved digit
+    by digit by one CTA, the second (random bf16) ranks its ~1100 candidates in every
+    CTA.  Both sets must equal the oracle's except for fp32 near-ties, and a second call
+    on the same workspace must repeat them."""
+    B, nq, n_hI, cI, N_cap, m, k = 1, 2, 64, 128, 30000, 4, 4000
+    qI = randint_values((B, nq, n_hI, cI), 270, 0, 2, torch.bfloat16)
+    qI[0, 1] = randn((n_hI, cI), 275, torch.bfloat16)
+    KI = randint_values((B, N_cap, cI), 271, 0, 2, torch.bfloat16)
+    KI[0, :, :64] += randn((N_cap, 64), 276, torch.bfloat16, scale=1.0)   # spread for query 1
+    KI = KI.to(torch.bfloat16)
+    wI = torch.ones((B, nq, n_hI), dtype=torch.float32)
+    wI[0, 1] = randn((n_hI,), 277, torch.float32)
+    t = [4 * N_cap, 4 * N_cap]
+    idx, sc, ws = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k)
+    widths = []
+    for q in range(nq):
+        q64, w64, K64 = to_f64(qI[0, q]), to_f64(wI[0, q]), to_f64(KI[0])
+        s = oracle.index_scores(q64, w64, K64, N_cap)
+        want = oracle.topk(s, k)
+        u = s.astype(np.float32).view(np.uint32)
+        d0 = np.where(u >> 31, ~u, u | np.uint32(0x80000000)) >> 20
+        widths.append(int(np.sum(d0 == d0[want[k - 1]])))
+        check_topk_sets(idx[0, q], s, k, lambda d: score_error_bound(q64, w64, K64, d))
+    assert widths[0] > 4096 >= widths[1]  # one query on each select path
+    idx2, _, _ = run_indexer(dev(qI), dev(wI), dev(KI), t, m, k, ws=ws)
+    for q in range(nq):
+        assert sorted(idx2[0, q].tolist()) == sorted(idx[0, q].tolist())
+
+
 @pytest.mark.parametrize("k,N_cap,run", [(200, 40000, 300), (1024, 262144, 2048)])
 def test_indexer_topk_clustered_top_keys(k, N_cap, run):
     """The top keys crowd into a few consecutive key tiles (a run of keys scaled by 3, so
