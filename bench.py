@@ -35,9 +35,10 @@ METRIC = "CSA/HCA decode tokens/s at 128K–1M ctx; achieved HBM GB/s vs ~8 TB/s
 WORKLOAD = "hybrid_1m_decode"
 N_PAIRS = 8
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one scan_tc_kernel launch
-# over 262144 keys, from one ncu capture of the current kernel (67.21 MB read, 0.73 MB
-# written; algorithmic 67.11 MB).  Must be retaken (or set to None) when the kernel changes.
-SCAN_TRAFFIC_BYTES = 67_941_888
+# over 262144 keys, per key format, from one ncu capture of the current kernel each: bf16
+# 67.21 MB read + 0.73 MB written (algorithmic 67.11 MB), E4M3 34.70 MB read (34.60 MB),
+# E2M1 17.93 MB read (17.83 MB).  Must be retaken (or set to None) when the kernel changes.
+SCAN_TRAFFIC_BYTES = {"bf16": 67_941_888, "e4m3": 34_704_640, "e2m1": 17_926_912}
 IDX_SAMPLE = 8  # steps per CUDA graph; the indexer call of each graph's first step is timed
 
 
@@ -1004,7 +1005,7 @@ def main():
 
     roof = roofline_obj("csa_indexer_topk%s (scan_tc_kernel: indexer scan with the top-k select in place)"
                         % ("" if not dec.quant else "_" + dec.kfmt), idx_bytes, t_idx, hbm, src,
-                        None if dec.quant else SCAN_TRAFFIC_BYTES, HOW_B2B % (64, 8))
+                        SCAN_TRAFFIC_BYTES.get(dec.kfmt), HOW_B2B % (64, 8))
     roof["in_step_event_nodes_us_mean"] = float(idx_ms.mean() * 1e3)
     roof["in_step_event_nodes_samples"] = int(len(idx_ms))
     line = {
