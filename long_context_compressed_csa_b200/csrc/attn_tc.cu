@@ -64,7 +64,9 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_const
                   const __grid_constant__ CUtensorMap tmap_w, AttnArgs a, uint32_t* status)
 {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned; an offset from the __shared__ array keeps every derived pointer in
+    // the shared window, so its accesses compile to shared-memory instructions
+    uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sQ = smem;
     uint8_t* sC0 = sQ + kQBytes;                      // chunk buffer b at sC0 + b * kCBytes
     uint8_t* sP = sC0 + 2 * kCBytes;

@@ -248,7 +248,9 @@ stream_pool_kernel(const __grid_constant__ CUtensorMap t0, const __grid_constant
     constexpr int kStreamBytes = kRows * kSpCols * 2;
     constexpr float kL2e = 1.4426950408889634f;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    // 128-byte aligned; an offset from the __shared__ array keeps derived pointers in the
+    // shared window (shared-memory instructions)
+    uint8_t* smem = smem_raw + ((128u - (tc::smem_u32(smem_raw) & 127u)) & 127u);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kSpStages * kSpStageBytes);
     uint64_t* empty = full + kSpStages;
     volatile uint32_t* abort_flag = reinterpret_cast<uint32_t*>(empty + kSpStages);

@@ -124,7 +124,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tmap, const void* __restrict_
     using Cfg = ScanCfg<NH, CI, KB>;
     constexpr int S = Cfg::kStages;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned; an offset from the __shared__ array keeps every derived pointer in
+    // the shared window, so its accesses compile to shared-memory instructions
+    uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sA = smem;
     uint8_t* sB = sA + S * Cfg::kAStage;
     float* s_sc = reinterpret_cast<float*>(sB + Cfg::kBBytes);  // [kCacheTiles * 128] own scores

@@ -105,7 +105,9 @@ hca_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __
                             const __grid_constant__ CUtensorMap tmap_wz, PcArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned; an offset from the __shared__ array keeps every derived pointer in
+    // the shared window, so its accesses compile to shared-memory instructions
+    uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPcStages * kPcStage);
     uint64_t* empty = full + kPcStages;
     uint64_t* tfull = empty + kPcStages;   // MMA -> epilogue: the tile's accumulators are complete
@@ -405,7 +407,9 @@ csa_project_compress_kernel(const __grid_constant__ CUtensorMap tmap_h, const __
                             const __grid_constant__ CUtensorMap tmap_wb_z, CsArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned; an offset from the __shared__ array keeps every derived pointer in
+    // the shared window, so its accesses compile to shared-memory instructions
+    uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kCsStages * kCsStage);  // leader's are used
     uint64_t* empty = full + kCsStages;    // each CTA's: its stage may be overwritten
     uint64_t* tfull = empty + kCsStages;   // each CTA's: the pass's accumulators are complete
