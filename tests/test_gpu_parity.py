@@ -713,6 +713,43 @@ def test_indexer_topk_e2m1(n_hI, cI, N_cap, k):
     assert np.array_equal(np.sort(idx2.cpu().numpy(), axis=-1), np.sort(idx, axis=-1))
 
 
+@pytest.mark.parametrize("fmt", ["e4m3", "e2m1"])
+def test_low_precision_indexer_many_queries(fmt):
+    """More queries than resident CTAs (200 > 148): the low-precision scan writes the
+    scores to the workspace and the stand-alone select follows.  Sets and scores against
+    the oracle on the GPU's decoded keys and the oracle-quantised queries."""
+    import long_context_compressed_csa_b200 as lib
+    quant = lib.csa_quantize_e4m3 if fmt == "e4m3" else lib.csa_quantize_e2m1
+    topk = lib.csa_indexer_topk_e4m3 if fmt == "e4m3" else lib.csa_indexer_topk_e2m1
+    decode = decode_e4m3 if fmt == "e4m3" else decode_e2m1
+    B, nq, n_hI, cI, N_cap, m, k = 1, 200, 64, 128, 2000, 4, 100
+    qI = randn((B, nq, n_hI, cI), 385, torch.bfloat16)
+    KI = randn((B, N_cap, cI), 386, torch.bfloat16)
+    wI = randn((B, nq, n_hI), 387, torch.float32)
+    codes = torch.empty((B, N_cap, cI if fmt == "e4m3" else cI // 2), dtype=torch.uint8, device=DEV)
+    ksc = torch.empty((B, N_cap), dtype=torch.float32, device=DEV)
+    quant(dev(KI), codes, ksc)
+    t = [m * (N_cap // 2) + 4 * q for q in range(nq)]  # visible counts 1000 .. 1199
+    tt = torch.tensor(t, dtype=torch.int64, device=DEV).reshape(B, nq)
+    ws = torch.zeros(csa_indexer_topk_workspace_size(B, nq, N_cap, k), dtype=torch.uint8, device=DEV)
+    idx = torch.full((B, nq, k), -7, dtype=torch.int32, device=DEV)
+    sc = torch.full((B, nq, k), float("nan"), dtype=torch.float32, device=DEV)
+    topk(dev(qI), dev(wI), codes, ksc, tt, m, k, idx, ws, scores_out=sc)
+    torch.cuda.synchronize()
+    assert csa_workspace_status(ws) == 0
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    K64 = decode(codes[0].cpu().numpy()) * ksc[0].cpu().numpy().astype(np.float64)[:, None]
+    for q in (0, 57, 123, 199):
+        vis = oracle.visible(t[q], m, N_cap)
+        qc, qs = oracle.quantize_rows_e4m3(qI[0, q].float().numpy())
+        q64, w64 = qc * qs[:, None], to_f64(wI[0, q])
+        s = oracle.index_scores(q64, w64, K64, vis)
+        check_topk_sets(idx[0, q], s, k, lambda d: score_error_bound(q64, w64, K64, d))
+        got = idx[0, q]
+        band = score_error_bound(q64, w64, K64, got) + 1e-6 * np.abs(s[got])
+        assert np.all(np.abs(sc[0, q] - s[got]) <= band)
+
+
 def test_indexer_wait_timeout_is_reported_then_cleared():
     """Failure detection without a GPU fault: a wait budget of a few cycles for the grid
     meeting of the in-place top-k (the workspace's test hook) makes that bounded wait run
