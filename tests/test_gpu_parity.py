@@ -940,6 +940,32 @@ def test_dense_attn_random(dtype, n_h, c):
                                    rtol=0)
 
 
+@pytest.mark.parametrize("B,N_cap,vis", [
+    (1, 200, [75]),                                          # one 32-entry chunk per split
+    (8, 2048, [2048, 1000, 700, 64, 63, 0, 130, 1]),         # CTA pairs, four 64-entry chunks per split
+])
+def test_dense_attn_ignores_rows_past_visible(B, N_cap, vis):
+    """Cache rows at or past the visible count hold NaN: a split whose range the count cuts
+    (a partial chunk), or that lies past it, must neither read them into the output nor
+    leave them in shared memory for the products."""
+    n_h, c, mp = 128, 512, 128
+    q = randn((B, 1, n_h, c), 480, torch.bfloat16)
+    cache = randn((B, N_cap, c), 481, torch.bfloat16)
+    for b, v in enumerate(vis):
+        cache[b, v:] = float("nan")
+    t = [mp * v + (b * 37) % mp for b, v in enumerate(vis)]
+    o, lse = run_dense(dev(q), dev(cache), t, mp)
+    for b, v in enumerate(vis):
+        assert oracle.visible(t[b], mp, N_cap) == v
+        if v == 0:
+            assert np.all(o[b, 0] == 0) and np.all(np.isneginf(lse[b, 0]))
+            continue
+        ref, ref_lse = _ref_attn(to_f64(q[b, 0]), to_f64(cache[b]), np.arange(v, dtype=np.int32))
+        assert np.all(np.isfinite(o[b, 0]))
+        assert max_rel_rowwise(o[b, 0], ref).max() <= TOL[torch.bfloat16]
+        np.testing.assert_allclose(lse[b, 0], ref_lse, atol=2e-3, rtol=0)
+
+
 def test_attn_many_queries_and_workspace_reuse():
     """80 queries of 128 heads in one call (one CTA pair per query, padding inside one
     list); then one dense workspace reused across calls whose visible counts, hence split
