@@ -193,6 +193,101 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(PoolArgs p)
     }
 }
 
+// Decode-sized calls (at most one wave of entries): one CTA per (entry, batch row).
+// pool_kernel gives a thread one column group and walks the 2m (or m') candidate rows in
+// dependent batches of kUnroll; at a block end of a decode that chain of round trips is
+// the whole cost.  Here the candidate rows are fetched into L2 before the dependency wait,
+// the whole CTA loads a chunk of up to kSmallChunk candidates at once (logits with their
+// bias, and values, as fp32 into shared memory), and one thread per column folds the
+// chunk's candidates, in pool_kernel's order, into the same online softmax: the result
+// is bit-identical to pool_kernel's.
+constexpr int kSmallChunk = 32;             // candidates per chunk
+constexpr int kSmallSmem = 160 * 1024;      // shared-memory bound of a chunk: [chunk][c] x 2 fp32
+constexpr int kSmallItems = 4;              // (candidate, column group) loads per thread per round
+
+template <typename T, int V>
+__global__ void __launch_bounds__(1024, 1) pool_small_kernel(PoolArgs p, int chunk)
+{
+    pdl_launch_dependents();
+    extern __shared__ float s_zx[];         // [chunk][c] logits (bias added), then [chunk][c] values
+    const int64_t i = p.e0 + blockIdx.x;    // entry
+    const int64_t b = blockIdx.y;           // batch row
+    const int c = p.c, vecs = c / V;
+    const int ncand = p.has_b && i > 0 ? 2 * p.m : p.m;
+    const int64_t ra = (int64_t)p.m * i - p.tok0;        // first a-row of block i
+    const int64_t rb = (int64_t)p.m * (i - 1) - p.tok0;  // block i-1 via stream b
+    const int64_t boff = b * p.ld_batch;
+    // candidate q: a-row q for q < m, then b-row q - m (pool_kernel's order)
+    auto row_of = [&](const void* sa, const void* sb, int q) -> const T* {
+        return q < p.m ? static_cast<const T*>(sa) + boff + (ra + q) * p.ld_row
+                       : static_cast<const T*>(sb) + boff + (rb + q - p.m) * p.ld_row;
+    };
+    if constexpr (V * sizeof(T) == 16) {
+        // whole rows into L2 while the previous kernel finishes (16-byte aligned rows of
+        // c * sizeof(T) bytes, a multiple of 16, on this path)
+        for (int u = threadIdx.x; u < 2 * ncand; u += blockDim.x)
+            tc::prefetch_l2(u & 1 ? row_of(p.Xa, p.Xb, u >> 1) : row_of(p.Za, p.Zb, u >> 1), (uint32_t)(c * sizeof(T)));
+    }
+    pdl_wait();
+    float* sz = s_zx;
+    float* sx = s_zx + (size_t)chunk * c;
+    const int j = threadIdx.x;  // the column this thread folds
+    OnlineSoftmax st;
+    st.init();
+    for (int q0 = 0; q0 < ncand; q0 += chunk) {
+        const int nq = min(chunk, ncand - q0);
+        const int items = nq * vecs;
+        for (int w0 = threadIdx.x; w0 < items; w0 += kSmallItems * blockDim.x) {
+            typename RowLoad<T, V>::Raw zr[kSmallItems], xr[kSmallItems];
+#pragma unroll
+            for (int u = 0; u < kSmallItems; ++u) {
+                const int w = w0 + u * blockDim.x;
+                if (w < items) {
+                    const int q = q0 + w / vecs, col = (w % vecs) * V;
+                    RowLoad<T, V>::load(row_of(p.Za, p.Zb, q) + col, zr[u]);
+                    RowLoad<T, V>::load(row_of(p.Xa, p.Xb, q) + col, xr[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kSmallItems; ++u) {
+                const int w = w0 + u * blockDim.x;
+                if (w < items) {
+                    const int q = q0 + w / vecs, col = (w % vecs) * V;
+                    float z[V], x[V];
+                    RowLoad<T, V>::unpack(zr[u], z);
+                    RowLoad<T, V>::unpack(xr[u], x);
+                    const float* bias = q < p.m ? (p.Ba ? p.Ba + (int64_t)q * c : nullptr)
+                                                : (p.Bb ? p.Bb + (int64_t)(q - p.m) * c : nullptr);
+                    const int o = (q - q0) * c + col;
+#pragma unroll
+                    for (int v = 0; v < V; ++v) {
+                        sz[o + v] = bias ? z[v] + __ldg(bias + col + v) : z[v];
+                        sx[o + v] = x[v];
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (j < c)
+            for (int q = 0; q < nq; ++q) st.add(sz[q * c + j], sx[q * c + j]);
+        __syncthreads();  // the chunk's buffer is rewritten by the next chunk
+    }
+    if (j < c) static_cast<T*>(p.out)[b * p.out_ld_batch + i * c + j] = from_f32<T>(st.acc / st.sum);
+}
+
+// The chunk (candidates held in shared memory at once) of pool_small_kernel, or 0 when
+// the call is not decode-sized or its columns exceed one CTA.
+int small_pool_chunk(const PoolArgs& p)
+{
+    const int64_t nent = p.e1 - p.e0;
+    if (nent <= 0 || (int64_t)p.B * nent > kNumSMs || p.B > 65535 || p.c > 1024) return 0;
+    const int ncand = p.has_b ? 2 * p.m : p.m;
+    int chunk = kSmallSmem / (8 * p.c);
+    if (chunk > kSmallChunk) chunk = kSmallChunk;
+    if (chunk > ncand) chunk = ncand;
+    return chunk;
+}
+
 // ----------------------------------------------------------------------------------
 // TMA-staged streaming path (bf16, c a multiple of 256, prefill-sized calls; CSA with
 // m = 4, HCA with m' a multiple of 32).
@@ -562,6 +657,17 @@ int launch_pool(const PoolArgs& p, int dtype, cudaStream_t stream)
     const int V = vec ? 16 / elem_bytes(dtype) : 1;
     const int64_t total = (int64_t)p.B * (p.e1 - p.e0) * (p.c / V);
     if (total == 0) return CSA_OK;
+    if (const int chunk = small_pool_chunk(p)) {
+        const dim3 grid((unsigned)(p.e1 - p.e0), (unsigned)p.B);
+        const dim3 block((unsigned)((p.c + 31) / 32 * 32));
+        const size_t smem = (size_t)chunk * p.c * 8;
+        void (*kern)(PoolArgs, int) =
+            dtype == CSA_BF16 ? (vec ? pool_small_kernel<__nv_bfloat16, 8> : pool_small_kernel<__nv_bfloat16, 1>)
+                              : (vec ? pool_small_kernel<float, 4> : pool_small_kernel<float, 1>);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        launch_pdl(kern, grid, block, smem, stream, p, chunk);
+        return launch_status();
+    }
     int64_t blocks = (total + kThreads - 1) / kThreads;
     const int64_t cap = (int64_t)kNumSMs * 64;
     if (blocks > cap) blocks = cap;

@@ -269,6 +269,43 @@ def test_hca_compress_prefill_size(B, mp, nent, c, e0, bias):
         assert np.all(np.isnan(got[b, :e0]))
 
 
+@pytest.mark.parametrize("dtype,mp", [(torch.bfloat16, 16), (torch.float32, 128)])
+def test_compress_block_end_entries_match_wide_calls_bit_exactly(dtype, mp):
+    """Single block-end entries, as a decode appends them (one CTA per entry, the candidate
+    rows of a chunk loaded at once), against the same entries of calls over 100 entries x 2
+    batch rows (one thread per column group and entry), bit for bit: CSA with biases, entry
+    0 without a b-part; HCA with m' = 16 and m' = 128 (four chunks of 32 candidates).  The
+    wide calls are checked against the oracle on sampled entries."""
+    B, c, m, nent = 2, 512, 4, 100
+    S = [randn((B, m * nent, c), 490 + i, dtype) for i in range(4)]
+    Ba, Bb = randn((m, c), 495, torch.float32), randn((m, c), 496, torch.float32)
+    Sd = [dev(x) for x in S]
+    full = run_csa_compress(*Sd, m, Ba=dev(Ba), Bb=dev(Bb))
+    for i in (0, 1, 57, 99):
+        lo = max(0, m * (i - 1))
+        part = run_csa_compress(*(x[:, lo:m * (i + 1)] for x in Sd), m, Ba=dev(Ba), Bb=dev(Bb), i0=i, i1=i + 1,
+                                tok0=lo, N_cap=nent)
+        torch.testing.assert_close(part[:, i], full[:, i], rtol=0, atol=0)
+    for b in range(B):
+        ref = oracle.csa_compress(*(to_f64(x[b]) for x in S), m, Ba=to_f64(Ba), Bb=to_f64(Bb), i0=0, i1=8)
+        assert max_rel_rowwise(full[b, :8].double().cpu().numpy(), ref).max() <= TOL[dtype]
+    n_h = mp * nent
+    C, Z = randn((B, n_h, c), 497, dtype), randn((B, n_h, c), 498, dtype)
+    Bias = randn((mp, c), 499, torch.float32)
+    Cd, Zd = dev(C), dev(Z)
+    hfull = torch.full((B, nent, c), float("nan"), dtype=dtype, device=DEV)
+    hca_compress(Cd, Zd, hfull, mp, Bias=dev(Bias))
+    for i in (0, 63, 99):
+        part = torch.full((B, nent, c), float("nan"), dtype=dtype, device=DEV)
+        hca_compress(Cd[:, mp * i:mp * (i + 1)], Zd[:, mp * i:mp * (i + 1)], part, mp, i, i + 1, Bias=dev(Bias),
+                     tok0=mp * i)
+        torch.cuda.synchronize()
+        torch.testing.assert_close(part[:, i], hfull[:, i], rtol=0, atol=0)
+    for b in range(B):
+        ref = oracle.hca_compress(to_f64(C[b]), to_f64(Z[b]), mp, Bias=to_f64(Bias), i0=90, i1=100)
+        assert max_rel_rowwise(hfull[b, 90:].double().cpu().numpy(), ref).max() <= TOL[dtype]
+
+
 def test_compress_extreme_logits_one_hot():
     B, n, c, m = 1, 32, 64, 4
     Ca, Cb = randn((B, n, c), 140, torch.float32), randn((B, n, c), 141, torch.float32)
